@@ -1,0 +1,442 @@
+"""fp64 CPU oracle for Megatron-style tensor-parallel layers.
+
+TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and
+the CPU-baseline leg of ``bench.py`` may import this module.  The CUDA path
+in ``linear_layers_b200`` never imports it and shares no code with it.
+
+Everything here is plain numpy in float64 (matrix products through ``@``,
+element-wise maps through numpy ufuncs).  There is no blocking, fusion or
+reordering beyond what the definitions below state.  Inputs arrive in their
+storage dtype (bf16 / fp32 torch tensors or numpy arrays) and are widened
+exactly to float64 before any arithmetic.
+
+Sources (web pages on Megatron-LM tensor parallelism), cited by page title
+and section:
+
+* [MLP-TP] "Megatron-LM：张量并行与大规模训练" (astro-blog-cod.pages.dev),
+  §2.1 "MLP 层的张量并行": Y = GeLU(XA)B with A [h,4h] split by columns,
+  B [4h,h] split by rows, one all-reduce of the Z_i after the row GEMM;
+  §2.2 "Self-Attention 的张量并行": per-shard heads, QKV column-split,
+  output projection row-split followed by one all-reduce.
+* [TP-ILL] 张量模型并行图解 page (m.youleyou.com/wenzhang/3143730),
+  §1.1 "按行切分权重" and §1.2 "按列切分权重" (the f and g operators and
+  their backward), §2.1 "MLP层的张量模型并行计算方法", §3.1
+  "Multihead-Attention的计算方法", §4.1 "输入层Embedding", §4.2
+  "输出层Embedding", §5 "Cross-Entropy层".
+* [APX] "Megatron-LM 介绍" (apxml.com), §"核心贡献": column-parallel
+  Y_i = X A_i and the Linear(1024→4096), TP=2 shape example.
+
+Readings where the pages are silent or garbled (each also listed with the
+design notes):
+
+* GeLU has no formula on any page.  Default: the tanh closed form
+  0.5·x·(1 + tanh(√(2/π)·(x + 0.044715·x³))); the erf form x·Φ(x) is the
+  selectable alternative.
+* No page has a bias.  A column bias [F] is added before the activation and
+  is split with A's columns.
+* The vocabulary split of §4.1's example is printed as [0,150) and
+  [150,299) for v=300; read as contiguous half-open ranges
+  [i·v/N, (i+1)·v/N).
+* §5 sums raw exponentials; the per-shard maximum is subtracted first
+  (mathematically equal, numerically safe).  The loss is returned per token
+  and as the sum over tokens ("按行加总得到 scalar Loss").
+* Ties in the arg-max go to the lowest vocabulary index.
+
+Pins (tests that hold this oracle to something other than itself) live in
+``tests/test_oracle_pins.py`` and ``tests/test_oracle_mutations.py``.
+No function here is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+ACT_NONE = 0
+ACT_GELU_TANH = 1
+ACT_GELU_ERF = 2
+
+_SQRT_2_OVER_PI = math.sqrt(2.0 / math.pi)
+_GELU_CUBIC = 0.044715
+
+
+# ----------------------------------------------------------------------------
+# conversions
+# ----------------------------------------------------------------------------
+def f64(x) -> np.ndarray:
+    """Widen a torch tensor (any float dtype, incl. bf16) or array to float64."""
+    if hasattr(x, "detach"):  # torch tensor; bf16 has no numpy dtype
+        import torch
+
+        return x.detach().to(device="cpu", dtype=torch.float64).numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def i64(x) -> np.ndarray:
+    if hasattr(x, "detach"):
+        return x.detach().cpu().numpy().astype(np.int64)
+    return np.asarray(x, dtype=np.int64)
+
+
+# ----------------------------------------------------------------------------
+# activation (no page gives the formula; see module docstring)
+# ----------------------------------------------------------------------------
+def _erf(x: np.ndarray) -> np.ndarray:
+    from scipy.special import erf
+
+    return erf(x)
+
+
+def act_fwd(u: np.ndarray, act: int) -> np.ndarray:
+    if act == ACT_NONE:
+        return u.copy()
+    if act == ACT_GELU_TANH:
+        inner = _SQRT_2_OVER_PI * (u + _GELU_CUBIC * u ** 3)
+        return 0.5 * u * (1.0 + np.tanh(inner))
+    if act == ACT_GELU_ERF:
+        return 0.5 * u * (1.0 + _erf(u / math.sqrt(2.0)))
+    raise ValueError(f"unknown activation {act}")
+
+
+def act_grad(u: np.ndarray, act: int) -> np.ndarray:
+    """d act(u) / du, element-wise."""
+    if act == ACT_NONE:
+        return np.ones_like(u)
+    if act == ACT_GELU_TANH:
+        t = np.tanh(_SQRT_2_OVER_PI * (u + _GELU_CUBIC * u ** 3))
+        dinner = _SQRT_2_OVER_PI * (1.0 + 3.0 * _GELU_CUBIC * u ** 2)
+        return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * dinner
+    if act == ACT_GELU_ERF:
+        cdf = 0.5 * (1.0 + _erf(u / math.sqrt(2.0)))
+        pdf = np.exp(-0.5 * u * u) / math.sqrt(2.0 * math.pi)
+        return cdf + u * pdf
+    raise ValueError(f"unknown activation {act}")
+
+
+# ----------------------------------------------------------------------------
+# shards
+# ----------------------------------------------------------------------------
+def even_offsets(total: int, N: int) -> list[int]:
+    """Contiguous half-open ranges [i·total/N, (i+1)·total/N); needs N | total.
+
+    [TP-ILL] §4.1 splits the vocabulary into contiguous ranges, one per GPU;
+    [MLP-TP] §2.1 gives each GPU 1/N of A's columns ([h, 4h/N]).
+    """
+    if total % N:
+        raise ValueError(f"{total} is not divisible by {N}")
+    step = total // N
+    return [i * step for i in range(N + 1)]
+
+
+def all_reduce_sum(parts):
+    """The all-reduce of the pages, written out: sum the N partials in shard order."""
+    acc = np.array(parts[0], dtype=np.float64, copy=True)
+    for p in parts[1:]:
+        acc = acc + p
+    return acc
+
+
+# ----------------------------------------------------------------------------
+# TP-MLP, unsharded definition  ([MLP-TP] §2.1; [TP-ILL] §2.1)
+# ----------------------------------------------------------------------------
+def mlp_fwd(X, A, bias, B, act=ACT_GELU_TANH):
+    """U = X·A + bias, Y = act(U), Z = Y·B.   Returns (U, Y, Z) in fp64."""
+    X, A, B = f64(X), f64(A), f64(B)
+    U = X @ A
+    if bias is not None:
+        U = U + f64(bias)[None, :]
+    Y = act_fwd(U, act)
+    Z = Y @ B
+    return U, Y, Z
+
+
+def mlp_bwd(X, A, bias, B, dZ, act=ACT_GELU_TANH):
+    """Gradient of L = Σ Z⊙dZ for Z = act(X·A + bias)·B.
+
+    Returns dict(dX, dA, dbias, dB, dU, dY).  The forward is recomputed here
+    in fp64 from the inputs.
+    """
+    X, A, B, dZ = f64(X), f64(A), f64(B), f64(dZ)
+    U, Y, _ = mlp_fwd(X, A, bias, B, act)
+    dY = dZ @ B.T
+    dU = dY * act_grad(U, act)
+    return {
+        "dY": dY,
+        "dU": dU,
+        "dB": Y.T @ dZ,
+        "dA": X.T @ dU,
+        "dbias": dU.sum(axis=0),
+        "dX": dU @ A.T,
+    }
+
+
+# ----------------------------------------------------------------------------
+# TP-MLP, sharded algorithm with an explicit host all-reduce
+# ([MLP-TP] §2.1 pseudocode; [TP-ILL] §1.1, §1.2 and §2.1 f/g operators)
+# ----------------------------------------------------------------------------
+def mlp_fwd_sharded(X, A, bias, B, N, offsets=None, act=ACT_GELU_TANH):
+    """Per shard i: Y_i = act(X·A_i + bias_i), Z_i = Y_i·B_i; Z = all-reduce(Z_i).
+
+    f forward is the identity (every shard sees the same X).  Returns
+    dict(Z, Zparts, U, Y) with U, Y assembled from the shards' column blocks.
+    """
+    X, A, B = f64(X), f64(A), f64(B)
+    F = A.shape[1]
+    offs = even_offsets(F, N) if offsets is None else list(offsets)
+    b = np.zeros(F) if bias is None else f64(bias)
+    Zparts, Us, Ys = [], [], []
+    for i in range(N):
+        lo, hi = offs[i], offs[i + 1]
+        Ui = X @ A[:, lo:hi] + b[None, lo:hi]
+        Yi = act_fwd(Ui, act)
+        Zparts.append(Yi @ B[lo:hi, :])
+        Us.append(Ui)
+        Ys.append(Yi)
+    return {
+        "Z": all_reduce_sum(Zparts),
+        "Zparts": Zparts,
+        "U": np.concatenate(Us, axis=1),
+        "Y": np.concatenate(Ys, axis=1),
+    }
+
+
+def mlp_bwd_sharded(X, A, bias, B, dZ, N, offsets=None, act=ACT_GELU_TANH):
+    """g backward = identity (dZ to every shard); local dA_i, dB_i, dbias_i;
+    f backward = all-reduce of the N partials dX_i = dU_i·A_iᵀ."""
+    X, A, B, dZ = f64(X), f64(A), f64(B), f64(dZ)
+    F = A.shape[1]
+    offs = even_offsets(F, N) if offsets is None else list(offsets)
+    b = np.zeros(F) if bias is None else f64(bias)
+    dXparts, dAs, dBs, dbs, dUs = [], [], [], [], []
+    for i in range(N):
+        lo, hi = offs[i], offs[i + 1]
+        Ai, Bi = A[:, lo:hi], B[lo:hi, :]
+        Ui = X @ Ai + b[None, lo:hi]
+        Yi = act_fwd(Ui, act)
+        dYi = dZ @ Bi.T
+        dUi = dYi * act_grad(Ui, act)
+        dBs.append(Yi.T @ dZ)
+        dAs.append(X.T @ dUi)
+        dbs.append(dUi.sum(axis=0))
+        dUs.append(dUi)
+        dXparts.append(dUi @ Ai.T)
+    return {
+        "dX": all_reduce_sum(dXparts),
+        "dXparts": dXparts,
+        "dA": np.concatenate(dAs, axis=1),
+        "dB": np.concatenate(dBs, axis=0),
+        "dbias": np.concatenate(dbs),
+        "dU": np.concatenate(dUs, axis=1),
+    }
+
+
+# ----------------------------------------------------------------------------
+# Linear building blocks ([TP-ILL] §1.1, §1.2; [APX] §核心贡献)
+# ----------------------------------------------------------------------------
+def col_linear_fwd(X, W, bias=None, act=ACT_NONE):
+    """Column-parallel linear over all shards: U = X·W + bias, Y = act(U)."""
+    X, W = f64(X), f64(W)
+    U = X @ W
+    if bias is not None:
+        U = U + f64(bias)[None, :]
+    return U, act_fwd(U, act)
+
+
+def col_linear_bwd(X, W, U, dY, act=ACT_NONE):
+    """dU = dY ⊙ act'(U); dW = Xᵀ·dU; dbias = Σ_rows dU; dX = dU·Wᵀ (the f sum)."""
+    X, W, U, dY = f64(X), f64(W), f64(U), f64(dY)
+    dU = dY * act_grad(U, act)
+    return {"dU": dU, "dW": X.T @ dU, "dbias": dU.sum(axis=0), "dX": dU @ W.T}
+
+
+def row_linear_fwd(Xin, W, offsets=None, N=None):
+    """Row-parallel linear: Z = Σ_i Xin[:, lo_i:hi_i]·W[lo_i:hi_i, :] (the g sum).
+
+    With no offsets this is the unsharded product Xin·W.
+    Returns (Z, parts) where parts is None for the unsharded call.
+    """
+    Xin, W = f64(Xin), f64(W)
+    if offsets is None and N is None:
+        return Xin @ W, None
+    offs = even_offsets(W.shape[0], N) if offsets is None else list(offsets)
+    parts = [Xin[:, offs[i]:offs[i + 1]] @ W[offs[i]:offs[i + 1], :]
+             for i in range(len(offs) - 1)]
+    return all_reduce_sum(parts), parts
+
+
+def row_linear_bwd(Xin, W, dZ):
+    """g backward is the identity: dXin = dZ·Wᵀ (per shard columns), dW = Xinᵀ·dZ."""
+    Xin, W, dZ = f64(Xin), f64(W), f64(dZ)
+    return {"dXin": dZ @ W.T, "dW": Xin.T @ dZ}
+
+
+def qkv_shard_columns(n_heads: int, head_dim: int, heads_per_shard):
+    """Column permutation from the standard [Q | K | V] layout (heads in order
+    inside each block) to the shard-major layout in which shard i holds its
+    own Q heads, then its K heads, then its V heads ([MLP-TP] §2.2;
+    [TP-ILL] §3.1: Q, K and V are column-split, one or more heads per GPU).
+
+    Returns (perm, offsets): shard-major column j holds standard column
+    perm[j]; shard i owns shard-major columns [offsets[i], offsets[i+1]).
+    """
+    hd = head_dim
+    h = n_heads * hd
+    perm, offsets, head0 = [], [0], 0
+    for nh in heads_per_shard:
+        for block in range(3):  # Q, K, V
+            for hh in range(head0, head0 + nh):
+                base = block * h + hh * hd
+                perm.extend(range(base, base + hd))
+        head0 += nh
+        offsets.append(len(perm))
+    if head0 != n_heads:
+        raise ValueError("heads_per_shard does not cover all heads")
+    return np.asarray(perm, dtype=np.int64), offsets
+
+
+# ----------------------------------------------------------------------------
+# Vocabulary-parallel embedding ([TP-ILL] §4.1)
+# ----------------------------------------------------------------------------
+def embed_lookup(ids, E):
+    """Plain row lookup out[t] = E[id_t]; ids outside [0, v) give a zero row."""
+    ids, E = i64(ids), f64(E)
+    v, h = E.shape
+    out = np.zeros((ids.shape[0], h))
+    ok = (ids >= 0) & (ids < v)
+    out[ok] = E[ids[ok]]
+    return out
+
+
+def vp_embed_sharded(ids, E, N):
+    """Each shard looks up the ids inside its vocabulary range and writes a
+    zero row for the rest; the N partial outputs are then all-reduced."""
+    ids, E = i64(ids), f64(E)
+    v, h = E.shape
+    offs = even_offsets(v, N)
+    parts = []
+    for i in range(N):
+        lo, hi = offs[i], offs[i + 1]
+        Ei = E[lo:hi]
+        mine = (ids >= lo) & (ids < hi)
+        part = np.zeros((ids.shape[0], h))
+        part[mine] = Ei[ids[mine] - lo]
+        parts.append(part)
+    return all_reduce_sum(parts)
+
+
+def embed_owner(ids, v, N):
+    """Index of the shard whose vocabulary range holds each id (-1 if none)."""
+    ids = i64(ids)
+    offs = even_offsets(v, N)
+    own = np.full(ids.shape, -1, dtype=np.int64)
+    for i in range(N):
+        own[(ids >= offs[i]) & (ids < offs[i + 1])] = i
+    return own
+
+
+# ----------------------------------------------------------------------------
+# Output embedding / logits ([TP-ILL] §4.2)
+# ----------------------------------------------------------------------------
+def logits(H, E):
+    """logits = H·Eᵀ (shared word-embedding table E [v,h])."""
+    return f64(H) @ f64(E).T
+
+
+def logits_sharded(H, E, N):
+    """Shard i computes H·E_iᵀ for its vocabulary rows; the blocks sit side by side."""
+    H, E = f64(H), f64(E)
+    offs = even_offsets(E.shape[0], N)
+    return [H @ E[offs[i]:offs[i + 1]].T for i in range(N)]
+
+
+# ----------------------------------------------------------------------------
+# Vocabulary-parallel softmax cross-entropy ([TP-ILL] §5)
+# ----------------------------------------------------------------------------
+def xent(logits_, targets, grad_scale=1.0):
+    """Unsharded softmax cross-entropy per row.
+
+    loss_t = log Σ_j exp(l_tj) − l_t,y_t;  loss_sum = Σ_t loss_t;
+    dlogits = grad_scale · (softmax(l_t) − onehot(y_t));
+    argmax_t = smallest j with l_tj = max_j l_tj.
+    Targets outside [0, v) give loss NaN and a dlogits row of NaN.
+    """
+    L = f64(logits_)
+    y = i64(targets)
+    T, v = L.shape
+    m = L.max(axis=1)
+    lse = m + np.log(np.exp(L - m[:, None]).sum(axis=1))
+    ok = (y >= 0) & (y < v)
+    tgt = np.full(T, np.nan)
+    tgt[ok] = L[np.nonzero(ok)[0], y[ok]]
+    loss = lse - tgt
+    p = np.exp(L - lse[:, None])
+    d = p.copy()
+    d[np.nonzero(ok)[0], y[ok]] -= 1.0
+    d[~ok] = np.nan
+    return {
+        "loss": loss,
+        "loss_sum": loss.sum(),
+        "dlogits": grad_scale * d,
+        "argmax": np.argmax(L, axis=1).astype(np.int64),  # first maximum
+    }
+
+
+def xent_sharded(logits_, targets, N, grad_scale=1.0):
+    """The vocabulary-parallel algorithm of [TP-ILL] §5, written out per shard.
+
+    Shard i holds columns [lo_i, hi_i).  It computes its maximum m_i, its sum
+    s_i = Σ exp(l − m_i), its masked target logit and its local arg-max; the
+    all-reduce combines m = max m_i, S = Σ s_i·exp(m_i − m) and the target
+    logit; every shard then forms its own block of softmax − onehot and its
+    share of the loss, and a last all-reduce sums the per-shard loss scalars.
+    """
+    L = f64(logits_)
+    y = i64(targets)
+    T, v = L.shape
+    offs = even_offsets(v, N)
+    ms, ss, tg, amax_i, amax_v = [], [], [], [], []
+    for i in range(N):
+        Li = L[:, offs[i]:offs[i + 1]]
+        mi = Li.max(axis=1)
+        ms.append(mi)
+        ss.append(np.exp(Li - mi[:, None]).sum(axis=1))
+        mine = (y >= offs[i]) & (y < offs[i + 1])
+        t = np.zeros(T)
+        t[mine] = Li[np.nonzero(mine)[0], y[mine] - offs[i]]
+        tg.append(t)
+        amax_i.append(np.argmax(Li, axis=1) + offs[i])
+        amax_v.append(mi)
+    # all-reduce (max) of the maxima, then (sum) of the rescaled sums
+    m = ms[0].copy()
+    for mi in ms[1:]:
+        m = np.maximum(m, mi)
+    S = all_reduce_sum([ss[i] * np.exp(ms[i] - m) for i in range(N)])
+    tgt = all_reduce_sum(tg)
+    ok = (y >= 0) & (y < v)
+    tgt[~ok] = np.nan
+    lse = m + np.log(S)
+    loss = lse - tgt
+    dblocks, loss_parts = [], []
+    for i in range(N):
+        Li = L[:, offs[i]:offs[i + 1]]
+        d = np.exp(Li - lse[:, None])
+        mine = (y >= offs[i]) & (y < offs[i + 1])
+        d[np.nonzero(mine)[0], y[mine] - offs[i]] -= 1.0
+        d[~ok] = np.nan
+        dblocks.append(grad_scale * d)
+        loss_parts.append(np.where(mine, loss, 0.0).sum())
+    # arg-max across shards: larger value wins, equal values go to the lower shard
+    best_v = amax_v[0].copy()
+    best_i = amax_i[0].copy()
+    for i in range(1, N):
+        better = amax_v[i] > best_v
+        best_v = np.where(better, amax_v[i], best_v)
+        best_i = np.where(better, amax_i[i], best_i)
+    return {
+        "loss": loss,
+        "loss_sum": all_reduce_sum([np.array(x) for x in loss_parts]),
+        "dlogits": np.concatenate(dblocks, axis=1),
+        "argmax": best_i.astype(np.int64),
+        "m": m,
+        "S": S,
+    }

@@ -1,0 +1,385 @@
+"""Checks that pin the fp64 oracle to facts outside itself.
+
+Each ``check_*`` takes the oracle module and raises AssertionError when the
+oracle disagrees with what the pages or the mathematics fix.  The pin tests
+run every check on the real oracle; the mutation tests plant plausible
+mistakes in the oracle and require at least one check to fail for each.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    den = max(np.linalg.norm(b), 1e-300)
+    return float(np.linalg.norm(a - b) / den)
+
+
+def _rng(seed=0):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------
+# GeLU
+# ----------------------------------------------------------------------------
+def check_gelu_erf_table(o):
+    """x·Φ(x) at the textbook values of the normal CDF."""
+    g = _golden("normal_cdf.json")
+    x = np.array(g["x"])
+    want = x * np.array(g["phi"])
+    got = o.act_fwd(x, o.ACT_GELU_ERF)
+    assert np.max(np.abs(got - want)) < 1e-15, (got, want)
+
+
+def check_gelu_tanh_vs_erf(o):
+    """The tanh closed form approximates x·Φ(x) to within 1e-3 on [-10, 10]
+    (the measured gap of this approximation is 4.73e-4, at |x| ≈ 2.70)."""
+    x = np.linspace(-10.0, 10.0, 200001)
+    gap = np.max(np.abs(o.act_fwd(x, o.ACT_GELU_TANH) - o.act_fwd(x, o.ACT_GELU_ERF)))
+    assert 1e-5 < gap < 1e-3, gap
+
+
+def check_gelu_special_values(o):
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF):
+        assert o.act_fwd(np.array([0.0]), act)[0] == 0.0
+        assert abs(o.act_grad(np.array([0.0]), act)[0] - 0.5) < 1e-15
+        big = o.act_fwd(np.array([10.0, -10.0]), act)
+        assert abs(big[0] - 10.0) < 1e-12 and abs(big[1]) < 1e-12, big
+        # gelu(x) - gelu(-x) = x for both forms (Φ(x) + Φ(-x) = 1, tanh odd)
+        x = np.linspace(-6, 6, 1001)
+        assert np.max(np.abs(o.act_fwd(x, act) - o.act_fwd(-x, act) - x)) < 1e-12
+    # identity "activation"
+    x = np.linspace(-3, 3, 7)
+    assert np.array_equal(o.act_fwd(x, o.ACT_NONE), x)
+    assert np.array_equal(o.act_grad(x, o.ACT_NONE), np.ones_like(x))
+
+
+def check_gelu_derivative_fd(o):
+    x = np.linspace(-8.0, 8.0, 3201)
+    eps = 1e-6
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF):
+        fd = (o.act_fwd(x + eps, act) - o.act_fwd(x - eps, act)) / (2 * eps)
+        assert np.max(np.abs(fd - o.act_grad(x, act))) < 1e-8, act
+
+
+# ----------------------------------------------------------------------------
+# TP-MLP
+# ----------------------------------------------------------------------------
+def _tiny_mlp(seed=0, M=3, h=4, F=8):
+    r = _rng(seed)
+    return (r.normal(size=(M, h)), r.normal(size=(h, F)) * 0.5,
+            r.normal(size=F) * 0.3, r.normal(size=(F, h)) * 0.5,
+            r.normal(size=(M, h)))
+
+
+def check_mlp_bruteforce_loops(o):
+    """Z of the oracle against triple loops over scalars (act = NONE and the
+    erf form, whose Φ comes from math.erf)."""
+    X, A, b, B, _ = _tiny_mlp(1, M=3, h=4, F=6)
+    M, h = X.shape
+    F = A.shape[1]
+    for act, fn in ((o.ACT_NONE, lambda u: u),
+                    (o.ACT_GELU_ERF, lambda u: u * 0.5 * (1 + math.erf(u / math.sqrt(2))))):
+        U = [[sum(X[m][k] * A[k][f] for k in range(h)) + b[f] for f in range(F)]
+             for m in range(M)]
+        Y = [[fn(U[m][f]) for f in range(F)] for m in range(M)]
+        Z = [[sum(Y[m][f] * B[f][j] for f in range(F)) for j in range(h)]
+             for m in range(M)]
+        oU, oY, oZ = o.mlp_fwd(X, A, b, B, act)
+        assert _rel(oU, U) < 1e-14 and _rel(oY, Y) < 1e-14 and _rel(oZ, Z) < 1e-14, act
+
+
+def check_mlp_identity_closed_form(o):
+    """With the identity activation Z = X·(A·B) + bias·B (re-associated)."""
+    X, A, b, B, _ = _tiny_mlp(2, M=5, h=6, F=12)
+    _, _, Z = o.mlp_fwd(X, A, b, B, o.ACT_NONE)
+    AB = A @ B
+    want = X @ AB + (b @ B)[None, :]
+    assert _rel(Z, want) < 1e-13
+
+
+def check_mlp_fd_gradients(o):
+    """Central differences of L = Σ Z⊙dZ against dX, dA, dbias, dB
+    (M=2, h=4, F=8, eps=1e-6)."""
+    X, A, b, B, dZ = _tiny_mlp(3, M=2, h=4, F=8)
+    eps = 1e-6
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF):
+        g = o.mlp_bwd(X, A, b, B, dZ, act)
+
+        def loss(X_, A_, b_, B_):
+            return float((o.mlp_fwd(X_, A_, b_, B_, act)[2] * dZ).sum())
+
+        for name, arr in (("dX", X), ("dA", A), ("dbias", b), ("dB", B)):
+            fd = np.zeros_like(arr)
+            it = np.nditer(arr, flags=["multi_index"])
+            for _ in it:
+                idx = it.multi_index
+                args = {"X": X, "A": A, "b": b, "B": B}
+                key = {"dX": "X", "dA": "A", "dbias": "b", "dB": "B"}[name]
+                plus = arr.copy()
+                plus[idx] += eps
+                minus = arr.copy()
+                minus[idx] -= eps
+                args[key] = plus
+                lp = loss(args["X"], args["A"], args["b"], args["B"])
+                args[key] = minus
+                lm = loss(args["X"], args["A"], args["b"], args["B"])
+                fd[idx] = (lp - lm) / (2 * eps)
+            assert _rel(g[name], fd) < 1e-7, (act, name, _rel(g[name], fd))
+
+
+def check_mlp_sharded_equals_unsharded(o):
+    """Column split of A and row split of B with one all-reduce reproduce the
+    unsharded layer exactly up to rounding (N = 1, 2, 4, 8 and uneven shards)."""
+    X, A, b, B, dZ = _tiny_mlp(4, M=6, h=8, F=32)
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF, o.ACT_NONE):
+        U, Y, Z = o.mlp_fwd(X, A, b, B, act)
+        g = o.mlp_bwd(X, A, b, B, dZ, act)
+        cases = [dict(N=n) for n in (1, 2, 4, 8)] + [dict(N=3, offsets=[0, 5, 19, 32])]
+        for c in cases:
+            s = o.mlp_fwd_sharded(X, A, b, B, c["N"], c.get("offsets"), act)
+            assert _rel(s["Z"], Z) < 1e-12 and _rel(s["U"], U) < 1e-14 and _rel(s["Y"], Y) < 1e-14
+            sb = o.mlp_bwd_sharded(X, A, b, B, dZ, c["N"], c.get("offsets"), act)
+            for k in ("dX", "dA", "dB", "dbias", "dU"):
+                assert _rel(sb[k], g[k]) < 1e-12, (act, c, k)
+            # each partial is its shard's own product (not a share of the sum)
+            offs = c.get("offsets") or o.even_offsets(32, c["N"])
+            for i, Zi in enumerate(s["Zparts"]):
+                lo, hi = offs[i], offs[i + 1]
+                assert _rel(Zi, Y[:, lo:hi] @ B[lo:hi]) < 1e-13
+
+
+def check_row_split_of_A_breaks_gelu(o):
+    """Why A is split by columns: splitting A by rows (X by columns) and
+    applying GeLU per shard before the sum does not give GeLU(X·A)."""
+    X, A, b, B, _ = _tiny_mlp(5, M=4, h=8, F=8)
+    full = o.act_fwd(X @ A, o.ACT_GELU_TANH)
+    wrong = sum(o.act_fwd(X[:, i * 4:(i + 1) * 4] @ A[i * 4:(i + 1) * 4], o.ACT_GELU_TANH)
+                for i in range(2))
+    assert _rel(wrong, full) > 1e-2
+    # column split: GeLU of each column block equals the block of GeLU
+    blocks = np.concatenate([o.act_fwd(X @ A[:, i * 4:(i + 1) * 4], o.ACT_GELU_TANH)
+                             for i in range(2)], axis=1)
+    assert np.array_equal(blocks, full)
+
+
+def check_apx_shape_example(o):
+    g = _golden("apx_linear_shapes.json")
+    r = _rng(6)
+    x = r.normal(size=(g["batch"], g["in_features"]))
+    W = r.normal(size=(g["in_features"], g["out_features"])) * 0.02
+    _, full = o.col_linear_fwd(x, W)
+    assert list(full.shape) == g["full_shape"]
+    offs = o.even_offsets(g["out_features"], g["tp"])
+    parts = [o.col_linear_fwd(x, W[:, offs[i]:offs[i + 1]])[1] for i in range(g["tp"])]
+    for p in parts:
+        assert list(p.shape) == g["shard_shape"]
+    assert np.array_equal(np.concatenate(parts, axis=1), full)
+
+
+def check_linear_blocks(o):
+    """Column/row linear blocks: sharded == unsharded, gradients by FD."""
+    r = _rng(7)
+    X = r.normal(size=(5, 6))
+    W = r.normal(size=(6, 10))
+    b = r.normal(size=10)
+    U, Y = o.col_linear_fwd(X, W, b, o.ACT_GELU_TANH)
+    assert _rel(U, X @ W + b) < 1e-14
+    dY = r.normal(size=U.shape)
+    g = o.col_linear_bwd(X, W, U, dY, o.ACT_GELU_TANH)
+    eps = 1e-6
+    fdW = np.zeros_like(W)
+    for i in range(W.shape[0]):
+        for j in range(W.shape[1]):
+            Wp, Wm = W.copy(), W.copy()
+            Wp[i, j] += eps
+            Wm[i, j] -= eps
+            fdW[i, j] = ((o.col_linear_fwd(X, Wp, b, o.ACT_GELU_TANH)[1]
+                          - o.col_linear_fwd(X, Wm, b, o.ACT_GELU_TANH)[1]) * dY).sum() / (2 * eps)
+    assert _rel(g["dW"], fdW) < 1e-7
+    fdX = np.zeros_like(X)
+    for i in range(X.shape[0]):
+        for j in range(X.shape[1]):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[i, j] += eps
+            Xm[i, j] -= eps
+            fdX[i, j] = ((o.col_linear_fwd(Xp, W, b, o.ACT_GELU_TANH)[1]
+                          - o.col_linear_fwd(Xm, W, b, o.ACT_GELU_TANH)[1]) * dY).sum() / (2 * eps)
+    assert _rel(g["dX"], fdX) < 1e-7
+    # row-parallel: sum of per-shard partials == unsharded product
+    Xin = r.normal(size=(4, 12))
+    Wr = r.normal(size=(12, 5))
+    Z, _ = o.row_linear_fwd(Xin, Wr)
+    Zs, parts = o.row_linear_fwd(Xin, Wr, offsets=[0, 7, 12])
+    assert _rel(Zs, Z) < 1e-14 and len(parts) == 2
+    dZ = r.normal(size=Z.shape)
+    gb = o.row_linear_bwd(Xin, Wr, dZ)
+    assert _rel(gb["dW"], np.einsum("mi,mj->ij", Xin, dZ)) < 1e-14
+    assert _rel(gb["dXin"], np.einsum("mj,ij->mi", dZ, Wr)) < 1e-14
+
+
+def check_qkv_head_split(o):
+    """25 heads over 4 shards -> 7, 6, 6, 6; shard-major columns are a
+    permutation of [Q | K | V] and shard i's block holds exactly its heads."""
+    perm, offs = o.qkv_shard_columns(25, 64, [7, 6, 6, 6])
+    assert offs == [0, 7 * 192, 13 * 192, 19 * 192, 25 * 192]
+    assert sorted(perm.tolist()) == list(range(3 * 1600))
+    # shard 1 starts with Q of head 7, then its K block starts at Q-offset 1600 + 7*64
+    s1 = perm[offs[1]:offs[2]]
+    assert s1[0] == 7 * 64 and s1[6 * 64] == 1600 + 7 * 64 and s1[12 * 64] == 3200 + 7 * 64
+
+
+# ----------------------------------------------------------------------------
+# embedding
+# ----------------------------------------------------------------------------
+def check_embed_page_example(o):
+    g = _golden("embed_vocab300_n2.json")
+    v, N, ids = g["v"], g["N"], np.array(g["ids"])
+    assert [[o.even_offsets(v, N)[i], o.even_offsets(v, N)[i + 1]] for i in range(N)] == g["shard_ranges"]
+    assert o.embed_owner(ids, v, N).tolist() == g["owner"]
+    E = _rng(8).normal(size=(v, 16))
+    out = o.vp_embed_sharded(ids, E, N)
+    for t, i in enumerate(ids):
+        assert np.array_equal(out[t], E[i])
+
+
+def check_embed_sharded_equals_lookup(o):
+    import torch
+
+    r = _rng(9)
+    v, h = 96, 24
+    E = r.normal(size=(v, h))
+    ids = r.integers(0, v, size=50)
+    ref = torch.nn.functional.embedding(torch.from_numpy(ids), torch.from_numpy(E)).numpy()
+    assert np.array_equal(o.embed_lookup(ids, E), ref)
+    for N in (1, 2, 3, 4, 8):
+        assert np.array_equal(o.vp_embed_sharded(ids, E, N), ref), N
+    bad = np.array([-1, v, 5])
+    out = o.vp_embed_sharded(bad, E, 4)
+    assert not out[0].any() and not out[1].any() and np.array_equal(out[2], E[5])
+    assert np.array_equal(o.embed_lookup(bad, E), out)
+
+
+# ----------------------------------------------------------------------------
+# logits
+# ----------------------------------------------------------------------------
+def check_logits(o):
+    import torch
+
+    r = _rng(10)
+    H = r.normal(size=(7, 16))
+    E = r.normal(size=(40, 16))
+    L = o.logits(H, E)
+    ref = torch.nn.functional.linear(torch.from_numpy(H), torch.from_numpy(E)).numpy()
+    assert _rel(L, ref) < 1e-14
+    blocks = o.logits_sharded(H, E, 4)
+    assert _rel(np.concatenate(blocks, axis=1), L) < 1e-15
+    # brute force single entry
+    assert abs(L[3, 17] - sum(H[3, k] * E[17, k] for k in range(16))) < 1e-12
+
+
+# ----------------------------------------------------------------------------
+# cross-entropy
+# ----------------------------------------------------------------------------
+def check_xent_uniform(o):
+    """Equal logits: loss = log v, dlogits = 1/v − onehot."""
+    v = 48
+    L = np.full((3, v), 0.7)
+    y = np.array([0, 17, 47])
+    r = o.xent(L, y)
+    assert np.max(np.abs(r["loss"] - math.log(v))) < 1e-13
+    want = np.full((3, v), 1.0 / v)
+    want[[0, 1, 2], y] -= 1.0
+    assert np.max(np.abs(r["dlogits"] - want)) < 1e-15
+    assert r["argmax"].tolist() == [0, 0, 0]
+
+
+def check_xent_dominant(o):
+    v = 32
+    L = np.zeros((2, v))
+    L[0, 5] = 1000.0
+    L[1, 9] = 1000.0
+    r = o.xent(L, np.array([5, 3]))
+    assert abs(r["loss"][0]) < 1e-12 and abs(r["loss"][1] - 1000.0) < 1e-9
+    assert r["argmax"].tolist() == [5, 9]
+
+
+def check_xent_vs_torch(o):
+    import torch
+
+    r = _rng(11)
+    L = r.normal(size=(9, 37)) * 2.0
+    y = r.integers(0, 37, size=9)
+    Lt = torch.from_numpy(L).requires_grad_(True)
+    loss = torch.nn.functional.cross_entropy(Lt, torch.from_numpy(y), reduction="none")
+    loss.sum().backward()
+    got = o.xent(L, y, grad_scale=1.0)
+    assert _rel(got["loss"], loss.detach().numpy()) < 1e-13
+    assert abs(got["loss_sum"] - float(loss.detach().sum())) < 1e-12
+    assert _rel(got["dlogits"], Lt.grad.numpy()) < 1e-13
+    assert np.array_equal(got["argmax"], np.argmax(L, axis=1))
+    got2 = o.xent(L, y, grad_scale=0.25)
+    assert _rel(got2["dlogits"], 0.25 * Lt.grad.numpy()) < 1e-14
+
+
+def check_xent_invariants(o):
+    r = _rng(12)
+    L = r.normal(size=(6, 50)) * 3
+    y = r.integers(0, 50, size=6)
+    a = o.xent(L, y)
+    assert np.max(np.abs(a["dlogits"].sum(axis=1))) < 1e-14      # rows sum to 0
+    b = o.xent(L + 123.0, y)                                       # shift invariance
+    assert np.max(np.abs(a["loss"] - b["loss"])) < 1e-10
+    eps = 1e-6                                                     # FD of loss_t
+    for t in range(2):
+        for j in (0, y[t], 49):
+            Lp, Lm = L.copy(), L.copy()
+            Lp[t, j] += eps
+            Lm[t, j] -= eps
+            fd = (o.xent(Lp, y)["loss"][t] - o.xent(Lm, y)["loss"][t]) / (2 * eps)
+            assert abs(fd - a["dlogits"][t, j]) < 1e-8
+    bad = o.xent(L[:2], np.array([-1, 50]))
+    assert np.all(np.isnan(bad["loss"]))
+
+
+def check_xent_sharded(o):
+    r = _rng(13)
+    v = 48
+    L = r.normal(size=(11, v)) * 2
+    y = r.integers(0, v, size=11)
+    ref = o.xent(L, y, grad_scale=0.5)
+    for N in (1, 2, 3, 4, 8):
+        s = o.xent_sharded(L, y, N, grad_scale=0.5)
+        assert _rel(s["loss"], ref["loss"]) < 1e-12, N
+        assert abs(s["loss_sum"] - ref["loss_sum"]) < 1e-11
+        assert _rel(s["dlogits"], ref["dlogits"]) < 1e-12
+        assert np.array_equal(s["argmax"], ref["argmax"])
+        assert _rel(np.log(s["S"]) + s["m"], ref["loss"] + L[np.arange(11), y]) < 1e-12
+
+
+def check_xent_argmax_ties(o):
+    """Equal maxima go to the lowest index, also across shard boundaries."""
+    v = 16
+    L = np.zeros((3, v))
+    L[0, [3, 12]] = 5.0   # tie across shards (N=4: ranges of 4)
+    L[1, [9, 10]] = 2.0   # tie inside one shard
+    L[2, :] = -1.0        # all equal
+    y = np.array([0, 0, 0])
+    for fn in (lambda: o.xent(L, y), lambda: o.xent_sharded(L, y, 4)):
+        assert fn()["argmax"].tolist() == [3, 9, 0]
+
+
+ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -1,0 +1,156 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and require the pins
+to catch each one: a pin set that a dropped term, a wrong sign or index, or
+a transposed operand slips through would not be worth trusting."""
+import math
+
+import numpy as np
+import pytest
+
+from oracle import tp_oracle as O
+from tests import oracle_checks as C
+
+
+def _m_gelu_grad_drop_term(mp):
+    def bad(u, act):
+        if act == O.ACT_GELU_TANH:
+            t = np.tanh(math.sqrt(2 / math.pi) * (u + 0.044715 * u ** 3))
+            return 0.5 * (1.0 + t)           # dropped the x·(1 − t²)·dinner term
+        return O.__dict__["_orig_act_grad"](u, act)
+    mp.setitem(O.__dict__, "_orig_act_grad", O.act_grad)
+    mp.setattr(O, "act_grad", bad)
+
+
+def _m_gelu_wrong_constant(mp):
+    mp.setattr(O, "_SQRT_2_OVER_PI", math.sqrt(math.pi / 2))
+
+
+def _m_gelu_sign(mp):
+    orig = O.act_fwd
+
+    def bad(u, act):
+        if act == O.ACT_GELU_TANH:
+            return 0.5 * u * (1.0 - np.tanh(O._SQRT_2_OVER_PI * (u + O._GELU_CUBIC * u ** 3)))
+        return orig(u, act)
+    mp.setattr(O, "act_fwd", bad)
+
+
+def _m_fwd_drop_bias(mp):
+    orig = O.mlp_fwd
+    mp.setattr(O, "mlp_fwd", lambda X, A, bias, B, act=O.ACT_GELU_TANH: orig(X, A, None, B, act))
+
+
+def _m_bwd_no_act_grad(mp):
+    orig = O.mlp_bwd
+
+    def bad(X, A, bias, B, dZ, act=O.ACT_GELU_TANH):
+        g = orig(X, A, bias, B, dZ, act)
+        g["dA"] = O.f64(X).T @ g["dY"]
+        return g
+    mp.setattr(O, "mlp_bwd", bad)
+
+
+def _m_bwd_transposed_dB(mp):
+    orig = O.mlp_bwd
+
+    def bad(X, A, bias, B, dZ, act=O.ACT_GELU_TANH):
+        g = orig(X, A, bias, B, dZ, act)
+        g["dB"] = g["dB"].reshape(g["dB"].shape[1], g["dB"].shape[0]).T.copy()  # wrong index order
+        return g
+    mp.setattr(O, "mlp_bwd", bad)
+
+
+def _m_bwd_dX_no_sum_of_shards(mp):
+    orig = O.mlp_bwd_sharded
+
+    def bad(*a, **k):
+        r = orig(*a, **k)
+        r["dX"] = r["dXparts"][0]        # f backward without its all-reduce
+        return r
+    mp.setattr(O, "mlp_bwd_sharded", bad)
+
+
+def _m_allreduce_drops_last(mp):
+    mp.setattr(O, "all_reduce_sum", lambda parts: np.sum(np.stack(parts[:-1] or parts), axis=0)
+               if len(parts) > 1 else np.array(parts[0], dtype=np.float64))
+
+
+def _m_offsets_off_by_one(mp):
+    def bad(total, N):
+        step = total // N
+        return [0] + [i * step - 1 for i in range(1, N)] + [total]
+    mp.setattr(O, "even_offsets", bad)
+
+
+def _m_embed_index_shift(mp):
+    def bad(ids, E):
+        ids, E = O.i64(ids), O.f64(E)
+        out = np.zeros((ids.shape[0], E.shape[1]))
+        ok = (ids >= 0) & (ids < E.shape[0])
+        out[ok] = E[np.maximum(ids[ok] - 1, 0)]
+        return out
+    mp.setattr(O, "embed_lookup", bad)
+
+
+def _m_xent_loss_sign(mp):
+    orig = O.xent
+
+    def bad(L, y, grad_scale=1.0):
+        r = orig(L, y, grad_scale)
+        Lf, yy = O.f64(L), O.i64(y)
+        tgt = Lf[np.arange(Lf.shape[0]), np.clip(yy, 0, Lf.shape[1] - 1)]
+        r["loss"] = r["loss"] + 2 * tgt
+        return r
+    mp.setattr(O, "xent", bad)
+
+
+def _m_xent_no_onehot(mp):
+    orig = O.xent
+
+    def bad(L, y, grad_scale=1.0):
+        r = orig(L, y, grad_scale)
+        Lf = O.f64(L)
+        p = np.exp(Lf - Lf.max(1, keepdims=True))
+        r["dlogits"] = grad_scale * p / p.sum(1, keepdims=True)
+        return r
+    mp.setattr(O, "xent", bad)
+
+
+def _m_xent_combine_no_rescale(mp):
+    orig = O.xent_sharded
+
+    def bad(L, y, N, grad_scale=1.0):
+        r = orig(L, y, N, grad_scale)
+        Lf = O.f64(L)
+        offs = O.even_offsets(Lf.shape[1], N)
+        S = sum(np.exp(Lf[:, offs[i]:offs[i + 1]] - Lf[:, offs[i]:offs[i + 1]].max(1, keepdims=True)).sum(1)
+                for i in range(N))
+        r["S"] = S
+        r["loss"] = r["m"] + np.log(S) - Lf[np.arange(Lf.shape[0]), O.i64(y)]
+        return r
+    mp.setattr(O, "xent_sharded", bad)
+
+
+def _m_argmax_last(mp):
+    orig = O.xent
+
+    def bad(L, y, grad_scale=1.0):
+        r = orig(L, y, grad_scale)
+        Lf = O.f64(L)
+        r["argmax"] = Lf.shape[1] - 1 - np.argmax(Lf[:, ::-1], axis=1)
+        return r
+    mp.setattr(O, "xent", bad)
+
+
+MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
+
+
+@pytest.mark.parametrize("mutate", MUTATIONS, ids=lambda f: f.__name__[3:])
+def test_pins_catch_mutation(mutate, monkeypatch):
+    mutate(monkeypatch)
+    failed = []
+    for check in C.ALL_CHECKS:
+        try:
+            check(O)
+        except Exception:  # AssertionError, or a shape error from a bad transpose
+            failed.append(check.__name__)
+    assert failed, "no pin caught this planted mistake"
