@@ -1,0 +1,266 @@
+/*
+ * tplayers.h — C ABI of the B200 tensor-parallel layers library (libtplayers.so).
+ *
+ * Megatron-style tensor parallelism on ONE GPU: the N shards of a layer are
+ * partitions of device memory, and the sums the pages perform with
+ * all-reduces (the g operator after the row-parallel GEMM, the f operator in
+ * backward, the embedding and the cross-entropy reductions) are on-device
+ * reductions fused into the kernels that produce the partials.
+ *
+ * Sources, cited by page title and section:
+ *   [MLP-TP] "Megatron-LM：张量并行与大规模训练" (astro-blog-cod.pages.dev),
+ *            §2.1 MLP 层的张量并行, §2.2 Self-Attention 的张量并行.
+ *   [TP-ILL] tensor-model-parallel illustrated (m.youleyou.com/wenzhang/3143730),
+ *            §1.1 按行切分权重, §1.2 按列切分权重, §2.1 MLP层的张量模型并行计算方法,
+ *            §3.1 Multihead-Attention的计算方法, §4.1 输入层Embedding,
+ *            §4.2 输出层Embedding, §5 Cross-Entropy层.
+ *   [APX]    "Megatron-LM 介绍" (apxml.com), §核心贡献 (column-parallel Y_i = X·A_i).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All matrices are dense ROW-MAJOR with no padding: X [M,h], A [h,F],
+ *    bias [F], B [F,h], Z [M,h] (the pages' math orientation, not the
+ *    [out,in] weight layout).  Shard i of A owns columns [off_i, off_{i+1});
+ *    shard i of B owns the same range of rows.
+ *  - shard_offsets: nullable int64 HOST array of N+1 increasing offsets with
+ *    off_0 = 0 and off_N = F.  NULL means the even split off_i = i*F/N, which
+ *    requires F % N == 0 (else TP_ERR_SHAPE).
+ *  - The CALLER OWNS EVERY BUFFER.  The library never allocates or frees
+ *    memory and never synchronises; all work is enqueued on `stream`
+ *    (a cudaStream_t, passed as void*; NULL = legacy default stream) and the
+ *    call returns before it completes.
+ *  - Argument errors are returned synchronously, before anything is
+ *    enqueued.  Errors found on the device (an id or target out of range, a
+ *    bounded wait that ran out) are OR-ed as TP_DEVERR_* bits into
+ *    *dev_status, an int32 in device memory (nullable); read it after the
+ *    stream has completed.
+ *  - bf16 tensors: base pointers 16-byte aligned and every row length a
+ *    multiple of 8 elements (the tensor-memory-accelerator copy rule);
+ *    fp32 tensors: 16-byte aligned, row lengths a multiple of 4.  Violations
+ *    return TP_ERR_ALIGN.
+ *  - bf16 storage, fp32 accumulation; every bf16 store rounds to nearest even.
+ *  - Thread safety: calls on different streams may overlap as long as they
+ *    do not share output or workspace buffers.
+ */
+#ifndef TPLAYERS_H_
+#define TPLAYERS_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TP_API __attribute__((visibility("default")))
+#else
+#define TP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t tp_status;
+
+enum {
+  TP_OK = 0,
+  TP_ERR_NULL = 1,        /* a required pointer is NULL */
+  TP_ERR_SHAPE = 2,       /* a size is <= 0, inconsistent, or not divisible as required */
+  TP_ERR_ALIGN = 3,       /* a pointer or row length breaks the alignment rules above */
+  TP_ERR_DTYPE = 4,       /* unknown dtype or activation code */
+  TP_ERR_UNSUPPORTED = 5, /* valid request this build does not implement */
+  TP_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed while enqueueing */
+  TP_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than tp_workspace_bytes() */
+  TP_ERR_DEVICE = 8       /* no usable sm_100 device is current */
+};
+
+/* Bits OR-ed into *dev_status by the kernels. */
+enum {
+  TP_DEVERR_RANGE = 1,    /* an embedding id or xent target outside [0, v) */
+  TP_DEVERR_TIMEOUT = 2   /* a bounded pipeline wait ran out; outputs are garbage */
+};
+
+typedef enum { TP_DTYPE_BF16 = 0, TP_DTYPE_F32 = 1 } tp_dtype;
+
+/* Activation of the column-parallel GEMM.  The pages name GeLU without a
+ * formula; GELU_TANH = 0.5·x·(1 + tanh(√(2/π)·(x + 0.044715·x³))) is the
+ * default, GELU_ERF = x·Φ(x). */
+typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU_TANH = 1, TP_ACT_GELU_ERF = 2 } tp_act;
+
+/* Operations whose workspace size tp_workspace_bytes() reports. */
+typedef enum {
+  TP_OP_MLP_FWD = 0,
+  TP_OP_MLP_BWD = 1,
+  TP_OP_ROW_LINEAR_FWD = 2,
+  TP_OP_COL_LINEAR_BWD = 3,
+  TP_OP_ROW_LINEAR_BWD = 4
+} tp_op;
+
+/* Human-readable text of a status code (static storage, never NULL). */
+TP_API const char* tp_status_string(tp_status s);
+
+/* Library version as 10000*major + 100*minor + patch. */
+TP_API int32_t tp_version(void);
+
+/*
+ * Workspace bytes an op needs for these sizes (M rows, h model width,
+ * F = ffn / output width, N shards).  For TP_OP_ROW_LINEAR_FWD pass
+ * (M, Nout, Kin, N).  Returns 0 when the op needs none.  The library
+ * clears the parts that must start at zero on every call.
+ */
+TP_API size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N);
+
+/*
+ * TP-MLP forward   [MLP-TP] §2.1 (formula and pseudocode); [TP-ILL] §2.1.
+ *
+ *   f forward is the identity: every shard reads the same X.
+ *   Shard i:  U_i = X·A_i + bias_i,  Y_i = act(U_i),  Z_i = Y_i·B_i.
+ *   g forward: Z = Σ_i Z_i (the all-reduce), fused on the device: the
+ *   row-parallel GEMM walks the shards' K ranges and sums them in its
+ *   accumulator or, in split mode, in a fixed-order epilogue reduction.
+ *
+ *   X    [M,h]   dt           in
+ *   A    [h,F]   dt           in   (column shards)
+ *   bias [F]     dt           in   nullable (= zero)
+ *   B    [F,h]   dt           in   (row shards)
+ *   U    [M,F]   dt           out  pre-activation, kept for backward
+ *   Y    [M,F]   dt           out  activation, kept for backward
+ *   Z    [M,h]   dt           out
+ *   Zpart [N,M,h] fp32        out  nullable: each shard's partial Z_i before
+ *                                  the sum (needs every off_i % 64 == 0 in bf16)
+ *   ws, ws_bytes                   workspace, >= tp_workspace_bytes(TP_OP_MLP_FWD, M, h, F, N)
+ *                                  (may be NULL when that is 0)
+ */
+TP_API tp_status tp_mlp_fwd(const void* X, const void* A, const void* bias, const void* B,
+                     int64_t M, int64_t h, int64_t F, int32_t N,
+                     const int64_t* shard_offsets, tp_dtype dt, tp_act act,
+                     void* U, void* Y, void* Z, float* Zpart,
+                     void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * TP-MLP backward   [TP-ILL] §1.1, §1.2, §2.1 (f and g backward).
+ *
+ *   g backward is the identity: dZ reaches every shard.
+ *   Shard i:  dU_i = (dZ·B_iᵀ) ⊙ act'(U_i)     (dGeLU fused in the epilogue)
+ *             dB_i = Y_iᵀ·dZ,  dA_i = Xᵀ·dU_i,  dbias_i = Σ_rows dU_i
+ *   f backward: dX = Σ_i dU_i·A_iᵀ (the all-reduce), fused like Z above.
+ *
+ *   X, A, B, U, Y, dZ   as in/out of the forward (U, Y from tp_mlp_fwd)
+ *   dU    [M,F] dt      out  (also the intermediate that dA and dX read)
+ *   dX    [M,h] dt      out
+ *   dA    [h,F] dt      out
+ *   dbias [F]   fp32    out  nullable
+ *   dB    [F,h] dt      out
+ *   ws, ws_bytes        >= tp_workspace_bytes(TP_OP_MLP_BWD, M, h, F, N)
+ */
+TP_API tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const void* U,
+                     const void* Y, const void* dZ,
+                     int64_t M, int64_t h, int64_t F, int32_t N,
+                     const int64_t* shard_offsets, tp_dtype dt, tp_act act,
+                     void* dU, void* dX, void* dA, float* dbias, void* dB,
+                     void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Column-parallel linear, forward   [TP-ILL] §1.2; [APX] §核心贡献; the QKV
+ * projection of [MLP-TP] §2.2 / [TP-ILL] §3.1 with per-shard heads.
+ *
+ *   U = X·W + bias, Y = act(U) over all N column shards of W in one launch.
+ *   X [M,K] in; W [K,Nout] in; bias [Nout] nullable; Y [M,Nout] out;
+ *   U [M,Nout] out, required unless act == TP_ACT_NONE (then may be NULL).
+ *   shard_offsets partition Nout (e.g. 3·64·heads_i for per-shard heads).
+ *   The shard boundaries do not change any value: a column split is exact.
+ */
+TP_API tp_status tp_col_linear_fwd(const void* X, const void* W, const void* bias,
+                            int64_t M, int64_t K, int64_t Nout, int32_t N,
+                            const int64_t* shard_offsets, tp_dtype dt, tp_act act,
+                            void* U, void* Y, int32_t* dev_status, void* stream);
+
+/*
+ * Column-parallel linear, backward   [TP-ILL] §1.2 (f backward sums the
+ * shards' dX partials).
+ *
+ *   dU = dY ⊙ act'(U) (dU may alias dY when act == NONE: then it is not
+ *   written); dW = Xᵀ·dU [K,Nout]; dbias = Σ_rows dU [Nout] fp32 (nullable);
+ *   dX = Σ_i dU_i·W_iᵀ [M,K].
+ */
+TP_API tp_status tp_col_linear_bwd(const void* X, const void* W, const void* U, const void* dY,
+                            int64_t M, int64_t K, int64_t Nout, int32_t N,
+                            const int64_t* shard_offsets, tp_dtype dt, tp_act act,
+                            void* dU, void* dX, void* dW, float* dbias,
+                            void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Row-parallel linear, forward   [TP-ILL] §1.1; the output projection of
+ * [MLP-TP] §2.2 followed by its all-reduce.
+ *
+ *   Z = Σ_i Xin[:, off_i:off_{i+1}]·W[off_i:off_{i+1}, :]   Xin [M,Kin],
+ *   W [Kin,Nout], Z [M,Nout] dt; Zpart [N,M,Nout] fp32 nullable as above.
+ */
+TP_API tp_status tp_row_linear_fwd(const void* Xin, const void* W,
+                            int64_t M, int64_t Kin, int64_t Nout, int32_t N,
+                            const int64_t* shard_offsets, tp_dtype dt,
+                            void* Z, float* Zpart,
+                            void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Row-parallel linear, backward   [TP-ILL] §1.1 (g backward is the identity).
+ *
+ *   dXin = dZ·Wᵀ [M,Kin] (each shard's columns are its own dX_i);
+ *   dW = Xinᵀ·dZ [Kin,Nout].
+ */
+TP_API tp_status tp_row_linear_bwd(const void* Xin, const void* W, const void* dZ,
+                            int64_t M, int64_t Kin, int64_t Nout, int32_t N,
+                            const int64_t* shard_offsets, tp_dtype dt,
+                            void* dXin, void* dW, int32_t* dev_status, void* stream);
+
+/*
+ * Vocabulary-parallel input embedding   [TP-ILL] §4.1.
+ *
+ *   The table E [v,h] is split into N contiguous row ranges
+ *   [i·v/N, (i+1)·v/N) (needs v % N == 0).  Shard i returns E[id] for the ids
+ *   in its range and a zero row otherwise; the N results are summed.  The
+ *   kernel forms that sum as an owner select: exactly one shard owns each
+ *   in-range id, so the sum is that shard's row (bit for bit, for every
+ *   value except -0.0, which the literal sum with +0.0 would turn into +0.0).
+ *   Ids outside [0, v) give a zero row and set TP_DEVERR_RANGE.
+ *
+ *   ids [T] int64 in (device); E [v,h] dt in; out [T,h] dt out.
+ */
+TP_API tp_status vp_embed(const int64_t* ids, int64_t T, const void* E, int64_t v, int64_t h,
+                   int32_t N, tp_dtype dt, void* out, int32_t* dev_status, void* stream);
+
+/*
+ * Output-embedding logits   [TP-ILL] §4.2 (the output layer shares the word
+ * embedding table): logits[:, lo_i:hi_i] = H·E_iᵀ for every vocabulary
+ * shard i, one launch, no gather (the blocks are written side by side).
+ *
+ *   H [T,h] bf16 in; E [v,h] bf16 in; logits [T,v] fp32 out.  v % N == 0.
+ */
+TP_API tp_status tp_logits_fwd(const void* H, const void* E, int64_t T, int64_t h, int64_t v,
+                        int32_t N, float* logits, int32_t* dev_status, void* stream);
+
+/*
+ * Vocabulary-parallel softmax cross-entropy   [TP-ILL] §5.
+ *
+ *   Row t of logits [T,v] fp32 is split into N contiguous vocabulary ranges
+ *   (v % N == 0).  Each shard computes its maximum m_i, its sum
+ *   s_i = Σ exp(l − m_i), its share of the target logit and its arg-max; the
+ *   shards combine m = max m_i, S = Σ s_i·exp(m_i − m) (the all-reduce of the
+ *   softmax denominators, with the maxima added for range safety) and
+ *
+ *     loss[t]    = log S + m − l[t, y_t]
+ *     dlogits    = grad_scale · (exp(l − m)/S − onehot(y_t))   (nullable)
+ *     argmax[t]  = lowest index of the row maximum (int32, nullable)
+ *     loss_sum   = Σ_t loss[t] in a fixed order (fp32 [1], nullable)
+ *
+ *   targets [T] int64 (device).  A target outside [0, v) sets
+ *   TP_DEVERR_RANGE, its loss is NaN and its dlogits row is NaN.
+ *   dlogits may alias logits (in-place gradient).
+ */
+TP_API tp_status vp_xent(const float* logits, const int64_t* targets, int64_t T, int64_t v,
+                  int32_t N, float grad_scale, float* loss, float* loss_sum,
+                  float* dlogits, int32_t* argmax, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPLAYERS_H_ */

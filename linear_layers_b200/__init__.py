@@ -1,0 +1,311 @@
+"""Megatron-style tensor-parallel layers on one B200 (sm_100a).
+
+Thin ctypes binding over ``libtplayers.so`` (declared in ``include/tplayers.h``).
+Every function here has the name of the C entry point it calls and does
+argument marshalling only: it reads sizes from the tensors' shapes,
+allocates missing outputs with torch (device memory is torch's job), passes
+raw device pointers and the current CUDA stream, and raises ``TPError`` on a
+non-zero status.  All arithmetic happens in the library's CUDA kernels; there
+is no CPU or PyTorch fallback, and importing a function whose library is
+missing fails loudly.
+
+The N tensor-parallel shards are partitions of the same device tensors:
+shard i of A owns columns [off_i, off_{i+1}), shard i of B the same rows,
+shard i of the vocabulary the rows [i·v/N, (i+1)·v/N) of E.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "TPError", "lib", "library_path", "ACT_NONE", "ACT_GELU_TANH", "ACT_GELU_ERF",
+    "tp_status_string", "tp_version", "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
+    "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
+    "vp_embed", "tp_logits_fwd", "vp_xent", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
+    "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
+]
+
+ACT_NONE, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
+DTYPE_BF16, DTYPE_F32 = 0, 1
+OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD = range(5)
+DEVERR_RANGE, DEVERR_TIMEOUT = 1, 2
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libtplayers.so")
+_lib = None
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+_SIGS = {
+    "tp_status_string": ([_I32], ctypes.c_char_p),
+    "tp_version": ([], _I32),
+    "tp_workspace_bytes": ([_I32, _I64, _I64, _I64, _I32], _SZ),
+    "tp_mlp_fwd": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
+                    _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
+    "tp_mlp_bwd": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
+                    _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
+    "tp_col_linear_fwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
+                           _P, _P, _P, _P], _I32),
+    "tp_col_linear_bwd": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
+                           _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
+    "tp_row_linear_fwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _SZ,
+                           _P, _P], _I32),
+    "tp_row_linear_bwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _P], _I32),
+    "vp_embed": ([_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P], _I32),
+    "tp_logits_fwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _P, _P], _I32),
+    "vp_xent": ([_P, _P, _I64, _I64, _I32, _F, _P, _P, _P, _P, _P, _P], _I32),
+}
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({_status_text(status)})")
+
+
+def lib():
+    """Load libtplayers.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(
+                f"{library_path} is missing: build it with `python -m linear_layers_b200.build`")
+        handle = ctypes.CDLL(library_path)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def _status_text(s: int) -> str:
+    try:
+        return lib().tp_status_string(int(s)).decode()
+    except Exception:  # pragma: no cover - library missing while formatting an error
+        return "?"
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise TPError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    if torch.device(device).type != "cuda":
+        raise RuntimeError("linear_layers_b200 runs on CUDA tensors only; there is no CPU path")
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _offsets(offsets, N):
+    if offsets is None:
+        return None, None
+    arr = (ctypes.c_int64 * (N + 1))(*[int(x) for x in offsets])
+    return arr, arr
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous (row-major, no padding)")
+
+
+def new_status(device="cuda") -> torch.Tensor:
+    """A zeroed int32 device word for the kernels' TP_DEVERR_* bits."""
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def tp_status_string(s: int) -> str:
+    return _status_text(s)
+
+
+def tp_version() -> int:
+    return int(lib().tp_version())
+
+
+def tp_workspace_bytes(op: int, M: int, h: int, F: int, N: int) -> int:
+    return int(lib().tp_workspace_bytes(int(op), int(M), int(h), int(F), int(N)))
+
+
+def _workspace(ws, op, M, h, F, N, device):
+    need = tp_workspace_bytes(op, M, h, F, N)
+    if ws is None and need > 0:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws, (0 if ws is None else ws.numel() * ws.element_size())
+
+
+def tp_mlp_fwd(X, A, bias, B, N, *, shard_offsets=None, act=ACT_GELU_TANH, U=None, Y=None,
+               Z=None, Zpart=None, ws=None, dev_status=None):
+    """Z = Σ_i act(X·A_i + bias_i)·B_i.  Returns (Z, U, Y)."""
+    M, h = X.shape
+    F = A.shape[1]
+    dev = X.device
+    U = torch.empty(M, F, dtype=X.dtype, device=dev) if U is None else U
+    Y = torch.empty(M, F, dtype=X.dtype, device=dev) if Y is None else Y
+    Z = torch.empty(M, h, dtype=X.dtype, device=dev) if Z is None else Z
+    _contig(X, A, bias, B, U, Y, Z, Zpart)
+    ws, wsb = _workspace(ws, OP_MLP_FWD, M, h, F, N, dev)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(bias), _ptr(B), M, h, F, N, offs, _dt(X),
+                            act, _ptr(U), _ptr(Y), _ptr(Z), _ptr(Zpart), _ptr(ws), wsb,
+                            _ptr(dev_status), _stream(dev)), "tp_mlp_fwd")
+    return Z, U, Y
+
+
+def tp_mlp_bwd(X, A, B, U, Y, dZ, N, *, shard_offsets=None, act=ACT_GELU_TANH, with_dbias=True,
+               dU=None, dX=None, dA=None, dbias=None, dB=None, ws=None, dev_status=None):
+    """Returns dict(dX, dA, dbias, dB, dU)."""
+    M, h = X.shape
+    F = A.shape[1]
+    dev = X.device
+    dt = X.dtype
+    dU = torch.empty(M, F, dtype=dt, device=dev) if dU is None else dU
+    dX = torch.empty(M, h, dtype=dt, device=dev) if dX is None else dX
+    dA = torch.empty(h, F, dtype=dt, device=dev) if dA is None else dA
+    dB = torch.empty(F, h, dtype=dt, device=dev) if dB is None else dB
+    if dbias is None and with_dbias:
+        dbias = torch.empty(F, dtype=torch.float32, device=dev)
+    _contig(X, A, B, U, Y, dZ, dU, dX, dA, dB, dbias)
+    ws, wsb = _workspace(ws, OP_MLP_BWD, M, h, F, N, dev)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_mlp_bwd(_ptr(X), _ptr(A), _ptr(B), _ptr(U), _ptr(Y), _ptr(dZ), M, h, F, N,
+                            offs, _dt(X), act, _ptr(dU), _ptr(dX), _ptr(dA), _ptr(dbias), _ptr(dB),
+                            _ptr(ws), wsb, _ptr(dev_status), _stream(dev)), "tp_mlp_bwd")
+    return {"dX": dX, "dA": dA, "dbias": dbias, "dB": dB, "dU": dU}
+
+
+def tp_col_linear_fwd(X, W, bias, N, *, shard_offsets=None, act=ACT_NONE, U=None, Y=None,
+                      dev_status=None):
+    """Y = act(X·W + bias) over all column shards.  Returns (Y, U) (U is None for act NONE
+    unless given)."""
+    M, K = X.shape
+    Nout = W.shape[1]
+    dev = X.device
+    if U is None and act != ACT_NONE:
+        U = torch.empty(M, Nout, dtype=X.dtype, device=dev)
+    Y = torch.empty(M, Nout, dtype=X.dtype, device=dev) if Y is None else Y
+    _contig(X, W, bias, U, Y)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_col_linear_fwd(_ptr(X), _ptr(W), _ptr(bias), M, K, Nout, N, offs, _dt(X),
+                                   act, _ptr(U), _ptr(Y), _ptr(dev_status), _stream(dev)),
+           "tp_col_linear_fwd")
+    return Y, U
+
+
+def tp_col_linear_bwd(X, W, U, dY, N, *, shard_offsets=None, act=ACT_NONE, with_dbias=True,
+                      dU=None, dX=None, dW=None, dbias=None, ws=None, dev_status=None):
+    """Returns dict(dX, dW, dbias, dU)."""
+    M, K = X.shape
+    Nout = W.shape[1]
+    dev = X.device
+    dt = X.dtype
+    if dU is None and act != ACT_NONE:
+        dU = torch.empty(M, Nout, dtype=dt, device=dev)
+    dX = torch.empty(M, K, dtype=dt, device=dev) if dX is None else dX
+    dW = torch.empty(K, Nout, dtype=dt, device=dev) if dW is None else dW
+    if dbias is None and with_dbias:
+        dbias = torch.empty(Nout, dtype=torch.float32, device=dev)
+    _contig(X, W, U, dY, dU, dX, dW, dbias)
+    ws, wsb = _workspace(ws, OP_COL_LINEAR_BWD, M, K, Nout, N, dev)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_col_linear_bwd(_ptr(X), _ptr(W), _ptr(U), _ptr(dY), M, K, Nout, N, offs,
+                                   _dt(X), act, _ptr(dU), _ptr(dX), _ptr(dW), _ptr(dbias),
+                                   _ptr(ws), wsb, _ptr(dev_status), _stream(dev)),
+           "tp_col_linear_bwd")
+    return {"dX": dX, "dW": dW, "dbias": dbias, "dU": dU if dU is not None else dY}
+
+
+def tp_row_linear_fwd(Xin, W, N, *, shard_offsets=None, Z=None, Zpart=None, ws=None,
+                      dev_status=None):
+    """Z = Σ_i Xin_i·W_i.  Returns Z."""
+    M, Kin = Xin.shape
+    Nout = W.shape[1]
+    dev = Xin.device
+    Z = torch.empty(M, Nout, dtype=Xin.dtype, device=dev) if Z is None else Z
+    _contig(Xin, W, Z, Zpart)
+    ws, wsb = _workspace(ws, OP_ROW_LINEAR_FWD, M, Nout, Kin, N, dev)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_row_linear_fwd(_ptr(Xin), _ptr(W), M, Kin, Nout, N, offs, _dt(Xin), _ptr(Z),
+                                   _ptr(Zpart), _ptr(ws), wsb, _ptr(dev_status), _stream(dev)),
+           "tp_row_linear_fwd")
+    return Z
+
+
+def tp_row_linear_bwd(Xin, W, dZ, N, *, shard_offsets=None, dXin=None, dW=None, dev_status=None):
+    """Returns dict(dXin, dW)."""
+    M, Kin = Xin.shape
+    Nout = W.shape[1]
+    dev = Xin.device
+    dXin = torch.empty(M, Kin, dtype=Xin.dtype, device=dev) if dXin is None else dXin
+    dW = torch.empty(Kin, Nout, dtype=Xin.dtype, device=dev) if dW is None else dW
+    _contig(Xin, W, dZ, dXin, dW)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_row_linear_bwd(_ptr(Xin), _ptr(W), _ptr(dZ), M, Kin, Nout, N, offs, _dt(Xin),
+                                   _ptr(dXin), _ptr(dW), _ptr(dev_status), _stream(dev)),
+           "tp_row_linear_bwd")
+    return {"dXin": dXin, "dW": dW}
+
+
+def vp_embed(ids, E, N, *, out=None, dev_status=None):
+    """out[t] = E[ids[t]] through the vocabulary shards (zero row for ids outside [0, v))."""
+    T = ids.shape[0]
+    v, h = E.shape
+    dev = E.device
+    out = torch.empty(T, h, dtype=E.dtype, device=dev) if out is None else out
+    _contig(ids, E, out)
+    if ids.dtype != torch.int64:
+        raise TypeError("ids must be int64")
+    _check(lib().vp_embed(_ptr(ids), T, _ptr(E), v, h, N, _dt(E), _ptr(out), _ptr(dev_status),
+                          _stream(dev)), "vp_embed")
+    return out
+
+
+def tp_logits_fwd(H, E, N, *, logits=None, dev_status=None):
+    """logits [T, v] fp32 = H·Eᵀ, written shard block by shard block."""
+    T, h = H.shape
+    v = E.shape[0]
+    dev = H.device
+    logits = torch.empty(T, v, dtype=torch.float32, device=dev) if logits is None else logits
+    _contig(H, E, logits)
+    _check(lib().tp_logits_fwd(_ptr(H), _ptr(E), T, h, v, N, _ptr(logits), _ptr(dev_status),
+                               _stream(dev)), "tp_logits_fwd")
+    return logits
+
+
+def vp_xent(logits, targets, N, *, grad_scale=1.0, with_grad=True, with_argmax=True,
+            loss=None, loss_sum=None, dlogits=None, argmax=None, dev_status=None):
+    """Returns dict(loss [T], loss_sum [1], dlogits [T,v] or None, argmax [T] or None)."""
+    T, v = logits.shape
+    dev = logits.device
+    loss = torch.empty(T, dtype=torch.float32, device=dev) if loss is None else loss
+    loss_sum = torch.empty(1, dtype=torch.float32, device=dev) if loss_sum is None else loss_sum
+    if with_grad and dlogits is None:
+        dlogits = torch.empty_like(logits)
+    if with_argmax and argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=dev)
+    _contig(logits, targets, loss, dlogits, argmax)
+    if targets.dtype != torch.int64:
+        raise TypeError("targets must be int64")
+    _check(lib().vp_xent(_ptr(logits), _ptr(targets), T, v, N, float(grad_scale), _ptr(loss),
+                         _ptr(loss_sum), _ptr(dlogits), _ptr(argmax), _ptr(dev_status),
+                         _stream(dev)), "vp_xent")
+    return {"loss": loss, "loss_sum": loss_sum, "dlogits": dlogits, "argmax": argmax}

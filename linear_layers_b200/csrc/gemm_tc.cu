@@ -1,0 +1,670 @@
+// gemm_tc.cu — persistent, warp-specialised bf16 GEMM engine for sm_100a.
+//
+// Every contraction of the tensor-parallel layers runs through this kernel:
+// the column-parallel GEMM with its bias + GeLU epilogue, the row-parallel
+// GEMM whose shard sum (the g operator's all-reduce, and the f operator's in
+// backward) is fused into the accumulator or into an ordered split
+// reduction, the dGeLU GEMM, the two weight-gradient GEMMs and the
+// output-embedding logits GEMM.
+//
+// Structure of one CTA (one per SM, persistent over output tiles):
+//   warp 0   TMA producer: one elected lane streams A and B k-blocks
+//            (64 bf16 of K) into a ring of shared-memory stages;
+//   warp 1   owns tensor memory (512 columns = two 128x256 fp32
+//            accumulators) and one elected lane issues tcgen05.mma;
+//   warps 2-5 epilogue: tcgen05.ld of the finished accumulator, the fused
+//            element-wise work, stores to global memory.
+// The accumulator is double buffered, so the epilogue of tile t overlaps
+// the main loop of tile t+1.  Tiles are 128 x BN with BN = 256.
+//
+// Operands may be K-major or MN-major in global memory; both are loaded by
+// TMA with 128-byte swizzle and described to the tensor core by matching
+// shared-memory descriptors, so no operand is ever transposed in memory.
+// No TMA load uses cluster multicast.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <cuda_bf16.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "sm100_ptx.cuh"
+
+namespace tpl {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;              // bf16 elements per k-block (= one 128-byte swizzle row)
+constexpr int kThreads = 192;       // 6 warps
+constexpr int kEpiThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+
+struct GemmArgs {
+  int M, N, K;
+  int a_mn, b_mn;
+  int tiles_m, tiles_n, splits, group_m;
+  int num_units;
+  int split_kb[kMaxSplits + 1];     // k-block boundaries of the splits
+  int epi, act;
+  void* out0;
+  void* out1;
+  int64_t ldo;
+  const __nv_bfloat16* bias;
+  const __nv_bfloat16* aux;
+  int64_t ld_aux;
+  float* dbias_part;
+  float* part;                      // split partials: zpart [splits,M,N] or tile-chunk buffer
+  int part_is_zpart;
+  int* counters;
+  int32_t* dev_status;
+  uint64_t wait_ns;
+};
+
+struct __align__(64) GemmParams {
+  CUtensorMap tmA;
+  CUtensorMap tmB;
+  GemmArgs a;
+};
+
+// -------------------------------------------------------------------------
+// activation (no page gives a formula: tanh closed form by default)
+// 0.5·u·(1 + tanh(z)) is written as u·σ(2z), which stays accurate in the
+// negative tail where 1 + tanh(z) cancels.
+// -------------------------------------------------------------------------
+__device__ __forceinline__ float act_apply(float u, int act) {
+  if (act == TP_ACT_GELU_TANH) {
+    const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);
+    return __fdividef(u, 1.0f + __expf(-2.0f * z));
+  }
+  if (act == TP_ACT_GELU_ERF) {
+    return 0.5f * u * (1.0f + erff(u * 0.7071067811865476f));
+  }
+  return u;
+}
+
+__device__ __forceinline__ float act_deriv(float u, int act) {
+  if (act == TP_ACT_GELU_TANH) {
+    const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);
+    const float s = __fdividef(1.0f, 1.0f + __expf(-2.0f * z));
+    const float dz = 0.7978845608028654f * (1.0f + 3.0f * 0.044715f * u * u);
+    return s + 2.0f * u * s * (1.0f - s) * dz;
+  }
+  if (act == TP_ACT_GELU_ERF) {
+    const float cdf = 0.5f * (1.0f + erff(u * 0.7071067811865476f));
+    return cdf + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  }
+  return 1.0f;
+}
+
+// -------------------------------------------------------------------------
+// tile scheduling: unit -> (tile row, tile column, split)
+// Tiles are visited in bands of group_m tile rows, column by column inside a
+// band, so that one wave of CTAs shares A rows and B columns through L2.
+// The splits of one tile are adjacent units, so their partials meet in L2.
+// -------------------------------------------------------------------------
+__device__ __forceinline__ void unit_map(const GemmArgs& a, int unit, int& tm, int& tn, int& s,
+                                         int& tile) {
+  s = unit % a.splits;
+  tile = unit / a.splits;
+  const int per_group = a.group_m * a.tiles_n;
+  const int g = tile / per_group;
+  const int first_m = g * a.group_m;
+  const int gm = min(a.tiles_m - first_m, a.group_m);
+  const int r = tile - g * per_group;
+  tm = first_m + r % gm;
+  tn = r / gm;
+}
+
+__device__ __forceinline__ void flag_timeout(const GemmArgs& a, volatile int* abort_flag) {
+  *abort_flag = 1;
+  if (a.dev_status) atomicOr(a.dev_status, TP_DEVERR_TIMEOUT);
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v, int ncols_left) {
+  // ncols_left is a multiple of 8 (row lengths are multiples of 8)
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (8 * j < ncols_left) {
+      uint4 w;
+      w.x = pack_bf16x2(v[8 * j + 0], v[8 * j + 1]);
+      w.y = pack_bf16x2(v[8 * j + 2], v[8 * j + 3]);
+      w.z = pack_bf16x2(v[8 * j + 4], v[8 * j + 5]);
+      w.w = pack_bf16x2(v[8 * j + 6], v[8 * j + 7]);
+      *reinterpret_cast<uint4*>(dst + 8 * j) = w;
+    }
+  }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v, int ncols_left) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (8 * j < ncols_left) w = __ldg(reinterpret_cast<const uint4*>(src + 8 * j));
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&ww[q]);
+      float2 f = __bfloat1622float2(b);
+      v[8 * j + 2 * q] = f.x;
+      v[8 * j + 2 * q + 1] = f.y;
+    }
+  }
+}
+
+// Transpose-reduce across the warp: lane l ends with Σ_lanes v[l].
+__device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {
+    const bool upper = (lane & off) != 0;
+#pragma unroll
+    for (int i = 0; i < off; ++i) {
+      const float send = upper ? v[i] : v[i + off];
+      const float keep = upper ? v[i + off] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+    }
+  }
+  return v[0];
+}
+
+template <int BN, int STAGES>
+struct SmemLayout {
+  static constexpr uint32_t kABytes = BM * BK * 2;
+  static constexpr uint32_t kBBytes = BN * BK * 2;
+  static constexpr uint32_t kOffB = STAGES * kABytes;
+  static constexpr uint32_t kOffBar = kOffB + STAGES * kBBytes;
+  static constexpr uint32_t kNumBars = 2 * STAGES + 5;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;
+  static constexpr uint32_t kBytes = kOffRed + 4 * BN * 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
+};
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
+  using L = SmemLayout<BN, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const GemmArgs& a = P.a;
+
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::kOffB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* mma_done = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
+  volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
+  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&tfull[s], 1);
+      mbar_init(&tempty[s], kEpiThreads);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (elect_one_sync()) {
+      tma_prefetch_desc(&P.tmA);
+      tma_prefetch_desc(&P.tmB);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int unit = blockIdx.x; ok && unit < a.num_units; unit += gridDim.x) {
+        int tm, tn, s, tile;
+        unit_map(a, unit, tm, tn, s, tile);
+        for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
+            if (!*abort_flag) flag_timeout(a, abort_flag);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], L::kABytes + L::kBBytes);
+          const int k0 = kb * BK;
+          uint8_t* dA = sA + stage * L::kABytes;
+          uint8_t* dB = sB + stage * L::kBBytes;
+          if (!a.a_mn) {
+            tma_load_2d(dA, &P.tmA, &full[stage], k0, tm * BM);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BM / 64; ++j)
+              tma_load_2d(dA + j * 8192, &P.tmA, &full[stage], tm * BM + j * 64, k0);
+          }
+          if (!a.b_mn) {
+            tma_load_2d(dB, &P.tmB, &full[stage], k0, tn * BN);
+          } else {
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+              tma_load_2d(dB + j * 8192, &P.tmB, &full[stage], tn * BN + j * 64, k0);
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Let every copy this thread started land before the CTA can exit
+      // (bounded in time, but not cut short by the abort flag).
+      volatile int keep_waiting = 0;
+      const int inflight = issued < STAGES ? issued : STAGES;
+      for (int i = 0; i < inflight; ++i) {
+        if (--stage < 0) {
+          stage = STAGES - 1;
+          phase ^= 1u;
+        }
+        mbar_wait_bounded(&full[stage], phase, a.wait_ns, &keep_waiting);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one_sync()) {
+      const uint32_t idesc = idesc_bf16_f32(BM, BN, a.a_mn != 0, a.b_mn != 0);
+      const uint32_t a_lbo = a.a_mn ? 8192u : 16u;
+      const uint32_t b_lbo = a.b_mn ? 8192u : 16u;
+      const uint32_t a_kstep = a.a_mn ? 2048u : 32u;   // bytes per 16-element K step
+      const uint32_t b_kstep = a.b_mn ? 2048u : 32u;
+      int stage = 0;
+      uint32_t phase = 0;
+      int t = 0;
+      bool ok = true, any = false;
+      for (int unit = blockIdx.x; ok && unit < a.num_units; unit += gridDim.x, ++t) {
+        int tm, tn, s, tile;
+        unit_map(a, unit, tm, tn, s, tile);
+        const int acc = t & 1;
+        const uint32_t use = static_cast<uint32_t>(t >> 1);
+        if (!mbar_wait_bounded(&tempty[acc], (use & 1u) ^ 1u, a.wait_ns, abort_flag)) {
+          if (!*abort_flag) flag_timeout(a, abort_flag);
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const int kb0 = a.split_kb[s], kb1 = a.split_kb[s + 1];
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
+            if (!*abort_flag) flag_timeout(a, abort_flag);
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t a_base = smem_u32(sA + stage * L::kABytes);
+          const uint32_t b_base = smem_u32(sB + stage * L::kBBytes);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            const uint64_t adesc = smem_desc_sw128(a_base + k * a_kstep, a_lbo, 1024);
+            const uint64_t bdesc = smem_desc_sw128(b_base + k * b_kstep, b_lbo, 1024);
+            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          }
+          any = true;
+          tc_commit(&empty[stage]);   // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) tc_commit(&tfull[acc]);   // accumulator ready for the epilogue
+      }
+      if (any) {   // every issued MMA must finish before tensor memory is freed
+        volatile int keep_waiting = 0;
+        tc_commit(mma_done);
+        mbar_wait_bounded(mma_done, 0, a.wait_ns, &keep_waiting);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;               // TMEM lane quadrant this warp may access
+    const int row_in_tile = q * 32 + lane;
+    const int et = threadIdx.x - 64;      // 0..127 among the epilogue threads
+    int t = 0;
+    for (int unit = blockIdx.x; unit < a.num_units; unit += gridDim.x, ++t) {
+      int tm, tn, s, tile;
+      unit_map(a, unit, tm, tn, s, tile);
+      const int acc = t & 1;
+      const uint32_t use = static_cast<uint32_t>(t >> 1);
+      const bool got = mbar_wait_bounded(&tfull[acc], use & 1u, a.wait_ns, abort_flag);
+      // all 128 epilogue threads leave together or go on together, so no
+      // warp can be left waiting in a later named barrier
+      if (!named_barrier_and(1, kEpiThreads, got)) {
+        if (et == 0 && !*abort_flag) flag_timeout(a, abort_flag);
+        break;
+      }
+      tc_fence_after_sync();
+      const int row = tm * BM + row_in_tile;
+      const bool row_ok = row < a.M;
+      const uint32_t t_base =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+
+      if (a.epi == EPI_SPLIT_SUM) {
+        // 1) publish this split's fp32 partial
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tc_wait_ld();
+          const int col0 = tn * BN + c * 32;
+          if (a.part_is_zpart) {
+            if (row_ok) {
+              float* dst = a.part + (static_cast<int64_t>(s) * a.M + row) * a.N + col0;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (col0 + 4 * j < a.N)
+                  __stcg(reinterpret_cast<float4*>(dst + 4 * j),
+                         make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+            }
+          } else {
+            float* dst = a.part +
+                         ((static_cast<int64_t>(tile) * a.splits + s) * (BN / 32) + c) * (BM * 32) +
+                         row_in_tile * 32;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              __stcg(reinterpret_cast<float4*>(dst + 4 * j),
+                     make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                 __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+          }
+        }
+        __threadfence();
+        named_barrier_sync(1, kEpiThreads);
+        if (et == 0) {
+          const int prev = atomicAdd(&a.counters[tile], 1);
+          const int last = (prev == a.splits - 1);
+          if (last) a.counters[tile] = 0;   // ready for the next call
+          *bcast = last;
+        }
+        named_barrier_sync(1, kEpiThreads);
+        const bool last = *bcast != 0;
+        if (last) {
+          __threadfence();
+          // 2) the last split of this tile sums all partials in split order
+#pragma unroll 1
+          for (int c = 0; c < BN / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_base + c * 32, r);
+            tc_wait_ld();
+            const int col0 = tn * BN + c * 32;
+            float sum[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
+            for (int ss = 0; ss < a.splits; ++ss) {
+              float p[32];
+              if (ss == s) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) p[j] = __uint_as_float(r[j]);
+              } else if (a.part_is_zpart) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) p[j] = 0.0f;
+                if (row_ok) {
+                  const float* src = a.part + (static_cast<int64_t>(ss) * a.M + row) * a.N + col0;
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    if (col0 + 4 * j < a.N) {
+                      const float4 f = __ldcg(reinterpret_cast<const float4*>(src + 4 * j));
+                      p[4 * j] = f.x; p[4 * j + 1] = f.y; p[4 * j + 2] = f.z; p[4 * j + 3] = f.w;
+                    }
+                }
+              } else {
+                const float* src =
+                    a.part +
+                    ((static_cast<int64_t>(tile) * a.splits + ss) * (BN / 32) + c) * (BM * 32) +
+                    row_in_tile * 32;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 f = __ldcg(reinterpret_cast<const float4*>(src + 4 * j));
+                  p[4 * j] = f.x; p[4 * j + 1] = f.y; p[4 * j + 2] = f.z; p[4 * j + 3] = f.w;
+                }
+              }
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sum[j] += p[j];
+            }
+            if (row_ok && col0 < a.N)
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, sum,
+                            a.N - col0);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = tn * BN + c * 32;
+          float aux_v[32];
+          if (a.epi == EPI_DACT) {
+            if (row_ok && col0 < a.N) {
+              load_bf16x32(a.aux + row * a.ld_aux + col0, aux_v, a.N - col0);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) aux_v[j] = 0.0f;
+            }
+          }
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tc_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          const bool store_ok = row_ok && col0 < a.N;
+
+          if (a.epi == EPI_STORE_BF16) {
+            if (store_ok)
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
+                            a.N - col0);
+          } else if (a.epi == EPI_STORE_F32) {
+            if (store_ok) {
+              float* dst = static_cast<float*>(a.out0) + row * a.ldo + col0;
+#pragma unroll
+              for (int j = 0; j < 8; ++j)
+                if (col0 + 4 * j < a.N)
+                  *reinterpret_cast<float4*>(dst + 4 * j) =
+                      make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+            }
+          } else if (a.epi == EPI_BIAS_ACT) {
+            if (a.bias != nullptr && col0 < a.N) {
+              float b[32];
+              load_bf16x32(a.bias + col0, b, a.N - col0);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] += b[j];
+            }
+            if (store_ok && a.out0 != nullptr)
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
+                            a.N - col0);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+            if (store_ok)
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
+                            a.N - col0);
+          } else {  // EPI_DACT
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = store_ok ? v[j] * act_deriv(aux_v[j], a.act) : 0.0f;
+            if (store_ok)
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
+                            a.N - col0);
+            if (a.dbias_part != nullptr) {
+              const float colsum = warp_column_sums(v, lane);
+              red[q * BN + c * 32 + lane] = colsum;
+            }
+          }
+        }
+        if (a.epi == EPI_DACT && a.dbias_part != nullptr) {
+          named_barrier_sync(1, kEpiThreads);
+          for (int cc = et; cc < BN; cc += kEpiThreads) {
+            const int col = tn * BN + cc;
+            // fixed order over the four row quarters of the tile
+            const float sum = ((red[cc] + red[BN + cc]) + red[2 * BN + cc]) + red[3 * BN + cc];
+            if (col < a.N) a.dbias_part[static_cast<int64_t>(tm) * a.N + col] = sum;
+          }
+          named_barrier_sync(1, kEpiThreads);
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+// -------------------------------------------------------------------------
+// host side
+// -------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major bf16 matrix [outer, inner] with row stride ld (elements); box of
+// box_inner x box_outer elements, 128-byte swizzle, zero fill outside.
+bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+               uint32_t box_inner, uint32_t box_outer) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int BN, int STAGES>
+tp_status launch_impl(const GemmParams& prm, int grid, cudaStream_t stream) {
+  using L = SmemLayout<BN, STAGES>;
+  static_assert(L::kAlloc <= 232448, "shared memory budget");
+  static int configured_device = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured_device != dev) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+      return TP_ERR_CUDA;
+    configured_device = dev;
+  }
+  gemm_tc_kernel<BN, STAGES><<<grid, kThreads, L::kAlloc, stream>>>(prm);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+
+}  // namespace
+
+size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
+  if (splits <= 1) return 0;
+  const size_t tiles = static_cast<size_t>((M + BM - 1) / BM) * ((N + kBN - 1) / kBN);
+  size_t bytes = with_zpart ? 0 : tiles * splits * BM * kBN * sizeof(float);
+  bytes += tiles * sizeof(int);
+  return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0) return TP_ERR_SHAPE;
+  if (p.splits < 1 || p.splits > kMaxSplits) return TP_ERR_SHAPE;
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  GemmArgs& a = prm.a;
+  a.M = p.M;
+  a.N = p.N;
+  a.K = p.K;
+  a.a_mn = p.a_mn;
+  a.b_mn = p.b_mn;
+  a.tiles_m = (p.M + BM - 1) / BM;
+  a.tiles_n = (p.N + kBN - 1) / kBN;
+  a.splits = p.splits;
+  a.group_m = 16;
+  const int kblocks = (p.K + BK - 1) / BK;
+  if (p.splits == 1) {
+    a.split_kb[0] = 0;
+    a.split_kb[1] = kblocks;
+  } else {
+    for (int s = 0; s <= p.splits; ++s) {
+      const int k = p.split_k[s];
+      if (s > 0 && s < p.splits && (k % BK) != 0) return TP_ERR_UNSUPPORTED;
+      a.split_kb[s] = (k + BK - 1) / BK;
+      if (s > 0 && a.split_kb[s] <= a.split_kb[s - 1]) return TP_ERR_SHAPE;
+    }
+    if (p.split_k[0] != 0 || p.split_k[p.splits] != p.K) return TP_ERR_SHAPE;
+  }
+  a.num_units = a.tiles_m * a.tiles_n * a.splits;
+  a.epi = p.splits > 1 ? EPI_SPLIT_SUM : p.epi;
+  a.act = p.act;
+  a.out0 = p.out0;
+  a.out1 = p.out1;
+  a.ldo = p.ldo;
+  a.bias = static_cast<const __nv_bfloat16*>(p.bias);
+  a.aux = static_cast<const __nv_bfloat16*>(p.aux);
+  a.ld_aux = p.ld_aux;
+  a.dbias_part = p.dbias_part;
+  a.dev_status = p.dev_status;
+  a.wait_ns = wait_limit_ns();
+  if (p.splits > 1) {
+    const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
+    if (p.ws == nullptr || p.ws_bytes < need) return TP_ERR_WORKSPACE;
+    const size_t tiles = static_cast<size_t>(a.tiles_m) * a.tiles_n;
+    if (p.zpart) {
+      a.part = p.zpart;
+      a.part_is_zpart = 1;
+      a.counters = static_cast<int*>(p.ws);
+    } else {
+      a.part = static_cast<float*>(p.ws);
+      a.part_is_zpart = 0;
+      a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(p.ws) +
+                                          tiles * p.splits * BM * kBN * sizeof(float));
+    }
+    if (cudaMemsetAsync(a.counters, 0, tiles * sizeof(int), stream) != cudaSuccess)
+      return TP_ERR_CUDA;
+  }
+  // operand maps
+  bool ok;
+  if (!p.a_mn)
+    ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, BM);
+  else
+    ok = make_tmap(&prm.tmA, p.A, p.M, p.K, p.lda, 64, BK);
+  if (!ok) return TP_ERR_CUDA;
+  if (!p.b_mn)
+    ok = make_tmap(&prm.tmB, p.B, p.K, p.N, p.ldb, BK, kBN);
+  else
+    ok = make_tmap(&prm.tmB, p.B, p.N, p.K, p.ldb, 64, BK);
+  if (!ok) return TP_ERR_CUDA;
+  const int grid = a.num_units < num_sms() ? a.num_units : num_sms();
+  return launch_impl<kBN, kStages>(prm, grid, stream);
+}
+
+}  // namespace tpl

@@ -1,0 +1,70 @@
+// internal.h — declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstdint>
+#include <cstddef>
+
+#include "../../include/tplayers.h"
+
+namespace tpl {
+
+constexpr int kMaxSplits = 16;   // K splits of one row-parallel GEMM (and shards with Zpart)
+
+enum EpiKind : int {
+  EPI_STORE_BF16 = 0,   // out0 = bf16(acc)
+  EPI_BIAS_ACT = 1,     // U = acc + bias; Y = act(U); out0 = U (nullable), out1 = Y
+  EPI_DACT = 2,         // dU = acc ⊙ act'(aux); out0 = dU; per-tile column sums of dU
+  EPI_STORE_F32 = 3,    // out0 = acc (fp32)
+  EPI_SPLIT_SUM = 4     // fp32 partial per split; the last split of a tile sums them
+                        // in split order and stores bf16 to out0
+};
+
+// C[M,N] = A[M,K] · B[K,N] with the operands in one of two storages each:
+//   A: a_mn == 0  ->  A stored [M,K] row-major (lda >= K)      (K-major)
+//      a_mn == 1  ->  A stored [K,M] row-major (lda >= M)      (MN-major)
+//   B: b_mn == 0  ->  B stored [N,K] row-major (ldb >= K)      (K-major)
+//      b_mn == 1  ->  B stored [K,N] row-major (ldb >= N)      (MN-major)
+struct GemmProblem {
+  const void* A = nullptr;
+  const void* B = nullptr;
+  int64_t lda = 0, ldb = 0;
+  int a_mn = 0, b_mn = 0;
+  int M = 0, N = 0, K = 0;
+  int epi = EPI_STORE_BF16;
+  void* out0 = nullptr;
+  void* out1 = nullptr;
+  int64_t ldo = 0;
+  const void* bias = nullptr;      // EPI_BIAS_ACT (bf16 [N]) nullable
+  const void* aux = nullptr;       // EPI_DACT: U (bf16, row stride ld_aux)
+  int64_t ld_aux = 0;
+  float* dbias_part = nullptr;     // EPI_DACT: [ceil(M/128), N] fp32, nullable
+  int act = TP_ACT_NONE;
+  // EPI_SPLIT_SUM
+  int splits = 1;
+  int split_k[kMaxSplits + 1] = {0};   // K offsets of the splits (multiples of 64)
+  float* zpart = nullptr;          // nullable [splits, M, N] fp32: partials land here
+  void* ws = nullptr;              // partial buffer + tile counters (see gemm_ws_bytes)
+  size_t ws_bytes = 0;
+  int32_t* dev_status = nullptr;
+};
+
+// Workspace a split GEMM needs: fp32 partial tiles (unless zpart carries
+// them) plus one int counter per output tile.
+size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart);
+
+tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream);
+
+// fp32 SIMT path (same problem description; operands fp32).
+tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream);
+
+// Column sums of the per-tile dbias partials: dbias[n] = Σ_t part[t, n].
+tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
+                              cudaStream_t stream);
+
+// Device checks shared by the entry points.
+tp_status require_sm100();
+int num_sms();
+uint64_t wait_limit_ns();
+
+}  // namespace tpl
