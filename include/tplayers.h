@@ -100,6 +100,11 @@ TP_API const char* tp_status_string(tp_status s);
 /* Library version as 10000*major + 100*minor + patch. */
 TP_API int32_t tp_version(void);
 
+/* Number of kernels this library has enqueued since it was loaded (all
+ * devices, all threads).  Diagnostics only: lets a caller count the
+ * library's launches inside a timed region. */
+TP_API uint64_t tp_launch_count(void);
+
 /*
  * Workspace bytes an op needs for these sizes (M rows, h model width,
  * F = ffn / output width, N shards).  For TP_OP_ROW_LINEAR_FWD pass

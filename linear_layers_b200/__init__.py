@@ -22,7 +22,7 @@ import torch
 
 __all__ = [
     "TPError", "lib", "library_path", "ACT_NONE", "ACT_GELU_TANH", "ACT_GELU_ERF",
-    "tp_status_string", "tp_version", "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
+    "tp_status_string", "tp_version", "tp_launch_count", "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
     "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
     "vp_embed", "tp_logits_fwd", "vp_xent", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
@@ -46,6 +46,7 @@ _F = ctypes.c_float
 _SIGS = {
     "tp_status_string": ([_I32], ctypes.c_char_p),
     "tp_version": ([], _I32),
+    "tp_launch_count": ([], ctypes.c_uint64),
     "tp_workspace_bytes": ([_I32, _I64, _I64, _I64, _I32], _SZ),
     "tp_mlp_fwd": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                     _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
@@ -140,6 +141,11 @@ def tp_status_string(s: int) -> str:
 
 def tp_version() -> int:
     return int(lib().tp_version())
+
+
+def tp_launch_count() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(lib().tp_launch_count())
 
 
 def tp_workspace_bytes(op: int, M: int, h: int, F: int, N: int) -> int:

@@ -195,6 +195,7 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream) {
     a.k0 = 0;
     a.k1 = p.K;
     gemm_simt_kernel<<<grid, block, 0, stream>>>(a);
+    note_launches(1);
     return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
   }
   // per-split partials into zpart (required here), then an ordered sum
@@ -208,10 +209,12 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream) {
     a.k0 = p.split_k[s];
     a.k1 = p.split_k[s + 1];
     gemm_simt_kernel<<<grid, block, 0, stream>>>(a);
+    note_launches(1);
   }
   const int blocks = static_cast<int>((count + 255) / 256 < 4096 ? (count + 255) / 256 : 4096);
   sum_splits_kernel<<<blocks, 256, 0, stream>>>(p.zpart, p.splits, count,
                                                  static_cast<float*>(p.out0));
+  note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
@@ -226,12 +229,14 @@ tp_status dact_colsum_launch(const void* dY, const void* U, int64_t M, int64_t N
     dact_colsum_kernel<float><<<grid, 256, 0, stream>>>(static_cast<const float*>(dY),
                                                         static_cast<const float*>(U), M, Nout, act,
                                                         static_cast<float*>(dU), dbias_part);
+  note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
                               cudaStream_t stream) {
   dbias_finish_kernel<<<(N + 255) / 256, 256, 0, stream>>>(part, tiles, N, dbias);
+  note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 

@@ -578,6 +578,7 @@ tp_status launch_impl(const GemmParams& prm, int grid, cudaStream_t stream) {
     configured_device = dev;
   }
   gemm_tc_kernel<BN, STAGES><<<grid, kThreads, L::kAlloc, stream>>>(prm);
+  note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 

@@ -62,6 +62,9 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream);
 tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
                               cudaStream_t stream);
 
+// Counts every kernel the library enqueues (tp_launch_count).
+void note_launches(int n);
+
 // Device checks shared by the entry points.
 tp_status require_sm100();
 int num_sms();

@@ -7,6 +7,7 @@
 // synchronises.
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -199,6 +200,10 @@ std::once_flag g_wait_once;
 
 }  // namespace
 
+std::atomic<uint64_t> g_launches{0};
+
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
+
 int num_sms() { return sms_or_default(); }
 
 uint64_t wait_limit_ns() {
@@ -240,6 +245,8 @@ const char* tp_status_string(tp_status s) {
 }
 
 int32_t tp_version(void) { return 100; }
+
+uint64_t tp_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) {
   if (M <= 0 || h <= 0 || F <= 0 || N < 1) return 0;

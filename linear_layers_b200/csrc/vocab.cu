@@ -342,6 +342,7 @@ tp_status vp_embed_launch(const int64_t* ids, int64_t T, const void* E, int64_t 
   vp_embed_kernel<<<static_cast<unsigned>(blocks), kEmbedWarps * 32, 0, stream>>>(
       ids, T, static_cast<const uint4*>(E), v, vec_per_row, v / N, static_cast<uint4*>(out),
       dev_status);
+  note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
@@ -379,13 +380,16 @@ tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T,
     if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel, logits, targets, v, static_cast<int>(vs),
                            grad_scale, loss, dlogits, argmax, dev_status) != cudaSuccess)
       return TP_ERR_CUDA;
+    note_launches(1);
   } else {
     vp_xent_rowwise_kernel<<<static_cast<unsigned>(T), kXentThreads, 0, stream>>>(
         logits, targets, v, N, grad_scale, loss, dlogits, argmax, dev_status);
+    note_launches(1);
     if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   }
   if (loss_sum) {
     loss_sum_kernel<<<1, 1024, 0, stream>>>(loss, T, loss_sum);
+    note_launches(1);
     if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   }
   return TP_OK;
