@@ -217,6 +217,39 @@ TP_API tp_status tp_row_linear_bwd(const void* Xin, const void* W, const void* d
                             void* dXin, void* dW, int32_t* dev_status, void* stream);
 
 /*
+ * Row-parallel linear forward that allocates nothing.  (No counterpart on
+ * the pages: this is a deployment variant of tp_row_linear_fwd.)
+ *
+ * Some callers cannot call cudaMalloc or pass in a workspace: code that runs
+ * inside a host framework which owns every device allocation, or a plugin
+ * whose interface only hands over input and output pointers.  This entry
+ * point computes the same Z = Σ_i Xin_i·W_i as tp_row_linear_fwd, always
+ * with one partial product per shard and the fused fixed-order sum, but keeps
+ * the shards' fp32 partials and the per-tile counters in a scratch array
+ * that is a static __device__ variable of the library.
+ *
+ *   - Scratch: TP_NOALLOC_SCRATCH_BYTES per GPU, reserved on every GPU that
+ *     loads the library and held until the process exits.  Calls whose
+ *     partials do not fit (ceil(M/128)·ceil(Nout/256)·N tiles of 128 KB plus
+ *     a counter each) return TP_ERR_WORKSPACE without enqueueing anything.
+ *   - bf16 only (TP_ERR_DTYPE otherwise); N <= 16; every shard offset a
+ *     multiple of 64 (TP_ERR_UNSUPPORTED otherwise).
+ *   - The first call on a device looks up the scratch address on that device
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture.  No call allocates or frees memory.
+ *   - Every call on a device shares the one scratch array, and it keeps the
+ *     previous call's contents (the counters are cleared by each call).
+ *     Calls that overlap on the GPU — on two streams, or from two threads —
+ *     race on it and give wrong results: serialise them.
+ *   Arguments as for tp_row_linear_fwd (no Zpart, no workspace).
+ */
+#define TP_NOALLOC_SCRATCH_BYTES (32u << 20)
+TP_API tp_status tp_row_linear_fwd_noalloc(const void* Xin, const void* W,
+                                           int64_t M, int64_t Kin, int64_t Nout, int32_t N,
+                                           const int64_t* shard_offsets, tp_dtype dt,
+                                           void* Z, int32_t* dev_status, void* stream);
+
+/*
  * Vocabulary-parallel input embedding   [TP-ILL] §4.1.
  *
  *   The table E [v,h] is split into N contiguous row ranges

@@ -24,6 +24,7 @@ __all__ = [
     "TPError", "lib", "library_path", "ACT_NONE", "ACT_GELU_TANH", "ACT_GELU_ERF",
     "tp_status_string", "tp_version", "tp_launch_count", "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
     "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
+    "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "vp_embed", "tp_logits_fwd", "vp_xent", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
@@ -59,6 +60,7 @@ _SIGS = {
     "tp_row_linear_fwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _SZ,
                            _P, _P], _I32),
     "tp_row_linear_bwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _P, _P, _P, _P], _I32),
+    "tp_row_linear_fwd_noalloc": ([_P, _P, _I64, _I64, _I64, _I32, _P, _I32, _P, _P, _P], _I32),
     "vp_embed": ([_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P], _I32),
     "tp_logits_fwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _P, _P], _I32),
     "vp_xent": ([_P, _P, _I64, _I64, _I32, _F, _P, _P, _P, _P, _P, _P], _I32),
@@ -253,6 +255,31 @@ def tp_row_linear_fwd(Xin, W, N, *, shard_offsets=None, Z=None, Zpart=None, ws=N
     _check(lib().tp_row_linear_fwd(_ptr(Xin), _ptr(W), M, Kin, Nout, N, offs, _dt(Xin), _ptr(Z),
                                    _ptr(Zpart), _ptr(ws), wsb, _ptr(dev_status), _stream(dev)),
            "tp_row_linear_fwd")
+    return Z
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20   # TP_NOALLOC_SCRATCH_BYTES in tplayers.h
+
+
+def tp_row_linear_fwd_noalloc(Xin, W, N, *, shard_offsets=None, Z=None, dev_status=None):
+    """Z = Σ_i Xin_i·W_i without any device allocation by the library.
+
+    For callers that cannot allocate device memory (a host framework that
+    owns every allocation, or a plugin interface that only passes input and
+    output pointers): the shards' partials live in the library's static
+    scratch of NOALLOC_SCRATCH_BYTES per GPU.  Only Z is allocated here, and
+    only if the caller does not pass it.  Calls that overlap on the GPU share
+    that scratch and race: serialise them.
+    """
+    M, Kin = Xin.shape
+    Nout = W.shape[1]
+    dev = Xin.device
+    Z = torch.empty(M, Nout, dtype=Xin.dtype, device=dev) if Z is None else Z
+    _contig(Xin, W, Z)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_row_linear_fwd_noalloc(_ptr(Xin), _ptr(W), M, Kin, Nout, N, offs, _dt(Xin),
+                                           _ptr(Z), _ptr(dev_status), _stream(dev)),
+           "tp_row_linear_fwd_noalloc")
     return Z
 
 
