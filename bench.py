@@ -132,16 +132,27 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 # the GPU arm
 # ----------------------------------------------------------------------------
-def _prepare(dev):
+def _prepare(dev, parts):
     import torch
 
     import linear_layers_b200 as tpl
     import tp_inputs
 
+    g = pr = vo = None
+    bf = dict(dtype=torch.bfloat16, device=dev)
+    if any(p.startswith("mlp") for p in parts):
+        g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
+    if "proj" in parts:
+        pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
+    if any(p in parts for p in ("embed", "logits", "xent")):
+        vo = _prepare_vocab(dev, tpl, tp_inputs, torch, bf, "logits" not in parts and "xent" in parts)
+    return g, pr, vo
+
+
+def _prepare_mlp(dev, tpl, tp_inputs, torch, bf):
     m = tp_inputs.mlp_inputs(MLP["M"], MLP["h"], MLP["F"], w_std=MLP["w_std"], seed=0)
     g = {k: v.to(dev) for k, v in m.items()}
     M, h, F = MLP["M"], MLP["h"], MLP["F"]
-    bf = dict(dtype=torch.bfloat16, device=dev)
     g.update(U=torch.empty(M, F, **bf), Y=torch.empty(M, F, **bf), Z=torch.empty(M, h, **bf),
              dU=torch.empty(M, F, **bf), dX=torch.empty(M, h, **bf), dA=torch.empty(h, F, **bf),
              dB=torch.empty(F, h, **bf), dbias=torch.empty(F, dtype=torch.float32, device=dev))
@@ -149,7 +160,10 @@ def _prepare(dev):
                             dtype=torch.uint8, device=dev)
     g["ws_b"] = torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_MLP_BWD, M, h, F, MLP["N"])),
                             dtype=torch.uint8, device=dev)
+    return g
 
+
+def _prepare_proj(dev, tpl, tp_inputs, torch, bf):
     p = tp_inputs.attn_proj_inputs(PROJ["M"], PROJ["h"], PROJ["n_heads"], PROJ["head_dim"],
                                    PROJ["N"], seed=0)
     pr = {k: v.to(dev) for k, v in p.items()}
@@ -167,7 +181,10 @@ def _prepare(dev):
                                                            PROJ["N"])), dtype=torch.uint8, device=dev)
     pr["ws_o"] = torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_ROW_LINEAR_FWD, Mp, hp, hp,
                                                            PROJ["N"])), dtype=torch.uint8, device=dev)
+    return pr
 
+
+def _prepare_vocab(dev, tpl, tp_inputs, torch, bf, fill_logits):
     vi = tp_inputs.vocab_inputs(VOC["T"], VOC["v"], VOC["h"], e_std=VOC["e_std"], seed=0)
     vo = {k: x.to(dev) for k, x in vi.items()}
     T, v = VOC["T"], VOC["v"]
@@ -175,7 +192,10 @@ def _prepare(dev):
               loss=torch.empty(T, dtype=torch.float32, device=dev),
               loss_sum=torch.empty(1, dtype=torch.float32, device=dev),
               argmax=torch.empty(T, dtype=torch.int32, device=dev))
-    return g, pr, vo
+    if fill_logits:   # the loss alone is timed: give it real logits once
+        tpl.tp_logits_fwd(vo["H"], vo["E"], VOC["N"], logits=vo["logits"])
+        torch.cuda.synchronize(dev)
+    return vo
 
 
 def _mlp_fwd(tpl, g, st):
@@ -274,7 +294,13 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    g, pr, vo = _prepare(dev)
+    parts = [p for p in PARTS if p in args.parts.split(",")]
+    if not parts:
+        raise SystemExit(f"--parts must name some of {','.join(PARTS)}")
+    if args.vocab_tokens:
+        VOC["T"] = args.vocab_tokens
+    full = parts == list(PARTS) and VOC["T"] == 16384
+    g, pr, vo = _prepare(dev, parts)
     st = tpl.new_status(dev)
     fns = {"mlp_fwd": lambda: _mlp_fwd(tpl, g, st), "mlp_bwd": lambda: _mlp_bwd(tpl, g, st),
            "proj": lambda: _proj(tpl, pr, st), "embed": lambda: _embed(tpl, vo, st),
@@ -282,12 +308,12 @@ def run_gpu(args):
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        for p in PARTS:
+        for p in parts:
             fns[p]()
     torch.cuda.synchronize(dev)
     assert int(st.item()) == 0, f"device status {int(st.item())} after warm-up"
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(PARTS) + 1)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
           for _ in range(args.steps)]
     if world > 1:
         torch.distributed.barrier()
@@ -297,7 +323,7 @@ def run_gpu(args):
         t_wall = time.perf_counter()
         for s in range(args.steps):
             ev[s][0].record(stream)
-            for i, p in enumerate(PARTS):
+            for i, p in enumerate(parts):
                 fns[p]()
                 ev[s][i + 1].record(stream)
         torch.cuda.synchronize(dev)
@@ -307,19 +333,33 @@ def run_gpu(args):
         torch.distributed.barrier()
     assert int(st.item()) == 0, f"device status {int(st.item())}"
 
-    part_ms = {p: 0.0 for p in PARTS}
+    part_ms = {p: 0.0 for p in parts}
     total_ms = 0.0
     for s in range(args.steps):
         total_ms += ev[s][0].elapsed_time(ev[s][-1])
-        for i, p in enumerate(PARTS):
+        for i, p in enumerate(parts):
             part_ms[p] += ev[s][i].elapsed_time(ev[s][i + 1])
-    times = torch.tensor([total_ms] + [part_ms[p] for p in PARTS], dtype=torch.float64, device=dev)
+    times = torch.tensor([total_ms] + [part_ms[p] for p in parts], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(times, op=torch.distributed.ReduceOp.MAX)
     total_ms = float(times[0])
-    part_ms = {p: float(times[i + 1]) for i, p in enumerate(PARTS)}
+    part_ms = {p: float(times[i + 1]) for i, p in enumerate(parts)}
+    if not full:   # a partial run (profiling): report the part times only
+        if rank == 0:
+            print(json.dumps({"partial_run": True, "parts": parts, "vocab_tokens": VOC["T"],
+                              "steps": args.steps, "warmup": args.warmup,
+                              "parts_ms_per_step": {p: round(part_ms[p] / args.steps, 4)
+                                                    for p in parts},
+                              "gpu_launches": int(launches)}), flush=True)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
 
-    e2e_ms, h2d, d2h = _e2e_mlp(tpl, torch, g, dev, max(2, min(args.steps, 5)))
+    if args.no_e2e:
+        e2e_ms, h2d, d2h = float("nan"), 0, 0
+    else:
+        e2e_ms, h2d, d2h = _e2e_mlp(tpl, torch, g, dev, max(2, min(args.steps, 5)))
     e2e = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(e2e, op=torch.distributed.ReduceOp.MAX)
@@ -488,6 +528,12 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-rows", type=int, default=128)
+    ap.add_argument("--parts", default=",".join(PARTS),
+                    help="comma-separated subset of the step (profiling runs); the JSON line of "
+                         "a partial run only carries part times")
+    ap.add_argument("--vocab-tokens", type=int, default=0,
+                    help="tokens of the vocabulary path (profiling runs; default 16384)")
+    ap.add_argument("--no-e2e", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always
     if args.impl == "reference":

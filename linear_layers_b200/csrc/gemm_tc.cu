@@ -7,25 +7,32 @@
 // reduction, the dGeLU GEMM, the two weight-gradient GEMMs and the
 // output-embedding logits GEMM.
 //
-// Structure of one CTA (one per SM, persistent over output tiles):
-//   warp 0   TMA producer: one elected lane streams A and B k-blocks
-//            (64 bf16 of K) into a ring of shared-memory stages;
-//   warp 1   owns tensor memory (512 columns = two 128x256 fp32
-//            accumulators) and one elected lane issues tcgen05.mma;
-//   warps 2-5 epilogue: tcgen05.ld of the finished accumulator, the fused
-//            element-wise work, stores to global memory.
-// The accumulator is double buffered, so the epilogue of tile t overlaps
-// the main loop of tile t+1.  Tiles are 128 x BN with BN = 256.
+// Two tile configurations share one kernel template:
+//   CG = 2  a pair of CTAs (a 2-CTA cluster on neighbouring SMs) computes a
+//           256 x 256 output tile with tcgen05.mma.cta_group::2: each CTA
+//           stages 128 rows of A and 128 columns of B per k-block, and each
+//           CTA's tensor memory holds its 128 rows x 256 fp32 columns;
+//   CG = 1  one CTA computes a 128 x 256 tile (problems one tile high).
+// Roles inside each CTA (persistent over output tiles):
+//   warp 0    TMA producer: one elected lane streams k-blocks of 64 bf16
+//             into a ring of shared-memory stages (no cluster multicast);
+//   warp 1    owns tensor memory (512 columns = two accumulators); in the
+//             pair leader one elected lane issues the MMAs;
+//   warps 2-9 epilogue: tcgen05.ld of the finished accumulator (two warps per
+//             TMEM lane quadrant, 128 columns each), fused element-wise
+//             work, stores to global memory.
+// The accumulator is double buffered, so the epilogue of one tile overlaps
+// the main loop of the next.
 //
 // Operands may be K-major or MN-major in global memory; both are loaded by
 // TMA with 128-byte swizzle and described to the tensor core by matching
 // shared-memory descriptors, so no operand is ever transposed in memory.
-// No TMA load uses cluster multicast.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 
+#include <cstdlib>
 #include <mutex>
 
 #include "internal.h"
@@ -35,10 +42,12 @@ namespace tpl {
 
 namespace {
 
-constexpr int BM = 128;
-constexpr int BK = 64;              // bf16 elements per k-block (= one 128-byte swizzle row)
-constexpr int kThreads = 192;       // 6 warps
-constexpr int kEpiThreads = 128;
+constexpr int BM = 128;              // rows of A per CTA
+constexpr int BN = 256;              // output columns per tile
+constexpr int BK = 64;               // bf16 elements per k-block (one 128-byte swizzle row)
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = 32 * kEpiWarps;
+constexpr int kThreads = 64 + kEpiThreads;
 constexpr uint32_t kTmemCols = 512;
 
 struct GemmArgs {
@@ -47,7 +56,7 @@ struct GemmArgs {
   int tiles_m, tiles_n, splits, group_m;
   int num_units;
   int split_kb[kMaxSplits + 1];     // k-block boundaries of the splits
-  int epi, act;
+  int act;
   void* out0;
   void* out1;
   int64_t ldo;
@@ -66,6 +75,22 @@ struct __align__(64) GemmParams {
   CUtensorMap tmA;
   CUtensorMap tmB;
   GemmArgs a;
+};
+
+template <int CG>
+struct Cfg {
+  static constexpr int kStages = CG == 2 ? 6 : 4;
+  static constexpr int kRows = BM * CG;          // output rows per tile
+  static constexpr int kBCols = BN / CG;         // B columns staged per CTA
+  static constexpr uint32_t kABytes = BM * BK * 2;
+  static constexpr uint32_t kBBytes = kBCols * BK * 2;
+  static constexpr uint32_t kOffB = kStages * kABytes;
+  static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
+  static constexpr uint32_t kNumBars = 2 * kStages + 5;
+  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;
+  static constexpr uint32_t kBytes = kOffRed + 4 * BN * 4;
+  static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
 };
 
 // -------------------------------------------------------------------------
@@ -137,12 +162,19 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float* v
   }
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float* v, int ncols_left) {
+__device__ __forceinline__ void load_raw_bf16x32(const __nv_bfloat16* src, uint4 (&w)[4],
+                                                 int ncols_left) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (8 * j < ncols_left) w = __ldg(reinterpret_cast<const uint4*>(src + 8 * j));
-    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    w[j] = make_uint4(0, 0, 0, 0);
+    if (8 * j < ncols_left) w[j] = __ldg(reinterpret_cast<const uint4*>(src + 8 * j));
+  }
+}
+
+__device__ __forceinline__ void unpack_bf16x32(const uint4 (&w)[4], float* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&ww[q]);
@@ -168,41 +200,32 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
   return v[0];
 }
 
-template <int BN, int STAGES>
-struct SmemLayout {
-  static constexpr uint32_t kABytes = BM * BK * 2;
-  static constexpr uint32_t kBBytes = BN * BK * 2;
-  static constexpr uint32_t kOffB = STAGES * kABytes;
-  static constexpr uint32_t kOffBar = kOffB + STAGES * kBBytes;
-  static constexpr uint32_t kNumBars = 2 * STAGES + 5;
-  static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;
-  static constexpr uint32_t kBytes = kOffRed + 4 * BN * 4;
-  static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
-};
-
-template <int BN, int STAGES>
+template <int CG, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
-  using L = SmemLayout<BN, STAGES>;
+  using C = Cfg<CG>;
+  constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const GemmArgs& a = P.a;
 
   uint8_t* sA = smem;
-  uint8_t* sB = smem + L::kOffB;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kOffBar);
+  uint8_t* sB = smem + C::kOffB;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* mma_done = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 4);
-  volatile int* bcast = reinterpret_cast<volatile int*>(smem + L::kOffMisc + 8);
-  float* red = reinterpret_cast<float*>(smem + L::kOffRed);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+  volatile int* bcast = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;   // 0 = pair leader
+  const int slot0 = CG == 2 ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int nslots = CG == 2 ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -211,18 +234,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(&tfull[s], 1);
-      mbar_init(&tempty[s], kEpiThreads);
+      mbar_init(&tempty[s], kEpiWarps * CG);   // one arrival per epilogue warp of the pair
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_cg<CG>(tmem_slot, kTmemCols);
+    tmem_relinquish_cg<CG>();
   }
   tc_fence_before_sync();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();   // peer barriers initialised before any signal
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -235,32 +259,52 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int unit = blockIdx.x; ok && unit < a.num_units; unit += gridDim.x) {
+      for (int unit = slot0; ok && unit < a.num_units; unit += nslots) {
         int tm, tn, s, tile;
         unit_map(a, unit, tm, tn, s, tile);
+        const int a_row = tm * C::kRows + static_cast<int>(rank) * BM;
+        const int b_col = tn * BN + static_cast<int>(rank) * C::kBCols;
         for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
             if (!*abort_flag) flag_timeout(a, abort_flag);
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], L::kABytes + L::kBBytes);
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], CG * (C::kABytes + C::kBBytes));
           const int k0 = kb * BK;
-          uint8_t* dA = sA + stage * L::kABytes;
-          uint8_t* dB = sB + stage * L::kBBytes;
-          if (!a.a_mn) {
-            tma_load_2d(dA, &P.tmA, &full[stage], k0, tm * BM);
-          } else {
+          uint8_t* dA = sA + stage * C::kABytes;
+          uint8_t* dB = sB + stage * C::kBBytes;
+          if constexpr (CG == 2) {
+            const uint32_t bar = mapa_shared(&full[stage], 0);
+            if (!a.a_mn) {
+              tma_load_2d_cg2(dA, &P.tmA, bar, k0, a_row);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BM / 64; ++j)
-              tma_load_2d(dA + j * 8192, &P.tmA, &full[stage], tm * BM + j * 64, k0);
-          }
-          if (!a.b_mn) {
-            tma_load_2d(dB, &P.tmB, &full[stage], k0, tn * BN);
-          } else {
+              for (int j = 0; j < BM / 64; ++j)
+                tma_load_2d_cg2(dA + j * 8192, &P.tmA, bar, a_row + j * 64, k0);
+            }
+            if (!a.b_mn) {
+              tma_load_2d_cg2(dB, &P.tmB, bar, k0, b_col);
+            } else {
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-              tma_load_2d(dB + j * 8192, &P.tmB, &full[stage], tn * BN + j * 64, k0);
+              for (int j = 0; j < C::kBCols / 64; ++j)
+                tma_load_2d_cg2(dB + j * 8192, &P.tmB, bar, b_col + j * 64, k0);
+            }
+          } else {
+            if (!a.a_mn) {
+              tma_load_2d(dA, &P.tmA, &full[stage], k0, a_row);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BM / 64; ++j)
+                tma_load_2d(dA + j * 8192, &P.tmA, &full[stage], a_row + j * 64, k0);
+            }
+            if (!a.b_mn) {
+              tma_load_2d(dB, &P.tmB, &full[stage], k0, b_col);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::kBCols / 64; ++j)
+                tma_load_2d(dB + j * 8192, &P.tmB, &full[stage], b_col + j * 64, k0);
+            }
           }
           ++issued;
           if (++stage == STAGES) {
@@ -269,31 +313,35 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           }
         }
       }
-      // Let every copy this thread started land before the CTA can exit
-      // (bounded in time, but not cut short by the abort flag).
-      volatile int keep_waiting = 0;
-      const int inflight = issued < STAGES ? issued : STAGES;
-      for (int i = 0; i < inflight; ++i) {
-        if (--stage < 0) {
-          stage = STAGES - 1;
-          phase ^= 1u;
+      // Let every copy started by this pair land before the CTAs can exit
+      // (bounded in time, not cut short by the abort flag).  The stage
+      // barriers live in the leader and count both CTAs' bytes.
+      if (rank == 0) {
+        volatile int keep_waiting = 0;
+        const int inflight = issued < STAGES ? issued : STAGES;
+        for (int i = 0; i < inflight; ++i) {
+          if (--stage < 0) {
+            stage = STAGES - 1;
+            phase ^= 1u;
+          }
+          mbar_wait_bounded(&full[stage], phase, a.wait_ns, &keep_waiting);
         }
-        mbar_wait_bounded(&full[stage], phase, a.wait_ns, &keep_waiting);
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (elect_one_sync()) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN, a.a_mn != 0, a.b_mn != 0);
+    // ------------------------------------------------------------ MMA issuer (pair leader)
+    if (rank == 0 && elect_one_sync()) {
+      const uint32_t idesc = idesc_bf16_f32(C::kRows, BN, a.a_mn != 0, a.b_mn != 0);
       const uint32_t a_lbo = a.a_mn ? 8192u : 16u;
       const uint32_t b_lbo = a.b_mn ? 8192u : 16u;
       const uint32_t a_kstep = a.a_mn ? 2048u : 32u;   // bytes per 16-element K step
       const uint32_t b_kstep = a.b_mn ? 2048u : 32u;
+      const uint16_t pair_mask = CG == 2 ? 0x3 : 0x1;
       int stage = 0;
       uint32_t phase = 0;
       int t = 0;
       bool ok = true, any = false;
-      for (int unit = blockIdx.x; ok && unit < a.num_units; unit += gridDim.x, ++t) {
+      for (int unit = slot0; ok && unit < a.num_units; unit += nslots, ++t) {
         int tm, tn, s, tile;
         unit_map(a, unit, tm, tn, s, tile);
         const int acc = t & 1;
@@ -312,57 +360,62 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             break;
           }
           tc_fence_after_sync();
-          const uint32_t a_base = smem_u32(sA + stage * L::kABytes);
-          const uint32_t b_base = smem_u32(sB + stage * L::kBBytes);
+          const uint32_t a_base = smem_u32(sA + stage * C::kABytes);
+          const uint32_t b_base = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
             const uint64_t adesc = smem_desc_sw128(a_base + k * a_kstep, a_lbo, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_base + k * b_kstep, b_lbo, 1024);
-            tc_mma_bf16(d_tmem, adesc, bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+            tc_mma_bf16_cg<CG>(d_tmem, adesc, bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
           }
           any = true;
-          tc_commit(&empty[stage]);   // frees the stage once these MMAs have read it
+          tc_commit_mc<CG>(&empty[stage], pair_mask);   // frees the stage in both CTAs
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
-        if (ok) tc_commit(&tfull[acc]);   // accumulator ready for the epilogue
+        if (ok) tc_commit_mc<CG>(&tfull[acc], pair_mask);   // accumulators ready
       }
       if (any) {   // every issued MMA must finish before tensor memory is freed
         volatile int keep_waiting = 0;
-        tc_commit(mma_done);
+        tc_commit_local<CG>(mma_done);
         mbar_wait_bounded(mma_done, 0, a.wait_ns, &keep_waiting);
       }
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    const int ew = warp - 2;              // 0..7
     const int q = warp & 3;               // TMEM lane quadrant this warp may access
+    const int half = ew >> 2;             // which 128 of the 256 accumulator columns
     const int row_in_tile = q * 32 + lane;
-    const int et = threadIdx.x - 64;      // 0..127 among the epilogue threads
+    const int et = threadIdx.x - 64;      // 0..255 among the epilogue threads
+    const uint32_t tempty_addr0 = CG == 2 ? mapa_shared(&tempty[0], 0) : smem_u32(&tempty[0]);
     int t = 0;
-    for (int unit = blockIdx.x; unit < a.num_units; unit += gridDim.x, ++t) {
+    for (int unit = slot0; unit < a.num_units; unit += nslots, ++t) {
       int tm, tn, s, tile;
       unit_map(a, unit, tm, tn, s, tile);
       const int acc = t & 1;
       const uint32_t use = static_cast<uint32_t>(t >> 1);
       const bool got = mbar_wait_bounded(&tfull[acc], use & 1u, a.wait_ns, abort_flag);
-      // all 128 epilogue threads leave together or go on together, so no
-      // warp can be left waiting in a later named barrier
+      // all epilogue threads leave together or go on together, so no warp
+      // can be left waiting in a later named barrier
       if (!named_barrier_and(1, kEpiThreads, got)) {
         if (et == 0 && !*abort_flag) flag_timeout(a, abort_flag);
         break;
       }
       tc_fence_after_sync();
-      const int row = tm * BM + row_in_tile;
+      const int row = tm * C::kRows + static_cast<int>(rank) * BM + row_in_tile;
       const bool row_ok = row < a.M;
+      const int htile = tile * CG + static_cast<int>(rank);   // this CTA's 128-row half tile
       const uint32_t t_base =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const int c0 = half * 4;
 
-      if (a.epi == EPI_SPLIT_SUM) {
+      if constexpr (EPI == EPI_SPLIT_SUM) {
         // 1) publish this split's fp32 partial
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = c0; c < c0 + 4; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           tc_wait_ld();
@@ -379,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           } else {
             float* dst = a.part +
-                         ((static_cast<int64_t>(tile) * a.splits + s) * (BN / 32) + c) * (BM * 32) +
+                         ((static_cast<int64_t>(htile) * a.splits + s) * (BN / 32) + c) * (BM * 32) +
                          row_in_tile * 32;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -391,18 +444,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         __threadfence();
         named_barrier_sync(1, kEpiThreads);
         if (et == 0) {
-          const int prev = atomicAdd(&a.counters[tile], 1);
+          const int prev = atomicAdd(&a.counters[htile], 1);
           const int last = (prev == a.splits - 1);
-          if (last) a.counters[tile] = 0;   // ready for the next call
+          if (last) a.counters[htile] = 0;   // ready for the next call
           *bcast = last;
         }
         named_barrier_sync(1, kEpiThreads);
         const bool last = *bcast != 0;
         if (last) {
           __threadfence();
-          // 2) the last split of this tile sums all partials in split order
+          // 2) the last split of this half tile sums all partials in split order
 #pragma unroll 1
-          for (int c = 0; c < BN / 32; ++c) {
+          for (int c = c0; c < c0 + 4; ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_base + c * 32, r);
             tc_wait_ld();
@@ -430,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               } else {
                 const float* src =
                     a.part +
-                    ((static_cast<int64_t>(tile) * a.splits + ss) * (BN / 32) + c) * (BM * 32) +
+                    ((static_cast<int64_t>(htile) * a.splits + ss) * (BN / 32) + c) * (BM * 32) +
                     row_in_tile * 32;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -447,31 +500,43 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           }
         }
       } else {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          const int col0 = tn * BN + c * 32;
-          float aux_v[32];
-          if (a.epi == EPI_DACT) {
-            if (row_ok && col0 < a.N) {
-              load_bf16x32(a.aux + row * a.ld_aux + col0, aux_v, a.N - col0);
-            } else {
+        uint4 aux_w[4];
+        if constexpr (EPI == EPI_DACT) {   // U for the first chunk
+          const int col0 = tn * BN + c0 * 32;
+          if (row_ok && col0 < a.N) {
+            load_raw_bf16x32(a.aux + row * a.ld_aux + col0, aux_w, a.N - col0);
+          } else {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) aux_v[j] = 0.0f;
-            }
+            for (int j = 0; j < 4; ++j) aux_w[j] = make_uint4(0, 0, 0, 0);
           }
+        }
+#pragma unroll 1
+        for (int c = c0; c < c0 + 4; ++c) {
+          const int col0 = tn * BN + c * 32;
+          const bool store_ok = row_ok && col0 < a.N;
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
+          float aux_v[32];
+          if constexpr (EPI == EPI_DACT) {
+            unpack_bf16x32(aux_w, aux_v);
+            const int coln = col0 + 32;   // prefetch U of the next chunk while this one runs
+            if (c + 1 < c0 + 4 && row_ok && coln < a.N) {
+              load_raw_bf16x32(a.aux + row * a.ld_aux + coln, aux_w, a.N - coln);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) aux_w[j] = make_uint4(0, 0, 0, 0);
+            }
+          }
           tc_wait_ld();
           float v[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
-          const bool store_ok = row_ok && col0 < a.N;
 
-          if (a.epi == EPI_STORE_BF16) {
+          if constexpr (EPI == EPI_STORE_BF16) {
             if (store_ok)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
                             a.N - col0);
-          } else if (a.epi == EPI_STORE_F32) {
+          } else if constexpr (EPI == EPI_STORE_F32) {
             if (store_ok) {
               float* dst = static_cast<float*>(a.out0) + row * a.ldo + col0;
 #pragma unroll
@@ -480,10 +545,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                   *reinterpret_cast<float4*>(dst + 4 * j) =
                       make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
             }
-          } else if (a.epi == EPI_BIAS_ACT) {
+          } else if constexpr (EPI == EPI_BIAS_ACT) {
             if (a.bias != nullptr && col0 < a.N) {
+              uint4 bw[4];
               float b[32];
-              load_bf16x32(a.bias + col0, b, a.N - col0);
+              load_raw_bf16x32(a.bias + col0, bw, a.N - col0);
+              unpack_bf16x32(bw, b);
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] += b[j];
             }
@@ -507,27 +574,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           }
         }
-        if (a.epi == EPI_DACT && a.dbias_part != nullptr) {
-          named_barrier_sync(1, kEpiThreads);
-          for (int cc = et; cc < BN; cc += kEpiThreads) {
+        if constexpr (EPI == EPI_DACT) {
+          if (a.dbias_part != nullptr) {
+            named_barrier_sync(1, kEpiThreads);
+            const int cc = et;   // one column per epilogue thread (256 columns)
             const int col = tn * BN + cc;
-            // fixed order over the four row quarters of the tile
+            // fixed order over the four row quarters of the half tile
             const float sum = ((red[cc] + red[BN + cc]) + red[2 * BN + cc]) + red[3 * BN + cc];
-            if (col < a.N) a.dbias_part[static_cast<int64_t>(tm) * a.N + col] = sum;
+            if (col < a.N)
+              a.dbias_part[static_cast<int64_t>(tm * CG + static_cast<int>(rank)) * a.N + col] = sum;
+            named_barrier_sync(1, kEpiThreads);
           }
-          named_barrier_sync(1, kEpiThreads);
         }
       }
       tc_fence_before_sync();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {   // release the accumulator to the pair leader's MMA
+        if constexpr (CG == 2)
+          mbar_arrive_cluster(tempty_addr0 + static_cast<uint32_t>(acc * 8));
+        else
+          mbar_arrive(&tempty[acc]);
+      }
     }
   }
 
   tc_fence_before_sync();
   __syncthreads();
+  if constexpr (CG == 2) cluster_sync_all();   // no CTA leaves while its peer may touch it
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem_base, kTmemCols);
+    tmem_dealloc_cg<CG>(tmem_base, kTmemCols);
   }
 }
 
@@ -564,40 +640,93 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
-template <int BN, int STAGES>
-tp_status launch_impl(const GemmParams& prm, int grid, cudaStream_t stream) {
-  using L = SmemLayout<BN, STAGES>;
-  static_assert(L::kAlloc <= 232448, "shared memory budget");
-  static int configured_device = -1;
+// Launch with `slots` persistent CTAs (CG = 1) or CTA pairs (CG = 2), capped
+// at the number that can be resident at once, so that no persistent slot
+// starts only after another has finished.
+template <int CG, int EPI>
+tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
+  using C = Cfg<CG>;
+  static_assert(C::kAlloc <= 232448, "shared memory budget");
+  static int max_resident[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (configured_device != dev) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, L::kAlloc) != cudaSuccess)
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CG;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!max_resident[dev & 63]) {
+    if (cudaFuncSetAttribute(gemm_tc_kernel<CG, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kAlloc) != cudaSuccess)
       return TP_ERR_CUDA;
-    configured_device = dev;
+    int clusters = 0;
+    cfg.gridDim = dim3(static_cast<unsigned>(CG * num_sms()));
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<CG, EPI>, &cfg) != cudaSuccess ||
+        clusters <= 0) {
+      cudaGetLastError();
+      clusters = num_sms() / CG;
+    }
+    max_resident[dev & 63] = clusters;
   }
-  gemm_tc_kernel<BN, STAGES><<<grid, kThreads, L::kAlloc, stream>>>(prm);
+  if (slots > max_resident[dev & 63]) slots = max_resident[dev & 63];
+  const int grid = CG * slots;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<CG, EPI>, prm) != cudaSuccess) return TP_ERR_CUDA;
   note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  return TP_OK;
 }
 
-constexpr int kBN = 256;
-constexpr int kStages = 4;
+template <int CG>
+tp_status launch_epi(const GemmParams& prm, int epi, int slots, cudaStream_t stream) {
+  switch (epi) {
+    case EPI_STORE_BF16: return launch_impl<CG, EPI_STORE_BF16>(prm, slots, stream);
+    case EPI_BIAS_ACT: return launch_impl<CG, EPI_BIAS_ACT>(prm, slots, stream);
+    case EPI_DACT: return launch_impl<CG, EPI_DACT>(prm, slots, stream);
+    case EPI_STORE_F32: return launch_impl<CG, EPI_STORE_F32>(prm, slots, stream);
+    case EPI_SPLIT_SUM: return launch_impl<CG, EPI_SPLIT_SUM>(prm, slots, stream);
+  }
+  return TP_ERR_UNSUPPORTED;
+}
+
+// Tile configuration: pairs of CTAs (256-row tiles) unless the problem is a
+// single 128-row tile high; TP_GEMM_CTA_GROUP=1|2 forces one (tests).
+int choose_cg(int M) {
+  static int forced = -1;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    forced = 0;
+    if (const char* e = std::getenv("TP_GEMM_CTA_GROUP")) {
+      const int v = std::atoi(e);
+      if (v == 1 || v == 2) forced = v;
+    }
+  });
+  if (forced) return forced;
+  return M > BM ? 2 : 1;
+}
 
 }  // namespace
 
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
   if (splits <= 1) return 0;
-  const size_t tiles = static_cast<size_t>((M + BM - 1) / BM) * ((N + kBN - 1) / kBN);
-  size_t bytes = with_zpart ? 0 : tiles * splits * BM * kBN * sizeof(float);
-  bytes += tiles * sizeof(int);
+  // 128-row half tiles of the 256-row tiling (covers the 128-row tiling too)
+  const size_t htiles = static_cast<size_t>((M + 2 * BM - 1) / (2 * BM)) * 2 * ((N + BN - 1) / BN);
+  size_t bytes = with_zpart ? 0 : htiles * splits * BM * BN * sizeof(float);
+  bytes += htiles * sizeof(int);
   return (bytes + 255) & ~static_cast<size_t>(255);
 }
 
 tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return TP_ERR_SHAPE;
   if (p.splits < 1 || p.splits > kMaxSplits) return TP_ERR_SHAPE;
+  const int CG = choose_cg(p.M);
+  const int rows = BM * CG;
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
   GemmArgs& a = prm.a;
@@ -606,10 +735,10 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.K = p.K;
   a.a_mn = p.a_mn;
   a.b_mn = p.b_mn;
-  a.tiles_m = (p.M + BM - 1) / BM;
-  a.tiles_n = (p.N + kBN - 1) / kBN;
+  a.tiles_m = (p.M + rows - 1) / rows;
+  a.tiles_n = (p.N + BN - 1) / BN;
   a.splits = p.splits;
-  a.group_m = 16;
+  a.group_m = CG == 2 ? 8 : 16;
   const int kblocks = (p.K + BK - 1) / BK;
   if (p.splits == 1) {
     a.split_kb[0] = 0;
@@ -624,7 +753,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     if (p.split_k[0] != 0 || p.split_k[p.splits] != p.K) return TP_ERR_SHAPE;
   }
   a.num_units = a.tiles_m * a.tiles_n * a.splits;
-  a.epi = p.splits > 1 ? EPI_SPLIT_SUM : p.epi;
+  const int epi = p.splits > 1 ? EPI_SPLIT_SUM : p.epi;
   a.act = p.act;
   a.out0 = p.out0;
   a.out1 = p.out1;
@@ -638,7 +767,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (p.splits > 1) {
     const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
     if (p.ws == nullptr || p.ws_bytes < need) return TP_ERR_WORKSPACE;
-    const size_t tiles = static_cast<size_t>(a.tiles_m) * a.tiles_n;
+    const size_t htiles = static_cast<size_t>(a.tiles_m) * CG * a.tiles_n;
     if (p.zpart) {
       a.part = p.zpart;
       a.part_is_zpart = 1;
@@ -647,12 +776,14 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
       a.part = static_cast<float*>(p.ws);
       a.part_is_zpart = 0;
       a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(p.ws) +
-                                          tiles * p.splits * BM * kBN * sizeof(float));
+                                          htiles * p.splits * BM * BN * sizeof(float));
     }
-    if (cudaMemsetAsync(a.counters, 0, tiles * sizeof(int), stream) != cudaSuccess)
+    if (cudaMemsetAsync(a.counters, 0, htiles * sizeof(int), stream) != cudaSuccess)
       return TP_ERR_CUDA;
   }
-  // operand maps
+  // operand maps: A boxes of 128 rows (K-major) or 64 x 64 blocks (MN-major);
+  // B boxes of BN / CG rows (K-major) or 64 x 64 blocks (MN-major)
+  const uint32_t b_rows = static_cast<uint32_t>(BN / CG);
   bool ok;
   if (!p.a_mn)
     ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, BM);
@@ -660,12 +791,13 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     ok = make_tmap(&prm.tmA, p.A, p.M, p.K, p.lda, 64, BK);
   if (!ok) return TP_ERR_CUDA;
   if (!p.b_mn)
-    ok = make_tmap(&prm.tmB, p.B, p.K, p.N, p.ldb, BK, kBN);
+    ok = make_tmap(&prm.tmB, p.B, p.K, p.N, p.ldb, BK, b_rows);
   else
     ok = make_tmap(&prm.tmB, p.B, p.N, p.K, p.ldb, 64, BK);
   if (!ok) return TP_ERR_CUDA;
-  const int grid = a.num_units < num_sms() ? a.num_units : num_sms();
-  return launch_impl<kBN, kStages>(prm, grid, stream);
+  const int slots = CG == 2 ? num_sms() / 2 : num_sms();
+  const int used = a.num_units < slots ? a.num_units : slots;
+  return CG == 2 ? launch_epi<2>(prm, epi, used, stream) : launch_epi<1>(prm, epi, used, stream);
 }
 
 }  // namespace tpl
