@@ -23,6 +23,7 @@
 #include <cstdint>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace tpl {
 namespace {
@@ -81,38 +82,18 @@ __global__ void __launch_bounds__(kEmbedWarps * 32)
 // ---------------------------------------------------------------------------
 constexpr int kXentThreads = 256;
 
-struct ShardStat {   // what one shard publishes for its row
-  float m;           // max of the shard's logits
-  float s;           // Σ exp(l − m) over the shard
-  float tgt;         // target logit if the target is in this shard, else 0
-  int amax;          // global index of the first maximum in the shard
-};
 
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
-                   : "memory");
-}
-__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
-               : "=r"(r)
-               : "r"(static_cast<uint32_t>(__cvta_generic_to_shared(p))), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ int ld_dsmem_s32(uint32_t addr) {
-  int v;
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-  return v;
+
+
+// 1-D bulk copy global -> this CTA's shared memory, completion counted in
+// bytes on `bar` (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
 }
 
 // (value, index) max with ties to the lower index
@@ -154,118 +135,231 @@ __device__ __forceinline__ float block_sum(float x, float* sv) {
   return s;
 }
 
-// grid = T * N CTAs, cluster = N CTAs (one token), CTA rank = shard.
-// Dynamic shared memory: the shard's slice of the row (vs floats).
-__global__ void __launch_bounds__(kXentThreads)
-    vp_xent_cluster_kernel(const float* logits, const int64_t* __restrict__ targets, int64_t v,
-                           int vs, float grad_scale, float* __restrict__ loss, float* dlogits,
-                           int32_t* __restrict__ argmax, int32_t* dev_status) {
-  extern __shared__ float4 slice4[];
-  __shared__ ShardStat stat;
-  __shared__ float red_v[kXentThreads / 32];
-  __shared__ int red_i[kXentThreads / 32];
-  __shared__ float comb[3];   // lse, target logit, valid
+// Persistent form: grid = (clusters) x N CTAs, cluster = N CTAs, CTA rank =
+// vocabulary shard.  Cluster c handles tokens c, c + C, c + 2C, ...
+// Each CTA's slice of a row arrives in shared memory by bulk copy, two
+// tokens ahead (double buffered); every thread copies its R float4 into
+// registers and the buffer is refilled at once, so HBM reads never wait on
+// the reductions.  One HBM read and one HBM write per logit, one exp per
+// logit (kept in registers for the gradient).  The shards exchange their
+// (max, sum-exp, target logit, arg-max) point to point: lane r of warp 0
+// writes the CTA's 16-byte record into shard r's shared memory with an
+// asynchronous store that counts its bytes on shard r's barrier; each CTA
+// expects N records on its own barrier and combines them in shard order.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
+__device__ __forceinline__ float max4(const float4& a) {
+  return fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w));
+}
+
+template <int R>
+__global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
+    vp_xent_cluster_kernel(const float* logits, const int64_t* __restrict__ targets, int64_t T,
+                           int64_t v, int vs, float grad_scale, float* __restrict__ loss,
+                           float* dlogits, int32_t* __restrict__ argmax, int32_t* dev_status,
+                           uint64_t wait_ns) {
+  extern __shared__ __align__(128) unsigned char xsm[];   // two slices of the row
+  __shared__ __align__(16) float rec[2][8][4];   // [token parity][shard] (m, s, tgt, amax)
+  __shared__ __align__(8) uint64_t xbar[2];
+  __shared__ __align__(8) uint64_t load_bar[2];
+  // block-reduction scratch, double buffered by token parity: a warp that
+  // runs ahead writes the other half while slow warps still read this one
+  __shared__ float red_m2[2][kXentThreads / 32];
+  __shared__ float red_s2[2][kXentThreads / 32];
+  __shared__ int red_i2[2][kXentThreads / 32];
+
+  constexpr float kLog2e = 1.4426950408889634f;
   const uint32_t shard = cluster_ctarank();
   const int N = static_cast<int>(v / vs);
-  const int64_t tok = blockIdx.x / N;
+  const int64_t cluster_id = blockIdx.x / N;
+  const int64_t nclusters = gridDim.x / N;
   const int64_t lo = static_cast<int64_t>(shard) * vs;
-  const float4* src4 = reinterpret_cast<const float4*>(logits + tok * v + lo);
   const int nvec = vs >> 2;
-
-  // 1) stage the slice, track the first maximum
-  float mv = -CUDART_INF_F;
-  int mi = 0x7fffffff;
-  for (int j = threadIdx.x; j < nvec; j += kXentThreads) {
-    const float4 x = __ldcs(src4 + j);
-    slice4[j] = x;
-    argmax_merge(mv, mi, x.x, 4 * j);
-    argmax_merge(mv, mi, x.y, 4 * j + 1);
-    argmax_merge(mv, mi, x.z, 4 * j + 2);
-    argmax_merge(mv, mi, x.w, 4 * j + 3);
-  }
-  block_argmax(mv, mi, red_v, red_i);   // includes __syncthreads: slice visible
-  const float m_i = mv;
-
-  const int64_t y = __ldg(targets + tok);
-  const bool y_ok = y >= 0 && y < v;
-  const bool mine = y_ok && y >= lo && y < lo + vs;
-  // read from global: the slice is overwritten in place below, and no CTA
-  // writes dlogits (which may alias logits) before the first cluster barrier
-  const float tgt_i = (mine && threadIdx.x == 0) ? logits[tok * v + y] : 0.0f;
-
-  // 2) e = exp(l − m_i) in place, and its sum
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const bool need_grad = dlogits != nullptr;
-  float sacc = 0.f;
-  for (int j = threadIdx.x; j < nvec; j += kXentThreads) {
-    float4 x = slice4[j];
-    x.x = __expf(x.x - m_i);
-    x.y = __expf(x.y - m_i);
-    x.z = __expf(x.z - m_i);
-    x.w = __expf(x.w - m_i);
-    sacc += (x.x + x.y) + (x.z + x.w);
-    if (need_grad) slice4[j] = x;
-  }
-  const float s_i = block_sum(sacc, red_v);
+  const uint32_t slice_bytes = static_cast<uint32_t>(vs) * 4u;
+  const uint32_t buf_stride = (slice_bytes + 127u) & ~127u;
 
-  // 3) publish this shard's scalars; combine all shards' through DSMEM
   if (threadIdx.x == 0) {
-    stat.m = m_i;
-    stat.s = s_i;
-    stat.tgt = tgt_i;
-    stat.amax = static_cast<int>(lo) + mi;
+    mbar_init(&xbar[0], 1);
+    mbar_init(&xbar[1], 1);
+    mbar_init(&load_bar[0], 1);
+    mbar_init(&load_bar[1], 1);
+    fence_mbarrier_init();
   }
-  cluster_sync_all();
-  if (threadIdx.x == 0) {
-    float m = -CUDART_INF_F;
-    float ms[16];
-    float ss[16];
-    float best_v = -CUDART_INF_F;
-    int best_i = 0x7fffffff;
-    float tgt = 0.f;
-    for (int r = 0; r < N; ++r) {
-      const uint32_t base = map_to_rank(&stat, r);
-      ms[r] = ld_dsmem_f32(base + offsetof(ShardStat, m));
-      ss[r] = ld_dsmem_f32(base + offsetof(ShardStat, s));
-      tgt += ld_dsmem_f32(base + offsetof(ShardStat, tgt));
-      argmax_merge(best_v, best_i, ms[r], ld_dsmem_s32(base + offsetof(ShardStat, amax)));
-      m = fmaxf(m, ms[r]);
+  __syncthreads();
+  cluster_sync_all();   // every CTA's barriers exist before any peer signals them
+
+  auto issue = [&](int b, int64_t tok) {   // one thread
+    mbar_arrive_expect_tx(&load_bar[b], slice_bytes);
+    const char* src = reinterpret_cast<const char*>(logits + tok * v + lo);
+    char* dst = reinterpret_cast<char*>(xsm + b * buf_stride);
+    for (uint32_t off = 0; off < slice_bytes; off += 16384u) {
+      const uint32_t n = slice_bytes - off < 16384u ? slice_bytes - off : 16384u;
+      bulk_load(dst + off, src + off, n, &load_bar[b]);
     }
-    float S = 0.f;
-    for (int r = 0; r < N; ++r) S += ss[r] * __expf(ms[r] - m);   // shard order
-    const float lse = m + logf(S);
-    comb[0] = lse;
-    comb[1] = tgt;
-    comb[2] = y_ok ? 1.f : 0.f;
-    if (shard == 0) {
+  };
+  if (threadIdx.x == 0) {
+    if (cluster_id < T) issue(0, cluster_id);
+    if (cluster_id + nclusters < T) issue(1, cluster_id + nclusters);
+  }
+
+  int k = 0;
+  for (int64_t tok = cluster_id; tok < T; tok += nclusters, ++k) {
+    const int p = k & 1;
+    const int64_t y = __ldg(targets + tok);
+    const bool y_ok = y >= 0 && y < v;
+    const bool mine = y_ok && y >= lo && y < lo + vs;
+    // this token's N incoming records: 16 bytes each on xbar[p]
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(&xbar[p], static_cast<uint32_t>(N) * 16u);
+    if (!mbar_wait_cluster_bounded(&load_bar[p], static_cast<uint32_t>(k >> 1) & 1u, wait_ns)) {
+      if (threadIdx.x == 0 && dev_status) atomicOr(dev_status, TP_DEVERR_TIMEOUT);
+    }
+    const float4* buf4 = reinterpret_cast<const float4*>(xsm + p * buf_stride);
+    float4 x[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const int j = threadIdx.x + r * kXentThreads;
+      x[r] = j < nvec ? buf4[j]
+                      : make_float4(-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F);
+    }
+    const float tgt_i =
+        (mine && threadIdx.x == 0) ? reinterpret_cast<const float*>(buf4)[y - lo] : 0.0f;
+
+    // 1) shard maximum
+    float mt = max4(x[0]);
+#pragma unroll
+    for (int r = 1; r < R; ++r) mt = fmaxf(mt, max4(x[r]));
+    float wm = mt;
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, off));
+    if (lane == 0) red_m2[p][warp] = wm;
+    __syncthreads();   // also: every thread has its slice in registers
+    if (threadIdx.x == 0 && tok + 2 * nclusters < T) {   // refill two tokens ahead
+      fence_proxy_async_smem();
+      issue(p, tok + 2 * nclusters);
+    }
+    float m_i = red_m2[p][0];
+#pragma unroll
+    for (int w = 1; w < kXentThreads / 32; ++w) m_i = fmaxf(m_i, red_m2[p][w]);
+
+    // 2) first position of the maximum (only threads that hold it search)
+    int it = 0x7fffffff;
+    if (mt == m_i) {
+#pragma unroll
+      for (int r = R - 1; r >= 0; --r) {   // elements ascend with r: keep the lowest
+        const int j = threadIdx.x + r * kXentThreads;
+        if (x[r].w == m_i) it = 4 * j + 3;
+        if (x[r].z == m_i) it = 4 * j + 2;
+        if (x[r].y == m_i) it = 4 * j + 1;
+        if (x[r].x == m_i) it = 4 * j;
+      }
+    }
+
+    // 3) e = exp(l − m_i) kept in registers, and the shard's sum
+    const float mL = m_i * kLog2e;
+    float st = 0.f;
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      x[r].x = ex2_approx(fmaf(x[r].x, kLog2e, -mL));
+      x[r].y = ex2_approx(fmaf(x[r].y, kLog2e, -mL));
+      x[r].z = ex2_approx(fmaf(x[r].z, kLog2e, -mL));
+      x[r].w = ex2_approx(fmaf(x[r].w, kLog2e, -mL));
+      st += (x[r].x + x[r].y) + (x[r].z + x[r].w);
+    }
+#pragma unroll
+    for (int off = 16; off >= 1; off >>= 1) {
+      st += __shfl_xor_sync(0xffffffffu, st, off);
+      it = min(it, __shfl_xor_sync(0xffffffffu, it, off));
+    }
+    if (lane == 0) {
+      red_s2[p][warp] = st;
+      red_i2[p][warp] = it;
+    }
+    __syncthreads();
+    float s_i = 0.f;
+    int a_i = 0x7fffffff;
+#pragma unroll
+    for (int w = 0; w < kXentThreads / 32; ++w) {   // fixed order
+      s_i += red_s2[p][w];
+      a_i = min(a_i, red_i2[p][w]);
+    }
+
+    // 4) send this shard's record to every shard of the cluster (itself included)
+    if (warp == 0) {
+      const float tg = __shfl_sync(0xffffffffu, tgt_i, 0);   // held by thread 0
+      if (lane < N)
+        st_async_v4(mapa_shared(&rec[p][shard][0], static_cast<uint32_t>(lane)),
+                    mapa_shared(&xbar[p], static_cast<uint32_t>(lane)), m_i, s_i, tg,
+                    __int_as_float(static_cast<int>(lo) + a_i));
+    }
+    if (!mbar_wait_cluster_bounded(&xbar[p], static_cast<uint32_t>(k >> 1) & 1u, wait_ns)) {
+      if (threadIdx.x == 0 && dev_status) atomicOr(dev_status, TP_DEVERR_TIMEOUT);
+    }
+
+    // 5) combine the N records inside each warp: lane r holds shard r's
+    float rm = -CUDART_INF_F, rs = 0.f, rt = 0.f;
+    int ri = 0x7fffffff;
+    if (lane < N) {
+      const float4 q = *reinterpret_cast<const float4*>(&rec[p][lane][0]);
+      rm = q.x;
+      rs = q.y;
+      rt = q.z;
+      ri = __float_as_int(q.w);
+    }
+    float M = rm;
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float term = lane < N ? rs * ex2_approx((rm - M) * kLog2e) : 0.f;
+    int bi = rm == M ? ri : 0x7fffffff;   // lowest index among the shards holding M
+#pragma unroll
+    for (int off = 4; off >= 1; off >>= 1) {
+      term += __shfl_xor_sync(0xffffffffu, term, off);
+      rt += __shfl_xor_sync(0xffffffffu, rt, off);
+      bi = min(bi, __shfl_xor_sync(0xffffffffu, bi, off));
+    }
+    const float S = __shfl_sync(0xffffffffu, term, 0);
+    const float tgt = __shfl_sync(0xffffffffu, rt, 0);
+    M = __shfl_sync(0xffffffffu, M, 0);
+    bi = __shfl_sync(0xffffffffu, bi, 0);
+    const float lse = M + logf(S);
+    if (shard == 0 && threadIdx.x == 0) {
       loss[tok] = y_ok ? lse - tgt : CUDART_NAN_F;
-      if (argmax) argmax[tok] = best_i;
+      if (argmax) argmax[tok] = bi;
       if (!y_ok && dev_status) atomicOr(dev_status, TP_DEVERR_RANGE);
     }
-  }
-  cluster_sync_all();   // no CTA leaves while a peer may still read its `stat`
-  if (!need_grad) return;
 
-  // 4) dlogits block = grad_scale · (e · exp(m_i − lse) − onehot)
-  const float lse = comb[0];
-  const float scale = y_ok ? grad_scale * __expf(m_i - lse) : CUDART_NAN_F;
-  float4* dst4 = reinterpret_cast<float4*>(dlogits + tok * v + lo);
-  const int yl = mine ? static_cast<int>(y - lo) : -1;
-  for (int j = threadIdx.x; j < nvec; j += kXentThreads) {
-    float4 e = slice4[j];
-    e.x *= scale;
-    e.y *= scale;
-    e.z *= scale;
-    e.w *= scale;
-    if ((yl >> 2) == j) {
-      const int k = yl & 3;
-      if (k == 0) e.x -= grad_scale;
-      if (k == 1) e.y -= grad_scale;
-      if (k == 2) e.z -= grad_scale;
-      if (k == 3) e.w -= grad_scale;
+    // 6) dlogits block = grad_scale · (e · exp(m_i − lse) − onehot)
+    if (need_grad) {
+      const float scale = y_ok ? grad_scale * ex2_approx((m_i - lse) * kLog2e) : CUDART_NAN_F;
+      float4* dst4 = reinterpret_cast<float4*>(dlogits + tok * v + lo);
+      const int yl = mine ? static_cast<int>(y - lo) : -1;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const int j = threadIdx.x + r * kXentThreads;
+        if (j < nvec) {
+          float4 e = x[r];
+          e.x *= scale;
+          e.y *= scale;
+          e.z *= scale;
+          e.w *= scale;
+          if ((yl >> 2) == j) {
+            const int q = yl & 3;
+            if (q == 0) e.x -= grad_scale;
+            if (q == 1) e.y -= grad_scale;
+            if (q == 2) e.z -= grad_scale;
+            if (q == 3) e.w -= grad_scale;
+          }
+          __stcs(dst4 + j, e);
+        }
+      }
     }
-    __stcs(dst4 + j, e);
   }
+  cluster_sync_all();   // every peer's writes into this CTA have landed
 }
 
 // General path (any N, any alignment): one CTA per token walks the shards'
@@ -329,6 +423,58 @@ __global__ void __launch_bounds__(1024) loss_sum_kernel(const float* loss, int64
   if (threadIdx.x == 0) *out = part[0];
 }
 
+tp_status loss_sum_launch(const float* loss, int64_t T, float* loss_sum, cudaStream_t stream) {
+  loss_sum_kernel<<<1, 1024, 0, stream>>>(loss, T, loss_sum);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+template <int R>
+tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v,
+                              int N, float grad_scale, float* loss, float* loss_sum, float* dlogits,
+                              int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
+  static int cap[64][9] = {{0}};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t slice = static_cast<size_t>(v / N) * sizeof(float);
+  const size_t smem = 2 * ((slice + 127) & ~static_cast<size_t>(127));
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kXentThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = N;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  static size_t cap_smem[64][9] = {{0}};
+  int& c = cap[dev & 63][N];
+  if (c == 0 || cap_smem[dev & 63][N] != smem) {
+    if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return TP_ERR_CUDA;
+    cap_smem[dev & 63][N] = smem;
+    int clusters = 0;
+    cfg.gridDim = dim3(static_cast<unsigned>(N * num_sms()));
+    if (cudaOccupancyMaxActiveClusters(&clusters, vp_xent_cluster_kernel<R>, &cfg) != cudaSuccess ||
+        clusters <= 0) {
+      cudaGetLastError();
+      clusters = num_sms() / N > 0 ? num_sms() / N : 1;
+    }
+    c = clusters;
+  }
+  const int64_t clusters = T < c ? T : c;
+  cfg.gridDim = dim3(static_cast<unsigned>(clusters * N));
+  if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel<R>, logits, targets, T, v,
+                         static_cast<int>(v / N), grad_scale, loss, dlogits, argmax, dev_status,
+                         wait_limit_ns()) != cudaSuccess)
+    return TP_ERR_CUDA;
+  note_launches(1);
+  return loss_sum ? loss_sum_launch(loss, T, loss_sum, stream) : TP_OK;
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -350,37 +496,22 @@ tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T,
                          float grad_scale, float* loss, float* loss_sum, float* dlogits,
                          int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
   const int64_t vs = v / N;
-  const size_t slice_bytes = static_cast<size_t>(vs) * sizeof(float);
-  const bool cluster_ok = N >= 1 && N <= 8 && (vs % 4) == 0 && slice_bytes <= 200 * 1024 &&
-                          (T * N) < (1ll << 31) &&
+  const bool cluster_ok = N >= 1 && N <= 8 && (vs % 4) == 0 && vs <= 16 * 4 * kXentThreads &&
+                          (v % 4) == 0 &&
                           (reinterpret_cast<uintptr_t>(logits) % 16) == 0 &&
                           (dlogits == nullptr || (reinterpret_cast<uintptr_t>(dlogits) % 16) == 0);
   if (cluster_ok) {
-    static int configured_bytes[64] = {0};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (slice_bytes > 48 * 1024 && configured_bytes[dev & 63] < static_cast<int>(slice_bytes)) {
-      if (cudaFuncSetAttribute(vp_xent_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(slice_bytes)) != cudaSuccess)
-        return TP_ERR_CUDA;
-      configured_bytes[dev & 63] = static_cast<int>(slice_bytes);
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(T * N));
-    cfg.blockDim = dim3(kXentThreads);
-    cfg.dynamicSmemBytes = slice_bytes;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = N;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel, logits, targets, v, static_cast<int>(vs),
-                           grad_scale, loss, dlogits, argmax, dev_status) != cudaSuccess)
-      return TP_ERR_CUDA;
-    note_launches(1);
+    // float4 per thread: the smallest supported R with R * 256 * 4 >= vs
+    const int need = static_cast<int>((vs / 4 + kXentThreads - 1) / kXentThreads);
+    const int R = need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : 16;
+    if (R == 2) return xent_cluster_launch<2>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                              dlogits, argmax, dev_status, stream);
+    if (R == 4) return xent_cluster_launch<4>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                              dlogits, argmax, dev_status, stream);
+    if (R == 8) return xent_cluster_launch<8>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                              dlogits, argmax, dev_status, stream);
+    return xent_cluster_launch<16>(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits,
+                                   argmax, dev_status, stream);
   } else {
     vp_xent_rowwise_kernel<<<static_cast<unsigned>(T), kXentThreads, 0, stream>>>(
         logits, targets, v, N, grad_scale, loss, dlogits, argmax, dev_status);

@@ -99,7 +99,8 @@ def _xent_check(logits, targets, N, grad_scale, rows=None):
     return r, st
 
 
-@pytest.mark.parametrize("v,N", [(1024, 4), (48, 8), (50304, 8), (1002, 3), (4096, 1), (4000, 16)])
+@pytest.mark.parametrize("v,N", [(1024, 4), (48, 8), (50304, 8), (1002, 3), (4096, 1), (4000, 16),
+                                 (32768, 2), (8192, 8)])
 def test_xent_small(v, N):
     inp = tp_inputs.xent_logits(257, v, seed=5)
     r, st = _xent_check(inp["logits"], inp["targets"], N, 1.0 / 257)
