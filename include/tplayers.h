@@ -94,6 +94,15 @@ typedef enum {
   TP_OP_ROW_LINEAR_BWD = 4
 } tp_op;
 
+/*
+ * Diagnostics: check the bounded-wait path on the device.  Launches one CTA
+ * that waits, with the same bounded mbarrier wait the kernels use, on a
+ * barrier that nothing arrives on.  After limit_us microseconds the wait
+ * gives up, the kernel ORs TP_DEVERR_TIMEOUT into *dev_status (required) and
+ * returns normally: no trap, no fault, the context stays usable.
+ */
+TP_API tp_status tp_selftest_wait_timeout(int32_t* dev_status, uint32_t limit_us, void* stream);
+
 /* Human-readable text of a status code (static storage, never NULL). */
 TP_API const char* tp_status_string(tp_status s);
 

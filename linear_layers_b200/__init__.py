@@ -22,7 +22,8 @@ import torch
 
 __all__ = [
     "TPError", "lib", "library_path", "ACT_NONE", "ACT_GELU_TANH", "ACT_GELU_ERF",
-    "tp_status_string", "tp_version", "tp_launch_count", "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
+    "tp_status_string", "tp_version", "tp_launch_count", "tp_selftest_wait_timeout",
+    "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
     "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
     "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "vp_embed", "tp_logits_fwd", "vp_xent", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
@@ -48,6 +49,7 @@ _SIGS = {
     "tp_status_string": ([_I32], ctypes.c_char_p),
     "tp_version": ([], _I32),
     "tp_launch_count": ([], ctypes.c_uint64),
+    "tp_selftest_wait_timeout": ([_P, ctypes.c_uint32, _P], _I32),
     "tp_workspace_bytes": ([_I32, _I64, _I64, _I64, _I32], _SZ),
     "tp_mlp_fwd": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                     _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
@@ -148,6 +150,13 @@ def tp_version() -> int:
 def tp_launch_count() -> int:
     """Kernels the library has enqueued since it was loaded."""
     return int(lib().tp_launch_count())
+
+
+def tp_selftest_wait_timeout(dev_status, limit_us=1000):
+    """Run the device self-test of the bounded wait; returns the status word."""
+    _check(lib().tp_selftest_wait_timeout(_ptr(dev_status), int(limit_us),
+                                          _stream(dev_status.device)), "tp_selftest_wait_timeout")
+    return dev_status
 
 
 def tp_workspace_bytes(op: int, M: int, h: int, F: int, N: int) -> int:

@@ -75,17 +75,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// The sleeping form: a thread whose phase is not complete is suspended in
+// hardware until the phase completes or about kSuspendHintNs pass, instead
+// of spinning on issue slots the working warps of the SM need.  For waits
+// that are long by design (an epilogue waiting out a whole main loop); the
+// producer's and the MMA issuer's short, latency-critical waits spin.
+constexpr uint32_t kSuspendHintNs = 1000000u;
+
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // when `limit_ns` of global-timer time pass first or `*abort` is set by
 // another role of the same CTA.
+template <bool kSleep = false>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity,
                                                   uint64_t limit_ns,
                                                   const volatile int* abort) {
-  if (mbar_try_wait(bar, parity)) return true;
+  auto test = [&]() { return kSleep ? mbar_try_wait_sleep(bar, parity) : mbar_try_wait(bar, parity); };
+  if (test()) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
+    if (test()) return true;
+    if (kSleep || (it & 63u) == 0) {
       if (*abort) return false;
       if (global_timer_ns() - t0 > limit_ns) return false;
     }
@@ -285,10 +306,10 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred P;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 P, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, P;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -297,9 +318,9 @@ __device__ __forceinline__ bool mbar_wait_cluster_bounded(uint64_t* bar, uint32_
                                                           uint64_t limit_ns) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
-  for (uint32_t it = 1;; ++it) {
+  for (;;) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((it & 63u) == 0 && global_timer_ns() - t0 > limit_ns) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
