@@ -440,3 +440,54 @@ def xent_sharded(logits_, targets, N, grad_scale=1.0):
         "m": m,
         "S": S,
     }
+
+
+# ----------------------------------------------------------------------------
+# Vocabulary-parallel backward ([TP-ILL] §4.2: the output layer shares the
+# word embedding with the input layer; the table's gradient is the sum of the
+# two layers' gradients)
+# ----------------------------------------------------------------------------
+def logits_bwd(dlogits, H, E):
+    """Backward of logits = H·Eᵀ:  dH = dlogits·E,  dE = dlogitsᵀ·H."""
+    G, H, E = f64(dlogits), f64(H), f64(E)
+    return {"dH": G @ E, "dE": G.T @ H}
+
+
+def logits_bwd_sharded(dlogits, H, E, N):
+    """Shard i owns vocabulary rows [lo_i, hi_i): dE_i = dlogits_iᵀ·H is local,
+    dH = Σ_i dlogits_i·E_i is the all-reduce of the shards' partials."""
+    G, H, E = f64(dlogits), f64(H), f64(E)
+    offs = even_offsets(E.shape[0], N)
+    parts = [G[:, offs[i]:offs[i + 1]] @ E[offs[i]:offs[i + 1]] for i in range(N)]
+    dE = np.concatenate([G[:, offs[i]:offs[i + 1]].T @ H for i in range(N)], axis=0)
+    return {"dH": all_reduce_sum(parts), "dHparts": parts, "dE": dE}
+
+
+def embed_bwd(ids, dout, v):
+    """Gradient of out[t] = E[id_t] with respect to E: row x of the result is
+    the sum of dout[t] over the tokens with id_t = x (ids outside [0, v)
+    contribute nothing)."""
+    ids, G = i64(ids), f64(dout)
+    dE = np.zeros((v, G.shape[1]))
+    ok = (ids >= 0) & (ids < v)
+    np.add.at(dE, ids[ok], G[ok])
+    return dE
+
+
+def embed_bwd_sharded(ids, dout, v, N):
+    """Each shard accumulates the gradient rows of the ids in its own range."""
+    ids, G = i64(ids), f64(dout)
+    offs = even_offsets(v, N)
+    blocks = []
+    for i in range(N):
+        lo, hi = offs[i], offs[i + 1]
+        blk = np.zeros((hi - lo, G.shape[1]))
+        mine = (ids >= lo) & (ids < hi)
+        np.add.at(blk, ids[mine] - lo, G[mine])
+        blocks.append(blk)
+    return np.concatenate(blocks, axis=0)
+
+
+def tied_embedding_grad(dE_output, dE_input):
+    """The shared table's gradient: output-layer part plus input-layer part."""
+    return f64(dE_output) + f64(dE_input)

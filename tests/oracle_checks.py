@@ -382,4 +382,81 @@ def check_xent_argmax_ties(o):
         assert fn()["argmax"].tolist() == [3, 9, 0]
 
 
+# ----------------------------------------------------------------------------
+# vocabulary-parallel backward
+# ----------------------------------------------------------------------------
+def check_logits_bwd_fd_through_xent(o):
+    """dH, dE of L = Σ_t xent(H·Eᵀ)_t against central differences, and the
+    sharded form (per-shard dH partials summed) equal to the unsharded one."""
+    r = _rng(21)
+    T, h, v = 3, 4, 12
+    H = r.normal(size=(T, h))
+    E = r.normal(size=(v, h)) * 0.5
+    y = np.array([1, 7, 11])
+
+    def loss(H_, E_):
+        return float(o.xent(o.logits(H_, E_), y)["loss_sum"])
+
+    G = o.xent(o.logits(H, E), y, grad_scale=1.0)["dlogits"]
+    g = o.logits_bwd(G, H, E)
+    eps = 1e-6
+    for name, arr in (("dH", H), ("dE", E)):
+        fd = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            p, m = arr.copy(), arr.copy()
+            p[idx] += eps
+            m[idx] -= eps
+            fd[idx] = ((loss(p, E) - loss(m, E)) if name == "dH" else (loss(H, p) - loss(H, m))) / (2 * eps)
+        assert _rel(g[name], fd) < 1e-7, (name, _rel(g[name], fd))
+    for N in (1, 2, 3, 4):
+        s = o.logits_bwd_sharded(G, H, E, N)
+        assert _rel(s["dH"], g["dH"]) < 1e-13 and _rel(s["dE"], g["dE"]) < 1e-14
+        assert len(s["dHparts"]) == N
+
+
+def check_embed_bwd_vs_torch(o):
+    """Scatter-add of the embedding gradient against torch autograd (float64),
+    with repeated ids, and the sharded accumulation equal to it."""
+    import torch
+
+    r = _rng(22)
+    v, h = 40, 6
+    ids = np.array([3, 17, 3, 39, 0, 17, 3, 25])
+    G = r.normal(size=(ids.shape[0], h))
+    E = torch.from_numpy(r.normal(size=(v, h))).requires_grad_(True)
+    out = torch.nn.functional.embedding(torch.from_numpy(ids), E)
+    (out * torch.from_numpy(G)).sum().backward()
+    got = o.embed_bwd(ids, G, v)
+    assert _rel(got, E.grad.numpy()) < 1e-15
+    assert abs(got[3] - (G[0] + G[2] + G[6])).max() < 1e-15      # three repeats of id 3
+    for N in (1, 2, 4, 5, 8):
+        assert np.array_equal(o.embed_bwd_sharded(ids, G, v, N), got), N
+    bad = o.embed_bwd(np.array([-1, 40, 2]), r.normal(size=(3, h)), v)
+    assert not bad[:2].any() and bad[2].any() and not np.delete(bad, 2, axis=0).any()
+
+
+def check_tied_embedding_grad(o):
+    """One table used twice (input lookup and output logits): its gradient is
+    the sum of both paths' gradients (torch autograd in float64)."""
+    import torch
+
+    r = _rng(23)
+    v, h, T = 10, 4, 5
+    ids = np.array([1, 4, 4, 9, 0])
+    y = np.array([2, 4, 8, 0, 1])
+    W = r.normal(size=(h, h)) * 0.7
+    E = torch.from_numpy(r.normal(size=(v, h))).requires_grad_(True)
+    x = torch.nn.functional.embedding(torch.from_numpy(ids), E)
+    Hh = torch.tanh(x @ torch.from_numpy(W))            # any layer between the two uses
+    L = torch.nn.functional.cross_entropy(Hh @ E.T, torch.from_numpy(y), reduction="sum")
+    L.backward()
+    Hn = Hh.detach().numpy()
+    G = o.xent(o.logits(Hn, E.detach().numpy()), y)["dlogits"]
+    g_out = o.logits_bwd(G, Hn, E.detach().numpy())
+    # back through tanh(x W) to the looked-up rows
+    dx = (g_out["dH"] * (1 - Hn ** 2)) @ W.T
+    total = o.tied_embedding_grad(g_out["dE"], o.embed_bwd(ids, dx, v))
+    assert _rel(total, E.grad.numpy()) < 1e-12
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

@@ -141,6 +141,38 @@ def _m_argmax_last(mp):
     mp.setattr(O, "xent", bad)
 
 
+def _m_embed_bwd_overwrites_repeats(mp):
+    def bad(ids, dout, v):
+        ids, G = O.i64(ids), O.f64(dout)
+        dE = np.zeros((v, G.shape[1]))
+        ok = (ids >= 0) & (ids < v)
+        dE[ids[ok]] = G[ok]            # assignment instead of accumulation
+        return dE
+    mp.setattr(O, "embed_bwd", bad)
+
+
+def _m_logits_bwd_shards_reversed(mp):
+    orig = O.logits_bwd_sharded
+
+    def bad(dlogits, H, E, N):
+        r = orig(dlogits, H, E, N)
+        offs = O.even_offsets(O.f64(E).shape[0], N)
+        blocks = [r["dE"][offs[i]:offs[i + 1]] for i in range(N)]
+        r["dE"] = np.concatenate(blocks[::-1], axis=0)
+        return r
+    mp.setattr(O, "logits_bwd_sharded", bad)
+
+
+def _m_logits_bwd_drops_scale(mp):
+    orig = O.logits_bwd
+
+    def bad(dlogits, H, E):
+        r = orig(dlogits, H, E)
+        r["dE"] = 0.5 * r["dE"]
+        return r
+    mp.setattr(O, "logits_bwd", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
