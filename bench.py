@@ -11,7 +11,10 @@ input, all through the library's C ABI on the current stream:
      row-parallel output projection, forward + backward: 0.2516 TFLOP;
   3. vocabulary path, T=16384 (b=8, s=2048), v=50304 over N=8, h=4096:
      embedding lookup, logits = H·Eᵀ (fp32, 6.752 TFLOP), softmax
-     cross-entropy with loss, loss_sum, in-place dlogits and arg-max.
+     cross-entropy with loss, loss_sum, in-place dlogits and arg-max;
+  4. vocabulary backward: the cross-entropy gradient in bf16, dH = dlogits·E
+     and dE = dlogitsᵀ·H (13.5 TFLOP), and the input-embedding scatter-add
+     onto that dE (the gradient of the shared table).
 
 value = TP-MLP forward+backward TFLOP/s (all ranks' FLOPs / max-over-ranks
 device time of the MLP part); the cross-entropy half of the metric is the
@@ -45,9 +48,12 @@ VOC = dict(T=16384, v=50304, h=4096, N=8, e_std=0.02)
 MLP_FLOP = 12.0 * MLP["M"] * MLP["h"] * MLP["F"]                       # 6 GEMMs x 2MhF
 PROJ_FLOP = 6.0 * PROJ["M"] * PROJ["h"] * 3 * PROJ["h"] + 6.0 * PROJ["M"] * PROJ["h"] ** 2
 LOGITS_FLOP = 2.0 * VOC["T"] * VOC["v"] * VOC["h"]
+LOGITS_BWD_FLOP = 2.0 * LOGITS_FLOP
 # algorithmic bytes: read + write every logit once, plus targets / loss / argmax
 XENT_BYTES = 2 * 4 * VOC["T"] * VOC["v"] + VOC["T"] * (8 + 4 + 4)
 EMBED_BYTES = 2 * 2 * VOC["T"] * VOC["h"] + 8 * VOC["T"]
+# bf16-gradient cross-entropy: read fp32 logits, write bf16 dlogits
+XENT_BF16_BYTES = (4 + 2) * VOC["T"] * VOC["v"] + VOC["T"] * (8 + 4 + 4)
 
 SPEC_BF16_TFLOPS = 2250.0
 SPEC_HBM_GBS = 8000.0
@@ -171,8 +177,8 @@ def _prepare(dev, parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
     if "proj" in parts:
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
-    if any(p in parts for p in ("embed", "logits", "xent")):
-        vo = _prepare_vocab(dev, tpl, tp_inputs, torch, bf, "logits" not in parts and "xent" in parts)
+    if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd")):
+        vo = _prepare_vocab(dev, tpl, tp_inputs, torch, bf, "logits" not in parts)
     return g, pr, vo
 
 
@@ -215,6 +221,13 @@ def _prepare_vocab(dev, tpl, tp_inputs, torch, bf, fill_logits):
     vi = tp_inputs.vocab_inputs(VOC["T"], VOC["v"], VOC["h"], e_std=VOC["e_std"], seed=0)
     vo = {k: x.to(dev) for k, x in vi.items()}
     T, v = VOC["T"], VOC["v"]
+    vb = tp_inputs.vocab_bwd_inputs(T, v, VOC["h"], seed=1)
+    vo.update(dout=vb["dout"].to(dev), dlogits_bf=torch.empty(T, v, **bf),
+              dH=torch.empty(T, VOC["h"], **bf),
+              dE=torch.empty(v, VOC["h"], dtype=torch.float32, device=dev),
+              ws_eb=torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_EMBED_BWD, T, VOC["h"], v,
+                                                              VOC["N"])),
+                                dtype=torch.uint8, device=dev))
     vo.update(emb=torch.empty(T, VOC["h"], **bf), logits=torch.empty(T, v, dtype=torch.float32, device=dev),
               loss=torch.empty(T, dtype=torch.float32, device=dev),
               loss_sum=torch.empty(1, dtype=torch.float32, device=dev),
@@ -260,7 +273,27 @@ def _xent(tpl, vo, st):
                 loss_sum=vo["loss_sum"], dlogits=vo["logits"], argmax=vo["argmax"], dev_status=st)
 
 
+def _xent_bf16(tpl, vo, st):
+    tpl.vp_xent_bf16_grad(vo["logits"], vo["targets"], VOC["N"], grad_scale=1.0 / VOC["T"],
+                          loss=vo["loss"], loss_sum=vo["loss_sum"], dlogits=vo["dlogits_bf"],
+                          argmax=vo["argmax"], dev_status=st)
+
+
+def _logits_bwd(tpl, vo, st):
+    tpl.tp_logits_bwd(vo["dlogits_bf"], vo["H"], vo["E"], VOC["N"], dH=vo["dH"], dE=vo["dE"],
+                      dev_status=st)
+
+
+def _embed_bwd(tpl, vo, st):
+    tpl.vp_embed_bwd(vo["ids"], vo["dout"], vo["dE"], VOC["N"], ws=vo["ws_eb"], dev_status=st)
+
+
+# the step: every row of the hot path
 PARTS = ("mlp_fwd", "mlp_bwd", "proj", "embed", "logits", "xent")
+# the vocabulary backward (the next row beyond the hot path), timed in its own
+# loop after the step: logits (re-made, not reported) -> bf16-gradient loss ->
+# dH, dE -> input-embedding scatter-add onto dE
+BWD_PARTS = ("logits", "xent_bf16", "logits_bwd", "embed_bwd")
 
 
 def _e2e_mlp(tpl, torch, g, dev, steps):
@@ -350,17 +383,25 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    parts = [p for p in PARTS if p in args.parts.split(",")]
+    known = PARTS + BWD_PARTS[1:]
+    parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
-        raise SystemExit(f"--parts must name some of {','.join(PARTS)}")
+        raise SystemExit(f"--parts must name some of {','.join(known)}")
     if args.vocab_tokens:
         VOC["T"] = args.vocab_tokens
     full = parts == list(PARTS) and VOC["T"] == 16384
-    g, pr, vo = _prepare(dev, parts)
+    if full:   # the backward loop needs its vocabulary buffers too
+        parts_prep = parts + list(BWD_PARTS)
+    else:
+        parts_prep = parts
+    g, pr, vo = _prepare(dev, parts_prep)
     st = tpl.new_status(dev)
     fns = {"mlp_fwd": lambda: _mlp_fwd(tpl, g, st), "mlp_bwd": lambda: _mlp_bwd(tpl, g, st),
            "proj": lambda: _proj(tpl, pr, st), "embed": lambda: _embed(tpl, vo, st),
-           "logits": lambda: _logits(tpl, vo, st), "xent": lambda: _xent(tpl, vo, st)}
+           "logits": lambda: _logits(tpl, vo, st), "xent": lambda: _xent(tpl, vo, st),
+           "xent_bf16": lambda: _xent_bf16(tpl, vo, st),
+           "logits_bwd": lambda: _logits_bwd(tpl, vo, st),
+           "embed_bwd": lambda: _embed_bwd(tpl, vo, st)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -411,6 +452,28 @@ def run_gpu(args):
             torch.distributed.barrier()
             torch.distributed.destroy_process_group()
         return
+
+    # vocabulary backward: its own timed loop (not part of the step)
+    bwd_steps = max(5, min(args.steps, 20))
+    for _ in range(2):
+        for p in BWD_PARTS:
+            fns[p]()
+    torch.cuda.synchronize(dev)
+    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(BWD_PARTS) + 1)]
+           for _ in range(bwd_steps)]
+    for s in range(bwd_steps):
+        bev[s][0].record(stream)
+        for i, p in enumerate(BWD_PARTS):
+            fns[p]()
+            bev[s][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
+    bwd_ms = {p: sum(bev[s][i].elapsed_time(bev[s][i + 1]) for s in range(bwd_steps)) / bwd_steps
+              for i, p in enumerate(BWD_PARTS)}
+    bt = torch.tensor([bwd_ms[p] for p in BWD_PARTS], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(bt, op=torch.distributed.ReduceOp.MAX)
+    bwd_ms = {p: float(bt[i]) for i, p in enumerate(BWD_PARTS)}
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
@@ -467,9 +530,17 @@ def run_gpu(args):
                            "ms": round(part_ms["xent"] / K, 4)},
             "vp_embed": {"GBps": round(embed_gbs, 1), "frac_of_measured_hbm": round(embed_gbs / peaks["hbm_gbs"], 4),
                          "us": round(part_ms["embed"] / K * 1e3, 2)},
+            "vocab_bwd": {
+                "what": "next row, own loop of %d iterations after the step" % bwd_steps,
+                "xent_bf16_grad_ms": round(bwd_ms["xent_bf16"], 4),
+                "xent_bf16_grad_GBps": round(XENT_BF16_BYTES / (bwd_ms["xent_bf16"] / 1e3) / 1e9, 1),
+                "logits_bwd_ms": round(bwd_ms["logits_bwd"], 4),
+                "logits_bwd_tflops": round(LOGITS_BWD_FLOP / (bwd_ms["logits_bwd"] / 1e3) / 1e12, 1),
+                "embed_bwd_us": round(bwd_ms["embed_bwd"] * 1e3, 1),
+            },
             "parts_ms_per_step": {p: round(part_ms[p] / K, 4) for p in PARTS},
             "roofline": {
-                "kernel": "gemm_tc_kernel (all GEMM launches of the step)",
+                "kernel": "gemm_tc_kernel (all 13 GEMM launches of the step)",
                 "bound": "tensor",
                 "achieved": round(achieved, 2),
                 "peak": peak,

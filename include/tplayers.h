@@ -91,7 +91,8 @@ typedef enum {
   TP_OP_MLP_BWD = 1,
   TP_OP_ROW_LINEAR_FWD = 2,
   TP_OP_COL_LINEAR_BWD = 3,
-  TP_OP_ROW_LINEAR_BWD = 4
+  TP_OP_ROW_LINEAR_BWD = 4,
+  TP_OP_EMBED_BWD = 5     /* pass (T, h, v, N): T tokens */
 } tp_op;
 
 /*
@@ -305,6 +306,53 @@ TP_API tp_status tp_logits_fwd(const void* H, const void* E, int64_t T, int64_t 
 TP_API tp_status vp_xent(const float* logits, const int64_t* targets, int64_t T, int64_t v,
                   int32_t N, float grad_scale, float* loss, float* loss_sum,
                   float* dlogits, int32_t* argmax, int32_t* dev_status, void* stream);
+
+/*
+ * Vocabulary-parallel cross-entropy with a bf16 gradient   [TP-ILL] §5.
+ *
+ *   Exactly vp_xent, except that dlogits [T,v] is written in bf16 (round to
+ *   nearest even), the storage the output-layer backward GEMMs read; it is
+ *   required here and may not alias the fp32 logits.
+ */
+TP_API tp_status vp_xent_bf16_grad(const float* logits, const int64_t* targets, int64_t T,
+                                   int64_t v, int32_t N, float grad_scale, float* loss,
+                                   float* loss_sum, void* dlogits, int32_t* argmax,
+                                   int32_t* dev_status, void* stream);
+
+/*
+ * Output-embedding backward   [TP-ILL] §4.2 (the output layer shares the word
+ * embedding table).
+ *
+ *   dH = Σ_i dlogits_i·E_i   [T,h] bf16 — vocabulary shard i holds columns
+ *        [i·v/N, (i+1)·v/N) of dlogits and rows of E; the shards' partials are
+ *        summed in one accumulator (the all-reduce of the pages' layout);
+ *   dE = dlogitsᵀ·H          [v,h] fp32 — each shard's block of rows is its own.
+ *
+ *   dlogits [T,v] bf16, H [T,h] bf16, E [v,h] bf16 in; v % N == 0,
+ *   v % 8 == 0, h % 8 == 0.  dE is overwritten (see vp_embed_bwd to add the
+ *   input-side gradient of a tied table).
+ */
+TP_API tp_status tp_logits_bwd(const void* dlogits, const void* H, const void* E, int64_t T,
+                               int64_t h, int64_t v, int32_t N, void* dH, float* dE,
+                               int32_t* dev_status, void* stream);
+
+/*
+ * Vocabulary-parallel input-embedding backward   [TP-ILL] §4.1, §4.2.
+ *
+ *   dE[x] += Σ_{t: ids[t] = x} dout[t]   for every x in [0, v): shard i adds
+ *   the gradient rows of the ids in its own range [i·v/N, (i+1)·v/N).  The
+ *   sum over repeated ids runs in token order (tokens sorted by (id, token)),
+ *   so the result is bitwise reproducible; each touched row is written once.
+ *   Adding onto the dE of tp_logits_bwd gives the gradient of a table shared
+ *   by the input and output layers (the sum the pages prescribe).
+ *
+ *   ids [T] int64 (device), dout [T,h] bf16, dE [v,h] fp32 (read and
+ *   written); ids outside [0, v) are skipped and set TP_DEVERR_RANGE.
+ *   ws, ws_bytes >= tp_workspace_bytes(TP_OP_EMBED_BWD, T, h, v, N).
+ */
+TP_API tp_status vp_embed_bwd(const int64_t* ids, const void* dout, int64_t T, int64_t v,
+                              int64_t h, int32_t N, float* dE, void* ws, size_t ws_bytes,
+                              int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -26,13 +26,14 @@ __all__ = [
     "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
     "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
     "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
-    "vp_embed", "tp_logits_fwd", "vp_xent", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
+    "vp_embed", "tp_logits_fwd", "vp_xent", "vp_xent_bf16_grad", "tp_logits_bwd", "vp_embed_bwd",
+    "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
 ACT_NONE, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
-OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD = range(5)
+OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD, OP_EMBED_BWD = range(6)
 DEVERR_RANGE, DEVERR_TIMEOUT = 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -66,6 +67,9 @@ _SIGS = {
     "vp_embed": ([_P, _I64, _P, _I64, _I64, _I32, _I32, _P, _P, _P], _I32),
     "tp_logits_fwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _P, _P], _I32),
     "vp_xent": ([_P, _P, _I64, _I64, _I32, _F, _P, _P, _P, _P, _P, _P], _I32),
+    "vp_xent_bf16_grad": ([_P, _P, _I64, _I64, _I32, _F, _P, _P, _P, _P, _P, _P], _I32),
+    "tp_logits_bwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P], _I32),
+    "vp_embed_bwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _P, _SZ, _P, _P], _I32),
 }
 
 
@@ -351,3 +355,50 @@ def vp_xent(logits, targets, N, *, grad_scale=1.0, with_grad=True, with_argmax=T
                          _ptr(loss_sum), _ptr(dlogits), _ptr(argmax), _ptr(dev_status),
                          _stream(dev)), "vp_xent")
     return {"loss": loss, "loss_sum": loss_sum, "dlogits": dlogits, "argmax": argmax}
+
+
+def vp_xent_bf16_grad(logits, targets, N, *, grad_scale=1.0, with_argmax=True, loss=None,
+                      loss_sum=None, dlogits=None, argmax=None, dev_status=None):
+    """vp_xent with the gradient written in bf16.  Returns the same dict."""
+    T, v = logits.shape
+    dev = logits.device
+    loss = torch.empty(T, dtype=torch.float32, device=dev) if loss is None else loss
+    loss_sum = torch.empty(1, dtype=torch.float32, device=dev) if loss_sum is None else loss_sum
+    dlogits = torch.empty(T, v, dtype=torch.bfloat16, device=dev) if dlogits is None else dlogits
+    if with_argmax and argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=dev)
+    _contig(logits, targets, loss, dlogits, argmax)
+    if targets.dtype != torch.int64:
+        raise TypeError("targets must be int64")
+    _check(lib().vp_xent_bf16_grad(_ptr(logits), _ptr(targets), T, v, N, float(grad_scale),
+                                   _ptr(loss), _ptr(loss_sum), _ptr(dlogits), _ptr(argmax),
+                                   _ptr(dev_status), _stream(dev)), "vp_xent_bf16_grad")
+    return {"loss": loss, "loss_sum": loss_sum, "dlogits": dlogits, "argmax": argmax}
+
+
+def tp_logits_bwd(dlogits, H, E, N, *, dH=None, dE=None, dev_status=None):
+    """dH = Σ_i dlogits_i·E_i (bf16), dE = dlogitsᵀ·H (fp32).  Returns (dH, dE)."""
+    T, v = dlogits.shape
+    h = H.shape[1]
+    dev = H.device
+    dH = torch.empty(T, h, dtype=H.dtype, device=dev) if dH is None else dH
+    dE = torch.empty(v, h, dtype=torch.float32, device=dev) if dE is None else dE
+    _contig(dlogits, H, E, dH, dE)
+    _check(lib().tp_logits_bwd(_ptr(dlogits), _ptr(H), _ptr(E), T, h, v, N, _ptr(dH), _ptr(dE),
+                               _ptr(dev_status), _stream(dev)), "tp_logits_bwd")
+    return dH, dE
+
+
+def vp_embed_bwd(ids, dout, dE, N, *, ws=None, dev_status=None):
+    """dE[x] += Σ_{t: ids[t] = x} dout[t] (in place, token order).  Returns dE."""
+    T, h = dout.shape
+    v = dE.shape[0]
+    dev = dout.device
+    _contig(ids, dout, dE)
+    if ids.dtype != torch.int64:
+        raise TypeError("ids must be int64")
+    ws, wsb = _workspace(ws, OP_EMBED_BWD, T, h, v, N, dev)
+    _check(lib().vp_embed_bwd(_ptr(ids), _ptr(dout), T, v, h, N, _ptr(dE), _ptr(ws), wsb,
+                              _ptr(dev_status), _stream(dev)), "vp_embed_bwd")
+    return dE
+

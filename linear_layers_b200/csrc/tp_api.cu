@@ -21,8 +21,13 @@ tp_status vp_embed_launch(const int64_t* ids, int64_t T, const void* E, int64_t 
                           int N, int elem_bytes, void* out, int32_t* dev_status,
                           cudaStream_t stream);
 tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v, int N,
-                         float grad_scale, float* loss, float* loss_sum, float* dlogits,
-                         int32_t* argmax, int32_t* dev_status, cudaStream_t stream);
+                         float grad_scale, float* loss, float* loss_sum, void* dlogits,
+                         bool bf16_grad, int32_t* argmax, int32_t* dev_status,
+                         cudaStream_t stream);
+
+size_t embed_bwd_ws_bytes(int64_t T);
+tp_status vp_embed_bwd_launch(const int64_t* ids, const void* dout, int64_t T, int64_t v, int64_t h,
+                              float* dE, void* ws, int32_t* dev_status, cudaStream_t stream);
 
 namespace {
 
@@ -261,6 +266,8 @@ size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) 
       return row_split_ws(M, h, F, N, false) + dbias_ws(M, F);
     case TP_OP_ROW_LINEAR_BWD:
       return 0;
+    case TP_OP_EMBED_BWD:   // (T, h, v, N): sort keys of the T tokens
+      return align256(embed_bwd_ws_bytes(M));
   }
   return 0;
 }
@@ -556,8 +563,69 @@ tp_status vp_xent(const float* logits, const int64_t* targets, int64_t T, int64_
   if ((reinterpret_cast<uintptr_t>(logits) & 3) || (reinterpret_cast<uintptr_t>(targets) & 7))
     return TP_ERR_ALIGN;
   if (tp_status s = require_sm100()) return s;
-  return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, argmax,
+  return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, false,
+                        argmax, dev_status, as_stream(stream));
+}
+
+}  // extern "C"
+
+extern "C" {
+
+tp_status vp_xent_bf16_grad(const float* logits, const int64_t* targets, int64_t T, int64_t v,
+                            int32_t N, float grad_scale, float* loss, float* loss_sum,
+                            void* dlogits, int32_t* argmax, int32_t* dev_status, void* stream) {
+  if (!logits || !targets || !loss || !dlogits) return TP_ERR_NULL;
+  if (!dims_ok({T, v}) || N < 1 || v % N) return TP_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(logits) & 3) || (reinterpret_cast<uintptr_t>(targets) & 7) ||
+      (reinterpret_cast<uintptr_t>(dlogits) & 1))
+    return TP_ERR_ALIGN;
+  if (static_cast<const void*>(logits) == dlogits) return TP_ERR_UNSUPPORTED;
+  if (tp_status s = require_sm100()) return s;
+  return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, true, argmax,
                         dev_status, as_stream(stream));
+}
+
+tp_status tp_logits_bwd(const void* dlogits, const void* H, const void* E, int64_t T, int64_t h,
+                        int64_t v, int32_t N, void* dH, float* dE, int32_t* dev_status,
+                        void* stream) {
+  if (!dlogits || !H || !E || !dH || !dE) return TP_ERR_NULL;
+  if (!dims_ok({T, h, v}) || N < 1 || v % N) return TP_ERR_SHAPE;
+  if (h % 8 || v % 8 || !ptrs_aligned({dlogits, H, E, dH, dE})) return TP_ERR_ALIGN;
+  if (tp_status s = require_sm100()) return s;
+  cudaStream_t st = as_stream(stream);
+  std::vector<int64_t> offs;
+  if (tp_status s = shard_offsets(nullptr, v, N, offs)) return s;
+  // dH = Σ_i dlogits_i·E_i: the vocabulary shards are the K ranges of one accumulator
+  GemmProblem gh;
+  gh.A = dlogits; gh.lda = v; gh.a_mn = 0;
+  gh.B = E; gh.ldb = h; gh.b_mn = 1;            // E [v,h] = [K, N]
+  gh.M = static_cast<int>(T); gh.N = static_cast<int>(h); gh.K = static_cast<int>(v);
+  gh.epi = EPI_STORE_BF16;
+  gh.out0 = dH; gh.ldo = h;
+  gh.dev_status = dev_status;
+  if (tp_status s = run_row_parallel(gh, offs, nullptr, nullptr, 0, true, st)) return s;
+  // dE = dlogitsᵀ·H, one block of rows per shard
+  GemmProblem ge;
+  ge.A = dlogits; ge.lda = v; ge.a_mn = 1;      // dlogits [T,v] read as [K, M]
+  ge.B = H; ge.ldb = h; ge.b_mn = 1;            // H [T,h] = [K, N]
+  ge.M = static_cast<int>(v); ge.N = static_cast<int>(h); ge.K = static_cast<int>(T);
+  ge.epi = EPI_STORE_F32;
+  ge.out0 = dE; ge.ldo = h;
+  ge.dev_status = dev_status;
+  return gemm_tc_launch(ge, st);
+}
+
+tp_status vp_embed_bwd(const int64_t* ids, const void* dout, int64_t T, int64_t v, int64_t h,
+                       int32_t N, float* dE, void* ws, size_t ws_bytes, int32_t* dev_status,
+                       void* stream) {
+  if (!ids || !dout || !dE) return TP_ERR_NULL;
+  if (!dims_ok({T, v, h}) || N < 1 || v % N || T > (1ll << 31) || v > (1ll << 31))
+    return TP_ERR_SHAPE;
+  if (h % 8 || !ptrs_aligned({dout, dE, ws}) || (reinterpret_cast<uintptr_t>(ids) & 7))
+    return TP_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < embed_bwd_ws_bytes(T)) return TP_ERR_WORKSPACE;
+  if (tp_status s = require_sm100()) return s;
+  return vp_embed_bwd_launch(ids, dout, T, v, h, dE, ws, dev_status, as_stream(stream));
 }
 
 }  // extern "C"

@@ -18,8 +18,10 @@
 // distributed shared memory — the on-chip form of the all-reduce.  Each CTA
 // then writes its block of dlogits (one HBM write).
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <math_constants.h>
 
+#include <algorithm>
 #include <cstdint>
 
 #include "internal.h"
@@ -156,11 +158,28 @@ __device__ __forceinline__ float max4(const float4& a) {
   return fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w));
 }
 
-template <int R>
+// Gradient stores: fp32 float4, or four bf16 (round to nearest even) in 8 bytes.
+__device__ __forceinline__ void store_grad4(float* dst, int j, float4 e) {
+  __stcs(reinterpret_cast<float4*>(dst) + j, e);
+}
+__device__ __forceinline__ void store_grad4(__nv_bfloat16* dst, int j, float4 e) {
+  __nv_bfloat162 lo = __floats2bfloat162_rn(e.x, e.y);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(e.z, e.w);
+  uint2 w;
+  w.x = *reinterpret_cast<uint32_t*>(&lo);
+  w.y = *reinterpret_cast<uint32_t*>(&hi);
+  __stcs(reinterpret_cast<uint2*>(dst) + j, w);
+}
+__device__ __forceinline__ void store_grad1(float* dst, float e) { *dst = e; }
+__device__ __forceinline__ void store_grad1(__nv_bfloat16* dst, float e) {
+  *dst = __float2bfloat16_rn(e);
+}
+
+template <int R, typename GT>
 __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
     vp_xent_cluster_kernel(const float* logits, const int64_t* __restrict__ targets, int64_t T,
                            int64_t v, int vs, float grad_scale, float* __restrict__ loss,
-                           float* dlogits, int32_t* __restrict__ argmax, int32_t* dev_status,
+                           GT* dlogits, int32_t* __restrict__ argmax, int32_t* dev_status,
                            uint64_t wait_ns) {
   extern __shared__ __align__(128) unsigned char xsm[];   // two slices of the row
   __shared__ __align__(16) float rec[2][8][4];   // [token parity][shard] (m, s, tgt, amax)
@@ -336,7 +355,7 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
     // 6) dlogits block = grad_scale · (e · exp(m_i − lse) − onehot)
     if (need_grad) {
       const float scale = y_ok ? grad_scale * ex2_approx((m_i - lse) * kLog2e) : CUDART_NAN_F;
-      float4* dst4 = reinterpret_cast<float4*>(dlogits + tok * v + lo);
+      GT* dst = dlogits + tok * v + lo;
       const int yl = mine ? static_cast<int>(y - lo) : -1;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
@@ -354,7 +373,7 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
             if (q == 2) e.z -= grad_scale;
             if (q == 3) e.w -= grad_scale;
           }
-          __stcs(dst4 + j, e);
+          store_grad4(dst, j, e);
         }
       }
     }
@@ -364,9 +383,10 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
 
 // General path (any N, any alignment): one CTA per token walks the shards'
 // ranges in order, reading the row from global memory twice.
+template <typename GT>
 __global__ void __launch_bounds__(kXentThreads)
     vp_xent_rowwise_kernel(const float* logits, const int64_t* __restrict__ targets, int64_t v,
-                           int N, float grad_scale, float* __restrict__ loss, float* dlogits,
+                           int N, float grad_scale, float* __restrict__ loss, GT* dlogits,
                            int32_t* __restrict__ argmax, int32_t* dev_status) {
   __shared__ float red_v[kXentThreads / 32];
   __shared__ int red_i[kXentThreads / 32];
@@ -405,7 +425,7 @@ __global__ void __launch_bounds__(kXentThreads)
   for (int64_t j = threadIdx.x; j < v; j += kXentThreads) {
     float d = y_ok ? grad_scale * __expf(row[j] - lse) : CUDART_NAN_F;
     if (j == y) d -= grad_scale;
-    dlogits[tok * v + j] = d;
+    store_grad1(dlogits + tok * v + j, d);
   }
 }
 
@@ -429,9 +449,9 @@ tp_status loss_sum_launch(const float* loss, int64_t T, float* loss_sum, cudaStr
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
-template <int R>
+template <int R, typename GT>
 tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v,
-                              int N, float grad_scale, float* loss, float* loss_sum, float* dlogits,
+                              int N, float grad_scale, float* loss, float* loss_sum, GT* dlogits,
                               int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
   static int cap[64][9] = {{0}};
   int dev = 0;
@@ -452,13 +472,13 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   static size_t cap_smem[64][9] = {{0}};
   int& c = cap[dev & 63][N];
   if (c == 0 || cap_smem[dev & 63][N] != smem) {
-    if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return TP_ERR_CUDA;
     cap_smem[dev & 63][N] = smem;
     int clusters = 0;
     cfg.gridDim = dim3(static_cast<unsigned>(N * num_sms()));
-    if (cudaOccupancyMaxActiveClusters(&clusters, vp_xent_cluster_kernel<R>, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&clusters, vp_xent_cluster_kernel<R, GT>, &cfg) != cudaSuccess ||
         clusters <= 0) {
       cudaGetLastError();
       clusters = num_sms() / N > 0 ? num_sms() / N : 1;
@@ -467,12 +487,177 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   }
   const int64_t clusters = T < c ? T : c;
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * N));
-  if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel<R>, logits, targets, T, v,
+  if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel<R, GT>, logits, targets, T, v,
                          static_cast<int>(v / N), grad_scale, loss, dlogits, argmax, dev_status,
                          wait_limit_ns()) != cudaSuccess)
     return TP_ERR_CUDA;
   note_launches(1);
   return loss_sum ? loss_sum_launch(loss, T, loss_sum, stream) : TP_OK;
+}
+
+// ---------------------------------------------------------------------------
+// embedding backward: deterministic scatter-add of dOut rows into dE
+// ---------------------------------------------------------------------------
+// Sort keys (id << 32 | token) ascending: tokens with the same id become a
+// contiguous run in token order.  Ids outside [0, v) get the largest key and
+// are skipped.
+constexpr int64_t kSortSmemKeys = 16384;   // keys sorted inside one CTA (128 KB)
+constexpr uint64_t kNoKey = ~0ull;
+
+__device__ __forceinline__ uint64_t embed_key(const int64_t* ids, int64_t T, int64_t v, int64_t i,
+                                              int32_t* dev_status) {
+  if (i >= T) return kNoKey;
+  const int64_t id = ids[i];
+  if (id < 0 || id >= v) {
+    if (dev_status) atomicOr(dev_status, TP_DEVERR_RANGE);
+    return kNoKey;
+  }
+  return (static_cast<uint64_t>(id) << 32) | static_cast<uint32_t>(i);
+}
+
+// Bucketed sort (T <= kSortSmemKeys): CTA b owns ids [b·span, (b+1)·span).
+// It scans every token once, gathers its own tokens in token order (warp
+// ballots + a block scan), counts the in-range tokens with smaller ids (its
+// output offset), sorts its keys in shared memory and writes them in place,
+// so keys_out ends up sorted by (id, token); the last CTA fills the tail
+// (out-of-range tokens) with the no-key marker.
+constexpr int kBucketThreads = 1024;
+
+__global__ void __launch_bounds__(kBucketThreads)
+    embed_bucket_sort_kernel(const int64_t* __restrict__ ids, int64_t T, int64_t v, int64_t span,
+                             uint64_t* __restrict__ keys_out, int32_t* dev_status) {
+  extern __shared__ uint64_t sk[];
+  __shared__ int warp_cnt[kBucketThreads / 32];
+  __shared__ int warp_below[kBucketThreads / 32];
+  __shared__ int scan_tot[2];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t lo = blockIdx.x * span;
+  const int64_t hi = lo + span < v ? lo + span : v;
+  int count = 0;       // this bucket's tokens so far (uniform over the block)
+  int64_t below = 0;   // in-range tokens with id < lo
+  int64_t inrange = 0; // all in-range tokens (for the tail fill)
+  for (int64_t base = 0; base < T; base += kBucketThreads) {
+    const int64_t t = base + threadIdx.x;
+    const int64_t id = t < T ? ids[t] : -1;
+    const bool ok = t < T && id >= 0 && id < v;
+    if (t < T && !ok && blockIdx.x == 0 && dev_status) atomicOr(dev_status, TP_DEVERR_RANGE);
+    const bool mine = ok && id >= lo && id < hi;
+    const unsigned bm = __ballot_sync(0xffffffffu, mine);
+    const unsigned bb = __ballot_sync(0xffffffffu, ok && id < lo);
+    const unsigned bo = __ballot_sync(0xffffffffu, ok);
+    if (lane == 0) {
+      warp_cnt[warp] = __popc(bm);
+      warp_below[warp] = __popc(bb) + (__popc(bo) << 16);
+    }
+    __syncthreads();
+    if (warp == 0) {   // exclusive scan of the warp counts in warp order
+      const int c = warp_cnt[lane];
+      int incl = c;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int o = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += o;
+      }
+      int wb = warp_below[lane];
+#pragma unroll
+      for (int off = 16; off >= 1; off >>= 1) wb += __shfl_xor_sync(0xffffffffu, wb, off);
+      warp_cnt[lane] = incl - c;
+      if (lane == 31) scan_tot[0] = incl;
+      if (lane == 0) scan_tot[1] = wb;
+    }
+    __syncthreads();
+    const int pos = count + warp_cnt[warp] + __popc(bm & ((1u << lane) - 1u));
+    if (mine && pos < kSortSmemKeys)
+      sk[pos] = (static_cast<uint64_t>(id) << 32) | static_cast<uint32_t>(t);
+    count += scan_tot[0];
+    below += scan_tot[1] & 0xffff;
+    inrange += scan_tot[1] >> 16;
+    __syncthreads();
+  }
+  int P = 1;
+  while (P < count) P <<= 1;
+  for (int i = count + threadIdx.x; i < P; i += kBucketThreads) sk[i] = kNoKey;
+  __syncthreads();
+  for (int k = 2; k <= P; k <<= 1) {          // bitonic sort, ascending
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < P; i += kBucketThreads) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint64_t a = sk[i], b = sk[l];
+          if ((a > b) == ((i & k) == 0)) {
+            sk[i] = b;
+            sk[l] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int i = threadIdx.x; i < count; i += kBucketThreads) keys_out[below + i] = sk[i];
+  if (blockIdx.x == gridDim.x - 1)
+    for (int64_t i = inrange + threadIdx.x; i < T; i += kBucketThreads) keys_out[i] = kNoKey;
+}
+
+__global__ void embed_keys_kernel(const int64_t* __restrict__ ids, int64_t T, int64_t v, int64_t P,
+                                  uint64_t* __restrict__ keys, int32_t* dev_status) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i < P) keys[i] = embed_key(ids, T, v, i, dev_status);
+}
+
+// one compare-exchange stage of a global-memory bitonic sort (large T)
+__global__ void bitonic_stage_kernel(uint64_t* keys, int64_t P, int64_t j, int64_t k) {
+  const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  if (i >= P) return;
+  const int64_t l = i ^ j;
+  if (l > i) {
+    const uint64_t a = keys[i], b = keys[l];
+    if ((a > b) == ((i & k) == 0)) {
+      keys[i] = b;
+      keys[l] = a;
+    }
+  }
+}
+
+// One warp per (sorted position, 256-column chunk).  A warp whose position
+// starts a run of equal ids sums the run's dOut rows in token order (fp32)
+// and adds the sum into dE[id] — the only writer of that chunk of that row.
+constexpr int kSegWarps = 8;
+
+__global__ void __launch_bounds__(kSegWarps * 32)
+    embed_segsum_kernel(const uint64_t* __restrict__ keys, int64_t T,
+                        const __nv_bfloat16* __restrict__ dout, int64_t h, int64_t nchunks,
+                        float* __restrict__ dE) {
+  const int lane = threadIdx.x & 31;
+  const int64_t w = blockIdx.x * static_cast<int64_t>(kSegWarps) + (threadIdx.x >> 5);
+  const int64_t i = w / nchunks;
+  const int64_t chunk = w - i * nchunks;
+  if (i >= T) return;
+  const uint64_t key = keys[i];
+  if (key == kNoKey) return;
+  const uint32_t id = static_cast<uint32_t>(key >> 32);
+  if (i > 0 && keys[i - 1] != kNoKey && static_cast<uint32_t>(keys[i - 1] >> 32) == id) return;
+  const int64_t col = chunk * 256 + lane * 8;
+  if (col >= h) return;
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int64_t j = i; j < T; ++j) {
+    const uint64_t kj = keys[j];
+    if (kj == kNoKey || static_cast<uint32_t>(kj >> 32) != id) break;
+    const int64_t t = static_cast<int64_t>(static_cast<uint32_t>(kj));
+    const uint4 wv = __ldg(reinterpret_cast<const uint4*>(dout + t * h + col));
+    const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ww[q]));
+      acc[2 * q] += f.x;
+      acc[2 * q + 1] += f.y;
+    }
+  }
+  float4* dst = reinterpret_cast<float4*>(dE + static_cast<int64_t>(id) * h + col);
+  float4 a = dst[0], b = dst[1];
+  a.x += acc[0]; a.y += acc[1]; a.z += acc[2]; a.w += acc[3];
+  b.x += acc[4]; b.y += acc[5]; b.z += acc[6]; b.w += acc[7];
+  dst[0] = a;
+  dst[1] = b;
 }
 
 }  // namespace
@@ -492,9 +677,10 @@ tp_status vp_embed_launch(const int64_t* ids, int64_t T, const void* E, int64_t 
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
-tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v, int N,
-                         float grad_scale, float* loss, float* loss_sum, float* dlogits,
-                         int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
+template <typename GT>
+tp_status vp_xent_launch_t(const float* logits, const int64_t* targets, int64_t T, int64_t v,
+                           int N, float grad_scale, float* loss, float* loss_sum, GT* dlogits,
+                           int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
   const int64_t vs = v / N;
   const bool cluster_ok = N >= 1 && N <= 8 && (vs % 4) == 0 && vs <= 16 * 4 * kXentThreads &&
                           (v % 4) == 0 &&
@@ -504,26 +690,80 @@ tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T,
     // float4 per thread: the smallest supported R with R * 256 * 4 >= vs
     const int need = static_cast<int>((vs / 4 + kXentThreads - 1) / kXentThreads);
     const int R = need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : 16;
-    if (R == 2) return xent_cluster_launch<2>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
-                                              dlogits, argmax, dev_status, stream);
-    if (R == 4) return xent_cluster_launch<4>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
-                                              dlogits, argmax, dev_status, stream);
-    if (R == 8) return xent_cluster_launch<8>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
-                                              dlogits, argmax, dev_status, stream);
-    return xent_cluster_launch<16>(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits,
-                                   argmax, dev_status, stream);
+    if (R == 2) return xent_cluster_launch<2, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                  loss_sum, dlogits, argmax, dev_status, stream);
+    if (R == 4) return xent_cluster_launch<4, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                  loss_sum, dlogits, argmax, dev_status, stream);
+    if (R == 8) return xent_cluster_launch<8, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                  loss_sum, dlogits, argmax, dev_status, stream);
+    return xent_cluster_launch<16, GT>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                       dlogits, argmax, dev_status, stream);
+  }
+  vp_xent_rowwise_kernel<GT><<<static_cast<unsigned>(T), kXentThreads, 0, stream>>>(
+      logits, targets, v, N, grad_scale, loss, dlogits, argmax, dev_status);
+  note_launches(1);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  return loss_sum ? loss_sum_launch(loss, T, loss_sum, stream) : TP_OK;
+}
+
+tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v, int N,
+                         float grad_scale, float* loss, float* loss_sum, void* dlogits,
+                         bool bf16_grad, int32_t* argmax, int32_t* dev_status,
+                         cudaStream_t stream) {
+  if (bf16_grad)
+    return vp_xent_launch_t<__nv_bfloat16>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                           static_cast<__nv_bfloat16*>(dlogits), argmax,
+                                           dev_status, stream);
+  return vp_xent_launch_t<float>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                 static_cast<float*>(dlogits), argmax, dev_status, stream);
+}
+
+size_t embed_bwd_ws_bytes(int64_t T) {
+  int64_t P = 1;
+  while (P < T) P <<= 1;
+  return static_cast<size_t>(P) * sizeof(uint64_t);
+}
+
+tp_status vp_embed_bwd_launch(const int64_t* ids, const void* dout, int64_t T, int64_t v, int64_t h,
+                              float* dE, void* ws, int32_t* dev_status, cudaStream_t stream) {
+  int64_t P = 1;
+  while (P < T) P <<= 1;
+  uint64_t* keys = static_cast<uint64_t*>(ws);
+  if (P <= kSortSmemKeys) {
+    // a bucket may hold every token: room for min(P, kSortSmemKeys) keys
+    const int smem = static_cast<int>(P * sizeof(uint64_t));
+    static int configured[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (smem > 48 * 1024 && configured[dev & 63] < smem) {
+      if (cudaFuncSetAttribute(embed_bucket_sort_kernel,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kSortSmemKeys * sizeof(uint64_t))) != cudaSuccess)
+        return TP_ERR_CUDA;
+      configured[dev & 63] = static_cast<int>(kSortSmemKeys * sizeof(uint64_t));
+    }
+    const int64_t buckets = std::min<int64_t>(v, 2 * static_cast<int64_t>(num_sms()));
+    const int64_t span = (v + buckets - 1) / buckets;
+    embed_bucket_sort_kernel<<<static_cast<unsigned>((v + span - 1) / span), kBucketThreads, smem,
+                               stream>>>(ids, T, v, span, keys, dev_status);
+    note_launches(1);
   } else {
-    vp_xent_rowwise_kernel<<<static_cast<unsigned>(T), kXentThreads, 0, stream>>>(
-        logits, targets, v, N, grad_scale, loss, dlogits, argmax, dev_status);
+    const unsigned blocks = static_cast<unsigned>((P + 255) / 256);
+    embed_keys_kernel<<<blocks, 256, 0, stream>>>(ids, T, v, P, keys, dev_status);
     note_launches(1);
-    if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+    for (int64_t k = 2; k <= P; k <<= 1)
+      for (int64_t j = k >> 1; j > 0; j >>= 1) {
+        bitonic_stage_kernel<<<blocks, 256, 0, stream>>>(keys, P, j, k);
+        note_launches(1);
+      }
   }
-  if (loss_sum) {
-    loss_sum_kernel<<<1, 1024, 0, stream>>>(loss, T, loss_sum);
-    note_launches(1);
-    if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
-  }
-  return TP_OK;
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const int64_t nchunks = (h + 255) / 256;
+  const int64_t warps = T * nchunks;
+  embed_segsum_kernel<<<static_cast<unsigned>((warps + kSegWarps - 1) / kSegWarps), kSegWarps * 32,
+                        0, stream>>>(keys, T, static_cast<const __nv_bfloat16*>(dout), h, nchunks, dE);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 }  // namespace tpl

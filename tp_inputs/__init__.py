@@ -26,6 +26,7 @@ __all__ = [
     "vocab_inputs",
     "xent_logits",
     "attn_proj_inputs",
+    "vocab_bwd_inputs",
     "head_split",
     "WORKLOADS",
 ]
@@ -78,6 +79,19 @@ def xent_logits(T, v, *, logit_std=1.28, seed=0):
     logits = _randn(g, (T, v), logit_std, torch.float32)
     targets = torch.randint(0, v, (T,), generator=g, dtype=torch.int64)
     return {"logits": logits, "targets": targets}
+
+
+def vocab_bwd_inputs(T, v, h, *, seed=0, dlogit_std=1e-4):
+    """Inputs of the vocabulary backward: dlogits [T,v] bf16 ~ N(0, dlogit_std),
+    dout [T,h] bf16 ~ N(0,1) (gradient at the embedding output), dE0 [v,h]
+    fp32 ~ N(0, 1e-3) (a gradient the scatter-add accumulates onto), ids [T]
+    uniform in [0, v)."""
+    g = _gen(seed)
+    dlogits = _randn(g, (T, v), dlogit_std, torch.bfloat16)
+    dout = _randn(g, (T, h), 1.0, torch.bfloat16)
+    dE0 = _randn(g, (v, h), 1e-3, torch.float32)
+    ids = torch.randint(0, v, (T,), generator=g, dtype=torch.int64)
+    return {"dlogits": dlogits, "dout": dout, "dE0": dE0, "ids": ids}
 
 
 def head_split(n_heads: int, N: int):
