@@ -82,7 +82,8 @@ __global__ void __launch_bounds__(kEmbedWarps * 32)
 // ---------------------------------------------------------------------------
 // cross-entropy
 // ---------------------------------------------------------------------------
-constexpr int kXentThreads = 256;
+constexpr int kXentThreads = 256;          // row-wise fallback
+constexpr int kXentClusterThreads = 128;   // per CTA of the cluster kernel
 
 
 
@@ -175,8 +176,8 @@ __device__ __forceinline__ void store_grad1(__nv_bfloat16* dst, float e) {
   *dst = __float2bfloat16_rn(e);
 }
 
-template <int R, typename GT>
-__global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
+template <int R, int NT, typename GT>
+__global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
     vp_xent_cluster_kernel(const float* logits, const int64_t* __restrict__ targets, int64_t T,
                            int64_t v, int vs, float grad_scale, float* __restrict__ loss,
                            GT* dlogits, int32_t* __restrict__ argmax, int32_t* dev_status,
@@ -187,9 +188,9 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
   __shared__ __align__(8) uint64_t load_bar[2];
   // block-reduction scratch, double buffered by token parity: a warp that
   // runs ahead writes the other half while slow warps still read this one
-  __shared__ float red_m2[2][kXentThreads / 32];
-  __shared__ float red_s2[2][kXentThreads / 32];
-  __shared__ int red_i2[2][kXentThreads / 32];
+  __shared__ float red_m2[2][NT / 32];
+  __shared__ float red_s2[2][NT / 32];
+  __shared__ int red_i2[2][NT / 32];
 
   constexpr float kLog2e = 1.4426950408889634f;
   const uint32_t shard = cluster_ctarank();
@@ -242,7 +243,7 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
     float4 x[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const int j = threadIdx.x + r * kXentThreads;
+      const int j = threadIdx.x + r * NT;
       x[r] = j < nvec ? buf4[j]
                       : make_float4(-CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F, -CUDART_INF_F);
     }
@@ -264,14 +265,14 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
     }
     float m_i = red_m2[p][0];
 #pragma unroll
-    for (int w = 1; w < kXentThreads / 32; ++w) m_i = fmaxf(m_i, red_m2[p][w]);
+    for (int w = 1; w < NT / 32; ++w) m_i = fmaxf(m_i, red_m2[p][w]);
 
     // 2) first position of the maximum (only threads that hold it search)
     int it = 0x7fffffff;
     if (mt == m_i) {
 #pragma unroll
       for (int r = R - 1; r >= 0; --r) {   // elements ascend with r: keep the lowest
-        const int j = threadIdx.x + r * kXentThreads;
+        const int j = threadIdx.x + r * NT;
         if (x[r].w == m_i) it = 4 * j + 3;
         if (x[r].z == m_i) it = 4 * j + 2;
         if (x[r].y == m_i) it = 4 * j + 1;
@@ -303,7 +304,7 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
     float s_i = 0.f;
     int a_i = 0x7fffffff;
 #pragma unroll
-    for (int w = 0; w < kXentThreads / 32; ++w) {   // fixed order
+    for (int w = 0; w < NT / 32; ++w) {   // fixed order
       s_i += red_s2[p][w];
       a_i = min(a_i, red_i2[p][w]);
     }
@@ -359,7 +360,7 @@ __global__ void __launch_bounds__(kXentThreads, R <= 8 ? 4 : 2)
       const int yl = mine ? static_cast<int>(y - lo) : -1;
 #pragma unroll
       for (int r = 0; r < R; ++r) {
-        const int j = threadIdx.x + r * kXentThreads;
+        const int j = threadIdx.x + r * NT;
         if (j < nvec) {
           float4 e = x[r];
           e.x *= scale;
@@ -449,7 +450,7 @@ tp_status loss_sum_launch(const float* loss, int64_t T, float* loss_sum, cudaStr
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
-template <int R, typename GT>
+template <int R, int NT, typename GT>
 tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64_t T, int64_t v,
                               int N, float grad_scale, float* loss, float* loss_sum, GT* dlogits,
                               int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
@@ -459,7 +460,7 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   const size_t slice = static_cast<size_t>(v / N) * sizeof(float);
   const size_t smem = 2 * ((slice + 127) & ~static_cast<size_t>(127));
   cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kXentThreads);
+  cfg.blockDim = dim3(NT);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -472,13 +473,13 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   static size_t cap_smem[64][9] = {{0}};
   int& c = cap[dev & 63][N];
   if (c == 0 || cap_smem[dev & 63][N] != smem) {
-    if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R, NT, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return TP_ERR_CUDA;
     cap_smem[dev & 63][N] = smem;
     int clusters = 0;
     cfg.gridDim = dim3(static_cast<unsigned>(N * num_sms()));
-    if (cudaOccupancyMaxActiveClusters(&clusters, vp_xent_cluster_kernel<R, GT>, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&clusters, vp_xent_cluster_kernel<R, NT, GT>, &cfg) != cudaSuccess ||
         clusters <= 0) {
       cudaGetLastError();
       clusters = num_sms() / N > 0 ? num_sms() / N : 1;
@@ -487,7 +488,7 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   }
   const int64_t clusters = T < c ? T : c;
   cfg.gridDim = dim3(static_cast<unsigned>(clusters * N));
-  if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel<R, GT>, logits, targets, T, v,
+  if (cudaLaunchKernelEx(&cfg, vp_xent_cluster_kernel<R, NT, GT>, logits, targets, T, v,
                          static_cast<int>(v / N), grad_scale, loss, dlogits, argmax, dev_status,
                          wait_limit_ns()) != cudaSuccess)
     return TP_ERR_CUDA;
@@ -682,22 +683,26 @@ tp_status vp_xent_launch_t(const float* logits, const int64_t* targets, int64_t 
                            int N, float grad_scale, float* loss, float* loss_sum, GT* dlogits,
                            int32_t* argmax, int32_t* dev_status, cudaStream_t stream) {
   const int64_t vs = v / N;
-  const bool cluster_ok = N >= 1 && N <= 8 && (vs % 4) == 0 && vs <= 16 * 4 * kXentThreads &&
+  const bool cluster_ok = N >= 1 && N <= 8 && (vs % 4) == 0 && vs <= 16 * 4 * kXentClusterThreads &&
                           (v % 4) == 0 &&
                           (reinterpret_cast<uintptr_t>(logits) % 16) == 0 &&
                           (dlogits == nullptr || (reinterpret_cast<uintptr_t>(dlogits) % 16) == 0);
   if (cluster_ok) {
-    // float4 per thread: the smallest supported R with R * 256 * 4 >= vs
-    const int need = static_cast<int>((vs / 4 + kXentThreads - 1) / kXentThreads);
-    const int R = need <= 2 ? 2 : need <= 4 ? 4 : need <= 8 ? 8 : 16;
-    if (R == 2) return xent_cluster_launch<2, GT>(logits, targets, T, v, N, grad_scale, loss,
-                                                  loss_sum, dlogits, argmax, dev_status, stream);
-    if (R == 4) return xent_cluster_launch<4, GT>(logits, targets, T, v, N, grad_scale, loss,
-                                                  loss_sum, dlogits, argmax, dev_status, stream);
-    if (R == 8) return xent_cluster_launch<8, GT>(logits, targets, T, v, N, grad_scale, loss,
-                                                  loss_sum, dlogits, argmax, dev_status, stream);
-    return xent_cluster_launch<16, GT>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
-                                       dlogits, argmax, dev_status, stream);
+    // threads per CTA and float4 per thread (the smallest supported R with
+    // R * NT * 4 >= vs): fewer, fuller threads amortise the per-token reductions
+    constexpr int NT = kXentClusterThreads;
+    const int need = static_cast<int>((vs / 4 + NT - 1) / NT);
+    if (need <= 2) return xent_cluster_launch<2, NT, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                         loss_sum, dlogits, argmax, dev_status, stream);
+    if (need <= 4) return xent_cluster_launch<4, NT, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                         loss_sum, dlogits, argmax, dev_status, stream);
+    if (need <= 8) return xent_cluster_launch<8, NT, GT>(logits, targets, T, v, N, grad_scale, loss,
+                                                         loss_sum, dlogits, argmax, dev_status, stream);
+    if (need <= 13) return xent_cluster_launch<13, NT, GT>(logits, targets, T, v, N, grad_scale,
+                                                           loss, loss_sum, dlogits, argmax,
+                                                           dev_status, stream);
+    return xent_cluster_launch<16, NT, GT>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
+                                           dlogits, argmax, dev_status, stream);
   }
   vp_xent_rowwise_kernel<GT><<<static_cast<unsigned>(T), kXentThreads, 0, stream>>>(
       logits, targets, v, N, grad_scale, loss, dlogits, argmax, dev_status);
