@@ -378,13 +378,16 @@ def xent(logits_, targets, grad_scale=1.0):
         "loss_sum": loss.sum(),
         "dlogits": grad_scale * d,
         "argmax": np.argmax(L, axis=1).astype(np.int64),  # first maximum
+        "lse": lse,
     }
 
 
-def xent_sharded(logits_, targets, N, grad_scale=1.0):
+def xent_sharded(logits_, targets, N, grad_scale=1.0, offsets=None):
     """The vocabulary-parallel algorithm of [TP-ILL] §5, written out per shard.
 
-    Shard i holds columns [lo_i, hi_i).  It computes its maximum m_i, its sum
+    Shard i holds columns [lo_i, hi_i): the even split [i·v/N, (i+1)·v/N) of
+    §4.1, or the boundaries ``offsets`` (N+1 increasing column indices from 0
+    to v) when given.  It computes its maximum m_i, its sum
     s_i = Σ exp(l − m_i), its masked target logit and its local arg-max; the
     all-reduce combines m = max m_i, S = Σ s_i·exp(m_i − m) and the target
     logit; every shard then forms its own block of softmax − onehot and its
@@ -393,7 +396,8 @@ def xent_sharded(logits_, targets, N, grad_scale=1.0):
     L = f64(logits_)
     y = i64(targets)
     T, v = L.shape
-    offs = even_offsets(v, N)
+    offs = even_offsets(v, N) if offsets is None else [int(o) for o in offsets]
+    assert len(offs) == N + 1 and offs[0] == 0 and offs[-1] == v
     ms, ss, tg, amax_i, amax_v = [], [], [], [], []
     for i in range(N):
         Li = L[:, offs[i]:offs[i + 1]]
@@ -439,7 +443,30 @@ def xent_sharded(logits_, targets, N, grad_scale=1.0):
         "argmax": best_i.astype(np.int64),
         "m": m,
         "S": S,
+        "lse": lse,
     }
+
+
+# ----------------------------------------------------------------------------
+# Output layer and loss together ([TP-ILL] §4.2 followed by §5)
+# ----------------------------------------------------------------------------
+def linear_xent(H, E, targets, grad_scale=1.0):
+    """Softmax cross-entropy of the output-layer logits l = H·Eᵀ.
+
+    The result is defined by the two steps in sequence: the logits of §4.2
+    (vocabulary rows of the shared table E against the hidden states H), then
+    §5's loss on them.  Returns xent's outputs, among them the per-token
+    log-sum-exp lse_t = log Σ_j exp(l_tj) that the gradient
+    grad_scale·(exp(l − lse) − onehot(y)) is formed from.
+    """
+    return xent(logits(H, E), targets, grad_scale)
+
+
+def linear_xent_partitioned(H, E, targets, offsets, grad_scale=1.0):
+    """The same loss with the vocabulary cut at ``offsets`` (any increasing
+    column boundaries, not only an even split): per-part maxima, rescaled
+    sums and target logits combined by §5's rule."""
+    return xent_sharded(logits(H, E), targets, len(offsets) - 1, grad_scale, offsets=offsets)
 
 
 # ----------------------------------------------------------------------------

@@ -459,4 +459,94 @@ def check_tied_embedding_grad(o):
     assert _rel(total, E.grad.numpy()) < 1e-12
 
 
+# ----------------------------------------------------------------------------
+# output layer and loss together
+# ----------------------------------------------------------------------------
+def check_linear_xent_zero_hidden(o):
+    """H = 0 makes every logit 0: loss = lse = log v, dlogits = 1/v − onehot,
+    arg-max 0 (the lowest index of a v-way tie)."""
+    v, h = 37, 6
+    E = _rng(30).normal(size=(v, h))
+    y = np.array([0, 36, 5])
+    r = o.linear_xent(np.zeros((3, h)), E, y, grad_scale=2.0)
+    assert np.allclose(r["loss"], math.log(v), rtol=0, atol=1e-14)
+    assert np.allclose(r["lse"], math.log(v), rtol=0, atol=1e-14)
+    want = np.full((3, v), 1.0 / v)
+    want[np.arange(3), y] -= 1.0
+    assert np.allclose(r["dlogits"], 2.0 * want, rtol=0, atol=1e-15)
+    assert list(r["argmax"]) == [0, 0, 0]
+
+
+def check_linear_xent_permutation_table(o):
+    """E = c·P (a permutation that is not its own inverse, v = h) gives logits
+    c·H[:, π]; torch's cross_entropy and logsumexp in float64 on those."""
+    import torch
+
+    h = 9
+    perm = np.array([3, 0, 7, 1, 8, 2, 4, 6, 5])      # row j of E picks hidden unit perm[j]
+    assert not np.array_equal(perm[perm], np.arange(h))
+    c = 1.7
+    E = np.zeros((h, h))
+    E[np.arange(h), perm] = c
+    H = _rng(31).normal(size=(6, h))
+    y = np.array([0, 8, 3, 3, 5, 1])
+    r = o.linear_xent(H, E, y, grad_scale=1.0)
+    Lt = torch.from_numpy(c * H[:, perm])
+    yt = torch.from_numpy(y)
+    ref = torch.nn.functional.cross_entropy(Lt, yt, reduction="none").numpy()
+    assert _rel(r["loss"], ref) < 1e-14
+    assert _rel(r["lse"], torch.logsumexp(Lt, dim=1).numpy()) < 1e-14
+    assert np.array_equal(r["argmax"], torch.argmax(Lt, dim=1).numpy())
+    Lg = Lt.clone().requires_grad_(True)
+    torch.nn.functional.cross_entropy(Lg, yt, reduction="sum").backward()
+    assert _rel(r["dlogits"], Lg.grad.numpy()) < 1e-14
+
+
+def check_linear_xent_bruteforce(o):
+    """Scalar loops: loss_t = log Σ_j exp(Σ_k H_tk·E_jk) − Σ_k H_tk·E_{y_t,k}."""
+    r = _rng(32)
+    T, v, h = 3, 7, 5
+    H = r.normal(size=(T, h))
+    E = r.normal(size=(v, h))
+    y = [4, 0, 6]
+    got = o.linear_xent(H, E, np.array(y), grad_scale=0.5)
+    for t in range(T):
+        lt = [sum(H[t][k] * E[j][k] for k in range(h)) for j in range(v)]
+        z = sum(math.exp(x) for x in lt)
+        assert abs(got["lse"][t] - math.log(z)) < 1e-12
+        assert abs(got["loss"][t] - (math.log(z) - lt[y[t]])) < 1e-12
+        best = 0
+        for j in range(1, v):
+            if lt[j] > lt[best]:
+                best = j
+        assert got["argmax"][t] == best
+        for j in range(v):
+            want = 0.5 * (math.exp(lt[j]) / z - (1.0 if j == y[t] else 0.0))
+            assert abs(got["dlogits"][t, j] - want) < 1e-13
+
+
+def check_linear_xent_partitioned(o):
+    """Any cut of the vocabulary (128-wide slices with a short tail, a single
+    column, the whole range) combines to the unpartitioned loss; a maximum
+    tied across a cut goes to the lower index."""
+    r = _rng(33)
+    T, v, h = 5, 300, 8
+    H = r.normal(size=(T, h))
+    E = r.normal(size=(v, h))
+    y = np.array([0, 127, 128, 299, 150])
+    ref = o.linear_xent(H, E, y, grad_scale=0.25)
+    for offs in ([0, 128, 256, 300], [0, 1, 300], [0, 300], [0, 7, 8, 200, 299, 300]):
+        got = o.linear_xent_partitioned(H, E, y, offs, grad_scale=0.25)
+        assert _rel(got["loss"], ref["loss"]) < 1e-13, offs
+        assert _rel(got["lse"], ref["lse"]) < 1e-13, offs
+        assert _rel(got["dlogits"], ref["dlogits"]) < 1e-13, offs
+        assert np.array_equal(got["argmax"], ref["argmax"]), offs
+    # rows 40 and 200 of the table are equal: the tie straddles the cut at 128
+    E2 = E.copy()
+    E2[200] = E2[40] = 10.0 * H[2] / np.linalg.norm(H[2])
+    tie = o.linear_xent_partitioned(H, E2, y, [0, 128, 256, 300])
+    assert tie["argmax"][2] == 40
+    assert o.linear_xent(H, E2, y)["argmax"][2] == 40
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

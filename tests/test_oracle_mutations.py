@@ -173,6 +173,34 @@ def _m_logits_bwd_drops_scale(mp):
     mp.setattr(O, "logits_bwd", bad)
 
 
+def _m_lxent_transposed_table(mp):
+    def bad(H, E, targets, grad_scale=1.0):
+        return O.xent(O.f64(H) @ O.f64(E), targets, grad_scale)   # E used as [h,v]
+    mp.setattr(O, "linear_xent", bad)
+
+
+def _m_lxent_lse_without_max(mp):
+    orig = O.linear_xent
+
+    def bad(H, E, targets, grad_scale=1.0):
+        r = orig(H, E, targets, grad_scale)
+        L = O.logits(H, E)
+        r["lse"] = np.log(np.exp(L - L.max(axis=1)[:, None]).sum(axis=1))   # dropped + m
+        return r
+    mp.setattr(O, "linear_xent", bad)
+
+
+def _m_partitioned_tie_to_later_part(mp):
+    orig = O.xent_sharded
+
+    def bad(logits_, targets, N, grad_scale=1.0, offsets=None):
+        r = orig(logits_, targets, N, grad_scale, offsets)
+        L = O.f64(logits_)
+        r["argmax"] = (L.shape[1] - 1 - np.argmax(L[:, ::-1], axis=1)).astype(np.int64)
+        return r
+    mp.setattr(O, "xent_sharded", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
