@@ -177,7 +177,8 @@ def _prepare(dev, parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
     if "proj" in parts:
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
-    if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd")):
+    if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd",
+                                "lxent_fwd", "lxent_dlogits")):
         vo = _prepare_vocab(dev, tpl, tp_inputs, torch, bf, "logits" not in parts)
     return g, pr, vo
 
@@ -227,6 +228,9 @@ def _prepare_vocab(dev, tpl, tp_inputs, torch, bf, fill_logits):
               dE=torch.empty(v, VOC["h"], dtype=torch.float32, device=dev),
               ws_eb=torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_EMBED_BWD, T, VOC["h"], v,
                                                               VOC["N"])),
+                                dtype=torch.uint8, device=dev))
+    vo.update(lse=torch.empty(T, dtype=torch.float32, device=dev),
+              ws_lx=torch.empty(tpl.tp_workspace_bytes(tpl.OP_LINEAR_XENT, T, VOC["h"], v, VOC["N"]),
                                 dtype=torch.uint8, device=dev))
     vo.update(emb=torch.empty(T, VOC["h"], **bf), logits=torch.empty(T, v, dtype=torch.float32, device=dev),
               loss=torch.empty(T, dtype=torch.float32, device=dev),
@@ -288,12 +292,27 @@ def _embed_bwd(tpl, vo, st):
     tpl.vp_embed_bwd(vo["ids"], vo["dout"], vo["dE"], VOC["N"], ws=vo["ws_eb"], dev_status=st)
 
 
+def _lxent_fwd(tpl, vo, st):
+    tpl.tp_linear_xent_fwd(vo["H"], vo["E"], vo["targets"], VOC["N"], loss=vo["loss"],
+                           loss_sum=vo["loss_sum"], lse=vo["lse"], argmax=vo["argmax"],
+                           ws=vo["ws_lx"], dev_status=st)
+
+
+def _lxent_dlogits(tpl, vo, st):
+    tpl.tp_linear_xent_dlogits(vo["H"], vo["E"], vo["targets"], vo["lse"], VOC["N"],
+                               grad_scale=1.0 / VOC["T"], dlogits=vo["dlogits_bf"], dev_status=st)
+
+
 # the step: every row of the hot path
 PARTS = ("mlp_fwd", "mlp_bwd", "proj", "embed", "logits", "xent")
 # the vocabulary backward (the next row beyond the hot path), timed in its own
 # loop after the step: logits (re-made, not reported) -> bf16-gradient loss ->
 # dH, dE -> input-embedding scatter-add onto dE
 BWD_PARTS = ("logits", "xent_bf16", "logits_bwd", "embed_bwd")
+# output layer + loss without the logits matrix (the next row after that),
+# also in its own loop: statistics GEMM + combine, then the recomputing
+# gradient GEMM
+FUSED_PARTS = ("lxent_fwd", "lxent_dlogits")
 
 
 def _e2e_mlp(tpl, torch, g, dev, steps):
@@ -361,6 +380,30 @@ def _e2e_mlp(tpl, torch, g, dev, steps):
     return ms, h2d, d2h
 
 
+def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world):
+    """Average ms per part over nsteps iterations of plist (2 untimed first),
+    CUDA events on the launching stream, max over ranks."""
+    for _ in range(2):
+        for p in plist:
+            fns[p]()
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plist) + 1)]
+          for _ in range(nsteps)]
+    for s in range(nsteps):
+        ev[s][0].record(stream)
+        for i, p in enumerate(plist):
+            fns[p]()
+            ev[s][i + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
+    ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(nsteps)) / nsteps
+          for i in range(len(plist))]
+    t = torch.tensor(ms, dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return {p: float(t[i]) for i, p in enumerate(plist)}
+
+
 def run_gpu(args):
     import torch
 
@@ -383,15 +426,15 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    known = PARTS + BWD_PARTS[1:]
+    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS
     parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
         raise SystemExit(f"--parts must name some of {','.join(known)}")
     if args.vocab_tokens:
         VOC["T"] = args.vocab_tokens
     full = parts == list(PARTS) and VOC["T"] == 16384
-    if full:   # the backward loop needs its vocabulary buffers too
-        parts_prep = parts + list(BWD_PARTS)
+    if full:   # the side loops need their vocabulary buffers too
+        parts_prep = parts + list(BWD_PARTS) + list(FUSED_PARTS)
     else:
         parts_prep = parts
     g, pr, vo = _prepare(dev, parts_prep)
@@ -401,7 +444,9 @@ def run_gpu(args):
            "logits": lambda: _logits(tpl, vo, st), "xent": lambda: _xent(tpl, vo, st),
            "xent_bf16": lambda: _xent_bf16(tpl, vo, st),
            "logits_bwd": lambda: _logits_bwd(tpl, vo, st),
-           "embed_bwd": lambda: _embed_bwd(tpl, vo, st)}
+           "embed_bwd": lambda: _embed_bwd(tpl, vo, st),
+           "lxent_fwd": lambda: _lxent_fwd(tpl, vo, st),
+           "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -453,27 +498,11 @@ def run_gpu(args):
             torch.distributed.destroy_process_group()
         return
 
-    # vocabulary backward: its own timed loop (not part of the step)
-    bwd_steps = max(5, min(args.steps, 20))
-    for _ in range(2):
-        for p in BWD_PARTS:
-            fns[p]()
-    torch.cuda.synchronize(dev)
-    bev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(BWD_PARTS) + 1)]
-           for _ in range(bwd_steps)]
-    for s in range(bwd_steps):
-        bev[s][0].record(stream)
-        for i, p in enumerate(BWD_PARTS):
-            fns[p]()
-            bev[s][i + 1].record(stream)
-    torch.cuda.synchronize(dev)
-    assert int(st.item()) == 0, f"device status {int(st.item())}"
-    bwd_ms = {p: sum(bev[s][i].elapsed_time(bev[s][i + 1]) for s in range(bwd_steps)) / bwd_steps
-              for i, p in enumerate(BWD_PARTS)}
-    bt = torch.tensor([bwd_ms[p] for p in BWD_PARTS], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(bt, op=torch.distributed.ReduceOp.MAX)
-    bwd_ms = {p: float(bt[i]) for i, p in enumerate(BWD_PARTS)}
+    # vocabulary backward and the fused output layer + loss: their own timed
+    # loops (not part of the step)
+    side_steps = max(5, min(args.steps, 20))
+    bwd_ms = _side_loop(torch, fns, BWD_PARTS, side_steps, stream, dev, st, world)
+    fused_ms = _side_loop(torch, fns, FUSED_PARTS, side_steps, stream, dev, st, world)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
@@ -531,12 +560,23 @@ def run_gpu(args):
             "vp_embed": {"GBps": round(embed_gbs, 1), "frac_of_measured_hbm": round(embed_gbs / peaks["hbm_gbs"], 4),
                          "us": round(part_ms["embed"] / K * 1e3, 2)},
             "vocab_bwd": {
-                "what": "next row, own loop of %d iterations after the step" % bwd_steps,
+                "what": "next row, own loop of %d iterations after the step" % side_steps,
                 "xent_bf16_grad_ms": round(bwd_ms["xent_bf16"], 4),
                 "xent_bf16_grad_GBps": round(XENT_BF16_BYTES / (bwd_ms["xent_bf16"] / 1e3) / 1e9, 1),
                 "logits_bwd_ms": round(bwd_ms["logits_bwd"], 4),
                 "logits_bwd_tflops": round(LOGITS_BWD_FLOP / (bwd_ms["logits_bwd"] / 1e3) / 1e12, 1),
                 "embed_bwd_us": round(bwd_ms["embed_bwd"] * 1e3, 1),
+            },
+            "linear_xent": {
+                "what": "output layer + loss without the [T,v] logits: statistics GEMM + combine "
+                        "(loss, lse, argmax), then the recomputing bf16-gradient GEMM; own loop of "
+                        "%d iterations" % side_steps,
+                "fwd_ms": round(fused_ms["lxent_fwd"], 4),
+                "fwd_tflops": round(LOGITS_FLOP / (fused_ms["lxent_fwd"] / 1e3) / 1e12, 1),
+                "unfused_logits_plus_xent_ms": round((part_ms["logits"] + part_ms["xent"]) / K, 4),
+                "dlogits_ms": round(fused_ms["lxent_dlogits"], 4),
+                "dlogits_tflops": round(LOGITS_FLOP / (fused_ms["lxent_dlogits"] / 1e3) / 1e12, 1),
+                "logits_bytes_not_stored": VOC["T"] * VOC["v"] * 4,
             },
             "parts_ms_per_step": {p: round(part_ms[p] / K, 4) for p in PARTS},
             "roofline": {

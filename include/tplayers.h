@@ -92,7 +92,8 @@ typedef enum {
   TP_OP_ROW_LINEAR_FWD = 2,
   TP_OP_COL_LINEAR_BWD = 3,
   TP_OP_ROW_LINEAR_BWD = 4,
-  TP_OP_EMBED_BWD = 5     /* pass (T, h, v, N): T tokens */
+  TP_OP_EMBED_BWD = 5,    /* pass (T, h, v, N): T tokens */
+  TP_OP_LINEAR_XENT = 6   /* pass (T, h, v, N) */
 } tp_op;
 
 /*
@@ -353,6 +354,54 @@ TP_API tp_status tp_logits_bwd(const void* dlogits, const void* H, const void* E
 TP_API tp_status vp_embed_bwd(const int64_t* ids, const void* dout, int64_t T, int64_t v,
                               int64_t h, int32_t N, float* dE, void* ws, size_t ws_bytes,
                               int32_t* dev_status, void* stream);
+
+/*
+ * Output layer and cross-entropy in one pass, without the logits matrix
+ *   [TP-ILL] §4.2 (logits = H·Eᵀ against the shared table) and §5 (the loss
+ *   from per-part maxima and rescaled sums, so that no part of the [T,v]
+ *   logits has to be gathered).
+ *
+ *   The logits GEMM keeps its accumulators on chip: for every 128-column
+ *   slice of every row it records the maximum m_k, s_k = Σ exp(l − m_k), the
+ *   first column holding m_k and, in the slice that holds the target, the
+ *   target logit.  A second kernel combines the slices by §5's rule,
+ *   m = max m_k, S = Σ s_k·exp(m_k − m), and writes
+ *
+ *     loss[t]    = m + log S − l[t, y_t]            fp32 [T]
+ *     lse[t]     = m + log S                        fp32 [T]   (nullable)
+ *     argmax[t]  = lowest index of the row maximum  int32 [T]  (nullable)
+ *     loss_sum   = Σ_t loss[t], fixed order         fp32 [1]   (nullable)
+ *
+ *   The vocabulary shards i (rows [i·v/N, (i+1)·v/N) of E, v % N == 0) are
+ *   memory partitions of E; the slices are a finer partition of the same
+ *   columns, combined by the same rule.  H [T,h] bf16, E [v,h] bf16,
+ *   targets [T] int64; h % 8 == 0, H and E 16-byte aligned.  A target outside
+ *   [0, v) sets TP_DEVERR_RANGE and gives loss NaN.
+ *   ws, ws_bytes >= tp_workspace_bytes(TP_OP_LINEAR_XENT, T, h, v, N)
+ *   (the slice statistics: 12·ceil(v/128)·T bytes plus 4·T).
+ *   No counterpart of the fused form is printed on the pages: it is their
+ *   output-layer GEMM and §5 loss evaluated without storing the logits.
+ */
+TP_API tp_status tp_linear_xent_fwd(const void* H, const void* E, const int64_t* targets,
+                                    int64_t T, int64_t h, int64_t v, int32_t N, float* loss,
+                                    float* loss_sum, float* lse, int32_t* argmax, void* ws,
+                                    size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * Gradient of that loss with respect to the logits, recomputed   [TP-ILL] §5.
+ *
+ *   dlogits[t, j] = grad_scale · (exp(l[t, j] − lse[t]) − [j = y_t])   bf16 [T,v]
+ *
+ *   with l = H·Eᵀ recomputed by the GEMM in fp32 and lse from
+ *   tp_linear_xent_fwd, so that the fp32 logits are never stored; the result
+ *   is the input of tp_logits_bwd.  v % 8 == 0, h % 8 == 0, H, E and dlogits
+ *   16-byte aligned.  A row whose target lies outside [0, v) is NaN and sets
+ *   TP_DEVERR_RANGE.
+ */
+TP_API tp_status tp_linear_xent_dlogits(const void* H, const void* E, const int64_t* targets,
+                                        const float* lse, int64_t T, int64_t h, int64_t v,
+                                        int32_t N, float grad_scale, void* dlogits,
+                                        int32_t* dev_status, void* stream);
 
 #ifdef __cplusplus
 }

@@ -28,12 +28,14 @@ __all__ = [
     "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "vp_embed", "tp_logits_fwd", "vp_xent", "vp_xent_bf16_grad", "tp_logits_bwd", "vp_embed_bwd",
     "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
+    "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
 ACT_NONE, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
-OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD, OP_EMBED_BWD = range(6)
+(OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD, OP_EMBED_BWD,
+ OP_LINEAR_XENT) = range(7)
 DEVERR_RANGE, DEVERR_TIMEOUT = 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -70,6 +72,9 @@ _SIGS = {
     "vp_xent_bf16_grad": ([_P, _P, _I64, _I64, _I32, _F, _P, _P, _P, _P, _P, _P], _I32),
     "tp_logits_bwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P], _I32),
     "vp_embed_bwd": ([_P, _P, _I64, _I64, _I64, _I32, _P, _P, _SZ, _P, _P], _I32),
+    "tp_linear_xent_fwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _SZ,
+                            _P, _P], _I32),
+    "tp_linear_xent_dlogits": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _F, _P, _P, _P], _I32),
 }
 
 
@@ -402,3 +407,42 @@ def vp_embed_bwd(ids, dout, dE, N, *, ws=None, dev_status=None):
                               _ptr(dev_status), _stream(dev)), "vp_embed_bwd")
     return dE
 
+
+def tp_linear_xent_fwd(H, E, targets, N, *, with_argmax=True, loss=None, loss_sum=None, lse=None,
+                       argmax=None, ws=None, dev_status=None):
+    """Cross-entropy of logits = H·Eᵀ without storing the logits.
+
+    Returns {"loss" [T] fp32, "loss_sum" [1] fp32, "lse" [T] fp32, "argmax" [T] int32 or None}.
+    """
+    T, h = H.shape
+    v = E.shape[0]
+    dev = H.device
+    loss = torch.empty(T, dtype=torch.float32, device=dev) if loss is None else loss
+    loss_sum = torch.empty(1, dtype=torch.float32, device=dev) if loss_sum is None else loss_sum
+    lse = torch.empty(T, dtype=torch.float32, device=dev) if lse is None else lse
+    if with_argmax and argmax is None:
+        argmax = torch.empty(T, dtype=torch.int32, device=dev)
+    _contig(H, E, targets, loss, lse, argmax)
+    if targets.dtype != torch.int64:
+        raise TypeError("targets must be int64")
+    ws, wsb = _workspace(ws, OP_LINEAR_XENT, T, h, v, N, dev)
+    _check(lib().tp_linear_xent_fwd(_ptr(H), _ptr(E), _ptr(targets), T, h, v, N, _ptr(loss),
+                                    _ptr(loss_sum), _ptr(lse), _ptr(argmax), _ptr(ws), wsb,
+                                    _ptr(dev_status), _stream(dev)), "tp_linear_xent_fwd")
+    return {"loss": loss, "loss_sum": loss_sum, "lse": lse, "argmax": argmax}
+
+
+def tp_linear_xent_dlogits(H, E, targets, lse, N, *, grad_scale=1.0, dlogits=None,
+                           dev_status=None):
+    """bf16 dlogits = grad_scale·(exp(H·Eᵀ − lse) − onehot), logits recomputed on chip."""
+    T, h = H.shape
+    v = E.shape[0]
+    dev = H.device
+    dlogits = torch.empty(T, v, dtype=torch.bfloat16, device=dev) if dlogits is None else dlogits
+    _contig(H, E, targets, lse, dlogits)
+    if targets.dtype != torch.int64:
+        raise TypeError("targets must be int64")
+    _check(lib().tp_linear_xent_dlogits(_ptr(H), _ptr(E), _ptr(targets), _ptr(lse), T, h, v, N,
+                                        float(grad_scale), _ptr(dlogits), _ptr(dev_status),
+                                        _stream(dev)), "tp_linear_xent_dlogits")
+    return dlogits

@@ -69,6 +69,13 @@ struct GemmArgs {
   int* counters;
   int32_t* dev_status;
   uint64_t wait_ns;
+  const int64_t* targets;           // EPI_XENT_*
+  float* stat_m;
+  float* stat_s;
+  int32_t* stat_i;
+  float* tgt_logit;
+  const float* row_lse;
+  float grad_scale;
 };
 
 struct __align__(64) GemmParams {
@@ -194,6 +201,14 @@ __device__ __forceinline__ void unpack_bf16x32(const uint4 (&w)[4], float* v) {
     }
   }
 }
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
 
 // Transpose-reduce across the warp: lane l ends with Σ_lanes v[l].
 __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
@@ -509,6 +524,96 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                             a.N - col0);
           }
         }
+      } else if constexpr (EPI == EPI_XENT_STATS) {
+        // Softmax statistics of this warp's 128-column slice of each row: the
+        // maximum m, s = Σ exp(acc − m) (rescaled whenever m grows) and the
+        // first column holding m; the thread whose slice holds the row's
+        // target keeps that accumulator.  Columns past the vocabulary are
+        // left out.  Nothing of the logits matrix is written.
+        const int slice = tn * (BN / kXentSlice) + half;
+        if (slice * kXentSlice < a.N) {   // warp-uniform
+          const int64_t tgt = row_ok ? a.targets[row] : -1;
+          float m = -INFINITY, ssum = 0.0f;
+          int arg = 0;
+#pragma unroll 1
+          for (int c = c0; c < c0 + 4; ++c) {
+            const int col0 = tn * BN + c * 32;
+            if (col0 >= a.N) break;        // warp-uniform
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_base + c * 32, r);
+            tc_wait_ld();
+            float v[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+            if (col0 + 32 > a.N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j >= a.N) v[j] = -INFINITY;
+            }
+            if (tgt >= col0 && tgt < col0 + 32) {
+              float tl = 0.0f;
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (col0 + j == tgt) tl = v[j];
+              a.tgt_logit[row] = tl;
+            }
+            float cm[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              cm[j] = fmaxf(fmaxf(v[4 * j], v[4 * j + 1]), fmaxf(v[4 * j + 2], v[4 * j + 3]));
+            const float cmax = fmaxf(fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3])),
+                                     fmaxf(fmaxf(cm[4], cm[5]), fmaxf(cm[6], cm[7])));
+            int ci = 31;
+#pragma unroll
+            for (int j = 31; j >= 0; --j)
+              if (v[j] == cmax) ci = j;
+            if (cmax > m) arg = col0 + ci;
+            const float mn = fmaxf(m, cmax);
+            const float mn_l2 = mn * kLog2e;
+            float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+            for (int j = 0; j < 32; ++j) ps[j & 3] += ex2_approx(fmaf(v[j], kLog2e, -mn_l2));
+            // m = −inf before the first chunk: the old sum (0) is scaled by 0
+            ssum = fmaf(ssum, ex2_approx((m - mn) * kLog2e), (ps[0] + ps[1]) + (ps[2] + ps[3]));
+            m = mn;
+          }
+          if (row_ok) {
+            const int64_t o = static_cast<int64_t>(slice) * a.M + row;
+            a.stat_m[o] = m;
+            a.stat_s[o] = ssum;
+            a.stat_i[o] = arg;
+          }
+        }
+      } else if constexpr (EPI == EPI_XENT_GRAD) {
+        // grad_scale·(softmax − onehot) from the recomputed logits and the
+        // row's log-sum-exp; a row whose target lies outside the vocabulary
+        // gets NaN (its loss is undefined)
+        float lse_l2 = 0.0f;
+        int64_t tgt = -1;
+        bool tgt_ok = false;
+        if (row_ok) {
+          lse_l2 = a.row_lse[row] * kLog2e;
+          tgt = a.targets[row];
+          tgt_ok = tgt >= 0 && tgt < a.N;
+          if (!tgt_ok && tn == 0 && half == 0 && a.dev_status) atomicOr(a.dev_status, TP_DEVERR_RANGE);
+        }
+        const float gs = tgt_ok ? a.grad_scale : __int_as_float(0x7fc00000);
+#pragma unroll 1
+        for (int c = c0; c < c0 + 4; ++c) {
+          const int col0 = tn * BN + c * 32;
+          if (col0 >= a.N) break;          // warp-uniform
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tc_wait_ld();
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            const float p = ex2_approx(fmaf(__uint_as_float(r[j]), kLog2e, -lse_l2));
+            v[j] = gs * (col0 + j == tgt ? p - 1.0f : p);
+          }
+          if (row_ok)
+            store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v, a.N - col0);
+        }
       } else {
         uint4 aux_w[4];
         if constexpr (EPI == EPI_DACT) {   // U for the first chunk
@@ -701,6 +806,8 @@ tp_status launch_epi(const GemmParams& prm, int epi, int slots, cudaStream_t str
     case EPI_DACT: return launch_impl<CG, EPI_DACT>(prm, slots, stream);
     case EPI_STORE_F32: return launch_impl<CG, EPI_STORE_F32>(prm, slots, stream);
     case EPI_SPLIT_SUM: return launch_impl<CG, EPI_SPLIT_SUM>(prm, slots, stream);
+    case EPI_XENT_STATS: return launch_impl<CG, EPI_XENT_STATS>(prm, slots, stream);
+    case EPI_XENT_GRAD: return launch_impl<CG, EPI_XENT_GRAD>(prm, slots, stream);
   }
   return TP_ERR_UNSUPPORTED;
 }
@@ -774,6 +881,14 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.dbias_part = p.dbias_part;
   a.dev_status = p.dev_status;
   a.wait_ns = wait_limit_ns();
+  a.targets = p.targets;
+  a.stat_m = p.stat_m;
+  a.stat_s = p.stat_s;
+  a.stat_i = p.stat_i;
+  a.tgt_logit = p.tgt_logit;
+  a.row_lse = p.row_lse;
+  a.grad_scale = p.grad_scale;
+  if ((p.epi == EPI_XENT_STATS || p.epi == EPI_XENT_GRAD) && p.splits != 1) return TP_ERR_UNSUPPORTED;
   if (p.splits > 1) {
     const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
     if (p.ws == nullptr || p.ws_bytes < need) return TP_ERR_WORKSPACE;

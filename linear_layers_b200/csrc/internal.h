@@ -16,9 +16,15 @@ enum EpiKind : int {
   EPI_BIAS_ACT = 1,     // U = acc + bias; Y = act(U); out0 = U (nullable), out1 = Y
   EPI_DACT = 2,         // dU = acc ⊙ act'(aux); out0 = dU; per-tile column sums of dU
   EPI_STORE_F32 = 3,    // out0 = acc (fp32)
-  EPI_SPLIT_SUM = 4     // fp32 partial per split; the last split of a tile sums them
+  EPI_SPLIT_SUM = 4,    // fp32 partial per split; the last split of a tile sums them
                         // in split order and stores bf16 to out0
+  EPI_XENT_STATS = 5,   // softmax statistics of each 128-column slice of every row:
+                        // maximum, Σ exp(acc − maximum), first arg-max; the target
+                        // column's accumulator; no output matrix
+  EPI_XENT_GRAD = 6     // out0 = bf16(grad_scale·(exp(acc − lse_row) − [col = target]))
 };
+
+constexpr int kXentSlice = 128;   // columns per softmax-statistics slice
 
 // C[M,N] = A[M,K] · B[K,N] with the operands in one of two storages each:
 //   A: a_mn == 0  ->  A stored [M,K] row-major (lda >= K)      (K-major)
@@ -47,6 +53,14 @@ struct GemmProblem {
   void* ws = nullptr;              // partial buffer + tile counters (see gemm_ws_bytes)
   size_t ws_bytes = 0;
   int32_t* dev_status = nullptr;
+  // EPI_XENT_STATS / EPI_XENT_GRAD (row = token, column = vocabulary entry)
+  const int64_t* targets = nullptr;  // [M]
+  float* stat_m = nullptr;           // [ceil(N/128), M] slice maxima
+  float* stat_s = nullptr;           // [ceil(N/128), M] slice sums of exp(acc − max)
+  int32_t* stat_i = nullptr;         // [ceil(N/128), M] slice arg-max (column index)
+  float* tgt_logit = nullptr;        // [M] accumulator at the target column
+  const float* row_lse = nullptr;    // [M] log-sum-exp of each row (EPI_XENT_GRAD)
+  float grad_scale = 1.0f;
 };
 
 // Workspace a split GEMM needs: fp32 partial tiles (unless zpart carries

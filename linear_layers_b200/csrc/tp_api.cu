@@ -26,6 +26,11 @@ tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T,
                          cudaStream_t stream);
 
 size_t embed_bwd_ws_bytes(int64_t T);
+tp_status linear_xent_combine_launch(const float* stat_m, const float* stat_s,
+                                     const int32_t* stat_i, const float* tgt_logit,
+                                     const int64_t* targets, int64_t T, int64_t v, float* loss,
+                                     float* loss_sum, float* lse, int32_t* argmax,
+                                     int32_t* dev_status, cudaStream_t stream);
 tp_status vp_embed_bwd_launch(const int64_t* ids, const void* dout, int64_t T, int64_t v, int64_t h,
                               float* dE, void* ws, int32_t* dev_status, cudaStream_t stream);
 
@@ -173,6 +178,12 @@ size_t row_split_ws(int64_t M, int64_t Nout, int64_t K, int32_t N, bool zpart) {
 }
 
 // dbias partials: one fp32 row per 32-row tile (the finest tiling any path uses)
+// slice maxima, slice sums, slice arg-max ([ceil(v/128), T] each), target logits [T]
+size_t linear_xent_ws_bytes(int64_t T, int64_t v) {
+  const size_t plane = align256(static_cast<size_t>((v + kXentSlice - 1) / kXentSlice) * T * 4);
+  return 3 * plane + align256(static_cast<size_t>(T) * 4);
+}
+
 size_t dbias_ws(int64_t M, int64_t F) { return align256(((M + 31) / 32) * F * sizeof(float)); }
 
 // Run a row-parallel GEMM C[M,Nout] = Σ_i A[:, off_i:off_{i+1}]·B[off_i:off_{i+1}, :]
@@ -268,6 +279,8 @@ size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) 
       return 0;
     case TP_OP_EMBED_BWD:   // (T, h, v, N): sort keys of the T tokens
       return align256(embed_bwd_ws_bytes(M));
+    case TP_OP_LINEAR_XENT:   // (T, h, v, N): slice statistics + target logits
+      return linear_xent_ws_bytes(M, F);
   }
   return 0;
 }
@@ -583,6 +596,59 @@ tp_status vp_xent_bf16_grad(const float* logits, const int64_t* targets, int64_t
   if (tp_status s = require_sm100()) return s;
   return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, true, argmax,
                         dev_status, as_stream(stream));
+}
+
+tp_status tp_linear_xent_fwd(const void* H, const void* E, const int64_t* targets, int64_t T,
+                             int64_t h, int64_t v, int32_t N, float* loss, float* loss_sum,
+                             float* lse, int32_t* argmax, void* ws, size_t ws_bytes,
+                             int32_t* dev_status, void* stream) {
+  if (!H || !E || !targets || !loss) return TP_ERR_NULL;
+  if (!dims_ok({T, h, v}) || N < 1 || v % N) return TP_ERR_SHAPE;
+  if (h % 8 || !ptrs_aligned({H, E}) || (reinterpret_cast<uintptr_t>(targets) & 7)) return TP_ERR_ALIGN;
+  const size_t need = linear_xent_ws_bytes(T, v);
+  if (ws == nullptr || ws_bytes < need) return TP_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255) return TP_ERR_ALIGN;
+  if (tp_status s = require_sm100()) return s;
+  const size_t plane = align256(static_cast<size_t>((v + kXentSlice - 1) / kXentSlice) * T * 4);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  GemmProblem g;
+  g.A = H; g.lda = h; g.a_mn = 0;
+  g.B = E; g.ldb = h; g.b_mn = 0;               // E [v,h] read as Eᵀ: K-major
+  g.M = static_cast<int>(T); g.N = static_cast<int>(v); g.K = static_cast<int>(h);
+  g.epi = EPI_XENT_STATS;
+  g.targets = targets;
+  g.stat_m = reinterpret_cast<float*>(w);
+  g.stat_s = reinterpret_cast<float*>(w + plane);
+  g.stat_i = reinterpret_cast<int32_t*>(w + 2 * plane);
+  g.tgt_logit = reinterpret_cast<float*>(w + 3 * plane);
+  g.dev_status = dev_status;
+  cudaStream_t st = as_stream(stream);
+  if (tp_status s = gemm_tc_launch(g, st)) return s;
+  return linear_xent_combine_launch(g.stat_m, g.stat_s, g.stat_i, g.tgt_logit, targets, T, v, loss,
+                                    loss_sum, lse, argmax, dev_status, st);
+}
+
+tp_status tp_linear_xent_dlogits(const void* H, const void* E, const int64_t* targets,
+                                 const float* lse, int64_t T, int64_t h, int64_t v, int32_t N,
+                                 float grad_scale, void* dlogits, int32_t* dev_status,
+                                 void* stream) {
+  if (!H || !E || !targets || !lse || !dlogits) return TP_ERR_NULL;
+  if (!dims_ok({T, h, v}) || N < 1 || v % N) return TP_ERR_SHAPE;
+  if (h % 8 || v % 8 || !ptrs_aligned({H, E, dlogits}) ||
+      (reinterpret_cast<uintptr_t>(targets) & 7) || (reinterpret_cast<uintptr_t>(lse) & 3))
+    return TP_ERR_ALIGN;
+  if (tp_status s = require_sm100()) return s;
+  GemmProblem g;
+  g.A = H; g.lda = h; g.a_mn = 0;
+  g.B = E; g.ldb = h; g.b_mn = 0;
+  g.M = static_cast<int>(T); g.N = static_cast<int>(v); g.K = static_cast<int>(h);
+  g.epi = EPI_XENT_GRAD;
+  g.out0 = dlogits; g.ldo = v;
+  g.targets = targets;
+  g.row_lse = lse;
+  g.grad_scale = grad_scale;
+  g.dev_status = dev_status;
+  return gemm_tc_launch(g, as_stream(stream));
 }
 
 tp_status tp_logits_bwd(const void* dlogits, const void* H, const void* E, int64_t T, int64_t h,

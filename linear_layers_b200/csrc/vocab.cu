@@ -444,6 +444,73 @@ __global__ void __launch_bounds__(1024) loss_sum_kernel(const float* loss, int64
   if (threadIdx.x == 0) *out = part[0];
 }
 
+// Combine of the per-slice softmax statistics the logits GEMM records
+// (slice k of row t at [k·T + t]): 32 tokens per block, one per lane; warp w
+// reads slices w, w + 8, … so that each load is 32 consecutive tokens.  First
+// the maximum with its first column, then the sum of s_k·exp(m_k − m); both
+// fold the eight warps in warp order, so the result does not depend on timing.
+constexpr int kCombWarps = 8;
+
+__global__ void __launch_bounds__(kCombWarps * 32) linear_xent_combine_kernel(
+    const float* __restrict__ stat_m, const float* __restrict__ stat_s,
+    const int32_t* __restrict__ stat_i, const float* __restrict__ tgt_logit,
+    const int64_t* __restrict__ targets, int64_t T, int64_t v, int nslices, float* __restrict__ loss,
+    float* __restrict__ lse_out, int32_t* __restrict__ argmax, int32_t* dev_status) {
+  __shared__ float part_m[kCombWarps][32];
+  __shared__ int part_i[kCombWarps][32];
+  __shared__ float part_s[kCombWarps][32];
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  const bool ok = t < T;
+  float m = -INFINITY;
+  int arg = 0x7fffffff;
+  if (ok) {
+#pragma unroll 4
+    for (int k = w; k < nslices; k += kCombWarps) {
+      const float mk = __ldcs(stat_m + k * T + t);
+      if (mk > m) {   // slices in increasing column order: ties keep the first
+        m = mk;
+        arg = stat_i[k * T + t];
+      }
+    }
+  }
+  part_m[w][lane] = m;
+  part_i[w][lane] = arg;
+  __syncthreads();
+  float M = part_m[0][lane];
+  int A = part_i[0][lane];
+#pragma unroll
+  for (int q = 1; q < kCombWarps; ++q) {
+    const float mq = part_m[q][lane];
+    const int aq = part_i[q][lane];
+    if (mq > M || (mq == M && aq < A)) {
+      M = mq;
+      A = aq;
+    }
+  }
+  float S = 0.0f;
+  if (ok) {
+#pragma unroll 4
+    for (int k = w; k < nslices; k += kCombWarps)
+      S += __ldcs(stat_s + k * T + t) * expf(stat_m[k * T + t] - M);
+  }
+  part_s[w][lane] = S;
+  __syncthreads();
+  if (w == 0 && ok) {
+    float tot = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kCombWarps; ++q) tot += part_s[q][lane];
+    const float lse = M + logf(tot);
+    const int64_t y = targets[t];
+    const bool y_ok = y >= 0 && y < v;
+    if (!y_ok && dev_status) atomicOr(dev_status, TP_DEVERR_RANGE);
+    loss[t] = y_ok ? lse - tgt_logit[t] : CUDART_NAN_F;
+    if (lse_out) lse_out[t] = lse;
+    if (argmax) argmax[t] = A;
+  }
+}
+
 tp_status loss_sum_launch(const float* loss, int64_t T, float* loss_sum, cudaStream_t stream) {
   loss_sum_kernel<<<1, 1024, 0, stream>>>(loss, T, loss_sum);
   note_launches(1);
@@ -471,11 +538,18 @@ tp_status xent_cluster_launch(const float* logits, const int64_t* targets, int64
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   static size_t cap_smem[64][9] = {{0}};
-  int& c = cap[dev & 63][N];
-  if (c == 0 || cap_smem[dev & 63][N] != smem) {
+  // The shared-memory opt-in belongs to the kernel, not to (device, N): it
+  // only ever grows, so that a call with a smaller slice cannot lower the
+  // limit under a larger one whose occupancy is already cached.
+  static size_t attr_smem[64] = {0};
+  if (smem > attr_smem[dev & 63]) {
     if (cudaFuncSetAttribute(vp_xent_cluster_kernel<R, NT, GT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem)) != cudaSuccess)
       return TP_ERR_CUDA;
+    attr_smem[dev & 63] = smem;
+  }
+  int& c = cap[dev & 63][N];
+  if (c == 0 || cap_smem[dev & 63][N] != smem) {
     cap_smem[dev & 63][N] = smem;
     int clusters = 0;
     cfg.gridDim = dim3(static_cast<unsigned>(N * num_sms()));
@@ -721,6 +795,20 @@ tp_status vp_xent_launch(const float* logits, const int64_t* targets, int64_t T,
                                            dev_status, stream);
   return vp_xent_launch_t<float>(logits, targets, T, v, N, grad_scale, loss, loss_sum,
                                  static_cast<float*>(dlogits), argmax, dev_status, stream);
+}
+
+tp_status linear_xent_combine_launch(const float* stat_m, const float* stat_s,
+                                     const int32_t* stat_i, const float* tgt_logit,
+                                     const int64_t* targets, int64_t T, int64_t v, float* loss,
+                                     float* loss_sum, float* lse, int32_t* argmax,
+                                     int32_t* dev_status, cudaStream_t stream) {
+  const int nslices = static_cast<int>((v + kXentSlice - 1) / kXentSlice);
+  const unsigned blocks = static_cast<unsigned>((T + 31) / 32);
+  linear_xent_combine_kernel<<<blocks, kCombWarps * 32, 0, stream>>>(
+      stat_m, stat_s, stat_i, tgt_logit, targets, T, v, nslices, loss, lse, argmax, dev_status);
+  note_launches(1);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  return loss_sum ? loss_sum_launch(loss, T, loss_sum, stream) : TP_OK;
 }
 
 size_t embed_bwd_ws_bytes(int64_t T) {

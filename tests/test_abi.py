@@ -99,6 +99,20 @@ def test_validation_errors_before_any_launch(L):
     assert L.vp_embed(None, 4, FAKE, 300, 64, 2, 0, FAKE, None, None) == TP_ERR_NULL
     assert L.vp_xent(FAKE, FAKE, 4, 300, 7, 1.0, FAKE, None, None, None, None, None) == TP_ERR_SHAPE
     assert L.tp_logits_fwd(FAKE, FAKE, 4, 64, 302, 2, FAKE, None, None) == TP_ERR_ALIGN
+    # fused output layer + loss: workspace is checked before the device
+    wsb = tpl.tp_workspace_bytes(tpl.OP_LINEAR_XENT, 4, 64, 300, 2)
+    assert wsb >= 3 * 3 * 4 * 4 + 4 * 4                       # 3 slices x 4 tokens, 3 planes
+    lx = L.tp_linear_xent_fwd
+    assert lx(FAKE, FAKE, FAKE, 4, 64, 300, 7, FAKE, None, None, None, FAKE, wsb, None,
+              None) == TP_ERR_SHAPE
+    assert lx(FAKE, FAKE, None, 4, 64, 300, 2, FAKE, None, None, None, FAKE, wsb, None,
+              None) == TP_ERR_NULL
+    assert lx(FAKE, FAKE, FAKE, 4, 60, 300, 2, FAKE, None, None, None, FAKE, wsb, None,
+              None) == TP_ERR_ALIGN
+    assert lx(FAKE, FAKE, FAKE, 4, 64, 300, 2, FAKE, None, None, None, FAKE, wsb - 1, None,
+              None) == 7                                       # TP_ERR_WORKSPACE
+    assert L.tp_linear_xent_dlogits(FAKE, FAKE, FAKE, FAKE, 4, 64, 300, 2, 1.0, FAKE, None,
+                                    None) == TP_ERR_ALIGN     # bf16 rows need 8 | v
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
@@ -106,6 +120,11 @@ def test_valid_call_without_gpu_fails_loudly(L):
     assert _mlp_fwd(L) == TP_ERR_DEVICE
     assert L.vp_embed(FAKE, 4, FAKE, 300, 64, 2, 0, FAKE, None, None) == TP_ERR_DEVICE
     assert L.vp_xent(FAKE, FAKE, 4, 300, 2, 1.0, FAKE, None, None, None, None, None) == TP_ERR_DEVICE
+    wsb = tpl.tp_workspace_bytes(tpl.OP_LINEAR_XENT, 4, 64, 304, 2)
+    assert L.tp_linear_xent_fwd(FAKE, FAKE, FAKE, 4, 64, 304, 2, FAKE, None, None, None, FAKE,
+                                wsb, None, None) == TP_ERR_DEVICE
+    assert L.tp_linear_xent_dlogits(FAKE, FAKE, FAKE, FAKE, 4, 64, 304, 2, 1.0, FAKE, None,
+                                    None) == TP_ERR_DEVICE
     with pytest.raises(RuntimeError, match="no CPU path"):
         X = torch.zeros(16, 64, dtype=torch.bfloat16)
         tpl.tp_mlp_fwd(X, torch.zeros(64, 256, dtype=torch.bfloat16), None,

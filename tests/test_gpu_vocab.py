@@ -109,6 +109,14 @@ def test_xent_small(v, N):
     assert abs(float(r["loss_sum"].item()) - ref["loss_sum"]) <= TOL_XENT * abs(ref["loss_sum"])
 
 
+def test_xent_alternating_slice_sizes():
+    """Calls with a smaller shard slice between two with a larger one (the
+    same kernel instance): every launch keeps enough shared memory."""
+    for v, N in [(8192, 8), (1024, 4), (8192, 8), (1024, 4)]:
+        inp = tp_inputs.xent_logits(64, v, seed=v + N)
+        _xent_check(inp["logits"], inp["targets"], N, 1.0)
+
+
 def test_xent_ties_uniform_and_bad_targets():
     v, N = 64, 4
     L = torch.zeros(5, v)
