@@ -25,6 +25,12 @@ and section:
   "输出层Embedding", §5 "Cross-Entropy层".
 * [APX] "Megatron-LM 介绍" (apxml.com), §"核心贡献": column-parallel
   Y_i = X A_i and the Linear(1024→4096), TP=2 shape example.
+* [FW] "Megatron-LM框架概览" page (5688vip.com, chapter 03), §3.2
+  "核心特性": activation recompute drops activations and rebuilds them in
+  the backward.
+* [EVO] Megatron history page (discosf.com/news/5875844), §2.3
+  "序列并行与激活重计算": recompute keeps only each layer's inputs, or
+  selectively the costliest part of the MLP or attention.
 
 Readings where the pages are silent or garbled (each also listed with the
 design notes):
@@ -161,6 +167,30 @@ def mlp_bwd(X, A, bias, B, dZ, act=ACT_GELU_TANH):
     dY = dZ @ B.T
     dU = dY * act_grad(U, act)
     return {
+        "dY": dY,
+        "dU": dU,
+        "dB": Y.T @ dZ,
+        "dA": X.T @ dU,
+        "dbias": dU.sum(axis=0),
+        "dX": dU @ A.T,
+    }
+
+
+def mlp_bwd_recompute(X, A, B, U, dZ, act=ACT_GELU_TANH):
+    """The same gradient when the forward kept only the pre-activation U.
+
+    Activation recompute ([FW] §3.2, the recompute row of its feature table;
+    [EVO] §2.3): the activation Y is dropped after the forward and rebuilt
+    from the saved U when the backward needs it, Y = act(U); everything else
+    is mlp_bwd.  ``U`` is taken as given (the saved tensor), so the result is
+    the gradient at that U.
+    """
+    X, A, B, U, dZ = f64(X), f64(A), f64(B), f64(U), f64(dZ)
+    Y = act_fwd(U, act)                      # recomputed, not stored
+    dY = dZ @ B.T
+    dU = dY * act_grad(U, act)
+    return {
+        "Y": Y,
         "dY": dY,
         "dU": dU,
         "dB": Y.T @ dZ,

@@ -141,6 +141,30 @@ def check_mlp_fd_gradients(o):
             assert _rel(g[name], fd) < 1e-7, (act, name, _rel(g[name], fd))
 
 
+def check_mlp_recompute(o):
+    """Backward from the saved pre-activation alone: with U = X·A + bias it is
+    the full backward; with a perturbed U it is the gradient at that U (torch
+    autograd through Y = gelu(U) in float64 on the recomputed path)."""
+    import torch
+
+    X, A, b, B, dZ = _tiny_mlp(5, M=3, h=4, F=8)
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF, o.ACT_NONE):
+        full = o.mlp_bwd(X, A, b, B, dZ, act)
+        U = X @ A + b[None, :]
+        rc = o.mlp_bwd_recompute(X, A, B, U, dZ, act)
+        for k in ("dX", "dA", "dbias", "dB", "dU"):
+            assert _rel(rc[k], full[k]) < 1e-15, (act, k)
+    U2 = X @ A + b[None, :] + 0.3                       # any saved tensor
+    Ut = torch.from_numpy(U2).requires_grad_(True)
+    Bt = torch.from_numpy(B).requires_grad_(True)
+    Yt = torch.nn.functional.gelu(Ut, approximate="tanh")
+    ((Yt @ Bt) * torch.from_numpy(dZ)).sum().backward()
+    rc = o.mlp_bwd_recompute(X, A, B, U2, dZ, o.ACT_GELU_TANH)
+    assert _rel(rc["Y"], Yt.detach().numpy()) < 1e-15
+    assert _rel(rc["dB"], Bt.grad.numpy()) < 1e-14
+    assert _rel(rc["dU"], Ut.grad.numpy()) < 1e-14
+
+
 def check_mlp_sharded_equals_unsharded(o):
     """Column split of A and row split of B with one all-reduce reproduce the
     unsharded layer exactly up to rounding (N = 1, 2, 4, 8 and uneven shards)."""

@@ -201,6 +201,18 @@ def _m_partitioned_tie_to_later_part(mp):
     mp.setattr(O, "xent_sharded", bad)
 
 
+def _m_recompute_uses_derivative(mp):
+    orig = O.mlp_bwd_recompute
+
+    def bad(X, A, B, U, dZ, act=O.ACT_GELU_TANH):
+        r = orig(X, A, B, U, dZ, act)
+        Y = O.act_grad(O.f64(U), act)                     # derivative in place of the value
+        r["Y"] = Y
+        r["dB"] = Y.T @ O.f64(dZ)
+        return r
+    mp.setattr(O, "mlp_bwd_recompute", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
