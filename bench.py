@@ -292,6 +292,12 @@ def _embed_bwd(tpl, vo, st):
     tpl.vp_embed_bwd(vo["ids"], vo["dout"], vo["dE"], VOC["N"], ws=vo["ws_eb"], dev_status=st)
 
 
+def _mlp_bwd_rc(tpl, g, st):
+    tpl.tp_mlp_bwd_recompute(g["X"], g["A"], g["B"], g["U"], g["dZ"], MLP["N"], Y=g["Y"],
+                             dU=g["dU"], dX=g["dX"], dA=g["dA"], dbias=g["dbias"], dB=g["dB"],
+                             ws=g["ws_b"], dev_status=st)
+
+
 def _lxent_fwd(tpl, vo, st):
     tpl.tp_linear_xent_fwd(vo["H"], vo["E"], vo["targets"], VOC["N"], loss=vo["loss"],
                            loss_sum=vo["loss_sum"], lse=vo["lse"], argmax=vo["argmax"],
@@ -313,6 +319,8 @@ BWD_PARTS = ("logits", "xent_bf16", "logits_bwd", "embed_bwd")
 # also in its own loop: statistics GEMM + combine, then the recomputing
 # gradient GEMM
 FUSED_PARTS = ("lxent_fwd", "lxent_dlogits")
+# the MLP backward with activation recompute (Y rebuilt from U), own loop
+RECOMPUTE_PARTS = ("mlp_bwd_rc",)
 
 
 def _e2e_mlp(tpl, torch, g, dev, steps):
@@ -426,7 +434,7 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS
+    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS
     parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
         raise SystemExit(f"--parts must name some of {','.join(known)}")
@@ -446,7 +454,8 @@ def run_gpu(args):
            "logits_bwd": lambda: _logits_bwd(tpl, vo, st),
            "embed_bwd": lambda: _embed_bwd(tpl, vo, st),
            "lxent_fwd": lambda: _lxent_fwd(tpl, vo, st),
-           "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st)}
+           "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st),
+           "mlp_bwd_rc": lambda: _mlp_bwd_rc(tpl, g, st)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -503,6 +512,7 @@ def run_gpu(args):
     side_steps = max(5, min(args.steps, 20))
     bwd_ms = _side_loop(torch, fns, BWD_PARTS, side_steps, stream, dev, st, world)
     fused_ms = _side_loop(torch, fns, FUSED_PARTS, side_steps, stream, dev, st, world)
+    rc_ms = _side_loop(torch, fns, RECOMPUTE_PARTS, side_steps, stream, dev, st, world)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
@@ -577,6 +587,14 @@ def run_gpu(args):
                 "dlogits_ms": round(fused_ms["lxent_dlogits"], 4),
                 "dlogits_tflops": round(LOGITS_FLOP / (fused_ms["lxent_dlogits"] / 1e3) / 1e12, 1),
                 "logits_bytes_not_stored": VOC["T"] * VOC["v"] * 4,
+            },
+            "mlp_bwd_recompute": {
+                "what": "TP-MLP backward from the saved pre-activation U alone (Y = GeLU(U) rebuilt "
+                        "in the dGeLU GEMM's epilogue); own loop of %d iterations" % side_steps,
+                "ms": round(rc_ms["mlp_bwd_rc"], 4),
+                "tflops": round(4.0 * MLP["M"] * MLP["h"] * MLP["F"] * 2 / (rc_ms["mlp_bwd_rc"] / 1e3) / 1e12, 1),
+                "saved_activation_ms": round(part_ms["mlp_bwd"] / K, 4),
+                "activation_bytes_not_kept": MLP["M"] * MLP["F"] * 2,
             },
             "parts_ms_per_step": {p: round(part_ms[p] / K, 4) for p in PARTS},
             "roofline": {

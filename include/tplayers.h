@@ -175,6 +175,29 @@ TP_API tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const v
                      void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
+ * TP-MLP backward with activation recompute   [FW] "Megatron-LM框架概览"
+ * §3.2 (the recompute row of the feature table: activations are dropped
+ * after the forward and rebuilt in the backward); [EVO] Megatron history page
+ * §2.3 "序列并行与激活重计算" (selective recompute of the MLP's costliest part).
+ *
+ *   Exactly tp_mlp_bwd, except that the forward's activation Y is not an
+ *   input: only the pre-activation U [M,F] was kept.  The dGeLU GEMM, which
+ *   reads U for act'(U) anyway, also writes Y = act(U) into Y [M,F] (an
+ *   output here, bf16 or fp32 like U), and the dB GEMM reads it from there.
+ *   Y may be a scratch buffer shared between layers, or U itself: every
+ *   element of U is read by the thread that then overwrites it, so Y == U
+ *   recomputes in place (U is then lost).  Same workspace as
+ *   TP_OP_MLP_BWD; same errors.
+ */
+TP_API tp_status tp_mlp_bwd_recompute(const void* X, const void* A, const void* B, const void* U,
+                                      void* Y, const void* dZ,
+                                      int64_t M, int64_t h, int64_t F, int32_t N,
+                                      const int64_t* shard_offsets, tp_dtype dt, tp_act act,
+                                      void* dU, void* dX, void* dA, float* dbias, void* dB,
+                                      void* ws, size_t ws_bytes, int32_t* dev_status,
+                                      void* stream);
+
+/*
  * Column-parallel linear, forward   [TP-ILL] §1.2; [APX] §核心贡献; the QKV
  * projection of [MLP-TP] §2.2 / [TP-ILL] §3.1 with per-shard heads.
  *

@@ -28,7 +28,7 @@ __all__ = [
     "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
     "vp_embed", "tp_logits_fwd", "vp_xent", "vp_xent_bf16_grad", "tp_logits_bwd", "vp_embed_bwd",
     "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
-    "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT",
+    "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT", "tp_mlp_bwd_recompute",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
@@ -75,6 +75,8 @@ _SIGS = {
     "tp_linear_xent_fwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _SZ,
                             _P, _P], _I32),
     "tp_linear_xent_dlogits": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _F, _P, _P, _P], _I32),
+    "tp_mlp_bwd_recompute": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
+                              _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
 }
 
 
@@ -217,6 +219,33 @@ def tp_mlp_bwd(X, A, B, U, Y, dZ, N, *, shard_offsets=None, act=ACT_GELU_TANH, w
                             offs, _dt(X), act, _ptr(dU), _ptr(dX), _ptr(dA), _ptr(dbias), _ptr(dB),
                             _ptr(ws), wsb, _ptr(dev_status), _stream(dev)), "tp_mlp_bwd")
     return {"dX": dX, "dA": dA, "dbias": dbias, "dB": dB, "dU": dU}
+
+
+def tp_mlp_bwd_recompute(X, A, B, U, dZ, N, *, Y=None, shard_offsets=None, act=ACT_GELU_TANH,
+                         with_dbias=True, dU=None, dX=None, dA=None, dbias=None, dB=None, ws=None,
+                         dev_status=None):
+    """Backward from the saved pre-activation U alone: Y = act(U) is rebuilt
+    into ``Y`` (scratch, or U itself for in place).  Returns dict(dX, dA,
+    dbias, dB, dU, Y)."""
+    M, h = X.shape
+    F = A.shape[1]
+    dev = X.device
+    dt = X.dtype
+    Y = torch.empty(M, F, dtype=dt, device=dev) if Y is None else Y
+    dU = torch.empty(M, F, dtype=dt, device=dev) if dU is None else dU
+    dX = torch.empty(M, h, dtype=dt, device=dev) if dX is None else dX
+    dA = torch.empty(h, F, dtype=dt, device=dev) if dA is None else dA
+    dB = torch.empty(F, h, dtype=dt, device=dev) if dB is None else dB
+    if dbias is None and with_dbias:
+        dbias = torch.empty(F, dtype=torch.float32, device=dev)
+    _contig(X, A, B, U, Y, dZ, dU, dX, dA, dB, dbias)
+    ws, wsb = _workspace(ws, OP_MLP_BWD, M, h, F, N, dev)
+    offs, keep = _offsets(shard_offsets, N)
+    _check(lib().tp_mlp_bwd_recompute(_ptr(X), _ptr(A), _ptr(B), _ptr(U), _ptr(Y), _ptr(dZ), M, h,
+                                      F, N, offs, _dt(X), act, _ptr(dU), _ptr(dX), _ptr(dA),
+                                      _ptr(dbias), _ptr(dB), _ptr(ws), wsb, _ptr(dev_status),
+                                      _stream(dev)), "tp_mlp_bwd_recompute")
+    return {"dX": dX, "dA": dA, "dbias": dbias, "dB": dB, "dU": dU, "Y": Y}
 
 
 def tp_col_linear_fwd(X, W, bias, N, *, shard_offsets=None, act=ACT_NONE, U=None, Y=None,

@@ -99,9 +99,11 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(SimtArgs a) {
       if (a.out0) a.out0[o] = v;
       a.out1[o] = act_apply32(v, a.act);
     } else if (a.epi == EPI_DACT) {
-      v *= act_deriv32(a.aux[static_cast<int64_t>(row) * a.ld_aux + col], a.act);
+      const float u = a.aux[static_cast<int64_t>(row) * a.ld_aux + col];
+      v *= act_deriv32(u, a.act);
       a.out0[o] = v;
       colsum += v;
+      if (a.out1) a.out1[o] = act_apply32(u, a.act);   // activation recompute
     } else {
       a.out0[o] = v;
     }

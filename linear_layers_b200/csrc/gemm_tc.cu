@@ -687,6 +687,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               const float colsum = warp_column_sums(v, lane);
               red[q * BN + c * 32 + lane] = colsum;
             }
+            if (a.out1 != nullptr && store_ok) {   // activation recompute: Y = act(U)
+#pragma unroll
+              for (int j = 0; j < 32; ++j) v[j] = act_apply(aux_v[j], a.act);
+              store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
+                            a.N - col0);
+            }
           }
         }
         if constexpr (EPI == EPI_DACT) {

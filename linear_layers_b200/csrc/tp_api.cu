@@ -323,11 +323,19 @@ tp_status tp_mlp_fwd(const void* X, const void* A, const void* bias, const void*
   return run_row_parallel(g2, offs, Zpart, ws, ws_bytes, bf16, st);
 }
 
-tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const void* U, const void* Y,
-                     const void* dZ, int64_t M, int64_t h, int64_t F, int32_t N,
-                     const int64_t* shard_offsets_, tp_dtype dt, tp_act act, void* dU, void* dX,
-                     void* dA, float* dbias, void* dB, void* ws, size_t ws_bytes,
-                     int32_t* dev_status, void* stream) {
+}  // extern "C"
+
+namespace tpl {
+namespace {
+
+// The MLP backward; with recompute the dGeLU GEMM's epilogue also writes
+// Y = act(U) into Y (which the dB GEMM then reads), otherwise Y is the saved
+// activation.
+tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* U, void* Y,
+                       bool recompute, const void* dZ, int64_t M, int64_t h, int64_t F, int32_t N,
+                       const int64_t* shard_offsets_, tp_dtype dt, tp_act act, void* dU, void* dX,
+                       void* dA, float* dbias, void* dB, void* ws, size_t ws_bytes,
+                       int32_t* dev_status, void* stream) {
   if (!X || !A || !B || !U || !Y || !dZ || !dU || !dX || !dA || !dB) return TP_ERR_NULL;
   if (dt != TP_DTYPE_BF16 && dt != TP_DTYPE_F32) return TP_ERR_DTYPE;
   if (act < TP_ACT_NONE || act > TP_ACT_GELU_ERF) return TP_ERR_DTYPE;
@@ -357,6 +365,7 @@ tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const void* U,
   g3.M = static_cast<int>(M); g3.N = static_cast<int>(F); g3.K = static_cast<int>(h);
   g3.epi = EPI_DACT; g3.act = act; g3.aux = U; g3.ld_aux = F;
   g3.out0 = dU; g3.ldo = F; g3.dbias_part = dbias_part;
+  if (recompute) g3.out1 = Y;
   g3.dev_status = dev_status;
   tp_status s = bf16 ? gemm_tc_launch(g3, st) : gemm_simt_launch(g3, st);
   if (s) return s;
@@ -395,6 +404,34 @@ tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const void* U,
                                         dbias, st);
   return TP_OK;
 }
+
+}  // namespace
+}  // namespace tpl
+
+extern "C" {
+
+tp_status tp_mlp_bwd(const void* X, const void* A, const void* B, const void* U, const void* Y,
+                     const void* dZ, int64_t M, int64_t h, int64_t F, int32_t N,
+                     const int64_t* shard_offsets_, tp_dtype dt, tp_act act, void* dU, void* dX,
+                     void* dA, float* dbias, void* dB, void* ws, size_t ws_bytes,
+                     int32_t* dev_status, void* stream) {
+  return tpl::mlp_bwd_impl(X, A, B, U, const_cast<void*>(Y), false, dZ, M, h, F, N,
+                           shard_offsets_, dt, act, dU, dX, dA, dbias, dB, ws, ws_bytes,
+                           dev_status, stream);
+}
+
+tp_status tp_mlp_bwd_recompute(const void* X, const void* A, const void* B, const void* U,
+                               void* Y, const void* dZ, int64_t M, int64_t h, int64_t F,
+                               int32_t N, const int64_t* shard_offsets_, tp_dtype dt, tp_act act,
+                               void* dU, void* dX, void* dA, float* dbias, void* dB, void* ws,
+                               size_t ws_bytes, int32_t* dev_status, void* stream) {
+  return tpl::mlp_bwd_impl(X, A, B, U, Y, true, dZ, M, h, F, N, shard_offsets_, dt, act, dU, dX,
+                           dA, dbias, dB, ws, ws_bytes, dev_status, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
 
 tp_status tp_col_linear_fwd(const void* X, const void* W, const void* bias, int64_t M, int64_t K,
                             int64_t Nout, int32_t N, const int64_t* shard_offsets_, tp_dtype dt,

@@ -1,0 +1,102 @@
+"""TP-MLP backward with activation recompute on the GPU against the fp64
+oracle (through the C ABI).
+
+The forward keeps U only; tp_mlp_bwd_recompute rebuilds Y = GeLU(U) in the
+dGeLU GEMM's epilogue.  Gradients are compared with the oracle's full
+backward from the same inputs (TOL_BF16, TOL_F32 for the fp32 path).  Every
+output that does not depend on Y (dX, dA, dU, dbias) must be bit-identical to
+the saved-activation backward: the same GEMMs run on the same operands.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_layers_b200 as tpl
+import tp_inputs
+from oracle import tp_oracle as O
+from tests.gpu_helpers import TOL_BF16, TOL_F32, assert_close, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+def _fwd(d, N, act, offsets=None):
+    st = tpl.new_status()
+    Z, U, Y = tpl.tp_mlp_fwd(d["X"], d["A"], d["bias"], d["B"], N, shard_offsets=offsets,
+                             act=act, dev_status=st)
+    return Z, U, Y, st
+
+
+@pytest.mark.parametrize("act", [tpl.ACT_GELU_TANH, tpl.ACT_GELU_ERF, tpl.ACT_NONE])
+def test_recompute_ragged_tiles(act):
+    # M=200 (a ragged 128-row tile), h=264 (ragged k-block), F=1024 over N=4
+    inp = tp_inputs.mlp_inputs(200, 264, 1024, w_std=0.05, bias_std=0.02, seed=1)
+    d = to_dev(inp)
+    _, U, Y_saved, st = _fwd(d, 4, act)
+    g = tpl.tp_mlp_bwd_recompute(d["X"], d["A"], d["B"], U, d["dZ"], 4, act=act, dev_status=st)
+    ref = tpl.tp_mlp_bwd(d["X"], d["A"], d["B"], U, Y_saved, d["dZ"], 4, act=act, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ob = O.mlp_bwd(inp["X"], inp["A"], inp["bias"], inp["B"], inp["dZ"], act)
+    oU, oY, _ = O.mlp_fwd(inp["X"], inp["A"], inp["bias"], inp["B"], act)
+    assert_close("recomputed Y", g["Y"], oY, TOL_BF16)
+    for k in ("dX", "dA", "dB", "dbias", "dU"):
+        assert_close(k, g[k], ob[k], TOL_BF16)
+    for k in ("dX", "dA", "dbias", "dU"):
+        assert torch.equal(g[k], ref[k]), k
+
+
+def test_recompute_in_place_and_uneven_shards():
+    """Y written over U gives the same gradients as a separate scratch."""
+    inp = tp_inputs.mlp_inputs(130, 128, 768, w_std=0.05, bias_std=0.02, seed=2)
+    d = to_dev(inp)
+    offs = [0, 128, 448, 768]
+    _, U, _, st = _fwd(d, 3, tpl.ACT_GELU_TANH, offs)
+    a = tpl.tp_mlp_bwd_recompute(d["X"], d["A"], d["B"], U, d["dZ"], 3, shard_offsets=offs,
+                                 dev_status=st)
+    U2 = U.clone()
+    b = tpl.tp_mlp_bwd_recompute(d["X"], d["A"], d["B"], U2, d["dZ"], 3, shard_offsets=offs,
+                                 Y=U2, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for k in ("dX", "dA", "dB", "dbias", "dU"):
+        assert torch.equal(a[k], b[k]), k
+    assert torch.equal(U2, a["Y"])            # U2 now holds the recomputed activation
+    ob = O.mlp_bwd(inp["X"], inp["A"], inp["bias"], inp["B"], inp["dZ"])
+    for k in ("dX", "dA", "dB", "dbias"):
+        assert_close(k, a[k], ob[k], TOL_BF16)
+
+
+def test_recompute_fp32_path():
+    w = tp_inputs.WORKLOADS["mlp_tiny_fp32"]
+    inp = tp_inputs.mlp_inputs(w["M"], w["h"], w["F"], dtype=torch.float32, w_std=0.5,
+                               bias_std=0.1, seed=5)
+    d = to_dev(inp)
+    _, U, _, st = _fwd(d, w["N"], tpl.ACT_GELU_TANH)
+    g = tpl.tp_mlp_bwd_recompute(d["X"], d["A"], d["B"], U, d["dZ"], w["N"], dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ob = O.mlp_bwd(inp["X"], inp["A"], inp["bias"], inp["B"], inp["dZ"])
+    for k in ("dX", "dA", "dB", "dbias", "dU"):
+        assert_close(k, g[k], ob[k], TOL_F32)
+
+
+@pytest.mark.slow
+def test_recompute_h4096_sampled_columns():
+    """M=4096, h=4096, ffn=16384 over 8 shards: dB on 96 sampled ffn columns
+    against the oracle; the Y-independent gradients bit-identical to the
+    saved-activation backward."""
+    w = tp_inputs.WORKLOADS["mlp_h4096"]
+    inp = tp_inputs.mlp_inputs(w["M"], w["h"], w["F"], w_std=w["w_std"], seed=0)
+    d = to_dev(inp)
+    _, U, Y_saved, st = _fwd(d, w["N"], tpl.ACT_GELU_TANH)
+    ref = tpl.tp_mlp_bwd(d["X"], d["A"], d["B"], U, Y_saved, d["dZ"], w["N"], dev_status=st)
+    del Y_saved
+    g = tpl.tp_mlp_bwd_recompute(d["X"], d["A"], d["B"], U, d["dZ"], w["N"], Y=U, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for k in ("dX", "dA", "dbias", "dU"):
+        assert torch.equal(g[k], ref[k]), k
+    cols = np.sort(np.random.default_rng(3).choice(w["F"], 96, replace=False))
+    c = torch.as_tensor(cols)
+    ob = O.mlp_bwd(inp["X"], inp["A"][:, c], inp["bias"][c], inp["B"][c], inp["dZ"])
+    assert_close("dB[cols]", g["dB"][c.cuda()], ob["dB"], TOL_BF16)
