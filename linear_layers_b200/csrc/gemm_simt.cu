@@ -98,17 +98,17 @@ __global__ void __launch_bounds__(256) gemm_simt_kernel(SimtArgs a) {
       if (a.bias) v += a.bias[col];
       if (a.out0) a.out0[o] = v;
       a.out1[o] = act_apply32(v, a.act);
-    } else if (a.epi == EPI_DACT) {
+    } else if (a.epi == EPI_DACT || a.epi == EPI_DACT_Y) {
       const float u = a.aux[static_cast<int64_t>(row) * a.ld_aux + col];
       v *= act_deriv32(u, a.act);
       a.out0[o] = v;
       colsum += v;
-      if (a.out1) a.out1[o] = act_apply32(u, a.act);   // activation recompute
+      if (a.epi == EPI_DACT_Y) a.out1[o] = act_apply32(u, a.act);   // activation recompute
     } else {
       a.out0[o] = v;
     }
   }
-  if (a.epi == EPI_DACT && a.dbias_part) {
+  if ((a.epi == EPI_DACT || a.epi == EPI_DACT_Y) && a.dbias_part) {
     sred[ty][tx] = colsum;
     __syncthreads();
     if (ty == 0 && col < a.N) {

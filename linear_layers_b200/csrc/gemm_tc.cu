@@ -133,10 +133,33 @@ __device__ __forceinline__ float act_deriv(float u, int act) {
     const float half_dz = fmaf(1.5f * c * a, u2, 0.5f * c);   // 0.5·c·(1 + 3a·u²)
     return fmaf(u * half_dz, fmaf(-t, t, 1.0f), fmaf(0.5f, t, 0.5f));
   }
-  if (act == TP_ACT_GELU_ERF) {
-    const float cdf = 0.5f * (1.0f + erff(u * 0.7071067811865476f));
-    return cdf + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  if (act == TP_ACT_GELU_ERF) {   // explicit fmaf: the same bits as act_deriv_value
+    const float cdf = fmaf(0.5f, erff(u * 0.7071067811865476f), 0.5f);
+    return fmaf(u * 0.3989422804014327f, __expf(-0.5f * u * u), cdf);
   }
+  return 1.0f;
+}
+
+// act'(u) and act(u) together.  For the tanh form the value 0.5·u·(1 + t)
+// reuses the derivative's t; where 1 + t cancels (u < 0) its absolute
+// error stays below 2.5e-4·|u|, the size of a bf16 rounding step of values
+// near 0.1.
+__device__ __forceinline__ float act_deriv_value(float u, int act, float& y) {
+  if (act == TP_ACT_GELU_TANH) {
+    constexpr float c = 0.7978845608028654f, a = 0.044715f;
+    const float u2 = u * u;
+    const float t = tanh_approx(u * fmaf(c * a, u2, c));
+    const float half_dz = fmaf(1.5f * c * a, u2, 0.5f * c);
+    const float hu = 0.5f * u;
+    y = fmaf(hu, t, hu);
+    return fmaf(u * half_dz, fmaf(-t, t, 1.0f), fmaf(0.5f, t, 0.5f));
+  }
+  if (act == TP_ACT_GELU_ERF) {
+    const float cdf = fmaf(0.5f, erff(u * 0.7071067811865476f), 0.5f);
+    y = u * cdf;
+    return fmaf(u * 0.3989422804014327f, __expf(-0.5f * u * u), cdf);
+  }
+  y = u;
   return 1.0f;
 }
 
@@ -188,16 +211,17 @@ __device__ __forceinline__ void load_raw_bf16x32(const __nv_bfloat16* src, uint4
   }
 }
 
+// bf16 -> fp32 is exact as a 16-bit shift of the bit pattern: two integer
+// ops per pair, which keeps the conversions off the transcendental unit the
+// epilogues' exp / tanh already load.
 __device__ __forceinline__ void unpack_bf16x32(const uint4 (&w)[4], float* v) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
     const uint32_t ww[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&ww[q]);
-      float2 f = __bfloat1622float2(b);
-      v[8 * j + 2 * q] = f.x;
-      v[8 * j + 2 * q + 1] = f.y;
+      v[8 * j + 2 * q] = __uint_as_float(ww[q] << 16);
+      v[8 * j + 2 * q + 1] = __uint_as_float(ww[q] & 0xffff0000u);
     }
   }
 }
@@ -616,7 +640,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
       } else {
         uint4 aux_w[4];
-        if constexpr (EPI == EPI_DACT) {   // U for the first chunk
+        constexpr bool kDact = EPI == EPI_DACT || EPI == EPI_DACT_Y;
+        if constexpr (kDact) {   // U for the first chunk
           const int col0 = tn * BN + c0 * 32;
           if (row_ok && col0 < a.N) {
             load_raw_bf16x32(a.aux + row * a.ld_aux + col0, aux_w, a.N - col0);
@@ -632,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           float aux_v[32];
-          if constexpr (EPI == EPI_DACT) {
+          if constexpr (kDact) {
             unpack_bf16x32(aux_w, aux_v);
             const int coln = col0 + 32;   // prefetch U of the next chunk while this one runs
             if (c + 1 < c0 + 4 && row_ok && coln < a.N) {
@@ -677,25 +702,36 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (store_ok)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
                             a.N - col0);
-          } else {  // EPI_DACT
+          } else {  // EPI_DACT, EPI_DACT_Y
+            if constexpr (EPI == EPI_DACT_Y) {
+              // U is dead after its derivative: its registers take Y = act(U)
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = store_ok ? v[j] * act_deriv(aux_v[j], a.act) : 0.0f;
+              for (int j = 0; j < 32; ++j) {
+                float y;
+                const float d = act_deriv_value(aux_v[j], a.act, y);
+                v[j] = store_ok ? v[j] * d : 0.0f;
+                aux_v[j] = y;
+              }
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                v[j] = store_ok ? v[j] * act_deriv(aux_v[j], a.act) : 0.0f;
+            }
             if (store_ok)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
                             a.N - col0);
+            if constexpr (EPI == EPI_DACT_Y) {
+              if (store_ok)
+                store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, aux_v,
+                              a.N - col0);
+            }
             if (a.dbias_part != nullptr) {
               const float colsum = warp_column_sums(v, lane);
               red[q * BN + c * 32 + lane] = colsum;
             }
-            if (a.out1 != nullptr && store_ok) {   // activation recompute: Y = act(U)
-#pragma unroll
-              for (int j = 0; j < 32; ++j) v[j] = act_apply(aux_v[j], a.act);
-              store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
-                            a.N - col0);
-            }
           }
         }
-        if constexpr (EPI == EPI_DACT) {
+        if constexpr (kDact) {
           if (a.dbias_part != nullptr) {
             named_barrier_sync(1, kEpiThreads);
             const int cc = et;   // one column per epilogue thread (256 columns)
@@ -810,6 +846,7 @@ tp_status launch_epi(const GemmParams& prm, int epi, int slots, cudaStream_t str
     case EPI_STORE_BF16: return launch_impl<CG, EPI_STORE_BF16>(prm, slots, stream);
     case EPI_BIAS_ACT: return launch_impl<CG, EPI_BIAS_ACT>(prm, slots, stream);
     case EPI_DACT: return launch_impl<CG, EPI_DACT>(prm, slots, stream);
+    case EPI_DACT_Y: return launch_impl<CG, EPI_DACT_Y>(prm, slots, stream);
     case EPI_STORE_F32: return launch_impl<CG, EPI_STORE_F32>(prm, slots, stream);
     case EPI_SPLIT_SUM: return launch_impl<CG, EPI_SPLIT_SUM>(prm, slots, stream);
     case EPI_XENT_STATS: return launch_impl<CG, EPI_XENT_STATS>(prm, slots, stream);

@@ -14,15 +14,16 @@ constexpr int kMaxSplits = 16;   // K splits of one row-parallel GEMM (and shard
 enum EpiKind : int {
   EPI_STORE_BF16 = 0,   // out0 = bf16(acc)
   EPI_BIAS_ACT = 1,     // U = acc + bias; Y = act(U); out0 = U (nullable), out1 = Y
-  EPI_DACT = 2,         // dU = acc ⊙ act'(aux); out0 = dU; per-tile column sums of dU;
-                        // out1 (nullable) = act(aux), the recomputed activation
+  EPI_DACT = 2,         // dU = acc ⊙ act'(aux); out0 = dU; per-tile column sums of dU
   EPI_STORE_F32 = 3,    // out0 = acc (fp32)
   EPI_SPLIT_SUM = 4,    // fp32 partial per split; the last split of a tile sums them
                         // in split order and stores bf16 to out0
   EPI_XENT_STATS = 5,   // softmax statistics of each 128-column slice of every row:
                         // maximum, Σ exp(acc − maximum), first arg-max; the target
                         // column's accumulator; no output matrix
-  EPI_XENT_GRAD = 6     // out0 = bf16(grad_scale·(exp(acc − lse_row) − [col = target]))
+  EPI_XENT_GRAD = 6,    // out0 = bf16(grad_scale·(exp(acc − lse_row) − [col = target]))
+  EPI_DACT_Y = 7        // EPI_DACT, and out1 = act(aux): the activation rebuilt from the
+                        // saved pre-activation (recompute), from the same tanh as act'
 };
 
 constexpr int kXentSlice = 128;   // columns per softmax-statistics slice

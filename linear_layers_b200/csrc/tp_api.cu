@@ -363,7 +363,7 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   g3.A = dZ; g3.lda = h; g3.a_mn = 0;
   g3.B = B; g3.ldb = h; g3.b_mn = 0;            // B [F,h] read as Bᵀ: K-major
   g3.M = static_cast<int>(M); g3.N = static_cast<int>(F); g3.K = static_cast<int>(h);
-  g3.epi = EPI_DACT; g3.act = act; g3.aux = U; g3.ld_aux = F;
+  g3.epi = recompute ? EPI_DACT_Y : EPI_DACT; g3.act = act; g3.aux = U; g3.ld_aux = F;
   g3.out0 = dU; g3.ldo = F; g3.dbias_part = dbias_part;
   if (recompute) g3.out1 = Y;
   g3.dev_status = dev_status;
