@@ -47,6 +47,9 @@ design notes):
   (mathematically equal, numerically safe).  The loss is returned per token
   and as the sum over tokens ("按行加总得到 scalar Loss").
 * Ties in the arg-max go to the lowest vocabulary index.
+* The attention core's formula is an image lost from the pages; the plain
+  reading is scaled dot-product attention softmax(Q·Kᵀ/√d)·V per head, with
+  the causal mask of a decoder (the GPT-2 layer) selectable, and no dropout.
 
 Pins (tests that hold this oracle to something other than itself) live in
 ``tests/test_oracle_pins.py`` and ``tests/test_oracle_mutations.py``.
@@ -322,6 +325,62 @@ def qkv_shard_columns(n_heads: int, head_dim: int, heads_per_shard):
     if head0 != n_heads:
         raise ValueError("heads_per_shard does not cover all heads")
     return np.asarray(perm, dtype=np.int64), offsets
+
+
+# ----------------------------------------------------------------------------
+# Attention core between the projections ([MLP-TP] §2.2; [TP-ILL] §3.1)
+# ----------------------------------------------------------------------------
+def attention_head(Q, K, V, causal=True, scale=None):
+    """One head of scaled dot-product attention over one sequence.
+
+    O = softmax(Q·Kᵀ·scale + mask)·V with Q, K, V [s, d], scale = 1/√d by
+    default and, when causal, position j masked out of row i for j > i (the
+    decoder form of the GPT-2 layer).  Each row's softmax subtracts its
+    maximum first.  Returns (O [s, d], lse [s]) with lse the natural-log
+    sum of exp of the scaled, masked scores.
+    """
+    Q, K, V = f64(Q), f64(K), f64(V)
+    s, d = Q.shape
+    sc = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    S = (Q @ K.T) * sc
+    if causal:
+        S = np.where(np.tril(np.ones((s, K.shape[0]), dtype=bool)), S, -np.inf)
+    m = S.max(axis=1)
+    P = np.exp(S - m[:, None])
+    l = P.sum(axis=1)
+    return (P / l[:, None]) @ V, m + np.log(l)
+
+
+def attention_sharded(QKV, b, s, n_heads, head_dim, heads_per_shard, causal=True, scale=None):
+    """The attention core of the tensor-parallel layer, shard by shard.
+
+    QKV [b·s, 3h] is the column-parallel projection's output in the
+    shard-major layout (shard i: its Q heads, then its K heads, then its V
+    heads; see qkv_shard_columns).  Each shard runs attention on its own heads
+    with no communication; the context [b·s, h] keeps the heads in order,
+    so shard i's block of columns is the input of its rows of the
+    row-parallel output projection.  Returns (ctx, lse [b, n_heads, s]).
+    """
+    X = f64(QKV)
+    hd = head_dim
+    ctx = np.zeros((b * s, n_heads * hd))
+    lse = np.zeros((b, n_heads, s))
+    col, head = 0, 0
+    for nh in heads_per_shard:
+        q0, k0, v0 = col, col + nh * hd, col + 2 * nh * hd
+        for j in range(nh):
+            for bb in range(b):
+                rows = slice(bb * s, (bb + 1) * s)
+                O, L = attention_head(X[rows, q0 + j * hd:q0 + (j + 1) * hd],
+                                      X[rows, k0 + j * hd:k0 + (j + 1) * hd],
+                                      X[rows, v0 + j * hd:v0 + (j + 1) * hd], causal, scale)
+                ctx[rows, (head + j) * hd:(head + j + 1) * hd] = O
+                lse[bb, head + j] = L
+        col += 3 * nh * hd
+        head += nh
+    if head != n_heads:
+        raise ValueError("heads_per_shard does not cover all heads")
+    return ctx, lse
 
 
 # ----------------------------------------------------------------------------

@@ -573,4 +573,68 @@ def check_linear_xent_partitioned(o):
     assert o.linear_xent(H, E2, y)["argmax"][2] == 40
 
 
+# ----------------------------------------------------------------------------
+# attention core
+# ----------------------------------------------------------------------------
+def check_attention_vs_torch(o):
+    """One head against torch's scaled_dot_product_attention in float64,
+    causal and not, default and explicit scale."""
+    import torch
+
+    r = _rng(40)
+    s, d = 9, 8
+    Q, K, V = (r.normal(size=(s, d)) for _ in range(3))
+    for causal in (True, False):
+        for scale in (None, 0.3):
+            O, lse = o.attention_head(Q, K, V, causal, scale)
+            t = lambda x: torch.from_numpy(x)[None, None]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                t(Q), t(K), t(V), is_causal=causal, scale=scale)[0, 0].numpy()
+            assert _rel(O, ref) < 1e-14, (causal, scale)
+            sc = 1 / math.sqrt(d) if scale is None else scale
+            S = torch.from_numpy(Q @ K.T * sc)
+            if causal:
+                S = S.masked_fill(~torch.ones(s, s, dtype=torch.bool).tril(), float("-inf"))
+            assert _rel(lse, torch.logsumexp(S, dim=1).numpy()) < 1e-14
+
+
+def check_attention_bruteforce_and_closed_forms(o):
+    """Scalar loops on a tiny head; constant V gives V back; zero scores give
+    the running mean of V under the causal mask (row i averages rows 0..i)."""
+    r = _rng(41)
+    s, d = 5, 3
+    Q, K, V = (r.normal(size=(s, d)) for _ in range(3))
+    O, _ = o.attention_head(Q, K, V, causal=True, scale=0.7)
+    for i in range(s):
+        w = [math.exp(0.7 * sum(Q[i][k] * K[j][k] for k in range(d))) for j in range(i + 1)]
+        for c in range(d):
+            want = sum(w[j] * V[j][c] for j in range(i + 1)) / sum(w)
+            assert abs(O[i, c] - want) < 1e-13
+    Vc = np.tile(r.normal(size=(1, d)), (s, 1))
+    assert np.allclose(o.attention_head(Q, K, Vc)[0], Vc, rtol=0, atol=1e-14)
+    O0, lse0 = o.attention_head(np.zeros((s, d)), K, V, causal=True)
+    want = np.cumsum(V, axis=0) / np.arange(1, s + 1)[:, None]
+    assert _rel(O0, want) < 1e-14
+    assert np.allclose(lse0, np.log(np.arange(1, s + 1)), rtol=0, atol=1e-14)
+
+
+def check_attention_sharded_layout(o):
+    """Shard-major QKV of uneven head shards: the per-shard core equals
+    standard multi-head attention on the [Q | K | V] layout (torch, float64),
+    batch rows kept apart."""
+    import torch
+
+    r = _rng(42)
+    b, s, nh, hd = 2, 6, 5, 4
+    shards = [2, 1, 1, 1]
+    std = r.normal(size=(b * s, 3 * nh * hd))            # standard [Q | K | V], heads in order
+    perm, offs = o.qkv_shard_columns(nh, hd, shards)
+    ctx, lse = o.attention_sharded(std[:, perm], b, s, nh, hd, shards, causal=True)
+    t = torch.from_numpy(std).view(b, s, 3, nh, hd).permute(2, 0, 3, 1, 4)   # [3, b, nh, s, hd]
+    ref = torch.nn.functional.scaled_dot_product_attention(t[0], t[1], t[2], is_causal=True)
+    ref = ref.permute(0, 2, 1, 3).reshape(b * s, nh * hd).numpy()
+    assert _rel(ctx, ref) < 1e-14
+    assert lse.shape == (b, nh, s)
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

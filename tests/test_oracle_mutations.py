@@ -213,6 +213,40 @@ def _m_recompute_uses_derivative(mp):
     mp.setattr(O, "mlp_bwd_recompute", bad)
 
 
+def _m_attention_mask_off_by_one(mp):
+    orig = O.attention_head
+
+    def bad(Q, K, V, causal=True, scale=None):
+        if not causal:
+            return orig(Q, K, V, causal, scale)
+        Q, K, V = O.f64(Q), O.f64(K), O.f64(V)
+        s, d = Q.shape
+        sc = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+        S = (Q @ K.T) * sc
+        S = np.where(np.tril(np.ones((s, s), dtype=bool), k=-1), S, -np.inf)   # drops the diagonal
+        S[0, 0] = 0.0
+        m = S.max(axis=1)
+        P = np.exp(S - m[:, None])
+        l = P.sum(axis=1)
+        return (P / l[:, None]) @ V, m + np.log(l)
+    mp.setattr(O, "attention_head", bad)
+
+
+def _m_attention_kv_swapped(mp):
+    orig = O.attention_sharded
+
+    def bad(QKV, b, s, n_heads, head_dim, heads_per_shard, causal=True, scale=None):
+        X = O.f64(QKV).copy()
+        col = 0
+        for nh in heads_per_shard:                    # reads V where K should be and back
+            k0, v0 = col + nh * head_dim, col + 2 * nh * head_dim
+            X[:, k0:k0 + nh * head_dim], X[:, v0:v0 + nh * head_dim] = (
+                X[:, v0:v0 + nh * head_dim].copy(), X[:, k0:k0 + nh * head_dim].copy())
+            col += 3 * nh * head_dim
+        return orig(X, b, s, n_heads, head_dim, heads_per_shard, causal, scale)
+    mp.setattr(O, "attention_sharded", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
