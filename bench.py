@@ -48,6 +48,7 @@ VOC = dict(T=16384, v=50304, h=4096, N=8, e_std=0.02)
 MLP_FLOP = 12.0 * MLP["M"] * MLP["h"] * MLP["F"]                       # 6 GEMMs x 2MhF
 PROJ_FLOP = 6.0 * PROJ["M"] * PROJ["h"] * 3 * PROJ["h"] + 6.0 * PROJ["M"] * PROJ["h"] ** 2
 LOGITS_FLOP = 2.0 * VOC["T"] * VOC["v"] * VOC["h"]
+ATTN_FLOP = 4.0 * 4 * 25 * 64 * (1024 * 1025 / 2)                      # b=4, 25 heads, s=1024
 LOGITS_BWD_FLOP = 2.0 * LOGITS_FLOP
 # algorithmic bytes: read + write every logit once, plus targets / loss / argmax
 XENT_BYTES = 2 * 4 * VOC["T"] * VOC["v"] + VOC["T"] * (8 + 4 + 4)
@@ -175,7 +176,7 @@ def _prepare(dev, parts):
     bf = dict(dtype=torch.bfloat16, device=dev)
     if any(p.startswith("mlp") for p in parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
-    if "proj" in parts:
+    if "proj" in parts or "attn_fwd" in parts:
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
     if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd",
                                 "lxent_fwd", "lxent_dlogits")):
@@ -210,7 +211,12 @@ def _prepare_proj(dev, tpl, tp_inputs, torch, bf):
     Mp, hp = PROJ["M"], PROJ["h"]
     pr.update(QKV=torch.empty(Mp, 3 * hp, **bf), dXq=torch.empty(Mp, hp, **bf),
               dWq=torch.empty(hp, 3 * hp, **bf), dbq=torch.empty(3 * hp, dtype=torch.float32, device=dev),
-              Zo=torch.empty(Mp, hp, **bf), dctx=torch.empty(Mp, hp, **bf), dWo=torch.empty(hp, hp, **bf))
+              Zo=torch.empty(Mp, hp, **bf), dctx=torch.empty(Mp, hp, **bf), dWo=torch.empty(hp, hp, **bf),
+              ctx_attn=torch.empty(Mp, hp, **bf))
+    # the attention core reads the QKV projection of these inputs
+    tpl.tp_col_linear_fwd(pr["X"], pr["Wqkv"], pr["bqkv"], PROJ["N"], shard_offsets=pr["qkv_offs"],
+                          Y=pr["QKV"])
+    torch.cuda.synchronize(dev)
     pr["ws_q"] = torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_COL_LINEAR_BWD, Mp, hp, 3 * hp,
                                                            PROJ["N"])), dtype=torch.uint8, device=dev)
     pr["ws_o"] = torch.empty(max(1, tpl.tp_workspace_bytes(tpl.OP_ROW_LINEAR_FWD, Mp, hp, hp,
@@ -298,6 +304,11 @@ def _mlp_bwd_rc(tpl, g, st):
                              ws=g["ws_b"], dev_status=st)
 
 
+def _attn_fwd(tpl, pr, st):
+    tpl.tp_attention_fwd(pr["QKV"], PROJ["M"] // 1024, 1024, PROJ["n_heads"], PROJ["N"],
+                         causal=True, ctx=pr["ctx_attn"], dev_status=st)
+
+
 def _lxent_fwd(tpl, vo, st):
     tpl.tp_linear_xent_fwd(vo["H"], vo["E"], vo["targets"], VOC["N"], loss=vo["loss"],
                            loss_sum=vo["loss_sum"], lse=vo["lse"], argmax=vo["argmax"],
@@ -321,6 +332,8 @@ BWD_PARTS = ("logits", "xent_bf16", "logits_bwd", "embed_bwd")
 FUSED_PARTS = ("lxent_fwd", "lxent_dlogits")
 # the MLP backward with activation recompute (Y rebuilt from U), own loop
 RECOMPUTE_PARTS = ("mlp_bwd_rc",)
+# the attention core between the projections (b=4, s=1024, causal), own loop
+ATTN_PARTS = ("attn_fwd",)
 
 
 def _e2e_mlp(tpl, torch, g, dev, steps):
@@ -434,7 +447,7 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS
+    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS + ATTN_PARTS
     parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
         raise SystemExit(f"--parts must name some of {','.join(known)}")
@@ -455,7 +468,8 @@ def run_gpu(args):
            "embed_bwd": lambda: _embed_bwd(tpl, vo, st),
            "lxent_fwd": lambda: _lxent_fwd(tpl, vo, st),
            "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st),
-           "mlp_bwd_rc": lambda: _mlp_bwd_rc(tpl, g, st)}
+           "mlp_bwd_rc": lambda: _mlp_bwd_rc(tpl, g, st),
+           "attn_fwd": lambda: _attn_fwd(tpl, pr, st)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -513,6 +527,7 @@ def run_gpu(args):
     bwd_ms = _side_loop(torch, fns, BWD_PARTS, side_steps, stream, dev, st, world)
     fused_ms = _side_loop(torch, fns, FUSED_PARTS, side_steps, stream, dev, st, world)
     rc_ms = _side_loop(torch, fns, RECOMPUTE_PARTS, side_steps, stream, dev, st, world)
+    at_ms = _side_loop(torch, fns, ATTN_PARTS, side_steps, stream, dev, st, world)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
@@ -595,6 +610,13 @@ def run_gpu(args):
                 "tflops": round(4.0 * MLP["M"] * MLP["h"] * MLP["F"] * 2 / (rc_ms["mlp_bwd_rc"] / 1e3) / 1e12, 1),
                 "saved_activation_ms": round(part_ms["mlp_bwd"] / K, 4),
                 "activation_bytes_not_kept": MLP["M"] * MLP["F"] * 2,
+            },
+            "attention_fwd": {
+                "what": "causal attention core between the projections, b=4 s=1024, 25 heads of 64 "
+                        "over 4 shards (7/6/6/6); own loop of %d iterations" % side_steps,
+                "us": round(at_ms["attn_fwd"] * 1e3, 2),
+                "tflops": round(ATTN_FLOP / (at_ms["attn_fwd"] / 1e3) / 1e12, 1),
+                "flop_note": "4·b·heads·d·s(s+1)/2 (the unmasked half of Q·Kᵀ and P·V)",
             },
             "parts_ms_per_step": {p: round(part_ms[p] / K, 4) for p in PARTS},
             "roofline": {

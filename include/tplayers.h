@@ -379,6 +379,36 @@ TP_API tp_status vp_embed_bwd(const int64_t* ids, const void* dout, int64_t T, i
                               int32_t* dev_status, void* stream);
 
 /*
+ * Attention core between the projections, per-shard heads   [MLP-TP] §2.2;
+ * [TP-ILL] §3.1 (heads are independent, so each GPU computes attention for
+ * its own heads with no communication; only the output projection's sum
+ * follows).
+ *
+ *   For every sequence and head:  O = softmax(Q·Kᵀ·scale + mask)·V, with the
+ *   causal mask (key j hidden from query i for j > i) when causal != 0.
+ *
+ *   QKV [b·s, 3·n_heads·64] bf16: the column-parallel projection's output in
+ *   the shard-major layout — shard i (heads [head_offsets[i],
+ *   head_offsets[i+1])) holds its Q heads, then its K heads, then its V
+ *   heads, each head 64 columns; row = batch·s + position.
+ *   ctx [b·s, n_heads·64] bf16 out: heads in order, so shard i's context is
+ *   the column block [64·head_offsets[i], 64·head_offsets[i+1]) — the input of
+ *   its rows of tp_row_linear_fwd.  lse [b, n_heads, s] fp32 (nullable): the
+ *   natural-log sum of exp of each query's scaled, masked scores.
+ *   head_offsets: N+1 increasing head indices from 0 to n_heads, or NULL for
+ *   the contiguous split that gives the first n_heads mod N shards one head
+ *   more (25 heads over 4: 7, 6, 6, 6).  scale <= 0 selects 1/sqrt(64).
+ *   head_dim must be 64 and n_heads <= 256 (else TP_ERR_UNSUPPORTED); any
+ *   s >= 1.  QKV and ctx 16-byte aligned.
+ *   The formula is an image lost from the pages; this is the standard
+ *   scaled dot-product attention of the GPT-2 layer, without dropout.
+ */
+TP_API tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t n_heads,
+                                  int32_t head_dim, int32_t N, const int64_t* head_offsets,
+                                  int32_t causal, float scale, void* ctx, float* lse,
+                                  int32_t* dev_status, void* stream);
+
+/*
  * Output layer and cross-entropy in one pass, without the logits matrix
  *   [TP-ILL] §4.2 (logits = H·Eᵀ against the shared table) and §5 (the loss
  *   from per-part maxima and rescaled sums, so that no part of the [T,v]

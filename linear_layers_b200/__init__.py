@@ -29,6 +29,7 @@ __all__ = [
     "vp_embed", "tp_logits_fwd", "vp_xent", "vp_xent_bf16_grad", "tp_logits_bwd", "vp_embed_bwd",
     "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT", "tp_mlp_bwd_recompute",
+    "tp_attention_fwd",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
@@ -75,6 +76,7 @@ _SIGS = {
     "tp_linear_xent_fwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _SZ,
                             _P, _P], _I32),
     "tp_linear_xent_dlogits": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _F, _P, _P, _P], _I32),
+    "tp_attention_fwd": ([_P, _I64, _I64, _I32, _I32, _I32, _P, _I32, _F, _P, _P, _P, _P], _I32),
     "tp_mlp_bwd_recompute": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                               _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
 }
@@ -475,3 +477,21 @@ def tp_linear_xent_dlogits(H, E, targets, lse, N, *, grad_scale=1.0, dlogits=Non
                                         float(grad_scale), _ptr(dlogits), _ptr(dev_status),
                                         _stream(dev)), "tp_linear_xent_dlogits")
     return dlogits
+
+
+def tp_attention_fwd(QKV, b, s, n_heads, N, *, head_offsets=None, causal=True, scale=None,
+                     ctx=None, lse=None, with_lse=False, dev_status=None):
+    """Per-shard attention core on the shard-major QKV [b·s, 3·n_heads·64].
+
+    Returns (ctx [b·s, n_heads·64] bf16, lse [b, n_heads, s] fp32 or None)."""
+    dev = QKV.device
+    hd = 64
+    ctx = torch.empty(b * s, n_heads * hd, dtype=QKV.dtype, device=dev) if ctx is None else ctx
+    if with_lse and lse is None:
+        lse = torch.empty(b, n_heads, s, dtype=torch.float32, device=dev)
+    _contig(QKV, ctx, lse)
+    offs, keep = _offsets(head_offsets, N)
+    _check(lib().tp_attention_fwd(_ptr(QKV), b, s, n_heads, hd, N, offs, 1 if causal else 0,
+                                  float(scale) if scale else 0.0, _ptr(ctx), _ptr(lse),
+                                  _ptr(dev_status), _stream(dev)), "tp_attention_fwd")
+    return ctx, lse

@@ -873,6 +873,11 @@ int choose_cg(int M) {
 
 }  // namespace
 
+bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                          uint32_t box_inner, uint32_t box_outer) {
+  return make_tmap(static_cast<CUtensorMap*>(tmap), ptr, inner, outer, ld, box_inner, box_outer);
+}
+
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
   if (splits <= 1) return 0;
   // 128-row half tiles of the 256-row tiling (covers the 128-row tiling too)

@@ -78,6 +78,17 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream);
 tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
                               cudaStream_t stream);
 
+// Tensor map (a CUtensorMap, 128 bytes) of a row-major bf16 matrix
+// [outer, inner] with row stride ld elements: boxes of box_inner x box_outer
+// elements, 128-byte swizzle, zero fill outside the matrix.
+bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                          uint32_t box_inner, uint32_t box_outer);
+
+// Attention core (attn.cu): see tp_attention_fwd.
+tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
+                               const int64_t* head_offsets, int N, bool causal, float scale,
+                               void* ctx, float* lse, int32_t* dev_status, cudaStream_t stream);
+
 // Counts every kernel the library enqueues (tp_launch_count).
 void note_launches(int n);
 

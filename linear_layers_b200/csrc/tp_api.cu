@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -633,6 +634,31 @@ tp_status vp_xent_bf16_grad(const float* logits, const int64_t* targets, int64_t
   if (tp_status s = require_sm100()) return s;
   return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, true, argmax,
                         dev_status, as_stream(stream));
+}
+
+tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t n_heads,
+                           int32_t head_dim, int32_t N, const int64_t* head_offsets,
+                           int32_t causal, float scale, void* ctx, float* lse,
+                           int32_t* dev_status, void* stream) {
+  if (!QKV || !ctx) return TP_ERR_NULL;
+  if (b <= 0 || s <= 0 || n_heads <= 0 || N < 1 || N > n_heads || b * s > (1ll << 30))
+    return TP_ERR_SHAPE;
+  if (head_dim != 64 || n_heads > 256) return TP_ERR_UNSUPPORTED;
+  if (!ptrs_aligned({QKV, ctx}) || (reinterpret_cast<uintptr_t>(lse) & 3)) return TP_ERR_ALIGN;
+  std::vector<int64_t> offs(N + 1);
+  if (head_offsets == nullptr) {   // contiguous split, the first n_heads mod N shards one larger
+    offs[0] = 0;
+    for (int i = 0; i < N; ++i) offs[i + 1] = offs[i] + n_heads / N + (i < n_heads % N ? 1 : 0);
+  } else {
+    for (int i = 0; i <= N; ++i) offs[i] = head_offsets[i];
+    if (offs[0] != 0 || offs[N] != n_heads) return TP_ERR_SHAPE;
+    for (int i = 0; i < N; ++i)
+      if (offs[i + 1] <= offs[i]) return TP_ERR_SHAPE;
+  }
+  if (!(scale > 0.0f) || !std::isfinite(scale)) scale = 1.0f / std::sqrt(static_cast<float>(head_dim));
+  if (tp_status st = require_sm100()) return st;
+  return attention_fwd_launch(QKV, b, s, n_heads, offs.data(), N, causal != 0, scale, ctx, lse,
+                              dev_status, as_stream(stream));
 }
 
 tp_status tp_linear_xent_fwd(const void* H, const void* E, const int64_t* targets, int64_t T,

@@ -113,6 +113,13 @@ def test_validation_errors_before_any_launch(L):
               None) == 7                                       # TP_ERR_WORKSPACE
     assert L.tp_linear_xent_dlogits(FAKE, FAKE, FAKE, FAKE, 4, 64, 300, 2, 1.0, FAKE, None,
                                     None) == TP_ERR_ALIGN     # bf16 rows need 8 | v
+    # attention core: head_dim 64 only, shards cover the heads
+    at = L.tp_attention_fwd
+    assert at(FAKE, 2, 16, 4, 128, 2, None, 1, 0.0, FAKE, None, None, None) == 5   # UNSUPPORTED
+    assert at(FAKE, 2, 16, 4, 64, 5, None, 1, 0.0, FAKE, None, None, None) == TP_ERR_SHAPE
+    bad = (ctypes.c_int64 * 3)(0, 3, 3)                        # empty shard
+    assert at(FAKE, 2, 16, 3, 64, 2, bad, 1, 0.0, FAKE, None, None, None) == TP_ERR_SHAPE
+    assert at(None, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, None, None, None) == TP_ERR_NULL
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
@@ -125,6 +132,8 @@ def test_valid_call_without_gpu_fails_loudly(L):
                                 wsb, None, None) == TP_ERR_DEVICE
     assert L.tp_linear_xent_dlogits(FAKE, FAKE, FAKE, FAKE, 4, 64, 304, 2, 1.0, FAKE, None,
                                     None) == TP_ERR_DEVICE
+    assert L.tp_attention_fwd(FAKE, 2, 16, 25, 64, 4, None, 1, 0.0, FAKE, None, None,
+                              None) == TP_ERR_DEVICE
     with pytest.raises(RuntimeError, match="no CPU path"):
         X = torch.zeros(16, 64, dtype=torch.bfloat16)
         tpl.tp_mlp_fwd(X, torch.zeros(64, 256, dtype=torch.bfloat16), None,

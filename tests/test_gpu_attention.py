@@ -1,0 +1,120 @@
+"""Attention core between the projections (per-shard heads) on the GPU
+against the fp64 oracle (through the C ABI).
+
+The scores are fp32 accumulations of bf16 Q·Kᵀ; P is rounded to bf16 for the
+P·V product and the context is stored in bf16, so the context is compared
+with TOL_BF16 (relative Frobenius per head and sequence) and the
+log-sum-exp per query with TOL_XENT.
+"""
+import numpy as np
+import pytest
+import torch
+
+import linear_layers_b200 as tpl
+import tp_inputs
+from oracle import tp_oracle as O
+from tests.gpu_helpers import TOL_BF16, TOL_XENT, assert_close, f64
+
+pytestmark = pytest.mark.gpu
+
+HD = 64
+
+
+def _qkv(b, s, nh, seed, std=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (std * torch.randn(b * s, 3 * nh * HD, generator=g)).bfloat16()
+
+
+def _offsets(nh, N):
+    heads = tp_inputs.head_split(nh, N)
+    return [0] + list(np.cumsum(heads))
+
+
+def _check(QKV, b, s, nh, N, causal, offs=None, scale=None):
+    st = tpl.new_status()
+    ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, head_offsets=offs, causal=causal,
+                                    scale=scale, with_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    shards = np.diff(offs if offs is not None else _offsets(nh, N)).tolist()
+    rctx, rlse = O.attention_sharded(QKV, b, s, nh, HD, shards, causal=causal, scale=scale)
+    g = f64(ctx)
+    for bb in range(b):
+        for hh in range(nh):
+            rows, cols = slice(bb * s, (bb + 1) * s), slice(hh * HD, (hh + 1) * HD)
+            assert_close(f"ctx[b={bb},h={hh}]", g[rows, cols], rctx[rows, cols], TOL_BF16)
+    gl = f64(lse)
+    assert (np.abs(gl - rlse) / np.maximum(np.abs(rlse), 1.0)).max() <= TOL_XENT
+    return ctx
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("b,s,nh,N", [(2, 200, 5, 3),     # ragged second query tile
+                                      (1, 128, 2, 2),     # one full tile
+                                      (3, 37, 4, 1),      # shorter than one tile
+                                      (1, 1, 1, 1),       # a single token
+                                      (2, 384, 3, 3)])    # three tiles, causal diagonal blocks
+def test_attention_small(b, s, nh, N, causal):
+    _check(_qkv(b, s, nh, seed=s + nh), b, s, nh, N, causal)
+
+
+def test_attention_explicit_offsets_and_scale():
+    b, s, nh = 2, 260, 6
+    _check(_qkv(b, s, nh, seed=7), b, s, nh, 3, True, offs=[0, 1, 4, 6], scale=0.05)
+
+
+def test_attention_large_scores():
+    """Scores of size ~±60 after scaling: the running maximum and the
+    rescaling of O keep the softmax exact in fp32."""
+    b, s, nh = 1, 512, 2
+    _check(_qkv(b, s, nh, seed=8, std=3.0), b, s, nh, 2, True)
+
+
+@pytest.mark.slow
+def test_attention_gpt2_slice():
+    """b=4, s=1024, 25 heads of 64 over 4 shards (7, 6, 6, 6): every head of
+    two sequences against the oracle; the other two by their log-sum-exp."""
+    w = tp_inputs.WORKLOADS["gpt2_1p5b_slice"]
+    b, s, nh, N = 4, 1024, w["n_heads"], w["N"]
+    QKV = _qkv(b, s, nh, seed=9)
+    st = tpl.new_status()
+    ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, with_lse=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    shards = tp_inputs.head_split(nh, N)
+    for bb in (0, 3):
+        rows = slice(bb * s, (bb + 1) * s)
+        rctx, rlse = O.attention_sharded(QKV[rows], 1, s, nh, HD, shards, causal=True)
+        assert_close(f"ctx[b={bb}]", ctx[rows], rctx, TOL_BF16)
+        assert (np.abs(f64(lse[bb]) - rlse[0]) / np.maximum(np.abs(rlse[0]), 1.0)).max() <= TOL_XENT
+
+
+def test_attention_layer_chain():
+    """X -> column-parallel QKV (per-shard heads) -> attention core ->
+    row-parallel output projection with its shard sum, against the oracle's
+    chain of the same three steps."""
+    b, s, nh, N, h = 2, 192, 5, 2, 5 * HD
+    inp = tp_inputs.attn_proj_inputs(b * s, h, nh, HD, N, seed=10, w_std=0.05)
+    shards = tp_inputs.head_split(nh, N)
+    qkv_offs = [0] + list(np.cumsum([3 * k * HD for k in shards]))
+    ctx_offs = [0] + list(np.cumsum([k * HD for k in shards]))
+    X, Wqkv, Wo = (inp[k].cuda() for k in ("X", "Wqkv", "Wo"))
+    QKV, _ = tpl.tp_col_linear_fwd(X, Wqkv, None, N, shard_offsets=qkv_offs)
+    ctx, _ = tpl.tp_attention_fwd(QKV, b, s, nh, N)
+    Z = tpl.tp_row_linear_fwd(ctx, Wo, N, shard_offsets=ctx_offs)
+    torch.cuda.synchronize()
+    _, rQKV = O.col_linear_fwd(inp["X"], inp["Wqkv"])
+    rctx, _ = O.attention_sharded(rQKV, b, s, nh, HD, shards, causal=True)
+    rZ, _ = O.row_linear_fwd(rctx, inp["Wo"], offsets=ctx_offs)
+    assert_close("QKV", QKV, rQKV, TOL_BF16)
+    assert_close("ctx", ctx, rctx, TOL_BF16)
+    assert_close("Z", Z, rZ, TOL_BF16)
+
+
+def test_attention_deterministic():
+    b, s, nh = 2, 300, 4
+    QKV = _qkv(b, s, nh, seed=11).cuda()
+    a, _ = tpl.tp_attention_fwd(QKV, b, s, nh, 2)
+    c, _ = tpl.tp_attention_fwd(QKV, b, s, nh, 2)
+    torch.cuda.synchronize()
+    assert torch.equal(a, c)
