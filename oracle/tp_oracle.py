@@ -47,6 +47,13 @@ design notes):
   (mathematically equal, numerically safe).  The loss is returned per token
   and as the sum over tokens ("按行加总得到 scalar Loss").
 * Ties in the arg-max go to the lowest vocabulary index.
+* [EVO] §2.3 names sequence-parallel LayerNorm and Dropout without
+  formulas; the plain reading is the transformer's residual step
+  hs = residual + dropout(x + bias), y = LayerNorm(hs) (biased variance,
+  eps = 1e-5) on each shard's token rows, with the parameter gradients
+  summed over shards.  Dropout draws from Philox4x32-10 (its published
+  definition), one 32-bit word per element, kept when the word is at least
+  floor(p·2^32).
 * The attention core's formula is an image lost from the pages; the plain
   reading is scaled dot-product attention softmax(Q·Kᵀ/√d)·V per head, with
   the causal mask of a decoder (the GPT-2 layer) selectable, and no dropout.
@@ -381,6 +388,107 @@ def attention_sharded(QKV, b, s, n_heads, head_dim, heads_per_shard, causal=True
     if head != n_heads:
         raise ValueError("heads_per_shard does not cover all heads")
     return ctx, lse
+
+
+# ----------------------------------------------------------------------------
+# Sequence-parallel dropout-add-LayerNorm ([EVO] §2.3: LayerNorm and Dropout
+# split along the sequence, each shard handling its own token rows)
+# ----------------------------------------------------------------------------
+_PHILOX_M0, _PHILOX_M1 = 0xD2511F53, 0xCD9E8D57
+_PHILOX_W0, _PHILOX_W1 = 0x9E3779B9, 0xBB67AE85
+_U32 = 0xFFFFFFFF
+
+
+def philox4x32_10(ctr, key):
+    """Philox4x32 with 10 rounds (Salmon, Moraes, Dror, Shaw, "Parallel random
+    numbers: as easy as 1, 2, 3", SC 2011).  ctr: uint32 array [..., 4], key:
+    uint32 array [..., 2].  Each round multiplies words 0 and 2 by the two
+    constants, crosses the high halves with words 1 and 3 and the key, and
+    bumps the key by the two Weyl constants.  Returns uint32 [..., 4]."""
+    c = np.asarray(ctr, dtype=np.uint64) & _U32
+    k = np.asarray(key, dtype=np.uint64) & _U32
+    c0, c1, c2, c3 = (c[..., i].copy() for i in range(4))
+    k0, k1 = k[..., 0].copy(), k[..., 1].copy()
+    for rnd in range(10):
+        if rnd:
+            k0 = (k0 + _PHILOX_W0) & _U32
+            k1 = (k1 + _PHILOX_W1) & _U32
+        p0 = c0 * _PHILOX_M0                      # exact in uint64
+        p1 = c2 * _PHILOX_M1
+        hi0, lo0 = p0 >> 32, p0 & _U32
+        hi1, lo1 = p1 >> 32, p1 & _U32
+        c0, c1, c2, c3 = hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0
+    return np.stack([c0, c1, c2, c3], axis=-1).astype(np.uint32)
+
+
+def dropout_keep(M, h, p, seed, offset):
+    """Keep mask [M, h] of dropout with drop probability p.
+
+    Element e = row·h + col draws word e mod 4 of Philox4x32-10 at counter
+    (e div 4 as two 32-bit words, offset as two 32-bit words) under key
+    seed (two 32-bit words); it is kept when that word u satisfies
+    u >= floor(p·2^32), so the keep probability is 1 − p to 2^-32.
+    """
+    n = M * h
+    q = np.arange((n + 3) // 4, dtype=np.uint64)
+    ctr = np.stack([q & _U32, q >> 32, np.full_like(q, offset & _U32),
+                    np.full_like(q, (offset >> 32) & _U32)], axis=-1)
+    key = np.broadcast_to(np.array([seed & _U32, (seed >> 32) & _U32], dtype=np.uint64),
+                          (q.size, 2))
+    words = philox4x32_10(ctr, key).reshape(-1)[:n]
+    thr = np.uint64(int(math.floor(p * 2.0 ** 32)))
+    return (words.astype(np.uint64) >= thr).reshape(M, h)
+
+
+def dropout_add_layernorm(x, bias, residual, gamma, beta, p, seed, offset, eps=1e-5):
+    """Forward: hs = residual + keep·(x + bias)/(1 − p);  y = LayerNorm(hs)·gamma + beta,
+    the LayerNorm over the hidden dimension with the biased variance.
+    Returns dict(hs, y, mean, rstd, keep)."""
+    x, residual, gamma, beta = f64(x), f64(residual), f64(gamma), f64(beta)
+    M, h = x.shape
+    keep = dropout_keep(M, h, p, seed, offset)
+    xb = x + (f64(bias)[None, :] if bias is not None else 0.0)
+    hs = residual + np.where(keep, xb / (1.0 - p), 0.0)
+    mean = hs.mean(axis=1)
+    var = ((hs - mean[:, None]) ** 2).mean(axis=1)
+    rstd = 1.0 / np.sqrt(var + eps)
+    xhat = (hs - mean[:, None]) * rstd[:, None]
+    return {"hs": hs, "y": xhat * gamma[None, :] + beta[None, :], "mean": mean, "rstd": rstd,
+            "keep": keep}
+
+
+def dropout_add_layernorm_bwd(dy, dhs_in, hs, gamma, mean, rstd, keep, p):
+    """Backward of dropout_add_layernorm.  dy: gradient at y; dhs_in
+    (nullable): gradient reaching the residual stream hs from later layers.
+    Returns dict(dx, dresidual, dbias, dgamma, dbeta)."""
+    dy, hs, gamma = f64(dy), f64(hs), f64(gamma)
+    xhat = (hs - f64(mean)[:, None]) * f64(rstd)[:, None]
+    g = dy * gamma[None, :]
+    dh = f64(rstd)[:, None] * (g - g.mean(axis=1, keepdims=True)
+                               - xhat * (g * xhat).mean(axis=1, keepdims=True))
+    if dhs_in is not None:
+        dh = dh + f64(dhs_in)
+    dx = np.where(keep, dh / (1.0 - p), 0.0)
+    return {"dx": dx, "dresidual": dh, "dbias": dx.sum(axis=0),
+            "dgamma": (dy * xhat).sum(axis=0), "dbeta": dy.sum(axis=0)}
+
+
+def dropout_add_layernorm_bwd_sharded(dy, dhs_in, hs, gamma, mean, rstd, keep, p, N):
+    """The sequence-parallel backward: shard i owns token rows [i·M/N, (i+1)·M/N)
+    and computes its rows' gradients and its partial dgamma, dbeta, dbias;
+    the parameter gradients are the all-reduce of the shards' partials."""
+    M = f64(dy).shape[0]
+    offs = even_offsets(M, N)
+    parts = []
+    for i in range(N):
+        r = slice(offs[i], offs[i + 1])
+        parts.append(dropout_add_layernorm_bwd(
+            f64(dy)[r], None if dhs_in is None else f64(dhs_in)[r], f64(hs)[r], gamma,
+            f64(mean)[r], f64(rstd)[r], keep[r], p))
+    out = {k: np.concatenate([q[k] for q in parts], axis=0) for k in ("dx", "dresidual")}
+    for k in ("dbias", "dgamma", "dbeta"):
+        out[k] = all_reduce_sum([q[k] for q in parts])
+    return out
 
 
 # ----------------------------------------------------------------------------

@@ -637,4 +637,75 @@ def check_attention_sharded_layout(o):
     assert lse.shape == (b, nh, s)
 
 
+# ----------------------------------------------------------------------------
+# sequence-parallel dropout-add-LayerNorm
+# ----------------------------------------------------------------------------
+def check_philox_known_answers(o):
+    """Philox4x32-10 against the generator's published known-answer vectors."""
+    g = _golden("philox4x32_10_kat.json")
+    for v in g["vectors"]:
+        got = o.philox4x32_10(np.array([int(w, 16) for w in v["ctr"]], dtype=np.uint64),
+                              np.array([int(w, 16) for w in v["key"]], dtype=np.uint64))
+        assert ["%08x" % w for w in got] == v["out"], (v, got)
+
+
+def check_dropout_mask_properties(o):
+    """Keep fraction within 5 sigma of 1 − p; p = 0 keeps everything; the mask is a
+    function of (seed, offset) alone; element e uses word e mod 4 of counter e div 4."""
+    M, h, p = 512, 1000, 0.1
+    k = o.dropout_keep(M, h, p, seed=1234, offset=7)
+    n = M * h
+    assert abs(k.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
+    assert o.dropout_keep(M, h, 0.0, 1234, 7).all()
+    assert np.array_equal(k, o.dropout_keep(M, h, p, 1234, 7))
+    assert not np.array_equal(k, o.dropout_keep(M, h, p, 1234, 8))
+    assert not np.array_equal(k, o.dropout_keep(M, h, p, 1235, 7))
+    w = o.philox4x32_10(np.array([2, 0, 7, 0], dtype=np.uint64), np.array([1234, 0], dtype=np.uint64))
+    e = 2 * 4 + 3                                         # counter 2, word 3
+    assert k.reshape(-1)[e] == (int(w[3]) >= int(math.floor(p * 2 ** 32)))
+
+
+def check_layernorm_vs_torch(o):
+    """Forward and backward of hs = residual + dropout(x + bias), y = LN(hs)
+    against torch (float64 autograd) with the oracle's keep mask as input."""
+    import torch
+
+    r = _rng(50)
+    M, h, p, eps = 6, 10, 0.25, 1e-5
+    x, res, bias = r.normal(size=(M, h)), r.normal(size=(M, h)), r.normal(size=h)
+    gamma, beta = 1 + 0.3 * r.normal(size=h), 0.2 * r.normal(size=h)
+    f = o.dropout_add_layernorm(x, bias, res, gamma, beta, p, seed=3, offset=11, eps=eps)
+    keep = torch.from_numpy(f["keep"].astype(np.float64))
+    T = {k: torch.from_numpy(v).requires_grad_(True)
+         for k, v in dict(x=x, res=res, bias=bias, gamma=gamma, beta=beta).items()}
+    hs = T["res"] + keep * (T["x"] + T["bias"]) / (1 - p)
+    y = torch.nn.functional.layer_norm(hs, (h,), T["gamma"], T["beta"], eps)
+    assert _rel(f["hs"], hs.detach().numpy()) < 1e-15
+    assert _rel(f["y"], y.detach().numpy()) < 1e-14
+    dy, dhs = r.normal(size=(M, h)), r.normal(size=(M, h))
+    (y * torch.from_numpy(dy)).sum().add((hs * torch.from_numpy(dhs)).sum()).backward()
+    b = o.dropout_add_layernorm_bwd(dy, dhs, f["hs"], gamma, f["mean"], f["rstd"], f["keep"], p)
+    for name, t in (("dx", "x"), ("dresidual", "res"), ("dbias", "bias"), ("dgamma", "gamma"),
+                    ("dbeta", "beta")):
+        assert _rel(b[name], T[t].grad.numpy()) < 1e-13, name
+    assert f["keep"].any() and not f["keep"].all()
+
+
+def check_layernorm_sequence_shards(o):
+    """Each shard of token rows gives its own rows' gradients; the parameter
+    gradients are the sum of the shards' partials (uneven last shard)."""
+    r = _rng(51)
+    M, h, p = 12, 8, 0.1
+    x, res = r.normal(size=(M, h)), r.normal(size=(M, h))
+    gamma, beta = 1 + 0.3 * r.normal(size=h), 0.2 * r.normal(size=h)
+    f = o.dropout_add_layernorm(x, None, res, gamma, beta, p, seed=9, offset=0)
+    dy = r.normal(size=(M, h))
+    ref = o.dropout_add_layernorm_bwd(dy, None, f["hs"], gamma, f["mean"], f["rstd"], f["keep"], p)
+    for N in (1, 3, 4):
+        s = o.dropout_add_layernorm_bwd_sharded(dy, None, f["hs"], gamma, f["mean"], f["rstd"],
+                                                f["keep"], p, N)
+        for k in ref:
+            assert _rel(s[k], ref[k]) < 1e-14, (N, k)
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

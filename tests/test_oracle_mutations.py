@@ -247,6 +247,45 @@ def _m_attention_kv_swapped(mp):
     mp.setattr(O, "attention_sharded", bad)
 
 
+def _m_philox_wrong_weyl(mp):
+    mp.setattr(O, "_PHILOX_W1", 0xBB67AE86)
+
+
+def _m_layernorm_unbiased_variance(mp):
+    orig = O.dropout_add_layernorm
+
+    def bad(x, bias, residual, gamma, beta, p, seed, offset, eps=1e-5):
+        f = orig(x, bias, residual, gamma, beta, p, seed, offset, eps)
+        hs = f["hs"]
+        var = hs.var(axis=1, ddof=1)                     # n − 1 in place of n
+        f["rstd"] = 1.0 / np.sqrt(var + eps)
+        xhat = (hs - f["mean"][:, None]) * f["rstd"][:, None]
+        f["y"] = xhat * O.f64(gamma)[None, :] + O.f64(beta)[None, :]
+        return f
+    mp.setattr(O, "dropout_add_layernorm", bad)
+
+
+def _m_dropout_no_rescale(mp):
+    orig = O.dropout_add_layernorm_bwd
+
+    def bad(dy, dhs_in, hs, gamma, mean, rstd, keep, p):
+        r = orig(dy, dhs_in, hs, gamma, mean, rstd, keep, p)
+        r["dx"] = r["dx"] * (1.0 - p)                   # dropped the 1/(1 − p)
+        r["dbias"] = r["dx"].sum(axis=0)
+        return r
+    mp.setattr(O, "dropout_add_layernorm_bwd", bad)
+
+
+def _m_layernorm_dgamma_without_xhat(mp):
+    orig = O.dropout_add_layernorm_bwd
+
+    def bad(dy, dhs_in, hs, gamma, mean, rstd, keep, p):
+        r = orig(dy, dhs_in, hs, gamma, mean, rstd, keep, p)
+        r["dgamma"] = O.f64(dy).sum(axis=0)
+        return r
+    mp.setattr(O, "dropout_add_layernorm_bwd", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
