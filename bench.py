@@ -49,6 +49,8 @@ MLP_FLOP = 12.0 * MLP["M"] * MLP["h"] * MLP["F"]                       # 6 GEMMs
 PROJ_FLOP = 6.0 * PROJ["M"] * PROJ["h"] * 3 * PROJ["h"] + 6.0 * PROJ["M"] * PROJ["h"] ** 2
 LOGITS_FLOP = 2.0 * VOC["T"] * VOC["v"] * VOC["h"]
 ATTN_FLOP = 4.0 * 4 * 25 * 64 * (1024 * 1025 / 2)                      # b=4, 25 heads, s=1024
+LN_FWD_BYTES = 8.0 * 4096 * 1600
+LN_BWD_BYTES = 10.0 * 4096 * 1600
 LOGITS_BWD_FLOP = 2.0 * LOGITS_FLOP
 # algorithmic bytes: read + write every logit once, plus targets / loss / argmax
 XENT_BYTES = 2 * 4 * VOC["T"] * VOC["v"] + VOC["T"] * (8 + 4 + 4)
@@ -176,7 +178,7 @@ def _prepare(dev, parts):
     bf = dict(dtype=torch.bfloat16, device=dev)
     if any(p.startswith("mlp") for p in parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
-    if "proj" in parts or "attn_fwd" in parts:
+    if "proj" in parts or "attn_fwd" in parts or "ln_fwd" in parts or "ln_bwd" in parts:
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
     if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd",
                                 "lxent_fwd", "lxent_dlogits")):
@@ -211,8 +213,22 @@ def _prepare_proj(dev, tpl, tp_inputs, torch, bf):
     Mp, hp = PROJ["M"], PROJ["h"]
     pr.update(QKV=torch.empty(Mp, 3 * hp, **bf), dXq=torch.empty(Mp, hp, **bf),
               dWq=torch.empty(hp, 3 * hp, **bf), dbq=torch.empty(3 * hp, dtype=torch.float32, device=dev),
-              Zo=torch.empty(Mp, hp, **bf), dctx=torch.empty(Mp, hp, **bf), dWo=torch.empty(hp, hp, **bf),
+              Zo=torch.zeros(Mp, hp, **bf), dctx=torch.zeros(Mp, hp, **bf), dWo=torch.empty(hp, hp, **bf),
               ctx_attn=torch.empty(Mp, hp, **bf))
+    # the residual step after the output projection: hs = X + dropout(Zo + b), y = LN(hs)
+    gl = torch.Generator().manual_seed(5)
+    pr.update(ln_bias=(0.1 * torch.randn(hp, generator=gl)).to(**bf),
+              ln_gamma=(1 + 0.1 * torch.randn(hp, generator=gl)).to(**bf),
+              ln_beta=(0.1 * torch.randn(hp, generator=gl)).to(**bf),
+              ln_hs=torch.empty(Mp, hp, **bf), ln_y=torch.empty(Mp, hp, **bf),
+              ln_mean=torch.empty(Mp, dtype=torch.float32, device=dev),
+              ln_rstd=torch.empty(Mp, dtype=torch.float32, device=dev),
+              ln_dx=torch.empty(Mp, hp, **bf), ln_dres=torch.empty(Mp, hp, **bf),
+              ln_dg=torch.empty(hp, dtype=torch.float32, device=dev),
+              ln_db=torch.empty(hp, dtype=torch.float32, device=dev),
+              ln_dbias=torch.empty(hp, dtype=torch.float32, device=dev),
+              ln_ws=torch.empty(tpl.tp_workspace_bytes(tpl.OP_SP_LN_BWD, Mp, hp, hp, PROJ["N"]),
+                                dtype=torch.uint8, device=dev))
     # the attention core reads the QKV projection of these inputs
     tpl.tp_col_linear_fwd(pr["X"], pr["Wqkv"], pr["bqkv"], PROJ["N"], shard_offsets=pr["qkv_offs"],
                           Y=pr["QKV"])
@@ -309,6 +325,23 @@ def _attn_fwd(tpl, pr, st):
                          causal=True, ctx=pr["ctx_attn"], dev_status=st)
 
 
+LN_P, LN_SEED = 0.1, 1234
+
+
+def _ln_fwd(tpl, pr, st):
+    tpl.tp_sp_dropout_add_ln_fwd(pr["Zo"], pr["ln_bias"], pr["X"], pr["ln_gamma"], pr["ln_beta"],
+                                 PROJ["N"], p=LN_P, seed=LN_SEED, offset=0, hs=pr["ln_hs"],
+                                 y=pr["ln_y"], mean=pr["ln_mean"], rstd=pr["ln_rstd"], dev_status=st)
+
+
+def _ln_bwd(tpl, pr, st):
+    tpl.tp_sp_dropout_add_ln_bwd(pr["dZ"], pr["dctx"], pr["ln_hs"], pr["ln_gamma"], pr["ln_mean"],
+                                 pr["ln_rstd"], PROJ["N"], p=LN_P, seed=LN_SEED, offset=0,
+                                 dx=pr["ln_dx"], dresidual=pr["ln_dres"], dgamma=pr["ln_dg"],
+                                 dbeta=pr["ln_db"], dbias=pr["ln_dbias"], ws=pr["ln_ws"],
+                                 dev_status=st)
+
+
 def _lxent_fwd(tpl, vo, st):
     tpl.tp_linear_xent_fwd(vo["H"], vo["E"], vo["targets"], VOC["N"], loss=vo["loss"],
                            loss_sum=vo["loss_sum"], lse=vo["lse"], argmax=vo["argmax"],
@@ -334,6 +367,8 @@ FUSED_PARTS = ("lxent_fwd", "lxent_dlogits")
 RECOMPUTE_PARTS = ("mlp_bwd_rc",)
 # the attention core between the projections (b=4, s=1024, causal), own loop
 ATTN_PARTS = ("attn_fwd",)
+# sequence-parallel dropout-add-LayerNorm after the output projection, own loop
+LN_PARTS = ("ln_fwd", "ln_bwd")
 
 
 E2E_DATA = (("X", "dZ"), ("Z", "dX"))
@@ -453,7 +488,7 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS + ATTN_PARTS
+    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS + ATTN_PARTS + LN_PARTS
     parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
         raise SystemExit(f"--parts must name some of {','.join(known)}")
@@ -475,7 +510,9 @@ def run_gpu(args):
            "lxent_fwd": lambda: _lxent_fwd(tpl, vo, st),
            "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st),
            "mlp_bwd_rc": lambda: _mlp_bwd_rc(tpl, g, st),
-           "attn_fwd": lambda: _attn_fwd(tpl, pr, st)}
+           "attn_fwd": lambda: _attn_fwd(tpl, pr, st),
+           "ln_fwd": lambda: _ln_fwd(tpl, pr, st),
+           "ln_bwd": lambda: _ln_bwd(tpl, pr, st)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
@@ -534,6 +571,7 @@ def run_gpu(args):
     fused_ms = _side_loop(torch, fns, FUSED_PARTS, side_steps, stream, dev, st, world)
     rc_ms = _side_loop(torch, fns, RECOMPUTE_PARTS, side_steps, stream, dev, st, world)
     at_ms = _side_loop(torch, fns, ATTN_PARTS, side_steps, stream, dev, st, world)
+    ln_ms = _side_loop(torch, fns, LN_PARTS, side_steps, stream, dev, st, world)
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
@@ -625,6 +663,17 @@ def run_gpu(args):
                 "us": round(at_ms["attn_fwd"] * 1e3, 2),
                 "tflops": round(ATTN_FLOP / (at_ms["attn_fwd"] / 1e3) / 1e12, 1),
                 "flop_note": "4·b·heads·d·s(s+1)/2 (the unmasked half of Q·Kᵀ and P·V)",
+            },
+            "sp_layernorm": {
+                "what": "hs = X + dropout(Zo + b), y = LayerNorm(hs) and its backward, M=4096 "
+                        "h=1600 over 4 sequence shards, p=0.1 (Philox masks regenerated in the "
+                        "backward); own loop of %d iterations" % side_steps,
+                "fwd_us": round(ln_ms["ln_fwd"] * 1e3, 2),
+                "fwd_GBps": round(LN_FWD_BYTES / (ln_ms["ln_fwd"] / 1e3) / 1e9, 1),
+                "bwd_us": round(ln_ms["ln_bwd"] * 1e3, 2),
+                "bwd_GBps": round(LN_BWD_BYTES / (ln_ms["ln_bwd"] / 1e3) / 1e9, 1),
+                "bytes_note": "8 B/element forward (x, residual in; hs, y out), 10 B/element "
+                              "backward (dy, dhs, hs in; dx, dresidual out)",
             },
             "parts_ms_per_step": {p: round(part_ms[p] / K, 4) for p in PARTS},
             "roofline": {

@@ -93,7 +93,8 @@ typedef enum {
   TP_OP_COL_LINEAR_BWD = 3,
   TP_OP_ROW_LINEAR_BWD = 4,
   TP_OP_EMBED_BWD = 5,    /* pass (T, h, v, N): T tokens */
-  TP_OP_LINEAR_XENT = 6   /* pass (T, h, v, N) */
+  TP_OP_LINEAR_XENT = 6,  /* pass (T, h, v, N) */
+  TP_OP_SP_LN_BWD = 7     /* pass (M, h, h, N): M token rows of width h */
 } tp_op;
 
 /*
@@ -407,6 +408,55 @@ TP_API tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t
                                   int32_t head_dim, int32_t N, const int64_t* head_offsets,
                                   int32_t causal, float scale, void* ctx, float* lse,
                                   int32_t* dev_status, void* stream);
+
+/*
+ * Sequence-parallel dropout-add-LayerNorm   [EVO] Megatron history page §2.3
+ * "序列并行与激活重计算" (LayerNorm and Dropout split along the sequence:
+ * each shard handles its own token rows, so their activations are split too).
+ *
+ *   hs = residual + keep · (x + bias) / (1 − p)            [M,h] bf16 out
+ *   y  = (hs − mean)·rstd·gamma + beta                      [M,h] bf16 out
+ *   mean, rstd [M] fp32 out: mean and 1/sqrt(biased variance + eps) of hs
+ *   as stored (bf16).
+ *
+ *   Shard i owns rows [i·M/N, (i+1)·M/N) (M % N == 0); on one device all
+ *   shards run in one launch.  keep: element e = row·h + col uses word e mod 4
+ *   of Philox4x32-10 (Salmon et al., SC 2011) at counter (e div 4 as two
+ *   32-bit words, offset as two 32-bit words) under key seed (two 32-bit
+ *   words), and is kept when the word is >= floor(p·2^32); 0 <= p < 1, p = 0
+ *   disables dropout.  keep_out [M,h] uint8 (nullable) receives the mask.
+ *   x, residual, gamma, beta bf16; bias [h] bf16 nullable; h % 8 == 0,
+ *   h <= 8192, pointers 16-byte aligned.  The formulas are not printed on
+ *   the pages: this is the transformer's residual step as Megatron writes it.
+ */
+TP_API tp_status tp_sp_dropout_add_ln_fwd(const void* x, const void* bias, const void* residual,
+                                          const void* gamma, const void* beta, int64_t M,
+                                          int64_t h, int32_t N, float p, uint64_t seed,
+                                          uint64_t offset, float eps, void* hs, void* y,
+                                          float* mean, float* rstd, uint8_t* keep_out,
+                                          int32_t* dev_status, void* stream);
+
+/*
+ * Its backward, same passage.  dy [M,h]: gradient at y; dhs_in [M,h]
+ * (nullable): gradient reaching the residual stream hs from later layers.
+ *
+ *   dresidual = rstd·(g − mean(g) − xhat·mean(g·xhat)) + dhs_in,
+ *               g = dy·gamma, xhat = (hs − mean)·rstd      [M,h] bf16 out
+ *   dx        = keep · dresidual / (1 − p)                   [M,h] bf16 out
+ *   dgamma = Σ_rows dy·xhat, dbeta = Σ_rows dy, dbias = Σ_rows dx   [h] fp32
+ *
+ *   The row sums are each shard's partial gradients summed over the shards
+ *   (the sequence-parallel all-reduce), in a fixed order.  keep is
+ *   regenerated from (p, seed, offset), which must be the forward's.
+ *   dbias nullable.  ws, ws_bytes >= tp_workspace_bytes(TP_OP_SP_LN_BWD, M,
+ *   h, h, N).
+ */
+TP_API tp_status tp_sp_dropout_add_ln_bwd(const void* dy, const void* dhs_in, const void* hs,
+                                          const void* gamma, const float* mean, const float* rstd,
+                                          int64_t M, int64_t h, int32_t N, float p, uint64_t seed,
+                                          uint64_t offset, void* dx, void* dresidual,
+                                          float* dgamma, float* dbeta, float* dbias, void* ws,
+                                          size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
  * Output layer and cross-entropy in one pass, without the logits matrix

@@ -29,14 +29,14 @@ __all__ = [
     "vp_embed", "tp_logits_fwd", "vp_xent", "vp_xent_bf16_grad", "tp_logits_bwd", "vp_embed_bwd",
     "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT", "tp_mlp_bwd_recompute",
-    "tp_attention_fwd",
+    "tp_attention_fwd", "tp_sp_dropout_add_ln_fwd", "tp_sp_dropout_add_ln_bwd", "OP_SP_LN_BWD",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
 ACT_NONE, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 (OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD, OP_EMBED_BWD,
- OP_LINEAR_XENT) = range(7)
+ OP_LINEAR_XENT, OP_SP_LN_BWD) = range(8)
 DEVERR_RANGE, DEVERR_TIMEOUT = 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -76,6 +76,10 @@ _SIGS = {
     "tp_linear_xent_fwd": ([_P, _P, _P, _I64, _I64, _I64, _I32, _P, _P, _P, _P, _P, _SZ,
                             _P, _P], _I32),
     "tp_linear_xent_dlogits": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _F, _P, _P, _P], _I32),
+    "tp_sp_dropout_add_ln_fwd": ([_P, _P, _P, _P, _P, _I64, _I64, _I32, _F, ctypes.c_uint64,
+                                  ctypes.c_uint64, _F, _P, _P, _P, _P, _P, _P, _P], _I32),
+    "tp_sp_dropout_add_ln_bwd": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _F, ctypes.c_uint64,
+                                  ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
     "tp_attention_fwd": ([_P, _I64, _I64, _I32, _I32, _I32, _P, _I32, _F, _P, _P, _P, _P], _I32),
     "tp_mlp_bwd_recompute": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                               _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
@@ -495,3 +499,49 @@ def tp_attention_fwd(QKV, b, s, n_heads, N, *, head_offsets=None, causal=True, s
                                   float(scale) if scale else 0.0, _ptr(ctx), _ptr(lse),
                                   _ptr(dev_status), _stream(dev)), "tp_attention_fwd")
     return ctx, lse
+
+
+def tp_sp_dropout_add_ln_fwd(x, bias, residual, gamma, beta, N, *, p=0.0, seed=0, offset=0,
+                             eps=1e-5, with_keep=False, hs=None, y=None, mean=None, rstd=None,
+                             keep=None, dev_status=None):
+    """hs = residual + dropout(x + bias), y = LayerNorm(hs) on N sequence shards.
+
+    Returns dict(hs, y, mean, rstd, keep or None)."""
+    M, h = x.shape
+    dev = x.device
+    hs = torch.empty_like(x) if hs is None else hs
+    y = torch.empty_like(x) if y is None else y
+    mean = torch.empty(M, dtype=torch.float32, device=dev) if mean is None else mean
+    rstd = torch.empty(M, dtype=torch.float32, device=dev) if rstd is None else rstd
+    if with_keep and keep is None:
+        keep = torch.empty(M, h, dtype=torch.uint8, device=dev)
+    _contig(x, bias, residual, gamma, beta, hs, y, mean, rstd, keep)
+    _check(lib().tp_sp_dropout_add_ln_fwd(_ptr(x), _ptr(bias), _ptr(residual), _ptr(gamma),
+                                          _ptr(beta), M, h, N, float(p), int(seed), int(offset),
+                                          float(eps), _ptr(hs), _ptr(y), _ptr(mean), _ptr(rstd),
+                                          _ptr(keep), _ptr(dev_status), _stream(dev)),
+           "tp_sp_dropout_add_ln_fwd")
+    return {"hs": hs, "y": y, "mean": mean, "rstd": rstd, "keep": keep}
+
+
+def tp_sp_dropout_add_ln_bwd(dy, dhs_in, hs, gamma, mean, rstd, N, *, p=0.0, seed=0, offset=0,
+                             with_dbias=True, dx=None, dresidual=None, dgamma=None, dbeta=None,
+                             dbias=None, ws=None, dev_status=None):
+    """Backward of tp_sp_dropout_add_ln_fwd.  Returns dict(dx, dresidual, dgamma, dbeta, dbias)."""
+    M, h = dy.shape
+    dev = dy.device
+    dx = torch.empty_like(dy) if dx is None else dx
+    dresidual = torch.empty_like(dy) if dresidual is None else dresidual
+    dgamma = torch.empty(h, dtype=torch.float32, device=dev) if dgamma is None else dgamma
+    dbeta = torch.empty(h, dtype=torch.float32, device=dev) if dbeta is None else dbeta
+    if with_dbias and dbias is None:
+        dbias = torch.empty(h, dtype=torch.float32, device=dev)
+    _contig(dy, dhs_in, hs, gamma, mean, rstd, dx, dresidual, dgamma, dbeta, dbias)
+    ws, wsb = _workspace(ws, OP_SP_LN_BWD, M, h, h, N, dev)
+    _check(lib().tp_sp_dropout_add_ln_bwd(_ptr(dy), _ptr(dhs_in), _ptr(hs), _ptr(gamma),
+                                          _ptr(mean), _ptr(rstd), M, h, N, float(p), int(seed),
+                                          int(offset), _ptr(dx), _ptr(dresidual), _ptr(dgamma),
+                                          _ptr(dbeta), _ptr(dbias), _ptr(ws), wsb,
+                                          _ptr(dev_status), _stream(dev)),
+           "tp_sp_dropout_add_ln_bwd")
+    return {"dx": dx, "dresidual": dresidual, "dgamma": dgamma, "dbeta": dbeta, "dbias": dbias}

@@ -89,6 +89,18 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
                                const int64_t* head_offsets, int N, bool causal, float scale,
                                void* ctx, float* lse, int32_t* dev_status, cudaStream_t stream);
 
+// Sequence-parallel dropout-add-LayerNorm (layernorm.cu): see
+// tp_sp_dropout_add_ln_fwd / _bwd.  h % 8 == 0, h <= 8192.
+size_t sp_ln_bwd_ws_bytes(int64_t M, int64_t h);
+tp_status sp_ln_fwd_launch(const void* x, const void* bias, const void* residual, const void* gamma,
+                           const void* beta, int64_t M, int64_t h, float p, uint64_t seed,
+                           uint64_t offset, float eps, void* hs, void* y, float* mean, float* rstd,
+                           uint8_t* keep, cudaStream_t stream);
+tp_status sp_ln_bwd_launch(const void* dy, const void* dhs_in, const void* hs, const void* gamma,
+                           const float* mean, const float* rstd, int64_t M, int64_t h, float p,
+                           uint64_t seed, uint64_t offset, void* dx, void* dres, float* dgamma,
+                           float* dbeta, float* dbias, void* ws, cudaStream_t stream);
+
 // Counts every kernel the library enqueues (tp_launch_count).
 void note_launches(int n);
 

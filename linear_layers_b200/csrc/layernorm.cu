@@ -1,0 +1,369 @@
+// layernorm.cu — sequence-parallel dropout-add-LayerNorm for sm_100a.
+//
+// The residual step of the transformer layer, computed by each sequence
+// shard on its own token rows (LayerNorm and Dropout split along the
+// sequence; the parameter gradients are summed over shards):
+//
+//   hs = residual + keep · (x + bias) / (1 − p)        (bf16, the residual stream)
+//   y  = (hs − mean) · rstd · gamma + beta              (bf16)
+//
+// with the mean and the biased variance of each row over the hidden size.
+// keep comes from Philox4x32-10 (Salmon et al., SC 2011), written here from
+// its definition: element e = row·h + col uses word e mod 4 of the block at
+// counter (e div 4, offset) under key seed, and is kept when the word is at
+// least floor(p · 2^32).  The backward regenerates the same words instead of
+// storing the mask.
+//
+// HBM-bound: one 16-byte chunk of 8 elements per access, rows held in
+// registers between the reductions.  The LayerNorm statistics are taken
+// from hs as stored (bf16), so forward and backward see the same values.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cmath>
+
+#include "internal.h"
+
+namespace tpl {
+
+namespace {
+
+constexpr int kLnThreads = 128;            // threads per row (forward) / per block (backward)
+constexpr int kLnBwdRows = 8;              // rows per backward block
+
+struct DropoutRng {
+  uint32_t key_lo, key_hi, off_lo, off_hi;
+  uint32_t threshold;                      // keep when the word >= threshold
+  float inv_keep;                          // 1 / (1 − p)
+};
+
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// Keep bits of the 8 elements starting at element e (e a multiple of 8).
+__device__ __forceinline__ uint32_t keep_bits8(const DropoutRng& g, uint64_t e) {
+  if (g.threshold == 0) return 0xffu;
+  const uint64_t q = e >> 2;
+  const uint4 w0 = philox4x32_10(make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32),
+                                            g.off_lo, g.off_hi), g.key_lo, g.key_hi);
+  const uint4 w1 = philox4x32_10(make_uint4(static_cast<uint32_t>(q + 1),
+                                            static_cast<uint32_t>((q + 1) >> 32), g.off_lo, g.off_hi),
+                                 g.key_lo, g.key_hi);
+  const uint32_t t = g.threshold;
+  return (w0.x >= t ? 1u : 0u) | (w0.y >= t ? 2u : 0u) | (w0.z >= t ? 4u : 0u) |
+         (w0.w >= t ? 8u : 0u) | (w1.x >= t ? 16u : 0u) | (w1.y >= t ? 32u : 0u) |
+         (w1.z >= t ? 64u : 0u) | (w1.w >= t ? 128u : 0u);
+}
+
+__device__ __forceinline__ void unpack8(const uint4& w, float (&v)[8]) {
+  const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    v[2 * q] = __uint_as_float(ww[q] << 16);
+    v[2 * q + 1] = __uint_as_float(ww[q] & 0xffff0000u);
+  }
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&b);
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&v)[8]) {
+  return make_uint4(pack2(v[0], v[1]), pack2(v[2], v[3]), pack2(v[4], v[5]), pack2(v[6], v[7]));
+}
+
+// Sum over the block's threads in a fixed order (warp tree, then warps in order).
+template <int NV>
+__device__ __forceinline__ void block_sum(float (&v)[NV], float (*red)[kLnThreads / 32]) {
+#pragma unroll
+  for (int i = 0; i < NV; ++i)
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v[i] += __shfl_xor_sync(0xffffffffu, v[i], o);
+  const int w = threadIdx.x >> 5;
+  __syncthreads();   // the previous use of red is finished
+  if ((threadIdx.x & 31) == 0)
+#pragma unroll
+    for (int i = 0; i < NV; ++i) red[i][w] = v[i];
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
+    float s = 0.0f;
+#pragma unroll
+    for (int q = 0; q < kLnThreads / 32; ++q) s += red[i][q];
+    v[i] = s;
+  }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ bias, const uint4* __restrict__ residual,
+    const uint4* __restrict__ gamma, const uint4* __restrict__ beta, int h8, float inv_h, float eps,
+    DropoutRng rng, uint4* __restrict__ hs_out, uint4* __restrict__ y_out, float* __restrict__ mean_out,
+    float* __restrict__ rstd_out, uint8_t* __restrict__ keep_out) {
+  __shared__ float red[2][kLnThreads / 32];
+  const int64_t row = blockIdx.x;
+  float hv[CH][8];
+  float s[1] = {0.0f};
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = threadIdx.x + k * kLnThreads;
+    if (c < h8) {
+      const int64_t o = row * h8 + c;
+      float xv[8], rv[8], bv[8];
+      unpack8(__ldcs(x + o), xv);
+      unpack8(__ldcs(residual + o), rv);
+      if (bias) {
+        unpack8(__ldg(bias + c), bv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bv[i] = 0.0f;
+      }
+      const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        t[i] = rv[i] + (((kb >> i) & 1u) ? (xv[i] + bv[i]) * rng.inv_keep : 0.0f);
+      const uint4 packed = pack8(t);
+      __stcs(hs_out + o, packed);
+      if (keep_out)
+        *reinterpret_cast<uint2*>(keep_out + o * 8) = make_uint2(
+            ((kb >> 0) & 1u) | (((kb >> 1) & 1u) << 8) | (((kb >> 2) & 1u) << 16) | (((kb >> 3) & 1u) << 24),
+            ((kb >> 4) & 1u) | (((kb >> 5) & 1u) << 8) | (((kb >> 6) & 1u) << 16) | (((kb >> 7) & 1u) << 24));
+      unpack8(packed, hv[k]);   // the statistics of hs as stored
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s[0] += hv[k][i];
+    }
+  }
+  block_sum<1>(s, red);
+  const float mean = s[0] * inv_h;
+  float q[1] = {0.0f};
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = threadIdx.x + k * kLnThreads;
+    if (c < h8)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float d = hv[k][i] - mean;
+        q[0] = fmaf(d, d, q[0]);
+      }
+  }
+  block_sum<1>(q, red);
+  const float rstd = 1.0f / sqrtf(q[0] * inv_h + eps);
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = threadIdx.x + k * kLnThreads;
+    if (c < h8) {
+      float gv[8], bv[8], yv[8];
+      unpack8(__ldg(gamma + c), gv);
+      unpack8(__ldg(beta + c), bv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) yv[i] = fmaf((hv[k][i] - mean) * rstd, gv[i], bv[i]);
+      __stcs(y_out + row * h8 + c, pack8(yv));
+    }
+  }
+  if (threadIdx.x == 0) {
+    mean_out[row] = mean;
+    rstd_out[row] = rstd;
+  }
+}
+
+// Backward, kLnBwdRows rows per block.  Pass A of a row forms Σ g and
+// Σ g·xhat (g = dy·gamma); pass B reads the row again (from L1) and writes
+// dresidual = rstd·(g − mean(g) − xhat·mean(g·xhat)) + dhs_in and
+// dx = keep·dresidual/(1 − p).  Only the block's column sums of dy·xhat, dy
+// and dx stay in registers across rows; they are written as this block's
+// partial and summed over blocks in block order afterwards.
+template <int CH>
+__global__ void __launch_bounds__(kLnThreads) sp_ln_bwd_kernel(
+    const uint4* __restrict__ dy, const uint4* __restrict__ dhs_in, const uint4* __restrict__ hs,
+    const uint4* __restrict__ gamma, const float* __restrict__ mean, const float* __restrict__ rstd,
+    int64_t M, int h8, float inv_h, DropoutRng rng, uint4* __restrict__ dx,
+    uint4* __restrict__ dresidual, float* __restrict__ part_gamma, float* __restrict__ part_beta,
+    float* __restrict__ part_bias) {
+  __shared__ float red[2][kLnThreads / 32];
+  float ag[CH][8], ab[CH][8], ax[CH][8];   // this block's column sums
+#pragma unroll
+  for (int k = 0; k < CH; ++k)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ag[k][i] = ab[k][i] = ax[k][i] = 0.0f;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kLnBwdRows;
+  for (int rr = 0; rr < kLnBwdRows; ++rr) {
+    const int64_t row = r0 + rr;
+    if (row >= M) break;   // uniform across the block
+    const float mu = mean[row], rs = rstd[row];
+    float sums[2] = {0.0f, 0.0f};   // Σ g, Σ g·xhat
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const int c = threadIdx.x + k * kLnThreads;
+      if (c < h8) {
+        const int64_t o = row * h8 + c;
+        float hv[8], dv[8], gv[8];
+        unpack8(__ldg(hs + o), hv);
+        unpack8(__ldg(dy + o), dv);
+        unpack8(__ldg(gamma + c), gv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float g = dv[i] * gv[i];
+          sums[0] += g;
+          sums[1] = fmaf(g, (hv[i] - mu) * rs, sums[1]);
+        }
+      }
+    }
+    block_sum<2>(sums, red);
+    const float mg = sums[0] * inv_h, mgx = sums[1] * inv_h;
+#pragma unroll
+    for (int k = 0; k < CH; ++k) {
+      const int c = threadIdx.x + k * kLnThreads;
+      if (c < h8) {
+        const int64_t o = row * h8 + c;
+        float hv[8], dv[8], gv[8], din[8], d[8], dxv[8];
+        unpack8(__ldg(hs + o), hv);
+        unpack8(__ldg(dy + o), dv);
+        unpack8(__ldg(gamma + c), gv);
+        if (dhs_in) {
+          unpack8(__ldcs(dhs_in + o), din);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) din[i] = 0.0f;
+        }
+        const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float xh = (hv[i] - mu) * rs;
+          d[i] = fmaf(rs, dv[i] * gv[i] - mg - xh * mgx, din[i]);
+          dxv[i] = ((kb >> i) & 1u) ? d[i] * rng.inv_keep : 0.0f;
+          ag[k][i] = fmaf(dv[i], xh, ag[k][i]);
+          ab[k][i] += dv[i];
+          ax[k][i] += dxv[i];
+        }
+        __stcs(dresidual + o, pack8(d));
+        __stcs(dx + o, pack8(dxv));
+      }
+    }
+  }
+  const int64_t h = static_cast<int64_t>(h8) * 8;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = threadIdx.x + k * kLnThreads;
+    if (c < h8) {
+      float* pg = part_gamma + blockIdx.x * h + c * 8;
+      float* pb = part_beta + blockIdx.x * h + c * 8;
+      *reinterpret_cast<float4*>(pg) = make_float4(ag[k][0], ag[k][1], ag[k][2], ag[k][3]);
+      *reinterpret_cast<float4*>(pg + 4) = make_float4(ag[k][4], ag[k][5], ag[k][6], ag[k][7]);
+      *reinterpret_cast<float4*>(pb) = make_float4(ab[k][0], ab[k][1], ab[k][2], ab[k][3]);
+      *reinterpret_cast<float4*>(pb + 4) = make_float4(ab[k][4], ab[k][5], ab[k][6], ab[k][7]);
+      if (part_bias) {
+        float* px = part_bias + blockIdx.x * h + c * 8;
+        *reinterpret_cast<float4*>(px) = make_float4(ax[k][0], ax[k][1], ax[k][2], ax[k][3]);
+        *reinterpret_cast<float4*>(px + 4) = make_float4(ax[k][4], ax[k][5], ax[k][6], ax[k][7]);
+      }
+    }
+  }
+}
+
+DropoutRng make_rng(float p, uint64_t seed, uint64_t offset) {
+  DropoutRng g;
+  g.key_lo = static_cast<uint32_t>(seed);
+  g.key_hi = static_cast<uint32_t>(seed >> 32);
+  g.off_lo = static_cast<uint32_t>(offset);
+  g.off_hi = static_cast<uint32_t>(offset >> 32);
+  const double t = std::floor(static_cast<double>(p) * 4294967296.0);
+  g.threshold = t >= 4294967295.0 ? 0xffffffffu : static_cast<uint32_t>(t);
+  g.inv_keep = static_cast<float>(1.0 / (1.0 - static_cast<double>(p)));
+  return g;
+}
+
+template <int CH>
+tp_status ln_fwd_t(const void* x, const void* bias, const void* residual, const void* gamma,
+                   const void* beta, int64_t M, int64_t h, const DropoutRng& g, float eps, void* hs,
+                   void* y, float* mean, float* rstd, uint8_t* keep, cudaStream_t stream) {
+  sp_ln_fwd_kernel<CH><<<static_cast<unsigned>(M), kLnThreads, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<const uint4*>(bias),
+      static_cast<const uint4*>(residual), static_cast<const uint4*>(gamma),
+      static_cast<const uint4*>(beta), static_cast<int>(h / 8), 1.0f / static_cast<float>(h), eps, g,
+      static_cast<uint4*>(hs), static_cast<uint4*>(y), mean, rstd, keep);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+template <int CH>
+tp_status ln_bwd_t(const void* dy, const void* dhs_in, const void* hs, const void* gamma,
+                   const float* mean, const float* rstd, int64_t M, int64_t h, const DropoutRng& g,
+                   void* dx, void* dres, float* pg, float* pb, float* px, cudaStream_t stream) {
+  const int64_t blocks = (M + kLnBwdRows - 1) / kLnBwdRows;
+  sp_ln_bwd_kernel<CH><<<static_cast<unsigned>(blocks), kLnThreads, 0, stream>>>(
+      static_cast<const uint4*>(dy), static_cast<const uint4*>(dhs_in),
+      static_cast<const uint4*>(hs), static_cast<const uint4*>(gamma), mean, rstd, M,
+      static_cast<int>(h / 8), 1.0f / static_cast<float>(h), g, static_cast<uint4*>(dx),
+      static_cast<uint4*>(dres), pg, pb, px);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+int chunks_per_thread(int64_t h) {
+  const int64_t c = (h / 8 + kLnThreads - 1) / kLnThreads;
+  return c <= 1 ? 1 : c <= 2 ? 2 : c <= 4 ? 4 : c <= 8 ? 8 : 0;
+}
+
+}  // namespace
+
+size_t sp_ln_bwd_ws_bytes(int64_t M, int64_t h) {
+  const size_t blocks = static_cast<size_t>((M + kLnBwdRows - 1) / kLnBwdRows);
+  const size_t plane = (blocks * static_cast<size_t>(h) * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  return 3 * plane;
+}
+
+tp_status sp_ln_fwd_launch(const void* x, const void* bias, const void* residual, const void* gamma,
+                           const void* beta, int64_t M, int64_t h, float p, uint64_t seed,
+                           uint64_t offset, float eps, void* hs, void* y, float* mean, float* rstd,
+                           uint8_t* keep, cudaStream_t stream) {
+  const DropoutRng g = make_rng(p, seed, offset);
+  switch (chunks_per_thread(h)) {
+    case 1: return ln_fwd_t<1>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+    case 2: return ln_fwd_t<2>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+    case 4: return ln_fwd_t<4>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+    case 8: return ln_fwd_t<8>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+  }
+  return TP_ERR_UNSUPPORTED;
+}
+
+tp_status sp_ln_bwd_launch(const void* dy, const void* dhs_in, const void* hs, const void* gamma,
+                           const float* mean, const float* rstd, int64_t M, int64_t h, float p,
+                           uint64_t seed, uint64_t offset, void* dx, void* dres, float* dgamma,
+                           float* dbeta, float* dbias, void* ws, cudaStream_t stream) {
+  const DropoutRng g = make_rng(p, seed, offset);
+  const int blocks = static_cast<int>((M + kLnBwdRows - 1) / kLnBwdRows);
+  const size_t plane = sp_ln_bwd_ws_bytes(M, h) / 3;
+  float* pg = static_cast<float*>(ws);
+  float* pb = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + plane);
+  float* px = dbias ? reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + 2 * plane) : nullptr;
+  tp_status s;
+  switch (chunks_per_thread(h)) {
+    case 1: s = ln_bwd_t<1>(dy, dhs_in, hs, gamma, mean, rstd, M, h, g, dx, dres, pg, pb, px, stream); break;
+    case 2: s = ln_bwd_t<2>(dy, dhs_in, hs, gamma, mean, rstd, M, h, g, dx, dres, pg, pb, px, stream); break;
+    case 4: s = ln_bwd_t<4>(dy, dhs_in, hs, gamma, mean, rstd, M, h, g, dx, dres, pg, pb, px, stream); break;
+    case 8: s = ln_bwd_t<8>(dy, dhs_in, hs, gamma, mean, rstd, M, h, g, dx, dres, pg, pb, px, stream); break;
+    default: return TP_ERR_UNSUPPORTED;
+  }
+  if (s) return s;
+  // the shards' (blocks') partial parameter gradients summed in block order
+  const int hi = static_cast<int>(h);
+  if ((s = dbias_finish_launch(pg, blocks, hi, dgamma, stream))) return s;
+  if ((s = dbias_finish_launch(pb, blocks, hi, dbeta, stream))) return s;
+  if (dbias) return dbias_finish_launch(px, blocks, hi, dbias, stream);
+  return TP_OK;
+}
+
+}  // namespace tpl

@@ -282,6 +282,8 @@ size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) 
       return align256(embed_bwd_ws_bytes(M));
     case TP_OP_LINEAR_XENT:   // (T, h, v, N): slice statistics + target logits
       return linear_xent_ws_bytes(M, F);
+    case TP_OP_SP_LN_BWD:     // (M, h, h, N): per-block partial parameter gradients
+      return sp_ln_bwd_ws_bytes(M, h);
   }
   return 0;
 }
@@ -634,6 +636,44 @@ tp_status vp_xent_bf16_grad(const float* logits, const int64_t* targets, int64_t
   if (tp_status s = require_sm100()) return s;
   return vp_xent_launch(logits, targets, T, v, N, grad_scale, loss, loss_sum, dlogits, true, argmax,
                         dev_status, as_stream(stream));
+}
+
+tp_status tp_sp_dropout_add_ln_fwd(const void* x, const void* bias, const void* residual,
+                                   const void* gamma, const void* beta, int64_t M, int64_t h,
+                                   int32_t N, float p, uint64_t seed, uint64_t offset, float eps,
+                                   void* hs, void* y, float* mean, float* rstd, uint8_t* keep_out,
+                                   int32_t* dev_status, void* stream) {
+  (void)dev_status;
+  if (!x || !residual || !gamma || !beta || !hs || !y || !mean || !rstd) return TP_ERR_NULL;
+  if (!dims_ok({M, h}) || N < 1 || M % N) return TP_ERR_SHAPE;
+  if (!(p >= 0.0f && p < 1.0f) || !(eps > 0.0f)) return TP_ERR_SHAPE;
+  if (h % 8 || h > 8192) return h % 8 ? TP_ERR_ALIGN : TP_ERR_UNSUPPORTED;
+  if (!ptrs_aligned({x, bias, residual, gamma, beta, hs, y}) ||
+      (reinterpret_cast<uintptr_t>(keep_out) & 7))
+    return TP_ERR_ALIGN;
+  if (tp_status st = require_sm100()) return st;
+  return sp_ln_fwd_launch(x, bias, residual, gamma, beta, M, h, p, seed, offset, eps, hs, y, mean,
+                          rstd, keep_out, as_stream(stream));
+}
+
+tp_status tp_sp_dropout_add_ln_bwd(const void* dy, const void* dhs_in, const void* hs,
+                                   const void* gamma, const float* mean, const float* rstd,
+                                   int64_t M, int64_t h, int32_t N, float p, uint64_t seed,
+                                   uint64_t offset, void* dx, void* dresidual, float* dgamma,
+                                   float* dbeta, float* dbias, void* ws, size_t ws_bytes,
+                                   int32_t* dev_status, void* stream) {
+  (void)dev_status;
+  if (!dy || !hs || !gamma || !mean || !rstd || !dx || !dresidual || !dgamma || !dbeta)
+    return TP_ERR_NULL;
+  if (!dims_ok({M, h}) || N < 1 || M % N) return TP_ERR_SHAPE;
+  if (!(p >= 0.0f && p < 1.0f)) return TP_ERR_SHAPE;
+  if (h % 8 || h > 8192) return h % 8 ? TP_ERR_ALIGN : TP_ERR_UNSUPPORTED;
+  if (!ptrs_aligned({dy, dhs_in, hs, gamma, dx, dresidual, dgamma, dbeta, dbias, ws}))
+    return TP_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < sp_ln_bwd_ws_bytes(M, h)) return TP_ERR_WORKSPACE;
+  if (tp_status st = require_sm100()) return st;
+  return sp_ln_bwd_launch(dy, dhs_in, hs, gamma, mean, rstd, M, h, p, seed, offset, dx, dresidual,
+                          dgamma, dbeta, dbias, ws, as_stream(stream));
 }
 
 tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t n_heads,
