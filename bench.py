@@ -442,24 +442,45 @@ def _e2e_mlp(tpl, torch, g, dev, steps, keys=E2E_DATA):
     return ms, h2d, d2h
 
 
-def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world):
-    """Average ms per part over nsteps iterations of plist (2 untimed first),
-    CUDA events on the launching stream, max over ranks."""
+def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world, reps=10):
+    """Average ms per call of each part in plist, max over ranks.
+
+    Each part is captured into a CUDA graph of `reps` back-to-back calls and
+    the graph is replayed `nsteps` times between two CUDA events, so host
+    launch overhead cannot leave the GPU idle inside the timed interval (it
+    would for parts of a few tens of microseconds).  Parts that cannot be
+    captured are timed as a plain loop of calls instead."""
     for _ in range(2):
         for p in plist:
             fns[p]()
     torch.cuda.synchronize(dev)
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(plist) + 1)]
-          for _ in range(nsteps)]
-    for s in range(nsteps):
-        ev[s][0].record(stream)
-        for i, p in enumerate(plist):
-            fns[p]()
-            ev[s][i + 1].record(stream)
-    torch.cuda.synchronize(dev)
+    ms = []
+    for p in plist:
+        try:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for _ in range(reps):
+                    fns[p]()
+            graph.replay()
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(nsteps):
+                graph.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(e0.elapsed_time(e1) / (nsteps * reps))
+            del graph
+        except RuntimeError:
+            torch.cuda.synchronize(dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(nsteps):
+                fns[p]()
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            ms.append(e0.elapsed_time(e1) / nsteps)
     assert int(st.item()) == 0, f"device status {int(st.item())}"
-    ms = [sum(ev[s][i].elapsed_time(ev[s][i + 1]) for s in range(nsteps)) / nsteps
-          for i in range(len(plist))]
     t = torch.tensor(ms, dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)

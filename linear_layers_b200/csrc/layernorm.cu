@@ -107,7 +107,7 @@ __device__ __forceinline__ void block_sum(float (&v)[NV], float (*red)[kLnThread
 }
 
 template <int CH>
-__global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_kernel(
+__global__ void __launch_bounds__(kLnThreads, CH <= 2 ? 8 : 4) sp_ln_fwd_kernel(
     const uint4* __restrict__ x, const uint4* __restrict__ bias, const uint4* __restrict__ residual,
     const uint4* __restrict__ gamma, const uint4* __restrict__ beta, int h8, float inv_h, float eps,
     DropoutRng rng, uint4* __restrict__ hs_out, uint4* __restrict__ y_out, float* __restrict__ mean_out,
@@ -273,6 +273,41 @@ __global__ void __launch_bounds__(kLnThreads) sp_ln_bwd_kernel(
   }
 }
 
+// out_p[n] = Σ_t part_p[t, n] for the planes p = blockIdx.y, in a fixed
+// order: 32 columns per block, 32 row groups of 32 threads; group q sums
+// rows q, q+32, … (four loads in flight), then the 32 group sums are added
+// in group order.
+struct ColumnSums {
+  const float* part[3];
+  float* out[3];
+};
+
+__global__ void __launch_bounds__(1024) column_sums_kernel(ColumnSums cs, int rows, int n) {
+  __shared__ float red[32][33];
+  const float* part = cs.part[blockIdx.y];
+  const int col = blockIdx.x * 32 + (threadIdx.x & 31);
+  const int q = threadIdx.x >> 5;
+  float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+  if (col < n) {
+    int t = q;
+    for (; t + 96 < rows; t += 128) {
+      s0 += part[static_cast<int64_t>(t) * n + col];
+      s1 += part[static_cast<int64_t>(t + 32) * n + col];
+      s2 += part[static_cast<int64_t>(t + 64) * n + col];
+      s3 += part[static_cast<int64_t>(t + 96) * n + col];
+    }
+    for (; t < rows; t += 32) s0 += part[static_cast<int64_t>(t) * n + col];
+  }
+  red[q][threadIdx.x & 31] = (s0 + s1) + (s2 + s3);
+  __syncthreads();
+  if (q == 0 && col < n) {
+    float s = 0.0f;
+#pragma unroll
+    for (int g = 0; g < 32; ++g) s += red[g][threadIdx.x];
+    cs.out[blockIdx.y][col] = s;
+  }
+}
+
 DropoutRng make_rng(float p, uint64_t seed, uint64_t offset) {
   DropoutRng g;
   g.key_lo = static_cast<uint32_t>(seed);
@@ -360,10 +395,13 @@ tp_status sp_ln_bwd_launch(const void* dy, const void* dhs_in, const void* hs, c
   if (s) return s;
   // the shards' (blocks') partial parameter gradients summed in block order
   const int hi = static_cast<int>(h);
-  if ((s = dbias_finish_launch(pg, blocks, hi, dgamma, stream))) return s;
-  if ((s = dbias_finish_launch(pb, blocks, hi, dbeta, stream))) return s;
-  if (dbias) return dbias_finish_launch(px, blocks, hi, dbias, stream);
-  return TP_OK;
+  ColumnSums cs;
+  cs.part[0] = pg; cs.part[1] = pb; cs.part[2] = px;
+  cs.out[0] = dgamma; cs.out[1] = dbeta; cs.out[2] = dbias;
+  column_sums_kernel<<<dim3(static_cast<unsigned>((hi + 31) / 32), dbias ? 3u : 2u), 1024, 0,
+                       stream>>>(cs, blocks, hi);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 }  // namespace tpl
