@@ -32,21 +32,22 @@ constexpr int kLnThreads = 128;            // threads per row (forward) / per bl
 constexpr int kLnBwdRows = 8;              // rows per backward block
 
 struct DropoutRng {
-  uint32_t key_lo, key_hi, off_lo, off_hi;
+  uint32_t rk[10][2];                      // the key of each of the 10 rounds
+  uint32_t off_lo, off_hi;
   uint32_t threshold;                      // keep when the word >= threshold
   float inv_keep;                          // 1 / (1 − p)
 };
 
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+// Philox4x32-10 with the round keys (key + r·(0x9E3779B9, 0xBB67AE85))
+// precomputed on the host: per round two 32 x 32 -> 64-bit products and two
+// three-way XORs.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const DropoutRng& g) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    if (r) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    c = make_uint4(static_cast<uint32_t>(p1 >> 32) ^ c.y ^ g.rk[r][0], static_cast<uint32_t>(p1),
+                   static_cast<uint32_t>(p0 >> 32) ^ c.w ^ g.rk[r][1], static_cast<uint32_t>(p0));
   }
   return c;
 }
@@ -56,10 +57,10 @@ __device__ __forceinline__ uint32_t keep_bits8(const DropoutRng& g, uint64_t e) 
   if (g.threshold == 0) return 0xffu;
   const uint64_t q = e >> 2;
   const uint4 w0 = philox4x32_10(make_uint4(static_cast<uint32_t>(q), static_cast<uint32_t>(q >> 32),
-                                            g.off_lo, g.off_hi), g.key_lo, g.key_hi);
+                                            g.off_lo, g.off_hi), g);
   const uint4 w1 = philox4x32_10(make_uint4(static_cast<uint32_t>(q + 1),
                                             static_cast<uint32_t>((q + 1) >> 32), g.off_lo, g.off_hi),
-                                 g.key_lo, g.key_hi);
+                                 g);
   const uint32_t t = g.threshold;
   return (w0.x >= t ? 1u : 0u) | (w0.y >= t ? 2u : 0u) | (w0.z >= t ? 4u : 0u) |
          (w0.w >= t ? 8u : 0u) | (w1.x >= t ? 16u : 0u) | (w1.y >= t ? 32u : 0u) |
@@ -186,7 +187,7 @@ __global__ void __launch_bounds__(kLnThreads, CH <= 2 ? 8 : 4) sp_ln_fwd_kernel(
 // and dx stay in registers across rows; they are written as this block's
 // partial and summed over blocks in block order afterwards.
 template <int CH>
-__global__ void __launch_bounds__(kLnThreads) sp_ln_bwd_kernel(
+__global__ void __launch_bounds__(kLnThreads, CH == 1 ? 8 : CH == 2 ? 5 : CH == 4 ? 3 : 1) sp_ln_bwd_kernel(
     const uint4* __restrict__ dy, const uint4* __restrict__ dhs_in, const uint4* __restrict__ hs,
     const uint4* __restrict__ gamma, const float* __restrict__ mean, const float* __restrict__ rstd,
     int64_t M, int h8, float inv_h, DropoutRng rng, uint4* __restrict__ dx,
@@ -310,8 +311,13 @@ __global__ void __launch_bounds__(1024) column_sums_kernel(ColumnSums cs, int ro
 
 DropoutRng make_rng(float p, uint64_t seed, uint64_t offset) {
   DropoutRng g;
-  g.key_lo = static_cast<uint32_t>(seed);
-  g.key_hi = static_cast<uint32_t>(seed >> 32);
+  uint32_t k0 = static_cast<uint32_t>(seed), k1 = static_cast<uint32_t>(seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    g.rk[r][0] = k0;
+    g.rk[r][1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
   g.off_lo = static_cast<uint32_t>(offset);
   g.off_hi = static_cast<uint32_t>(offset >> 32);
   const double t = std::floor(static_cast<double>(p) * 4294967296.0);
