@@ -574,11 +574,13 @@ def run_gpu(args):
     total_ms = float(times[0])
     part_ms = {p: float(times[i + 1]) for i, p in enumerate(parts)}
     if not full:   # a partial run (profiling): report the part times only
+        graphed = _side_loop(torch, fns, parts, max(args.steps, 5), stream, dev, st, world)
         if rank == 0:
             print(json.dumps({"partial_run": True, "parts": parts, "vocab_tokens": VOC["T"],
                               "steps": args.steps, "warmup": args.warmup,
                               "parts_ms_per_step": {p: round(part_ms[p] / args.steps, 4)
                                                     for p in parts},
+                              "parts_ms_graph_replay": {p: round(graphed[p], 4) for p in parts},
                               "gpu_launches": int(launches)}), flush=True)
         if world > 1:
             torch.distributed.barrier()
