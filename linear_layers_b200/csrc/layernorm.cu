@@ -180,6 +180,88 @@ __global__ void __launch_bounds__(kLnThreads, CH <= 2 ? 8 : 4) sp_ln_fwd_kernel(
   }
 }
 
+// Warp-wide sum in a fixed order (xor butterfly: every lane ends with the
+// same value).
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Forward for rows of up to 32·CH chunks (h <= 2048): one warp per row, four
+// rows per block, the row in registers and both reductions by shuffles, so
+// no block barrier stands between a row's loads and its stores.
+template <int CH>
+__global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ bias, const uint4* __restrict__ residual,
+    const uint4* __restrict__ gamma, const uint4* __restrict__ beta, int64_t M, int h8,
+    float inv_h, float eps, DropoutRng rng, uint4* __restrict__ hs_out, uint4* __restrict__ y_out,
+    float* __restrict__ mean_out, float* __restrict__ rstd_out, uint8_t* __restrict__ keep_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * (kLnThreads / 32) + (threadIdx.x >> 5);
+  if (row >= M) return;   // whole warps only
+  float hv[CH][8];
+  float s = 0.0f;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = lane + 32 * k;
+    if (c < h8) {
+      const int64_t o = row * h8 + c;
+      float xv[8], rv[8], bv[8];
+      unpack8(__ldcs(x + o), xv);
+      unpack8(__ldcs(residual + o), rv);
+      if (bias) {
+        unpack8(__ldg(bias + c), bv);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) bv[i] = 0.0f;
+      }
+      const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+      float t[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        t[i] = rv[i] + (((kb >> i) & 1u) ? (xv[i] + bv[i]) * rng.inv_keep : 0.0f);
+      const uint4 packed = pack8(t);
+      __stcs(hs_out + o, packed);
+      if (keep_out)
+        *reinterpret_cast<uint2*>(keep_out + o * 8) = make_uint2(
+            ((kb >> 0) & 1u) | (((kb >> 1) & 1u) << 8) | (((kb >> 2) & 1u) << 16) | (((kb >> 3) & 1u) << 24),
+            ((kb >> 4) & 1u) | (((kb >> 5) & 1u) << 8) | (((kb >> 6) & 1u) << 16) | (((kb >> 7) & 1u) << 24));
+      unpack8(packed, hv[k]);   // the statistics of hs as stored
+#pragma unroll
+      for (int i = 0; i < 8; ++i) s += hv[k][i];
+    }
+  }
+  const float mean = warp_sum(s) * inv_h;
+  float q = 0.0f;
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    if (lane + 32 * k < h8)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float d = hv[k][i] - mean;
+        q = fmaf(d, d, q);
+      }
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(q) * inv_h + eps);
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = lane + 32 * k;
+    if (c < h8) {
+      float gv[8], bv[8], yv[8];
+      unpack8(__ldg(gamma + c), gv);
+      unpack8(__ldg(beta + c), bv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) yv[i] = fmaf((hv[k][i] - mean) * rstd, gv[i], bv[i]);
+      __stcs(y_out + row * h8 + c, pack8(yv));
+    }
+  }
+  if (lane == 0) {
+    mean_out[row] = mean;
+    rstd_out[row] = rstd;
+  }
+}
+
 // Backward, kLnBwdRows rows per block.  Pass A of a row forms Σ g and
 // Σ g·xhat (g = dy·gamma); pass B reads the row again (from L1) and writes
 // dresidual = rstd·(g − mean(g) − xhat·mean(g·xhat)) + dhs_in and
@@ -366,11 +448,33 @@ size_t sp_ln_bwd_ws_bytes(int64_t M, int64_t h) {
   return 3 * plane;
 }
 
+template <int CH>
+tp_status ln_fwd_warp_t(const void* x, const void* bias, const void* residual, const void* gamma,
+                        const void* beta, int64_t M, int64_t h, const DropoutRng& g, float eps,
+                        void* hs, void* y, float* mean, float* rstd, uint8_t* keep,
+                        cudaStream_t stream) {
+  constexpr int rows = kLnThreads / 32;
+  sp_ln_fwd_warp_kernel<CH><<<static_cast<unsigned>((M + rows - 1) / rows), kLnThreads, 0, stream>>>(
+      static_cast<const uint4*>(x), static_cast<const uint4*>(bias),
+      static_cast<const uint4*>(residual), static_cast<const uint4*>(gamma),
+      static_cast<const uint4*>(beta), M, static_cast<int>(h / 8), 1.0f / static_cast<float>(h), eps,
+      g, static_cast<uint4*>(hs), static_cast<uint4*>(y), mean, rstd, keep);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
 tp_status sp_ln_fwd_launch(const void* x, const void* bias, const void* residual, const void* gamma,
                            const void* beta, int64_t M, int64_t h, float p, uint64_t seed,
                            uint64_t offset, float eps, void* hs, void* y, float* mean, float* rstd,
                            uint8_t* keep, cudaStream_t stream) {
   const DropoutRng g = make_rng(p, seed, offset);
+  const int64_t h8 = h / 8;
+  if (h8 <= 32 * 2)
+    return ln_fwd_warp_t<2>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+  if (h8 <= 32 * 4)
+    return ln_fwd_warp_t<4>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
+  if (h8 <= 32 * 8)
+    return ln_fwd_warp_t<8>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
   switch (chunks_per_thread(h)) {
     case 1: return ln_fwd_t<1>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
     case 2: return ln_fwd_t<2>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
