@@ -167,12 +167,17 @@ __device__ __forceinline__ float act_deriv_value(float u, int act, float& y) {
 // tile scheduling: unit -> (tile row, tile column, split)
 // Tiles are visited in bands of group_m tile rows, column by column inside a
 // band, so that one wave of CTAs shares A rows and B columns through L2.
-// The splits of one tile are adjacent units, so their partials meet in L2.
+// Split-major: every tile's first K range, then every tile's second, … so a
+// wave reads one K range of its operands (a third less L2 footprint than
+// running a tile's splits side by side; about 1 % faster for the K = 16384
+// row-parallel GEMM of the MLP), and the last split of a tile sums the
+// partials the earlier splits left behind.
 // -------------------------------------------------------------------------
 __device__ __forceinline__ void unit_map(const GemmArgs& a, int unit, int& tm, int& tn, int& s,
                                          int& tile) {
-  s = unit % a.splits;
-  tile = unit / a.splits;
+  const int tiles = a.tiles_m * a.tiles_n;
+  s = unit / tiles;
+  tile = unit - s * tiles;
   const int per_group = a.group_m * a.tiles_n;
   const int g = tile / per_group;
   const int first_m = g * a.group_m;
