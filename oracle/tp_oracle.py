@@ -390,6 +390,53 @@ def attention_sharded(QKV, b, s, n_heads, head_dim, heads_per_shard, causal=True
     return ctx, lse
 
 
+def attention_head_bwd(Q, K, V, dO, causal=True, scale=None):
+    """Gradient of one head of attention_head for the upstream gradient dO.
+
+    With P = softmax(Q·Kᵀ·scale + mask) and O = P·V:
+    dV = Pᵀ·dO,  dP = dO·Vᵀ,  dS = P ⊙ (dP − rowsum(dO ⊙ O)),
+    dQ = scale·dS·K,  dK = scale·dSᵀ·Q.  Returns (dQ, dK, dV)."""
+    Q, K, V, dO = f64(Q), f64(K), f64(V), f64(dO)
+    s, d = Q.shape
+    sc = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+    S = (Q @ K.T) * sc
+    if causal:
+        S = np.where(np.tril(np.ones((s, K.shape[0]), dtype=bool)), S, -np.inf)
+    P = np.exp(S - S.max(axis=1)[:, None])
+    P = P / P.sum(axis=1)[:, None]
+    O = P @ V
+    dV = P.T @ dO
+    dP = dO @ V.T
+    dS = P * (dP - (dO * O).sum(axis=1)[:, None])
+    return sc * dS @ K, sc * dS.T @ Q, dV
+
+
+def attention_sharded_bwd(QKV, dctx, b, s, n_heads, head_dim, heads_per_shard, causal=True,
+                          scale=None):
+    """Backward of attention_sharded: each shard differentiates its own heads
+    with no communication.  Returns dQKV [b·s, 3h] in the same shard-major
+    layout as QKV (the upstream gradient of the column-parallel projection)."""
+    X, G = f64(QKV), f64(dctx)
+    hd = head_dim
+    dX = np.zeros_like(X)
+    col, head = 0, 0
+    for nh in heads_per_shard:
+        q0, k0, v0 = col, col + nh * hd, col + 2 * nh * hd
+        for j in range(nh):
+            cq = slice(q0 + j * hd, q0 + (j + 1) * hd)
+            ck = slice(k0 + j * hd, k0 + (j + 1) * hd)
+            cv = slice(v0 + j * hd, v0 + (j + 1) * hd)
+            co = slice((head + j) * hd, (head + j + 1) * hd)
+            for bb in range(b):
+                rows = slice(bb * s, (bb + 1) * s)
+                dq, dk, dv = attention_head_bwd(X[rows, cq], X[rows, ck], X[rows, cv],
+                                                G[rows, co], causal, scale)
+                dX[rows, cq], dX[rows, ck], dX[rows, cv] = dq, dk, dv
+        col += 3 * nh * hd
+        head += nh
+    return dX
+
+
 # ----------------------------------------------------------------------------
 # Sequence-parallel dropout-add-LayerNorm ([EVO] §2.3: LayerNorm and Dropout
 # split along the sequence, each shard handling its own token rows)

@@ -708,4 +708,36 @@ def check_layernorm_sequence_shards(o):
             assert _rel(s[k], ref[k]) < 1e-14, (N, k)
 
 
+def check_attention_backward_vs_torch(o):
+    """dQ, dK, dV of one head against torch autograd through
+    scaled_dot_product_attention in float64, causal and not; and the sharded
+    backward against autograd through the whole shard-major layout."""
+    import torch
+
+    r = _rng(43)
+    s, d = 7, 4
+    Q, K, V, dO = (r.normal(size=(s, d)) for _ in range(4))
+    for causal in (True, False):
+        for scale in (None, 0.4):
+            T = [torch.from_numpy(x).requires_grad_(True) for x in (Q, K, V)]
+            out = torch.nn.functional.scaled_dot_product_attention(
+                *(t[None, None] for t in T), is_causal=causal, scale=scale)[0, 0]
+            (out * torch.from_numpy(dO)).sum().backward()
+            got = o.attention_head_bwd(Q, K, V, dO, causal, scale)
+            for g, t in zip(got, T):
+                assert _rel(g, t.grad.numpy()) < 1e-13, (causal, scale)
+    b, s2, nh, hd = 2, 5, 3, 4
+    shards = [2, 1]
+    std = r.normal(size=(b * s2, 3 * nh * hd))
+    perm, _ = o.qkv_shard_columns(nh, hd, shards)
+    X = torch.from_numpy(std).requires_grad_(True)
+    t = X.view(b, s2, 3, nh, hd).permute(2, 0, 3, 1, 4)
+    ctx = torch.nn.functional.scaled_dot_product_attention(t[0], t[1], t[2], is_causal=True)
+    ctx = ctx.permute(0, 2, 1, 3).reshape(b * s2, nh * hd)
+    G = r.normal(size=(b * s2, nh * hd))
+    (ctx * torch.from_numpy(G)).sum().backward()
+    got = o.attention_sharded_bwd(std[:, perm], G, b, s2, nh, hd, shards, causal=True)
+    assert _rel(got, X.grad.numpy()[:, perm]) < 1e-13
+
+
 ALL_CHECKS = [v for k, v in sorted(globals().items()) if k.startswith("check_")]

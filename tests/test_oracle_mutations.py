@@ -286,6 +286,23 @@ def _m_layernorm_dgamma_without_xhat(mp):
     mp.setattr(O, "dropout_add_layernorm_bwd", bad)
 
 
+def _m_attention_bwd_drops_rowsum(mp):
+    orig = O.attention_head_bwd
+
+    def bad(Q, K, V, dO, causal=True, scale=None):
+        Qf, Kf, Vf, dOf = O.f64(Q), O.f64(K), O.f64(V), O.f64(dO)
+        s, d = Qf.shape
+        sc = (1.0 / math.sqrt(d)) if scale is None else float(scale)
+        S = (Qf @ Kf.T) * sc
+        if causal:
+            S = np.where(np.tril(np.ones((s, s), dtype=bool)), S, -np.inf)
+        P = np.exp(S - S.max(axis=1)[:, None])
+        P = P / P.sum(axis=1)[:, None]
+        dS = P * (dOf @ Vf.T)                         # dropped − rowsum(dO ⊙ O)
+        return sc * dS @ Kf, sc * dS.T @ Qf, P.T @ dOf
+    mp.setattr(O, "attention_head_bwd", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
