@@ -178,7 +178,7 @@ def _prepare(dev, parts):
     bf = dict(dtype=torch.bfloat16, device=dev)
     if any(p.startswith("mlp") for p in parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
-    if "proj" in parts or "attn_fwd" in parts or "ln_fwd" in parts or "ln_bwd" in parts:
+    if any(p in parts for p in ("proj", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd")):
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
     if any(p in parts for p in ("embed", "logits", "xent", "xent_bf16", "logits_bwd", "embed_bwd",
                                 "lxent_fwd", "lxent_dlogits")):
@@ -214,7 +214,11 @@ def _prepare_proj(dev, tpl, tp_inputs, torch, bf):
     pr.update(QKV=torch.empty(Mp, 3 * hp, **bf), dXq=torch.empty(Mp, hp, **bf),
               dWq=torch.empty(hp, 3 * hp, **bf), dbq=torch.empty(3 * hp, dtype=torch.float32, device=dev),
               Zo=torch.zeros(Mp, hp, **bf), dctx=torch.zeros(Mp, hp, **bf), dWo=torch.empty(hp, hp, **bf),
-              ctx_attn=torch.empty(Mp, hp, **bf))
+              ctx_attn=torch.empty(Mp, hp, **bf),
+              attn_lse=torch.empty(Mp // 1024, PROJ["n_heads"], 1024, dtype=torch.float32, device=dev),
+              dqkv_attn=torch.empty(Mp, 3 * hp, **bf),
+              attn_ws=torch.empty(tpl.tp_workspace_bytes(tpl.OP_ATTENTION_BWD, Mp, PROJ["n_heads"], 64,
+                                                         PROJ["N"]), dtype=torch.uint8, device=dev))
     # the residual step after the output projection: hs = X + dropout(Zo + b), y = LN(hs)
     gl = torch.Generator().manual_seed(5)
     pr.update(ln_bias=(0.1 * torch.randn(hp, generator=gl)).to(**bf),
@@ -322,7 +326,13 @@ def _mlp_bwd_rc(tpl, g, st):
 
 def _attn_fwd(tpl, pr, st):
     tpl.tp_attention_fwd(pr["QKV"], PROJ["M"] // 1024, 1024, PROJ["n_heads"], PROJ["N"],
-                         causal=True, ctx=pr["ctx_attn"], dev_status=st)
+                         causal=True, ctx=pr["ctx_attn"], lse=pr["attn_lse"], dev_status=st)
+
+
+def _attn_bwd(tpl, pr, st):
+    tpl.tp_attention_bwd(pr["QKV"], pr["ctx_attn"], pr["dZ"], pr["attn_lse"], PROJ["M"] // 1024,
+                         1024, PROJ["n_heads"], PROJ["N"], causal=True, dQKV=pr["dqkv_attn"],
+                         ws=pr["attn_ws"], dev_status=st)
 
 
 LN_P, LN_SEED = 0.1, 1234
@@ -366,7 +376,7 @@ FUSED_PARTS = ("lxent_fwd", "lxent_dlogits")
 # the MLP backward with activation recompute (Y rebuilt from U), own loop
 RECOMPUTE_PARTS = ("mlp_bwd_rc",)
 # the attention core between the projections (b=4, s=1024, causal), own loop
-ATTN_PARTS = ("attn_fwd",)
+ATTN_PARTS = ("attn_fwd", "attn_bwd")
 # sequence-parallel dropout-add-LayerNorm after the output projection, own loop
 LN_PARTS = ("ln_fwd", "ln_bwd")
 
@@ -532,6 +542,7 @@ def run_gpu(args):
            "lxent_dlogits": lambda: _lxent_dlogits(tpl, vo, st),
            "mlp_bwd_rc": lambda: _mlp_bwd_rc(tpl, g, st),
            "attn_fwd": lambda: _attn_fwd(tpl, pr, st),
+           "attn_bwd": lambda: _attn_bwd(tpl, pr, st),
            "ln_fwd": lambda: _ln_fwd(tpl, pr, st),
            "ln_bwd": lambda: _ln_bwd(tpl, pr, st)}
     stream = torch.cuda.current_stream(dev)
@@ -685,6 +696,10 @@ def run_gpu(args):
                         "over 4 shards (7/6/6/6); own loop of %d iterations" % side_steps,
                 "us": round(at_ms["attn_fwd"] * 1e3, 2),
                 "tflops": round(ATTN_FLOP / (at_ms["attn_fwd"] / 1e3) / 1e12, 1),
+                "bwd_us": round(at_ms["attn_bwd"] * 1e3, 2),
+                "bwd_tflops": round(2.5 * ATTN_FLOP / (at_ms["attn_bwd"] / 1e3) / 1e12, 1),
+                "bwd_flop_note": "2.5x the forward's: Sᵀ, dPᵀ, dV, dK in one kernel and S, dP, dQ "
+                                 "in the other (7 products of which 5 are the algorithmic ones)",
                 "flop_note": "4·b·heads·d·s(s+1)/2 (the unmasked half of Q·Kᵀ and P·V)",
             },
             "sp_layernorm": {

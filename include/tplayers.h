@@ -94,7 +94,8 @@ typedef enum {
   TP_OP_ROW_LINEAR_BWD = 4,
   TP_OP_EMBED_BWD = 5,    /* pass (T, h, v, N): T tokens */
   TP_OP_LINEAR_XENT = 6,  /* pass (T, h, v, N) */
-  TP_OP_SP_LN_BWD = 7     /* pass (M, h, h, N): M token rows of width h */
+  TP_OP_SP_LN_BWD = 7,    /* pass (M, h, h, N): M token rows of width h */
+  TP_OP_ATTENTION_BWD = 8 /* pass (b·s, n_heads, 64, N) */
 } tp_op;
 
 /*
@@ -408,6 +409,31 @@ TP_API tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t
                                   int32_t head_dim, int32_t N, const int64_t* head_offsets,
                                   int32_t causal, float scale, void* ctx, float* lse,
                                   int32_t* dev_status, void* stream);
+
+/*
+ * Backward of the attention core, per-shard heads   [MLP-TP] §2.2;
+ * [TP-ILL] §3.1 (each shard differentiates its own heads; no communication).
+ *
+ *   For every sequence and head, with P = softmax(Q·Kᵀ·scale + mask) and
+ *   dO the gradient at the context:
+ *     dV = Pᵀ·dO,  dS = P ⊙ (dO·Vᵀ − rowsum(dO ⊙ O)),
+ *     dQ = scale·dS·K,  dK = scale·dSᵀ·Q,
+ *   written into dQKV [b·s, 3·n_heads·64] bf16 in the same shard-major layout
+ *   as QKV (the upstream gradient of the column-parallel projection).
+ *
+ *   QKV as in tp_attention_fwd; ctx [b·s, n_heads·64] bf16 its output O;
+ *   dctx the same shape, the gradient dO; lse [b, n_heads, s] fp32 from
+ *   tp_attention_fwd.  causal, scale and head_offsets must be the forward's.
+ *   Every gradient row is produced by one CTA (one kernel for dK and dV per
+ *   key tile, one for dQ per query tile), so the result is reproducible.
+ *   ws, ws_bytes >= tp_workspace_bytes(TP_OP_ATTENTION_BWD, b·s, n_heads,
+ *   64, N) (rowsum(dO ⊙ O) per query and head).  head_dim 64, n_heads <= 256.
+ */
+TP_API tp_status tp_attention_bwd(const void* QKV, const void* ctx, const void* dctx,
+                                  const float* lse, int64_t b, int64_t s, int32_t n_heads,
+                                  int32_t head_dim, int32_t N, const int64_t* head_offsets,
+                                  int32_t causal, float scale, void* dQKV, void* ws,
+                                  size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
  * Sequence-parallel dropout-add-LayerNorm   [EVO] Megatron history page §2.3

@@ -30,13 +30,14 @@ __all__ = [
     "OP_EMBED_BWD", "new_status", "DEVERR_RANGE", "DEVERR_TIMEOUT",
     "tp_linear_xent_fwd", "tp_linear_xent_dlogits", "OP_LINEAR_XENT", "tp_mlp_bwd_recompute",
     "tp_attention_fwd", "tp_sp_dropout_add_ln_fwd", "tp_sp_dropout_add_ln_bwd", "OP_SP_LN_BWD",
+    "tp_attention_bwd", "OP_ATTENTION_BWD",
     "OP_MLP_FWD", "OP_MLP_BWD", "OP_ROW_LINEAR_FWD", "OP_COL_LINEAR_BWD", "OP_ROW_LINEAR_BWD",
 ]
 
 ACT_NONE, ACT_GELU_TANH, ACT_GELU_ERF = 0, 1, 2
 DTYPE_BF16, DTYPE_F32 = 0, 1
 (OP_MLP_FWD, OP_MLP_BWD, OP_ROW_LINEAR_FWD, OP_COL_LINEAR_BWD, OP_ROW_LINEAR_BWD, OP_EMBED_BWD,
- OP_LINEAR_XENT, OP_SP_LN_BWD) = range(8)
+ OP_LINEAR_XENT, OP_SP_LN_BWD, OP_ATTENTION_BWD) = range(9)
 DEVERR_RANGE, DEVERR_TIMEOUT = 1, 2
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -80,6 +81,8 @@ _SIGS = {
                                   ctypes.c_uint64, _F, _P, _P, _P, _P, _P, _P, _P], _I32),
     "tp_sp_dropout_add_ln_bwd": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I32, _F, ctypes.c_uint64,
                                   ctypes.c_uint64, _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
+    "tp_attention_bwd": ([_P, _P, _P, _P, _I64, _I64, _I32, _I32, _I32, _P, _I32, _F, _P, _P, _SZ,
+                          _P, _P], _I32),
     "tp_attention_fwd": ([_P, _I64, _I64, _I32, _I32, _I32, _P, _I32, _F, _P, _P, _P, _P], _I32),
     "tp_mlp_bwd_recompute": ([_P, _P, _P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                               _P, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
@@ -545,3 +548,19 @@ def tp_sp_dropout_add_ln_bwd(dy, dhs_in, hs, gamma, mean, rstd, N, *, p=0.0, see
                                           _ptr(dev_status), _stream(dev)),
            "tp_sp_dropout_add_ln_bwd")
     return {"dx": dx, "dresidual": dresidual, "dgamma": dgamma, "dbeta": dbeta, "dbias": dbias}
+
+
+def tp_attention_bwd(QKV, ctx, dctx, lse, b, s, n_heads, N, *, head_offsets=None, causal=True,
+                     scale=None, dQKV=None, ws=None, dev_status=None):
+    """Gradient of the attention core with respect to QKV (shard-major layout).
+    lse from tp_attention_fwd(..., with_lse=True).  Returns dQKV."""
+    dev = QKV.device
+    dQKV = torch.empty_like(QKV) if dQKV is None else dQKV
+    _contig(QKV, ctx, dctx, lse, dQKV)
+    offs, keep = _offsets(head_offsets, N)
+    ws, wsb = _workspace(ws, OP_ATTENTION_BWD, b * s, n_heads, 64, N, dev)
+    _check(lib().tp_attention_bwd(_ptr(QKV), _ptr(ctx), _ptr(dctx), _ptr(lse), b, s, n_heads, 64,
+                                  N, offs, 1 if causal else 0, float(scale) if scale else 0.0,
+                                  _ptr(dQKV), _ptr(ws), wsb, _ptr(dev_status), _stream(dev)),
+           "tp_attention_bwd")
+    return dQKV

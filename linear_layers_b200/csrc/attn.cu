@@ -418,6 +418,378 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   }
 }
 
+
+// ===========================================================================
+// Backward.  D = rowsum(dO ⊙ O) first; then two kernels of one template:
+//   kKV = true   one CTA per 128-key tile of a head: streams the query tiles,
+//                Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ in tensor memory, Pᵀ = exp(Sᵀ·scale
+//                − lse) and dSᵀ = Pᵀ ⊙ (dPᵀ − D) per key row, then
+//                dV += Pᵀ·dO and dK += dSᵀ·Q accumulated in tensor memory;
+//   kKV = false  one CTA per 128-query tile: streams the key tiles, S, dP,
+//                P, dS the same way per query row, dQ += dS·K.
+// Each gradient row is produced by exactly one CTA, so there are no atomics
+// and the result does not depend on timing.  dQ and dK carry the scale.
+// ===========================================================================
+constexpr int kBwdThreads = 192;                       // 6 warps
+constexpr uint32_t kBOffF1 = 0;                        // fixed tiles (K, V) or (Q, dO)
+constexpr uint32_t kBOffF2 = kTile;
+constexpr uint32_t kBOffG1 = 2 * kTile;                // streamed tiles, 2 stages each
+constexpr uint32_t kBOffG2 = kBOffG1 + 2 * kTile;
+constexpr uint32_t kBOffP = kBOffG2 + 2 * kTile;       // P (or Pᵀ) bf16: 2 chunks of 64
+constexpr uint32_t kBOffDS = kBOffP + 2 * kTile;       // dS (or dSᵀ) bf16
+constexpr uint32_t kBOffVec = kBOffDS + 2 * kTile;     // per-column lse·log2e and D, 2 stages
+constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * kBQ * 4;
+constexpr int kBNumBars = 10;
+constexpr uint32_t kBOffMisc = kBOffBar + kBNumBars * 8;
+constexpr uint32_t kBAlloc = kBOffMisc + 16 + 1024;
+constexpr uint32_t kTX = 0, kTY = 128, kTA1 = 256, kTA2 = 320;   // tensor memory columns
+
+struct AttnBwdArgs {
+  int b, s, heads, nqb;
+  int causal;
+  float scale, scale_log2;
+  const float* lse;          // [b, heads, s] natural log
+  const float* D;            // [b, heads, s]
+  __nv_bfloat16* dqkv;       // [b·s, 3h], the QKV layout
+  int64_t ldq;               // 3h
+  int32_t* dev_status;
+  uint64_t wait_ns;
+  int2 head_cols[kMaxHeads];
+};
+
+struct __align__(64) AttnBwdParams {
+  CUtensorMap tm_qkv;        // QKV [b·s, 3h], boxes of 64 columns x 128 rows
+  CUtensorMap tm_do;         // dO  [b·s, h],  boxes of 64 columns x 128 rows
+  AttnBwdArgs a;
+};
+
+__global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restrict__ O,
+                                                            const uint4* __restrict__ dO,
+                                                            int64_t rows, int heads, int s,
+                                                            float* __restrict__ D) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (row, head)
+  if (i >= rows * heads) return;
+  const int64_t row = i / heads;
+  const int head = static_cast<int>(i - row * heads);
+  const uint4* o = O + (row * heads + head) * 8;     // 64 bf16 of this head
+  const uint4* g = dO + (row * heads + head) * 8;
+  float acc = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 a = __ldg(o + k), c = __ldg(g + k);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc = fmaf(__uint_as_float(aw[q] << 16), __uint_as_float(cw[q] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[q] & 0xffff0000u), __uint_as_float(cw[q] & 0xffff0000u), acc);
+    }
+  }
+  const int64_t bb = row / s, pos = row - bb * s;
+  D[(bb * heads + head) * s + pos] = acc;
+}
+
+__device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* abort_flag) {
+  if (!*abort_flag) {
+    *abort_flag = 1;
+    if (a.dev_status) atomicOr(a.dev_status, TP_DEVERR_TIMEOUT);
+  }
+}
+
+template <bool kKV>
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const AttnBwdArgs& a = P.a;
+  uint8_t* sF1 = smem + kBOffF1;
+  uint8_t* sF2 = smem + kBOffF2;
+  uint8_t* sG1 = smem + kBOffG1;
+  uint8_t* sG2 = smem + kBOffG2;
+  uint8_t* sP = smem + kBOffP;
+  uint8_t* sDS = smem + kBOffDS;
+  float* vecL = reinterpret_cast<float*>(smem + kBOffVec);   // [2][128]
+  float* vecD = vecL + 2 * kBQ;                               // [2][128]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBOffBar);
+  uint64_t* f_full = bars;
+  uint64_t* g_full = bars + 1;       // [stage]
+  uint64_t* g_empty = bars + 3;      // [stage]
+  uint64_t* xy_full = bars + 5;
+  uint64_t* xy_empty = bars + 6;
+  uint64_t* pd_full = bars + 7;
+  uint64_t* pd_empty = bars + 8;
+  uint64_t* acc_done = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int bh = a.b * a.heads;
+  // fixed tile, longest first: under the causal mask key tile t streams the
+  // query tiles t.., query tile t the key tiles ..t
+  const int ft = kKV ? static_cast<int>(blockIdx.x) / bh
+                     : a.nqb - 1 - static_cast<int>(blockIdx.x) / bh;
+  const int rem = static_cast<int>(blockIdx.x) % bh;
+  const int head = rem / a.b;
+  const int batch = rem % a.b;
+  const int row0 = batch * a.s;
+  // streamed tiles: queries t >= ft (kKV) or keys t <= ft (dQ) under the causal mask
+  const int t_begin = (kKV && a.causal) ? ft : 0;
+  const int t_end = (!kKV && a.causal) ? ft + 1 : a.nqb;
+  const int nt = t_end - t_begin;
+  const int qcol = a.head_cols[head].x;
+  const int kcol = qcol + a.head_cols[head].y;
+  const int vcol = kcol + a.head_cols[head].y;
+  const int ocol = head * kHD;                         // this head's columns of dO
+  // fixed pair: (K, V) or (Q, dO); streamed pair: (Q, dO) or (K, V)
+  const int f1col = kKV ? kcol : qcol, f2col = kKV ? vcol : ocol;
+  const int g1col = kKV ? qcol : kcol, g2col = kKV ? ocol : vcol;
+  const CUtensorMap* f2map = kKV ? &P.tm_qkv : &P.tm_do;
+  const CUtensorMap* g2map = kKV ? &P.tm_do : &P.tm_qkv;
+
+  if (threadIdx.x == 0) {
+    mbar_init(f_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&g_full[i], 1);
+      mbar_init(&g_empty[i], 1);
+    }
+    mbar_init(xy_full, 1);
+    mbar_init(xy_empty, kSoftmaxThreads);
+    mbar_init(pd_full, kSoftmaxThreads);
+    mbar_init(pd_empty, 1);
+    mbar_init(acc_done, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  tc_fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA
+    if (elect_one_sync()) {
+      tma_prefetch_desc(&P.tm_qkv);
+      tma_prefetch_desc(&P.tm_do);
+      mbar_arrive_expect_tx(f_full, 2 * kTile);
+      tma_load_2d(sF1, &P.tm_qkv, f_full, f1col, row0 + ft * kBQ);
+      tma_load_2d(sF2, f2map, f_full, f2col, row0 + ft * kBQ);
+      int issued = 0;
+      for (int it = 0; it < nt; ++it) {
+        const int st = it & 1;
+        if (!mbar_wait_bounded(&g_empty[st], (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u, a.wait_ns,
+                               abort_flag)) {
+          bwd_timeout(a, abort_flag);
+          break;
+        }
+        const int r = row0 + (t_begin + it) * kBQ;
+        mbar_arrive_expect_tx(&g_full[st], 2 * kTile);
+        tma_load_2d(sG1 + st * kTile, &P.tm_qkv, &g_full[st], g1col, r);
+        tma_load_2d(sG2 + st * kTile, g2map, &g_full[st], g2col, r);
+        ++issued;
+      }
+      volatile int keep_waiting = 0;   // every copy lands before the CTA can exit
+      mbar_wait_bounded(f_full, 0, a.wait_ns, &keep_waiting);
+      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
+        mbar_wait_bounded(&g_full[it & 1], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns,
+                          &keep_waiting);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (elect_one_sync()) {
+      constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBQ, false, false);   // both K-major
+      constexpr uint32_t idA = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, G MN-major
+      bool ok = mbar_wait_bounded(f_full, 0, a.wait_ns, abort_flag);
+      bool any = false;
+      const uint32_t f1 = smem_u32(sF1), f2 = smem_u32(sF2);
+      const uint32_t pa = smem_u32(sP), da = smem_u32(sDS);
+      for (int it = 0; ok && it < nt; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = static_cast<uint32_t>(it & 1);
+        if (!mbar_wait_bounded(&g_full[st], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns, abort_flag) ||
+            !mbar_wait_bounded(xy_empty, ph ^ 1u, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t g1 = smem_u32(sG1 + st * kTile), g2 = smem_u32(sG2 + st * kTile);
+#pragma unroll
+        for (int k = 0; k < kHD / 16; ++k) {
+          tc_mma_bf16(tmem + kTX, smem_desc_sw128(f1 + k * 32, 16, 1024),
+                      smem_desc_sw128(g1 + k * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+          tc_mma_bf16(tmem + kTY, smem_desc_sw128(f2 + k * 32, 16, 1024),
+                      smem_desc_sw128(g2 + k * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
+        }
+        any = true;
+        tc_commit(xy_full);
+        if (!mbar_wait_bounded(pd_full, ph, a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+#pragma unroll
+        for (int k = 0; k < kBQ / 16; ++k) {   // K = the streamed tile's 128 rows
+          const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
+          const uint32_t off = (k >> 2) * kTile + (k & 3) * 32;
+          if constexpr (kKV)   // dV += Pᵀ·dO
+            tc_mma_bf16(tmem + kTA1, smem_desc_sw128(pa + off, 16, 1024),
+                        smem_desc_sw128(g2 + k * 2048, 8192, 1024), idA, acc);
+          // dK += dSᵀ·Q  or  dQ += dS·K
+          tc_mma_bf16(tmem + kTA2, smem_desc_sw128(da + off, 16, 1024),
+                      smem_desc_sw128(g1 + k * 2048, 8192, 1024), idA, acc);
+        }
+        tc_commit(pd_empty);
+        tc_commit(&g_empty[st]);
+      }
+      if (!ok) bwd_timeout(a, abort_flag);
+      if (any) tc_commit(acc_done);   // completes once every MMA above has
+      if (!any) mbar_arrive(acc_done);
+    }
+  } else {
+    // ------------------------------------------------------------ element-wise
+    const int qd = warp & 3;
+    const int r = qd * 32 + lane;                  // fixed row = TMEM lane
+    const int fpos = ft * kBQ + r;                 // its position in the sequence
+    const int sbase = (batch * a.heads + head) * a.s;
+    const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
+    const float sl = a.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    // the fixed row's own lse and D (dQ kernel)
+    const float own_l = (!kKV && fpos < a.s) ? a.lse[sbase + fpos] * kLog2e : 0.0f;
+    const float own_d = (!kKV && fpos < a.s) ? a.D[sbase + fpos] : 0.0f;
+    uint8_t* prow = sP + r * 128;
+    uint8_t* drow = sDS + r * 128;
+    const int et = threadIdx.x - 64;               // 0..127
+    bool ok = true;
+    for (int it = 0; it < nt; ++it) {
+      const int st = it & 1;
+      const uint32_t ph = static_cast<uint32_t>(it & 1);
+      const int t0 = (t_begin + it) * kBQ;         // first position of the streamed tile
+      if constexpr (kKV) {   // lse·log2e and D of the streamed queries, one per thread
+        const int q = t0 + et;
+        vecL[st * kBQ + et] = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
+        vecD[st * kBQ + et] = q < a.s ? a.D[sbase + q] : 0.0f;
+        // one barrier per tile that also carries every thread's state, so all
+        // 128 threads leave together and none is left waiting in it
+        ok = __all_sync(0xffffffffu, ok);          // the warp converged for the aligned barrier
+        if (!named_barrier_and(1, kSoftmaxThreads, ok)) {
+          ok = false;
+          break;
+        }
+      }
+      if (!mbar_wait_bounded(xy_full, ph, a.wait_ns, abort_flag) ||
+          !mbar_wait_bounded(pd_empty, ph ^ 1u, a.wait_ns, abort_flag)) {
+        ok = false;
+        if constexpr (kKV) continue;   // leave at the next tile's barrier, with the others
+        break;
+      }
+      tc_fence_after_sync();
+#pragma unroll 1
+      for (int c = 0; c < kBQ / 32; ++c) {
+        uint32_t xr[32], yr[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + kTX + c * 32, xr);
+        tmem_ld_32x32b_x32(tmem + lane_off + kTY + c * 32, yr);
+        tc_wait_ld();
+        float p[32], ds[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int tpos = t0 + c * 32 + j;        // streamed position of this column
+          bool masked;
+          float lcol, dcol;
+          if constexpr (kKV) {   // rows are keys, columns queries
+            masked = tpos >= a.s || (a.causal && tpos < fpos);
+            lcol = vecL[st * kBQ + c * 32 + j];
+            dcol = vecD[st * kBQ + c * 32 + j];
+          } else {               // rows are queries, columns keys
+            masked = tpos >= a.s || (a.causal && tpos > fpos);
+            lcol = own_l;
+            dcol = own_d;
+          }
+          p[j] = masked ? 0.0f : ex2f(fmaf(__uint_as_float(xr[j]), sl, -lcol));
+          ds[j] = p[j] * (__uint_as_float(yr[j]) - dcol);
+        }
+        uint8_t* pch = prow + (c >> 1) * kTile;
+        uint8_t* dch = drow + (c >> 1) * kTile;
+#pragma unroll
+        for (int g4 = 0; g4 < 4; ++g4) {
+          const int gr = (c & 1) * 4 + g4;
+          uint4 w;
+          w.x = pack_bf16x2(p[8 * g4 + 0], p[8 * g4 + 1]);
+          w.y = pack_bf16x2(p[8 * g4 + 2], p[8 * g4 + 3]);
+          w.z = pack_bf16x2(p[8 * g4 + 4], p[8 * g4 + 5]);
+          w.w = pack_bf16x2(p[8 * g4 + 6], p[8 * g4 + 7]);
+          *reinterpret_cast<uint4*>(pch + ((gr ^ (r & 7)) << 4)) = w;
+          w.x = pack_bf16x2(ds[8 * g4 + 0], ds[8 * g4 + 1]);
+          w.y = pack_bf16x2(ds[8 * g4 + 2], ds[8 * g4 + 3]);
+          w.z = pack_bf16x2(ds[8 * g4 + 4], ds[8 * g4 + 5]);
+          w.w = pack_bf16x2(ds[8 * g4 + 6], ds[8 * g4 + 7]);
+          *reinterpret_cast<uint4*>(dch + ((gr ^ (r & 7)) << 4)) = w;
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(xy_empty);
+      fence_proxy_async_smem();
+      mbar_arrive(pd_full);
+    }
+    // the accumulated gradients of the fixed rows
+    const bool done = ok && mbar_wait_bounded<true>(acc_done, 0, a.wait_ns, abort_flag);
+    if (!done) {
+      if (lane == 0) bwd_timeout(a, abort_flag);
+    } else if (fpos < a.s) {
+      tc_fence_after_sync();
+      __nv_bfloat16* dst_row = a.dqkv + static_cast<int64_t>(row0 + fpos) * a.ldq;
+#pragma unroll
+      for (int which = 0; which < (kKV ? 2 : 1); ++which) {
+        // kKV: which 0 -> dK (scaled, acc2), which 1 -> dV (acc1); else dQ (scaled, acc2)
+        const uint32_t col = which == 0 ? kTA2 : kTA1;
+        const float f = which == 0 ? a.scale : 1.0f;
+        __nv_bfloat16* dst = dst_row + (kKV ? (which == 0 ? kcol : vcol) : qcol);
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, rr);
+          tc_wait_ld();
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(rr[8 * g + 0]) * f, __uint_as_float(rr[8 * g + 1]) * f);
+            w.y = pack_bf16x2(__uint_as_float(rr[8 * g + 2]) * f, __uint_as_float(rr[8 * g + 3]) * f);
+            w.z = pack_bf16x2(__uint_as_float(rr[8 * g + 4]) * f, __uint_as_float(rr[8 * g + 5]) * f);
+            w.w = pack_bf16x2(__uint_as_float(rr[8 * g + 6]) * f, __uint_as_float(rr[8 * g + 7]) * f);
+            reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after_sync();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <bool kKV>
+tp_status attn_bwd_launch_t(const AttnBwdParams& prm, int64_t grid, cudaStream_t stream) {
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!configured[dev & 63]) {
+    if (cudaFuncSetAttribute(attn_bwd_kernel<kKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kBAlloc)) != cudaSuccess)
+      return TP_ERR_CUDA;
+    configured[dev & 63] = true;
+  }
+  attn_bwd_kernel<kKV><<<static_cast<unsigned>(grid), kBwdThreads, kBAlloc, stream>>>(prm);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
 }  // namespace
 
 tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
@@ -461,6 +833,56 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
   attn_fwd_kernel<<<static_cast<unsigned>(grid), kAttnThreads, kAttnAlloc, stream>>>(prm);
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+size_t attention_bwd_ws_bytes(int64_t b, int64_t s, int heads) {
+  return (static_cast<size_t>(b * s) * heads * sizeof(float) + 255) & ~static_cast<size_t>(255);
+}
+
+tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, const float* lse,
+                               int64_t b, int64_t s, int heads, const int64_t* head_offsets, int N,
+                               bool causal, float scale, void* dQKV, void* ws, int32_t* dev_status,
+                               cudaStream_t stream) {
+  if (heads > kMaxHeads) return TP_ERR_UNSUPPORTED;
+  float* D = static_cast<float*>(ws);
+  {
+    const int64_t n = b * s * heads;
+    attn_bwd_prep_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
+        static_cast<const uint4*>(O), static_cast<const uint4*>(dO), b * s, heads,
+        static_cast<int>(s), D);
+    note_launches(1);
+    if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  }
+  AttnBwdParams prm;
+  memset(&prm, 0, sizeof(prm));
+  AttnBwdArgs& a = prm.a;
+  a.b = static_cast<int>(b);
+  a.s = static_cast<int>(s);
+  a.heads = heads;
+  a.nqb = static_cast<int>((s + kBQ - 1) / kBQ);
+  a.causal = causal ? 1 : 0;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  a.lse = lse;
+  a.D = D;
+  a.dqkv = static_cast<__nv_bfloat16*>(dQKV);
+  a.ldq = static_cast<int64_t>(3) * heads * kHD;
+  a.dev_status = dev_status;
+  a.wait_ns = wait_limit_ns();
+  for (int i = 0; i < N; ++i) {
+    const int first = static_cast<int>(head_offsets[i]);
+    const int nh = static_cast<int>(head_offsets[i + 1] - head_offsets[i]);
+    for (int hh = 0; hh < nh; ++hh)
+      a.head_cols[first + hh] = make_int2(3 * kHD * first + hh * kHD, nh * kHD);
+  }
+  const uint64_t rows = static_cast<uint64_t>(b * s);
+  const uint64_t ncols = static_cast<uint64_t>(3) * heads * kHD;
+  if (!make_tmap_bf16_sw128(&prm.tm_qkv, QKV, ncols, rows, ncols, kHD, kBQ)) return TP_ERR_CUDA;
+  const uint64_t hcols = static_cast<uint64_t>(heads) * kHD;
+  if (!make_tmap_bf16_sw128(&prm.tm_do, dO, hcols, rows, hcols, kHD, kBQ)) return TP_ERR_CUDA;
+  const int64_t grid = b * heads * a.nqb;
+  if (tp_status st = attn_bwd_launch_t<true>(prm, grid, stream)) return st;
+  return attn_bwd_launch_t<false>(prm, grid, stream);
 }
 
 }  // namespace tpl

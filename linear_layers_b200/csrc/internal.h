@@ -89,6 +89,12 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
                                const int64_t* head_offsets, int N, bool causal, float scale,
                                void* ctx, float* lse, int32_t* dev_status, cudaStream_t stream);
 
+size_t attention_bwd_ws_bytes(int64_t b, int64_t s, int heads);
+tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, const float* lse,
+                               int64_t b, int64_t s, int heads, const int64_t* head_offsets, int N,
+                               bool causal, float scale, void* dQKV, void* ws, int32_t* dev_status,
+                               cudaStream_t stream);
+
 // Sequence-parallel dropout-add-LayerNorm (layernorm.cu): see
 // tp_sp_dropout_add_ln_fwd / _bwd.  h % 8 == 0, h <= 8192.
 size_t sp_ln_bwd_ws_bytes(int64_t M, int64_t h);

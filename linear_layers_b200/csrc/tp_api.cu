@@ -284,6 +284,8 @@ size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) 
       return linear_xent_ws_bytes(M, F);
     case TP_OP_SP_LN_BWD:     // (M, h, h, N): per-block partial parameter gradients
       return sp_ln_bwd_ws_bytes(M, h);
+    case TP_OP_ATTENTION_BWD: // (b·s, n_heads, 64, N): rowsum(dO ⊙ O) per query and head
+      return attention_bwd_ws_bytes(M, 1, static_cast<int>(h));
   }
   return 0;
 }
@@ -699,6 +701,33 @@ tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t n_head
   if (tp_status st = require_sm100()) return st;
   return attention_fwd_launch(QKV, b, s, n_heads, offs.data(), N, causal != 0, scale, ctx, lse,
                               dev_status, as_stream(stream));
+}
+
+tp_status tp_attention_bwd(const void* QKV, const void* ctx, const void* dctx, const float* lse,
+                           int64_t b, int64_t s, int32_t n_heads, int32_t head_dim, int32_t N,
+                           const int64_t* head_offsets, int32_t causal, float scale, void* dQKV,
+                           void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (!QKV || !ctx || !dctx || !lse || !dQKV) return TP_ERR_NULL;
+  if (b <= 0 || s <= 0 || n_heads <= 0 || N < 1 || N > n_heads || b * s > (1ll << 30))
+    return TP_ERR_SHAPE;
+  if (head_dim != 64 || n_heads > 256) return TP_ERR_UNSUPPORTED;
+  if (!ptrs_aligned({QKV, ctx, dctx, dQKV, ws}) || (reinterpret_cast<uintptr_t>(lse) & 3))
+    return TP_ERR_ALIGN;
+  if (ws == nullptr || ws_bytes < attention_bwd_ws_bytes(b, s, n_heads)) return TP_ERR_WORKSPACE;
+  std::vector<int64_t> offs(N + 1);
+  if (head_offsets == nullptr) {
+    offs[0] = 0;
+    for (int i = 0; i < N; ++i) offs[i + 1] = offs[i] + n_heads / N + (i < n_heads % N ? 1 : 0);
+  } else {
+    for (int i = 0; i <= N; ++i) offs[i] = head_offsets[i];
+    if (offs[0] != 0 || offs[N] != n_heads) return TP_ERR_SHAPE;
+    for (int i = 0; i < N; ++i)
+      if (offs[i + 1] <= offs[i]) return TP_ERR_SHAPE;
+  }
+  if (!(scale > 0.0f) || !std::isfinite(scale)) scale = 1.0f / std::sqrt(static_cast<float>(head_dim));
+  if (tp_status st = require_sm100()) return st;
+  return attention_bwd_launch(QKV, ctx, dctx, lse, b, s, n_heads, offs.data(), N, causal != 0,
+                              scale, dQKV, ws, dev_status, as_stream(stream));
 }
 
 tp_status tp_linear_xent_fwd(const void* H, const void* E, const int64_t* targets, int64_t T,

@@ -118,3 +118,61 @@ def test_attention_deterministic():
     c, _ = tpl.tp_attention_fwd(QKV, b, s, nh, 2)
     torch.cuda.synchronize()
     assert torch.equal(a, c)
+
+
+# ---------------------------------------------------------------- backward
+def _bwd_check(b, s, nh, N, causal, seed, offs=None, scale=None):
+    QKV = _qkv(b, s, nh, seed=seed)
+    g = torch.Generator().manual_seed(seed + 1)
+    dctx = torch.randn(b * s, nh * HD, generator=g).bfloat16()
+    st = tpl.new_status()
+    ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, head_offsets=offs, causal=causal,
+                                    scale=scale, with_lse=True, dev_status=st)
+    dQKV = tpl.tp_attention_bwd(QKV.cuda(), ctx, dctx.cuda(), lse, b, s, nh, N, head_offsets=offs,
+                                causal=causal, scale=scale, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    shards = np.diff(offs if offs is not None else _offsets(nh, N)).tolist()
+    ref = O.attention_sharded_bwd(QKV, dctx, b, s, nh, HD, shards, causal=causal, scale=scale)
+    got = f64(dQKV)
+    for bb in range(b):
+        rows = slice(bb * s, (bb + 1) * s)
+        for c0 in range(0, 3 * nh * HD, HD):     # every head's Q, K and V block
+            cols = slice(c0, c0 + HD)
+            assert_close(f"dQKV[b={bb},cols={c0}]", got[rows, cols], ref[rows, cols], TOL_BF16)
+    return dQKV
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("b,s,nh,N", [(2, 200, 5, 3), (1, 128, 2, 2), (3, 37, 4, 1), (1, 1, 1, 1),
+                                      (2, 384, 3, 3)])
+def test_attention_backward_small(b, s, nh, N, causal):
+    _bwd_check(b, s, nh, N, causal, seed=100 + s + nh)
+
+
+def test_attention_backward_offsets_and_scale():
+    _bwd_check(2, 260, 6, 3, True, seed=12, offs=[0, 1, 4, 6], scale=0.05)
+
+
+def test_attention_backward_deterministic():
+    a = _bwd_check(2, 300, 4, 2, True, seed=13)
+    c = _bwd_check(2, 300, 4, 2, True, seed=13)
+    assert torch.equal(a, c)
+
+
+@pytest.mark.slow
+def test_attention_backward_gpt2_slice():
+    """b=4, s=1024, 25 heads over 4 shards: every head of the first sequence
+    against the oracle."""
+    b, s, nh, N = 4, 1024, 25, 4
+    QKV = _qkv(b, s, nh, seed=14)
+    g = torch.Generator().manual_seed(15)
+    dctx = torch.randn(b * s, nh * HD, generator=g).bfloat16()
+    st = tpl.new_status()
+    ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, with_lse=True, dev_status=st)
+    dQKV = tpl.tp_attention_bwd(QKV.cuda(), ctx, dctx.cuda(), lse, b, s, nh, N, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    shards = tp_inputs.head_split(nh, N)
+    ref = O.attention_sharded_bwd(QKV[:s], dctx[:s], 1, s, nh, HD, shards, causal=True)
+    assert_close("dQKV[b=0]", dQKV[:s], ref, TOL_BF16)
