@@ -343,8 +343,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     bool ok = true;
     // O = O·2^(m_{j-2} − m_{j-1}) + P_{j-1}·V_{j-1}
     auto take_o = [&](int jb) -> bool {
-      if (!mbar_wait_bounded(&o_full[g], static_cast<uint32_t>(jb & 1), a.wait_ns,
-                                   abort_flag))
+      // the warp's lanes agree before the warp-collective tensor-memory loads
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[g], static_cast<uint32_t>(jb & 1),
+                                                     a.wait_ns, abort_flag)))
         return false;
       tc_fence_after_sync();
 #pragma unroll
@@ -360,8 +361,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       return true;
     };
     for (int j = 0; j < nk; ++j) {
-      if (!mbar_wait_bounded(&s_full[g], static_cast<uint32_t>(j & 1), a.wait_ns,
-                                   abort_flag)) {
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[g], static_cast<uint32_t>(j & 1),
+                                                     a.wait_ns, abort_flag))) {
         ok = false;
         break;
       }
@@ -680,8 +681,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
           break;
         }
       }
-      if (!mbar_wait_bounded(xy_full, ph, a.wait_ns, abort_flag) ||
-          !mbar_wait_bounded(pd_empty, ph ^ 1u, a.wait_ns, abort_flag)) {
+      // the warp's lanes agree before the warp-collective tensor-memory loads
+      const bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(xy_full, ph, a.wait_ns, abort_flag) &&
+                                      mbar_wait_bounded(pd_empty, ph ^ 1u, a.wait_ns, abort_flag));
+      if (!got) {
         ok = false;
         if constexpr (kKV) continue;   // leave at the next tile's barrier, with the others
         break;
@@ -734,11 +738,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       fence_proxy_async_smem();
       mbar_arrive(pd_full);
     }
-    // the accumulated gradients of the fixed rows
-    const bool done = ok && mbar_wait_bounded<true>(acc_done, 0, a.wait_ns, abort_flag);
+    // the accumulated gradients of the fixed rows: every lane takes part in
+    // the warp-collective tensor-memory loads, only rows inside the sequence
+    // are stored
+    const bool done =
+        __all_sync(0xffffffffu, ok && mbar_wait_bounded<true>(acc_done, 0, a.wait_ns, abort_flag));
     if (!done) {
       if (lane == 0) bwd_timeout(a, abort_flag);
-    } else if (fpos < a.s) {
+    } else {
       tc_fence_after_sync();
       __nv_bfloat16* dst_row = a.dqkv + static_cast<int64_t>(row0 + fpos) * a.ldq;
 #pragma unroll
@@ -759,7 +766,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
             w.y = pack_bf16x2(__uint_as_float(rr[8 * g + 2]) * f, __uint_as_float(rr[8 * g + 3]) * f);
             w.z = pack_bf16x2(__uint_as_float(rr[8 * g + 4]) * f, __uint_as_float(rr[8 * g + 5]) * f);
             w.w = pack_bf16x2(__uint_as_float(rr[8 * g + 6]) * f, __uint_as_float(rr[8 * g + 7]) * f);
-            reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
+            if (fpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
           }
         }
       }
