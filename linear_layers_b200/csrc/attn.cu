@@ -691,29 +691,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
         break;
       }
       tc_fence_after_sync();
+      // the mask can only cut the diagonal tile and the tile past the end
+      const bool need_mask = (a.causal && t_begin + it == ft) || t0 + kBQ > a.s;
 #pragma unroll 1
       for (int c = 0; c < kBQ / 32; ++c) {
         uint32_t xr[32], yr[32];
         tmem_ld_32x32b_x32(tmem + lane_off + kTX + c * 32, xr);
         tmem_ld_32x32b_x32(tmem + lane_off + kTY + c * 32, yr);
+        float lv[32], dv[32];   // per-column lse·log2e and D (the streamed queries)
+        if constexpr (kKV) {
+          const float4* l4 = reinterpret_cast<const float4*>(vecL + st * kBQ + c * 32);
+          const float4* d4 = reinterpret_cast<const float4*>(vecD + st * kBQ + c * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const float4 u = l4[q], w = d4[q];
+            lv[4 * q] = u.x; lv[4 * q + 1] = u.y; lv[4 * q + 2] = u.z; lv[4 * q + 3] = u.w;
+            dv[4 * q] = w.x; dv[4 * q + 1] = w.y; dv[4 * q + 2] = w.z; dv[4 * q + 3] = w.w;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            lv[j] = own_l;
+            dv[j] = own_d;
+          }
+        }
         tc_wait_ld();
         float p[32], ds[32];
+        if (need_mask) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int tpos = t0 + c * 32 + j;        // streamed position of this column
-          bool masked;
-          float lcol, dcol;
-          if constexpr (kKV) {   // rows are keys, columns queries
-            masked = tpos >= a.s || (a.causal && tpos < fpos);
-            lcol = vecL[st * kBQ + c * 32 + j];
-            dcol = vecD[st * kBQ + c * 32 + j];
-          } else {               // rows are queries, columns keys
-            masked = tpos >= a.s || (a.causal && tpos > fpos);
-            lcol = own_l;
-            dcol = own_d;
+          for (int j = 0; j < 32; ++j) {
+            const int tpos = t0 + c * 32 + j;      // streamed position of this column
+            // rows are keys and columns queries (kKV), or the other way round
+            const bool masked = tpos >= a.s || (a.causal && (kKV ? tpos < fpos : tpos > fpos));
+            p[j] = masked ? 0.0f : ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[j]));
+            ds[j] = p[j] * (__uint_as_float(yr[j]) - dv[j]);
           }
-          p[j] = masked ? 0.0f : ex2f(fmaf(__uint_as_float(xr[j]), sl, -lcol));
-          ds[j] = p[j] * (__uint_as_float(yr[j]) - dcol);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) {
+            p[j] = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[j]));
+            ds[j] = p[j] * (__uint_as_float(yr[j]) - dv[j]);
+          }
         }
         uint8_t* pch = prow + (c >> 1) * kTile;
         uint8_t* dch = drow + (c >> 1) * kTile;
