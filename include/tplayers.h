@@ -66,7 +66,7 @@ enum {
   TP_ERR_SHAPE = 2,       /* a size is <= 0, inconsistent, or not divisible as required */
   TP_ERR_ALIGN = 3,       /* a pointer or row length breaks the alignment rules above */
   TP_ERR_DTYPE = 4,       /* unknown dtype or activation code */
-  TP_ERR_UNSUPPORTED = 5, /* valid request this build does not implement */
+  TP_ERR_UNSUPPORTED = 5, /* valid request the library does not implement */
   TP_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed while enqueueing */
   TP_ERR_WORKSPACE = 7,   /* workspace NULL or smaller than tp_workspace_bytes() */
   TP_ERR_DEVICE = 8       /* no usable sm_100 device is current */

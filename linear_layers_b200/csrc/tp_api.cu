@@ -253,7 +253,7 @@ const char* tp_status_string(tp_status s) {
     case TP_ERR_SHAPE: return "invalid or inconsistent sizes";
     case TP_ERR_ALIGN: return "pointer or row length breaks the 16-byte alignment rule";
     case TP_ERR_DTYPE: return "unknown dtype or activation";
-    case TP_ERR_UNSUPPORTED: return "request not supported by this build";
+    case TP_ERR_UNSUPPORTED: return "request not supported by the library";
     case TP_ERR_CUDA: return "CUDA call failed while enqueueing";
     case TP_ERR_WORKSPACE: return "workspace missing or too small";
     case TP_ERR_DEVICE: return "no sm_100 device is current";
