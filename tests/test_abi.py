@@ -120,6 +120,35 @@ def test_validation_errors_before_any_launch(L):
     bad = (ctypes.c_int64 * 3)(0, 3, 3)                        # empty shard
     assert at(FAKE, 2, 16, 3, 64, 2, bad, 1, 0.0, FAKE, None, None, None) == TP_ERR_SHAPE
     assert at(None, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, None, None, None) == TP_ERR_NULL
+    # attention backward: the lse and a workspace are required
+    ab = L.tp_attention_bwd
+    wsa = tpl.tp_workspace_bytes(tpl.OP_ATTENTION_BWD, 32, 4, 64, 2)
+    assert wsa >= 32 * 4 * 4
+    assert ab(FAKE, FAKE, FAKE, None, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, FAKE, wsa, None,
+              None) == TP_ERR_NULL
+    assert ab(FAKE, FAKE, FAKE, FAKE, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, FAKE, wsa - 1, None,
+              None) == 7                                       # TP_ERR_WORKSPACE
+    assert ab(FAKE, FAKE, FAKE, FAKE, 2, 16, 4, 32, 2, None, 1, 0.0, FAKE, FAKE, wsa, None,
+              None) == 5                                       # head_dim 64 only
+    # dropout-add-LayerNorm: 0 <= p < 1, rows split evenly, h a multiple of 8
+    ln = L.tp_sp_dropout_add_ln_fwd
+    args = lambda **k: dict(dict(x=FAKE, b=None, r=FAKE, g=FAKE, be=FAKE, M=64, h=1600, N=4,
+                                 p=0.1, seed=1, off=0, eps=1e-5, hs=FAKE, y=FAKE, m=FAKE, rs=FAKE,
+                                 keep=None), **k)
+    call = lambda a: ln(a["x"], a["b"], a["r"], a["g"], a["be"], a["M"], a["h"], a["N"], a["p"],
+                        a["seed"], a["off"], a["eps"], a["hs"], a["y"], a["m"], a["rs"], a["keep"],
+                        None, None)
+    assert call(args(p=1.0)) == TP_ERR_SHAPE
+    assert call(args(p=-0.1)) == TP_ERR_SHAPE
+    assert call(args(M=66)) == TP_ERR_SHAPE                  # 4 ∤ 66
+    assert call(args(h=1604)) == TP_ERR_ALIGN
+    assert call(args(h=16384)) == 5                           # wider than 8192
+    assert call(args(x=None)) == TP_ERR_NULL
+    lb = L.tp_sp_dropout_add_ln_bwd
+    wsl = tpl.tp_workspace_bytes(tpl.OP_SP_LN_BWD, 64, 1600, 1600, 4)
+    assert wsl >= 3 * (64 // 8) * 1600 * 4
+    assert lb(FAKE, None, FAKE, FAKE, FAKE, FAKE, 64, 1600, 4, 0.1, 1, 0, FAKE, FAKE, FAKE, FAKE,
+              None, FAKE, wsl - 1, None, None) == 7           # TP_ERR_WORKSPACE
 
 
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
@@ -134,6 +163,11 @@ def test_valid_call_without_gpu_fails_loudly(L):
                                     None) == TP_ERR_DEVICE
     assert L.tp_attention_fwd(FAKE, 2, 16, 25, 64, 4, None, 1, 0.0, FAKE, None, None,
                               None) == TP_ERR_DEVICE
+    wsa = tpl.tp_workspace_bytes(tpl.OP_ATTENTION_BWD, 32, 25, 64, 4)
+    assert L.tp_attention_bwd(FAKE, FAKE, FAKE, FAKE, 2, 16, 25, 64, 4, None, 1, 0.0, FAKE, FAKE,
+                              wsa, None, None) == TP_ERR_DEVICE
+    assert L.tp_sp_dropout_add_ln_fwd(FAKE, None, FAKE, FAKE, FAKE, 64, 1600, 4, 0.1, 1, 0, 1e-5,
+                                      FAKE, FAKE, FAKE, FAKE, None, None, None) == TP_ERR_DEVICE
     with pytest.raises(RuntimeError, match="no CPU path"):
         X = torch.zeros(16, 64, dtype=torch.bfloat16)
         tpl.tp_mlp_fwd(X, torch.zeros(64, 256, dtype=torch.bfloat16), None,
