@@ -270,9 +270,12 @@ TP_API tp_status tp_row_linear_bwd(const void* Xin, const void* W, const void* d
  *     a counter each) return TP_ERR_WORKSPACE without enqueueing anything.
  *   - bf16 only (TP_ERR_DTYPE otherwise); N <= 16; every shard offset a
  *     multiple of 64 (TP_ERR_UNSUPPORTED otherwise).
- *   - The first call on a device looks up the scratch address on that device
- *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture.  No call allocates or frees memory.
+ *   - The first call in a CUDA context looks up the scratch address there
+ *     (cudaGetSymbolAddress, with the caller's device and context current)
+ *     and caches it for that context, so callers on their own contexts, or
+ *     on a primary context created again after cudaDeviceReset, get an
+ *     address valid where they run; make that first call before any stream
+ *     capture.  No call allocates or frees memory.
  *   - Every call on a device shares the one scratch array, and it keeps the
  *     previous call's contents (the counters are cleared by each call).
  *     Calls that overlap on the GPU — on two streams, or from two threads —

@@ -4,8 +4,12 @@
 // The shards' fp32 partial tiles and the per-tile arrival counters of the
 // split shard-sum GEMM live in g_noalloc_scratch, a file-scope static device
 // array.  In host code that name is only a host-side stand-in for the
-// symbol, never a device address: the address is looked up once per device
-// with cudaGetSymbolAddress (with that device current) and cached.
+// symbol, never a device address: the address is looked up with
+// cudaGetSymbolAddress while the caller's device (and context) is current,
+// and cached per CUDA context, so a caller on a context of its own (or on a
+// primary context created again after cudaDeviceReset) gets the address that
+// is valid in that context.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -16,31 +20,71 @@ namespace tpl {
 namespace {
 
 constexpr size_t kScratchBytes = TP_NOALLOC_SCRATCH_BYTES;
-constexpr int kMaxDevices = 64;
+constexpr int kCacheSlots = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-void* g_scratch_addr[kMaxDevices] = {nullptr};
+struct ScratchSlot {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+ScratchSlot g_scratch_cache[kCacheSlots];
+int g_scratch_next = 0;
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+  });
+  return fn;
+}
+
+// Device address of the scratch array in the current context.  The first
+// call in a context makes the runtime load the library's module there (and
+// may create the device's primary context), so it belongs before any stream
+// capture.
 tp_status scratch_address(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
     cudaGetLastError();
     return TP_ERR_DEVICE;
   }
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  if (get == nullptr) return TP_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (get(&ctx) != CUDA_SUCCESS) return TP_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess || p == nullptr) {
-      cudaGetLastError();
-      return TP_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
+  if (ctx != nullptr)
+    for (const ScratchSlot& s : g_scratch_cache)
+      if (s.ctx == ctx && s.addr != nullptr) {
+        *out = s.addr;
+        return TP_OK;
+      }
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess || p == nullptr) {
+    cudaGetLastError();
+    return TP_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  // with no context current before, the lookup made the device's primary
+  // context current
+  if (ctx == nullptr && (get(&ctx) != CUDA_SUCCESS || ctx == nullptr)) return TP_ERR_CUDA;
+  // A context handle can be reused after its context is destroyed; the new
+  // context then simply replaces the old entry's address on its first call.
+  ScratchSlot& slot = g_scratch_cache[g_scratch_next];
+  g_scratch_next = (g_scratch_next + 1) % kCacheSlots;
+  slot.ctx = ctx;
+  slot.addr = p;
+  *out = p;
   return TP_OK;
 }
 

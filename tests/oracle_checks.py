@@ -255,6 +255,54 @@ def check_linear_blocks(o):
     assert _rel(gb["dXin"], np.einsum("mj,ij->mi", dZ, Wr)) < 1e-14
 
 
+def _fd_grad(f, P, eps=1e-6):
+    """Central differences of the scalar f() with respect to every entry of
+    the array P (modified in place and restored)."""
+    g = np.zeros_like(P)
+    it = np.nditer(P, flags=["multi_index"])
+    for _ in it:
+        i = it.multi_index
+        keep = P[i]
+        P[i] = keep + eps
+        fp = f()
+        P[i] = keep - eps
+        fm = f()
+        P[i] = keep
+        g[i] = (fp - fm) / (2 * eps)
+    return g
+
+
+def check_linear_bwd_fd(o):
+    """Every gradient of the two linear blocks against central differences of
+    L = Σ out ⊙ dOut ([TP-ILL] §1.1/§1.2: each shard's gradient is the local
+    one, the f/g operators only sum or pass through):
+    - col_linear_bwd: dbias (with a GeLU, so dbias = Σ_rows dY ⊙ act'(U)
+      and not Σ_rows dY) and dU;
+    - row_linear_bwd: dXin and dW of Z = Σ_i Xin_i·W_i over uneven shards."""
+    r = _rng(71)
+    X = r.normal(size=(5, 6))
+    W = r.normal(size=(6, 10)) * 0.5
+    b = r.normal(size=10)
+    for act in (o.ACT_GELU_TANH, o.ACT_GELU_ERF, o.ACT_NONE):
+        U, _ = o.col_linear_fwd(X, W, b, act)
+        dY = r.normal(size=U.shape)
+        g = o.col_linear_bwd(X, W, U, dY, act)
+        L = lambda: float((o.col_linear_fwd(X, W, b, act)[1] * dY).sum())
+        assert _rel(g["dbias"], _fd_grad(L, b)) < 1e-7, act
+        # dU is the gradient with respect to the pre-activation itself
+        Uw = U.copy()
+        LU = lambda: float((o.act_fwd(Uw, act) * dY).sum())
+        assert _rel(g["dU"], _fd_grad(LU, Uw)) < 1e-7, act
+    Xin = r.normal(size=(4, 12))
+    Wr = r.normal(size=(12, 5))
+    dZ = r.normal(size=(4, 5))
+    offs = [0, 7, 12]
+    Lr = lambda: float((o.row_linear_fwd(Xin, Wr, offsets=offs)[0] * dZ).sum())
+    gb = o.row_linear_bwd(Xin, Wr, dZ)
+    assert _rel(gb["dXin"], _fd_grad(Lr, Xin)) < 1e-8
+    assert _rel(gb["dW"], _fd_grad(Lr, Wr)) < 1e-8
+
+
 def check_qkv_head_split(o):
     """25 heads over 4 shards -> 7, 6, 6, 6; shard-major columns are a
     permutation of [Q | K | V] and shard i's block holds exactly its heads."""

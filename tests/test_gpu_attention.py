@@ -13,7 +13,7 @@ import torch
 import linear_layers_b200 as tpl
 import tp_inputs
 from oracle import tp_oracle as O
-from tests.gpu_helpers import TOL_BF16, TOL_XENT, assert_close, f64
+from tests.gpu_helpers import TOL_BF16, TOL_XENT, assert_close, f64, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -32,10 +32,14 @@ def _offsets(nh, N):
 
 def _check(QKV, b, s, nh, N, causal, offs=None, scale=None):
     st = tpl.new_status()
-    ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, head_offsets=offs, causal=causal,
-                                    scale=scale, with_lse=True, dev_status=st)
+    ctx, gctx = guarded((b * s, nh * HD), torch.bfloat16)
+    lse, glse = guarded((b, nh, s), torch.float32)
+    tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, head_offsets=offs, causal=causal, scale=scale,
+                         ctx=ctx, lse=lse, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    gctx.check("ctx")
+    glse.check("lse")
     shards = np.diff(offs if offs is not None else _offsets(nh, N)).tolist()
     rctx, rlse = O.attention_sharded(QKV, b, s, nh, HD, shards, causal=causal, scale=scale)
     g = f64(ctx)
@@ -128,10 +132,12 @@ def _bwd_check(b, s, nh, N, causal, seed, offs=None, scale=None):
     st = tpl.new_status()
     ctx, lse = tpl.tp_attention_fwd(QKV.cuda(), b, s, nh, N, head_offsets=offs, causal=causal,
                                     scale=scale, with_lse=True, dev_status=st)
-    dQKV = tpl.tp_attention_bwd(QKV.cuda(), ctx, dctx.cuda(), lse, b, s, nh, N, head_offsets=offs,
-                                causal=causal, scale=scale, dev_status=st)
+    dQKV, gd = guarded((b * s, 3 * nh * HD), torch.bfloat16)
+    tpl.tp_attention_bwd(QKV.cuda(), ctx, dctx.cuda(), lse, b, s, nh, N, head_offsets=offs,
+                         causal=causal, scale=scale, dQKV=dQKV, dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    gd.check("dQKV")
     shards = np.diff(offs if offs is not None else _offsets(nh, N)).tolist()
     ref = O.attention_sharded_bwd(QKV, dctx, b, s, nh, HD, shards, causal=causal, scale=scale)
     got = f64(dQKV)

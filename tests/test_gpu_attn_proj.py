@@ -9,7 +9,7 @@ import torch
 import linear_layers_b200 as tpl
 import tp_inputs
 from oracle import tp_oracle as O
-from tests.gpu_helpers import TOL_BF16, assert_close, f64, to_dev
+from tests.gpu_helpers import TOL_BF16, assert_close, f64, guarded, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -31,20 +31,33 @@ def _case(M, seed, zpart):
     _, ctx_offs = _head_offsets(nh, hd, N, 1)
     assert heads == [7, 6, 6, 6]
     assert ctx_offs == [0, 448, 832, 1216, 1600]
+    bf = torch.bfloat16
+    # every output inside a guard band (NaN-filled, sentinel margins): the
+    # 1600-wide outputs end in a 64-column tile and M=640 in a half row tile
+    shapes = {"QKV": ((M, 3 * h), bf), "dX": ((M, h), bf), "dWq": ((h, 3 * h), bf),
+              "dbq": ((3 * h,), torch.float32), "Z": ((M, h), bf), "dctx": ((M, h), bf),
+              "dWo": ((h, h), bf)}
+    if zpart:
+        shapes["Zp"] = ((N, M, h), torch.float32)
+    o, guards = {}, {}
+    for k, (shape, t) in shapes.items():
+        o[k], guards[k] = guarded(shape, t)
     st = tpl.new_status()
     # QKV: column-parallel, shard-major columns (own Q, K, V heads per shard)
     QKV, _ = tpl.tp_col_linear_fwd(d["X"], d["Wqkv"], d["bqkv"], N, shard_offsets=qkv_offs,
-                                   dev_status=st)
+                                   Y=o["QKV"], dev_status=st)
     gq = tpl.tp_col_linear_bwd(d["X"], d["Wqkv"], None, d["dQKV"], N, shard_offsets=qkv_offs,
-                               dev_status=st)
+                               dX=o["dX"], dW=o["dWq"], dbias=o["dbq"], dev_status=st)
     # output projection: row-parallel over the per-shard context, summed
-    Zp = torch.empty(N, M, h, dtype=torch.float32, device="cuda") if zpart else None
-    Z = tpl.tp_row_linear_fwd(d["ctx"], d["Wo"], N, shard_offsets=ctx_offs, Zpart=Zp,
+    Zp = o.get("Zp")
+    Z = tpl.tp_row_linear_fwd(d["ctx"], d["Wo"], N, shard_offsets=ctx_offs, Zpart=Zp, Z=o["Z"],
                               dev_status=st)
     go = tpl.tp_row_linear_bwd(d["ctx"], d["Wo"], d["dZ"], N, shard_offsets=ctx_offs,
-                               dev_status=st)
+                               dXin=o["dctx"], dW=o["dWo"], dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
+    for k, gd in guards.items():
+        gd.check(k)
     return inp, qkv_offs, ctx_offs, QKV, gq, Z, Zp, go
 
 

@@ -13,24 +13,39 @@ import torch
 import linear_layers_b200 as tpl
 import tp_inputs
 from oracle import tp_oracle as O
-from tests.gpu_helpers import TOL_BF16, TOL_F32, assert_close, f64, to_dev
+from tests.gpu_helpers import TOL_BF16, TOL_F32, assert_close, f64, guarded, to_dev
 
 pytestmark = pytest.mark.gpu
 
 
 def _run(inp, N, act, offsets=None, zpart=False):
+    """Forward + backward with every output inside a guard band (NaN-filled,
+    sentinel margins before and after) so that a missed store fails the
+    parity check and a store past either end fails the guard check."""
     d = to_dev(inp)
     M, h = d["X"].shape
     F = d["A"].shape[1]
-    Zpart = torch.empty(N, M, h, dtype=torch.float32, device="cuda") if zpart else None
+    dt = d["X"].dtype
+    shapes = {"U": ((M, F), dt), "Y": ((M, F), dt), "Z": ((M, h), dt), "dU": ((M, F), dt),
+              "dX": ((M, h), dt), "dA": ((h, F), dt), "dB": ((F, h), dt),
+              "dbias": ((F,), torch.float32)}
+    if zpart:
+        shapes["Zpart"] = ((N, M, h), torch.float32)
+    out, guards = {}, {}
+    for k, (shape, t) in shapes.items():
+        out[k], guards[k] = guarded(shape, t)
     st = tpl.new_status()
     Z, U, Y = tpl.tp_mlp_fwd(d["X"], d["A"], d["bias"], d["B"], N, shard_offsets=offsets,
-                             act=act, Zpart=Zpart, dev_status=st)
+                             act=act, U=out["U"], Y=out["Y"], Z=out["Z"], Zpart=out.get("Zpart"),
+                             dev_status=st)
     g = tpl.tp_mlp_bwd(d["X"], d["A"], d["B"], U, Y, d["dZ"], N, shard_offsets=offsets, act=act,
+                       dU=out["dU"], dX=out["dX"], dA=out["dA"], dbias=out["dbias"], dB=out["dB"],
                        dev_status=st)
     torch.cuda.synchronize()
     assert int(st.item()) == 0
-    return Z, U, Y, g, Zpart
+    for k, gd in guards.items():
+        gd.check(k)
+    return Z, U, Y, g, out.get("Zpart")
 
 
 def _check_full(inp, N, act, tol, offsets=None, zpart=False):

@@ -9,7 +9,7 @@ import torch
 import linear_layers_b200 as tpl
 import tp_inputs
 from oracle import tp_oracle as O
-from tests.gpu_helpers import TOL_BF16, TOL_XENT, assert_close, f64
+from tests.gpu_helpers import TOL_BF16, TOL_XENT, assert_close, f64, guarded
 
 pytestmark = pytest.mark.gpu
 
@@ -62,8 +62,9 @@ def test_embed_full_size_bit_exact():
 # ---------------------------------------------------------------- logits
 def test_logits_ragged():
     inp = tp_inputs.vocab_inputs(300, 1000, 264, seed=4)
-    L = tpl.tp_logits_fwd(inp["H"].cuda(), inp["E"].cuda(), 4)
-    torch.cuda.synchronize()
+    L, gl = guarded((300, 1000), torch.float32)       # ragged row and column tiles
+    tpl.tp_logits_fwd(inp["H"].cuda(), inp["E"].cuda(), 4, logits=L)
+    gl.check("logits")
     assert_close("logits", L, O.logits(inp["H"], inp["E"]), TOL_BF16)
     blocks = O.logits_sharded(inp["H"], inp["E"], 4)
     for i, b in enumerate(blocks):
@@ -83,8 +84,10 @@ def test_logits_full_size_sampled_rows():
 # ---------------------------------------------------------------- cross-entropy
 def _xent_check(logits, targets, N, grad_scale, rows=None):
     st = tpl.new_status()
-    r = tpl.vp_xent(logits.cuda(), targets.cuda(), N, grad_scale=grad_scale, dev_status=st)
-    torch.cuda.synchronize()
+    dl, gdl = guarded(tuple(logits.shape), torch.float32)
+    r = tpl.vp_xent(logits.cuda(), targets.cuda(), N, grad_scale=grad_scale, dlogits=dl,
+                    dev_status=st)
+    gdl.check("dlogits")
     sel = torch.arange(logits.shape[0]) if rows is None else torch.as_tensor(rows)
     ref = O.xent(logits[sel], targets[sel], grad_scale)
     dsel = sel.cuda()

@@ -303,6 +303,46 @@ def _m_attention_bwd_drops_rowsum(mp):
     mp.setattr(O, "attention_head_bwd", bad)
 
 
+def _m_col_dbias_without_act_grad(mp):
+    orig = O.col_linear_bwd
+
+    def bad(X, W, U, dY, act=O.ACT_NONE):
+        g = orig(X, W, U, dY, act)
+        g["dbias"] = O.f64(dY).sum(axis=0)            # dbias from dY, act'(U) forgotten
+        return g
+    mp.setattr(O, "col_linear_bwd", bad)
+
+
+def _m_col_dbias_mean_not_sum(mp):
+    orig = O.col_linear_bwd
+
+    def bad(X, W, U, dY, act=O.ACT_NONE):
+        g = orig(X, W, U, dY, act)
+        g["dbias"] = g["dU"].mean(axis=0)             # averaged over rows instead of summed
+        return g
+    mp.setattr(O, "col_linear_bwd", bad)
+
+
+def _m_row_bwd_dW_rows_misaligned(mp):
+    orig = O.row_linear_bwd
+
+    def bad(Xin, W, dZ):
+        g = orig(Xin, W, dZ)
+        g["dW"] = O.f64(Xin)[::-1].T @ O.f64(dZ)      # token rows of Xin and dZ out of step
+        return g
+    mp.setattr(O, "row_linear_bwd", bad)
+
+
+def _m_row_bwd_dX_sign(mp):
+    orig = O.row_linear_bwd
+
+    def bad(Xin, W, dZ):
+        g = orig(Xin, W, dZ)
+        g["dXin"] = -g["dXin"]
+        return g
+    mp.setattr(O, "row_linear_bwd", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
