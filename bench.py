@@ -125,7 +125,7 @@ class ClockSampler:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -497,6 +497,82 @@ def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world, reps=10):
     return {p: float(t[i]) for i, p in enumerate(plist)}
 
 
+def _event_loop(torch, fn, n, stream, before=None):
+    """Average ms of fn() over n calls, each bracketed by its own CUDA events
+    on `stream`; before() (untimed) runs ahead of every call."""
+    total = 0.0
+    evs = []
+    for _ in range(n):
+        if before is not None:
+            before()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    for e0, e1 in evs:
+        total += e0.elapsed_time(e1)
+    return total / n
+
+
+def _embed_flushed(torch, tpl, vo, stream, st, n=10):
+    """vp_embed with a 256 MB memset between calls, so the table rows it
+    reads come from HBM and not from the 126 MB L2."""
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=vo["E"].device)
+    ms = _event_loop(torch, lambda: _embed(tpl, vo, st), n, stream, before=flush.zero_)
+    del flush
+    return ms
+
+
+def _library_context(torch, g, vo, stream, n=10):
+    """cuBLAS (torch.matmul, bf16 in, fp32 accumulate) on the six GEMM shapes
+    of the TP-MLP at h=4096 with the operand transposes the layer needs, and
+    torch.nn.functional.cross_entropy (sum, forward + backward) on the same
+    fp32 logits as vp_xent.  Library context, not the product's path."""
+    import torch.nn.functional as F
+
+    X, A, B, dZ, U, Y, dU = (g[k] for k in ("X", "A", "B", "dZ", "U", "Y", "dU"))
+    gemms = {
+        "a2 U=X·A": lambda: torch.matmul(X, A),
+        "a3 Z=Y·B": lambda: torch.matmul(Y, B),
+        "a4 dY=dZ·Bt": lambda: torch.matmul(dZ, B.t()),
+        "a5 dB=Yt·dZ": lambda: torch.matmul(Y.t(), dZ),
+        "a6 dA=Xt·dU": lambda: torch.matmul(X.t(), dU),
+        "a7 dX=dU·At": lambda: torch.matmul(dU, A.t()),
+    }
+    flop = 2.0 * MLP["M"] * MLP["h"] * MLP["F"]
+    out = {}
+    total = 0.0
+    for name, fn in gemms.items():
+        for _ in range(3):
+            fn()
+        ms = _event_loop(torch, fn, n, stream)
+        out[name] = {"ms": round(ms, 4), "tflops": round(flop / (ms / 1e3) / 1e12, 1)}
+        total += ms
+    ctx = {"what": "torch.matmul (cuBLAS) on the six TP-MLP GEMM shapes at h=4096 (no fused "
+                   "bias/GeLU/dGeLU, no shard sums), and torch cross_entropy forward+backward on "
+                   "the [16384, 50304] fp32 logits; timed in this process after the step, "
+                   "%d calls each" % n,
+           "mlp_gemms": out, "mlp_gemms_sum_ms": round(total, 4),
+           "mlp_gemms_sum_tflops": round(MLP_FLOP / (total / 1e3) / 1e12, 1)}
+    if vo is not None:
+        L = vo["logits"].detach().requires_grad_(True)
+        tg = vo["targets"]
+
+        def xent():
+            loss = F.cross_entropy(L, tg, reduction="sum")
+            loss.backward()
+            L.grad = None
+
+        for _ in range(2):
+            xent()
+        ms = _event_loop(torch, xent, max(3, n // 2), stream)
+        ctx["cross_entropy_fwd_bwd_ms"] = round(ms, 4)
+        ctx["cross_entropy_tokens_per_s"] = round(VOC["T"] / (ms / 1e3), 1)
+    return ctx
+
+
 def run_gpu(args):
     import torch
 
@@ -607,6 +683,9 @@ def run_gpu(args):
     at_ms = _side_loop(torch, fns, ATTN_PARTS, side_steps, stream, dev, st, world)
     ln_ms = _side_loop(torch, fns, LN_PARTS, side_steps, stream, dev, st, world)
 
+    embed_flush_ms = _embed_flushed(torch, tpl, vo, stream, st)
+    libctx = None if args.no_library_context else _library_context(torch, g, vo, stream)
+
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
         all_ms, all_h2d, all_d2h = float("nan"), 0, 0
@@ -663,7 +742,12 @@ def run_gpu(args):
                            "frac_of_spec_8000": round(xent_gbs / SPEC_HBM_GBS, 4),
                            "ms": round(part_ms["xent"] / K, 4)},
             "vp_embed": {"GBps": round(embed_gbs, 1), "frac_of_measured_hbm": round(embed_gbs / peaks["hbm_gbs"], 4),
-                         "us": round(part_ms["embed"] / K * 1e3, 2)},
+                         "us": round(part_ms["embed"] / K * 1e3, 2),
+                         "l2_flushed": {"us": round(embed_flush_ms * 1e3, 2),
+                                        "GBps": round(EMBED_BYTES / (embed_flush_ms / 1e3) / 1e9, 1),
+                                        "frac_of_measured_hbm": round(EMBED_BYTES / (embed_flush_ms / 1e3) / 1e9
+                                                                      / peaks["hbm_gbs"], 4),
+                                        "what": "a 256 MB memset before every call (untimed), 10 calls"}},
             "vocab_bwd": {
                 "what": "next row, own loop of %d iterations after the step" % side_steps,
                 "xent_bf16_grad_ms": round(bwd_ms["xent_bf16"], 4),
@@ -726,6 +810,7 @@ def run_gpu(args):
                 "traffic_unit": "bytes/launch (ncu dram__bytes_read.sum + dram__bytes_write.sum)",
                 "traffic_note": traffic_note,
             },
+            "library_context": libctx,
             "gpu_launches": int(launches),
             "clocks": clocks,
             "wall_s_timed": round(t_wall, 3),
@@ -735,7 +820,9 @@ def run_gpu(args):
                             "(X, dZ) from pinned host memory and reads its results (Z, dX) back inside "
                             "the timed region; weights and weight gradients stay resident on the device "
                             "as in a training loop; copies of neighbouring steps overlap the compute on "
-                            "their own streams",
+                            "their own streams; timed in its own TP-MLP-only loop after the step (the "
+                            "step's other parts do not run between its iterations), so it is not measured "
+                            "under the same conditions as value",
                     "all_tensors": {"value": round(world * MLP_FLOP / (all_ms / 1e3) / 1e12, 2),
                                     "h2d_bytes_per_step": int(all_h2d),
                                     "d2h_bytes_per_step": int(all_d2h),
@@ -848,6 +935,7 @@ def main():
     ap.add_argument("--vocab-tokens", type=int, default=0,
                     help="tokens of the vocabulary path (profiling runs; default 16384)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-library-context", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always
     if args.impl == "reference":

@@ -107,6 +107,25 @@ typedef enum {
  */
 TP_API tp_status tp_selftest_wait_timeout(int32_t* dev_status, uint32_t limit_us, void* stream);
 
+/*
+ * Diagnostics: exercise the real pipeline's failure path.  Arms a one-shot
+ * injection for the NEXT tensor-core GEMM launch of this process (any entry
+ * point; the TP-MLP forward's first launch is its column GEMM): in that
+ * launch the TMA producers of the CTA (pair) that owns work unit `unit`
+ * stop, without a word, before loading k-block `kblock` of it, as a
+ * producer that died would.  The MMA issuer's wait for that k-block then
+ * runs out after wait_limit_us (the launch's every bounded wait uses that
+ * limit); the kernel ORs TP_DEVERR_TIMEOUT into *dev_status, lets the copies
+ * and MMAs already issued finish, frees its tensor memory and returns.  The
+ * outputs of that launch are garbage; later launches are unaffected.  Units
+ * are numbered split-major over the output tiles (unit 0 is the first K range
+ * of the first tile); an injection naming a unit or k-block the launch does
+ * not reach does nothing.  Host-side only: nothing here faults or traps.
+ *   Returns TP_ERR_SHAPE for a negative unit or kblock, or a limit of 0 or
+ *   above 10 s.
+ */
+TP_API tp_status tp_debug_stall_next_gemm(int32_t unit, int32_t kblock, uint32_t wait_limit_us);
+
 /* Human-readable text of a status code (static storage, never NULL). */
 TP_API const char* tp_status_string(tp_status s);
 

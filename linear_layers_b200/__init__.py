@@ -23,6 +23,7 @@ import torch
 __all__ = [
     "TPError", "lib", "library_path", "ACT_NONE", "ACT_GELU_TANH", "ACT_GELU_ERF",
     "tp_status_string", "tp_version", "tp_launch_count", "tp_selftest_wait_timeout",
+    "tp_debug_stall_next_gemm",
     "tp_workspace_bytes", "tp_mlp_fwd", "tp_mlp_bwd",
     "tp_col_linear_fwd", "tp_col_linear_bwd", "tp_row_linear_fwd", "tp_row_linear_bwd",
     "tp_row_linear_fwd_noalloc", "NOALLOC_SCRATCH_BYTES",
@@ -55,6 +56,7 @@ _SIGS = {
     "tp_version": ([], _I32),
     "tp_launch_count": ([], ctypes.c_uint64),
     "tp_selftest_wait_timeout": ([_P, ctypes.c_uint32, _P], _I32),
+    "tp_debug_stall_next_gemm": ([_I32, _I32, ctypes.c_uint32], _I32),
     "tp_workspace_bytes": ([_I32, _I64, _I64, _I64, _I32], _SZ),
     "tp_mlp_fwd": ([_P, _P, _P, _P, _I64, _I64, _I64, _I32, _P, _I32, _I32,
                     _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
@@ -177,6 +179,13 @@ def tp_selftest_wait_timeout(dev_status, limit_us=1000):
     _check(lib().tp_selftest_wait_timeout(_ptr(dev_status), int(limit_us),
                                           _stream(dev_status.device)), "tp_selftest_wait_timeout")
     return dev_status
+
+
+def tp_debug_stall_next_gemm(unit: int, kblock: int, wait_limit_us: int = 50000):
+    """Arm the one-shot producer stall of the next tensor-core GEMM launch
+    (diagnostics of the bounded-wait failure path; see tplayers.h)."""
+    _check(lib().tp_debug_stall_next_gemm(int(unit), int(kblock), int(wait_limit_us)),
+           "tp_debug_stall_next_gemm")
 
 
 def tp_workspace_bytes(op: int, M: int, h: int, F: int, N: int) -> int:

@@ -191,7 +191,7 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream) {
   a.dbias_part = p.dbias_part;
   dim3 block(TS, 8);
   dim3 grid((p.N + TS - 1) / TS, (p.M + TS - 1) / TS);
-  if (p.splits <= 1) {
+  if (p.splits <= 1 && !p.zpart) {
     a.epi = p.epi;
     a.out0 = static_cast<float*>(p.out0);
     a.k0 = 0;

@@ -33,6 +33,7 @@
 #include <cuda_bf16.h>
 
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "internal.h"
@@ -43,12 +44,11 @@ namespace tpl {
 namespace {
 
 constexpr int BM = 128;              // rows of A per CTA
-constexpr int BN = 256;              // output columns per tile
+constexpr int BN = 256;              // output columns of the widest tile
 constexpr int BK = 64;               // bf16 elements per k-block (one 128-byte swizzle row)
 constexpr int kEpiWarps = 8;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kThreads = 64 + kEpiThreads;
-constexpr uint32_t kTmemCols = 512;
 
 struct GemmArgs {
   int M, N, K;
@@ -76,6 +76,7 @@ struct GemmArgs {
   float* tgt_logit;
   const float* row_lse;
   float grad_scale;
+  int inject_unit, inject_kb;       // debug: the producer stops before this k-block (-1: never)
 };
 
 struct __align__(64) GemmParams {
@@ -84,20 +85,25 @@ struct __align__(64) GemmParams {
   GemmArgs a;
 };
 
-template <int CG>
+// Tile configurations: CG CTAs (1 or 2, a cluster pair with cta_group::2)
+// compute a (128·CG) x BNT output tile, BNT = 256 or 128 columns.
+template <int CG, int BNT>
 struct Cfg {
-  static constexpr int kStages = CG == 2 ? 6 : 4;
   static constexpr int kRows = BM * CG;          // output rows per tile
-  static constexpr int kBCols = BN / CG;         // B columns staged per CTA
+  static constexpr int kBCols = BNT / CG;        // B columns staged per CTA
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr uint32_t kBBytes = kBCols * BK * 2;
+  // 192 KB of operand stages: 6 (2 x 256), 4 (1 x 256), 8 (2 x 128), 6 (1 x 128)
+  static constexpr int kStages = static_cast<int>(196608u / (kABytes + kBBytes));
   static constexpr uint32_t kOffB = kStages * kABytes;
   static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;
-  static constexpr uint32_t kBytes = kOffRed + 4 * BN * 4;
+  static constexpr uint32_t kBytes = kOffRed + 4 * BNT * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
+  static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators
+  static constexpr int kChunks = BNT / 64;            // 32-column chunks per epilogue warp
 };
 
 // -------------------------------------------------------------------------
@@ -254,9 +260,11 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
   return v[0];
 }
 
-template <int CG, int EPI>
+template <int CG, int BNT, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, BNT>;
+  static_assert(BNT == 256 || (EPI != EPI_XENT_STATS && EPI != EPI_XENT_GRAD),
+                "the cross-entropy epilogues take 128-column slices of a 256-column tile");
   constexpr int STAGES = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -295,7 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc_cg<CG>(tmem_slot, kTmemCols);
+    tmem_alloc_cg<CG>(tmem_slot, C::kTmemCols);
     tmem_relinquish_cg<CG>();
   }
   tc_fence_before_sync();
@@ -317,8 +325,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         int tm, tn, s, tile;
         unit_map(a, unit, tm, tn, s, tile);
         const int a_row = tm * C::kRows + static_cast<int>(rank) * BM;
-        const int b_col = tn * BN + static_cast<int>(rank) * C::kBCols;
+        const int b_col = tn * BNT + static_cast<int>(rank) * C::kBCols;
         for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
+          if (unit == a.inject_unit && kb == a.inject_kb) {
+            // debug injection: stop issuing without a word, as a producer
+            // that died would; the MMA issuer's bounded wait runs out
+            ok = false;
+            break;
+          }
           if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
             if (!*abort_flag) flag_timeout(a, abort_flag);
             ok = false;
@@ -385,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (pair leader)
     if (rank == 0 && elect_one_sync()) {
-      const uint32_t idesc = idesc_bf16_f32(C::kRows, BN, a.a_mn != 0, a.b_mn != 0);
+      const uint32_t idesc = idesc_bf16_f32(C::kRows, BNT, a.a_mn != 0, a.b_mn != 0);
       const uint32_t a_lbo = a.a_mn ? 8192u : 16u;
       const uint32_t b_lbo = a.b_mn ? 8192u : 16u;
       const uint32_t a_kstep = a.a_mn ? 2048u : 32u;   // bytes per 16-element K step
@@ -405,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           break;
         }
         tc_fence_after_sync();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BNT);
         const int kb0 = a.split_kb[s], kb1 = a.split_kb[s + 1];
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
@@ -463,17 +477,17 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const bool row_ok = row < a.M;
       const int htile = tile * CG + static_cast<int>(rank);   // this CTA's 128-row half tile
       const uint32_t t_base =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      const int c0 = half * 4;
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BNT);
+      const int c0 = half * C::kChunks;   // this warp's first 32-column chunk
 
       if constexpr (EPI == EPI_SPLIT_SUM) {
         // 1) publish this split's fp32 partial
 #pragma unroll 1
-        for (int c = c0; c < c0 + 4; ++c) {
+        for (int c = c0; c < c0 + C::kChunks; ++c) {
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
           tc_wait_ld();
-          const int col0 = tn * BN + c * 32;
+          const int col0 = tn * BNT + c * 32;
           if (a.part_is_zpart) {
             if (row_ok) {
               float* dst = a.part + (static_cast<int64_t>(s) * a.M + row) * a.N + col0;
@@ -486,7 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
           } else {
             float* dst = a.part +
-                         ((static_cast<int64_t>(htile) * a.splits + s) * (BN / 32) + c) * (BM * 32) +
+                         ((static_cast<int64_t>(htile) * a.splits + s) * (BNT / 32) + c) * (BM * 32) +
                          row_in_tile * 32;
 #pragma unroll
             for (int j = 0; j < 8; ++j)
@@ -509,11 +523,11 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           __threadfence();
           // 2) the last split of this half tile sums all partials in split order
 #pragma unroll 1
-          for (int c = c0; c < c0 + 4; ++c) {
+          for (int c = c0; c < c0 + C::kChunks; ++c) {
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_base + c * 32, r);
             tc_wait_ld();
-            const int col0 = tn * BN + c * 32;
+            const int col0 = tn * BNT + c * 32;
             float sum[32];
 #pragma unroll
             for (int j = 0; j < 32; ++j) sum[j] = 0.0f;
@@ -537,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               } else {
                 const float* src =
                     a.part +
-                    ((static_cast<int64_t>(htile) * a.splits + ss) * (BN / 32) + c) * (BM * 32) +
+                    ((static_cast<int64_t>(htile) * a.splits + ss) * (BNT / 32) + c) * (BM * 32) +
                     row_in_tile * 32;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
@@ -559,14 +573,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         // first column holding m; the thread whose slice holds the row's
         // target keeps that accumulator.  Columns past the vocabulary are
         // left out.  Nothing of the logits matrix is written.
-        const int slice = tn * (BN / kXentSlice) + half;
+        const int slice = tn * (BNT / kXentSlice) + half;
         if (slice * kXentSlice < a.N) {   // warp-uniform
           const int64_t tgt = row_ok ? a.targets[row] : -1;
           float m = -INFINITY, ssum = 0.0f;
           int arg = 0;
 #pragma unroll 1
-          for (int c = c0; c < c0 + 4; ++c) {
-            const int col0 = tn * BN + c * 32;
+          for (int c = c0; c < c0 + C::kChunks; ++c) {
+            const int col0 = tn * BNT + c * 32;
             if (col0 >= a.N) break;        // warp-uniform
             uint32_t r[32];
             tmem_ld_32x32b_x32(t_base + c * 32, r);
@@ -628,8 +642,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         }
         const float gs = tgt_ok ? a.grad_scale : __int_as_float(0x7fc00000);
 #pragma unroll 1
-        for (int c = c0; c < c0 + 4; ++c) {
-          const int col0 = tn * BN + c * 32;
+        for (int c = c0; c < c0 + C::kChunks; ++c) {
+          const int col0 = tn * BNT + c * 32;
           if (col0 >= a.N) break;          // warp-uniform
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
@@ -647,7 +661,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         uint4 aux_w[4];
         constexpr bool kDact = EPI == EPI_DACT || EPI == EPI_DACT_Y;
         if constexpr (kDact) {   // U for the first chunk
-          const int col0 = tn * BN + c0 * 32;
+          const int col0 = tn * BNT + c0 * 32;
           if (row_ok && col0 < a.N) {
             load_raw_bf16x32(a.aux + row * a.ld_aux + col0, aux_w, a.N - col0);
           } else {
@@ -656,8 +670,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           }
         }
 #pragma unroll 1
-        for (int c = c0; c < c0 + 4; ++c) {
-          const int col0 = tn * BN + c * 32;
+        for (int c = c0; c < c0 + C::kChunks; ++c) {
+          const int col0 = tn * BNT + c * 32;
           const bool store_ok = row_ok && col0 < a.N;
           uint32_t r[32];
           tmem_ld_32x32b_x32(t_base + c * 32, r);
@@ -665,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if constexpr (kDact) {
             unpack_bf16x32(aux_w, aux_v);
             const int coln = col0 + 32;   // prefetch U of the next chunk while this one runs
-            if (c + 1 < c0 + 4 && row_ok && coln < a.N) {
+            if (c + 1 < c0 + C::kChunks && row_ok && coln < a.N) {
               load_raw_bf16x32(a.aux + row * a.ld_aux + coln, aux_w, a.N - coln);
             } else {
 #pragma unroll
@@ -732,19 +746,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             }
             if (a.dbias_part != nullptr) {
               const float colsum = warp_column_sums(v, lane);
-              red[q * BN + c * 32 + lane] = colsum;
+              red[q * BNT + c * 32 + lane] = colsum;
             }
           }
         }
         if constexpr (kDact) {
           if (a.dbias_part != nullptr) {
             named_barrier_sync(1, kEpiThreads);
-            const int cc = et;   // one column per epilogue thread (256 columns)
-            const int col = tn * BN + cc;
-            // fixed order over the four row quarters of the half tile
-            const float sum = ((red[cc] + red[BN + cc]) + red[2 * BN + cc]) + red[3 * BN + cc];
-            if (col < a.N)
+            const int cc = et;   // one column per epilogue thread (BNT <= 256 columns)
+            const int col = tn * BNT + cc;
+            if (cc < BNT && col < a.N) {
+              // fixed order over the four row quarters of the half tile
+              const float sum = ((red[cc] + red[BNT + cc]) + red[2 * BNT + cc]) + red[3 * BNT + cc];
               a.dbias_part[static_cast<int64_t>(tm * CG + static_cast<int>(rank)) * a.N + col] = sum;
+            }
             named_barrier_sync(1, kEpiThreads);
           }
         }
@@ -765,7 +780,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if constexpr (CG == 2) cluster_sync_all();   // no CTA leaves while its peer may touch it
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc_cg<CG>(tmem_base, kTmemCols);
+    tmem_dealloc_cg<CG>(tmem_base, C::kTmemCols);
   }
 }
 
@@ -805,9 +820,9 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
 // Launch with `slots` persistent CTAs (CG = 1) or CTA pairs (CG = 2), capped
 // at the number that can be resident at once, so that no persistent slot
 // starts only after another has finished.
-template <int CG, int EPI>
+template <int CG, int BNT, int EPI>
 tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
-  using C = Cfg<CG>;
+  using C = Cfg<CG, BNT>;
   static_assert(C::kAlloc <= 232448, "shared memory budget");
   static int max_resident[64] = {0};
   int dev = 0;
@@ -824,12 +839,13 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!max_resident[dev & 63]) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<CG, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             C::kAlloc) != cudaSuccess)
+    if (cudaFuncSetAttribute(gemm_tc_kernel<CG, BNT, EPI>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
       return TP_ERR_CUDA;
     int clusters = 0;
     cfg.gridDim = dim3(static_cast<unsigned>(CG * num_sms()));
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<CG, EPI>, &cfg) != cudaSuccess ||
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<CG, BNT, EPI>, &cfg) !=
+            cudaSuccess ||
         clusters <= 0) {
       cudaGetLastError();
       clusters = num_sms() / CG;
@@ -840,40 +856,95 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   const int grid = CG * slots;
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
-  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<CG, EPI>, prm) != cudaSuccess) return TP_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<CG, BNT, EPI>, prm) != cudaSuccess)
+    return TP_ERR_CUDA;
   note_launches(1);
   return TP_OK;
 }
 
-template <int CG>
+template <int CG, int BNT>
 tp_status launch_epi(const GemmParams& prm, int epi, int slots, cudaStream_t stream) {
   switch (epi) {
-    case EPI_STORE_BF16: return launch_impl<CG, EPI_STORE_BF16>(prm, slots, stream);
-    case EPI_BIAS_ACT: return launch_impl<CG, EPI_BIAS_ACT>(prm, slots, stream);
-    case EPI_DACT: return launch_impl<CG, EPI_DACT>(prm, slots, stream);
-    case EPI_DACT_Y: return launch_impl<CG, EPI_DACT_Y>(prm, slots, stream);
-    case EPI_STORE_F32: return launch_impl<CG, EPI_STORE_F32>(prm, slots, stream);
-    case EPI_SPLIT_SUM: return launch_impl<CG, EPI_SPLIT_SUM>(prm, slots, stream);
-    case EPI_XENT_STATS: return launch_impl<CG, EPI_XENT_STATS>(prm, slots, stream);
-    case EPI_XENT_GRAD: return launch_impl<CG, EPI_XENT_GRAD>(prm, slots, stream);
+    case EPI_STORE_BF16: return launch_impl<CG, BNT, EPI_STORE_BF16>(prm, slots, stream);
+    case EPI_BIAS_ACT: return launch_impl<CG, BNT, EPI_BIAS_ACT>(prm, slots, stream);
+    case EPI_DACT: return launch_impl<CG, BNT, EPI_DACT>(prm, slots, stream);
+    case EPI_DACT_Y: return launch_impl<CG, BNT, EPI_DACT_Y>(prm, slots, stream);
+    case EPI_STORE_F32: return launch_impl<CG, BNT, EPI_STORE_F32>(prm, slots, stream);
+    case EPI_SPLIT_SUM: return launch_impl<CG, BNT, EPI_SPLIT_SUM>(prm, slots, stream);
+    case EPI_XENT_STATS:
+      if constexpr (BNT == 256) return launch_impl<CG, BNT, EPI_XENT_STATS>(prm, slots, stream);
+      break;
+    case EPI_XENT_GRAD:
+      if constexpr (BNT == 256) return launch_impl<CG, BNT, EPI_XENT_GRAD>(prm, slots, stream);
+      break;
   }
   return TP_ERR_UNSUPPORTED;
 }
 
-// Tile configuration: pairs of CTAs (256-row tiles) unless the problem is a
-// single 128-row tile high; TP_GEMM_CTA_GROUP=1|2 forces one (tests).
-int choose_cg(int M) {
-  static int forced = -1;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    forced = 0;
-    if (const char* e = std::getenv("TP_GEMM_CTA_GROUP")) {
-      const int v = std::atoi(e);
-      if (v == 1 || v == 2) forced = v;
+// One-shot debug injection (tp_debug_stall_next_gemm): the next launch's
+// producers stop before k-block `kb` of unit `unit`, and that launch's
+// bounded waits give up after `wait_ns`.
+std::mutex g_inject_mu;
+bool g_inject_armed = false;
+int g_inject_unit = -1, g_inject_kb = -1;
+uint64_t g_inject_wait_ns = 0;
+
+void take_injection(int& unit, int& kb, uint64_t& wait_ns) {
+  std::lock_guard<std::mutex> lk(g_inject_mu);
+  if (!g_inject_armed) return;
+  unit = g_inject_unit;
+  kb = g_inject_kb;
+  wait_ns = g_inject_wait_ns;
+  g_inject_armed = false;
+}
+
+struct TileChoice {
+  int cg;    // CTAs per tile (1, or a cluster pair with cta_group::2)
+  int bn;    // output columns per tile (256 or 128)
+};
+
+// Relative throughput of each tile shape per SM (the 256 x 256 pair tile is
+// the reference): narrower or single-CTA tiles read more operand bytes per
+// MMA and keep the tensor pipe a little less busy.
+double tile_efficiency(int cg, int bn) {
+  if (cg == 2) return bn == 256 ? 1.0 : 0.93;
+  return bn == 256 ? 0.95 : 0.85;
+}
+
+// Tile shape of a GEMM: the one with the least estimated time, counting
+// whole waves of units (tiles x splits) over the resident slots, each wave
+// costing one tile's work per SM.  Problems one 128-row tile high use
+// single-CTA tiles; the cross-entropy epilogues need 256-column tiles.
+// TP_GEMM_TILE=2x256|2x128|1x256|1x128 forces a shape (tests and sweeps).
+TileChoice choose_tile(int M, int N, int splits, int epi) {
+  const bool xent = epi == EPI_XENT_STATS || epi == EPI_XENT_GRAD;
+  if (const char* e = std::getenv("TP_GEMM_TILE")) {
+    TileChoice t{0, 0};
+    if (!std::strcmp(e, "2x256")) t = {2, 256};
+    else if (!std::strcmp(e, "2x128")) t = {2, 128};
+    else if (!std::strcmp(e, "1x256")) t = {1, 256};
+    else if (!std::strcmp(e, "1x128")) t = {1, 128};
+    if (t.cg && !(xent && t.bn != 256)) return t;
+  }
+  const TileChoice cands[4] = {{2, 256}, {2, 128}, {1, 256}, {1, 128}};
+  TileChoice best{M > BM ? 2 : 1, 256};
+  double best_cost = 0.0;
+  bool have = false;
+  for (const TileChoice& t : cands) {
+    if (xent && t.bn != 256) continue;
+    if (M <= BM && t.cg == 2) continue;
+    const long long tiles = static_cast<long long>((M + BM * t.cg - 1) / (BM * t.cg)) *
+                            ((N + t.bn - 1) / t.bn);
+    const long long slots = num_sms() / t.cg;
+    const long long waves = (tiles * splits + slots - 1) / slots;
+    const double cost = static_cast<double>(waves) * t.bn / tile_efficiency(t.cg, t.bn);
+    if (!have || cost < best_cost * 0.999) {
+      best = t;
+      best_cost = cost;
+      have = true;
     }
-  });
-  if (forced) return forced;
-  return M > BM ? 2 : 1;
+  }
+  return best;
 }
 
 }  // namespace
@@ -884,18 +955,35 @@ bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t 
 }
 
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
-  if (splits <= 1) return 0;
-  // 128-row half tiles of the 256-row tiling (covers the 128-row tiling too)
-  const size_t htiles = static_cast<size_t>((M + 2 * BM - 1) / (2 * BM)) * 2 * ((N + BN - 1) / BN);
-  size_t bytes = with_zpart ? 0 : htiles * splits * BM * BN * sizeof(float);
-  bytes += htiles * sizeof(int);
+  if (splits <= 1 && !with_zpart) return 0;
+  // 128-row half tiles of the 256-row tiling (covers the 128-row tiling
+  // too); the partial bytes of 256-column tiles bound those of 128-column
+  // tiles, whose counters are twice as many
+  const size_t hrows = static_cast<size_t>((M + 2 * BM - 1) / (2 * BM)) * 2;
+  size_t bytes = with_zpart ? 0 : hrows * ((N + BN - 1) / BN) * splits * BM * BN * sizeof(float);
+  bytes += hrows * ((N + 127) / 128) * sizeof(int);
   return (bytes + 255) & ~static_cast<size_t>(255);
+}
+
+double gemm_tc_estimate_s(int M, int N, int K, int splits, int epi) {
+  const TileChoice t = choose_tile(M, N, splits, epi);
+  const long long tiles =
+      static_cast<long long>((M + BM * t.cg - 1) / (BM * t.cg)) * ((N + t.bn - 1) / t.bn);
+  const long long slots = num_sms() / t.cg;
+  const long long waves = (tiles * splits + slots - 1) / slots;
+  const double k_split = static_cast<double>(K) / splits;
+  const double per_sm_flops = 1.5e15 / 148.0;   // bf16 dense, sustained
+  return static_cast<double>(waves) * 2.0 * BM * t.bn * k_split /
+         (per_sm_flops * tile_efficiency(t.cg, t.bn));
 }
 
 tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return TP_ERR_SHAPE;
   if (p.splits < 1 || p.splits > kMaxSplits) return TP_ERR_SHAPE;
-  const int CG = choose_cg(p.M);
+  const bool split_epi = p.splits > 1 || p.zpart != nullptr;
+  const TileChoice tile = choose_tile(p.M, p.N, p.splits, split_epi ? EPI_SPLIT_SUM : p.epi);
+  const int CG = tile.cg;
+  const int BNT = tile.bn;
   const int rows = BM * CG;
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
@@ -906,7 +994,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.a_mn = p.a_mn;
   a.b_mn = p.b_mn;
   a.tiles_m = (p.M + rows - 1) / rows;
-  a.tiles_n = (p.N + BN - 1) / BN;
+  a.tiles_n = (p.N + BNT - 1) / BNT;
   a.splits = p.splits;
   a.group_m = CG == 2 ? 8 : 16;
   const int kblocks = (p.K + BK - 1) / BK;
@@ -923,7 +1011,10 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     if (p.split_k[0] != 0 || p.split_k[p.splits] != p.K) return TP_ERR_SHAPE;
   }
   a.num_units = a.tiles_m * a.tiles_n * a.splits;
-  const int epi = p.splits > 1 ? EPI_SPLIT_SUM : p.epi;
+  // partials requested (Zpart) go through the split epilogue even for a
+  // single split: it publishes the partial and stores the (one-term) sum
+  if (p.zpart != nullptr && p.epi != EPI_STORE_BF16) return TP_ERR_UNSUPPORTED;
+  const int epi = split_epi ? EPI_SPLIT_SUM : p.epi;
   a.act = p.act;
   a.out0 = p.out0;
   a.out1 = p.out1;
@@ -941,8 +1032,11 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.tgt_logit = p.tgt_logit;
   a.row_lse = p.row_lse;
   a.grad_scale = p.grad_scale;
+  a.inject_unit = -1;
+  a.inject_kb = -1;
+  take_injection(a.inject_unit, a.inject_kb, a.wait_ns);
   if ((p.epi == EPI_XENT_STATS || p.epi == EPI_XENT_GRAD) && p.splits != 1) return TP_ERR_UNSUPPORTED;
-  if (p.splits > 1) {
+  if (split_epi) {
     const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
     if (p.ws == nullptr || p.ws_bytes < need) return TP_ERR_WORKSPACE;
     const size_t htiles = static_cast<size_t>(a.tiles_m) * CG * a.tiles_n;
@@ -954,14 +1048,14 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
       a.part = static_cast<float*>(p.ws);
       a.part_is_zpart = 0;
       a.counters = reinterpret_cast<int*>(static_cast<uint8_t*>(p.ws) +
-                                          htiles * p.splits * BM * BN * sizeof(float));
+                                          htiles * p.splits * BM * BNT * sizeof(float));
     }
     if (cudaMemsetAsync(a.counters, 0, htiles * sizeof(int), stream) != cudaSuccess)
       return TP_ERR_CUDA;
   }
   // operand maps: A boxes of 128 rows (K-major) or 64 x 64 blocks (MN-major);
-  // B boxes of BN / CG rows (K-major) or 64 x 64 blocks (MN-major)
-  const uint32_t b_rows = static_cast<uint32_t>(BN / CG);
+  // B boxes of BNT / CG rows (K-major) or 64 x 64 blocks (MN-major)
+  const uint32_t b_rows = static_cast<uint32_t>(BNT / CG);
   bool ok;
   if (!p.a_mn)
     ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, BM);
@@ -975,7 +1069,19 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (!ok) return TP_ERR_CUDA;
   const int slots = CG == 2 ? num_sms() / 2 : num_sms();
   const int used = a.num_units < slots ? a.num_units : slots;
-  return CG == 2 ? launch_epi<2>(prm, epi, used, stream) : launch_epi<1>(prm, epi, used, stream);
+  if (CG == 2)
+    return BNT == 256 ? launch_epi<2, 256>(prm, epi, used, stream)
+                      : launch_epi<2, 128>(prm, epi, used, stream);
+  return BNT == 256 ? launch_epi<1, 256>(prm, epi, used, stream)
+                    : launch_epi<1, 128>(prm, epi, used, stream);
+}
+
+void arm_gemm_injection(int unit, int kb, uint64_t wait_ns) {
+  std::lock_guard<std::mutex> lk(g_inject_mu);
+  g_inject_unit = unit;
+  g_inject_kb = kb;
+  g_inject_wait_ns = wait_ns;
+  g_inject_armed = true;
 }
 
 }  // namespace tpl

@@ -71,6 +71,13 @@ size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart);
 
 tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream);
 
+// Arm the one-shot debug injection of the next gemm_tc_launch.
+void arm_gemm_injection(int unit, int kb, uint64_t wait_ns);
+
+// Estimated run time (seconds) of a tensor-core GEMM with `splits` K ranges,
+// with the tile shape gemm_tc_launch would choose (whole waves of tiles).
+double gemm_tc_estimate_s(int M, int N, int K, int splits, int epi);
+
 // fp32 SIMT path (same problem description; operands fp32).
 tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream);
 

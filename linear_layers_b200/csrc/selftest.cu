@@ -41,3 +41,11 @@ extern "C" tp_status tp_selftest_wait_timeout(int32_t* dev_status, uint32_t limi
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
+
+extern "C" tp_status tp_debug_stall_next_gemm(int32_t unit, int32_t kblock, uint32_t wait_limit_us) {
+  using namespace tpl;
+  if (unit < 0 || kblock < 0) return TP_ERR_SHAPE;
+  if (wait_limit_us == 0 || wait_limit_us > 10000000u) return TP_ERR_SHAPE;
+  arm_gemm_injection(unit, kblock, static_cast<uint64_t>(wait_limit_us) * 1000ull);
+  return TP_OK;
+}

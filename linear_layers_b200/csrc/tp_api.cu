@@ -122,10 +122,9 @@ bool ptrs_aligned(std::initializer_list<const void*> ps) {
 // traffic at HBM speed.  Splits must be a divisor of N with every group
 // boundary on a 64-element k-block.
 int choose_splits(int64_t M, int64_t Nout, int64_t K, const std::vector<int64_t>& offs, int sms) {
+  (void)sms;
   const int N = static_cast<int>(offs.size()) - 1;
-  const int64_t tiles = ((M + 127) / 128) * ((Nout + 255) / 256);
-  const double flops = 2.0 * M * Nout * K;
-  const double tc_rate = 1.5e15, hbm = 6.5e12;
+  const double hbm = 6.5e12;
   double best_cost = 0;
   int best = 1;
   for (int S = 1; S <= N && S <= kMaxSplits; ++S) {
@@ -135,16 +134,14 @@ int choose_splits(int64_t M, int64_t Nout, int64_t K, const std::vector<int64_t>
       if (offs[g * (N / S)] % 64) aligned = false;
     if (!aligned) continue;
     if (S > 1 && K / S < 512) continue;   // keep main loops long enough
-    const int64_t units = tiles * S;
-    const int64_t waves = (units + sms - 1) / sms;
-    const double eff = static_cast<double>(units) / static_cast<double>(waves * sms);
-    double cost = flops / (tc_rate * eff);
-    if (S > 1) cost += static_cast<double>(S - 1) * M * Nout * 4.0 / hbm;
+    // whole waves of the chosen tile shape, plus the fp32 partials written
+    // and read back by the splits but the last
+    double cost = gemm_tc_estimate_s(static_cast<int>(M), static_cast<int>(Nout),
+                                     static_cast<int>(K), S, S > 1 ? EPI_SPLIT_SUM : EPI_STORE_BF16);
+    if (S > 1) cost += static_cast<double>(S - 1) * M * Nout * 4.0 * 2.0 / hbm;
     if (S == 1 || cost < best_cost * 0.98) {
-      if (S == 1 || cost < best_cost) {
-        best_cost = cost;
-        best = S;
-      }
+      best_cost = cost;
+      best = S;
     }
   }
   return best;

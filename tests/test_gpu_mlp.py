@@ -76,6 +76,9 @@ def test_mlp_shard_partials_and_uneven_shards():
     inp = tp_inputs.mlp_inputs(130, 128, 768, w_std=0.05, bias_std=0.02, seed=2)
     _check_full(inp, 3, tpl.ACT_GELU_TANH, TOL_BF16, offsets=[0, 128, 448, 768], zpart=True)
     _check_full(inp, 4, tpl.ACT_GELU_TANH, TOL_BF16, zpart=True)
+    # one shard: Zpart[0] is the whole product in fp32 (the per-rank partial
+    # a multi-GPU layer all-reduces)
+    _check_full(inp, 1, tpl.ACT_GELU_TANH, TOL_BF16, zpart=True)
 
 
 def test_mlp_degenerate_sizes():
@@ -154,3 +157,17 @@ def test_mlp_deterministic():
     for k in ("dX", "dA", "dB", "dbias", "dU"):
         assert torch.equal(a[3][k], b[3][k]), k
     assert torch.equal(a[4], b[4])
+
+
+@pytest.mark.parametrize("tile", ["2x256", "2x128", "1x256", "1x128"])
+def test_mlp_every_tile_shape(tile, monkeypatch):
+    """Each tile shape of the GEMM engine (CTA pairs or single CTAs, 256- or
+    128-column tiles), forced for every GEMM of the layer: ragged rows and
+    columns, uneven shards with their partials, and the split shard sum."""
+    monkeypatch.setenv("TP_GEMM_TILE", tile)
+    inp = tp_inputs.mlp_inputs(300, 264, 1024, w_std=0.05, bias_std=0.02, seed=21)
+    _check_full(inp, 4, tpl.ACT_GELU_TANH, TOL_BF16, zpart=True)
+    _check_full(inp, 3, tpl.ACT_GELU_TANH, TOL_BF16, offsets=[0, 128, 448, 1024])
+    # long K over 8 shards: the split shard sum (two or more K ranges per tile)
+    inp = tp_inputs.mlp_inputs(512, 256, 4096, w_std=0.02, bias_std=0.02, seed=22)
+    _check_full(inp, 8, tpl.ACT_GELU_TANH, TOL_BF16)
