@@ -53,11 +53,11 @@ constexpr uint32_t kOffV = kOffK + 2 * kTile;          // 2 stages
 constexpr uint32_t kOffP = kOffV + 2 * kTile;          // per tile: 2 chunks of 64 keys
 constexpr uint32_t kPBytes = 2 * kTile;
 constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
-constexpr int kNumBars = 18;
+constexpr int kNumBars = 12;
 constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
 constexpr uint32_t kAttnBytes = kOffMisc + 16;
 constexpr uint32_t kAttnAlloc = kAttnBytes + 1024;     // slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 512;                    // S: 2 x 128, O_blk: 2 x 64
+constexpr uint32_t kTmemCols = 512;                    // S: 2 x 128, O: 2 x 64
 constexpr uint32_t kTmemO = 256;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -90,66 +90,61 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
-// Row maximum of one 128-key block of S (TMEM, this thread's lane), 64
-// columns per tensor-memory round trip.  With kMask, keys at positions >=
-// klim are left out.
+// The running maximum only moves when a block's maximum exceeds it by more
+// than 2^kTau (log2 units): p = 2^(x·sl − m) then stays below 2^kTau = 256,
+// exact enough in bf16 and far from fp32 overflow, and O in tensor memory is
+// rescaled only on those rare moves instead of after every block.
+constexpr float kTau = 8.0f;
+
+// All 128 scores of this thread's row of one block, read from tensor memory
+// in one round trip (four 32-column loads, one wait).  With kMask, keys at
+// positions >= klim become −inf.  Returns the row maximum.
 template <bool kMask>
-__device__ __forceinline__ float block_row_max(uint32_t sbase, int kpos0, int klim) {
+__device__ __forceinline__ float load_block_row(uint32_t sbase, int kpos0, int klim,
+                                                uint32_t (&x)[kBK]) {
+#pragma unroll
+  for (int c = 0; c < kBK / 32; ++c)
+    tmem_ld_32x32b_x32(sbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
+  tc_wait_ld();
+  if (kMask) {
+#pragma unroll
+    for (int t = 0; t < kBK; ++t)
+      if (kpos0 + t >= klim) x[t] = 0xff800000u;   // −inf
+  }
   float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll 1
-  for (int c = 0; c < kBK / 32; c += 2) {
-    uint32_t rr[64];
-    tmem_ld_32x32b_x32(sbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
-    tmem_ld_32x32b_x32(sbase + c * 32 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
-    tc_wait_ld();
-    float x[64];
 #pragma unroll
-    for (int t = 0; t < 64; ++t) {
-      x[t] = __uint_as_float(rr[t]);
-      if (kMask && kpos0 + c * 32 + t >= klim) x[t] = -INFINITY;
-    }
-#pragma unroll
-    for (int t = 0; t < 64; t += 8) {
-      float& a = acc[(t >> 3) & 3];
-      a = fmax3(a, x[t], x[t + 1]);
-      a = fmax3(a, x[t + 2], x[t + 3]);
-      a = fmax3(a, x[t + 4], x[t + 5]);
-      a = fmax3(a, x[t + 6], x[t + 7]);
-    }
+  for (int t = 0; t < kBK; t += 8) {
+    float& a = acc[(t >> 3) & 3];
+    a = fmax3(a, __uint_as_float(x[t]), __uint_as_float(x[t + 1]));
+    a = fmax3(a, __uint_as_float(x[t + 2]), __uint_as_float(x[t + 3]));
+    a = fmax3(a, __uint_as_float(x[t + 4]), __uint_as_float(x[t + 5]));
+    a = fmax3(a, __uint_as_float(x[t + 6]), __uint_as_float(x[t + 7]));
   }
   return fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]);
 }
 
-// p = 2^(x·sl − m) of one block, stored as bf16 into this row of the P tile
+// p = 2^(x·sl − m) of the row, stored as bf16 into this row of the P tile
 // (two 64-key chunks of 128-byte rows, 16-byte granule g at g ^ (row & 7):
-// the 128-byte swizzle the MMA's descriptor names).  One 64-key chunk per
-// tensor-memory round trip.  Returns Σ p.
-template <bool kMask>
-__device__ __forceinline__ float block_exp_store(uint32_t sbase, int kpos0, int klim, float sl,
-                                                 float m_use, uint8_t* prow, int r) {
+// the 128-byte swizzle the MMA's descriptor names).  Returns Σ p.
+__device__ __forceinline__ float exp_store_row(const uint32_t (&x)[kBK], float sl, float m,
+                                               uint8_t* prow, int r) {
   float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 1
-  for (int h = 0; h < kBK / 64; ++h) {
-    uint32_t rr[64];
-    tmem_ld_32x32b_x32(sbase + h * 64, *reinterpret_cast<uint32_t(*)[32]>(&rr[0]));
-    tmem_ld_32x32b_x32(sbase + h * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&rr[32]));
-    tc_wait_ld();
-    float p[64];
 #pragma unroll
-    for (int t = 0; t < 64; ++t) {
-      float x = __uint_as_float(rr[t]);
-      if (kMask && kpos0 + h * 64 + t >= klim) x = -INFINITY;
-      p[t] = ex2f(fmaf(x, sl, -m_use));
-      ps[t & 3] += p[t];
-    }
+  for (int h = 0; h < kBK / 64; ++h) {
     uint8_t* chunk = prow + h * kTile;
 #pragma unroll
     for (int gr = 0; gr < 8; ++gr) {            // 16-byte granule of the 128-byte row
+      float p[8];
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        p[t] = ex2f(fmaf(__uint_as_float(x[h * 64 + gr * 8 + t]), sl, -m));
+        ps[t & 3] += p[t];
+      }
       uint4 w;
-      w.x = pack_bf16x2(p[8 * gr + 0], p[8 * gr + 1]);
-      w.y = pack_bf16x2(p[8 * gr + 2], p[8 * gr + 3]);
-      w.z = pack_bf16x2(p[8 * gr + 4], p[8 * gr + 5]);
-      w.w = pack_bf16x2(p[8 * gr + 6], p[8 * gr + 7]);
+      w.x = pack_bf16x2(p[0], p[1]);
+      w.y = pack_bf16x2(p[2], p[3]);
+      w.z = pack_bf16x2(p[4], p[5]);
+      w.w = pack_bf16x2(p[6], p[7]);
       *reinterpret_cast<uint4*>(chunk + ((gr ^ (r & 7)) << 4)) = w;
     }
   }
@@ -163,7 +158,7 @@ __device__ __forceinline__ void attn_timeout(const AttnArgs& a, volatile int* ab
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
+__global__ void __maxnreg__(200) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -176,13 +171,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;        // [stage]
   uint64_t* kv_empty = bars + 3;       // [stage]
-  uint64_t* s_full = bars + 5;         // [tile]
-  uint64_t* s_empty = bars + 7;        // [tile]
-  uint64_t* p_full = bars + 9;         // [tile]
-  uint64_t* p_empty = bars + 11;       // [tile]
-  uint64_t* o_full = bars + 13;        // [tile]
-  uint64_t* o_empty = bars + 15;       // [tile]
-  uint64_t* mma_done = bars + 17;
+  uint64_t* s_full = bars + 5;         // [tile]: S_j ready, and every earlier MMA of the CTA done
+  uint64_t* p_full = bars + 7;         // [tile]: P_j written, S_j read, O rescaled
+  uint64_t* o_full = bars + 9;         // [tile]: the last P·V done (O final)
+  uint64_t* mma_done = bars + 11;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
 
@@ -213,11 +205,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], kSoftmaxThreads);
       mbar_init(&p_full[i], kSoftmaxThreads);
-      mbar_init(&p_empty[i], 1);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], kSoftmaxThreads);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -266,13 +255,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBK, false, false);   // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, V MN-major
       bool any = false;
-      // S_g(j) = Q_g·K_jᵀ into tile g's S buffer, once its softmax has read S_g(j-1)
+      // S_g(j) = Q_g·K_jᵀ.  Issued only after the softmax has released S_g(j-1)
+      // (p_full of j-1, taken by issue_pv) and after P·V of j-1, so the
+      // commit's arrival also tells the softmax that O_g holds every block
+      // before j and that the P buffer is free.
       auto issue_s = [&](int g, int j) -> bool {
         const int st = j & 1;
         if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.wait_ns,
-                               abort_flag))
-          return false;
-        if (!mbar_wait_bounded(&s_empty[g], static_cast<uint32_t>(j & 1) ^ 1u, a.wait_ns,
                                abort_flag))
           return false;
         tc_fence_after_sync();
@@ -285,11 +274,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         tc_commit(&s_full[g]);
         return true;
       };
-      // O_g = P_g(j)·V_j, once the softmax has written P_g(j) and taken O_g(j-1)
+      // O_g += P_g(j)·V_j in tensor memory, once the softmax has written P_g(j)
+      // and rescaled O_g where its running maximum moved
       auto issue_pv = [&](int g, int j) -> bool {
-        const uint32_t ph = static_cast<uint32_t>(j & 1);
-        if (!mbar_wait_bounded(&p_full[g], ph, a.wait_ns, abort_flag) ||
-            !mbar_wait_bounded(&o_empty[g], ph ^ 1u, a.wait_ns, abort_flag))
+        if (!mbar_wait_bounded(&p_full[g], static_cast<uint32_t>(j & 1), a.wait_ns, abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t pa = smem_u32(sP + g * kPBytes), vb = smem_u32(sV + (j & 1) * kTile);
@@ -297,9 +285,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         for (int k = 0; k < kBK / 16; ++k)   // 16 keys per step; chunk of 64 keys = 16 KB
           tc_mma_bf16(tmem + kTmemO + g * kHD,
                       smem_desc_sw128(pa + (k >> 2) * kTile + (k & 3) * 32, 16, 1024),
-                      smem_desc_sw128(vb + k * 2048, 8192, 1024), idO, k > 0 ? 1u : 0u);
-        tc_commit(&o_full[g]);
-        tc_commit(&p_empty[g]);
+                      smem_desc_sw128(vb + k * 2048, 8192, 1024), idO,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        if (j + 1 == nkb[g]) tc_commit(&o_full[g]);
         return true;
       };
       bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns, abort_flag);
@@ -336,31 +324,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     const int klim = a.causal ? min(qpos + 1, a.s) : a.s;   // keys [0, klim) are visible
     float m = -INFINITY;                            // running maximum (log2 units)
     float l = 0.0f;                                 // running sum of 2^(x − m)
-    float alpha_prev = 1.0f;
-    float o[kHD];
-#pragma unroll
-    for (int i = 0; i < kHD; ++i) o[i] = 0.0f;
     bool ok = true;
-    // O = O·2^(m_{j-2} − m_{j-1}) + P_{j-1}·V_{j-1}
-    auto take_o = [&](int jb) -> bool {
-      // the warp's lanes agree before the warp-collective tensor-memory loads
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[g], static_cast<uint32_t>(jb & 1),
-                                                     a.wait_ns, abort_flag)))
-        return false;
-      tc_fence_after_sync();
-#pragma unroll
-      for (int c = 0; c < kHD / 32; ++c) {
-        uint32_t rr[32];
-        tmem_ld_32x32b_x32(obase + c * 32, rr);
-        tc_wait_ld();
-#pragma unroll
-        for (int t = 0; t < 32; ++t) o[c * 32 + t] = fmaf(o[c * 32 + t], alpha_prev, __uint_as_float(rr[t]));
-      }
-      tc_fence_before_sync();
-      mbar_arrive(&o_empty[g]);
-      return true;
-    };
     for (int j = 0; j < nk; ++j) {
+      // the warp's lanes agree before the warp-collective tensor-memory loads
       if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[g], static_cast<uint32_t>(j & 1),
                                                      a.wait_ns, abort_flag))) {
         ok = false;
@@ -369,44 +335,58 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
       tc_fence_after_sync();
       const int kpos0 = j * kBK;
       const bool need_mask = (a.causal && j == qb) || kpos0 + kBK > a.s;
-      // pass 1: the row maximum of this block (the mask only where it cuts)
-      const float mx = need_mask ? block_row_max<true>(sbase, kpos0, klim)
-                                 : block_row_max<false>(sbase, kpos0, klim);
-      const float m_new = fmaxf(m, mx * sl);
-      const float m_use = m_new == -INFINITY ? 0.0f : m_new;
-      const float alpha_j = ex2f(m - m_use);        // 0 before the first block
-      // block j-1's P·V has finished (O taken, P buffer free) before P_j is written
-      if (j >= 1 && !take_o(j - 1)) {
-        ok = false;
-        break;
+      uint32_t x[kBK];
+      const float mx = need_mask ? load_block_row<true>(sbase, kpos0, klim, x)
+                                 : load_block_row<false>(sbase, kpos0, klim, x);
+      const float m_blk = mx * sl;   // finite: every block a tile visits has a visible key
+      bool move = j == 0 || m_blk > m + kTau;
+      const float alpha = (j > 0 && move) ? ex2f(m - m_blk) : 1.0f;
+      if (move) m = m_blk;
+      // p = 2^(x·sl − m), bf16 into the swizzled P tile, and the row sum
+      l = fmaf(l, alpha, exp_store_row(x, sl, m, prow, r));
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
+        // O_g holds blocks 0..j-1 (the s_full arrival covers their P·V):
+        // rescale the rows whose maximum moved, the others by 1, before the
+        // P·V of this block adds to it
+#pragma unroll
+        for (int c = 0; c < kHD / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(obase + c * 32, rr);
+          tc_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) rr[t] = __float_as_uint(__uint_as_float(rr[t]) * alpha);
+          tmem_st_32x32b_x32(obase + c * 32, rr);
+        }
+        tc_wait_st();
       }
-      alpha_prev = alpha_j;
-      // pass 2: p = 2^(x·sl − m), bf16 into the swizzled P tile, row sum
-      const float rs = need_mask ? block_exp_store<true>(sbase, kpos0, klim, sl, m_use, prow, r)
-                                 : block_exp_store<false>(sbase, kpos0, klim, sl, m_use, prow, r);
-      tc_fence_before_sync();
-      mbar_arrive(&s_empty[g]);                    // S buffer read out
+      tc_fence_before_sync();                      // S read and O written before the arrival
       fence_proxy_async_smem();                    // P visible to the tensor core
       mbar_arrive(&p_full[g]);
-      l = fmaf(l, alpha_j, rs);
-      m = m_new;
     }
-    if (ok && nk > 0) ok = take_o(nk - 1);
+    if (ok && nk > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_full[g], 0, a.wait_ns, abort_flag));
     if (!ok) {
       if (lane == 0) attn_timeout(a, abort_flag);
-    } else if (nk > 0 && qpos < a.s) {
+    } else if (nk > 0) {
+      tc_fence_after_sync();
       const float inv = 1.0f / l;
       __nv_bfloat16* dst = a.ctx + static_cast<int64_t>(row0 + qpos) * a.ldc + head * kHD;
 #pragma unroll
-      for (int gr = 0; gr < kHD / 8; ++gr) {
-        uint4 w;
-        w.x = pack_bf16x2(o[8 * gr + 0] * inv, o[8 * gr + 1] * inv);
-        w.y = pack_bf16x2(o[8 * gr + 2] * inv, o[8 * gr + 3] * inv);
-        w.z = pack_bf16x2(o[8 * gr + 4] * inv, o[8 * gr + 5] * inv);
-        w.w = pack_bf16x2(o[8 * gr + 6] * inv, o[8 * gr + 7] * inv);
-        reinterpret_cast<uint4*>(dst)[gr] = w;
+      for (int c = 0; c < kHD / 32; ++c) {
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(obase + c * 32, rr);   // every lane loads; rows past s store nothing
+        tc_wait_ld();
+#pragma unroll
+        for (int gr = 0; gr < 4; ++gr) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(rr[8 * gr + 0]) * inv, __uint_as_float(rr[8 * gr + 1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(rr[8 * gr + 2]) * inv, __uint_as_float(rr[8 * gr + 3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(rr[8 * gr + 4]) * inv, __uint_as_float(rr[8 * gr + 5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(rr[8 * gr + 6]) * inv, __uint_as_float(rr[8 * gr + 7]) * inv);
+          if (qpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[gr] = w;
+        }
       }
-      if (a.lse)
+      if (a.lse && qpos < a.s)
         a.lse[(static_cast<int64_t>(batch) * a.heads + head) * a.s + qpos] = m * kLn2 + logf(l);
     }
   }
@@ -422,31 +402,45 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
 
 // ===========================================================================
 // Backward.  D = rowsum(dO ⊙ O) first; then two kernels of one template:
-//   kKV = true   one CTA per 128-key tile of a head: streams the query tiles,
-//                Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ in tensor memory, Pᵀ = exp(Sᵀ·scale
-//                − lse) and dSᵀ = Pᵀ ⊙ (dPᵀ − D) per key row, then
-//                dV += Pᵀ·dO and dK += dSᵀ·Q accumulated in tensor memory;
-//   kKV = false  one CTA per 128-query tile: streams the key tiles, S, dP,
-//                P, dS the same way per query row, dQ += dS·K.
+//   kKV = true   one CTA per 128-key tile of a head: streams the queries in
+//                tiles of 64, Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ in tensor memory,
+//                Pᵀ = exp(Sᵀ·scale − lse) and dSᵀ = Pᵀ ⊙ (dPᵀ − D) per key
+//                row, then dV += Pᵀ·dO and dK += dSᵀ·Q accumulated in tensor
+//                memory;
+//   kKV = false  one CTA per 128-query tile: streams the keys in tiles of 64,
+//                S, dP, P, dS the same way per query row, dQ += dS·K.
 // Each gradient row is produced by exactly one CTA, so there are no atomics
 // and the result does not depend on timing.  dQ and dK carry the scale.
+//
+// Roles (10 warps): warp 0 TMA (the fixed 128-row tiles once, the streamed
+// 64-row tiles through a three-stage ring), warp 1 the MMA issuer, warps 2-5
+// and 6-9 two element-wise warpgroups taking the streamed tiles in turn.
+// S/dP and the bf16 P/dS tiles are double buffered, so the MMAs of one tile
+// (and the gradient MMAs of the one before) run while the other warpgroup
+// evaluates its exponentials.
 // ===========================================================================
-constexpr int kBwdThreads = 192;                       // 6 warps
+constexpr int kBG = 64;                                // streamed rows per tile
+constexpr int kGStages = 3;
+constexpr int kBwdThreads = 320;                       // 10 warps
+constexpr uint32_t kGTile = kBG * kHD * 2;             // 8 KB: 64 rows of 128 bytes
+constexpr uint32_t kPTile = kBQ * kBG * 2;             // 16 KB: 128 fixed rows x 64 streamed
 constexpr uint32_t kBOffF1 = 0;                        // fixed tiles (K, V) or (Q, dO)
 constexpr uint32_t kBOffF2 = kTile;
-constexpr uint32_t kBOffG1 = 2 * kTile;                // streamed tiles, 2 stages each
-constexpr uint32_t kBOffG2 = kBOffG1 + 2 * kTile;
-constexpr uint32_t kBOffP = kBOffG2 + 2 * kTile;       // P (or Pᵀ) bf16: 2 chunks of 64
-constexpr uint32_t kBOffDS = kBOffP + 2 * kTile;       // dS (or dSᵀ) bf16
-constexpr uint32_t kBOffVec = kBOffDS + 2 * kTile;     // per-column lse·log2e and D, 2 stages
-constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * kBQ * 4;
-constexpr int kBNumBars = 10;
+constexpr uint32_t kBOffG1 = 2 * kTile;                // streamed tiles, kGStages each
+constexpr uint32_t kBOffG2 = kBOffG1 + kGStages * kGTile;
+constexpr uint32_t kBOffP = kBOffG2 + kGStages * kGTile;   // Pᵀ [2 buffers] (dK/dV kernel)
+constexpr uint32_t kBOffDS = kBOffP + 2 * kPTile;          // dSᵀ or dS [2 buffers]
+constexpr uint32_t kBOffVec = kBOffDS + 2 * kPTile;        // [warpgroup][2][lse·log2e | D][64]
+constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * 2 * kBG * 4;
+constexpr int kBNumBars = 2 * kGStages + 10;
 constexpr uint32_t kBOffMisc = kBOffBar + kBNumBars * 8;
 constexpr uint32_t kBAlloc = kBOffMisc + 16 + 1024;
-constexpr uint32_t kTX = 0, kTY = 128, kTA1 = 256, kTA2 = 320;   // tensor memory columns
+// tensor memory columns: S/Sᵀ (X) and dP/dPᵀ (Y) double buffered, then the
+// accumulators dV (A1) and dK or dQ (A2)
+constexpr uint32_t kTX = 0, kTY = 128, kTA1 = 256, kTA2 = 320;
 
 struct AttnBwdArgs {
-  int b, s, heads, nqb;
+  int b, s, heads, nqb, ng;  // ng: streamed 64-row tiles of a sequence
   int causal;
   float scale, scale_log2;
   const float* lse;          // [b, heads, s] natural log
@@ -459,8 +453,10 @@ struct AttnBwdArgs {
 };
 
 struct __align__(64) AttnBwdParams {
-  CUtensorMap tm_qkv;        // QKV [b·s, 3h], boxes of 64 columns x 128 rows
+  CUtensorMap tm_qkv;        // QKV [b·s, 3h], boxes of 64 columns x 128 rows (fixed tiles)
   CUtensorMap tm_do;         // dO  [b·s, h],  boxes of 64 columns x 128 rows
+  CUtensorMap tm_qkv_g;      // QKV, boxes of 64 columns x 64 rows (streamed tiles)
+  CUtensorMap tm_do_g;       // dO, boxes of 64 columns x 64 rows
   AttnBwdArgs a;
 };
 
@@ -497,7 +493,7 @@ __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* 
 }
 
 template <bool kKV>
-__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
+__global__ void __maxnreg__(200) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -508,34 +504,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   uint8_t* sG2 = smem + kBOffG2;
   uint8_t* sP = smem + kBOffP;
   uint8_t* sDS = smem + kBOffDS;
-  float* vecL = reinterpret_cast<float*>(smem + kBOffVec);   // [2][128]
-  float* vecD = vecL + 2 * kBQ;                               // [2][128]
+  float* vec = reinterpret_cast<float*>(smem + kBOffVec);   // [warpgroup][buffer][lse | D][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBOffBar);
   uint64_t* f_full = bars;
-  uint64_t* g_full = bars + 1;       // [stage]
-  uint64_t* g_empty = bars + 3;      // [stage]
-  uint64_t* xy_full = bars + 5;
-  uint64_t* xy_empty = bars + 6;
-  uint64_t* pd_full = bars + 7;
-  uint64_t* pd_empty = bars + 8;
-  uint64_t* acc_done = bars + 9;
+  uint64_t* g_full = bars + 1;                   // [stage]
+  uint64_t* g_empty = g_full + kGStages;         // [stage]
+  uint64_t* x_full = g_empty + kGStages;         // [buffer]: S and dP of a tile in tensor memory
+  uint64_t* x_empty = x_full + 2;                // [buffer]: read out by the warpgroup
+  uint64_t* pd_full = x_empty + 2;               // [buffer]: P and dS tiles written
+  uint64_t* pd_empty = pd_full + 2;              // [buffer]: read by the gradient MMAs
+  uint64_t* acc_done = pd_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = a.b * a.heads;
-  // fixed tile, longest first: under the causal mask key tile t streams the
-  // query tiles t.., query tile t the key tiles ..t
+  // fixed 128-row tile, longest first: under the causal mask key tile t
+  // streams the queries from 128·t on, query tile t the keys up to 128·t + 127
   const int ft = kKV ? static_cast<int>(blockIdx.x) / bh
                      : a.nqb - 1 - static_cast<int>(blockIdx.x) / bh;
   const int rem = static_cast<int>(blockIdx.x) % bh;
   const int head = rem / a.b;
   const int batch = rem % a.b;
   const int row0 = batch * a.s;
-  // streamed tiles: queries t >= ft (kKV) or keys t <= ft (dQ) under the causal mask
-  const int t_begin = (kKV && a.causal) ? ft : 0;
-  const int t_end = (!kKV && a.causal) ? ft + 1 : a.nqb;
+  const int t_begin = (kKV && a.causal) ? 2 * ft : 0;                  // in 64-row tiles
+  const int t_end = (!kKV && a.causal) ? min(2 * ft + 2, a.ng) : a.ng;
   const int nt = t_end - t_begin;
   const int qcol = a.head_cols[head].x;
   const int kcol = qcol + a.head_cols[head].y;
@@ -545,18 +539,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   const int f1col = kKV ? kcol : qcol, f2col = kKV ? vcol : ocol;
   const int g1col = kKV ? qcol : kcol, g2col = kKV ? ocol : vcol;
   const CUtensorMap* f2map = kKV ? &P.tm_qkv : &P.tm_do;
-  const CUtensorMap* g2map = kKV ? &P.tm_do : &P.tm_qkv;
+  const CUtensorMap* g2map = kKV ? &P.tm_do_g : &P.tm_qkv_g;
 
   if (threadIdx.x == 0) {
     mbar_init(f_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kGStages; ++i) {
       mbar_init(&g_full[i], 1);
       mbar_init(&g_empty[i], 1);
     }
-    mbar_init(xy_full, 1);
-    mbar_init(xy_empty, kSoftmaxThreads);
-    mbar_init(pd_full, kSoftmaxThreads);
-    mbar_init(pd_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&x_full[i], 1);
+      mbar_init(&x_empty[i], kSoftmaxThreads);
+      mbar_init(&pd_full[i], kSoftmaxThreads);
+      mbar_init(&pd_empty[i], 1);
+    }
     mbar_init(acc_done, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -575,84 +571,101 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     if (elect_one_sync()) {
       tma_prefetch_desc(&P.tm_qkv);
       tma_prefetch_desc(&P.tm_do);
+      tma_prefetch_desc(&P.tm_qkv_g);
+      tma_prefetch_desc(&P.tm_do_g);
       mbar_arrive_expect_tx(f_full, 2 * kTile);
       tma_load_2d(sF1, &P.tm_qkv, f_full, f1col, row0 + ft * kBQ);
       tma_load_2d(sF2, f2map, f_full, f2col, row0 + ft * kBQ);
       int issued = 0;
       for (int it = 0; it < nt; ++it) {
-        const int st = it & 1;
-        if (!mbar_wait_bounded(&g_empty[st], (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u, a.wait_ns,
-                               abort_flag)) {
+        const int st = it % kGStages;
+        if (!mbar_wait_bounded(&g_empty[st], (static_cast<uint32_t>(it / kGStages) & 1u) ^ 1u,
+                               a.wait_ns, abort_flag)) {
           bwd_timeout(a, abort_flag);
           break;
         }
-        const int r = row0 + (t_begin + it) * kBQ;
-        mbar_arrive_expect_tx(&g_full[st], 2 * kTile);
-        tma_load_2d(sG1 + st * kTile, &P.tm_qkv, &g_full[st], g1col, r);
-        tma_load_2d(sG2 + st * kTile, g2map, &g_full[st], g2col, r);
+        const int r = row0 + (t_begin + it) * kBG;
+        mbar_arrive_expect_tx(&g_full[st], 2 * kGTile);
+        tma_load_2d(sG1 + st * kGTile, &P.tm_qkv_g, &g_full[st], g1col, r);
+        tma_load_2d(sG2 + st * kGTile, g2map, &g_full[st], g2col, r);
         ++issued;
       }
       volatile int keep_waiting = 0;   // every copy lands before the CTA can exit
       mbar_wait_bounded(f_full, 0, a.wait_ns, &keep_waiting);
-      for (int it = issued > 2 ? issued - 2 : 0; it < issued; ++it)
-        mbar_wait_bounded(&g_full[it & 1], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns,
-                          &keep_waiting);
+      for (int it = issued > kGStages ? issued - kGStages : 0; it < issued; ++it)
+        mbar_wait_bounded(&g_full[it % kGStages], static_cast<uint32_t>(it / kGStages) & 1u,
+                          a.wait_ns, &keep_waiting);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one_sync()) {
-      constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBQ, false, false);   // both K-major
+      constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBG, false, false);   // both K-major
       constexpr uint32_t idA = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, G MN-major
       bool ok = mbar_wait_bounded(f_full, 0, a.wait_ns, abort_flag);
       bool any = false;
       const uint32_t f1 = smem_u32(sF1), f2 = smem_u32(sF2);
-      const uint32_t pa = smem_u32(sP), da = smem_u32(sDS);
-      for (int it = 0; ok && it < nt; ++it) {
-        const int st = it & 1;
-        const uint32_t ph = static_cast<uint32_t>(it & 1);
-        if (!mbar_wait_bounded(&g_full[st], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns, abort_flag) ||
-            !mbar_wait_bounded(xy_empty, ph ^ 1u, a.wait_ns, abort_flag)) {
-          ok = false;
-          break;
-        }
+      // X_b = F1·G1ᵀ (S or Sᵀ) and Y_b = F2·G2ᵀ (dP or dPᵀ) of streamed tile it
+      auto issue_xy = [&](int it) -> bool {
+        const int st = it % kGStages, b = it & 1;
+        if (!mbar_wait_bounded(&g_full[st], static_cast<uint32_t>(it / kGStages) & 1u, a.wait_ns,
+                               abort_flag) ||
+            !mbar_wait_bounded(&x_empty[b], (static_cast<uint32_t>(it >> 1) & 1u) ^ 1u, a.wait_ns,
+                               abort_flag))
+          return false;
         tc_fence_after_sync();
-        const uint32_t g1 = smem_u32(sG1 + st * kTile), g2 = smem_u32(sG2 + st * kTile);
+        const uint32_t g1 = smem_u32(sG1 + st * kGTile), g2 = smem_u32(sG2 + st * kGTile);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k) {
-          tc_mma_bf16(tmem + kTX, smem_desc_sw128(f1 + k * 32, 16, 1024),
+          tc_mma_bf16(tmem + kTX + b * kBG, smem_desc_sw128(f1 + k * 32, 16, 1024),
                       smem_desc_sw128(g1 + k * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
-          tc_mma_bf16(tmem + kTY, smem_desc_sw128(f2 + k * 32, 16, 1024),
+          tc_mma_bf16(tmem + kTY + b * kBG, smem_desc_sw128(f2 + k * 32, 16, 1024),
                       smem_desc_sw128(g2 + k * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
         }
         any = true;
-        tc_commit(xy_full);
-        if (!mbar_wait_bounded(pd_full, ph, a.wait_ns, abort_flag)) {
+        tc_commit(&x_full[b]);
+        return true;
+      };
+      if (ok && nt > 0) ok = issue_xy(0);
+      if (ok && nt > 1) ok = issue_xy(1);
+      for (int it = 0; ok && it < nt; ++it) {
+        const int st = it % kGStages, b = it & 1;
+        if (!mbar_wait_bounded(&pd_full[b], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns,
+                               abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
+        const uint32_t g1 = smem_u32(sG1 + st * kGTile), g2 = smem_u32(sG2 + st * kGTile);
+        const uint32_t pa = smem_u32(sP + b * kPTile), da = smem_u32(sDS + b * kPTile);
 #pragma unroll
-        for (int k = 0; k < kBQ / 16; ++k) {   // K = the streamed tile's 128 rows
+        for (int k = 0; k < kBG / 16; ++k) {   // K = the streamed tile's 64 rows
           const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
-          const uint32_t off = (k >> 2) * kTile + (k & 3) * 32;
           if constexpr (kKV)   // dV += Pᵀ·dO
-            tc_mma_bf16(tmem + kTA1, smem_desc_sw128(pa + off, 16, 1024),
+            tc_mma_bf16(tmem + kTA1, smem_desc_sw128(pa + k * 32, 16, 1024),
                         smem_desc_sw128(g2 + k * 2048, 8192, 1024), idA, acc);
           // dK += dSᵀ·Q  or  dQ += dS·K
-          tc_mma_bf16(tmem + kTA2, smem_desc_sw128(da + off, 16, 1024),
+          tc_mma_bf16(tmem + kTA2, smem_desc_sw128(da + k * 32, 16, 1024),
                       smem_desc_sw128(g1 + k * 2048, 8192, 1024), idA, acc);
         }
-        tc_commit(pd_empty);
+        tc_commit(&pd_empty[b]);
         tc_commit(&g_empty[st]);
+        if (it + 2 < nt) ok = issue_xy(it + 2);
       }
       if (!ok) bwd_timeout(a, abort_flag);
-      if (any) tc_commit(acc_done);   // completes once every MMA above has
-      if (!any) mbar_arrive(acc_done);
+      if (any) {
+        tc_commit(acc_done);   // completes once every MMA above has
+        volatile int keep_waiting = 0;   // and this thread sees them done before teardown
+        mbar_wait_bounded(acc_done, 0, a.wait_ns, &keep_waiting);
+      } else {
+        mbar_arrive(acc_done);
+      }
     }
   } else {
     // ------------------------------------------------------------ element-wise
+    const int wg = (warp - 2) >> 2;                // warpgroup: streamed tiles wg, wg + 2, ...
     const int qd = warp & 3;
     const int r = qd * 32 + lane;                  // fixed row = TMEM lane
+    const int et = threadIdx.x - 64 - wg * kSoftmaxThreads;   // 0..127 in the warpgroup
     const int fpos = ft * kBQ + r;                 // its position in the sequence
     const int sbase = (batch * a.heads + head) * a.s;
     const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
@@ -661,104 +674,100 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     // the fixed row's own lse and D (dQ kernel)
     const float own_l = (!kKV && fpos < a.s) ? a.lse[sbase + fpos] * kLog2e : 0.0f;
     const float own_d = (!kKV && fpos < a.s) ? a.D[sbase + fpos] : 0.0f;
-    uint8_t* prow = sP + r * 128;
-    uint8_t* drow = sDS + r * 128;
-    const int et = threadIdx.x - 64;               // 0..127
+    uint8_t* prow = sP + wg * kPTile + r * 128;
+    uint8_t* drow = sDS + wg * kPTile + r * 128;
     bool ok = true;
-    for (int it = 0; it < nt; ++it) {
-      const int st = it & 1;
-      const uint32_t ph = static_cast<uint32_t>(it & 1);
-      const int t0 = (t_begin + it) * kBQ;         // first position of the streamed tile
-      if constexpr (kKV) {   // lse·log2e and D of the streamed queries, one per thread
-        const int q = t0 + et;
-        vecL[st * kBQ + et] = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
-        vecD[st * kBQ + et] = q < a.s ? a.D[sbase + q] : 0.0f;
+    for (int it = wg; it < nt; it += 2) {
+      const uint32_t use = static_cast<uint32_t>(it >> 1);   // this warpgroup's tile count
+      const int t0 = (t_begin + it) * kBG;         // first position of the streamed tile
+      const float* vL = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
+      const float* vD = vL + kBG;
+      if constexpr (kKV) {   // lse·log2e and D of the streamed queries
+        if (et < kBG) {
+          const int q = t0 + et;
+          float* w = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
+          w[et] = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
+          w[kBG + et] = q < a.s ? a.D[sbase + q] : 0.0f;
+        }
         // one barrier per tile that also carries every thread's state, so all
-        // 128 threads leave together and none is left waiting in it
-        ok = __all_sync(0xffffffffu, ok);          // the warp converged for the aligned barrier
-        if (!named_barrier_and(1, kSoftmaxThreads, ok)) {
+        // 128 threads of the warpgroup leave together and none is left in it
+        ok = __all_sync(0xffffffffu, ok);
+        if (!named_barrier_and(1 + wg, kSoftmaxThreads, ok)) {
           ok = false;
           break;
         }
       }
       // the warp's lanes agree before the warp-collective tensor-memory loads
-      const bool got = __all_sync(0xffffffffu,
-                                  mbar_wait_bounded(xy_full, ph, a.wait_ns, abort_flag) &&
-                                      mbar_wait_bounded(pd_empty, ph ^ 1u, a.wait_ns, abort_flag));
-      if (!got) {
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait_bounded(&x_full[wg], use & 1u, a.wait_ns, abort_flag))) {
         ok = false;
         if constexpr (kKV) continue;   // leave at the next tile's barrier, with the others
         break;
       }
       tc_fence_after_sync();
-      // the mask can only cut the diagonal tile and the tile past the end
-      const bool need_mask = (a.causal && t_begin + it == ft) || t0 + kBQ > a.s;
-#pragma unroll 1
-      for (int c = 0; c < kBQ / 32; ++c) {
-        uint32_t xr[32], yr[32];
-        tmem_ld_32x32b_x32(tmem + lane_off + kTX + c * 32, xr);
-        tmem_ld_32x32b_x32(tmem + lane_off + kTY + c * 32, yr);
-        float lv[32], dv[32];   // per-column lse·log2e and D (the streamed queries)
-        if constexpr (kKV) {
-          const float4* l4 = reinterpret_cast<const float4*>(vecL + st * kBQ + c * 32);
-          const float4* d4 = reinterpret_cast<const float4*>(vecD + st * kBQ + c * 32);
+      uint32_t xr[kBG], yr[kBG];
 #pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float4 u = l4[q], w = d4[q];
-            lv[4 * q] = u.x; lv[4 * q + 1] = u.y; lv[4 * q + 2] = u.z; lv[4 * q + 3] = u.w;
-            dv[4 * q] = w.x; dv[4 * q + 1] = w.y; dv[4 * q + 2] = w.z; dv[4 * q + 3] = w.w;
-          }
-        } else {
+      for (int c = 0; c < kBG / 32; ++c) {
+        tmem_ld_32x32b_x32(tmem + lane_off + kTX + wg * kBG + c * 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&xr[c * 32]));
+        tmem_ld_32x32b_x32(tmem + lane_off + kTY + wg * kBG + c * 32,
+                           *reinterpret_cast<uint32_t(*)[32]>(&yr[c * 32]));
+      }
+      tc_wait_ld();
+      tc_fence_before_sync();
+      mbar_arrive(&x_empty[wg]);                   // S and dP read: the MMA may refill them
+      // the P/dS buffer is free once the gradient MMAs of this warpgroup's
+      // previous tile have read it
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pd_empty[wg], (use & 1u) ^ 1u, a.wait_ns,
+                                                     abort_flag))) {
+        ok = false;
+        if constexpr (kKV) continue;
+        break;
+      }
+      // the mask can only cut the tiles that meet the diagonal or the end
+      const bool need_mask =
+          kKV ? ((a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s)
+              : ((a.causal && t0 + kBG - 1 > ft * kBQ) || t0 + kBG > a.s);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            lv[j] = own_l;
-            dv[j] = own_d;
-          }
-        }
-        tc_wait_ld();
-        float p[32], ds[32];
-        if (need_mask) {
+      for (int gr = 0; gr < kBG / 8; ++gr) {       // 16-byte granules of the 128-byte row
+        float p[8], ds[8];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int tpos = t0 + c * 32 + j;      // streamed position of this column
+        for (int t = 0; t < 8; ++t) {
+          const int j = gr * 8 + t;
+          const float lv = kKV ? vL[j] : own_l;
+          const float dv = kKV ? vD[j] : own_d;
+          float pv = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv));
+          if (need_mask) {
+            const int tpos = t0 + j;               // streamed position of this column
             // rows are keys and columns queries (kKV), or the other way round
             const bool masked = tpos >= a.s || (a.causal && (kKV ? tpos < fpos : tpos > fpos));
-            p[j] = masked ? 0.0f : ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[j]));
-            ds[j] = p[j] * (__uint_as_float(yr[j]) - dv[j]);
+            if (masked) pv = 0.0f;
           }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            p[j] = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[j]));
-            ds[j] = p[j] * (__uint_as_float(yr[j]) - dv[j]);
-          }
+          p[t] = pv;
+          ds[t] = pv * (__uint_as_float(yr[j]) - dv);
         }
-        uint8_t* pch = prow + (c >> 1) * kTile;
-        uint8_t* dch = drow + (c >> 1) * kTile;
-#pragma unroll
-        for (int g4 = 0; g4 < 4; ++g4) {
-          const int gr = (c & 1) * 4 + g4;
-          uint4 w;
-          w.x = pack_bf16x2(p[8 * g4 + 0], p[8 * g4 + 1]);
-          w.y = pack_bf16x2(p[8 * g4 + 2], p[8 * g4 + 3]);
-          w.z = pack_bf16x2(p[8 * g4 + 4], p[8 * g4 + 5]);
-          w.w = pack_bf16x2(p[8 * g4 + 6], p[8 * g4 + 7]);
-          *reinterpret_cast<uint4*>(pch + ((gr ^ (r & 7)) << 4)) = w;
-          w.x = pack_bf16x2(ds[8 * g4 + 0], ds[8 * g4 + 1]);
-          w.y = pack_bf16x2(ds[8 * g4 + 2], ds[8 * g4 + 3]);
-          w.z = pack_bf16x2(ds[8 * g4 + 4], ds[8 * g4 + 5]);
-          w.w = pack_bf16x2(ds[8 * g4 + 6], ds[8 * g4 + 7]);
-          *reinterpret_cast<uint4*>(dch + ((gr ^ (r & 7)) << 4)) = w;
+        const int off = (gr ^ (r & 7)) << 4;
+        uint4 w;
+        if constexpr (kKV) {
+          w.x = pack_bf16x2(p[0], p[1]);
+          w.y = pack_bf16x2(p[2], p[3]);
+          w.z = pack_bf16x2(p[4], p[5]);
+          w.w = pack_bf16x2(p[6], p[7]);
+          *reinterpret_cast<uint4*>(prow + off) = w;
         }
+        w.x = pack_bf16x2(ds[0], ds[1]);
+        w.y = pack_bf16x2(ds[2], ds[3]);
+        w.z = pack_bf16x2(ds[4], ds[5]);
+        w.w = pack_bf16x2(ds[6], ds[7]);
+        *reinterpret_cast<uint4*>(drow + off) = w;
       }
-      tc_fence_before_sync();
-      mbar_arrive(xy_empty);
-      fence_proxy_async_smem();
-      mbar_arrive(pd_full);
+      fence_proxy_async_smem();                    // P and dS visible to the tensor core
+      mbar_arrive(&pd_full[wg]);
     }
     // the accumulated gradients of the fixed rows: every lane takes part in
     // the warp-collective tensor-memory loads, only rows inside the sequence
-    // are stored
+    // are stored.  dK/dV kernel: warpgroup 0 stores dK, warpgroup 1 dV; dQ
+    // kernel: each warpgroup stores 32 of the 64 columns.
     const bool done =
         __all_sync(0xffffffffu, ok && mbar_wait_bounded<true>(acc_done, 0, a.wait_ns, abort_flag));
     if (!done) {
@@ -766,26 +775,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     } else {
       tc_fence_after_sync();
       __nv_bfloat16* dst_row = a.dqkv + static_cast<int64_t>(row0 + fpos) * a.ldq;
+      const uint32_t col = (kKV && wg == 1) ? kTA1 : kTA2;
+      const float f = (kKV && wg == 1) ? 1.0f : a.scale;
+      const int c_begin = kKV ? 0 : wg, c_end = kKV ? kHD / 32 : wg + 1;
+      __nv_bfloat16* dst = dst_row + (kKV ? (wg == 0 ? kcol : vcol) : qcol);
+#pragma unroll 1
+      for (int c = c_begin; c < c_end; ++c) {
+        uint32_t rr[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, rr);
+        tc_wait_ld();
 #pragma unroll
-      for (int which = 0; which < (kKV ? 2 : 1); ++which) {
-        // kKV: which 0 -> dK (scaled, acc2), which 1 -> dV (acc1); else dQ (scaled, acc2)
-        const uint32_t col = which == 0 ? kTA2 : kTA1;
-        const float f = which == 0 ? a.scale : 1.0f;
-        __nv_bfloat16* dst = dst_row + (kKV ? (which == 0 ? kcol : vcol) : qcol);
-#pragma unroll
-        for (int c = 0; c < kHD / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, rr);
-          tc_wait_ld();
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            uint4 w;
-            w.x = pack_bf16x2(__uint_as_float(rr[8 * g + 0]) * f, __uint_as_float(rr[8 * g + 1]) * f);
-            w.y = pack_bf16x2(__uint_as_float(rr[8 * g + 2]) * f, __uint_as_float(rr[8 * g + 3]) * f);
-            w.z = pack_bf16x2(__uint_as_float(rr[8 * g + 4]) * f, __uint_as_float(rr[8 * g + 5]) * f);
-            w.w = pack_bf16x2(__uint_as_float(rr[8 * g + 6]) * f, __uint_as_float(rr[8 * g + 7]) * f);
-            if (fpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
-          }
+        for (int g = 0; g < 4; ++g) {
+          uint4 w;
+          w.x = pack_bf16x2(__uint_as_float(rr[8 * g + 0]) * f, __uint_as_float(rr[8 * g + 1]) * f);
+          w.y = pack_bf16x2(__uint_as_float(rr[8 * g + 2]) * f, __uint_as_float(rr[8 * g + 3]) * f);
+          w.z = pack_bf16x2(__uint_as_float(rr[8 * g + 4]) * f, __uint_as_float(rr[8 * g + 5]) * f);
+          w.w = pack_bf16x2(__uint_as_float(rr[8 * g + 6]) * f, __uint_as_float(rr[8 * g + 7]) * f);
+          if (fpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
         }
       }
     }
@@ -885,6 +891,7 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
   a.s = static_cast<int>(s);
   a.heads = heads;
   a.nqb = static_cast<int>((s + kBQ - 1) / kBQ);
+  a.ng = static_cast<int>((s + kBG - 1) / kBG);
   a.causal = causal ? 1 : 0;
   a.scale = scale;
   a.scale_log2 = scale * 1.4426950408889634f;
@@ -905,6 +912,8 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
   if (!make_tmap_bf16_sw128(&prm.tm_qkv, QKV, ncols, rows, ncols, kHD, kBQ)) return TP_ERR_CUDA;
   const uint64_t hcols = static_cast<uint64_t>(heads) * kHD;
   if (!make_tmap_bf16_sw128(&prm.tm_do, dO, hcols, rows, hcols, kHD, kBQ)) return TP_ERR_CUDA;
+  if (!make_tmap_bf16_sw128(&prm.tm_qkv_g, QKV, ncols, rows, ncols, kHD, kBG)) return TP_ERR_CUDA;
+  if (!make_tmap_bf16_sw128(&prm.tm_do_g, dO, hcols, rows, hcols, kHD, kBG)) return TP_ERR_CUDA;
   const int64_t grid = b * heads * a.nqb;
   if (tp_status st = attn_bwd_launch_t<true>(prm, grid, stream)) return st;
   return attn_bwd_launch_t<false>(prm, grid, stream);

@@ -77,6 +77,7 @@ struct GemmArgs {
   const float* row_lse;
   float grad_scale;
   int inject_unit, inject_kb;       // debug: the producer stops before this k-block (-1: never)
+  int a_hint, b_hint;               // L2 policy of the operand loads: 0 none, 1 evict-first, 2 evict-last
 };
 
 struct __align__(64) GemmParams {
@@ -317,6 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     if (elect_one_sync()) {
       tma_prefetch_desc(&P.tmA);
       tma_prefetch_desc(&P.tmB);
+      const uint64_t pol_first = l2_policy_evict_first();
+      const uint64_t pol_last = l2_policy_evict_last();
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
@@ -344,34 +347,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           uint8_t* dB = sB + stage * C::kBBytes;
           if constexpr (CG == 2) {
             const uint32_t bar = mapa_shared(&full[stage], 0);
+            auto load = [&](uint8_t* dst, const CUtensorMap* m, int x, int y, int hint) {
+              if (hint) tma_load_2d_cg2_hint(dst, m, bar, x, y, hint == 1 ? pol_first : pol_last);
+              else tma_load_2d_cg2(dst, m, bar, x, y);
+            };
             if (!a.a_mn) {
-              tma_load_2d_cg2(dA, &P.tmA, bar, k0, a_row);
+              load(dA, &P.tmA, k0, a_row, a.a_hint);
             } else {
 #pragma unroll
-              for (int j = 0; j < BM / 64; ++j)
-                tma_load_2d_cg2(dA + j * 8192, &P.tmA, bar, a_row + j * 64, k0);
+              for (int j = 0; j < BM / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
             }
             if (!a.b_mn) {
-              tma_load_2d_cg2(dB, &P.tmB, bar, k0, b_col);
+              load(dB, &P.tmB, k0, b_col, a.b_hint);
             } else {
 #pragma unroll
               for (int j = 0; j < C::kBCols / 64; ++j)
-                tma_load_2d_cg2(dB + j * 8192, &P.tmB, bar, b_col + j * 64, k0);
+                load(dB + j * 8192, &P.tmB, b_col + j * 64, k0, a.b_hint);
             }
           } else {
+            auto load = [&](uint8_t* dst, const CUtensorMap* m, int x, int y, int hint) {
+              if (hint) tma_load_2d_hint(dst, m, &full[stage], x, y, hint == 1 ? pol_first : pol_last);
+              else tma_load_2d(dst, m, &full[stage], x, y);
+            };
             if (!a.a_mn) {
-              tma_load_2d(dA, &P.tmA, &full[stage], k0, a_row);
+              load(dA, &P.tmA, k0, a_row, a.a_hint);
             } else {
 #pragma unroll
-              for (int j = 0; j < BM / 64; ++j)
-                tma_load_2d(dA + j * 8192, &P.tmA, &full[stage], a_row + j * 64, k0);
+              for (int j = 0; j < BM / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
             }
             if (!a.b_mn) {
-              tma_load_2d(dB, &P.tmB, &full[stage], k0, b_col);
+              load(dB, &P.tmB, k0, b_col, a.b_hint);
             } else {
 #pragma unroll
               for (int j = 0; j < C::kBCols / 64; ++j)
-                tma_load_2d(dB + j * 8192, &P.tmB, &full[stage], b_col + j * 64, k0);
+                load(dB + j * 8192, &P.tmB, b_col + j * 64, k0, a.b_hint);
             }
           }
           ++issued;
@@ -898,6 +907,21 @@ void take_injection(int& unit, int& kb, uint64_t& wait_ns) {
   g_inject_armed = false;
 }
 
+// L2 eviction policies of the two operands.  TP_GEMM_L2HINT=<a><b> with
+// n (none), f (evict first) or l (evict last) for each operand overrides
+// the choice (sweeps).
+void choose_l2_hints(const GemmProblem& p, int& a_hint, int& b_hint) {
+  a_hint = 0;
+  b_hint = 0;
+  if (const char* e = std::getenv("TP_GEMM_L2HINT")) {
+    auto code = [](char c) { return c == 'f' ? 1 : c == 'l' ? 2 : 0; };
+    if (e[0] && e[1]) {
+      a_hint = code(e[0]);
+      b_hint = code(e[1]);
+    }
+  }
+}
+
 struct TileChoice {
   int cg;    // CTAs per tile (1, or a cluster pair with cta_group::2)
   int bn;    // output columns per tile (256 or 128)
@@ -1034,6 +1058,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.grad_scale = p.grad_scale;
   a.inject_unit = -1;
   a.inject_kb = -1;
+  choose_l2_hints(p, a.a_hint, a.b_hint);
   take_injection(a.inject_unit, a.inject_kb, a.wait_ns);
   if ((p.epi == EPI_XENT_STATS || p.epi == EPI_XENT_GRAD) && p.splits != 1) return TP_ERR_UNSUPPORTED;
   if (split_epi) {

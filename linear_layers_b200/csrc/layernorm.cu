@@ -202,14 +202,24 @@ __global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
   if (row >= M) return;   // whole warps only
   float hv[CH][8];
   float s = 0.0f;
+  // every load of the row first, so that all of them are in flight together
+  uint4 xw[CH], rw[CH];
+#pragma unroll
+  for (int k = 0; k < CH; ++k) {
+    const int c = lane + 32 * k;
+    if (c < h8) {
+      xw[k] = __ldcs(x + row * h8 + c);
+      rw[k] = __ldcs(residual + row * h8 + c);
+    }
+  }
 #pragma unroll
   for (int k = 0; k < CH; ++k) {
     const int c = lane + 32 * k;
     if (c < h8) {
       const int64_t o = row * h8 + c;
       float xv[8], rv[8], bv[8];
-      unpack8(__ldcs(x + o), xv);
-      unpack8(__ldcs(residual + o), rv);
+      unpack8(xw[k], xv);
+      unpack8(rw[k], rv);
       if (bias) {
         unpack8(__ldg(bias + c), bv);
       } else {
@@ -269,70 +279,97 @@ __global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
 // and dx stay in registers across rows; they are written as this block's
 // partial and summed over blocks in block order afterwards.
 template <int CH>
-__global__ void __launch_bounds__(kLnThreads, CH == 1 ? 8 : CH == 2 ? 5 : CH == 4 ? 3 : 1) sp_ln_bwd_kernel(
+__global__ void __launch_bounds__(kLnThreads, CH == 1 ? 6 : CH == 2 ? 4 : CH == 4 ? 2 : 1) sp_ln_bwd_kernel(
     const uint4* __restrict__ dy, const uint4* __restrict__ dhs_in, const uint4* __restrict__ hs,
     const uint4* __restrict__ gamma, const float* __restrict__ mean, const float* __restrict__ rstd,
     int64_t M, int h8, float inv_h, DropoutRng rng, uint4* __restrict__ dx,
     uint4* __restrict__ dresidual, float* __restrict__ part_gamma, float* __restrict__ part_beta,
     float* __restrict__ part_bias) {
-  __shared__ float red[2][kLnThreads / 32];
+  __shared__ float red[4][kLnThreads / 32];
   float ag[CH][8], ab[CH][8], ax[CH][8];   // this block's column sums
 #pragma unroll
   for (int k = 0; k < CH; ++k)
 #pragma unroll
     for (int i = 0; i < 8; ++i) ag[k][i] = ab[k][i] = ax[k][i] = 0.0f;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kLnBwdRows;
-  for (int rr = 0; rr < kLnBwdRows; ++rr) {
-    const int64_t row = r0 + rr;
-    if (row >= M) break;   // uniform across the block
-    const float mu = mean[row], rs = rstd[row];
-    float sums[2] = {0.0f, 0.0f};   // Σ g, Σ g·xhat
+  // up to two rows per iteration (RPI): their loads are in flight together
+  // and their reductions share one pair of block barriers; the widest rows
+  // take one at a time to stay within the registers
+  constexpr int RPI = CH <= 4 ? 2 : 1;
+  for (int rr = 0; rr < kLnBwdRows; rr += RPI) {
+    const int64_t rowA = r0 + rr;
+    if (rowA >= M) break;   // uniform across the block
+    const int nrows = RPI == 2 && rowA + 1 < M ? 2 : 1;
+    float mu[RPI], rs[RPI];
+    float sums[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // per row: Σ g, Σ g·xhat
 #pragma unroll
-    for (int k = 0; k < CH; ++k) {
-      const int c = threadIdx.x + k * kLnThreads;
-      if (c < h8) {
-        const int64_t o = row * h8 + c;
-        float hv[8], dv[8], gv[8];
-        unpack8(__ldg(hs + o), hv);
-        unpack8(__ldg(dy + o), dv);
-        unpack8(__ldg(gamma + c), gv);
+    for (int q = 0; q < RPI; ++q) {
+      mu[q] = q < nrows ? mean[rowA + q] : 0.0f;
+      rs[q] = q < nrows ? rstd[rowA + q] : 0.0f;
+    }
+    uint4 hw[RPI][CH], dw[RPI][CH];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float g = dv[i] * gv[i];
-          sums[0] += g;
-          sums[1] = fmaf(g, (hv[i] - mu) * rs, sums[1]);
+    for (int q = 0; q < RPI; ++q)
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int c = threadIdx.x + k * kLnThreads;
+        if (q < nrows && c < h8) {
+          hw[q][k] = __ldg(hs + (rowA + q) * h8 + c);
+          dw[q][k] = __ldg(dy + (rowA + q) * h8 + c);
         }
       }
-    }
-    block_sum<2>(sums, red);
-    const float mg = sums[0] * inv_h, mgx = sums[1] * inv_h;
 #pragma unroll
-    for (int k = 0; k < CH; ++k) {
-      const int c = threadIdx.x + k * kLnThreads;
-      if (c < h8) {
-        const int64_t o = row * h8 + c;
-        float hv[8], dv[8], gv[8], din[8], d[8], dxv[8];
-        unpack8(__ldg(hs + o), hv);
-        unpack8(__ldg(dy + o), dv);
-        unpack8(__ldg(gamma + c), gv);
-        if (dhs_in) {
-          unpack8(__ldcs(dhs_in + o), din);
-        } else {
+    for (int q = 0; q < RPI; ++q)
 #pragma unroll
-          for (int i = 0; i < 8; ++i) din[i] = 0.0f;
+      for (int k = 0; k < CH; ++k) {
+        const int c = threadIdx.x + k * kLnThreads;
+        if (q < nrows && c < h8) {
+          float hv[8], dv[8], gv[8];
+          unpack8(hw[q][k], hv);
+          unpack8(dw[q][k], dv);
+          unpack8(__ldg(gamma + c), gv);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float g = dv[i] * gv[i];
+            sums[2 * q] += g;
+            sums[2 * q + 1] = fmaf(g, (hv[i] - mu[q]) * rs[q], sums[2 * q + 1]);
+          }
         }
-        const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+      }
+    block_sum<2 * RPI>(*reinterpret_cast<float(*)[2 * RPI]>(sums), red);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float xh = (hv[i] - mu) * rs;
-          d[i] = fmaf(rs, dv[i] * gv[i] - mg - xh * mgx, din[i]);
-          dxv[i] = ((kb >> i) & 1u) ? d[i] * rng.inv_keep : 0.0f;
-          ag[k][i] = fmaf(dv[i], xh, ag[k][i]);
-          ab[k][i] += dv[i];
-          ax[k][i] += dxv[i];
+    for (int q = 0; q < RPI; ++q) {
+      if (q >= nrows) break;   // uniform
+      const int64_t row = rowA + q;
+      const float mg = sums[2 * q] * inv_h, mgx = sums[2 * q + 1] * inv_h;
+#pragma unroll
+      for (int k = 0; k < CH; ++k) {
+        const int c = threadIdx.x + k * kLnThreads;
+        if (c < h8) {
+          const int64_t o = row * h8 + c;
+          float hv[8], dv[8], gv[8], din[8], d[8], dxv[8];
+          unpack8(hw[q][k], hv);
+          unpack8(dw[q][k], dv);
+          unpack8(__ldg(gamma + c), gv);
+          if (dhs_in) {
+            unpack8(__ldcs(dhs_in + o), din);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) din[i] = 0.0f;
+          }
+          const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float xh = (hv[i] - mu[q]) * rs[q];
+            d[i] = fmaf(rs[q], dv[i] * gv[i] - mg - xh * mgx, din[i]);
+            dxv[i] = ((kb >> i) & 1u) ? d[i] * rng.inv_keep : 0.0f;
+            ag[k][i] = fmaf(dv[i], xh, ag[k][i]);
+            ab[k][i] += dv[i];
+            ax[k][i] += dxv[i];
+          }
+          __stcs(dresidual + o, pack8(d));
+          __stcs(dx + o, pack8(dxv));
         }
-        __stcs(dresidual + o, pack8(d));
-        __stcs(dx + o, pack8(dxv));
       }
     }
   }

@@ -250,38 +250,27 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
     const float tgt_i =
         (mine && threadIdx.x == 0) ? reinterpret_cast<const float*>(buf4)[y - lo] : 0.0f;
 
-    // 1) shard maximum
+    // 1) each warp's maximum, the first position of it, e = exp(l − m_w) kept
+    //    in registers and the warp's sum: one warp-level pass, no barrier
     float mt = max4(x[0]);
 #pragma unroll
     for (int r = 1; r < R; ++r) mt = fmaxf(mt, max4(x[r]));
-    float wm = mt;
+    float m_w = mt;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, off));
-    if (lane == 0) red_m2[p][warp] = wm;
-    __syncthreads();   // also: every thread has its slice in registers
-    if (threadIdx.x == 0 && tok + 2 * nclusters < T) {   // refill two tokens ahead
-      fence_proxy_async_smem();
-      issue(p, tok + 2 * nclusters);
-    }
-    float m_i = red_m2[p][0];
-#pragma unroll
-    for (int w = 1; w < NT / 32; ++w) m_i = fmaxf(m_i, red_m2[p][w]);
-
-    // 2) first position of the maximum (only threads that hold it search)
+    for (int off = 16; off >= 1; off >>= 1) m_w = fmaxf(m_w, __shfl_xor_sync(0xffffffffu, m_w, off));
     int it = 0x7fffffff;
-    if (mt == m_i) {
+    if (mt == m_w) {   // only lanes holding the warp maximum search
 #pragma unroll
       for (int r = R - 1; r >= 0; --r) {   // elements ascend with r: keep the lowest
         const int j = threadIdx.x + r * NT;
-        if (x[r].w == m_i) it = 4 * j + 3;
-        if (x[r].z == m_i) it = 4 * j + 2;
-        if (x[r].y == m_i) it = 4 * j + 1;
-        if (x[r].x == m_i) it = 4 * j;
+        if (x[r].w == m_w) it = 4 * j + 3;
+        if (x[r].z == m_w) it = 4 * j + 2;
+        if (x[r].y == m_w) it = 4 * j + 1;
+        if (x[r].x == m_w) it = 4 * j;
       }
     }
-
-    // 3) e = exp(l − m_i) kept in registers, and the shard's sum
-    const float mL = m_i * kLog2e;
+    // a warp whose elements are all padding (−inf) contributes nothing
+    const float mL = m_w == -CUDART_INF_F ? 0.0f : m_w * kLog2e;
     float st = 0.f;
 #pragma unroll
     for (int r = 0; r < R; ++r) {
@@ -297,16 +286,27 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
       it = min(it, __shfl_xor_sync(0xffffffffu, it, off));
     }
     if (lane == 0) {
+      red_m2[p][warp] = m_w;
       red_s2[p][warp] = st;
       red_i2[p][warp] = it;
     }
-    __syncthreads();
+    __syncthreads();   // also: every thread has its slice in registers
+    if (threadIdx.x == 0 && tok + 2 * nclusters < T) {   // refill two tokens ahead
+      fence_proxy_async_smem();
+      issue(p, tok + 2 * nclusters);
+    }
+    // 2) the shard's record from the warps' in a fixed order:
+    //    m_i = max m_w, s_i = Σ s_w·exp(m_w − m_i), first position of m_i
+    float m_i = red_m2[p][0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) m_i = fmaxf(m_i, red_m2[p][w]);
     float s_i = 0.f;
     int a_i = 0x7fffffff;
 #pragma unroll
-    for (int w = 0; w < NT / 32; ++w) {   // fixed order
-      s_i += red_s2[p][w];
-      a_i = min(a_i, red_i2[p][w]);
+    for (int w = 0; w < NT / 32; ++w) {
+      const float mw = red_m2[p][w];
+      if (mw != -CUDART_INF_F) s_i += red_s2[p][w] * ex2_approx((mw - m_i) * kLog2e);
+      if (mw == m_i) a_i = min(a_i, red_i2[p][w]);
     }
 
     // 4) send this shard's record to every shard of the cluster (itself included)
@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
 
     // 6) dlogits block = grad_scale · (e · exp(m_i − lse) − onehot)
     if (need_grad) {
-      const float scale = y_ok ? grad_scale * ex2_approx((m_i - lse) * kLog2e) : CUDART_NAN_F;
+      const float scale = y_ok ? grad_scale * ex2_approx((m_w - lse) * kLog2e) : CUDART_NAN_F;
       GT* dst = dlogits + tok * v + lo;
       const int yl = mine ? static_cast<int>(y - lo) : -1;
 #pragma unroll
