@@ -158,7 +158,7 @@ __device__ __forceinline__ void attn_timeout(const AttnArgs& a, volatile int* ab
   }
 }
 
-__global__ void __maxnreg__(200) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
+__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -493,7 +493,7 @@ __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* 
 }
 
 template <bool kKV>
-__global__ void __maxnreg__(200) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
+__global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -677,17 +677,27 @@ __global__ void __maxnreg__(200) attn_bwd_kernel(const __grid_constant__ AttnBwd
     uint8_t* prow = sP + wg * kPTile + r * 128;
     uint8_t* drow = sDS + wg * kPTile + r * 128;
     bool ok = true;
+    // lse·log2e and D of the streamed queries (dK/dV kernel): thread et < 64
+    // loads those of query et of a tile one tile ahead of its use, so the
+    // global loads are in flight while the warpgroup works on a tile
+    float nl = 0.0f, nd = 0.0f;
+    auto fetch_vec = [&](int tile) {
+      const int q = (t_begin + tile) * kBG + et;
+      nl = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
+      nd = q < a.s ? a.D[sbase + q] : 0.0f;
+    };
+    if (kKV && et < kBG && wg < nt) fetch_vec(wg);
     for (int it = wg; it < nt; it += 2) {
       const uint32_t use = static_cast<uint32_t>(it >> 1);   // this warpgroup's tile count
       const int t0 = (t_begin + it) * kBG;         // first position of the streamed tile
       const float* vL = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
       const float* vD = vL + kBG;
-      if constexpr (kKV) {   // lse·log2e and D of the streamed queries
+      if constexpr (kKV) {
         if (et < kBG) {
-          const int q = t0 + et;
           float* w = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
-          w[et] = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
-          w[kBG + et] = q < a.s ? a.D[sbase + q] : 0.0f;
+          w[et] = nl;
+          w[kBG + et] = nd;
+          if (it + 2 < nt) fetch_vec(it + 2);
         }
         // one barrier per tile that also carries every thread's state, so all
         // 128 threads of the warpgroup leave together and none is left in it

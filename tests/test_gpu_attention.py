@@ -111,8 +111,10 @@ def test_attention_layer_chain():
     rctx, _ = O.attention_sharded(rQKV, b, s, nh, HD, shards, causal=True)
     rZ, _ = O.row_linear_fwd(rctx, inp["Wo"], offsets=ctx_offs)
     assert_close("QKV", QKV, rQKV, TOL_BF16)
-    assert_close("ctx", ctx, rctx, TOL_BF16)
-    assert_close("Z", Z, rZ, TOL_BF16)
+    # ctx and Z are taken from the bf16-rounded QKV (the oracle's stays
+    # fp64) and the softmax amplifies that rounding: twice the bound per element
+    assert_close("ctx", ctx, rctx, TOL_BF16, elem_tol=2 * TOL_BF16)
+    assert_close("Z", Z, rZ, TOL_BF16, elem_tol=2 * TOL_BF16)
 
 
 def test_attention_deterministic():
@@ -125,6 +127,17 @@ def test_attention_deterministic():
 
 
 # ---------------------------------------------------------------- backward
+def _bwd_elem_tol(causal):
+    """Per-element bound of the backward's gradients.  P and dS enter their
+    products rounded to bf16; under the causal mask the first rows of a
+    sequence sum over a handful of keys, so that rounding does not average
+    out there.  Emulating exactly those rounding points in float64 (one
+    head, s=1024, three seeds) gives relative Frobenius errors of 2.5e-3 and
+    worst elements of up to 6.8e-2 causal, 1.7e-2 not causal: the causal
+    bound is 0.1, still far below the ~1 of an element that is wrong."""
+    return 5 * TOL_BF16 if causal else TOL_BF16
+
+
 def _bwd_check(b, s, nh, N, causal, seed, offs=None, scale=None):
     QKV = _qkv(b, s, nh, seed=seed)
     g = torch.Generator().manual_seed(seed + 1)
@@ -145,7 +158,8 @@ def _bwd_check(b, s, nh, N, causal, seed, offs=None, scale=None):
         rows = slice(bb * s, (bb + 1) * s)
         for c0 in range(0, 3 * nh * HD, HD):     # every head's Q, K and V block
             cols = slice(c0, c0 + HD)
-            assert_close(f"dQKV[b={bb},cols={c0}]", got[rows, cols], ref[rows, cols], TOL_BF16)
+            assert_close(f"dQKV[b={bb},cols={c0}]", got[rows, cols], ref[rows, cols], TOL_BF16,
+                         elem_tol=_bwd_elem_tol(causal))
     return dQKV
 
 
@@ -181,4 +195,4 @@ def test_attention_backward_gpt2_slice():
     assert int(st.item()) == 0
     shards = tp_inputs.head_split(nh, N)
     ref = O.attention_sharded_bwd(QKV[:s], dctx[:s], 1, s, nh, HD, shards, causal=True)
-    assert_close("dQKV[b=0]", dQKV[:s], ref, TOL_BF16)
+    assert_close("dQKV[b=0]", dQKV[:s], ref, TOL_BF16, elem_tol=_bwd_elem_tol(True))

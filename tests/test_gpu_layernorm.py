@@ -65,15 +65,17 @@ def test_layernorm_against_oracle(M, h, N, p, use_dhs, with_bias):
     assert_close("hs", f["hs"], ref["hs"], TOL_BF16)
     assert_close("y", f["y"], ref["y"], TOL_BF16)
     assert_close("mean", f["mean"], ref["mean"], TOL_MEAN)
-    assert_close("rstd", f["rstd"], ref["rstd"], TOL_STAT)
+    # per element twice TOL_STAT: a row of 8 values (the smallest case) has
+    # the statistics of 8 bf16-rounded hs values
+    assert_close("rstd", f["rstd"], ref["rstd"], TOL_STAT, elem_tol=2 * TOL_STAT)
     rb = O.dropout_add_layernorm_bwd_sharded(d["dy"], d["dhs"] if use_dhs else None, ref["hs"],
                                              d["gamma"], ref["mean"], ref["rstd"], ref["keep"], p, N)
     assert_close("dx", b["dx"], rb["dx"], TOL_BF16)
     assert_close("dresidual", b["dresidual"], rb["dresidual"], TOL_BF16)
-    assert_close("dgamma", b["dgamma"], rb["dgamma"], TOL_PGRAD)
-    assert_close("dbeta", b["dbeta"], rb["dbeta"], TOL_PGRAD)
+    assert_close("dgamma", b["dgamma"], rb["dgamma"], TOL_PGRAD, elem_tol=TOL_BF16)
+    assert_close("dbeta", b["dbeta"], rb["dbeta"], TOL_PGRAD, elem_tol=TOL_BF16)
     if with_bias:
-        assert_close("dbias", b["dbias"], rb["dbias"], TOL_PGRAD)
+        assert_close("dbias", b["dbias"], rb["dbias"], TOL_PGRAD, elem_tol=TOL_BF16)
 
 
 def test_dropout_mask_depends_only_on_seed_and_offset():
@@ -101,7 +103,7 @@ def test_layernorm_gpt2_slice_full():
     rb = O.dropout_add_layernorm_bwd(d["dy"], d["dhs"], ref["hs"], d["gamma"], ref["mean"],
                                      ref["rstd"], ref["keep"], p)
     assert_close("dx", b["dx"], rb["dx"], TOL_BF16)
-    assert_close("dgamma", b["dgamma"], rb["dgamma"], TOL_PGRAD)
+    assert_close("dgamma", b["dgamma"], rb["dgamma"], TOL_PGRAD, elem_tol=TOL_BF16)
 
 
 def test_layernorm_deterministic():

@@ -127,8 +127,11 @@ def test_linear_xent_backward_chain():
     torch.cuda.synchronize()
     ref = O.linear_xent(H, E, y, grad_scale=1.0 / T)
     g = O.logits_bwd(ref["dlogits"], H, E)
-    assert_close("dH", dH, g["dH"], TOL_BF16)
-    assert_close("dE", dE, g["dE"], TOL_BF16)
+    # dH and dE contract the bf16-rounded dlogits (the oracle's stay fp64):
+    # per tensor the stated 2e-2, per element twice that for the rounding
+    # the chain adds before the contraction
+    assert_close("dH", dH, g["dH"], TOL_BF16, elem_tol=2 * TOL_BF16)
+    assert_close("dE", dE, g["dE"], TOL_BF16, elem_tol=2 * TOL_BF16)
 
 
 @pytest.mark.slow
