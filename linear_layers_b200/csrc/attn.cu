@@ -492,6 +492,66 @@ __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* 
   }
 }
 
+// One fixed row of a streamed tile: p = 2^(x·sl − l) (zero where masked) and
+// dS = p·(y − D), written as bf16 into the row's 128-byte lines of the P
+// (dK/dV kernel only) and dS tiles, granule g at g ^ (row & 7).  The dK/dV
+// kernel takes l and D per column from shared memory (four at a time), the
+// dQ kernel has one pair for its row.
+template <bool kKV, bool kMask>
+__device__ __forceinline__ void bwd_tile_rows(const uint32_t (&xr)[kBG], const uint32_t (&yr)[kBG],
+                                              const float* vL, const float* vD, float own_l,
+                                              float own_d, float sl, int t0, int fpos, int s,
+                                              int causal, uint8_t* prow, uint8_t* drow, int r) {
+#pragma unroll
+  for (int gr = 0; gr < kBG / 8; ++gr) {       // 16-byte granules of the 128-byte row
+    float lv[8], dv[8];
+    if constexpr (kKV) {
+      const float4 l0 = reinterpret_cast<const float4*>(vL)[2 * gr];
+      const float4 l1 = reinterpret_cast<const float4*>(vL)[2 * gr + 1];
+      const float4 d0 = reinterpret_cast<const float4*>(vD)[2 * gr];
+      const float4 d1 = reinterpret_cast<const float4*>(vD)[2 * gr + 1];
+      lv[0] = l0.x; lv[1] = l0.y; lv[2] = l0.z; lv[3] = l0.w;
+      lv[4] = l1.x; lv[5] = l1.y; lv[6] = l1.z; lv[7] = l1.w;
+      dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w;
+      dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
+    } else {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        lv[t] = own_l;
+        dv[t] = own_d;
+      }
+    }
+    float p[8], ds[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      const int j = gr * 8 + t;
+      float pv = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[t]));
+      if constexpr (kMask) {
+        const int tpos = t0 + j;               // streamed position of this column
+        // rows are keys and columns queries (kKV), or the other way round
+        const bool masked = tpos >= s || (causal && (kKV ? tpos < fpos : tpos > fpos));
+        pv = masked ? 0.0f : pv;
+      }
+      p[t] = pv;
+      ds[t] = pv * (__uint_as_float(yr[j]) - dv[t]);
+    }
+    const int off = (gr ^ (r & 7)) << 4;
+    uint4 w;
+    if constexpr (kKV) {
+      w.x = pack_bf16x2(p[0], p[1]);
+      w.y = pack_bf16x2(p[2], p[3]);
+      w.z = pack_bf16x2(p[4], p[5]);
+      w.w = pack_bf16x2(p[6], p[7]);
+      *reinterpret_cast<uint4*>(prow + off) = w;
+    }
+    w.x = pack_bf16x2(ds[0], ds[1]);
+    w.y = pack_bf16x2(ds[2], ds[3]);
+    w.z = pack_bf16x2(ds[4], ds[5]);
+    w.w = pack_bf16x2(ds[6], ds[7]);
+    *reinterpret_cast<uint4*>(drow + off) = w;
+  }
+}
+
 template <bool kKV>
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
   extern __shared__ uint8_t smem_raw[];
@@ -738,39 +798,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       const bool need_mask =
           kKV ? ((a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s)
               : ((a.causal && t0 + kBG - 1 > ft * kBQ) || t0 + kBG > a.s);
-#pragma unroll
-      for (int gr = 0; gr < kBG / 8; ++gr) {       // 16-byte granules of the 128-byte row
-        float p[8], ds[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int j = gr * 8 + t;
-          const float lv = kKV ? vL[j] : own_l;
-          const float dv = kKV ? vD[j] : own_d;
-          float pv = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv));
-          if (need_mask) {
-            const int tpos = t0 + j;               // streamed position of this column
-            // rows are keys and columns queries (kKV), or the other way round
-            const bool masked = tpos >= a.s || (a.causal && (kKV ? tpos < fpos : tpos > fpos));
-            if (masked) pv = 0.0f;
-          }
-          p[t] = pv;
-          ds[t] = pv * (__uint_as_float(yr[j]) - dv);
-        }
-        const int off = (gr ^ (r & 7)) << 4;
-        uint4 w;
-        if constexpr (kKV) {
-          w.x = pack_bf16x2(p[0], p[1]);
-          w.y = pack_bf16x2(p[2], p[3]);
-          w.z = pack_bf16x2(p[4], p[5]);
-          w.w = pack_bf16x2(p[6], p[7]);
-          *reinterpret_cast<uint4*>(prow + off) = w;
-        }
-        w.x = pack_bf16x2(ds[0], ds[1]);
-        w.y = pack_bf16x2(ds[2], ds[3]);
-        w.z = pack_bf16x2(ds[4], ds[5]);
-        w.w = pack_bf16x2(ds[6], ds[7]);
-        *reinterpret_cast<uint4*>(drow + off) = w;
-      }
+      if (need_mask)
+        bwd_tile_rows<kKV, true>(xr, yr, vL, vD, own_l, own_d, sl, t0, fpos, a.s, a.causal, prow,
+                                 drow, r);
+      else
+        bwd_tile_rows<kKV, false>(xr, yr, vL, vD, own_l, own_d, sl, t0, fpos, a.s, a.causal,
+                                  prow, drow, r);
       fence_proxy_async_smem();                    // P and dS visible to the tensor core
       mbar_arrive(&pd_full[wg]);
     }

@@ -94,14 +94,13 @@ struct Cfg {
   static constexpr int kBCols = BNT / CG;        // B columns staged per CTA
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr uint32_t kBBytes = kBCols * BK * 2;
-  // 192 KB of operand stages: 6 (2 x 256), 4 (1 x 256), 8 (2 x 128), 6 (1 x 128)
-  static constexpr int kStages = static_cast<int>(196608u / (kABytes + kBBytes));
+  // 224 KB of operand stages: 7 (2 x 256), 4 (1 x 256), 9 (2 x 128), 7 (1 x 128)
+  static constexpr int kStages = static_cast<int>(229376u / (kABytes + kBBytes));
   static constexpr uint32_t kOffB = kStages * kABytes;
   static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;
-  static constexpr uint32_t kBytes = kOffRed + 4 * BNT * 4;
+  static constexpr uint32_t kBytes = kOffMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators
   static constexpr int kChunks = BNT / 64;            // 32-column chunks per epilogue warp
@@ -282,7 +281,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* bcast = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
-  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -381,6 +379,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
               for (int j = 0; j < C::kBCols / 64; ++j)
                 load(dB + j * 8192, &P.tmB, b_col + j * 64, k0, a.b_hint);
+            }
+          }
+          // L2 prefetch of the k-block one ring length ahead in this unit:
+          // by the time its load is issued it waits in L2, not in HBM
+          const int kbp = kb + STAGES;
+          if (kbp < a.split_kb[s + 1]) {
+            const int kp = kbp * BK;
+            if (!a.a_mn) {
+              tma_prefetch_l2_2d(&P.tmA, kp, a_row);
+            } else {
+#pragma unroll
+              for (int j = 0; j < BM / 64; ++j) tma_prefetch_l2_2d(&P.tmA, a_row + j * 64, kp);
+            }
+            if (!a.b_mn) {
+              tma_prefetch_l2_2d(&P.tmB, kp, b_col);
+            } else {
+#pragma unroll
+              for (int j = 0; j < C::kBCols / 64; ++j) tma_prefetch_l2_2d(&P.tmB, b_col + j * 64, kp);
             }
           }
           ++issued;
@@ -754,22 +770,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                               a.N - col0);
             }
             if (a.dbias_part != nullptr) {
+              // this warp's 32 rows: one partial row of the 32-row tiling,
+              // written only when it holds rows of the problem (rows past M
+              // contribute zeros and have no partial row)
               const float colsum = warp_column_sums(v, lane);
-              red[q * BNT + c * 32 + lane] = colsum;
+              const int prow = (tm * CG + static_cast<int>(rank)) * 4 + q;
+              if (prow * 32 < a.M && col0 + lane < a.N)
+                a.dbias_part[static_cast<int64_t>(prow) * a.N + col0 + lane] = colsum;
             }
-          }
-        }
-        if constexpr (kDact) {
-          if (a.dbias_part != nullptr) {
-            named_barrier_sync(1, kEpiThreads);
-            const int cc = et;   // one column per epilogue thread (BNT <= 256 columns)
-            const int col = tn * BNT + cc;
-            if (cc < BNT && col < a.N) {
-              // fixed order over the four row quarters of the half tile
-              const float sum = ((red[cc] + red[BNT + cc]) + red[2 * BNT + cc]) + red[3 * BNT + cc];
-              a.dbias_part[static_cast<int64_t>(tm * CG + static_cast<int>(rank)) * a.N + col] = sum;
-            }
-            named_barrier_sync(1, kEpiThreads);
           }
         }
       }

@@ -254,6 +254,15 @@ __device__ __forceinline__ void tma_load_2d_cg2(void* smem_dst, const CUtensorMa
       : "memory");
 }
 
+// Bring the box at (x, y) of a tensor map into L2 (no shared memory, no
+// completion): a later TMA load of the same box then hits L2.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 // L2 eviction policies for the cache-hinted TMA loads below.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t p;

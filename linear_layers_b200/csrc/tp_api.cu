@@ -351,8 +351,7 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   const bool bf16 = dt == TP_DTYPE_BF16;
   cudaStream_t st = as_stream(stream);
 
-  const int tile_rows = bf16 ? 128 : 32;
-  const int64_t mtiles = (M + tile_rows - 1) / tile_rows;
+  const int64_t mtiles = (M + 31) / 32;   // dbias partial rows: one per 32 token rows
   const size_t split_bytes = bf16 ? row_split_ws(M, h, F, N, false) : 0;
   const size_t dbias_bytes = dbias ? dbias_ws(M, F) : 0;
   if (split_bytes + dbias_bytes > 0 && (ws == nullptr || ws_bytes < split_bytes + dbias_bytes))
