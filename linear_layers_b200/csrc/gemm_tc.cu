@@ -39,6 +39,10 @@
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
+#ifndef TP_GEMM_STAGE_BUDGET
+#define TP_GEMM_STAGE_BUDGET 229376u
+#endif
+
 namespace tpl {
 
 namespace {
@@ -78,6 +82,7 @@ struct GemmArgs {
   float grad_scale;
   int inject_unit, inject_kb;       // debug: the producer stops before this k-block (-1: never)
   int a_hint, b_hint;               // L2 policy of the operand loads: 0 none, 1 evict-first, 2 evict-last
+  int l2_prefetch;                  // prefetch the k-block one ring ahead into L2
 };
 
 struct __align__(64) GemmParams {
@@ -94,8 +99,9 @@ struct Cfg {
   static constexpr int kBCols = BNT / CG;        // B columns staged per CTA
   static constexpr uint32_t kABytes = BM * BK * 2;
   static constexpr uint32_t kBBytes = kBCols * BK * 2;
-  // 224 KB of operand stages: 7 (2 x 256), 4 (1 x 256), 9 (2 x 128), 7 (1 x 128)
-  static constexpr int kStages = static_cast<int>(229376u / (kABytes + kBBytes));
+  // TP_GEMM_STAGE_BUDGET bytes of operand stages (default 224 KB: 7 stages of
+  // the 2 x 256 tile, 4 of 1 x 256, 9 of 2 x 128, 7 of 1 x 128)
+  static constexpr int kStages = static_cast<int>(TP_GEMM_STAGE_BUDGET / (kABytes + kBBytes));
   static constexpr uint32_t kOffB = kStages * kABytes;
   static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
@@ -384,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           // L2 prefetch of the k-block one ring length ahead in this unit:
           // by the time its load is issued it waits in L2, not in HBM
           const int kbp = kb + STAGES;
-          if (kbp < a.split_kb[s + 1]) {
+          if (a.l2_prefetch && kbp < a.split_kb[s + 1]) {
             const int kp = kbp * BK;
             if (!a.a_mn) {
               tma_prefetch_l2_2d(&P.tmA, kp, a_row);
@@ -1070,6 +1076,10 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.inject_unit = -1;
   a.inject_kb = -1;
   choose_l2_hints(p, a.a_hint, a.b_hint);
+  {
+    const char* e = std::getenv("TP_GEMM_L2PREFETCH");   // sweeps: 1 turns the prefetch on
+    a.l2_prefetch = (e && e[0] == '1') ? 1 : 0;
+  }
   take_injection(a.inject_unit, a.inject_kb, a.wait_ns);
   if ((p.epi == EPI_XENT_STATS || p.epi == EPI_XENT_GRAD) && p.splits != 1) return TP_ERR_UNSUPPORTED;
   if (split_epi) {
