@@ -39,6 +39,12 @@
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
+// per-SM throughput of the tall tile relative to the 256 x 256 pair tile
+// (below 1 keeps it off the default choice until measured)
+#ifndef TP_GEMM_TALL_EFF
+#define TP_GEMM_TALL_EFF 0.9
+#endif
+
 #ifndef TP_GEMM_STAGE_BUDGET
 #define TP_GEMM_STAGE_BUDGET 229376u
 #endif
@@ -47,7 +53,8 @@ namespace tpl {
 
 namespace {
 
-constexpr int BM = 128;              // rows of A per CTA
+constexpr int BM = 128;              // rows of A per CTA row half
+constexpr double kTallEfficiency = TP_GEMM_TALL_EFF;
 constexpr int BN = 256;              // output columns of the widest tile
 constexpr int BK = 64;               // bf16 elements per k-block (one 128-byte swizzle row)
 constexpr int kEpiWarps = 8;
@@ -92,15 +99,21 @@ struct __align__(64) GemmParams {
 };
 
 // Tile configurations: CG CTAs (1 or 2, a cluster pair with cta_group::2)
-// compute a (128·CG) x BNT output tile, BNT = 256 or 128 columns.
-template <int CG, int BNT>
+// compute a (128·RH·CG) x BNT output tile, BNT = 256 or 128 columns.  RH = 1:
+// each CTA holds 128 rows and tensor memory holds two accumulators, so one
+// tile's epilogue overlaps the next tile's main loop.  RH = 2 (the tall
+// tile, pairs of 256-column tiles only): each CTA holds 256 rows as two
+// halves that share every B stage, which halves the operand bytes per MMA;
+// the two halves fill tensor memory, so the epilogue does not overlap.
+template <int CG, int BNT, int RH>
 struct Cfg {
-  static constexpr int kRows = BM * CG;          // output rows per tile
+  static constexpr int kRowsCTA = BM * RH;       // output rows per CTA
+  static constexpr int kRows = kRowsCTA * CG;    // output rows per tile
   static constexpr int kBCols = BNT / CG;        // B columns staged per CTA
-  static constexpr uint32_t kABytes = BM * BK * 2;
+  static constexpr uint32_t kABytes = kRowsCTA * BK * 2;
   static constexpr uint32_t kBBytes = kBCols * BK * 2;
   // TP_GEMM_STAGE_BUDGET bytes of operand stages (default 224 KB: 7 stages of
-  // the 2 x 256 tile, 4 of 1 x 256, 9 of 2 x 128, 7 of 1 x 128)
+  // the 2 x 256 tile, 4 of 1 x 256 and of the tall tile, 9 of 2 x 128, 7 of 1 x 128)
   static constexpr int kStages = static_cast<int>(TP_GEMM_STAGE_BUDGET / (kABytes + kBBytes));
   static constexpr uint32_t kOffB = kStages * kABytes;
   static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
@@ -108,7 +121,8 @@ struct Cfg {
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kBytes = kOffMisc + 16;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
-  static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators
+  static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators, or two row halves
+  static constexpr int kAccBufs = RH == 2 ? 1 : 2;    // accumulator buffers in tensor memory
   static constexpr int kChunks = BNT / 64;            // 32-column chunks per epilogue warp
 };
 
@@ -266,9 +280,10 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
   return v[0];
 }
 
-template <int CG, int BNT, int EPI>
+template <int CG, int BNT, int RH, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
-  using C = Cfg<CG, BNT>;
+  using C = Cfg<CG, BNT, RH>;
+  static_assert(RH == 1 || (CG == 2 && BNT == 256), "tall tiles are 2-CTA 256-column tiles");
   static_assert(BNT == 256 || (EPI != EPI_XENT_STATS && EPI != EPI_XENT_GRAD),
                 "the cross-entropy epilogues take 128-column slices of a 256-column tile");
   constexpr int STAGES = C::kStages;
@@ -331,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       for (int unit = slot0; ok && unit < a.num_units; unit += nslots) {
         int tm, tn, s, tile;
         unit_map(a, unit, tm, tn, s, tile);
-        const int a_row = tm * C::kRows + static_cast<int>(rank) * BM;
+        const int a_row = tm * C::kRows + static_cast<int>(rank) * C::kRowsCTA;
         const int b_col = tn * BNT + static_cast<int>(rank) * C::kBCols;
         for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
           if (unit == a.inject_unit && kb == a.inject_kb) {
@@ -359,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               load(dA, &P.tmA, k0, a_row, a.a_hint);
             } else {
 #pragma unroll
-              for (int j = 0; j < BM / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
+              for (int j = 0; j < C::kRowsCTA / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
             }
             if (!a.b_mn) {
               load(dB, &P.tmB, k0, b_col, a.b_hint);
@@ -377,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               load(dA, &P.tmA, k0, a_row, a.a_hint);
             } else {
 #pragma unroll
-              for (int j = 0; j < BM / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
+              for (int j = 0; j < C::kRowsCTA / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
             }
             if (!a.b_mn) {
               load(dB, &P.tmB, k0, b_col, a.b_hint);
@@ -396,7 +411,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               tma_prefetch_l2_2d(&P.tmA, kp, a_row);
             } else {
 #pragma unroll
-              for (int j = 0; j < BM / 64; ++j) tma_prefetch_l2_2d(&P.tmA, a_row + j * 64, kp);
+              for (int j = 0; j < C::kRowsCTA / 64; ++j) tma_prefetch_l2_2d(&P.tmA, a_row + j * 64, kp);
             }
             if (!a.b_mn) {
               tma_prefetch_l2_2d(&P.tmB, kp, b_col);
@@ -443,13 +458,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       for (int unit = slot0; ok && unit < a.num_units; unit += nslots, ++t) {
         int tm, tn, s, tile;
         unit_map(a, unit, tm, tn, s, tile);
-        const int acc = t & 1;
-        const uint32_t use = static_cast<uint32_t>(t >> 1);
+        const int acc = t % C::kAccBufs;
+        const uint32_t use = static_cast<uint32_t>(t / C::kAccBufs);
         if (!mbar_wait_bounded(&tempty[acc], (use & 1u) ^ 1u, a.wait_ns, abort_flag)) {
           if (!*abort_flag) flag_timeout(a, abort_flag);
           break;
         }
         tc_fence_after_sync();
+        // RH = 1: accumulator buffer acc; RH = 2: row half h at column h·BNT
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BNT);
         const int kb0 = a.split_kb[s], kb1 = a.split_kb[s + 1];
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -463,9 +479,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           const uint32_t b_base = smem_u32(sB + stage * C::kBBytes);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            const uint64_t adesc = smem_desc_sw128(a_base + k * a_kstep, a_lbo, 1024);
             const uint64_t bdesc = smem_desc_sw128(b_base + k * b_kstep, b_lbo, 1024);
-            tc_mma_bf16_cg<CG>(d_tmem, adesc, bdesc, idesc, (kb > kb0 || k > 0) ? 1u : 0u);
+#pragma unroll
+            for (int h = 0; h < RH; ++h) {   // the row halves share the B stage
+              // a row half is 128 rows: 16 KB of the A stage in either layout
+              const uint64_t adesc =
+                  smem_desc_sw128(a_base + h * (BM * 128) + k * a_kstep, a_lbo, 1024);
+              tc_mma_bf16_cg<CG>(d_tmem + static_cast<uint32_t>(h * BNT), adesc, bdesc, idesc,
+                                 (kb > kb0 || k > 0) ? 1u : 0u);
+            }
           }
           any = true;
           tc_commit_mc<CG>(&empty[stage], pair_mask);   // frees the stage in both CTAs
@@ -494,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     for (int unit = slot0; unit < a.num_units; unit += nslots, ++t) {
       int tm, tn, s, tile;
       unit_map(a, unit, tm, tn, s, tile);
-      const int acc = t & 1;
-      const uint32_t use = static_cast<uint32_t>(t >> 1);
+      const int acc = t % C::kAccBufs;
+      const uint32_t use = static_cast<uint32_t>(t / C::kAccBufs);
       const bool got = mbar_wait_bounded<true>(&tfull[acc], use & 1u, a.wait_ns, abort_flag);
       // all epilogue threads leave together or go on together, so no warp
       // can be left waiting in a later named barrier
@@ -504,11 +526,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         break;
       }
       tc_fence_after_sync();
-      const int row = tm * C::kRows + static_cast<int>(rank) * BM + row_in_tile;
+#pragma unroll 1
+      for (int hr = 0; hr < RH; ++hr) {   // the CTA's 128-row halves (one unless tall)
+      const int row =
+          tm * C::kRows + static_cast<int>(rank) * C::kRowsCTA + hr * BM + row_in_tile;
       const bool row_ok = row < a.M;
-      const int htile = tile * CG + static_cast<int>(rank);   // this CTA's 128-row half tile
-      const uint32_t t_base =
-          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BNT);
+      // this CTA's 128-row piece of the tile: the unit of the split partials,
+      // the arrival counters and (times four) the dbias partial rows
+      const int htile = (tile * CG + static_cast<int>(rank)) * RH + hr;
+      const uint32_t t_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
+                              static_cast<uint32_t>((acc + hr) * BNT);
       const int c0 = half * C::kChunks;   // this warp's first 32-column chunk
 
       if constexpr (EPI == EPI_SPLIT_SUM) {
@@ -780,13 +807,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               // written only when it holds rows of the problem (rows past M
               // contribute zeros and have no partial row)
               const float colsum = warp_column_sums(v, lane);
-              const int prow = (tm * CG + static_cast<int>(rank)) * 4 + q;
+              const int prow = ((tm * CG + static_cast<int>(rank)) * RH + hr) * 4 + q;
               if (prow * 32 < a.M && col0 + lane < a.N)
                 a.dbias_part[static_cast<int64_t>(prow) * a.N + col0 + lane] = colsum;
             }
           }
         }
       }
+      }   // row halves
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) {   // release the accumulator to the pair leader's MMA
@@ -843,9 +871,9 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
 // Launch with `slots` persistent CTAs (CG = 1) or CTA pairs (CG = 2), capped
 // at the number that can be resident at once, so that no persistent slot
 // starts only after another has finished.
-template <int CG, int BNT, int EPI>
+template <int CG, int BNT, int RH, int EPI>
 tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
-  using C = Cfg<CG, BNT>;
+  using C = Cfg<CG, BNT, RH>;
   static_assert(C::kAlloc <= 232448, "shared memory budget");
   static int max_resident[64] = {0};
   int dev = 0;
@@ -862,12 +890,12 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (!max_resident[dev & 63]) {
-    if (cudaFuncSetAttribute(gemm_tc_kernel<CG, BNT, EPI>,
+    if (cudaFuncSetAttribute(gemm_tc_kernel<CG, BNT, RH, EPI>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
       return TP_ERR_CUDA;
     int clusters = 0;
     cfg.gridDim = dim3(static_cast<unsigned>(CG * num_sms()));
-    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<CG, BNT, EPI>, &cfg) !=
+    if (cudaOccupancyMaxActiveClusters(&clusters, gemm_tc_kernel<CG, BNT, RH, EPI>, &cfg) !=
             cudaSuccess ||
         clusters <= 0) {
       cudaGetLastError();
@@ -879,26 +907,26 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   const int grid = CG * slots;
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
-  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<CG, BNT, EPI>, prm) != cudaSuccess)
+  if (cudaLaunchKernelEx(&cfg, gemm_tc_kernel<CG, BNT, RH, EPI>, prm) != cudaSuccess)
     return TP_ERR_CUDA;
   note_launches(1);
   return TP_OK;
 }
 
-template <int CG, int BNT>
+template <int CG, int BNT, int RH>
 tp_status launch_epi(const GemmParams& prm, int epi, int slots, cudaStream_t stream) {
   switch (epi) {
-    case EPI_STORE_BF16: return launch_impl<CG, BNT, EPI_STORE_BF16>(prm, slots, stream);
-    case EPI_BIAS_ACT: return launch_impl<CG, BNT, EPI_BIAS_ACT>(prm, slots, stream);
-    case EPI_DACT: return launch_impl<CG, BNT, EPI_DACT>(prm, slots, stream);
-    case EPI_DACT_Y: return launch_impl<CG, BNT, EPI_DACT_Y>(prm, slots, stream);
-    case EPI_STORE_F32: return launch_impl<CG, BNT, EPI_STORE_F32>(prm, slots, stream);
-    case EPI_SPLIT_SUM: return launch_impl<CG, BNT, EPI_SPLIT_SUM>(prm, slots, stream);
+    case EPI_STORE_BF16: return launch_impl<CG, BNT, RH, EPI_STORE_BF16>(prm, slots, stream);
+    case EPI_BIAS_ACT: return launch_impl<CG, BNT, RH, EPI_BIAS_ACT>(prm, slots, stream);
+    case EPI_DACT: return launch_impl<CG, BNT, RH, EPI_DACT>(prm, slots, stream);
+    case EPI_DACT_Y: return launch_impl<CG, BNT, RH, EPI_DACT_Y>(prm, slots, stream);
+    case EPI_STORE_F32: return launch_impl<CG, BNT, RH, EPI_STORE_F32>(prm, slots, stream);
+    case EPI_SPLIT_SUM: return launch_impl<CG, BNT, RH, EPI_SPLIT_SUM>(prm, slots, stream);
     case EPI_XENT_STATS:
-      if constexpr (BNT == 256) return launch_impl<CG, BNT, EPI_XENT_STATS>(prm, slots, stream);
+      if constexpr (BNT == 256) return launch_impl<CG, BNT, RH, EPI_XENT_STATS>(prm, slots, stream);
       break;
     case EPI_XENT_GRAD:
-      if constexpr (BNT == 256) return launch_impl<CG, BNT, EPI_XENT_GRAD>(prm, slots, stream);
+      if constexpr (BNT == 256) return launch_impl<CG, BNT, RH, EPI_XENT_GRAD>(prm, slots, stream);
       break;
   }
   return TP_ERR_UNSUPPORTED;
@@ -939,46 +967,48 @@ void choose_l2_hints(const GemmProblem& p, int& a_hint, int& b_hint) {
 struct TileChoice {
   int cg;    // CTAs per tile (1, or a cluster pair with cta_group::2)
   int bn;    // output columns per tile (256 or 128)
+  int rh;    // 128-row halves per CTA (2: the tall 512 x 256 pair tile)
 };
 
 // Relative throughput of each tile shape per SM (the 256 x 256 pair tile is
 // the reference): narrower or single-CTA tiles read more operand bytes per
 // MMA and keep the tensor pipe a little less busy.
-double tile_efficiency(int cg, int bn) {
+double tile_efficiency(const TileChoice& t) {
   // measured per SM against the 256 x 256 pair tile on the layer's shapes
   // (h = 4096 MLP, h = 1600 projections, logits): 0.60-0.75 for 256 x 128,
   // 0.90-1.0 for 128 x 256, 0.55-0.70 for 128 x 128
-  if (cg == 2) return bn == 256 ? 1.0 : 0.70;
-  return bn == 256 ? 0.92 : 0.60;
+  if (t.cg == 2) return t.bn == 256 ? (t.rh == 2 ? kTallEfficiency : 1.0) : 0.70;
+  return t.bn == 256 ? 0.92 : 0.60;
 }
 
 // Tile shape of a GEMM: the one with the least estimated time, counting
 // whole waves of units (tiles x splits) over the resident slots, each wave
 // costing one tile's work per SM.  Problems one 128-row tile high use
 // single-CTA tiles; the cross-entropy epilogues need 256-column tiles.
-// TP_GEMM_TILE=2x256|2x128|1x256|1x128 forces a shape (tests and sweeps).
+// TP_GEMM_TILE=2x256|2x256t|2x128|1x256|1x128 forces a shape (tests, sweeps).
 TileChoice choose_tile(int M, int N, int splits, int epi) {
   const bool xent = epi == EPI_XENT_STATS || epi == EPI_XENT_GRAD;
   if (const char* e = std::getenv("TP_GEMM_TILE")) {
-    TileChoice t{0, 0};
-    if (!std::strcmp(e, "2x256")) t = {2, 256};
-    else if (!std::strcmp(e, "2x128")) t = {2, 128};
-    else if (!std::strcmp(e, "1x256")) t = {1, 256};
-    else if (!std::strcmp(e, "1x128")) t = {1, 128};
+    TileChoice t{0, 0, 1};
+    if (!std::strcmp(e, "2x256")) t = {2, 256, 1};
+    else if (!std::strcmp(e, "2x256t")) t = {2, 256, 2};
+    else if (!std::strcmp(e, "2x128")) t = {2, 128, 1};
+    else if (!std::strcmp(e, "1x256")) t = {1, 256, 1};
+    else if (!std::strcmp(e, "1x128")) t = {1, 128, 1};
     if (t.cg && !(xent && t.bn != 256)) return t;
   }
-  const TileChoice cands[4] = {{2, 256}, {2, 128}, {1, 256}, {1, 128}};
-  TileChoice best{M > BM ? 2 : 1, 256};
+  const TileChoice cands[5] = {{2, 256, 1}, {2, 256, 2}, {2, 128, 1}, {1, 256, 1}, {1, 128, 1}};
+  TileChoice best{M > BM ? 2 : 1, 256, 1};
   double best_cost = 0.0;
   bool have = false;
   for (const TileChoice& t : cands) {
     if (xent && t.bn != 256) continue;
     if (M <= BM && t.cg == 2) continue;
-    const long long tiles = static_cast<long long>((M + BM * t.cg - 1) / (BM * t.cg)) *
-                            ((N + t.bn - 1) / t.bn);
+    const int rows = BM * t.rh * t.cg;
+    const long long tiles = static_cast<long long>((M + rows - 1) / rows) * ((N + t.bn - 1) / t.bn);
     const long long slots = num_sms() / t.cg;
     const long long waves = (tiles * splits + slots - 1) / slots;
-    const double cost = static_cast<double>(waves) * t.bn / tile_efficiency(t.cg, t.bn);
+    const double cost = static_cast<double>(waves) * t.rh * t.bn / tile_efficiency(t);
     if (!have || cost < best_cost * 0.999) {
       best = t;
       best_cost = cost;
@@ -997,10 +1027,10 @@ bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t 
 
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
   if (splits <= 1 && !with_zpart) return 0;
-  // 128-row half tiles of the 256-row tiling (covers the 128-row tiling
-  // too); the partial bytes of 256-column tiles bound those of 128-column
-  // tiles, whose counters are twice as many
-  const size_t hrows = static_cast<size_t>((M + 2 * BM - 1) / (2 * BM)) * 2;
+  // 128-row pieces of the 512-row tall tiling (covers the 256- and 128-row
+  // tilings too); the partial bytes of 256-column tiles bound those of
+  // 128-column tiles, whose counters are twice as many
+  const size_t hrows = static_cast<size_t>((M + 4 * BM - 1) / (4 * BM)) * 4;
   size_t bytes = with_zpart ? 0 : hrows * ((N + BN - 1) / BN) * splits * BM * BN * sizeof(float);
   bytes += hrows * ((N + 127) / 128) * sizeof(int);
   return (bytes + 255) & ~static_cast<size_t>(255);
@@ -1008,14 +1038,14 @@ size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
 
 double gemm_tc_estimate_s(int M, int N, int K, int splits, int epi) {
   const TileChoice t = choose_tile(M, N, splits, epi);
-  const long long tiles =
-      static_cast<long long>((M + BM * t.cg - 1) / (BM * t.cg)) * ((N + t.bn - 1) / t.bn);
+  const int rows = BM * t.rh * t.cg;
+  const long long tiles = static_cast<long long>((M + rows - 1) / rows) * ((N + t.bn - 1) / t.bn);
   const long long slots = num_sms() / t.cg;
   const long long waves = (tiles * splits + slots - 1) / slots;
   const double k_split = static_cast<double>(K) / splits;
   const double per_sm_flops = 1.5e15 / 148.0;   // bf16 dense, sustained
-  return static_cast<double>(waves) * 2.0 * BM * t.bn * k_split /
-         (per_sm_flops * tile_efficiency(t.cg, t.bn));
+  return static_cast<double>(waves) * 2.0 * BM * t.rh * t.bn * k_split /
+         (per_sm_flops * tile_efficiency(t));
 }
 
 tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
@@ -1025,7 +1055,8 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   const TileChoice tile = choose_tile(p.M, p.N, p.splits, split_epi ? EPI_SPLIT_SUM : p.epi);
   const int CG = tile.cg;
   const int BNT = tile.bn;
-  const int rows = BM * CG;
+  const int RH = tile.rh;
+  const int rows = BM * RH * CG;
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
   GemmArgs& a = prm.a;
@@ -1085,7 +1116,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (split_epi) {
     const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
     if (p.ws == nullptr || p.ws_bytes < need) return TP_ERR_WORKSPACE;
-    const size_t htiles = static_cast<size_t>(a.tiles_m) * CG * a.tiles_n;
+    const size_t htiles = static_cast<size_t>(a.tiles_m) * CG * RH * a.tiles_n;
     if (p.zpart) {
       a.part = p.zpart;
       a.part_is_zpart = 1;
@@ -1104,7 +1135,7 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   const uint32_t b_rows = static_cast<uint32_t>(BNT / CG);
   bool ok;
   if (!p.a_mn)
-    ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, BM);
+    ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, static_cast<uint32_t>(BM * RH));
   else
     ok = make_tmap(&prm.tmA, p.A, p.M, p.K, p.lda, 64, BK);
   if (!ok) return TP_ERR_CUDA;
@@ -1115,11 +1146,13 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   if (!ok) return TP_ERR_CUDA;
   const int slots = CG == 2 ? num_sms() / 2 : num_sms();
   const int used = a.num_units < slots ? a.num_units : slots;
-  if (CG == 2)
-    return BNT == 256 ? launch_epi<2, 256>(prm, epi, used, stream)
-                      : launch_epi<2, 128>(prm, epi, used, stream);
-  return BNT == 256 ? launch_epi<1, 256>(prm, epi, used, stream)
-                    : launch_epi<1, 128>(prm, epi, used, stream);
+  if (CG == 2) {
+    if (RH == 2) return launch_epi<2, 256, 2>(prm, epi, used, stream);
+    return BNT == 256 ? launch_epi<2, 256, 1>(prm, epi, used, stream)
+                      : launch_epi<2, 128, 1>(prm, epi, used, stream);
+  }
+  return BNT == 256 ? launch_epi<1, 256, 1>(prm, epi, used, stream)
+                    : launch_epi<1, 128, 1>(prm, epi, used, stream);
 }
 
 void arm_gemm_injection(int unit, int kb, uint64_t wait_ns) {

@@ -57,7 +57,7 @@ def _clean_mlp_matches_oracle(seed):
         assert_close(k, g[k], ob[k], TOL_BF16)
 
 
-@pytest.mark.parametrize("tile", ["2x256", "2x128", "1x256", "1x128"])
+@pytest.mark.parametrize("tile", ["2x256", "2x256t", "2x128", "1x256", "1x128"])
 @pytest.mark.parametrize("unit,kblock", [(0, 1), (0, 0), (1, 2)])
 def test_gemm_producer_stall_times_out_drains_and_recovers(tile, unit, kblock, monkeypatch):
     """The real GEMM pipeline's failure path: the producers of one CTA (pair)

@@ -159,7 +159,7 @@ def test_mlp_deterministic():
     assert torch.equal(a[4], b[4])
 
 
-@pytest.mark.parametrize("tile", ["2x256", "2x128", "1x256", "1x128"])
+@pytest.mark.parametrize("tile", ["2x256", "2x256t", "2x128", "1x256", "1x128"])
 def test_mlp_every_tile_shape(tile, monkeypatch):
     """Each tile shape of the GEMM engine (CTA pairs or single CTAs, 256- or
     128-column tiles), forced for every GEMM of the layer: ragged rows and
