@@ -176,7 +176,7 @@ def _prepare(dev, parts):
 
     g = pr = vo = None
     bf = dict(dtype=torch.bfloat16, device=dev)
-    if any(p.startswith("mlp") for p in parts):
+    if any(p.startswith("mlp") or p.endswith("_gemm") for p in parts):
         g = _prepare_mlp(dev, tpl, tp_inputs, torch, bf)
     if any(p in parts for p in ("proj", "attn_fwd", "attn_bwd", "ln_fwd", "ln_bwd")):
         pr = _prepare_proj(dev, tpl, tp_inputs, torch, bf)
@@ -363,6 +363,17 @@ def _lxent_dlogits(tpl, vo, st):
                                grad_scale=1.0 / VOC["T"], dlogits=vo["dlogits_bf"], dev_status=st)
 
 
+def _col_gemm(tpl, g, st):
+    """The column GEMM of the h=4096 layer alone (U = X·A, no bias, no
+    activation): the engine's main loop on the a2 shape, for profiling."""
+    tpl.tp_col_linear_fwd(g["X"], g["A"], None, 1, Y=g["U"], dev_status=st)
+
+
+def _cublas_gemm(torch, g):
+    """torch.matmul (cuBLAS) on the same operands, for the same-box A/B."""
+    torch.matmul(g["X"], g["A"], out=g["U"])
+
+
 # the step: every row of the hot path
 PARTS = ("mlp_fwd", "mlp_bwd", "proj", "embed", "logits", "xent")
 # the vocabulary backward (the next row beyond the hot path), timed in its own
@@ -379,6 +390,8 @@ RECOMPUTE_PARTS = ("mlp_bwd_rc",)
 ATTN_PARTS = ("attn_fwd", "attn_bwd")
 # sequence-parallel dropout-add-LayerNorm after the output projection, own loop
 LN_PARTS = ("ln_fwd", "ln_bwd")
+# single GEMMs for profiling and the library A/B (partial runs only)
+GEMM_PARTS = ("col_gemm", "cublas_gemm")
 
 
 E2E_DATA = (("X", "dZ"), ("Z", "dX"))
@@ -595,7 +608,7 @@ def run_gpu(args):
         torch.distributed.barrier()
     tpl.lib()
 
-    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS + ATTN_PARTS + LN_PARTS
+    known = PARTS + BWD_PARTS[1:] + FUSED_PARTS + RECOMPUTE_PARTS + ATTN_PARTS + LN_PARTS + GEMM_PARTS
     parts = [p for p in known if p in args.parts.split(",")]
     if not parts:
         raise SystemExit(f"--parts must name some of {','.join(known)}")
@@ -620,7 +633,9 @@ def run_gpu(args):
            "attn_fwd": lambda: _attn_fwd(tpl, pr, st),
            "attn_bwd": lambda: _attn_bwd(tpl, pr, st),
            "ln_fwd": lambda: _ln_fwd(tpl, pr, st),
-           "ln_bwd": lambda: _ln_bwd(tpl, pr, st)}
+           "ln_bwd": lambda: _ln_bwd(tpl, pr, st),
+           "col_gemm": lambda: _col_gemm(tpl, g, st),
+           "cublas_gemm": lambda: _cublas_gemm(torch, g)}
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):

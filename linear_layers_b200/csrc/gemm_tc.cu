@@ -40,9 +40,9 @@
 #include "sm100_ptx.cuh"
 
 // per-SM throughput of the tall tile relative to the 256 x 256 pair tile
-// (below 1 keeps it off the default choice until measured)
+// (measured on the h = 4096 MLP GEMMs: 1.05-1.08)
 #ifndef TP_GEMM_TALL_EFF
-#define TP_GEMM_TALL_EFF 0.9
+#define TP_GEMM_TALL_EFF 1.08
 #endif
 
 #ifndef TP_GEMM_STAGE_BUDGET
@@ -88,14 +88,17 @@ struct GemmArgs {
   const float* row_lse;
   float grad_scale;
   int inject_unit, inject_kb;       // debug: the producer stops before this k-block (-1: never)
-  int a_hint, b_hint;               // L2 policy of the operand loads: 0 none, 1 evict-first, 2 evict-last
-  int l2_prefetch;                  // prefetch the k-block one ring ahead into L2
 };
 
+// One launch runs one problem, or two independent problems with the same
+// tile shape and epilogue one after the other in its unit order (a grouped
+// launch: the units of the second fill the first one's last wave).
 struct __align__(64) GemmParams {
-  CUtensorMap tmA;
-  CUtensorMap tmB;
-  GemmArgs a;
+  CUtensorMap tmA[2];
+  CUtensorMap tmB[2];
+  GemmArgs a[2];
+  int units0;                       // units of problem 0
+  int total_units;                  // units of both problems
 };
 
 // Tile configurations: CG CTAs (1 or 2, a cluster pair with cta_group::2)
@@ -290,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  const GemmArgs& a = P.a;
+  const GemmArgs& a0 = P.a[0];   // wait limit and status word (the same in both problems)
 
   uint8_t* sA = smem;
   uint8_t* sB = smem + C::kOffB;
@@ -331,32 +334,38 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   if constexpr (CG == 2) cluster_sync_all();   // peer barriers initialised before any signal
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
+  // launched as a programmatic dependent of the previous kernel in the
+  // stream: the set-up above overlapped its tail; nothing below touches
+  // global memory before that kernel has completed
+  grid_dependency_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (elect_one_sync()) {
-      tma_prefetch_desc(&P.tmA);
-      tma_prefetch_desc(&P.tmB);
-      const uint64_t pol_first = l2_policy_evict_first();
-      const uint64_t pol_last = l2_policy_evict_last();
+      tma_prefetch_desc(&P.tmA[0]);
+      tma_prefetch_desc(&P.tmB[0]);
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
       bool ok = true;
-      for (int unit = slot0; ok && unit < a.num_units; unit += nslots) {
+      for (int unit = slot0; ok && unit < P.total_units; unit += nslots) {
+        const int prob = unit >= P.units0 ? 1 : 0;
+        const GemmArgs& a = P.a[prob];
+        const CUtensorMap* tmA = &P.tmA[prob];
+        const CUtensorMap* tmB = &P.tmB[prob];
         int tm, tn, s, tile;
-        unit_map(a, unit, tm, tn, s, tile);
+        unit_map(a, unit - prob * P.units0, tm, tn, s, tile);
         const int a_row = tm * C::kRows + static_cast<int>(rank) * C::kRowsCTA;
         const int b_col = tn * BNT + static_cast<int>(rank) * C::kBCols;
         for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
-          if (unit == a.inject_unit && kb == a.inject_kb) {
+          if (unit == a0.inject_unit && kb == a0.inject_kb) {
             // debug injection: stop issuing without a word, as a producer
             // that died would; the MMA issuer's bounded wait runs out
             ok = false;
             break;
           }
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a.wait_ns, abort_flag)) {
-            if (!*abort_flag) flag_timeout(a, abort_flag);
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, a0.wait_ns, abort_flag)) {
+            if (!*abort_flag) flag_timeout(a0, abort_flag);
             ok = false;
             break;
           }
@@ -366,58 +375,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           uint8_t* dB = sB + stage * C::kBBytes;
           if constexpr (CG == 2) {
             const uint32_t bar = mapa_shared(&full[stage], 0);
-            auto load = [&](uint8_t* dst, const CUtensorMap* m, int x, int y, int hint) {
-              if (hint) tma_load_2d_cg2_hint(dst, m, bar, x, y, hint == 1 ? pol_first : pol_last);
-              else tma_load_2d_cg2(dst, m, bar, x, y);
-            };
             if (!a.a_mn) {
-              load(dA, &P.tmA, k0, a_row, a.a_hint);
+              tma_load_2d_cg2(dA, tmA, bar, k0, a_row);
             } else {
 #pragma unroll
-              for (int j = 0; j < C::kRowsCTA / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
+              for (int j = 0; j < C::kRowsCTA / 64; ++j)
+                tma_load_2d_cg2(dA + j * 8192, tmA, bar, a_row + j * 64, k0);
             }
             if (!a.b_mn) {
-              load(dB, &P.tmB, k0, b_col, a.b_hint);
+              tma_load_2d_cg2(dB, tmB, bar, k0, b_col);
             } else {
 #pragma unroll
               for (int j = 0; j < C::kBCols / 64; ++j)
-                load(dB + j * 8192, &P.tmB, b_col + j * 64, k0, a.b_hint);
+                tma_load_2d_cg2(dB + j * 8192, tmB, bar, b_col + j * 64, k0);
             }
           } else {
-            auto load = [&](uint8_t* dst, const CUtensorMap* m, int x, int y, int hint) {
-              if (hint) tma_load_2d_hint(dst, m, &full[stage], x, y, hint == 1 ? pol_first : pol_last);
-              else tma_load_2d(dst, m, &full[stage], x, y);
-            };
             if (!a.a_mn) {
-              load(dA, &P.tmA, k0, a_row, a.a_hint);
+              tma_load_2d(dA, tmA, &full[stage], k0, a_row);
             } else {
 #pragma unroll
-              for (int j = 0; j < C::kRowsCTA / 64; ++j) load(dA + j * 8192, &P.tmA, a_row + j * 64, k0, a.a_hint);
+              for (int j = 0; j < C::kRowsCTA / 64; ++j)
+                tma_load_2d(dA + j * 8192, tmA, &full[stage], a_row + j * 64, k0);
             }
             if (!a.b_mn) {
-              load(dB, &P.tmB, k0, b_col, a.b_hint);
+              tma_load_2d(dB, tmB, &full[stage], k0, b_col);
             } else {
 #pragma unroll
               for (int j = 0; j < C::kBCols / 64; ++j)
-                load(dB + j * 8192, &P.tmB, b_col + j * 64, k0, a.b_hint);
-            }
-          }
-          // L2 prefetch of the k-block one ring length ahead in this unit:
-          // by the time its load is issued it waits in L2, not in HBM
-          const int kbp = kb + STAGES;
-          if (a.l2_prefetch && kbp < a.split_kb[s + 1]) {
-            const int kp = kbp * BK;
-            if (!a.a_mn) {
-              tma_prefetch_l2_2d(&P.tmA, kp, a_row);
-            } else {
-#pragma unroll
-              for (int j = 0; j < C::kRowsCTA / 64; ++j) tma_prefetch_l2_2d(&P.tmA, a_row + j * 64, kp);
-            }
-            if (!a.b_mn) {
-              tma_prefetch_l2_2d(&P.tmB, kp, b_col);
-            } else {
-#pragma unroll
-              for (int j = 0; j < C::kBCols / 64; ++j) tma_prefetch_l2_2d(&P.tmB, b_col + j * 64, kp);
+                tma_load_2d(dB + j * 8192, tmB, &full[stage], b_col + j * 64, k0);
             }
           }
           ++issued;
@@ -438,30 +423,34 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             stage = STAGES - 1;
             phase ^= 1u;
           }
-          mbar_wait_bounded(&full[stage], phase, a.wait_ns, &keep_waiting);
+          mbar_wait_bounded(&full[stage], phase, a0.wait_ns, &keep_waiting);
         }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (pair leader)
     if (rank == 0 && elect_one_sync()) {
-      const uint32_t idesc = idesc_bf16_f32(C::kRows, BNT, a.a_mn != 0, a.b_mn != 0);
-      const uint32_t a_lbo = a.a_mn ? 8192u : 16u;
-      const uint32_t b_lbo = a.b_mn ? 8192u : 16u;
-      const uint32_t a_kstep = a.a_mn ? 2048u : 32u;   // bytes per 16-element K step
-      const uint32_t b_kstep = a.b_mn ? 2048u : 32u;
       const uint16_t pair_mask = CG == 2 ? 0x3 : 0x1;
       int stage = 0;
       uint32_t phase = 0;
       int t = 0;
       bool ok = true, any = false;
-      for (int unit = slot0; ok && unit < a.num_units; unit += nslots, ++t) {
+      for (int unit = slot0; ok && unit < P.total_units; unit += nslots, ++t) {
+        const int prob = unit >= P.units0 ? 1 : 0;
+        const GemmArgs& a = P.a[prob];
+        // one MMA covers 128 rows per CTA (256 for the pair); the tall tile
+        // issues one per row half
+        const uint32_t idesc = idesc_bf16_f32(BM * CG, BNT, a.a_mn != 0, a.b_mn != 0);
+        const uint32_t a_lbo = a.a_mn ? 8192u : 16u;
+        const uint32_t b_lbo = a.b_mn ? 8192u : 16u;
+        const uint32_t a_kstep = a.a_mn ? 2048u : 32u;   // bytes per 16-element K step
+        const uint32_t b_kstep = a.b_mn ? 2048u : 32u;
         int tm, tn, s, tile;
-        unit_map(a, unit, tm, tn, s, tile);
+        unit_map(a, unit - prob * P.units0, tm, tn, s, tile);
         const int acc = t % C::kAccBufs;
         const uint32_t use = static_cast<uint32_t>(t / C::kAccBufs);
-        if (!mbar_wait_bounded(&tempty[acc], (use & 1u) ^ 1u, a.wait_ns, abort_flag)) {
-          if (!*abort_flag) flag_timeout(a, abort_flag);
+        if (!mbar_wait_bounded(&tempty[acc], (use & 1u) ^ 1u, a0.wait_ns, abort_flag)) {
+          if (!*abort_flag) flag_timeout(a0, abort_flag);
           break;
         }
         tc_fence_after_sync();
@@ -469,8 +458,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BNT);
         const int kb0 = a.split_kb[s], kb1 = a.split_kb[s + 1];
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!mbar_wait_bounded(&full[stage], phase, a.wait_ns, abort_flag)) {
-            if (!*abort_flag) flag_timeout(a, abort_flag);
+          if (!mbar_wait_bounded(&full[stage], phase, a0.wait_ns, abort_flag)) {
+            if (!*abort_flag) flag_timeout(a0, abort_flag);
             ok = false;
             break;
           }
@@ -501,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       if (any) {   // every issued MMA must finish before tensor memory is freed
         volatile int keep_waiting = 0;
         tc_commit_local<CG>(mma_done);
-        mbar_wait_bounded(mma_done, 0, a.wait_ns, &keep_waiting);
+        mbar_wait_bounded(mma_done, 0, a0.wait_ns, &keep_waiting);
       }
     }
   } else {
@@ -513,16 +502,18 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
     const int et = threadIdx.x - 64;      // 0..255 among the epilogue threads
     const uint32_t tempty_addr0 = CG == 2 ? mapa_shared(&tempty[0], 0) : smem_u32(&tempty[0]);
     int t = 0;
-    for (int unit = slot0; unit < a.num_units; unit += nslots, ++t) {
+    for (int unit = slot0; unit < P.total_units; unit += nslots, ++t) {
+      const int prob = unit >= P.units0 ? 1 : 0;
+      const GemmArgs& a = P.a[prob];
       int tm, tn, s, tile;
-      unit_map(a, unit, tm, tn, s, tile);
+      unit_map(a, unit - prob * P.units0, tm, tn, s, tile);
       const int acc = t % C::kAccBufs;
       const uint32_t use = static_cast<uint32_t>(t / C::kAccBufs);
-      const bool got = mbar_wait_bounded<true>(&tfull[acc], use & 1u, a.wait_ns, abort_flag);
+      const bool got = mbar_wait_bounded<true>(&tfull[acc], use & 1u, a0.wait_ns, abort_flag);
       // all epilogue threads leave together or go on together, so no warp
       // can be left waiting in a later named barrier
       if (!named_barrier_and(1, kEpiThreads, got)) {
-        if (et == 0 && !*abort_flag) flag_timeout(a, abort_flag);
+        if (et == 0 && !*abort_flag) flag_timeout(a0, abort_flag);
         break;
       }
       tc_fence_after_sync();
@@ -882,13 +873,17 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kAlloc;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = CG;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the CTAs may be set up while the previous
+  // kernel drains (the kernel waits for it before any global access)
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (!max_resident[dev & 63]) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<CG, BNT, RH, EPI>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
@@ -949,21 +944,6 @@ void take_injection(int& unit, int& kb, uint64_t& wait_ns) {
   g_inject_armed = false;
 }
 
-// L2 eviction policies of the two operands.  TP_GEMM_L2HINT=<a><b> with
-// n (none), f (evict first) or l (evict last) for each operand overrides
-// the choice (sweeps).
-void choose_l2_hints(const GemmProblem& p, int& a_hint, int& b_hint) {
-  a_hint = 0;
-  b_hint = 0;
-  if (const char* e = std::getenv("TP_GEMM_L2HINT")) {
-    auto code = [](char c) { return c == 'f' ? 1 : c == 'l' ? 2 : 0; };
-    if (e[0] && e[1]) {
-      a_hint = code(e[0]);
-      b_hint = code(e[1]);
-    }
-  }
-}
-
 struct TileChoice {
   int cg;    // CTAs per tile (1, or a cluster pair with cta_group::2)
   int bn;    // output columns per tile (256 or 128)
@@ -986,8 +966,12 @@ double tile_efficiency(const TileChoice& t) {
 // costing one tile's work per SM.  Problems one 128-row tile high use
 // single-CTA tiles; the cross-entropy epilogues need 256-column tiles.
 // TP_GEMM_TILE=2x256|2x256t|2x128|1x256|1x128 forces a shape (tests, sweeps).
-TileChoice choose_tile(int M, int N, int splits, int epi) {
+TileChoice choose_tile(int M, int N, int K, int splits, int epi) {
   const bool xent = epi == EPI_XENT_STATS || epi == EPI_XENT_GRAD;
+  // the tall tile's epilogue does not overlap its main loop: only for long
+  // main loops (K per split >= 4096) with bf16 outputs (the fp32 logits and
+  // the cross-entropy epilogues stay on the overlapped tile)
+  const bool tall_ok = K / splits >= 4096 && !xent && epi != EPI_STORE_F32;
   if (const char* e = std::getenv("TP_GEMM_TILE")) {
     TileChoice t{0, 0, 1};
     if (!std::strcmp(e, "2x256")) t = {2, 256, 1};
@@ -1004,6 +988,7 @@ TileChoice choose_tile(int M, int N, int splits, int epi) {
   for (const TileChoice& t : cands) {
     if (xent && t.bn != 256) continue;
     if (M <= BM && t.cg == 2) continue;
+    if (t.rh == 2 && !tall_ok) continue;
     const int rows = BM * t.rh * t.cg;
     const long long tiles = static_cast<long long>((M + rows - 1) / rows) * ((N + t.bn - 1) / t.bn);
     const long long slots = num_sms() / t.cg;
@@ -1037,7 +1022,7 @@ size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
 }
 
 double gemm_tc_estimate_s(int M, int N, int K, int splits, int epi) {
-  const TileChoice t = choose_tile(M, N, splits, epi);
+  const TileChoice t = choose_tile(M, N, K, splits, epi);
   const int rows = BM * t.rh * t.cg;
   const long long tiles = static_cast<long long>((M + rows - 1) / rows) * ((N + t.bn - 1) / t.bn);
   const long long slots = num_sms() / t.cg;
@@ -1048,18 +1033,17 @@ double gemm_tc_estimate_s(int M, int N, int K, int splits, int epi) {
          (per_sm_flops * tile_efficiency(t));
 }
 
-tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
+namespace {
+
+// Kernel arguments, operand maps and (split epilogue) workspace of one
+// problem with the given tile shape.
+tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& a,
+                        CUtensorMap* tmA, CUtensorMap* tmB, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return TP_ERR_SHAPE;
   if (p.splits < 1 || p.splits > kMaxSplits) return TP_ERR_SHAPE;
   const bool split_epi = p.splits > 1 || p.zpart != nullptr;
-  const TileChoice tile = choose_tile(p.M, p.N, p.splits, split_epi ? EPI_SPLIT_SUM : p.epi);
-  const int CG = tile.cg;
-  const int BNT = tile.bn;
-  const int RH = tile.rh;
+  const int CG = tile.cg, BNT = tile.bn, RH = tile.rh;
   const int rows = BM * RH * CG;
-  GemmParams prm;
-  memset(&prm, 0, sizeof(prm));
-  GemmArgs& a = prm.a;
   a.M = p.M;
   a.N = p.N;
   a.K = p.K;
@@ -1086,7 +1070,6 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   // partials requested (Zpart) go through the split epilogue even for a
   // single split: it publishes the partial and stores the (one-term) sum
   if (p.zpart != nullptr && p.epi != EPI_STORE_BF16) return TP_ERR_UNSUPPORTED;
-  const int epi = split_epi ? EPI_SPLIT_SUM : p.epi;
   a.act = p.act;
   a.out0 = p.out0;
   a.out1 = p.out1;
@@ -1106,12 +1089,6 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   a.grad_scale = p.grad_scale;
   a.inject_unit = -1;
   a.inject_kb = -1;
-  choose_l2_hints(p, a.a_hint, a.b_hint);
-  {
-    const char* e = std::getenv("TP_GEMM_L2PREFETCH");   // sweeps: 1 turns the prefetch on
-    a.l2_prefetch = (e && e[0] == '1') ? 1 : 0;
-  }
-  take_injection(a.inject_unit, a.inject_kb, a.wait_ns);
   if ((p.epi == EPI_XENT_STATS || p.epi == EPI_XENT_GRAD) && p.splits != 1) return TP_ERR_UNSUPPORTED;
   if (split_epi) {
     const size_t need = gemm_split_ws_bytes(p.M, p.N, p.splits, p.zpart != nullptr);
@@ -1130,29 +1107,71 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
     if (cudaMemsetAsync(a.counters, 0, htiles * sizeof(int), stream) != cudaSuccess)
       return TP_ERR_CUDA;
   }
-  // operand maps: A boxes of 128 rows (K-major) or 64 x 64 blocks (MN-major);
-  // B boxes of BNT / CG rows (K-major) or 64 x 64 blocks (MN-major)
+  // operand maps: A boxes of 128·RH rows (K-major) or 64 x 64 blocks
+  // (MN-major); B boxes of BNT / CG rows (K-major) or 64 x 64 blocks (MN-major)
   const uint32_t b_rows = static_cast<uint32_t>(BNT / CG);
   bool ok;
   if (!p.a_mn)
-    ok = make_tmap(&prm.tmA, p.A, p.K, p.M, p.lda, BK, static_cast<uint32_t>(BM * RH));
+    ok = make_tmap(tmA, p.A, p.K, p.M, p.lda, BK, static_cast<uint32_t>(BM * RH));
   else
-    ok = make_tmap(&prm.tmA, p.A, p.M, p.K, p.lda, 64, BK);
+    ok = make_tmap(tmA, p.A, p.M, p.K, p.lda, 64, BK);
   if (!ok) return TP_ERR_CUDA;
   if (!p.b_mn)
-    ok = make_tmap(&prm.tmB, p.B, p.K, p.N, p.ldb, BK, b_rows);
+    ok = make_tmap(tmB, p.B, p.K, p.N, p.ldb, BK, b_rows);
   else
-    ok = make_tmap(&prm.tmB, p.B, p.N, p.K, p.ldb, 64, BK);
-  if (!ok) return TP_ERR_CUDA;
-  const int slots = CG == 2 ? num_sms() / 2 : num_sms();
-  const int used = a.num_units < slots ? a.num_units : slots;
-  if (CG == 2) {
-    if (RH == 2) return launch_epi<2, 256, 2>(prm, epi, used, stream);
-    return BNT == 256 ? launch_epi<2, 256, 1>(prm, epi, used, stream)
-                      : launch_epi<2, 128, 1>(prm, epi, used, stream);
+    ok = make_tmap(tmB, p.B, p.N, p.K, p.ldb, 64, BK);
+  return ok ? TP_OK : TP_ERR_CUDA;
+}
+
+tp_status dispatch(GemmParams& prm, const TileChoice& tile, int epi, cudaStream_t stream) {
+  take_injection(prm.a[0].inject_unit, prm.a[0].inject_kb, prm.a[0].wait_ns);
+  prm.a[1].wait_ns = prm.a[0].wait_ns;
+  const int slots = tile.cg == 2 ? num_sms() / 2 : num_sms();
+  const int used = prm.total_units < slots ? prm.total_units : slots;
+  if (tile.cg == 2) {
+    if (tile.rh == 2) return launch_epi<2, 256, 2>(prm, epi, used, stream);
+    return tile.bn == 256 ? launch_epi<2, 256, 1>(prm, epi, used, stream)
+                          : launch_epi<2, 128, 1>(prm, epi, used, stream);
   }
-  return BNT == 256 ? launch_epi<1, 256, 1>(prm, epi, used, stream)
-                    : launch_epi<1, 128, 1>(prm, epi, used, stream);
+  return tile.bn == 256 ? launch_epi<1, 256, 1>(prm, epi, used, stream)
+                        : launch_epi<1, 128, 1>(prm, epi, used, stream);
+}
+
+}  // namespace
+
+tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
+  const bool split_epi = p.splits > 1 || p.zpart != nullptr;
+  const int epi = split_epi ? EPI_SPLIT_SUM : p.epi;
+  const TileChoice tile = choose_tile(p.M, p.N, p.K, p.splits, epi);
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (tp_status st = setup_problem(p, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], stream)) return st;
+  prm.a[1] = prm.a[0];
+  prm.tmA[1] = prm.tmA[0];
+  prm.tmB[1] = prm.tmB[0];
+  prm.units0 = prm.a[0].num_units;
+  prm.total_units = prm.units0;
+  return dispatch(prm, tile, epi, stream);
+}
+
+tp_status gemm_tc_launch_pair(const GemmProblem& p0, const GemmProblem& p1, cudaStream_t stream) {
+  // two independent problems of one epilogue, no split, no partials: one launch
+  if (p0.splits != 1 || p1.splits != 1 || p0.zpart || p1.zpart || p0.epi != p1.epi ||
+      p0.epi == EPI_XENT_STATS || p0.epi == EPI_XENT_GRAD || p0.dbias_part || p1.dbias_part)
+    return TP_ERR_UNSUPPORTED;
+  // the tile shape of the larger problem, and pairs of CTAs only when both
+  // are more than one 128-row tile high
+  const bool first_larger = static_cast<double>(p0.M) * p0.N >= static_cast<double>(p1.M) * p1.N;
+  const GemmProblem& big = first_larger ? p0 : p1;
+  TileChoice tile = choose_tile(big.M, big.N, big.K, 1, p0.epi);
+  if ((p0.M <= BM || p1.M <= BM) && tile.cg == 2) tile = TileChoice{1, 256, 1};
+  GemmParams prm;
+  memset(&prm, 0, sizeof(prm));
+  if (tp_status st = setup_problem(p0, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], stream)) return st;
+  if (tp_status st = setup_problem(p1, tile, prm.a[1], &prm.tmA[1], &prm.tmB[1], stream)) return st;
+  prm.units0 = prm.a[0].num_units;
+  prm.total_units = prm.units0 + prm.a[1].num_units;
+  return dispatch(prm, tile, p0.epi, stream);
 }
 
 void arm_gemm_injection(int unit, int kb, uint64_t wait_ns) {

@@ -71,6 +71,11 @@ size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart);
 
 tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream);
 
+// Two independent problems with the same epilogue (no split, no partials, no
+// dbias) in one launch: the second's tiles fill the first's last wave.
+// Returns TP_ERR_UNSUPPORTED for problems it cannot pair.
+tp_status gemm_tc_launch_pair(const GemmProblem& p0, const GemmProblem& p1, cudaStream_t stream);
+
 // Arm the one-shot debug injection of the next gemm_tc_launch.
 void arm_gemm_injection(int unit, int kb, uint64_t wait_ns);
 

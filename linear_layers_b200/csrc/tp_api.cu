@@ -371,7 +371,7 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   tp_status s = bf16 ? gemm_tc_launch(g3, st) : gemm_simt_launch(g3, st);
   if (s) return s;
 
-  // dB_i = Y_iᵀ·dZ  (both operands MN-major)
+  // dB_i = Y_iᵀ·dZ and dA_i = Xᵀ·dU_i (independent: one launch in bf16)
   GemmProblem g4;
   g4.A = Y; g4.lda = F; g4.a_mn = 1;
   g4.B = dZ; g4.ldb = h; g4.b_mn = 1;
@@ -379,9 +379,6 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   g4.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   g4.out0 = dB; g4.ldo = h;
   g4.dev_status = dev_status;
-  if ((s = bf16 ? gemm_tc_launch(g4, st) : gemm_simt_launch(g4, st))) return s;
-
-  // dA_i = Xᵀ·dU_i
   GemmProblem g5;
   g5.A = X; g5.lda = h; g5.a_mn = 1;
   g5.B = dU; g5.ldb = F; g5.b_mn = 1;
@@ -389,7 +386,12 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   g5.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   g5.out0 = dA; g5.ldo = F;
   g5.dev_status = dev_status;
-  if ((s = bf16 ? gemm_tc_launch(g5, st) : gemm_simt_launch(g5, st))) return s;
+  if (bf16) {
+    if ((s = gemm_tc_launch_pair(g4, g5, st))) return s;
+  } else {
+    if ((s = gemm_simt_launch(g4, st))) return s;
+    if ((s = gemm_simt_launch(g5, st))) return s;
+  }
 
   // f backward: dX = Σ_i dU_i·A_iᵀ
   GemmProblem g6;
@@ -505,8 +507,6 @@ tp_status tp_col_linear_bwd(const void* X, const void* W, const void* U, const v
   gw.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   gw.out0 = dW; gw.ldo = Nout;
   gw.dev_status = dev_status;
-  tp_status s = bf16 ? gemm_tc_launch(gw, st) : gemm_simt_launch(gw, st);
-  if (s) return s;
   // f backward: dX = Σ_i dU_i·W_iᵀ
   GemmProblem gx;
   gx.A = grad; gx.lda = Nout; gx.a_mn = 0;
@@ -515,7 +515,15 @@ tp_status tp_col_linear_bwd(const void* X, const void* W, const void* U, const v
   gx.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   gx.out0 = dX; gx.ldo = K;
   gx.dev_status = dev_status;
-  if ((s = run_row_parallel(gx, offs, nullptr, ws, split_bytes, bf16, st))) return s;
+  tp_status s;
+  if (bf16 && choose_splits(M, K, Nout, offs, sms_or_default()) == 1) {
+    // the shard sum stays in the accumulator: dW and dX in one launch
+    fill_splits(gx, offs, 1);
+    if ((s = gemm_tc_launch_pair(gw, gx, st))) return s;
+  } else {
+    if ((s = bf16 ? gemm_tc_launch(gw, st) : gemm_simt_launch(gw, st))) return s;
+    if ((s = run_row_parallel(gx, offs, nullptr, ws, split_bytes, bf16, st))) return s;
+  }
   if (dbias) return dbias_finish_launch(dbias_part, static_cast<int>(mtiles),
                                         static_cast<int>(Nout), dbias, st);
   return TP_OK;
@@ -564,9 +572,7 @@ tp_status tp_row_linear_bwd(const void* Xin, const void* W, const void* dZ, int6
   gx.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   gx.out0 = dXin; gx.ldo = Kin;
   gx.dev_status = dev_status;
-  tp_status s = bf16 ? gemm_tc_launch(gx, st) : gemm_simt_launch(gx, st);
-  if (s) return s;
-  // dW = Xinᵀ·dZ
+  // dW = Xinᵀ·dZ (independent of dXin: one launch in bf16)
   GemmProblem gw;
   gw.A = Xin; gw.lda = Kin; gw.a_mn = 1;
   gw.B = dZ; gw.ldb = Nout; gw.b_mn = 1;
@@ -574,7 +580,10 @@ tp_status tp_row_linear_bwd(const void* Xin, const void* W, const void* dZ, int6
   gw.epi = bf16 ? EPI_STORE_BF16 : EPI_STORE_F32;
   gw.out0 = dW; gw.ldo = Nout;
   gw.dev_status = dev_status;
-  return bf16 ? gemm_tc_launch(gw, st) : gemm_simt_launch(gw, st);
+  if (bf16) return gemm_tc_launch_pair(gx, gw, st);
+  tp_status s = gemm_simt_launch(gx, st);
+  if (s) return s;
+  return gemm_simt_launch(gw, st);
 }
 
 tp_status vp_embed(const int64_t* ids, int64_t T, const void* E, int64_t v, int64_t h, int32_t N,
