@@ -614,7 +614,7 @@ def run_gpu(args):
         raise SystemExit(f"--parts must name some of {','.join(known)}")
     if args.vocab_tokens:
         VOC["T"] = args.vocab_tokens
-    full = parts == list(PARTS) and VOC["T"] == 16384
+    full = parts == list(PARTS) and VOC["T"] == 16384 and not args.partial
     if full:   # the side loops need their vocabulary buffers too
         parts_prep = parts + list(BWD_PARTS) + list(FUSED_PARTS)
     else:
@@ -951,6 +951,8 @@ def main():
                     help="tokens of the vocabulary path (profiling runs; default 16384)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-library-context", action="store_true")
+    ap.add_argument("--partial", action="store_true",
+                    help="report part times only, also for the whole step (sweeps)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, always
     if args.impl == "reference":

@@ -859,6 +859,13 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
   return r == CUDA_SUCCESS;
 }
 
+// Programmatic dependent launch of the GEMMs; TP_GEMM_NO_PDL=1 turns it off
+// (sweeps).
+bool pdl_enabled() {
+  const char* e = std::getenv("TP_GEMM_NO_PDL");
+  return !(e && e[0] == '1');
+}
+
 // Launch with `slots` persistent CTAs (CG = 1) or CTA pairs (CG = 2), capped
 // at the number that can be resident at once, so that no persistent slot
 // starts only after another has finished.
@@ -883,7 +890,7 @@ tp_status launch_impl(const GemmParams& prm, int slots, cudaStream_t stream) {
   attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   if (!max_resident[dev & 63]) {
     if (cudaFuncSetAttribute(gemm_tc_kernel<CG, BNT, RH, EPI>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::kAlloc) != cudaSuccess)
@@ -1155,6 +1162,12 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
 }
 
 tp_status gemm_tc_launch_pair(const GemmProblem& p0, const GemmProblem& p1, cudaStream_t stream) {
+  // TP_GEMM_NO_PAIR=1 runs the two problems as two launches (sweeps)
+  if (const char* e = std::getenv("TP_GEMM_NO_PAIR"))
+    if (e[0] == '1') {
+      if (tp_status st = gemm_tc_launch(p0, stream)) return st;
+      return gemm_tc_launch(p1, stream);
+    }
   // two independent problems of one epilogue, no split, no partials: one launch
   if (p0.splits != 1 || p1.splits != 1 || p0.zpart || p1.zpart || p0.epi != p1.epi ||
       p0.epi == EPI_XENT_STATS || p0.epi == EPI_XENT_GRAD || p0.dbias_part || p1.dbias_part)
