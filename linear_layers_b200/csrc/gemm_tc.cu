@@ -39,14 +39,14 @@
 #include "internal.h"
 #include "sm100_ptx.cuh"
 
-// per-SM throughput of the tall tile relative to the 256 x 256 pair tile
-// (measured on the h = 4096 MLP GEMMs: 1.05-1.08)
+// per-SM throughput of the tall tile relative to the 256 x 256 pair tile when
+// it is forced (alone on the h = 4096 MLP GEMMs: 1.0-1.05)
 #ifndef TP_GEMM_TALL_EFF
-#define TP_GEMM_TALL_EFF 1.08
+#define TP_GEMM_TALL_EFF 1.0
 #endif
 
 #ifndef TP_GEMM_STAGE_BUDGET
-#define TP_GEMM_STAGE_BUDGET 229376u
+#define TP_GEMM_STAGE_BUDGET 196608u
 #endif
 
 namespace tpl {
@@ -115,14 +115,16 @@ struct Cfg {
   static constexpr int kBCols = BNT / CG;        // B columns staged per CTA
   static constexpr uint32_t kABytes = kRowsCTA * BK * 2;
   static constexpr uint32_t kBBytes = kBCols * BK * 2;
-  // TP_GEMM_STAGE_BUDGET bytes of operand stages (default 224 KB: 7 stages of
-  // the 2 x 256 tile, 4 of 1 x 256 and of the tall tile, 9 of 2 x 128, 7 of 1 x 128)
+  // TP_GEMM_STAGE_BUDGET bytes of operand stages (default 192 KB: 6 stages of
+  // the 2 x 256 tile, 4 of 1 x 256 and of the tall tile, 8 of 2 x 128, 6 of
+  // 1 x 128; a seventh stage measured no faster)
   static constexpr int kStages = static_cast<int>(TP_GEMM_STAGE_BUDGET / (kABytes + kBBytes));
   static constexpr uint32_t kOffB = kStages * kABytes;
   static constexpr uint32_t kOffBar = kOffB + kStages * kBBytes;
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr uint32_t kBytes = kOffMisc + 16;
+  static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;   // dbias quadrant sums
+  static constexpr uint32_t kBytes = kOffRed + 4 * BNT * 4;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators, or two row halves
   static constexpr int kAccBufs = RH == 2 ? 1 : 2;    // accumulator buffers in tensor memory
@@ -305,6 +307,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
   volatile int* bcast = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 8);
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -794,14 +797,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                               a.N - col0);
             }
             if (a.dbias_part != nullptr) {
-              // this warp's 32 rows: one partial row of the 32-row tiling,
-              // written only when it holds rows of the problem (rows past M
-              // contribute zeros and have no partial row)
               const float colsum = warp_column_sums(v, lane);
-              const int prow = ((tm * CG + static_cast<int>(rank)) * RH + hr) * 4 + q;
-              if (prow * 32 < a.M && col0 + lane < a.N)
-                a.dbias_part[static_cast<int64_t>(prow) * a.N + col0 + lane] = colsum;
+              red[q * BNT + c * 32 + lane] = colsum;
             }
+          }
+        }
+        if constexpr (kDact) {
+          if (a.dbias_part != nullptr) {
+            // one partial row per 128-row piece: the four lane quadrants'
+            // column sums added in a fixed order
+            named_barrier_sync(1, kEpiThreads);
+            const int cc = et;   // one column per epilogue thread (BNT <= 256 columns)
+            const int col = tn * BNT + cc;
+            const int prow = (tm * CG + static_cast<int>(rank)) * RH + hr;
+            if (cc < BNT && col < a.N && prow * BM < a.M) {   // pieces past M hold no rows
+              const float sum = ((red[cc] + red[BNT + cc]) + red[2 * BNT + cc]) + red[3 * BNT + cc];
+              a.dbias_part[static_cast<int64_t>(prow) * a.N + col] = sum;
+            }
+            named_barrier_sync(1, kEpiThreads);
           }
         }
       }
@@ -988,7 +1001,11 @@ TileChoice choose_tile(int M, int N, int K, int splits, int epi) {
     else if (!std::strcmp(e, "1x128")) t = {1, 128, 1};
     if (t.cg && !(xent && t.bn != 256)) return t;
   }
-  const TileChoice cands[5] = {{2, 256, 1}, {2, 256, 2}, {2, 128, 1}, {1, 256, 1}, {1, 128, 1}};
+  // The tall tile is not among the automatic choices: in the whole layer
+  // step (after the logits and the cross-entropy have filled L2 with their
+  // write-backs) its non-overlapped epilogue made the MLP about 19 % slower,
+  // although alone it ties or beats the 256 x 256 pair tile.
+  const TileChoice cands[4] = {{2, 256, 1}, {2, 128, 1}, {1, 256, 1}, {1, 128, 1}};
   TileChoice best{M > BM ? 2 : 1, 256, 1};
   double best_cost = 0.0;
   bool have = false;

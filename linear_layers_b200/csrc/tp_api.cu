@@ -351,7 +351,8 @@ tp_status mlp_bwd_impl(const void* X, const void* A, const void* B, const void* 
   const bool bf16 = dt == TP_DTYPE_BF16;
   cudaStream_t st = as_stream(stream);
 
-  const int64_t mtiles = (M + 31) / 32;   // dbias partial rows: one per 32 token rows
+  // dbias partial rows: one per 128-row piece (tensor cores) or per 32-row tile (fp32 path)
+  const int64_t mtiles = bf16 ? (M + 127) / 128 : (M + 31) / 32;
   const size_t split_bytes = bf16 ? row_split_ws(M, h, F, N, false) : 0;
   const size_t dbias_bytes = dbias ? dbias_ws(M, F) : 0;
   if (split_bytes + dbias_bytes > 0 && (ws == nullptr || ws_bytes < split_bytes + dbias_bytes))
