@@ -9,21 +9,21 @@
 //
 //   O = softmax(Q·Kᵀ·scale + causal mask)·V,  head_dim 64, bf16 in and out
 //
-// One CTA computes two 128-query tiles (2p and 2p+1) of one head of one
-// sequence, streaming 128-key blocks shared by both (flash-style online
-// softmax), in the ping-pong order that keeps the tensor core busy while
-// either tile's softmax runs:
-//   warp 0    TMA: both Q tiles once, K and V blocks into a two-stage ring;
-//   warp 1    owns tensor memory; one lane issues, per tile g, S_g = Q_g·Kᵀ
-//             (128 x 128 fp32) and O_g = P_g·V (128 x 64 fp32) with
-//             tcgen05.mma: P·V of block j and S of block j+1 for one tile as
-//             soon as its softmax has released block j, then the other's;
-//   warps 2-5 and 6-9, one warpgroup per tile, one query row per thread (its
-//             TMEM lane): row maximum, p = 2^(x − m) in the log2 domain, P
-//             as bf16 written into shared memory in the 128-byte-swizzled
-//             K-major layout the MMA reads, the running sum, and O
-//             accumulated in registers as O = O·2^(m_old − m_new) + O_blk,
-//             so O never goes back to tensor memory.
+// One CTA computes one 128-query tile of one head of one sequence, streaming
+// 64-key blocks (flash-style online softmax); two or three CTAs share an SM,
+// each with its own pipeline, so one CTA's MMAs run while another's softmax
+// does and the uneven causal tiles (launched heaviest first) balance:
+//   warp 0    TMA: the Q tile once, K and V blocks into a two-stage ring;
+//   warp 1    owns 128 tensor-memory columns; one lane issues S = Q·Kᵀ
+//             (128 x 64 fp32) as soon as the softmax has read the previous
+//             S into registers, and O += P·V (128 x 64 fp32, accumulated in
+//             tensor memory) once the softmax has written P;
+//   warps 2-5 the softmax, one query row per thread (its TMEM lane): the
+//             block's scores read in one round trip and released, row
+//             maximum, p = 2^(x − m) in the log2 domain as bf16 into shared
+//             memory in the 128-byte-swizzled K-major layout the MMA reads,
+//             the running sum; O is rescaled in tensor memory only when a
+//             row's maximum grows by more than 2^8.
 // Every wait is bounded: on a timeout the kernel sets TP_DEVERR_TIMEOUT,
 // lets its copies and MMAs finish and returns.
 #include <cuda.h>
@@ -41,28 +41,29 @@ namespace tpl {
 namespace {
 
 constexpr int kBQ = 128;                       // queries per tile (TMEM lanes)
-constexpr int kBK = 128;                       // keys per block
+constexpr int kFK = 64;                        // keys per forward block
 constexpr int kHD = 64;                        // head dimension: one 128-byte row
-constexpr int kAttnThreads = 320;              // 10 warps
+constexpr int kFwdThreads = 192;               // 6 warps
 constexpr int kSoftmaxThreads = 128;           // one warpgroup per query tile
 constexpr int kMaxHeads = 256;
 constexpr uint32_t kTile = kBQ * kHD * 2;      // 16 KB: 128 rows of 128 bytes
-constexpr uint32_t kOffQ = 0;                          // 2 tiles
-constexpr uint32_t kOffK = kOffQ + 2 * kTile;          // 2 stages
-constexpr uint32_t kOffV = kOffK + 2 * kTile;          // 2 stages
-constexpr uint32_t kOffP = kOffV + 2 * kTile;          // per tile: 2 chunks of 64 keys
-constexpr uint32_t kPBytes = 2 * kTile;
-constexpr uint32_t kOffBar = kOffP + 2 * kPBytes;
-constexpr int kNumBars = 12;
-constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
-constexpr uint32_t kAttnBytes = kOffMisc + 16;
-constexpr uint32_t kAttnAlloc = kAttnBytes + 1024;     // slack for 1024-byte alignment
-constexpr uint32_t kTmemCols = 512;                    // S: 2 x 128, O: 2 x 64
-constexpr uint32_t kTmemO = 256;
+constexpr uint32_t kKVTile = kFK * kHD * 2;    // 8 KB: 64 rows of 128 bytes
+// forward shared memory: Q, K and V in a two-stage ring, P (128 rows x 64 keys)
+constexpr uint32_t kFOffQ = 0;
+constexpr uint32_t kFOffK = kFOffQ + kTile;
+constexpr uint32_t kFOffV = kFOffK + 2 * kKVTile;
+constexpr uint32_t kFOffP = kFOffV + 2 * kKVTile;
+constexpr uint32_t kFOffBar = kFOffP + kBQ * kFK * 2;
+constexpr int kFNumBars = 10;
+constexpr uint32_t kFOffMisc = kFOffBar + kFNumBars * 8;
+constexpr uint32_t kFwdAlloc = kFOffMisc + 16 + 1024;     // slack for 1024-byte alignment
+constexpr uint32_t kFwdTmemCols = 128;                     // S: 64, O: 64
+constexpr uint32_t kFTmemO = 64;
+constexpr uint32_t kTmemCols = 512;                        // backward
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct AttnArgs {
-  int b, s, heads, nqb, npairs;
+  int b, s, heads, nqb;
   int causal;
   float scale_log2;          // scale · log2(e)
   __nv_bfloat16* ctx;
@@ -74,7 +75,8 @@ struct AttnArgs {
 };
 
 struct __align__(64) AttnParams {
-  CUtensorMap tm;            // QKV [b·s, 3h], boxes of 64 columns x 128 rows
+  CUtensorMap tm;            // QKV [b·s, 3h], boxes of 64 columns x 128 rows (Q)
+  CUtensorMap tm_kv;         // QKV, boxes of 64 columns x 64 rows (K and V blocks)
   AttnArgs a;
 };
 
@@ -96,24 +98,24 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // rescaled only on those rare moves instead of after every block.
 constexpr float kTau = 8.0f;
 
-// All 128 scores of this thread's row of one block, read from tensor memory
-// in one round trip (four 32-column loads, one wait).  With kMask, keys at
+// All 64 scores of this thread's row of one block, read from tensor memory
+// in one round trip (two 32-column loads, one wait).  With kMask, keys at
 // positions >= klim become −inf.  Returns the row maximum.
 template <bool kMask>
 __device__ __forceinline__ float load_block_row(uint32_t sbase, int kpos0, int klim,
-                                                uint32_t (&x)[kBK]) {
+                                                uint32_t (&x)[kFK]) {
 #pragma unroll
-  for (int c = 0; c < kBK / 32; ++c)
+  for (int c = 0; c < kFK / 32; ++c)
     tmem_ld_32x32b_x32(sbase + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&x[c * 32]));
   tc_wait_ld();
   if (kMask) {
 #pragma unroll
-    for (int t = 0; t < kBK; ++t)
+    for (int t = 0; t < kFK; ++t)
       if (kpos0 + t >= klim) x[t] = 0xff800000u;   // −inf
   }
   float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int t = 0; t < kBK; t += 8) {
+  for (int t = 0; t < kFK; t += 8) {
     float& a = acc[(t >> 3) & 3];
     a = fmax3(a, __uint_as_float(x[t]), __uint_as_float(x[t + 1]));
     a = fmax3(a, __uint_as_float(x[t + 2]), __uint_as_float(x[t + 3]));
@@ -124,29 +126,25 @@ __device__ __forceinline__ float load_block_row(uint32_t sbase, int kpos0, int k
 }
 
 // p = 2^(x·sl − m) of the row, stored as bf16 into this row of the P tile
-// (two 64-key chunks of 128-byte rows, 16-byte granule g at g ^ (row & 7):
-// the 128-byte swizzle the MMA's descriptor names).  Returns Σ p.
-__device__ __forceinline__ float exp_store_row(const uint32_t (&x)[kBK], float sl, float m,
+// (one 128-byte row of 64 keys, 16-byte granule g at g ^ (row & 7): the
+// 128-byte swizzle the MMA's descriptor names).  Returns Σ p.
+__device__ __forceinline__ float exp_store_row(const uint32_t (&x)[kFK], float sl, float m,
                                                uint8_t* prow, int r) {
   float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int h = 0; h < kBK / 64; ++h) {
-    uint8_t* chunk = prow + h * kTile;
+  for (int gr = 0; gr < 8; ++gr) {            // 16-byte granule of the 128-byte row
+    float p[8];
 #pragma unroll
-    for (int gr = 0; gr < 8; ++gr) {            // 16-byte granule of the 128-byte row
-      float p[8];
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        p[t] = ex2f(fmaf(__uint_as_float(x[h * 64 + gr * 8 + t]), sl, -m));
-        ps[t & 3] += p[t];
-      }
-      uint4 w;
-      w.x = pack_bf16x2(p[0], p[1]);
-      w.y = pack_bf16x2(p[2], p[3]);
-      w.z = pack_bf16x2(p[4], p[5]);
-      w.w = pack_bf16x2(p[6], p[7]);
-      *reinterpret_cast<uint4*>(chunk + ((gr ^ (r & 7)) << 4)) = w;
+    for (int t = 0; t < 8; ++t) {
+      p[t] = ex2f(fmaf(__uint_as_float(x[gr * 8 + t]), sl, -m));
+      ps[t & 3] += p[t];
     }
+    uint4 w;
+    w.x = pack_bf16x2(p[0], p[1]);
+    w.y = pack_bf16x2(p[2], p[3]);
+    w.z = pack_bf16x2(p[4], p[5]);
+    w.w = pack_bf16x2(p[6], p[7]);
+    *reinterpret_cast<uint4*>(prow + ((gr ^ (r & 7)) << 4)) = w;
   }
   return (ps[0] + ps[1]) + (ps[2] + ps[3]);
 }
@@ -158,43 +156,39 @@ __device__ __forceinline__ void attn_timeout(const AttnArgs& a, volatile int* ab
   }
 }
 
-__global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
+__global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_constant__ AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const AttnArgs& a = P.a;
-  uint8_t* sQ = smem + kOffQ;
-  uint8_t* sK = smem + kOffK;
-  uint8_t* sV = smem + kOffV;
-  uint8_t* sP = smem + kOffP;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+  uint8_t* sQ = smem + kFOffQ;
+  uint8_t* sK = smem + kFOffK;
+  uint8_t* sV = smem + kFOffV;
+  uint8_t* sP = smem + kFOffP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFOffBar);
   uint64_t* q_full = bars;
   uint64_t* kv_full = bars + 1;        // [stage]
   uint64_t* kv_empty = bars + 3;       // [stage]
-  uint64_t* s_full = bars + 5;         // [tile]: S_j ready, and every earlier MMA of the CTA done
-  uint64_t* p_full = bars + 7;         // [tile]: P_j written, S_j read, O rescaled
-  uint64_t* o_full = bars + 9;         // [tile]: the last P·V done (O final)
-  uint64_t* mma_done = bars + 11;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffMisc + 4);
+  uint64_t* s_full = bars + 5;         // S(j) in tensor memory
+  uint64_t* s_free = bars + 6;         // S(j) read into the softmax's registers
+  uint64_t* p_full = bars + 7;         // P(j) written, O rescaled
+  uint64_t* o_full = bars + 8;         // P·V(j) done: O current, P buffer free
+  uint64_t* mma_done = bars + 9;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kFOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kFOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // the pairs of the last query tiles (the longest under the causal mask) first
+  // the last query tiles (the longest under the causal mask) first
   const int bh = a.b * a.heads;
-  const int pair = a.npairs - 1 - static_cast<int>(blockIdx.x) / bh;
+  const int qb = a.nqb - 1 - static_cast<int>(blockIdx.x) / bh;
   const int rem = static_cast<int>(blockIdx.x) % bh;
   const int head = rem / a.b;
   const int batch = rem % a.b;
   const int row0 = batch * a.s;                         // first token row of the sequence
-  const int nkb_all = (a.s + kBK - 1) / kBK;
-  int nkb[2];                                           // key blocks of each tile (0: absent)
-#pragma unroll
-  for (int g = 0; g < 2; ++g) {
-    const int qb = 2 * pair + g;
-    nkb[g] = qb >= a.nqb ? 0 : (a.causal ? min(qb + 1, nkb_all) : nkb_all);
-  }
-  const int nkb_max = max(nkb[0], nkb[1]);
+  const int nkb_all = (a.s + kFK - 1) / kFK;
+  // key blocks of this tile: up to the tile's last query under the causal mask
+  const int nk = a.causal ? min((qb + 1) * (kBQ / kFK), nkb_all) : nkb_all;
   const int qcol = a.head_cols[head].x;
   const int kcol = qcol + a.head_cols[head].y;
   const int vcol = kcol + a.head_cols[head].y;
@@ -204,16 +198,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     for (int i = 0; i < 2; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kSoftmaxThreads);
-      mbar_init(&o_full[i], 1);
     }
+    mbar_init(s_full, 1);
+    mbar_init(s_free, kSoftmaxThreads);
+    mbar_init(p_full, kSoftmaxThreads);
+    mbar_init(o_full, 1);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_alloc(tmem_slot, kFwdTmemCols);
     tmem_relinquish();
   }
   tc_fence_before_sync();
@@ -225,24 +220,24 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     // ------------------------------------------------------------ TMA
     if (elect_one_sync()) {
       tma_prefetch_desc(&P.tm);
-      mbar_arrive_expect_tx(q_full, nkb[1] > 0 ? 2 * kTile : kTile);
-      tma_load_2d(sQ, &P.tm, q_full, qcol, row0 + 2 * pair * kBQ);
-      if (nkb[1] > 0) tma_load_2d(sQ + kTile, &P.tm, q_full, qcol, row0 + (2 * pair + 1) * kBQ);
+      tma_prefetch_desc(&P.tm_kv);
+      mbar_arrive_expect_tx(q_full, kTile);
+      tma_load_2d(sQ, &P.tm, q_full, qcol, row0 + qb * kBQ);
       int issued = 0;
-      for (int j = 0; j < nkb_max; ++j) {
+      for (int j = 0; j < nk; ++j) {
         const int st = j & 1;
         const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
         if (!mbar_wait_bounded(&kv_empty[st], ph ^ 1u, a.wait_ns, abort_flag)) {
           attn_timeout(a, abort_flag);
           break;
         }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * kTile);
-        tma_load_2d(sK + st * kTile, &P.tm, &kv_full[st], kcol, row0 + j * kBK);
-        tma_load_2d(sV + st * kTile, &P.tm, &kv_full[st], vcol, row0 + j * kBK);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * kKVTile);
+        tma_load_2d(sK + st * kKVTile, &P.tm_kv, &kv_full[st], kcol, row0 + j * kFK);
+        tma_load_2d(sV + st * kKVTile, &P.tm_kv, &kv_full[st], vcol, row0 + j * kFK);
         ++issued;
       }
       // every copy lands before the CTA can exit (bounded, not cut short by
-      // the abort flag): the Q tiles and the last two K/V stages
+      // the abort flag): the Q tile and the last two K/V stages
       volatile int keep_waiting = 0;
       mbar_wait_bounded(q_full, 0, a.wait_ns, &keep_waiting);
       for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
@@ -252,54 +247,49 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (elect_one_sync()) {
-      constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBK, false, false);   // Q K-major, K K-major
+      constexpr uint32_t idS = idesc_bf16_f32(kBQ, kFK, false, false);   // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, V MN-major
       bool any = false;
-      // S_g(j) = Q_g·K_jᵀ.  Issued only after the softmax has released S_g(j-1)
-      // (p_full of j-1, taken by issue_pv) and after P·V of j-1, so the
-      // commit's arrival also tells the softmax that O_g holds every block
-      // before j and that the P buffer is free.
-      auto issue_s = [&](int g, int j) -> bool {
+      const uint32_t qa = smem_u32(sQ), pa = smem_u32(sP);
+      // S(j) = Q·K_jᵀ into the S columns
+      auto issue_s = [&](int j) -> bool {
         const int st = j & 1;
         if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.wait_ns,
                                abort_flag))
           return false;
         tc_fence_after_sync();
-        const uint32_t qa = smem_u32(sQ + g * kTile), kb = smem_u32(sK + st * kTile);
+        const uint32_t kb = smem_u32(sK + st * kKVTile);
 #pragma unroll
         for (int k = 0; k < kHD / 16; ++k)
-          tc_mma_bf16(tmem + g * kBK, smem_desc_sw128(qa + k * 32, 16, 1024),
+          tc_mma_bf16(tmem, smem_desc_sw128(qa + k * 32, 16, 1024),
                       smem_desc_sw128(kb + k * 32, 16, 1024), idS, k > 0 ? 1u : 0u);
         any = true;
-        tc_commit(&s_full[g]);
-        return true;
-      };
-      // O_g += P_g(j)·V_j in tensor memory, once the softmax has written P_g(j)
-      // and rescaled O_g where its running maximum moved
-      auto issue_pv = [&](int g, int j) -> bool {
-        if (!mbar_wait_bounded(&p_full[g], static_cast<uint32_t>(j & 1), a.wait_ns, abort_flag))
-          return false;
-        tc_fence_after_sync();
-        const uint32_t pa = smem_u32(sP + g * kPBytes), vb = smem_u32(sV + (j & 1) * kTile);
-#pragma unroll
-        for (int k = 0; k < kBK / 16; ++k)   // 16 keys per step; chunk of 64 keys = 16 KB
-          tc_mma_bf16(tmem + kTmemO + g * kHD,
-                      smem_desc_sw128(pa + (k >> 2) * kTile + (k & 3) * 32, 16, 1024),
-                      smem_desc_sw128(vb + k * 2048, 8192, 1024), idO,
-                      (j > 0 || k > 0) ? 1u : 0u);
-        if (j + 1 == nkb[g]) tc_commit(&o_full[g]);
+        tc_commit(s_full);
         return true;
       };
       bool ok = mbar_wait_bounded(q_full, 0, a.wait_ns, abort_flag);
-      for (int g = 0; ok && g < 2; ++g)
-        if (nkb[g] > 0) ok = issue_s(g, 0);
-      for (int j = 0; ok && j < nkb_max; ++j) {
-        for (int g = 0; ok && g < 2; ++g) {
-          if (j >= nkb[g]) continue;
-          ok = issue_pv(g, j);
-          if (ok && j + 1 < nkb[g]) ok = issue_s(g, j + 1);
+      if (ok && nk > 0) ok = issue_s(0);
+      for (int j = 0; ok && j < nk; ++j) {
+        // the next S as soon as the softmax holds S(j) in registers
+        if (j + 1 < nk) {
+          ok = mbar_wait_bounded(s_free, static_cast<uint32_t>(j & 1), a.wait_ns, abort_flag) &&
+               issue_s(j + 1);
+          if (!ok) break;
         }
-        if (ok) tc_commit(&kv_empty[j & 1]);   // K_j and V_j read by every MMA issued so far
+        // O += P(j)·V_j once the softmax has written P(j) (and rescaled O)
+        if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j & 1), a.wait_ns, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const uint32_t vb = smem_u32(sV + (j & 1) * kKVTile);
+#pragma unroll
+        for (int k = 0; k < kFK / 16; ++k)   // 16 keys per step
+          tc_mma_bf16(tmem + kFTmemO, smem_desc_sw128(pa + k * 32, 16, 1024),
+                      smem_desc_sw128(vb + k * 2048, 8192, 1024), idO,
+                      (j > 0 || k > 0) ? 1u : 0u);
+        tc_commit(o_full);
+        tc_commit(&kv_empty[j & 1]);   // K_j and V_j read by every MMA issued so far
       }
       if (!ok) attn_timeout(a, abort_flag);
       if (any) {   // every issued MMA completes before tensor memory is freed
@@ -310,16 +300,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int g = (warp - 2) >> 2;                  // query tile of this warpgroup
     const int qd = warp & 3;                        // TMEM lane quadrant of this warp
     const int r = qd * 32 + lane;                   // row of the query tile
-    const int qb = 2 * pair + g;
     const int qpos = qb * kBQ + r;                  // position in the sequence
-    const int nk = nkb[g];
     const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
-    const uint32_t sbase = tmem + lane_off + static_cast<uint32_t>(g * kBK);
-    const uint32_t obase = tmem + lane_off + kTmemO + static_cast<uint32_t>(g * kHD);
-    uint8_t* prow = sP + g * kPBytes + r * 128;
+    const uint32_t sbase = tmem + lane_off;
+    const uint32_t obase = tmem + lane_off + kFTmemO;
+    uint8_t* prow = sP + r * 128;
     const float sl = a.scale_log2;
     const int klim = a.causal ? min(qpos + 1, a.s) : a.s;   // keys [0, klim) are visible
     float m = -INFINITY;                            // running maximum (log2 units)
@@ -327,27 +314,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       // the warp's lanes agree before the warp-collective tensor-memory loads
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&s_full[g], static_cast<uint32_t>(j & 1),
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(s_full, static_cast<uint32_t>(j & 1),
                                                      a.wait_ns, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after_sync();
-      const int kpos0 = j * kBK;
-      const bool need_mask = (a.causal && j == qb) || kpos0 + kBK > a.s;
-      uint32_t x[kBK];
+      const int kpos0 = j * kFK;
+      const bool need_mask = (a.causal && kpos0 + kFK > qb * kBQ) || kpos0 + kFK > a.s;
+      uint32_t x[kFK];
       const float mx = need_mask ? load_block_row<true>(sbase, kpos0, klim, x)
                                  : load_block_row<false>(sbase, kpos0, klim, x);
-      const float m_blk = mx * sl;   // finite: every block a tile visits has a visible key
-      bool move = j == 0 || m_blk > m + kTau;
+      tc_fence_before_sync();
+      mbar_arrive(s_free);                          // S read: the MMA may compute S(j+1)
+      // finite at j = 0 (key 0 is visible to every row); a later block that
+      // is wholly masked for this row gives −inf and moves nothing
+      const float m_blk = mx * sl;
+      const bool move = j == 0 || m_blk > m + kTau;
       const float alpha = (j > 0 && move) ? ex2f(m - m_blk) : 1.0f;
       if (move) m = m_blk;
+      // P·V(j-1) has finished: the P buffer is free and O holds blocks 0..j-1
+      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(o_full, static_cast<uint32_t>((j - 1) & 1),
+                                                                a.wait_ns, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after_sync();
       // p = 2^(x·sl − m), bf16 into the swizzled P tile, and the row sum
       l = fmaf(l, alpha, exp_store_row(x, sl, m, prow, r));
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // O_g holds blocks 0..j-1 (the s_full arrival covers their P·V):
         // rescale the rows whose maximum moved, the others by 1, before the
-        // P·V of this block adds to it
+        // P·V of this block adds to O
 #pragma unroll
         for (int c = 0; c < kHD / 32; ++c) {
           uint32_t rr[32];
@@ -359,12 +356,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
         }
         tc_wait_st();
       }
-      tc_fence_before_sync();                      // S read and O written before the arrival
+      tc_fence_before_sync();                      // O written before the arrival
       fence_proxy_async_smem();                    // P visible to the tensor core
-      mbar_arrive(&p_full[g]);
+      mbar_arrive(p_full);
     }
     if (ok && nk > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_full[g], 0, a.wait_ns, abort_flag));
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_full, static_cast<uint32_t>((nk - 1) & 1),
+                                                     a.wait_ns, abort_flag));
     if (!ok) {
       if (lane == 0) attn_timeout(a, abort_flag);
     } else if (nk > 0) {
@@ -395,7 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_fwd_kernel(const __grid_
   __syncthreads();
   if (warp == 1) {
     tc_fence_after_sync();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, kFwdTmemCols);
   }
 }
 
@@ -877,7 +875,6 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
   a.s = static_cast<int>(s);
   a.heads = heads;
   a.nqb = static_cast<int>((s + kBQ - 1) / kBQ);
-  a.npairs = (a.nqb + 1) / 2;
   a.causal = causal ? 1 : 0;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.ctx = static_cast<__nv_bfloat16*>(ctx);
@@ -892,19 +889,21 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
       a.head_cols[first + hh] = make_int2(3 * kHD * first + hh * kHD, nh * kHD);
   }
   const uint64_t ncols = static_cast<uint64_t>(3) * heads * kHD;
-  if (!make_tmap_bf16_sw128(&prm.tm, QKV, ncols, static_cast<uint64_t>(b * s), ncols, kHD, kBQ))
+  if (!make_tmap_bf16_sw128(&prm.tm, QKV, ncols, static_cast<uint64_t>(b * s), ncols, kHD, kBQ) ||
+      !make_tmap_bf16_sw128(&prm.tm_kv, QKV, ncols, static_cast<uint64_t>(b * s), ncols, kHD, kFK))
     return TP_ERR_CUDA;
   static bool configured[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (!configured[dev & 63]) {
     if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kAttnAlloc)) != cudaSuccess)
+                             static_cast<int>(kFwdAlloc)) != cudaSuccess)
       return TP_ERR_CUDA;
     configured[dev & 63] = true;
   }
-  const int64_t grid = b * heads * a.npairs;
-  attn_fwd_kernel<<<static_cast<unsigned>(grid), kAttnThreads, kAttnAlloc, stream>>>(prm);
+  // one CTA per (sequence, head, query tile), the longest causal tiles first
+  const int64_t grid = b * heads * a.nqb;
+  attn_fwd_kernel<<<static_cast<unsigned>(grid), kFwdThreads, kFwdAlloc, stream>>>(prm);
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
