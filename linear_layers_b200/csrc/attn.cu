@@ -48,13 +48,15 @@ constexpr int kSoftmaxThreads = 128;           // one warpgroup per query tile
 constexpr int kMaxHeads = 256;
 constexpr uint32_t kTile = kBQ * kHD * 2;      // 16 KB: 128 rows of 128 bytes
 constexpr uint32_t kKVTile = kFK * kHD * 2;    // 8 KB: 64 rows of 128 bytes
-// forward shared memory: Q, K and V in a two-stage ring, P (128 rows x 64 keys)
+constexpr int kFStages = 3;                    // K/V ring depth
+constexpr uint32_t kPTileF = kBQ * kFK * 2;    // 16 KB: P of one block, bf16
+// forward shared memory: Q, K and V in a ring, P double buffered
 constexpr uint32_t kFOffQ = 0;
 constexpr uint32_t kFOffK = kFOffQ + kTile;
-constexpr uint32_t kFOffV = kFOffK + 2 * kKVTile;
-constexpr uint32_t kFOffP = kFOffV + 2 * kKVTile;
-constexpr uint32_t kFOffBar = kFOffP + kBQ * kFK * 2;
-constexpr int kFNumBars = 10;
+constexpr uint32_t kFOffV = kFOffK + kFStages * kKVTile;
+constexpr uint32_t kFOffP = kFOffV + kFStages * kKVTile;
+constexpr uint32_t kFOffBar = kFOffP + 2 * kPTileF;
+constexpr int kFNumBars = 4 + 2 * kFStages + 4;
 constexpr uint32_t kFOffMisc = kFOffBar + kFNumBars * 8;
 constexpr uint32_t kFwdAlloc = kFOffMisc + 16 + 1024;     // slack for 1024-byte alignment
 constexpr uint32_t kFwdTmemCols = 128;                     // S: 64, O: 64
@@ -128,16 +130,22 @@ __device__ __forceinline__ float load_block_row(uint32_t sbase, int kpos0, int k
 // p = 2^(x·sl − m) of the row, stored as bf16 into this row of the P tile
 // (one 128-byte row of 64 keys, 16-byte granule g at g ^ (row & 7): the
 // 128-byte swizzle the MMA's descriptor names).  Returns Σ p.
+// The scaling and the sums run on pairs (f32x2 FMA and add).
 __device__ __forceinline__ float exp_store_row(const uint32_t (&x)[kFK], float sl, float m,
                                                uint8_t* prow, int r) {
-  float ps[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  const float2 sl2 = make_float2(sl, sl);
+  const float2 nm2 = make_float2(-m, -m);
+  float2 ps[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
   for (int gr = 0; gr < 8; ++gr) {            // 16-byte granule of the 128-byte row
     float p[8];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      p[t] = ex2f(fmaf(__uint_as_float(x[gr * 8 + t]), sl, -m));
-      ps[t & 3] += p[t];
+    for (int t = 0; t < 8; t += 2) {
+      const float2 y = __ffma2_rn(make_float2(__uint_as_float(x[gr * 8 + t]),
+                                              __uint_as_float(x[gr * 8 + t + 1])), sl2, nm2);
+      p[t] = ex2f(y.x);
+      p[t + 1] = ex2f(y.y);
+      ps[(t >> 1) & 1] = __fadd2_rn(ps[(t >> 1) & 1], make_float2(p[t], p[t + 1]));
     }
     uint4 w;
     w.x = pack_bf16x2(p[0], p[1]);
@@ -146,7 +154,7 @@ __device__ __forceinline__ float exp_store_row(const uint32_t (&x)[kFK], float s
     w.w = pack_bf16x2(p[6], p[7]);
     *reinterpret_cast<uint4*>(prow + ((gr ^ (r & 7)) << 4)) = w;
   }
-  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+  return (ps[0].x + ps[1].x) + (ps[0].y + ps[1].y);
 }
 
 __device__ __forceinline__ void attn_timeout(const AttnArgs& a, volatile int* abort_flag) {
@@ -167,13 +175,13 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
   uint8_t* sP = smem + kFOffP;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kFOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;        // [stage]
-  uint64_t* kv_empty = bars + 3;       // [stage]
-  uint64_t* s_full = bars + 5;         // S(j) in tensor memory
-  uint64_t* s_free = bars + 6;         // S(j) read into the softmax's registers
-  uint64_t* p_full = bars + 7;         // P(j) written, O rescaled
-  uint64_t* o_full = bars + 8;         // P·V(j) done: O current, P buffer free
-  uint64_t* mma_done = bars + 9;
+  uint64_t* kv_full = bars + 1;                    // [stage]
+  uint64_t* kv_empty = kv_full + kFStages;         // [stage]
+  uint64_t* s_full = kv_empty + kFStages;          // S(j) in tensor memory
+  uint64_t* s_free = s_full + 1;                   // S(j) read into the softmax's registers
+  uint64_t* p_full = s_free + 1;                   // [j & 1] P(j) written, O rescaled
+  uint64_t* o_full = p_full + 2;                   // [j & 1] P·V(j) done: O current, P(j) free
+  uint64_t* mma_done = o_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kFOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kFOffMisc + 4);
 
@@ -195,14 +203,16 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kFStages; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(s_free, kSoftmaxThreads);
-    mbar_init(p_full, kSoftmaxThreads);
-    mbar_init(o_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&p_full[i], kSoftmaxThreads);
+      mbar_init(&o_full[i], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -225,8 +235,8 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
       tma_load_2d(sQ, &P.tm, q_full, qcol, row0 + qb * kBQ);
       int issued = 0;
       for (int j = 0; j < nk; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
+        const int st = j % kFStages;
+        const uint32_t ph = static_cast<uint32_t>(j / kFStages) & 1u;
         if (!mbar_wait_bounded(&kv_empty[st], ph ^ 1u, a.wait_ns, abort_flag)) {
           attn_timeout(a, abort_flag);
           break;
@@ -237,12 +247,12 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
         ++issued;
       }
       // every copy lands before the CTA can exit (bounded, not cut short by
-      // the abort flag): the Q tile and the last two K/V stages
+      // the abort flag): the Q tile and the last stages of the ring
       volatile int keep_waiting = 0;
       mbar_wait_bounded(q_full, 0, a.wait_ns, &keep_waiting);
-      for (int j = issued > 2 ? issued - 2 : 0; j < issued; ++j)
-        mbar_wait_bounded(&kv_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, a.wait_ns,
-                          &keep_waiting);
+      for (int j = issued > kFStages ? issued - kFStages : 0; j < issued; ++j)
+        mbar_wait_bounded(&kv_full[j % kFStages], static_cast<uint32_t>(j / kFStages) & 1u,
+                          a.wait_ns, &keep_waiting);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -250,11 +260,11 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
       constexpr uint32_t idS = idesc_bf16_f32(kBQ, kFK, false, false);   // Q K-major, K K-major
       constexpr uint32_t idO = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, V MN-major
       bool any = false;
-      const uint32_t qa = smem_u32(sQ), pa = smem_u32(sP);
+      const uint32_t qa = smem_u32(sQ);
       // S(j) = Q·K_jᵀ into the S columns
       auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>(j >> 1) & 1u, a.wait_ns,
+        const int st = j % kFStages;
+        if (!mbar_wait_bounded(&kv_full[st], static_cast<uint32_t>(j / kFStages) & 1u, a.wait_ns,
                                abort_flag))
           return false;
         tc_fence_after_sync();
@@ -277,19 +287,21 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
           if (!ok) break;
         }
         // O += P(j)·V_j once the softmax has written P(j) (and rescaled O)
-        if (!mbar_wait_bounded(p_full, static_cast<uint32_t>(j & 1), a.wait_ns, abort_flag)) {
+        if (!mbar_wait_bounded(&p_full[j & 1], static_cast<uint32_t>(j >> 1) & 1u, a.wait_ns,
+                               abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after_sync();
-        const uint32_t vb = smem_u32(sV + (j & 1) * kKVTile);
+        const uint32_t vb = smem_u32(sV + (j % kFStages) * kKVTile);
+        const uint32_t pa = smem_u32(sP + (j & 1) * kPTileF);
 #pragma unroll
         for (int k = 0; k < kFK / 16; ++k)   // 16 keys per step
           tc_mma_bf16(tmem + kFTmemO, smem_desc_sw128(pa + k * 32, 16, 1024),
                       smem_desc_sw128(vb + k * 2048, 8192, 1024), idO,
                       (j > 0 || k > 0) ? 1u : 0u);
-        tc_commit(o_full);
-        tc_commit(&kv_empty[j & 1]);   // K_j and V_j read by every MMA issued so far
+        tc_commit(&o_full[j & 1]);
+        tc_commit(&kv_empty[j % kFStages]);   // K_j and V_j read by every MMA issued so far
       }
       if (!ok) attn_timeout(a, abort_flag);
       if (any) {   // every issued MMA completes before tensor memory is freed
@@ -306,7 +318,6 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
     const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
     const uint32_t sbase = tmem + lane_off;
     const uint32_t obase = tmem + lane_off + kFTmemO;
-    uint8_t* prow = sP + r * 128;
     const float sl = a.scale_log2;
     const int klim = a.causal ? min(qpos + 1, a.s) : a.s;   // keys [0, klim) are visible
     float m = -INFINITY;                            // running maximum (log2 units)
@@ -333,35 +344,49 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
       const bool move = j == 0 || m_blk > m + kTau;
       const float alpha = (j > 0 && move) ? ex2f(m - m_blk) : 1.0f;
       if (move) m = m_blk;
-      // P·V(j-1) has finished: the P buffer is free and O holds blocks 0..j-1
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait_bounded(o_full, static_cast<uint32_t>((j - 1) & 1),
+      // P(j) reuses the buffer of P(j-2): P·V(j-2) must have finished
+      if (j > 1 && !__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[j & 1],
+                                                                static_cast<uint32_t>((j - 2) >> 1) & 1u,
                                                                 a.wait_ns, abort_flag))) {
         ok = false;
         break;
       }
-      tc_fence_after_sync();
       // p = 2^(x·sl − m), bf16 into the swizzled P tile, and the row sum
-      l = fmaf(l, alpha, exp_store_row(x, sl, m, prow, r));
+      l = fmaf(l, alpha, exp_store_row(x, sl, m, sP + (j & 1) * kPTileF + r * 128, r));
       if (j > 0 && __any_sync(0xffffffffu, move)) {
-        // rescale the rows whose maximum moved, the others by 1, before the
-        // P·V of this block adds to O
+        // rescale the rows whose maximum moved (the others by 1) once
+        // P·V(j-1) has finished, before the P·V of this block adds to O
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(&o_full[(j - 1) & 1],
+                                                       static_cast<uint32_t>((j - 1) >> 1) & 1u,
+                                                       a.wait_ns, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after_sync();
+        const float2 a2 = make_float2(alpha, alpha);
 #pragma unroll
         for (int c = 0; c < kHD / 32; ++c) {
           uint32_t rr[32];
           tmem_ld_32x32b_x32(obase + c * 32, rr);
           tc_wait_ld();
 #pragma unroll
-          for (int t = 0; t < 32; ++t) rr[t] = __float_as_uint(__uint_as_float(rr[t]) * alpha);
+          for (int t = 0; t < 32; t += 2) {
+            const float2 v = __fmul2_rn(make_float2(__uint_as_float(rr[t]), __uint_as_float(rr[t + 1])), a2);
+            rr[t] = __float_as_uint(v.x);
+            rr[t + 1] = __float_as_uint(v.y);
+          }
           tmem_st_32x32b_x32(obase + c * 32, rr);
         }
         tc_wait_st();
       }
       tc_fence_before_sync();                      // O written before the arrival
       fence_proxy_async_smem();                    // P visible to the tensor core
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[j & 1]);
     }
+    // the last P·V's commit covers every MMA before it
     if (ok && nk > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait_bounded(o_full, static_cast<uint32_t>((nk - 1) & 1),
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&o_full[(nk - 1) & 1],
+                                                     static_cast<uint32_t>((nk - 1) >> 1) & 1u,
                                                      a.wait_ns, abort_flag));
     if (!ok) {
       if (lane == 0) attn_timeout(a, abort_flag);
@@ -896,8 +921,11 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
   int dev = 0;
   cudaGetDevice(&dev);
   if (!configured[dev & 63]) {
+    // two CTAs per SM: the largest shared-memory carveout
     if (cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kFwdAlloc)) != cudaSuccess)
+                             static_cast<int>(kFwdAlloc)) != cudaSuccess ||
+        cudaFuncSetAttribute(attn_fwd_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
       return TP_ERR_CUDA;
     configured[dev & 63] = true;
   }
