@@ -446,10 +446,13 @@ TP_API tp_status tp_attention_fwd(const void* QKV, int64_t b, int64_t s, int32_t
  *   QKV as in tp_attention_fwd; ctx [b·s, n_heads·64] bf16 its output O;
  *   dctx the same shape, the gradient dO; lse [b, n_heads, s] fp32 from
  *   tp_attention_fwd.  causal, scale and head_offsets must be the forward's.
- *   Every gradient row is produced by one CTA (one kernel for dK and dV per
- *   key tile, one for dQ per query tile), so the result is reproducible.
+ *   One CTA per 128-key tile of a head computes that tile's dK and dV rows
+ *   (reproducible bit for bit) and adds its share of dQ into an fp32
+ *   accumulator in the workspace; the adds of different key tiles land in
+ *   any order, so dQ may differ between runs by the rounding of that sum.
  *   ws, ws_bytes >= tp_workspace_bytes(TP_OP_ATTENTION_BWD, b·s, n_heads,
- *   64, N) (rowsum(dO ⊙ O) per query and head).  head_dim 64, n_heads <= 256.
+ *   64, N) (rowsum(dO ⊙ O) per query and head, then the fp32 dQ
+ *   accumulator, b·s·n_heads·64 floats).  head_dim 64, n_heads <= 256.
  */
 TP_API tp_status tp_attention_bwd(const void* QKV, const void* ctx, const void* dctx,
                                   const float* lse, int64_t b, int64_t s, int32_t n_heads,

@@ -424,43 +424,51 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
 
 
 // ===========================================================================
-// Backward.  D = rowsum(dO ⊙ O) first; then two kernels of one template:
-//   kKV = true   one CTA per 128-key tile of a head: streams the queries in
-//                tiles of 64, Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ in tensor memory,
-//                Pᵀ = exp(Sᵀ·scale − lse) and dSᵀ = Pᵀ ⊙ (dPᵀ − D) per key
-//                row, then dV += Pᵀ·dO and dK += dSᵀ·Q accumulated in tensor
-//                memory;
-//   kKV = false  one CTA per 128-query tile: streams the keys in tiles of 64,
-//                S, dP, P, dS the same way per query row, dQ += dS·K.
-// Each gradient row is produced by exactly one CTA, so there are no atomics
-// and the result does not depend on timing.  dQ and dK carry the scale.
+// Backward.  A prep kernel computes D = rowsum(dO ⊙ O) and zeroes the fp32
+// dQ accumulator; then one CTA per 128-key tile of a head streams the queries
+// in tiles of 64:
+//   Sᵀ = K·Qᵀ and dPᵀ = V·dOᵀ in tensor memory,
+//   Pᵀ = exp(Sᵀ·scale − lse) and dSᵀ = Pᵀ ⊙ (dPᵀ − D) per key row,
+//   dV += Pᵀ·dO and dK += dSᵀ·Q accumulated in tensor memory,
+//   dQ_pair = dS·K for every two streamed tiles (one 128-row MMA over the two
+//   dS tiles, MN-major), staged in shared memory and added into the fp32
+//   accumulator in global memory by a TMA reduce (the adds happen in L2, off
+//   the load/store path the element-wise warps use);
+// a finish kernel scales the accumulated dQ and writes it as bf16.  dK and dV
+// of a key row come from exactly one CTA (reproducible bit for bit); dQ sums
+// the key tiles' contributions in fp32 in whatever order they arrive, so its
+// last bits may differ between runs.
 //
-// Roles (10 warps): warp 0 TMA (the fixed 128-row tiles once, the streamed
-// 64-row tiles through a three-stage ring), warp 1 the MMA issuer, warps 2-5
+// Roles (10 warps): warp 0 TMA (the fixed K and V tiles once, the streamed
+// Q and dO tiles through a three-stage ring), warp 1 the MMA issuer, warps 2-5
 // and 6-9 two element-wise warpgroups taking the streamed tiles in turn.
-// S/dP and the bf16 P/dS tiles are double buffered, so the MMAs of one tile
-// (and the gradient MMAs of the one before) run while the other warpgroup
-// evaluates its exponentials.
+// S/dP and the bf16 P tiles are double buffered and the dS tiles quadruple
+// buffered (a pair of them is read by the dQ MMA), so the MMAs of one tile
+// run while the other warpgroup evaluates its exponentials.  Warpgroup w also
+// reads out the dQ of the pairs p ≡ w (mod 2), two streamed tiles later.
 // ===========================================================================
 constexpr int kBG = 64;                                // streamed rows per tile
 constexpr int kGStages = 3;
 constexpr int kBwdThreads = 320;                       // 10 warps
+constexpr int kDSBufs = 4;
 constexpr uint32_t kGTile = kBG * kHD * 2;             // 8 KB: 64 rows of 128 bytes
-constexpr uint32_t kPTile = kBQ * kBG * 2;             // 16 KB: 128 fixed rows x 64 streamed
-constexpr uint32_t kBOffF1 = 0;                        // fixed tiles (K, V) or (Q, dO)
+constexpr uint32_t kPTile = kBQ * kBG * 2;             // 16 KB: 128 keys x 64 queries
+constexpr uint32_t kBOffF1 = 0;                        // fixed tiles: K, V
 constexpr uint32_t kBOffF2 = kTile;
-constexpr uint32_t kBOffG1 = 2 * kTile;                // streamed tiles, kGStages each
+constexpr uint32_t kBOffG1 = 2 * kTile;                // streamed tiles Q, dO, kGStages each
 constexpr uint32_t kBOffG2 = kBOffG1 + kGStages * kGTile;
-constexpr uint32_t kBOffP = kBOffG2 + kGStages * kGTile;   // Pᵀ [2 buffers] (dK/dV kernel)
-constexpr uint32_t kBOffDS = kBOffP + 2 * kPTile;          // dSᵀ or dS [2 buffers]
-constexpr uint32_t kBOffVec = kBOffDS + 2 * kPTile;        // [warpgroup][2][lse·log2e | D][64]
+constexpr uint32_t kBOffP = kBOffG2 + kGStages * kGTile;   // Pᵀ [2 buffers]
+constexpr uint32_t kBOffDS = kBOffP + 2 * kPTile;          // dSᵀ [kDSBufs buffers]
+constexpr uint32_t kBOffStage = kBOffDS + kDSBufs * kPTile;   // dQ of a pair, fp32, 2 x 16 KB
+constexpr uint32_t kStageHalf = kBQ * 32 * 4;                    // 128 rows x 32 columns
+constexpr uint32_t kBOffVec = kBOffStage + 2 * kStageHalf;      // [warpgroup][2][lse·log2e | D][64]
 constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * 2 * kBG * 4;
-constexpr int kBNumBars = 2 * kGStages + 10;
+constexpr int kBNumBars = 2 * kGStages + 15;
 constexpr uint32_t kBOffMisc = kBOffBar + kBNumBars * 8;
 constexpr uint32_t kBAlloc = kBOffMisc + 16 + 1024;
-// tensor memory columns: S/Sᵀ (X) and dP/dPᵀ (Y) double buffered, then the
-// accumulators dV (A1) and dK or dQ (A2)
-constexpr uint32_t kTX = 0, kTY = 128, kTA1 = 256, kTA2 = 320;
+// tensor memory columns: Sᵀ (X) and dPᵀ (Y) double buffered, the
+// accumulators dV (A1) and dK (A2), the dQ of a pair double buffered (Q)
+constexpr uint32_t kTX = 0, kTY = 128, kTA1 = 256, kTA2 = 320, kTQ = 384;
 
 struct AttnBwdArgs {
   int b, s, heads, nqb, ng;  // ng: streamed 64-row tiles of a sequence
@@ -468,6 +476,7 @@ struct AttnBwdArgs {
   float scale, scale_log2;
   const float* lse;          // [b, heads, s] natural log
   const float* D;            // [b, heads, s]
+  float* dq_acc;             // [b·s, heads·64] fp32, zeroed by the prep kernel
   __nv_bfloat16* dqkv;       // [b·s, 3h], the QKV layout
   int64_t ldq;               // 3h
   int32_t* dev_status;
@@ -477,16 +486,19 @@ struct AttnBwdArgs {
 
 struct __align__(64) AttnBwdParams {
   CUtensorMap tm_qkv;        // QKV [b·s, 3h], boxes of 64 columns x 128 rows (fixed tiles)
-  CUtensorMap tm_do;         // dO  [b·s, h],  boxes of 64 columns x 128 rows
   CUtensorMap tm_qkv_g;      // QKV, boxes of 64 columns x 64 rows (streamed tiles)
-  CUtensorMap tm_do_g;       // dO, boxes of 64 columns x 64 rows
+  CUtensorMap tm_do_g;       // dO [b·s, h], boxes of 64 columns x 64 rows
+  CUtensorMap tm_dq;         // dQ accumulator [b·s, h] fp32, boxes of 32 columns x 128 rows
   AttnBwdArgs a;
 };
 
+// D = rowsum(dO ⊙ O) per (token, head), and the dQ accumulator of that
+// (token, head) set to zero.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restrict__ O,
                                                             const uint4* __restrict__ dO,
                                                             int64_t rows, int heads, int s,
-                                                            float* __restrict__ D) {
+                                                            float* __restrict__ D,
+                                                            float4* __restrict__ dq_acc) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (row, head)
   if (i >= rows * heads) return;
   const int64_t row = i / heads;
@@ -506,6 +518,30 @@ __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restr
   }
   const int64_t bb = row / s, pos = row - bb * s;
   D[(bb * heads + head) * s + pos] = acc;
+  float4* z = dq_acc + (row * heads + head) * 16;    // 64 fp32 of this head
+#pragma unroll
+  for (int k = 0; k < 16; ++k) z[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+}
+
+// dQ = scale · (accumulated dS·K), bf16, into this head's Q columns of dQKV.
+// One thread per 8 columns of a (token, head).
+__global__ void __launch_bounds__(256) attn_dq_finish_kernel(const __grid_constant__ AttnBwdArgs a) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t rows = static_cast<int64_t>(a.b) * a.s;
+  if (i >= rows * a.heads * 8) return;
+  const int64_t rh = i >> 3;                           // (row, head)
+  const int g = static_cast<int>(i & 7);
+  const int64_t row = rh / a.heads;
+  const int head = static_cast<int>(rh - row * a.heads);
+  const float4* src = reinterpret_cast<const float4*>(a.dq_acc) + rh * 16 + g * 2;
+  const float4 v0 = src[0], v1 = src[1];
+  const float f = a.scale;
+  uint4 w;
+  w.x = pack_bf16x2(v0.x * f, v0.y * f);
+  w.y = pack_bf16x2(v0.z * f, v0.w * f);
+  w.z = pack_bf16x2(v1.x * f, v1.y * f);
+  w.w = pack_bf16x2(v1.z * f, v1.w * f);
+  *reinterpret_cast<uint4*>(a.dqkv + row * a.ldq + a.head_cols[head].x + g * 8) = w;
 }
 
 __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* abort_flag) {
@@ -515,58 +551,45 @@ __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* 
   }
 }
 
-// One fixed row of a streamed tile: p = 2^(x·sl − l) (zero where masked) and
-// dS = p·(y − D), written as bf16 into the row's 128-byte lines of the P
-// (dK/dV kernel only) and dS tiles, granule g at g ^ (row & 7).  The dK/dV
-// kernel takes l and D per column from shared memory (four at a time), the
-// dQ kernel has one pair for its row.
-template <bool kKV, bool kMask>
+// One key row of a streamed tile: p = 2^(x·sl − l) (zero where masked) and
+// dS = p·(y − D), written as bf16 into the row's 128-byte lines of the P and
+// dS tiles, granule g at g ^ (row & 7).  l and D come per query column from
+// shared memory, four at a time.
+template <bool kMask>
 __device__ __forceinline__ void bwd_tile_rows(const uint32_t (&xr)[kBG], const uint32_t (&yr)[kBG],
-                                              const float* vL, const float* vD, float own_l,
-                                              float own_d, float sl, int t0, int fpos, int s,
-                                              int causal, uint8_t* prow, uint8_t* drow, int r) {
+                                              const float* vL, const float* vD, float sl, int t0,
+                                              int kpos, int s, int causal, uint8_t* prow,
+                                              uint8_t* drow, int r) {
 #pragma unroll
   for (int gr = 0; gr < kBG / 8; ++gr) {       // 16-byte granules of the 128-byte row
     float lv[8], dv[8];
-    if constexpr (kKV) {
-      const float4 l0 = reinterpret_cast<const float4*>(vL)[2 * gr];
-      const float4 l1 = reinterpret_cast<const float4*>(vL)[2 * gr + 1];
-      const float4 d0 = reinterpret_cast<const float4*>(vD)[2 * gr];
-      const float4 d1 = reinterpret_cast<const float4*>(vD)[2 * gr + 1];
-      lv[0] = l0.x; lv[1] = l0.y; lv[2] = l0.z; lv[3] = l0.w;
-      lv[4] = l1.x; lv[5] = l1.y; lv[6] = l1.z; lv[7] = l1.w;
-      dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w;
-      dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
-    } else {
-#pragma unroll
-      for (int t = 0; t < 8; ++t) {
-        lv[t] = own_l;
-        dv[t] = own_d;
-      }
-    }
+    const float4 l0 = reinterpret_cast<const float4*>(vL)[2 * gr];
+    const float4 l1 = reinterpret_cast<const float4*>(vL)[2 * gr + 1];
+    const float4 d0 = reinterpret_cast<const float4*>(vD)[2 * gr];
+    const float4 d1 = reinterpret_cast<const float4*>(vD)[2 * gr + 1];
+    lv[0] = l0.x; lv[1] = l0.y; lv[2] = l0.z; lv[3] = l0.w;
+    lv[4] = l1.x; lv[5] = l1.y; lv[6] = l1.z; lv[7] = l1.w;
+    dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w;
+    dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
     float p[8], ds[8];
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       const int j = gr * 8 + t;
       float pv = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[t]));
       if constexpr (kMask) {
-        const int tpos = t0 + j;               // streamed position of this column
-        // rows are keys and columns queries (kKV), or the other way round
-        const bool masked = tpos >= s || (causal && (kKV ? tpos < fpos : tpos > fpos));
-        pv = masked ? 0.0f : pv;
+        const int qpos = t0 + j;               // query position of this column
+        pv = (qpos >= s || kpos >= s || (causal && qpos < kpos)) ? 0.0f : pv;
       }
       p[t] = pv;
       ds[t] = pv * (__uint_as_float(yr[j]) - dv[t]);
     }
     const int off = (gr ^ (r & 7)) << 4;
     uint4 w;
-    if constexpr (kKV) {
-      w.x = pack_bf16x2(p[0], p[1]);
-      w.y = pack_bf16x2(p[2], p[3]);
-      w.z = pack_bf16x2(p[4], p[5]);
-      w.w = pack_bf16x2(p[6], p[7]);
-      *reinterpret_cast<uint4*>(prow + off) = w;
-    }
+    w.x = pack_bf16x2(p[0], p[1]);
+    w.y = pack_bf16x2(p[2], p[3]);
+    w.z = pack_bf16x2(p[4], p[5]);
+    w.w = pack_bf16x2(p[6], p[7]);
+    *reinterpret_cast<uint4*>(prow + off) = w;
     w.x = pack_bf16x2(ds[0], ds[1]);
     w.y = pack_bf16x2(ds[2], ds[3]);
     w.z = pack_bf16x2(ds[4], ds[5]);
@@ -575,7 +598,6 @@ __device__ __forceinline__ void bwd_tile_rows(const uint32_t (&xr)[kBG], const u
   }
 }
 
-template <bool kKV>
 __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_constant__ AttnBwdParams P) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -587,42 +609,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   uint8_t* sG2 = smem + kBOffG2;
   uint8_t* sP = smem + kBOffP;
   uint8_t* sDS = smem + kBOffDS;
+  uint8_t* sStage = smem + kBOffStage;
   float* vec = reinterpret_cast<float*>(smem + kBOffVec);   // [warpgroup][buffer][lse | D][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBOffBar);
   uint64_t* f_full = bars;
   uint64_t* g_full = bars + 1;                   // [stage]
   uint64_t* g_empty = g_full + kGStages;         // [stage]
-  uint64_t* x_full = g_empty + kGStages;         // [buffer]: S and dP of a tile in tensor memory
+  uint64_t* x_full = g_empty + kGStages;         // [buffer]: Sᵀ and dPᵀ of a tile in tensor memory
   uint64_t* x_empty = x_full + 2;                // [buffer]: read out by the warpgroup
-  uint64_t* pd_full = x_empty + 2;               // [buffer]: P and dS tiles written
-  uint64_t* pd_empty = pd_full + 2;              // [buffer]: read by the gradient MMAs
-  uint64_t* acc_done = pd_empty + 2;
+  uint64_t* pd_full = x_empty + 2;               // [warpgroup]: P and dS tiles written
+  uint64_t* pd_empty = pd_full + 2;              // [warpgroup]: its buffers free again
+  uint64_t* q_full = pd_empty + 2;               // [pair & 1]: dQ of a pair in tensor memory
+  uint64_t* q_empty = q_full + 2;                // [pair & 1]: read out
+  uint64_t* acc_done = q_empty + 2;
+  uint64_t* stage_free = acc_done + 1;           // the staged dQ of a pair read by its reduce
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int bh = a.b * a.heads;
-  // fixed 128-row tile, longest first: under the causal mask key tile t
-  // streams the queries from 128·t on, query tile t the keys up to 128·t + 127
-  const int ft = kKV ? static_cast<int>(blockIdx.x) / bh
-                     : a.nqb - 1 - static_cast<int>(blockIdx.x) / bh;
+  // fixed 128-key tile, longest first: under the causal mask key tile t
+  // streams the queries from 128·t on
+  const int ft = static_cast<int>(blockIdx.x) / bh;
   const int rem = static_cast<int>(blockIdx.x) % bh;
   const int head = rem / a.b;
   const int batch = rem % a.b;
   const int row0 = batch * a.s;
-  const int t_begin = (kKV && a.causal) ? 2 * ft : 0;                  // in 64-row tiles
-  const int t_end = (!kKV && a.causal) ? min(2 * ft + 2, a.ng) : a.ng;
-  const int nt = t_end - t_begin;
+  const int t_begin = a.causal ? 2 * ft : 0;           // in 64-row tiles
+  const int nt = a.ng - t_begin;
+  const int npairs = (nt + 1) >> 1;
   const int qcol = a.head_cols[head].x;
   const int kcol = qcol + a.head_cols[head].y;
   const int vcol = kcol + a.head_cols[head].y;
   const int ocol = head * kHD;                         // this head's columns of dO
-  // fixed pair: (K, V) or (Q, dO); streamed pair: (Q, dO) or (K, V)
-  const int f1col = kKV ? kcol : qcol, f2col = kKV ? vcol : ocol;
-  const int g1col = kKV ? qcol : kcol, g2col = kKV ? ocol : vcol;
-  const CUtensorMap* f2map = kKV ? &P.tm_qkv : &P.tm_do;
-  const CUtensorMap* g2map = kKV ? &P.tm_do_g : &P.tm_qkv_g;
 
   if (threadIdx.x == 0) {
     mbar_init(f_full, 1);
@@ -635,8 +655,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       mbar_init(&x_empty[i], kSoftmaxThreads);
       mbar_init(&pd_full[i], kSoftmaxThreads);
       mbar_init(&pd_empty[i], 1);
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], kSoftmaxThreads);
     }
     mbar_init(acc_done, 1);
+    mbar_init(stage_free, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -653,12 +676,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     // ------------------------------------------------------------ TMA
     if (elect_one_sync()) {
       tma_prefetch_desc(&P.tm_qkv);
-      tma_prefetch_desc(&P.tm_do);
       tma_prefetch_desc(&P.tm_qkv_g);
       tma_prefetch_desc(&P.tm_do_g);
       mbar_arrive_expect_tx(f_full, 2 * kTile);
-      tma_load_2d(sF1, &P.tm_qkv, f_full, f1col, row0 + ft * kBQ);
-      tma_load_2d(sF2, f2map, f_full, f2col, row0 + ft * kBQ);
+      tma_load_2d(sF1, &P.tm_qkv, f_full, kcol, row0 + ft * kBQ);
+      tma_load_2d(sF2, &P.tm_qkv, f_full, vcol, row0 + ft * kBQ);
       int issued = 0;
       for (int it = 0; it < nt; ++it) {
         const int st = it % kGStages;
@@ -669,8 +691,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
         }
         const int r = row0 + (t_begin + it) * kBG;
         mbar_arrive_expect_tx(&g_full[st], 2 * kGTile);
-        tma_load_2d(sG1 + st * kGTile, &P.tm_qkv_g, &g_full[st], g1col, r);
-        tma_load_2d(sG2 + st * kGTile, g2map, &g_full[st], g2col, r);
+        tma_load_2d(sG1 + st * kGTile, &P.tm_qkv_g, &g_full[st], qcol, r);
+        tma_load_2d(sG2 + st * kGTile, &P.tm_do_g, &g_full[st], ocol, r);
         ++issued;
       }
       volatile int keep_waiting = 0;   // every copy lands before the CTA can exit
@@ -684,10 +706,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     if (elect_one_sync()) {
       constexpr uint32_t idS = idesc_bf16_f32(kBQ, kBG, false, false);   // both K-major
       constexpr uint32_t idA = idesc_bf16_f32(kBQ, kHD, false, true);    // P K-major, G MN-major
+      constexpr uint32_t idQ = idesc_bf16_f32(kBQ, kHD, true, true);     // dS MN-major, K MN-major
       bool ok = mbar_wait_bounded(f_full, 0, a.wait_ns, abort_flag);
       bool any = false;
       const uint32_t f1 = smem_u32(sF1), f2 = smem_u32(sF2);
-      // X_b = F1·G1ᵀ (S or Sᵀ) and Y_b = F2·G2ᵀ (dP or dPᵀ) of streamed tile it
+      // X_b = K·Qᵀ (Sᵀ) and Y_b = V·dOᵀ (dPᵀ) of streamed tile it
       auto issue_xy = [&](int it) -> bool {
         const int st = it % kGStages, b = it & 1;
         if (!mbar_wait_bounded(&g_full[st], static_cast<uint32_t>(it / kGStages) & 1u, a.wait_ns,
@@ -712,6 +735,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       if (ok && nt > 1) ok = issue_xy(1);
       for (int it = 0; ok && it < nt; ++it) {
         const int st = it % kGStages, b = it & 1;
+        // Sᵀ and dPᵀ of tile it+2 as soon as the warpgroup has read those of
+        // tile it, ahead of tile it's gradient MMAs: their commit then does
+        // not wait for those
+        if (it + 2 < nt && !issue_xy(it + 2)) {
+          ok = false;
+          break;
+        }
         if (!mbar_wait_bounded(&pd_full[b], static_cast<uint32_t>(it >> 1) & 1u, a.wait_ns,
                                abort_flag)) {
           ok = false;
@@ -719,20 +749,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
         }
         tc_fence_after_sync();
         const uint32_t g1 = smem_u32(sG1 + st * kGTile), g2 = smem_u32(sG2 + st * kGTile);
-        const uint32_t pa = smem_u32(sP + b * kPTile), da = smem_u32(sDS + b * kPTile);
+        const uint32_t pa = smem_u32(sP + b * kPTile);
+        const uint32_t da = smem_u32(sDS + (it % kDSBufs) * kPTile);
 #pragma unroll
-        for (int k = 0; k < kBG / 16; ++k) {   // K = the streamed tile's 64 rows
+        for (int k = 0; k < kBG / 16; ++k) {   // K = the streamed tile's 64 queries
           const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
-          if constexpr (kKV)   // dV += Pᵀ·dO
-            tc_mma_bf16(tmem + kTA1, smem_desc_sw128(pa + k * 32, 16, 1024),
-                        smem_desc_sw128(g2 + k * 2048, 8192, 1024), idA, acc);
-          // dK += dSᵀ·Q  or  dQ += dS·K
+          // dV += Pᵀ·dO
+          tc_mma_bf16(tmem + kTA1, smem_desc_sw128(pa + k * 32, 16, 1024),
+                      smem_desc_sw128(g2 + k * 2048, 8192, 1024), idA, acc);
+          // dK += dSᵀ·Q
           tc_mma_bf16(tmem + kTA2, smem_desc_sw128(da + k * 32, 16, 1024),
                       smem_desc_sw128(g1 + k * 2048, 8192, 1024), idA, acc);
         }
+        if ((it & 1) || it + 1 == nt) {
+          // dQ of the pair (tiles it & ~1 and it & ~1 | 1) = dS·K: M = the
+          // pair's 128 queries (two MN-major 64-query dS tiles, kPTile apart),
+          // K = the 128 keys of this CTA, N = 64 (K tile MN-major)
+          const int pr = it >> 1;
+          if (!mbar_wait_bounded(&q_empty[pr & 1], (static_cast<uint32_t>(pr >> 1) & 1u) ^ 1u,
+                                 a.wait_ns, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after_sync();
+          const uint32_t qa = smem_u32(sDS + ((2 * pr) % kDSBufs) * kPTile);
+#pragma unroll
+          for (int k = 0; k < kBQ / 16; ++k)
+            tc_mma_bf16(tmem + kTQ + (pr & 1) * kHD, smem_desc_sw128(qa + k * 2048, kPTile, 1024),
+                        smem_desc_sw128(f1 + k * 2048, 8192, 1024), idQ, k > 0 ? 1u : 0u);
+          tc_commit(&q_full[pr & 1]);
+        }
         tc_commit(&pd_empty[b]);
         tc_commit(&g_empty[st]);
-        if (it + 2 < nt) ok = issue_xy(it + 2);
       }
       if (!ok) bwd_timeout(a, abort_flag);
       if (any) {
@@ -747,106 +795,151 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     // ------------------------------------------------------------ element-wise
     const int wg = (warp - 2) >> 2;                // warpgroup: streamed tiles wg, wg + 2, ...
     const int qd = warp & 3;
-    const int r = qd * 32 + lane;                  // fixed row = TMEM lane
+    const int r = qd * 32 + lane;                  // key row = TMEM lane
     const int et = threadIdx.x - 64 - wg * kSoftmaxThreads;   // 0..127 in the warpgroup
-    const int fpos = ft * kBQ + r;                 // its position in the sequence
+    const int kpos = ft * kBQ + r;                 // its position in the sequence
     const int sbase = (batch * a.heads + head) * a.s;
     const uint32_t lane_off = static_cast<uint32_t>(qd * 32) << 16;
     const float sl = a.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
-    // the fixed row's own lse and D (dQ kernel)
-    const float own_l = (!kKV && fpos < a.s) ? a.lse[sbase + fpos] * kLog2e : 0.0f;
-    const float own_d = (!kKV && fpos < a.s) ? a.D[sbase + fpos] : 0.0f;
     uint8_t* prow = sP + wg * kPTile + r * 128;
-    uint8_t* drow = sDS + wg * kPTile + r * 128;
     bool ok = true;
-    // lse·log2e and D of the streamed queries (dK/dV kernel): thread et < 64
-    // loads those of query et of a tile one tile ahead of its use, so the
-    // global loads are in flight while the warpgroup works on a tile
+    // dQ of pair pr (queries of streamed tiles 2pr, 2pr+1 = TMEM lanes): read
+    // out, staged as two 128-byte-swizzled fp32 boxes of 32 columns (rows
+    // past s as zeros) and added into the accumulator by one thread's TMA
+    // reduce.  Every thread of the warpgroup enters (the call sites depend
+    // only on the tile and the warpgroup) with its own state `in`; the first
+    // barrier ANDs those, so all threads return the same answer and none is
+    // left waiting in the second barrier after a timeout.
+    auto drain_pair = [&](int pr, bool in) -> bool {
+      // the pair's dQ is in tensor memory and the staging buffer is free
+      // once the previous pair's reduce has read it
+      bool good = in &&
+                  mbar_wait_bounded(&q_full[pr & 1], static_cast<uint32_t>(pr >> 1) & 1u, a.wait_ns,
+                                    abort_flag) &&
+                  (pr == 0 || mbar_wait_bounded(stage_free, static_cast<uint32_t>(pr - 1) & 1u,
+                                                a.wait_ns, abort_flag));
+      if (!named_barrier_and(3 + wg, kSoftmaxThreads, good)) return false;
+      tc_fence_after_sync();
+      const bool valid = (t_begin + 2 * pr) * kBG + r < a.s;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t qr[32];
+        tmem_ld_32x32b_x32(tmem + lane_off + kTQ + (pr & 1) * kHD + h * 32, qr);
+        tc_wait_ld();
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const float4 v = valid ? make_float4(__uint_as_float(qr[4 * g]), __uint_as_float(qr[4 * g + 1]),
+                                               __uint_as_float(qr[4 * g + 2]), __uint_as_float(qr[4 * g + 3]))
+                                 : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          *reinterpret_cast<float4*>(sStage + h * kStageHalf + r * 128 + ((g ^ (r & 7)) << 4)) = v;
+        }
+      }
+      tc_fence_before_sync();
+      mbar_arrive(&q_empty[pr & 1]);               // dQ read: the MMA may reuse its columns
+      fence_proxy_async_smem();                    // staged dQ visible to the TMA unit
+      named_barrier_sync(3 + wg, kSoftmaxThreads);
+      if (et == 0) {
+        const int y = row0 + (t_begin + 2 * pr) * kBG;
+        tma_reduce_add_2d(&P.tm_dq, sStage, head * kHD, y);
+        tma_reduce_add_2d(&P.tm_dq, sStage + kStageHalf, head * kHD + 32, y);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(stage_free);
+      }
+      return true;
+    };
+    // lse·log2e and D of the streamed queries: thread et < 64 loads those of
+    // query et of a tile one tile ahead of its use, so the global loads are
+    // in flight while the warpgroup works on a tile
     float nl = 0.0f, nd = 0.0f;
     auto fetch_vec = [&](int tile) {
       const int q = (t_begin + tile) * kBG + et;
       nl = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
       nd = q < a.s ? a.D[sbase + q] : 0.0f;
     };
-    if (kKV && et < kBG && wg < nt) fetch_vec(wg);
+    if (et < kBG && wg < nt) fetch_vec(wg);
     for (int it = wg; it < nt; it += 2) {
       const uint32_t use = static_cast<uint32_t>(it >> 1);   // this warpgroup's tile count
-      const int t0 = (t_begin + it) * kBG;         // first position of the streamed tile
+      const int t0 = (t_begin + it) * kBG;         // first query of the streamed tile
       const float* vL = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
       const float* vD = vL + kBG;
-      if constexpr (kKV) {
-        if (et < kBG) {
-          float* w = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
-          w[et] = nl;
-          w[kBG + et] = nd;
-          if (it + 2 < nt) fetch_vec(it + 2);
-        }
-        // one barrier per tile that also carries every thread's state, so all
-        // 128 threads of the warpgroup leave together and none is left in it
-        ok = __all_sync(0xffffffffu, ok);
-        if (!named_barrier_and(1 + wg, kSoftmaxThreads, ok)) {
-          ok = false;
-          break;
-        }
+      if (et < kBG) {
+        float* w = vec + ((wg * 2 + (use & 1)) * 2) * kBG;
+        w[et] = nl;
+        w[kBG + et] = nd;
+        if (it + 2 < nt) fetch_vec(it + 2);
       }
-      // the warp's lanes agree before the warp-collective tensor-memory loads
-      if (!__all_sync(0xffffffffu,
-                      mbar_wait_bounded(&x_full[wg], use & 1u, a.wait_ns, abort_flag))) {
+      // one barrier per tile that also carries every thread's state, so all
+      // 128 threads of the warpgroup leave together and none is left in it
+      ok = __all_sync(0xffffffffu, ok);
+      if (!named_barrier_and(1 + wg, kSoftmaxThreads, ok)) {
         ok = false;
-        if constexpr (kKV) continue;   // leave at the next tile's barrier, with the others
         break;
       }
-      tc_fence_after_sync();
-      uint32_t xr[kBG], yr[kBG];
+      // the warp's lanes agree before the warp-collective tensor-memory
+      // loads; a warp that gives up skips the tile's work but still reaches
+      // the warpgroup's barriers (the dQ drain's, the next tile's), where
+      // the others learn of it
+      ok = __all_sync(0xffffffffu, mbar_wait_bounded(&x_full[wg], use & 1u, a.wait_ns, abort_flag));
+      if (ok) {
+        tc_fence_after_sync();
+        uint32_t xr[kBG], yr[kBG];
 #pragma unroll
-      for (int c = 0; c < kBG / 32; ++c) {
-        tmem_ld_32x32b_x32(tmem + lane_off + kTX + wg * kBG + c * 32,
-                           *reinterpret_cast<uint32_t(*)[32]>(&xr[c * 32]));
-        tmem_ld_32x32b_x32(tmem + lane_off + kTY + wg * kBG + c * 32,
-                           *reinterpret_cast<uint32_t(*)[32]>(&yr[c * 32]));
+        for (int c = 0; c < kBG / 32; ++c) {
+          tmem_ld_32x32b_x32(tmem + lane_off + kTX + wg * kBG + c * 32,
+                             *reinterpret_cast<uint32_t(*)[32]>(&xr[c * 32]));
+          tmem_ld_32x32b_x32(tmem + lane_off + kTY + wg * kBG + c * 32,
+                             *reinterpret_cast<uint32_t(*)[32]>(&yr[c * 32]));
+        }
+        tc_wait_ld();
+        tc_fence_before_sync();
+        mbar_arrive(&x_empty[wg]);               // Sᵀ and dPᵀ read: the MMA may refill them
+        // this warpgroup's P buffer and dS buffer it % 4 are free once the
+        // MMAs issued up to its previous tile (its dV/dK and the dQ of the
+        // pair before) have completed
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(&pd_empty[wg], (use & 1u) ^ 1u, a.wait_ns,
+                                                       abort_flag));
+        if (ok) {
+          uint8_t* drow = sDS + (it % kDSBufs) * kPTile + r * 128;
+          // the mask can only cut the tiles that meet the diagonal or the end
+          // (of the queries, or of the keys: key rows past s must add nothing
+          // to dQ)
+          const bool need_mask =
+              (a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s || ft * kBQ + kBQ > a.s;
+          if (need_mask)
+            bwd_tile_rows<true>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r);
+          else
+            bwd_tile_rows<false>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r);
+          fence_proxy_async_smem();              // P and dS visible to the tensor core
+          mbar_arrive(&pd_full[wg]);
+        }
       }
-      tc_wait_ld();
-      tc_fence_before_sync();
-      mbar_arrive(&x_empty[wg]);                   // S and dP read: the MMA may refill them
-      // the P/dS buffer is free once the gradient MMAs of this warpgroup's
-      // previous tile have read it
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&pd_empty[wg], (use & 1u) ^ 1u, a.wait_ns,
-                                                     abort_flag))) {
-        ok = false;
-        if constexpr (kKV) continue;
-        break;
-      }
-      // the mask can only cut the tiles that meet the diagonal or the end
-      const bool need_mask =
-          kKV ? ((a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s)
-              : ((a.causal && t0 + kBG - 1 > ft * kBQ) || t0 + kBG > a.s);
-      if (need_mask)
-        bwd_tile_rows<kKV, true>(xr, yr, vL, vD, own_l, own_d, sl, t0, fpos, a.s, a.causal, prow,
-                                 drow, r);
-      else
-        bwd_tile_rows<kKV, false>(xr, yr, vL, vD, own_l, own_d, sl, t0, fpos, a.s, a.causal,
-                                  prow, drow, r);
-      fence_proxy_async_smem();                    // P and dS visible to the tensor core
-      mbar_arrive(&pd_full[wg]);
+      // the dQ of pair (it − 2 − wg) / 2 when it belongs to this warpgroup:
+      // issued after the other warpgroup's tile, it is done by now
+      if (it >= 2 + wg && (((it - 2 - wg) >> 1) & 1) == wg)
+        ok = drain_pair((it - 2 - wg) >> 1, ok);
     }
-    // the accumulated gradients of the fixed rows: every lane takes part in
+    // every thread of the warpgroup agrees on the state, then drains this
+    // warpgroup's pairs not drained in the loop
+    ok = named_barrier_and(1 + wg, kSoftmaxThreads, __all_sync(0xffffffffu, ok));
+    for (int pr = wg; pr < npairs; pr += 2)
+      if (2 * pr + 2 + wg >= nt) ok = drain_pair(pr, ok);
+    if (et == 0) bulk_wait_group0();               // this thread's reduces have landed
+    // the accumulated gradients of the key rows: every lane takes part in
     // the warp-collective tensor-memory loads, only rows inside the sequence
-    // are stored.  dK/dV kernel: warpgroup 0 stores dK, warpgroup 1 dV; dQ
-    // kernel: each warpgroup stores 32 of the 64 columns.
+    // are stored.  Warpgroup 0 stores dK, warpgroup 1 dV.
     const bool done =
         __all_sync(0xffffffffu, ok && mbar_wait_bounded<true>(acc_done, 0, a.wait_ns, abort_flag));
     if (!done) {
       if (lane == 0) bwd_timeout(a, abort_flag);
     } else {
       tc_fence_after_sync();
-      __nv_bfloat16* dst_row = a.dqkv + static_cast<int64_t>(row0 + fpos) * a.ldq;
-      const uint32_t col = (kKV && wg == 1) ? kTA1 : kTA2;
-      const float f = (kKV && wg == 1) ? 1.0f : a.scale;
-      const int c_begin = kKV ? 0 : wg, c_end = kKV ? kHD / 32 : wg + 1;
-      __nv_bfloat16* dst = dst_row + (kKV ? (wg == 0 ? kcol : vcol) : qcol);
+      const uint32_t col = wg == 1 ? kTA1 : kTA2;
+      const float f = wg == 1 ? 1.0f : a.scale;
+      __nv_bfloat16* dst = a.dqkv + static_cast<int64_t>(row0 + kpos) * a.ldq + (wg == 0 ? kcol : vcol);
 #pragma unroll 1
-      for (int c = c_begin; c < c_end; ++c) {
+      for (int c = 0; c < kHD / 32; ++c) {
         uint32_t rr[32];
         tmem_ld_32x32b_x32(tmem + lane_off + col + c * 32, rr);
         tc_wait_ld();
@@ -857,7 +950,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
           w.y = pack_bf16x2(__uint_as_float(rr[8 * g + 2]) * f, __uint_as_float(rr[8 * g + 3]) * f);
           w.z = pack_bf16x2(__uint_as_float(rr[8 * g + 4]) * f, __uint_as_float(rr[8 * g + 5]) * f);
           w.w = pack_bf16x2(__uint_as_float(rr[8 * g + 6]) * f, __uint_as_float(rr[8 * g + 7]) * f);
-          if (fpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
+          if (kpos < a.s) reinterpret_cast<uint4*>(dst + c * 32)[g] = w;
         }
       }
     }
@@ -869,22 +962,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     tc_fence_after_sync();
     tmem_dealloc(tmem, kTmemCols);
   }
-}
-
-template <bool kKV>
-tp_status attn_bwd_launch_t(const AttnBwdParams& prm, int64_t grid, cudaStream_t stream) {
-  static bool configured[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!configured[dev & 63]) {
-    if (cudaFuncSetAttribute(attn_bwd_kernel<kKV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kBAlloc)) != cudaSuccess)
-      return TP_ERR_CUDA;
-    configured[dev & 63] = true;
-  }
-  attn_bwd_kernel<kKV><<<static_cast<unsigned>(grid), kBwdThreads, kBAlloc, stream>>>(prm);
-  note_launches(1);
-  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 }  // namespace
@@ -937,7 +1014,9 @@ tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,
 }
 
 size_t attention_bwd_ws_bytes(int64_t b, int64_t s, int heads) {
-  return (static_cast<size_t>(b * s) * heads * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  // D [b·s·heads] fp32, then the dQ accumulator [b·s, heads·64] fp32
+  const size_t d_bytes = (static_cast<size_t>(b * s) * heads * sizeof(float) + 255) & ~static_cast<size_t>(255);
+  return d_bytes + static_cast<size_t>(b * s) * heads * kHD * sizeof(float);
 }
 
 tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, const float* lse,
@@ -946,11 +1025,14 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
                                cudaStream_t stream) {
   if (heads > kMaxHeads) return TP_ERR_UNSUPPORTED;
   float* D = static_cast<float*>(ws);
+  float* dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) +
+                                           ((static_cast<size_t>(b * s) * heads * sizeof(float) + 255) &
+                                            ~static_cast<size_t>(255)));
   {
     const int64_t n = b * s * heads;
     attn_bwd_prep_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
         static_cast<const uint4*>(O), static_cast<const uint4*>(dO), b * s, heads,
-        static_cast<int>(s), D);
+        static_cast<int>(s), D, reinterpret_cast<float4*>(dq_acc));
     note_launches(1);
     if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
   }
@@ -967,6 +1049,7 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
   a.scale_log2 = scale * 1.4426950408889634f;
   a.lse = lse;
   a.D = D;
+  a.dq_acc = dq_acc;
   a.dqkv = static_cast<__nv_bfloat16*>(dQKV);
   a.ldq = static_cast<int64_t>(3) * heads * kHD;
   a.dev_status = dev_status;
@@ -979,14 +1062,30 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
   }
   const uint64_t rows = static_cast<uint64_t>(b * s);
   const uint64_t ncols = static_cast<uint64_t>(3) * heads * kHD;
-  if (!make_tmap_bf16_sw128(&prm.tm_qkv, QKV, ncols, rows, ncols, kHD, kBQ)) return TP_ERR_CUDA;
   const uint64_t hcols = static_cast<uint64_t>(heads) * kHD;
-  if (!make_tmap_bf16_sw128(&prm.tm_do, dO, hcols, rows, hcols, kHD, kBQ)) return TP_ERR_CUDA;
-  if (!make_tmap_bf16_sw128(&prm.tm_qkv_g, QKV, ncols, rows, ncols, kHD, kBG)) return TP_ERR_CUDA;
-  if (!make_tmap_bf16_sw128(&prm.tm_do_g, dO, hcols, rows, hcols, kHD, kBG)) return TP_ERR_CUDA;
+  if (!make_tmap_bf16_sw128(&prm.tm_qkv, QKV, ncols, rows, ncols, kHD, kBQ) ||
+      !make_tmap_bf16_sw128(&prm.tm_qkv_g, QKV, ncols, rows, ncols, kHD, kBG) ||
+      !make_tmap_bf16_sw128(&prm.tm_do_g, dO, hcols, rows, hcols, kHD, kBG) ||
+      !make_tmap_f32_sw128(&prm.tm_dq, dq_acc, hcols, rows, hcols, 32, kBQ))
+    return TP_ERR_CUDA;
+  static bool configured[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!configured[dev & 63]) {
+    if (cudaFuncSetAttribute(attn_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kBAlloc)) != cudaSuccess)
+      return TP_ERR_CUDA;
+    configured[dev & 63] = true;
+  }
+  // one CTA per (sequence, head, key tile), the longest causal tiles first
   const int64_t grid = b * heads * a.nqb;
-  if (tp_status st = attn_bwd_launch_t<true>(prm, grid, stream)) return st;
-  return attn_bwd_launch_t<false>(prm, grid, stream);
+  attn_bwd_kernel<<<static_cast<unsigned>(grid), kBwdThreads, kBAlloc, stream>>>(prm);
+  note_launches(1);
+  if (cudaGetLastError() != cudaSuccess) return TP_ERR_CUDA;
+  const int64_t nfin = b * s * heads * 8;
+  attn_dq_finish_kernel<<<static_cast<unsigned>((nfin + 255) / 256), 256, 0, stream>>>(a);
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
 }  // namespace tpl

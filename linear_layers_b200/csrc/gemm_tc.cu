@@ -1034,6 +1034,21 @@ bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t 
   return make_tmap(static_cast<CUtensorMap*>(tmap), ptr, inner, outer, ld, box_inner, box_outer);
 }
 
+bool make_tmap_f32_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                         uint32_t box_inner, uint32_t box_outer) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(static_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
   if (splits <= 1 && !with_zpart) return 0;
   // 128-row pieces of the 512-row tall tiling (covers the 256- and 128-row

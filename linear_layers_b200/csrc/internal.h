@@ -95,6 +95,9 @@ tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
 // elements, 128-byte swizzle, zero fill outside the matrix.
 bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
                           uint32_t box_inner, uint32_t box_outer);
+// The same for an fp32 matrix (box_inner <= 32: one 128-byte swizzle row).
+bool make_tmap_f32_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                         uint32_t box_inner, uint32_t box_outer);
 
 // Attention core (attn.cu): see tp_attention_fwd.
 tp_status attention_fwd_launch(const void* QKV, int64_t b, int64_t s, int heads,

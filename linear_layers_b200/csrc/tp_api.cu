@@ -281,7 +281,7 @@ size_t tp_workspace_bytes(tp_op op, int64_t M, int64_t h, int64_t F, int32_t N) 
       return linear_xent_ws_bytes(M, F);
     case TP_OP_SP_LN_BWD:     // (M, h, h, N): per-block partial parameter gradients
       return sp_ln_bwd_ws_bytes(M, h);
-    case TP_OP_ATTENTION_BWD: // (b·s, n_heads, 64, N): rowsum(dO ⊙ O) per query and head
+    case TP_OP_ATTENTION_BWD: // (b·s, n_heads, 64, N): rowsum(dO ⊙ O), fp32 dQ accumulator
       return attention_bwd_ws_bytes(M, 1, static_cast<int>(h));
   }
   return 0;

