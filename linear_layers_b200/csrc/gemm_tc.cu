@@ -136,15 +136,19 @@ struct Cfg {
 // 0.5·u·(1 + tanh(z)) is written as u·σ(2z), which stays accurate in the
 // negative tail where 1 + tanh(z) cancels.
 // -------------------------------------------------------------------------
-__device__ __forceinline__ float act_apply(float u, int act) {
-  if (act == TP_ACT_GELU_TANH) {
+// The activation is a template argument: the epilogues branch once per
+// 32-column chunk on the (uniform) runtime code and run straight-line code
+// for the one form, instead of carrying every form's arithmetic per element.
+template <int ACT>
+__device__ __forceinline__ float act_apply(float u) {
+  if constexpr (ACT == TP_ACT_GELU_TANH) {
     const float z = 0.7978845608028654f * (u + 0.044715f * u * u * u);
     return __fdividef(u, 1.0f + __expf(-2.0f * z));
-  }
-  if (act == TP_ACT_GELU_ERF) {
+  } else if constexpr (ACT == TP_ACT_GELU_ERF) {
     return 0.5f * u * (1.0f + erff(u * 0.7071067811865476f));
+  } else {
+    return u;
   }
-  return u;
 }
 
 __device__ __forceinline__ float tanh_approx(float x) {
@@ -156,27 +160,29 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // GeLU'(u) of the tanh form, 0.5·(1 + t) + 0.5·u·(1 − t²)·c·(1 + 3a·u²) with
 // t = tanh(c·(u + a·u³)), from one hardware tanh (absolute error of GeLU'
 // about 2.5e-4, below the bf16 rounding of the dU it scales).
-__device__ __forceinline__ float act_deriv(float u, int act) {
-  if (act == TP_ACT_GELU_TANH) {
+template <int ACT>
+__device__ __forceinline__ float act_deriv(float u) {
+  if constexpr (ACT == TP_ACT_GELU_TANH) {
     constexpr float c = 0.7978845608028654f, a = 0.044715f;
     const float u2 = u * u;
     const float t = tanh_approx(u * fmaf(c * a, u2, c));
     const float half_dz = fmaf(1.5f * c * a, u2, 0.5f * c);   // 0.5·c·(1 + 3a·u²)
     return fmaf(u * half_dz, fmaf(-t, t, 1.0f), fmaf(0.5f, t, 0.5f));
-  }
-  if (act == TP_ACT_GELU_ERF) {   // explicit fmaf: the same bits as act_deriv_value
+  } else if constexpr (ACT == TP_ACT_GELU_ERF) {   // explicit fmaf: the same bits as act_deriv_value
     const float cdf = fmaf(0.5f, erff(u * 0.7071067811865476f), 0.5f);
     return fmaf(u * 0.3989422804014327f, __expf(-0.5f * u * u), cdf);
+  } else {
+    return 1.0f;
   }
-  return 1.0f;
 }
 
 // act'(u) and act(u) together.  For the tanh form the value 0.5·u·(1 + t)
 // reuses the derivative's t; where 1 + t cancels (u < 0) its absolute
 // error stays below 2.5e-4·|u|, the size of a bf16 rounding step of values
 // near 0.1.
-__device__ __forceinline__ float act_deriv_value(float u, int act, float& y) {
-  if (act == TP_ACT_GELU_TANH) {
+template <int ACT>
+__device__ __forceinline__ float act_deriv_value(float u, float& y) {
+  if constexpr (ACT == TP_ACT_GELU_TANH) {
     constexpr float c = 0.7978845608028654f, a = 0.044715f;
     const float u2 = u * u;
     const float t = tanh_approx(u * fmaf(c * a, u2, c));
@@ -184,14 +190,37 @@ __device__ __forceinline__ float act_deriv_value(float u, int act, float& y) {
     const float hu = 0.5f * u;
     y = fmaf(hu, t, hu);
     return fmaf(u * half_dz, fmaf(-t, t, 1.0f), fmaf(0.5f, t, 0.5f));
-  }
-  if (act == TP_ACT_GELU_ERF) {
+  } else if constexpr (ACT == TP_ACT_GELU_ERF) {
     const float cdf = fmaf(0.5f, erff(u * 0.7071067811865476f), 0.5f);
     y = u * cdf;
     return fmaf(u * 0.3989422804014327f, __expf(-0.5f * u * u), cdf);
+  } else {
+    y = u;
+    return 1.0f;
   }
-  y = u;
-  return 1.0f;
+}
+
+// One 32-column chunk through the activation / its derivative.
+template <int ACT>
+__device__ __forceinline__ void act_chunk(float (&v)[32]) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = act_apply<ACT>(v[j]);
+}
+template <int ACT>
+__device__ __forceinline__ void dact_chunk(float (&v)[32], const float (&u)[32], bool ok) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) v[j] = ok ? v[j] * act_deriv<ACT>(u[j]) : 0.0f;
+}
+// dU = dY·act'(U) and, in place of U, Y = act(U)
+template <int ACT>
+__device__ __forceinline__ void dact_value_chunk(float (&v)[32], float (&u)[32], bool ok) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) {
+    float y;
+    const float d = act_deriv_value<ACT>(u[j], y);
+    v[j] = ok ? v[j] * d : 0.0f;
+    u[j] = y;
+  }
 }
 
 // -------------------------------------------------------------------------
@@ -768,25 +797,29 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
             if (store_ok && a.out0 != nullptr)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
                             a.N - col0);
-#pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = act_apply(v[j], a.act);
+            if (a.act == TP_ACT_GELU_TANH)
+              act_chunk<TP_ACT_GELU_TANH>(v);
+            else if (a.act == TP_ACT_GELU_ERF)
+              act_chunk<TP_ACT_GELU_ERF>(v);
             if (store_ok)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
                             a.N - col0);
           } else {  // EPI_DACT, EPI_DACT_Y
             if constexpr (EPI == EPI_DACT_Y) {
               // U is dead after its derivative: its registers take Y = act(U)
-#pragma unroll
-              for (int j = 0; j < 32; ++j) {
-                float y;
-                const float d = act_deriv_value(aux_v[j], a.act, y);
-                v[j] = store_ok ? v[j] * d : 0.0f;
-                aux_v[j] = y;
-              }
+              if (a.act == TP_ACT_GELU_TANH)
+                dact_value_chunk<TP_ACT_GELU_TANH>(v, aux_v, store_ok);
+              else if (a.act == TP_ACT_GELU_ERF)
+                dact_value_chunk<TP_ACT_GELU_ERF>(v, aux_v, store_ok);
+              else
+                dact_value_chunk<TP_ACT_NONE>(v, aux_v, store_ok);
             } else {
-#pragma unroll
-              for (int j = 0; j < 32; ++j)
-                v[j] = store_ok ? v[j] * act_deriv(aux_v[j], a.act) : 0.0f;
+              if (a.act == TP_ACT_GELU_TANH)
+                dact_chunk<TP_ACT_GELU_TANH>(v, aux_v, store_ok);
+              else if (a.act == TP_ACT_GELU_ERF)
+                dact_chunk<TP_ACT_GELU_ERF>(v, aux_v, store_ok);
+              else
+                dact_chunk<TP_ACT_NONE>(v, aux_v, store_ok);
             }
             if (store_ok)
               store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
