@@ -88,6 +88,7 @@ struct GemmArgs {
   const float* row_lse;
   float grad_scale;
   int inject_unit, inject_kb;       // debug: the producer stops before this k-block (-1: never)
+  int tma_out;                      // bf16 outputs leave through tensor maps (tmO)
 };
 
 // One launch runs one problem, or two independent problems with the same
@@ -96,6 +97,7 @@ struct GemmArgs {
 struct __align__(64) GemmParams {
   CUtensorMap tmA[2];
   CUtensorMap tmB[2];
+  CUtensorMap tmO[2][2];            // [problem][out0, out1]: 32 x 32 boxes, 64-byte swizzle
   GemmArgs a[2];
   int units0;                       // units of problem 0
   int total_units;                  // units of both problems
@@ -124,7 +126,10 @@ struct Cfg {
   static constexpr uint32_t kNumBars = 2 * kStages + 5;
   static constexpr uint32_t kOffMisc = kOffBar + kNumBars * 8;
   static constexpr uint32_t kOffRed = (kOffMisc + 16 + 15) & ~15u;   // dbias quadrant sums
-  static constexpr uint32_t kBytes = kOffRed + 4 * BNT * 4;
+  // per epilogue warp, one 32 x 32 bf16 chunk on its way to a TMA store
+  static constexpr uint32_t kOffStage = (kOffRed + 4 * BNT * 4 + 1023) & ~1023u;
+  static constexpr uint32_t kStageBytes = 32 * 32 * 2;
+  static constexpr uint32_t kBytes = kOffStage + 8 * kStageBytes;
   static constexpr uint32_t kAlloc = kBytes + 1024;   // slack for 1024-byte alignment
   static constexpr uint32_t kTmemCols = 2 * BNT;      // two accumulators, or two row halves
   static constexpr int kAccBufs = RH == 2 ? 1 : 2;    // accumulator buffers in tensor memory
@@ -312,6 +317,35 @@ __device__ __forceinline__ float warp_column_sums(float (&v)[32], int lane) {
     }
   }
   return v[0];
+}
+
+// One warp's 32 x 32 chunk (lane = row, 32 columns each) out through a TMA
+// store: the rows go to the warp's staging buffer as 64-byte lines in the
+// 64-byte swizzle (16-byte granule g of row r at g ^ ((r >> 1) & 3): the
+// eight lanes of each store phase hit eight different bank groups), then
+// one lane stores the box at (col0, row0).  Each store instruction of the
+// direct path touches 32 rows; this writes whole lines.  The previous
+// chunk's store must have read the buffer first.
+__device__ __forceinline__ void stage_store_bf16x32(const CUtensorMap* tm, uint8_t* stg,
+                                                    const float (&v)[32], int lane, int col0,
+                                                    int row0) {
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * g + 0], v[8 * g + 1]);
+    w.y = pack_bf16x2(v[8 * g + 2], v[8 * g + 3]);
+    w.z = pack_bf16x2(v[8 * g + 4], v[8 * g + 5]);
+    w.w = pack_bf16x2(v[8 * g + 6], v[8 * g + 7]);
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) = w;
+  }
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tm, stg, col0, row0);
+    bulk_commit_group();
+  }
 }
 
 template <int CG, int BNT, int RH, int EPI>
@@ -741,6 +775,16 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       } else {
         uint4 aux_w[4];
         constexpr bool kDact = EPI == EPI_DACT || EPI == EPI_DACT_Y;
+        // bf16 outputs through this warp's staging buffer and a TMA store
+        // when the outputs have tensor maps, else stored from registers
+        uint8_t* stg = smem + C::kOffStage + ew * C::kStageBytes;
+        const int row_w = row - lane;   // the warp's first row
+        auto put = [&](int o, void* out, const float (&vals)[32], int col0) {
+          if (a.tma_out)
+            stage_store_bf16x32(&P.tmO[prob][o], stg, vals, lane, col0, row_w);
+          else if (row_ok)
+            store_bf16x32(static_cast<__nv_bfloat16*>(out) + row * a.ldo + col0, vals, a.N - col0);
+        };
         if constexpr (kDact) {   // U for the first chunk
           const int col0 = tn * BNT + c0 * 32;
           if (row_ok && col0 < a.N) {
@@ -773,9 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
 
           if constexpr (EPI == EPI_STORE_BF16) {
-            if (store_ok)
-              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
-                            a.N - col0);
+            if (col0 < a.N) put(0, a.out0, v, col0);
           } else if constexpr (EPI == EPI_STORE_F32) {
             if (store_ok) {
               float* dst = static_cast<float*>(a.out0) + row * a.ldo + col0;
@@ -794,16 +836,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
 #pragma unroll
               for (int j = 0; j < 32; ++j) v[j] += b[j];
             }
-            if (store_ok && a.out0 != nullptr)
-              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
-                            a.N - col0);
+            if (col0 < a.N && a.out0 != nullptr) put(0, a.out0, v, col0);
             if (a.act == TP_ACT_GELU_TANH)
               act_chunk<TP_ACT_GELU_TANH>(v);
             else if (a.act == TP_ACT_GELU_ERF)
               act_chunk<TP_ACT_GELU_ERF>(v);
-            if (store_ok)
-              store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, v,
-                            a.N - col0);
+            if (col0 < a.N) put(1, a.out1, v, col0);
           } else {  // EPI_DACT, EPI_DACT_Y
             if constexpr (EPI == EPI_DACT_Y) {
               // U is dead after its derivative: its registers take Y = act(U)
@@ -821,13 +859,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
               else
                 dact_chunk<TP_ACT_NONE>(v, aux_v, store_ok);
             }
-            if (store_ok)
-              store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v,
-                            a.N - col0);
+            if (col0 < a.N) put(0, a.out0, v, col0);
             if constexpr (EPI == EPI_DACT_Y) {
-              if (store_ok)
-                store_bf16x32(static_cast<__nv_bfloat16*>(a.out1) + row * a.ldo + col0, aux_v,
-                              a.N - col0);
+              if (col0 < a.N) put(1, a.out1, aux_v, col0);
             }
             if (a.dbias_part != nullptr) {
               const float colsum = warp_column_sums(v, lane);
@@ -861,6 +895,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           mbar_arrive(&tempty[acc]);
       }
     }
+    if (lane == 0) bulk_wait_group0();   // this warp's TMA stores have landed
   }
 
   tc_fence_before_sync();
@@ -892,7 +927,8 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 // Row-major bf16 matrix [outer, inner] with row stride ld (elements); box of
 // box_inner x box_outer elements, 128-byte swizzle, zero fill outside.
 bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
-               uint32_t box_inner, uint32_t box_outer) {
+               uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = get_encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -900,9 +936,15 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// TP_GEMM_NO_TMA_STORE=1 stores the bf16 outputs from registers (sweeps).
+bool tma_store_disabled() {
+  const char* e = std::getenv("TP_GEMM_NO_TMA_STORE");
+  return e && e[0] == '1';
 }
 
 // Programmatic dependent launch of the GEMMs; TP_GEMM_NO_PDL=1 turns it off
@@ -1110,7 +1152,7 @@ namespace {
 // Kernel arguments, operand maps and (split epilogue) workspace of one
 // problem with the given tile shape.
 tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& a,
-                        CUtensorMap* tmA, CUtensorMap* tmB, cudaStream_t stream) {
+                        CUtensorMap* tmA, CUtensorMap* tmB, CUtensorMap* tmO, cudaStream_t stream) {
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return TP_ERR_SHAPE;
   if (p.splits < 1 || p.splits > kMaxSplits) return TP_ERR_SHAPE;
   const bool split_epi = p.splits > 1 || p.zpart != nullptr;
@@ -1192,7 +1234,24 @@ tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& 
     ok = make_tmap(tmB, p.B, p.K, p.N, p.ldb, BK, b_rows);
   else
     ok = make_tmap(tmB, p.B, p.N, p.K, p.ldb, 64, BK);
-  return ok ? TP_OK : TP_ERR_CUDA;
+  if (!ok) return TP_ERR_CUDA;
+  // the bf16 outputs of the plain, bias + activation and dGeLU epilogues
+  // leave through 32 x 32 TMA stores when both can be described (16-byte
+  // aligned base, row stride a multiple of 16 bytes); otherwise from
+  // registers
+  a.tma_out = 0;
+  const bool staged = !split_epi && (p.epi == EPI_STORE_BF16 || p.epi == EPI_BIAS_ACT ||
+                                     p.epi == EPI_DACT || p.epi == EPI_DACT_Y);
+  if (staged && !(tma_store_disabled())) {
+    bool mk = true;
+    void* outs[2] = {p.out0, p.out1};
+    for (int o = 0; o < 2 && mk; ++o)
+      if (outs[o] != nullptr)
+        mk = (reinterpret_cast<uintptr_t>(outs[o]) & 15) == 0 && (p.ldo * 2) % 16 == 0 &&
+             make_tmap(&tmO[o], outs[o], p.N, p.M, p.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
+    a.tma_out = mk ? 1 : 0;
+  }
+  return TP_OK;
 }
 
 tp_status dispatch(GemmParams& prm, const TileChoice& tile, int epi, cudaStream_t stream) {
@@ -1217,10 +1276,13 @@ tp_status gemm_tc_launch(const GemmProblem& p, cudaStream_t stream) {
   const TileChoice tile = choose_tile(p.M, p.N, p.K, p.splits, epi);
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
-  if (tp_status st = setup_problem(p, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], stream)) return st;
+  if (tp_status st = setup_problem(p, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], prm.tmO[0], stream))
+    return st;
   prm.a[1] = prm.a[0];
   prm.tmA[1] = prm.tmA[0];
   prm.tmB[1] = prm.tmB[0];
+  prm.tmO[1][0] = prm.tmO[0][0];
+  prm.tmO[1][1] = prm.tmO[0][1];
   prm.units0 = prm.a[0].num_units;
   prm.total_units = prm.units0;
   return dispatch(prm, tile, epi, stream);
@@ -1245,8 +1307,10 @@ tp_status gemm_tc_launch_pair(const GemmProblem& p0, const GemmProblem& p1, cuda
   if ((p0.M <= BM || p1.M <= BM) && tile.cg == 2) tile = TileChoice{1, 256, 1};
   GemmParams prm;
   memset(&prm, 0, sizeof(prm));
-  if (tp_status st = setup_problem(p0, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], stream)) return st;
-  if (tp_status st = setup_problem(p1, tile, prm.a[1], &prm.tmA[1], &prm.tmB[1], stream)) return st;
+  if (tp_status st = setup_problem(p0, tile, prm.a[0], &prm.tmA[0], &prm.tmB[0], prm.tmO[0], stream))
+    return st;
+  if (tp_status st = setup_problem(p1, tile, prm.a[1], &prm.tmA[1], &prm.tmB[1], prm.tmO[1], stream))
+    return st;
   prm.units0 = prm.a[0].num_units;
   prm.total_units = prm.units0 + prm.a[1].num_units;
   return dispatch(prm, tile, p0.epi, stream);
