@@ -348,6 +348,27 @@ __device__ __forceinline__ void stage_store_bf16x32(const CUtensorMap* tm, uint8
   }
 }
 
+// fp32 outputs: half h (16 of the chunk's 32 columns, 64-byte lines) of the
+// chunk through the same staging buffer and a TMA store with an evict-first
+// hint (the logits are written once and read by a later kernel).
+__device__ __forceinline__ void stage_store_f32x16(const CUtensorMap* tm, uint8_t* stg,
+                                                   const float (&v)[32], int h, int lane, int col0,
+                                                   int row0) {
+  if (lane == 0) bulk_wait_group_read0();
+  __syncwarp();
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    *reinterpret_cast<float4*>(stg + lane * 64 + ((g ^ ((lane >> 1) & 3)) << 4)) =
+        make_float4(v[16 * h + 4 * g], v[16 * h + 4 * g + 1], v[16 * h + 4 * g + 2],
+                    v[16 * h + 4 * g + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d_evict_first(tm, stg, col0 + 16 * h, row0);
+    bulk_commit_group();
+  }
+}
+
 template <int CG, int BNT, int RH, int EPI>
 __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_constant__ GemmParams P) {
   using C = Cfg<CG, BNT, RH>;
@@ -819,7 +840,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
           if constexpr (EPI == EPI_STORE_BF16) {
             if (col0 < a.N) put(0, a.out0, v, col0);
           } else if constexpr (EPI == EPI_STORE_F32) {
-            if (store_ok) {
+            if (a.tma_out) {
+              if (col0 < a.N) {
+                stage_store_f32x16(&P.tmO[prob][0], stg, v, 0, lane, col0, row_w);
+                if (col0 + 16 < a.N) stage_store_f32x16(&P.tmO[prob][0], stg, v, 1, lane, col0, row_w);
+              }
+            } else if (store_ok) {
               float* dst = static_cast<float*>(a.out0) + row * a.ldo + col0;
 #pragma unroll
               for (int j = 0; j < 8; ++j)
@@ -938,6 +964,35 @@ bool make_tmap(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, 
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// TP_GEMM_BAND_MB=<MB> sizes the rasterisation bands by the bytes of their
+// A rows instead (sweeps); 0 when unset.
+double band_budget_bytes() {
+  static double bytes = [] {
+    double mb = 0.0;
+    if (const char* e = std::getenv("TP_GEMM_BAND_MB")) {
+      const double v = std::atof(e);
+      if (v > 0.0) mb = v;
+    }
+    return mb * 1024.0 * 1024.0;
+  }();
+  return bytes;
+}
+
+// Row-major fp32 matrix [outer, inner], row stride ld elements.
+bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
+                   uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  auto fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {ld * 4};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -1111,17 +1166,8 @@ bool make_tmap_bf16_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t 
 
 bool make_tmap_f32_sw128(void* tmap, const void* ptr, uint64_t inner, uint64_t outer, uint64_t ld,
                          uint32_t box_inner, uint32_t box_outer) {
-  auto fn = get_encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {ld * 4};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(static_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
-                  const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_tmap_f32(static_cast<CUtensorMap*>(tmap), ptr, inner, outer, ld, box_inner, box_outer,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 size_t gemm_split_ws_bytes(int M, int N, int splits, bool with_zpart) {
@@ -1166,7 +1212,17 @@ tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& 
   a.tiles_m = (p.M + rows - 1) / rows;
   a.tiles_n = (p.N + BNT - 1) / BNT;
   a.splits = p.splits;
+  // bands of 2048 rows (inside a band the B columns are read once, so B is
+  // read once per band and A once in all).  Taller bands read less in
+  // principle but measured slower with more DRAM reads (the logits GEMM:
+  // 7.3 GB read with 32-tile-row bands against 6.5 GB with 8); the byte
+  // budget rule stays as a sweep switch
   a.group_m = CG == 2 ? 8 : 16;
+  if (band_budget_bytes() > 0.0) {
+    const double row_bytes = static_cast<double>(rows) * ((p.K + p.splits - 1) / p.splits) * 2.0;
+    const int band = static_cast<int>(band_budget_bytes() / row_bytes);
+    a.group_m = band < 1 ? 1 : (band > a.tiles_m ? a.tiles_m : band);
+  }
   const int kblocks = (p.K + BK - 1) / BK;
   if (p.splits == 1) {
     a.split_kb[0] = 0;
@@ -1250,6 +1306,10 @@ tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& 
         mk = (reinterpret_cast<uintptr_t>(outs[o]) & 15) == 0 && (p.ldo * 2) % 16 == 0 &&
              make_tmap(&tmO[o], outs[o], p.N, p.M, p.ldo, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B);
     a.tma_out = mk ? 1 : 0;
+  } else if (!split_epi && p.epi == EPI_STORE_F32 && !tma_store_disabled()) {
+    // fp32: boxes of 16 columns (64-byte lines) x 32 rows
+    a.tma_out = (reinterpret_cast<uintptr_t>(p.out0) & 15) == 0 && (p.ldo * 4) % 16 == 0 &&
+                make_tmap_f32(&tmO[0], p.out0, p.N, p.M, p.ldo, 16, 32, CU_TENSOR_MAP_SWIZZLE_64B);
   }
   return TP_OK;
 }
