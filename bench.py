@@ -465,14 +465,20 @@ def _e2e_mlp(tpl, torch, g, dev, steps, keys=E2E_DATA):
     return ms, h2d, d2h
 
 
+SETTLE_S = 0.1
+
+
 def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world, reps=10):
     """Average ms per call of each part in plist, max over ranks.
 
     Each part is captured into a CUDA graph of `reps` back-to-back calls and
     the graph is replayed `nsteps` times between two CUDA events, so host
     launch overhead cannot leave the GPU idle inside the timed interval (it
-    would for parts of a few tens of microseconds).  Parts that cannot be
-    captured are timed as a plain loop of calls instead."""
+    would for parts of a few tens of microseconds).  Before its timed
+    replays each part replays untimed for at least SETTLE_S seconds: a part
+    is then timed at the clocks its own load settles to, not at those the
+    previous (power-capped, GEMM-heavy) loop left behind.  Parts that cannot
+    be captured are timed as a plain loop of calls instead."""
     for _ in range(2):
         for p in plist:
             fns[p]()
@@ -486,6 +492,10 @@ def _side_loop(torch, fns, plist, nsteps, stream, dev, st, world, reps=10):
                     fns[p]()
             graph.replay()
             torch.cuda.synchronize(dev)
+            t_settle = time.perf_counter()
+            while time.perf_counter() - t_settle < SETTLE_S:
+                graph.replay()
+                torch.cuda.synchronize(dev)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for _ in range(nsteps):
