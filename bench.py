@@ -548,11 +548,13 @@ def _embed_flushed(torch, tpl, vo, stream, st, n=10):
     return ms
 
 
-def _library_context(torch, g, vo, stream, n=10):
+def _library_context(torch, g, vo, stream, n=10, ours=None):
     """cuBLAS (torch.matmul, bf16 in, fp32 accumulate) on the six GEMM shapes
     of the TP-MLP at h=4096 with the operand transposes the layer needs, and
     torch.nn.functional.cross_entropy (sum, forward + backward) on the same
-    fp32 logits as vp_xent.  Library context, not the product's path."""
+    fp32 logits as vp_xent.  Library context, not the product's path.
+    `ours` (mlp_fwd, mlp_bwd) are timed right after the GEMMs in the same
+    kind of loop, so the two sums compare under the same conditions."""
     import torch.nn.functional as F
 
     X, A, B, dZ, U, Y, dU = (g[k] for k in ("X", "A", "B", "dZ", "U", "Y", "dU"))
@@ -579,6 +581,21 @@ def _library_context(torch, g, vo, stream, n=10):
                    "%d calls each" % n,
            "mlp_gemms": out, "mlp_gemms_sum_ms": round(total, 4),
            "mlp_gemms_sum_tflops": round(MLP_FLOP / (total / 1e3) / 1e12, 1)}
+    if ours is not None:
+        fwd, bwd = ours
+        for _ in range(3):
+            fwd()
+            bwd()
+        ms_f = _event_loop(torch, fwd, n, stream)
+        ms_b = _event_loop(torch, bwd, n, stream)
+        ctx["tp_mlp_same_loop"] = {
+            "what": "this library's tp_mlp_fwd and tp_mlp_bwd (all six GEMMs with their fused "
+                    "bias/GeLU, dGeLU, dbias and shard-sum epilogues) timed the same way, "
+                    "%d calls each, right after the cuBLAS GEMMs" % n,
+            "fwd_ms": round(ms_f, 4), "bwd_ms": round(ms_b, 4),
+            "sum_ms": round(ms_f + ms_b, 4),
+            "tflops": round(MLP_FLOP / ((ms_f + ms_b) / 1e3) / 1e12, 1),
+            "vs_cublas_sum": round(total / (ms_f + ms_b), 4)}
     if vo is not None:
         L = vo["logits"].detach().requires_grad_(True)
         tg = vo["targets"]
@@ -709,7 +726,8 @@ def run_gpu(args):
     ln_ms = _side_loop(torch, fns, LN_PARTS, side_steps, stream, dev, st, world)
 
     embed_flush_ms = _embed_flushed(torch, tpl, vo, stream, st)
-    libctx = None if args.no_library_context else _library_context(torch, g, vo, stream)
+    libctx = (None if args.no_library_context else
+              _library_context(torch, g, vo, stream, ours=(fns["mlp_fwd"], fns["mlp_bwd"])))
 
     if args.no_e2e:
         e2e_ms, h2d, d2h = float("nan"), 0, 0
