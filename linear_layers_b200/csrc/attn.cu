@@ -439,17 +439,20 @@ __global__ void __launch_bounds__(kFwdThreads, 2) attn_fwd_kernel(const __grid_c
 // the key tiles' contributions in fp32 in whatever order they arrive, so its
 // last bits may differ between runs.
 //
-// Roles (10 warps): warp 0 TMA (the fixed K and V tiles once, the streamed
+// Roles (11 warps): warp 0 TMA (the fixed K and V tiles once, the streamed
 // Q and dO tiles through a three-stage ring), warp 1 the MMA issuer, warps 2-5
-// and 6-9 two element-wise warpgroups taking the streamed tiles in turn.
-// S/dP and the bf16 P tiles are double buffered and the dS tiles quadruple
-// buffered (a pair of them is read by the dQ MMA), so the MMAs of one tile
-// run while the other warpgroup evaluates its exponentials.  Warpgroup w also
-// reads out the dQ of the pairs p ≡ w (mod 2), two streamed tiles later.
+// and 6-9 two element-wise warpgroups taking the streamed tiles in turn,
+// warp 10 the dQ reduces.  S/dP and the bf16 P tiles are double buffered and
+// the dS tiles quadruple buffered (a pair of them is read by the dQ MMA), so
+// the MMAs of one tile run while the other warpgroup evaluates its
+// exponentials.  Warpgroup w also reads out and stages the dQ of the pairs
+// p ≡ w (mod 2), two streamed tiles later; warp 10 issues each pair's TMA
+// reduce and alone waits for it to have read the staging buffer.
 // ===========================================================================
 constexpr int kBG = 64;                                // streamed rows per tile
 constexpr int kGStages = 3;
-constexpr int kBwdThreads = 320;                       // 10 warps
+constexpr int kBwdThreads = 352;                       // 11 warps
+constexpr int kRedWarp = 10;                           // issues the dQ reduces
 constexpr int kDSBufs = 4;
 constexpr uint32_t kGTile = kBG * kHD * 2;             // 8 KB: 64 rows of 128 bytes
 constexpr uint32_t kPTile = kBQ * kBG * 2;             // 16 KB: 128 keys x 64 queries
@@ -461,9 +464,9 @@ constexpr uint32_t kBOffP = kBOffG2 + kGStages * kGTile;   // Pᵀ [2 buffers]
 constexpr uint32_t kBOffDS = kBOffP + 2 * kPTile;          // dSᵀ [kDSBufs buffers]
 constexpr uint32_t kBOffStage = kBOffDS + kDSBufs * kPTile;   // dQ of a pair, fp32, 2 x 16 KB
 constexpr uint32_t kStageHalf = kBQ * 32 * 4;                    // 128 rows x 32 columns
-constexpr uint32_t kBOffVec = kBOffStage + 2 * kStageHalf;      // [warpgroup][2][lse·log2e | D][64]
+constexpr uint32_t kBOffVec = kBOffStage + 2 * kStageHalf;      // [warpgroup][2][−lse·log2e | −D][64]
 constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * 2 * kBG * 4;
-constexpr int kBNumBars = 2 * kGStages + 15;
+constexpr int kBNumBars = 2 * kGStages + 16;
 constexpr uint32_t kBOffMisc = kBOffBar + kBNumBars * 8;
 constexpr uint32_t kBAlloc = kBOffMisc + 16 + 1024;
 // tensor memory columns: Sᵀ (X) and dPᵀ (Y) double buffered, the
@@ -551,50 +554,49 @@ __device__ __forceinline__ void bwd_timeout(const AttnBwdArgs& a, volatile int* 
   }
 }
 
-// One key row of a streamed tile: p = 2^(x·sl − l) (zero where masked) and
-// dS = p·(y − D), written as bf16 into the row's 128-byte lines of the P and
-// dS tiles, granule g at g ^ (row & 7).  l and D come per query column from
-// shared memory, four at a time.
+// Half h (32 query columns) of one key row of a streamed tile:
+// p = 2^(x·sl − l) (zero where masked) and dS = p·(y − D), written as bf16
+// into the row's 128-byte lines of the P and dS tiles, granule g at
+// g ^ (row & 7).  −l and −D come per query column from shared memory, four
+// at a time; the arithmetic runs on f32x2 pairs.
 template <bool kMask>
-__device__ __forceinline__ void bwd_tile_rows(const uint32_t (&xr)[kBG], const uint32_t (&yr)[kBG],
-                                              const float* vL, const float* vD, float sl, int t0,
+__device__ __forceinline__ void bwd_half_rows(const uint32_t (&xr)[32], const uint32_t (&yr)[32],
+                                              const float* vNL, const float* vND, float sl, int t0,
                                               int kpos, int s, int causal, uint8_t* prow,
-                                              uint8_t* drow, int r) {
+                                              uint8_t* drow, int r, int h) {
+  const float2 sl2 = make_float2(sl, sl);
 #pragma unroll
-  for (int gr = 0; gr < kBG / 8; ++gr) {       // 16-byte granules of the 128-byte row
-    float lv[8], dv[8];
-    const float4 l0 = reinterpret_cast<const float4*>(vL)[2 * gr];
-    const float4 l1 = reinterpret_cast<const float4*>(vL)[2 * gr + 1];
-    const float4 d0 = reinterpret_cast<const float4*>(vD)[2 * gr];
-    const float4 d1 = reinterpret_cast<const float4*>(vD)[2 * gr + 1];
-    lv[0] = l0.x; lv[1] = l0.y; lv[2] = l0.z; lv[3] = l0.w;
-    lv[4] = l1.x; lv[5] = l1.y; lv[6] = l1.z; lv[7] = l1.w;
-    dv[0] = d0.x; dv[1] = d0.y; dv[2] = d0.z; dv[3] = d0.w;
-    dv[4] = d1.x; dv[5] = d1.y; dv[6] = d1.z; dv[7] = d1.w;
-    float p[8], ds[8];
+  for (int g4 = 0; g4 < 4; ++g4) {             // 16-byte granule gr of the 128-byte row
+    const int gr = h * 4 + g4;
+    const float4 l0 = reinterpret_cast<const float4*>(vNL)[2 * gr];
+    const float4 l1 = reinterpret_cast<const float4*>(vNL)[2 * gr + 1];
+    const float4 d0 = reinterpret_cast<const float4*>(vND)[2 * gr];
+    const float4 d1 = reinterpret_cast<const float4*>(vND)[2 * gr + 1];
+    const float2 nl[4] = {make_float2(l0.x, l0.y), make_float2(l0.z, l0.w),
+                          make_float2(l1.x, l1.y), make_float2(l1.z, l1.w)};
+    const float2 nd[4] = {make_float2(d0.x, d0.y), make_float2(d0.z, d0.w),
+                          make_float2(d1.x, d1.y), make_float2(d1.z, d1.w)};
+    uint32_t pw[4], dw[4];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const int j = gr * 8 + t;
-      float pv = ex2f(fmaf(__uint_as_float(xr[j]), sl, -lv[t]));
+    for (int t = 0; t < 4; ++t) {
+      const int j = g4 * 8 + 2 * t;            // column within the half
+      const float2 e = __ffma2_rn(make_float2(__uint_as_float(xr[j]), __uint_as_float(xr[j + 1])),
+                                  sl2, nl[t]);
+      float p0 = ex2f(e.x), p1 = ex2f(e.y);
       if constexpr (kMask) {
-        const int qpos = t0 + j;               // query position of this column
-        pv = (qpos >= s || kpos >= s || (causal && qpos < kpos)) ? 0.0f : pv;
+        const int q0 = t0 + h * 32 + j;        // query positions of the two columns
+        p0 = (q0 >= s || kpos >= s || (causal && q0 < kpos)) ? 0.0f : p0;
+        p1 = (q0 + 1 >= s || kpos >= s || (causal && q0 + 1 < kpos)) ? 0.0f : p1;
       }
-      p[t] = pv;
-      ds[t] = pv * (__uint_as_float(yr[j]) - dv[t]);
+      const float2 dy = __fadd2_rn(make_float2(__uint_as_float(yr[j]), __uint_as_float(yr[j + 1])),
+                                   nd[t]);
+      const float2 ds = __fmul2_rn(make_float2(p0, p1), dy);
+      pw[t] = pack_bf16x2(p0, p1);
+      dw[t] = pack_bf16x2(ds.x, ds.y);
     }
     const int off = (gr ^ (r & 7)) << 4;
-    uint4 w;
-    w.x = pack_bf16x2(p[0], p[1]);
-    w.y = pack_bf16x2(p[2], p[3]);
-    w.z = pack_bf16x2(p[4], p[5]);
-    w.w = pack_bf16x2(p[6], p[7]);
-    *reinterpret_cast<uint4*>(prow + off) = w;
-    w.x = pack_bf16x2(ds[0], ds[1]);
-    w.y = pack_bf16x2(ds[2], ds[3]);
-    w.z = pack_bf16x2(ds[4], ds[5]);
-    w.w = pack_bf16x2(ds[6], ds[7]);
-    *reinterpret_cast<uint4*>(drow + off) = w;
+    *reinterpret_cast<uint4*>(prow + off) = make_uint4(pw[0], pw[1], pw[2], pw[3]);
+    *reinterpret_cast<uint4*>(drow + off) = make_uint4(dw[0], dw[1], dw[2], dw[3]);
   }
 }
 
@@ -610,7 +612,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   uint8_t* sP = smem + kBOffP;
   uint8_t* sDS = smem + kBOffDS;
   uint8_t* sStage = smem + kBOffStage;
-  float* vec = reinterpret_cast<float*>(smem + kBOffVec);   // [warpgroup][buffer][lse | D][64]
+  float* vec = reinterpret_cast<float*>(smem + kBOffVec);   // [warpgroup][buffer][−lse | −D][64]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kBOffBar);
   uint64_t* f_full = bars;
   uint64_t* g_full = bars + 1;                   // [stage]
@@ -622,7 +624,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
   uint64_t* q_full = pd_empty + 2;               // [pair & 1]: dQ of a pair in tensor memory
   uint64_t* q_empty = q_full + 2;                // [pair & 1]: read out
   uint64_t* acc_done = q_empty + 2;
-  uint64_t* stage_free = acc_done + 1;           // the staged dQ of a pair read by its reduce
+  uint64_t* stage_full = acc_done + 1;           // the dQ of a pair staged in shared memory
+  uint64_t* stage_free = stage_full + 1;         // ... and read by its TMA reduce
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kBOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kBOffMisc + 4);
 
@@ -659,6 +662,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       mbar_init(&q_empty[i], kSoftmaxThreads);
     }
     mbar_init(acc_done, 1);
+    mbar_init(stage_full, kSoftmaxThreads);
     mbar_init(stage_free, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -791,6 +795,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
         mbar_arrive(acc_done);
       }
     }
+  } else if (warp == kRedWarp) {
+    // ------------------------------------------------------------ dQ reduces
+    // each pair's staged dQ goes to L2 as two TMA reduce-adds; the buffer is
+    // handed back once they have read it (this thread alone waits for that)
+    if (elect_one_sync()) {
+      for (int pr = 0; pr < npairs; ++pr) {
+        if (!mbar_wait_bounded(stage_full, static_cast<uint32_t>(pr) & 1u, a.wait_ns, abort_flag)) {
+          bwd_timeout(a, abort_flag);
+          break;
+        }
+        const int y = row0 + (t_begin + 2 * pr) * kBG;
+        tma_reduce_add_2d(&P.tm_dq, sStage, head * kHD, y);
+        tma_reduce_add_2d(&P.tm_dq, sStage + kStageHalf, head * kHD + 32, y);
+        bulk_commit_group();
+        bulk_wait_group_read0();
+        mbar_arrive(stage_free);
+      }
+      bulk_wait_group0();              // the reduces have landed
+    }
   } else {
     // ------------------------------------------------------------ element-wise
     const int wg = (warp - 2) >> 2;                // warpgroup: streamed tiles wg, wg + 2, ...
@@ -805,21 +828,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     uint8_t* prow = sP + wg * kPTile + r * 128;
     bool ok = true;
     // dQ of pair pr (queries of streamed tiles 2pr, 2pr+1 = TMEM lanes): read
-    // out, staged as two 128-byte-swizzled fp32 boxes of 32 columns (rows
-    // past s as zeros) and added into the accumulator by one thread's TMA
-    // reduce.  Every thread of the warpgroup enters (the call sites depend
-    // only on the tile and the warpgroup) with its own state `in`; the first
-    // barrier ANDs those, so all threads return the same answer and none is
-    // left waiting in the second barrier after a timeout.
+    // out and staged as two 128-byte-swizzled fp32 boxes of 32 columns (rows
+    // past s as zeros) for the reduce warp.  `in` is the thread's state so
+    // far; the answer is uniform across the warp, and a warp that gives up
+    // does not arrive, so the reduce warp's bounded wait ends the pair.
     auto drain_pair = [&](int pr, bool in) -> bool {
       // the pair's dQ is in tensor memory and the staging buffer is free
       // once the previous pair's reduce has read it
-      bool good = in &&
-                  mbar_wait_bounded(&q_full[pr & 1], static_cast<uint32_t>(pr >> 1) & 1u, a.wait_ns,
-                                    abort_flag) &&
-                  (pr == 0 || mbar_wait_bounded(stage_free, static_cast<uint32_t>(pr - 1) & 1u,
-                                                a.wait_ns, abort_flag));
-      if (!named_barrier_and(3 + wg, kSoftmaxThreads, good)) return false;
+      if (!__all_sync(0xffffffffu,
+                      in &&
+                          mbar_wait_bounded(&q_full[pr & 1], static_cast<uint32_t>(pr >> 1) & 1u,
+                                            a.wait_ns, abort_flag) &&
+                          (pr == 0 || mbar_wait_bounded(stage_free, static_cast<uint32_t>(pr - 1) & 1u,
+                                                        a.wait_ns, abort_flag))))
+        return false;
       tc_fence_after_sync();
       const bool valid = (t_begin + 2 * pr) * kBG + r < a.s;
 #pragma unroll
@@ -838,25 +860,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       tc_fence_before_sync();
       mbar_arrive(&q_empty[pr & 1]);               // dQ read: the MMA may reuse its columns
       fence_proxy_async_smem();                    // staged dQ visible to the TMA unit
-      named_barrier_sync(3 + wg, kSoftmaxThreads);
-      if (et == 0) {
-        const int y = row0 + (t_begin + 2 * pr) * kBG;
-        tma_reduce_add_2d(&P.tm_dq, sStage, head * kHD, y);
-        tma_reduce_add_2d(&P.tm_dq, sStage + kStageHalf, head * kHD + 32, y);
-        bulk_commit_group();
-        bulk_wait_group_read0();
-        mbar_arrive(stage_free);
-      }
+      mbar_arrive(stage_full);
       return true;
     };
-    // lse·log2e and D of the streamed queries: thread et < 64 loads those of
+    // −lse·log2e and −D of the streamed queries: thread et < 64 loads those of
     // query et of a tile one tile ahead of its use, so the global loads are
     // in flight while the warpgroup works on a tile
     float nl = 0.0f, nd = 0.0f;
-    auto fetch_vec = [&](int tile) {
+    auto fetch_vec = [&](int tile) {   // −lse·log2e and −D
       const int q = (t_begin + tile) * kBG + et;
-      nl = q < a.s ? a.lse[sbase + q] * kLog2e : 0.0f;
-      nd = q < a.s ? a.D[sbase + q] : 0.0f;
+      nl = q < a.s ? -a.lse[sbase + q] * kLog2e : 0.0f;
+      nd = q < a.s ? -a.D[sbase + q] : 0.0f;
     };
     if (et < kBG && wg < nt) fetch_vec(wg);
     for (int it = wg; it < nt; it += 2) {
@@ -882,38 +896,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
       // the warpgroup's barriers (the dQ drain's, the next tile's), where
       // the others learn of it
       ok = __all_sync(0xffffffffu, mbar_wait_bounded(&x_full[wg], use & 1u, a.wait_ns, abort_flag));
-      if (ok) {
-        tc_fence_after_sync();
-        uint32_t xr[kBG], yr[kBG];
-#pragma unroll
-        for (int c = 0; c < kBG / 32; ++c) {
-          tmem_ld_32x32b_x32(tmem + lane_off + kTX + wg * kBG + c * 32,
-                             *reinterpret_cast<uint32_t(*)[32]>(&xr[c * 32]));
-          tmem_ld_32x32b_x32(tmem + lane_off + kTY + wg * kBG + c * 32,
-                             *reinterpret_cast<uint32_t(*)[32]>(&yr[c * 32]));
-        }
-        tc_wait_ld();
-        tc_fence_before_sync();
-        mbar_arrive(&x_empty[wg]);               // Sᵀ and dPᵀ read: the MMA may refill them
-        // this warpgroup's P buffer and dS buffer it % 4 are free once the
-        // MMAs issued up to its previous tile (its dV/dK and the dQ of the
-        // pair before) have completed
+      // this warpgroup's P buffer and dS buffer it % 4 are free once the
+      // MMAs issued up to its previous tile (its dV/dK and the dQ of the
+      // pair before) have completed
+      if (ok)
         ok = __all_sync(0xffffffffu, mbar_wait_bounded(&pd_empty[wg], (use & 1u) ^ 1u, a.wait_ns,
                                                        abort_flag));
-        if (ok) {
-          uint8_t* drow = sDS + (it % kDSBufs) * kPTile + r * 128;
-          // the mask can only cut the tiles that meet the diagonal or the end
-          // (of the queries, or of the keys: key rows past s must add nothing
-          // to dQ)
-          const bool need_mask =
-              (a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s || ft * kBQ + kBQ > a.s;
+      if (ok) {
+        tc_fence_after_sync();
+        uint8_t* drow = sDS + (it % kDSBufs) * kPTile + r * 128;
+        // the mask can only cut the tiles that meet the diagonal or the end
+        // (of the queries, or of the keys: key rows past s must add nothing
+        // to dQ)
+        const bool need_mask =
+            (a.causal && t0 < ft * kBQ + kBQ) || t0 + kBG > a.s || ft * kBQ + kBQ > a.s;
+        // the two 32-column halves one after the other (half the registers
+        // in flight); Sᵀ and dPᵀ are released after the second half's loads
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t xr[32], yr[32];
+          tmem_ld_32x32b_x32(tmem + lane_off + kTX + wg * kBG + h * 32, xr);
+          tmem_ld_32x32b_x32(tmem + lane_off + kTY + wg * kBG + h * 32, yr);
+          tc_wait_ld();
+          if (h == 1) {
+            tc_fence_before_sync();
+            mbar_arrive(&x_empty[wg]);           // Sᵀ and dPᵀ read: the MMA may refill them
+          }
           if (need_mask)
-            bwd_tile_rows<true>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r);
+            bwd_half_rows<true>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r, h);
           else
-            bwd_tile_rows<false>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r);
-          fence_proxy_async_smem();              // P and dS visible to the tensor core
-          mbar_arrive(&pd_full[wg]);
+            bwd_half_rows<false>(xr, yr, vL, vD, sl, t0, kpos, a.s, a.causal, prow, drow, r, h);
         }
+        fence_proxy_async_smem();                // P and dS visible to the tensor core
+        mbar_arrive(&pd_full[wg]);
       }
       // the dQ of pair (it − 2 − wg) / 2 when it belongs to this warpgroup:
       // issued after the other warpgroup's tile, it is done by now
@@ -925,7 +940,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1) attn_bwd_kernel(const __grid_c
     ok = named_barrier_and(1 + wg, kSoftmaxThreads, __all_sync(0xffffffffu, ok));
     for (int pr = wg; pr < npairs; pr += 2)
       if (2 * pr + 2 + wg >= nt) ok = drain_pair(pr, ok);
-    if (et == 0) bulk_wait_group0();               // this thread's reduces have landed
     // the accumulated gradients of the key rows: every lane takes part in
     // the warp-collective tensor-memory loads, only rows inside the sequence
     // are stored.  Warpgroup 0 stores dK, warpgroup 1 dV.
