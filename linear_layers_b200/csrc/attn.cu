@@ -59,6 +59,9 @@ constexpr uint32_t kFOffBar = kFOffP + 2 * kPTileF;
 constexpr int kFNumBars = 4 + 2 * kFStages + 4;
 constexpr uint32_t kFOffMisc = kFOffBar + kFNumBars * 8;
 constexpr uint32_t kFwdAlloc = kFOffMisc + 16 + 1024;     // slack for 1024-byte alignment
+static_assert(kFOffK % 1024 == 0 && kFOffV % 1024 == 0 && kFOffP % 1024 == 0 &&
+                  kKVTile % 1024 == 0 && kPTileF % 1024 == 0,
+              "forward shared-memory layout: swizzled tiles on 1024-byte boundaries");
 constexpr uint32_t kFwdTmemCols = 128;                     // S: 64, O: 64
 constexpr uint32_t kFTmemO = 64;
 constexpr uint32_t kTmemCols = 512;                        // backward
@@ -466,6 +469,11 @@ constexpr uint32_t kBOffStage = kBOffDS + kDSBufs * kPTile;   // dQ of a pair, f
 constexpr uint32_t kStageHalf = kBQ * 32 * 4;                    // 128 rows x 32 columns
 constexpr uint32_t kBOffVec = kBOffStage + 2 * kStageHalf;      // [warpgroup][2][−lse·log2e | −D][64]
 constexpr uint32_t kBOffBar = kBOffVec + 2 * 2 * 2 * kBG * 4;
+// every swizzled tile and TMA box starts on a 1024-byte boundary
+static_assert(kBOffG1 % 1024 == 0 && kBOffG2 % 1024 == 0 && kBOffP % 1024 == 0 &&
+                  kBOffDS % 1024 == 0 && kBOffStage % 1024 == 0 && kGTile % 1024 == 0 &&
+                  kPTile % 1024 == 0 && kStageHalf % 1024 == 0,
+              "backward shared-memory layout");
 constexpr int kBNumBars = 2 * kGStages + 16;
 constexpr uint32_t kBOffMisc = kBOffBar + kBNumBars * 8;
 constexpr uint32_t kBAlloc = kBOffMisc + 16 + 1024;
