@@ -504,34 +504,40 @@ struct __align__(64) AttnBwdParams {
 };
 
 // D = rowsum(dO ⊙ O) per (token, head), and the dQ accumulator of that
-// (token, head) set to zero.
+// (token, head) set to zero.  Eight lanes per (token, head): lane j takes
+// columns 8j..8j+7 (one 16-byte word of O and of dO, 32 bytes of the
+// accumulator), so a warp's loads and stores cover four heads' contiguous
+// bytes; the eight partial sums meet by shuffles.
 __global__ void __launch_bounds__(256) attn_bwd_prep_kernel(const uint4* __restrict__ O,
                                                             const uint4* __restrict__ dO,
                                                             int64_t rows, int heads, int s,
                                                             float* __restrict__ D,
                                                             float4* __restrict__ dq_acc) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;   // (row, head)
-  if (i >= rows * heads) return;
-  const int64_t row = i / heads;
-  const int head = static_cast<int>(i - row * heads);
-  const uint4* o = O + (row * heads + head) * 8;     // 64 bf16 of this head
-  const uint4* g = dO + (row * heads + head) * 8;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t rh = i >> 3;                           // (row, head)
+  const int j = static_cast<int>(i & 7);
+  const bool live = rh < rows * heads;                 // whole groups of 8 share it
   float acc = 0.0f;
-#pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint4 a = __ldg(o + k), c = __ldg(g + k);
+  if (live) {
+    const uint4 a = __ldg(O + rh * 8 + j), c = __ldg(dO + rh * 8 + j);
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      acc = fmaf(__uint_as_float(aw[q] << 16), __uint_as_float(cw[q] << 16), acc);
-      acc = fmaf(__uint_as_float(aw[q] & 0xffff0000u), __uint_as_float(cw[q] & 0xffff0000u), acc);
+    for (int w = 0; w < 4; ++w) {
+      acc = fmaf(__uint_as_float(aw[w] << 16), __uint_as_float(cw[w] << 16), acc);
+      acc = fmaf(__uint_as_float(aw[w] & 0xffff0000u), __uint_as_float(cw[w] & 0xffff0000u), acc);
     }
+    dq_acc[rh * 16 + 2 * j] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    dq_acc[rh * 16 + 2 * j + 1] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
   }
-  const int64_t bb = row / s, pos = row - bb * s;
-  D[(bb * heads + head) * s + pos] = acc;
-  float4* z = dq_acc + (row * heads + head) * 16;    // 64 fp32 of this head
-#pragma unroll
-  for (int k = 0; k < 16; ++k) z[k] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+  acc += __shfl_xor_sync(0xffffffffu, acc, 4);
+  if (live && j == 0) {
+    const int64_t row = rh / heads;
+    const int head = static_cast<int>(rh - row * heads);
+    const int64_t bb = row / s, pos = row - bb * s;
+    D[(bb * heads + head) * s + pos] = acc;
+  }
 }
 
 // dQ = scale · (accumulated dS·K), bf16, into this head's Q columns of dQKV.
@@ -1051,7 +1057,7 @@ tp_status attention_bwd_launch(const void* QKV, const void* O, const void* dO, c
                                            ((static_cast<size_t>(b * s) * heads * sizeof(float) + 255) &
                                             ~static_cast<size_t>(255)));
   {
-    const int64_t n = b * s * heads;
+    const int64_t n = b * s * heads * 8;   // eight lanes per (token, head)
     attn_bwd_prep_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, stream>>>(
         static_cast<const uint4*>(O), static_cast<const uint4*>(dO), b * s, heads,
         static_cast<int>(s), D, reinterpret_cast<float4*>(dq_acc));
