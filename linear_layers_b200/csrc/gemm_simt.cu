@@ -161,6 +161,60 @@ __global__ void dact_colsum_kernel(const T* dY, const T* U, int64_t M, int64_t N
   if (part) part[static_cast<int64_t>(blockIdx.y) * N + n] = s;
 }
 
+__device__ __forceinline__ uint32_t pack2_bf16(float lo, float hi) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// bf16, 8 columns per thread (16-byte loads and stores) over 32 rows per
+// block; the activation is a template argument.
+template <int ACT>
+__global__ void __launch_bounds__(128) dact_colsum_v8_kernel(const uint4* __restrict__ dY,
+                                                             const uint4* __restrict__ U,
+                                                             int64_t M, int64_t N,
+                                                             uint4* __restrict__ dU,
+                                                             float* __restrict__ part) {
+  const int64_t c8 = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t n8 = N / 8;
+  if (c8 >= n8) return;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * 32;
+  const int64_t r1 = r0 + 32 < M ? r0 + 32 : M;
+  float s[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+  for (int64_t r = r0; r < r1; ++r) {
+    const uint4 g = __ldg(dY + r * n8 + c8);
+    const uint32_t gw[4] = {g.x, g.y, g.z, g.w};
+    float v[8];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      v[2 * k] = __uint_as_float(gw[k] << 16);
+      v[2 * k + 1] = __uint_as_float(gw[k] & 0xffff0000u);
+    }
+    if constexpr (ACT != TP_ACT_NONE) {
+      const uint4 u = __ldg(U + r * n8 + c8);
+      const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        v[2 * k] *= act_deriv32(__uint_as_float(uw[k] << 16), ACT);
+        v[2 * k + 1] *= act_deriv32(__uint_as_float(uw[k] & 0xffff0000u), ACT);
+      }
+      uint4 o;
+      o.x = pack2_bf16(v[0], v[1]);
+      o.y = pack2_bf16(v[2], v[3]);
+      o.z = pack2_bf16(v[4], v[5]);
+      o.w = pack2_bf16(v[6], v[7]);
+      if (dU) dU[r * n8 + c8] = o;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) s[k] += v[k];
+  }
+  if (part) {
+    float4* dst = reinterpret_cast<float4*>(part + static_cast<int64_t>(blockIdx.y) * N + c8 * 8);
+    dst[0] = make_float4(s[0], s[1], s[2], s[3]);
+    dst[1] = make_float4(s[4], s[5], s[6], s[7]);
+  }
+}
+
 __global__ void dbias_finish_kernel(const float* part, int tiles, int N, float* dbias) {
   const int n = blockIdx.x * blockDim.x + threadIdx.x;
   if (n >= N) return;
@@ -221,8 +275,27 @@ tp_status gemm_simt_launch(const GemmProblem& p, cudaStream_t stream) {
 }
 
 tp_status dact_colsum_launch(const void* dY, const void* U, int64_t M, int64_t Nout, int act,
-                             bool bf16, void* dU, float* dbias_part, cudaStream_t stream) {
+                             bool bf16, void* dU, float* dbias_part, cudaStream_t stream,
+                             int* tiles) {
+  const auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (bf16 && Nout % 8 == 0 && al16(dY) && al16(U) && al16(dU) && al16(dbias_part)) {
+    // 32-row partial sums (the workspace holds ceil(M / 32) rows)
+    dim3 g(static_cast<unsigned>((Nout / 8 + 127) / 128), static_cast<unsigned>((M + 31) / 32));
+    const auto* y = static_cast<const uint4*>(dY);
+    const auto* u = static_cast<const uint4*>(U);
+    auto* d = static_cast<uint4*>(dU);
+    if (act == TP_ACT_GELU_TANH)
+      dact_colsum_v8_kernel<TP_ACT_GELU_TANH><<<g, 128, 0, stream>>>(y, u, M, Nout, d, dbias_part);
+    else if (act == TP_ACT_GELU_ERF)
+      dact_colsum_v8_kernel<TP_ACT_GELU_ERF><<<g, 128, 0, stream>>>(y, u, M, Nout, d, dbias_part);
+    else
+      dact_colsum_v8_kernel<TP_ACT_NONE><<<g, 128, 0, stream>>>(y, u, M, Nout, d, dbias_part);
+    *tiles = static_cast<int>(g.y);
+    note_launches(1);
+    return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+  }
   dim3 grid(static_cast<unsigned>((Nout + 255) / 256), static_cast<unsigned>((M + 127) / 128));
+  *tiles = static_cast<int>(grid.y);
   if (bf16)
     dact_colsum_kernel<__nv_bfloat16><<<grid, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(dY), static_cast<const __nv_bfloat16*>(U), M, Nout, act,

@@ -463,7 +463,8 @@ tp_status tp_col_linear_fwd(const void* X, const void* W, const void* bias, int6
 
 namespace tpl {
 tp_status dact_colsum_launch(const void* dY, const void* U, int64_t M, int64_t Nout, int act,
-                             bool bf16, void* dU, float* dbias_part, cudaStream_t stream);
+                             bool bf16, void* dU, float* dbias_part, cudaStream_t stream,
+                             int* tiles);
 }
 
 extern "C" {
@@ -486,7 +487,7 @@ tp_status tp_col_linear_bwd(const void* X, const void* W, const void* U, const v
   const bool bf16 = dt == TP_DTYPE_BF16;
   cudaStream_t st = as_stream(stream);
   const size_t split_bytes = bf16 ? row_split_ws(M, K, Nout, N, false) : 0;
-  const int64_t mtiles = (M + 127) / 128;
+  int64_t mtiles = (M + 127) / 128;   // partial rows of the column sums (set by their kernel)
   const size_t dbias_bytes = dbias ? dbias_ws(M, Nout) : 0;
   if (split_bytes + dbias_bytes > 0 && (ws == nullptr || ws_bytes < split_bytes + dbias_bytes))
     return TP_ERR_WORKSPACE;
@@ -497,7 +498,10 @@ tp_status tp_col_linear_bwd(const void* X, const void* W, const void* U, const v
   const void* grad = dY;
   if (act != TP_ACT_NONE || dbias) {
     void* dst = act != TP_ACT_NONE ? dU : nullptr;
-    if (tp_status s = dact_colsum_launch(dY, U, M, Nout, act, bf16, dst, dbias_part, st)) return s;
+    int tiles = static_cast<int>(mtiles);
+    if (tp_status s = dact_colsum_launch(dY, U, M, Nout, act, bf16, dst, dbias_part, st, &tiles))
+      return s;
+    mtiles = tiles;
     if (act != TP_ACT_NONE) grad = dU;
   }
   // dW = Xᵀ·dU

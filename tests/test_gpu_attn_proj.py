@@ -113,3 +113,36 @@ def test_attention_projections_full_m():
     obq = O.col_linear_bwd(inp["X"], inp["Wqkv"][:, cols], None, inp["dQKV"][:, cols])
     assert_close("dWqkv[:,cols]", gq["dW"][:, cols.cuda()], obq["dW"], TOL_BF16)
     assert_close("dbqkv[cols]", gq["dbias"][cols.cuda()], obq["dbias"], TOL_BF16)
+
+
+@pytest.mark.parametrize("act", [tpl.ACT_GELU_TANH, tpl.ACT_GELU_ERF, tpl.ACT_NONE])
+@pytest.mark.parametrize("M,K,Nout,N", [(200, 192, 1600, 4), (1000, 320, 648, 3)])
+def test_col_linear_bwd_with_activation(M, K, Nout, N, act):
+    """The column-parallel backward with an activation: dU = dY ⊙ act'(U)
+    and dbias = Σ_rows dU come from the element-wise column-sum kernel
+    (32-row partial sums, ragged last block), then dW and dX."""
+    g = torch.Generator().manual_seed(M + Nout + act)
+    X = (torch.randn(M, K, generator=g) * 0.5).bfloat16()
+    W = (torch.randn(K, Nout, generator=g) * 0.05).bfloat16()
+    U = torch.randn(M, Nout, generator=g).bfloat16()
+    dY = torch.randn(M, Nout, generator=g).bfloat16()
+    bf = torch.bfloat16
+    dX, gx = guarded((M, K), bf)
+    dW, gw = guarded((K, Nout), bf)
+    dbias, gb = guarded((Nout,), torch.float32)
+    dU, gu = guarded((M, Nout), bf) if act != tpl.ACT_NONE else (None, None)
+    st = tpl.new_status()
+    out = tpl.tp_col_linear_bwd(X.cuda(), W.cuda(), U.cuda() if act != tpl.ACT_NONE else None,
+                                dY.cuda(), N, act=act, dU=dU, dX=dX, dW=dW, dbias=dbias,
+                                dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    for gd, name in ((gx, "dX"), (gw, "dW"), (gb, "dbias"), (gu, "dU")):
+        if gd is not None:
+            gd.check(name)
+    ref = O.col_linear_bwd(X, W, U, dY, act)   # act' = 1 everywhere without an activation
+    if act != tpl.ACT_NONE:
+        assert_close("dU", f64(out["dU"]), ref["dU"], TOL_BF16)
+    assert_close("dbias", f64(out["dbias"]), ref["dbias"], TOL_BF16)
+    assert_close("dW", f64(out["dW"]), ref["dW"], TOL_BF16)
+    assert_close("dX", f64(out["dX"]), ref["dX"], TOL_BF16)
