@@ -155,8 +155,10 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ float max4(const float4& a) {
-  return fmaxf(fmaxf(a.x, a.y), fmaxf(a.z, a.w));
+__device__ __forceinline__ float max3f(float a, float b, float c) {   // three-input max
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
 }
 
 // Gradient stores: fp32 float4, or four bf16 (round to nearest even) in 8 bytes.
@@ -252,9 +254,9 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
 
     // 1) each warp's maximum, the first position of it, e = exp(l − m_w) kept
     //    in registers and the warp's sum: one warp-level pass, no barrier
-    float mt = max4(x[0]);
+    float mt = -CUDART_INF_F;
 #pragma unroll
-    for (int r = 1; r < R; ++r) mt = fmaxf(mt, max4(x[r]));
+    for (int r = 0; r < R; ++r) mt = max3f(max3f(mt, x[r].x, x[r].y), x[r].z, x[r].w);
     float m_w = mt;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) m_w = fmaxf(m_w, __shfl_xor_sync(0xffffffffu, m_w, off));
@@ -271,15 +273,22 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
     }
     // a warp whose elements are all padding (−inf) contributes nothing
     const float mL = m_w == -CUDART_INF_F ? 0.0f : m_w * kLog2e;
-    float st = 0.f;
+    // the exponent arguments, the sums and (below) the gradient scaling run
+    // on f32x2 pairs
+    const float2 l2e2 = make_float2(kLog2e, kLog2e), nml2 = make_float2(-mL, -mL);
+    float2 st2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      x[r].x = ex2_approx(fmaf(x[r].x, kLog2e, -mL));
-      x[r].y = ex2_approx(fmaf(x[r].y, kLog2e, -mL));
-      x[r].z = ex2_approx(fmaf(x[r].z, kLog2e, -mL));
-      x[r].w = ex2_approx(fmaf(x[r].w, kLog2e, -mL));
-      st += (x[r].x + x[r].y) + (x[r].z + x[r].w);
+      const float2 a = __ffma2_rn(make_float2(x[r].x, x[r].y), l2e2, nml2);
+      const float2 b = __ffma2_rn(make_float2(x[r].z, x[r].w), l2e2, nml2);
+      x[r].x = ex2_approx(a.x);
+      x[r].y = ex2_approx(a.y);
+      x[r].z = ex2_approx(b.x);
+      x[r].w = ex2_approx(b.y);
+      st2 = __fadd2_rn(st2, make_float2(x[r].x, x[r].y));
+      st2 = __fadd2_rn(st2, make_float2(x[r].z, x[r].w));
     }
+    float st = st2.x + st2.y;
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) {
       st += __shfl_xor_sync(0xffffffffu, st, off);
@@ -362,11 +371,13 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
       for (int r = 0; r < R; ++r) {
         const int j = threadIdx.x + r * NT;
         if (j < nvec) {
-          float4 e = x[r];
-          e.x *= scale;
-          e.y *= scale;
-          e.z *= scale;
-          e.w *= scale;
+          float4 e;
+          const float2 lo2 = __fmul2_rn(make_float2(x[r].x, x[r].y), make_float2(scale, scale));
+          const float2 hi2 = __fmul2_rn(make_float2(x[r].z, x[r].w), make_float2(scale, scale));
+          e.x = lo2.x;
+          e.y = lo2.y;
+          e.z = hi2.x;
+          e.w = hi2.y;
           if ((yl >> 2) == j) {
             const int q = yl & 3;
             if (q == 0) e.x -= grad_scale;
