@@ -65,6 +65,8 @@ struct GemmArgs {
   int M, N, K;
   int a_mn, b_mn;
   int tiles_m, tiles_n, splits, group_m;
+  int full_tiles;                   // split-sum GEMMs: the first full_tiles tiles (raster
+                                    // order) take their whole K range, the rest are split
   int num_units;
   int split_kb[kMaxSplits + 1];     // k-block boundaries of the splits
   int act;
@@ -232,17 +234,24 @@ __device__ __forceinline__ void dact_value_chunk(float (&v)[32], float (&u)[32],
 // tile scheduling: unit -> (tile row, tile column, split)
 // Tiles are visited in bands of group_m tile rows, column by column inside a
 // band, so that one wave of CTAs shares A rows and B columns through L2.
-// Split-major: every tile's first K range, then every tile's second, … so a
-// wave reads one K range of its operands (a third less L2 footprint than
-// running a tile's splits side by side; about 1 % faster for the K = 16384
-// row-parallel GEMM of the MLP), and the last split of a tile sums the
-// partials the earlier splits left behind.
+// Split-sum GEMMs: the first full_tiles tiles take their whole K range
+// (s = −1, stored directly); the tiles of the last, partial wave are split,
+// split-major (every tile's first K range, then every tile's second), and
+// the last split of a tile sums the partials the earlier splits left
+// behind.  Without full tiles every tile is split.
 // -------------------------------------------------------------------------
 __device__ __forceinline__ void unit_map(const GemmArgs& a, int unit, int& tm, int& tn, int& s,
                                          int& tile) {
   const int tiles = a.tiles_m * a.tiles_n;
-  s = unit / tiles;
-  tile = unit - s * tiles;
+  if (unit < a.full_tiles) {
+    s = -1;
+    tile = unit;
+  } else {
+    const int rem = tiles - a.full_tiles;
+    const int u = unit - a.full_tiles;
+    s = u / rem;
+    tile = a.full_tiles + (u - s * rem);
+  }
   const int per_group = a.group_m * a.tiles_n;
   const int g = tile / per_group;
   const int first_m = g * a.group_m;
@@ -444,7 +453,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         unit_map(a, unit - prob * P.units0, tm, tn, s, tile);
         const int a_row = tm * C::kRows + static_cast<int>(rank) * C::kRowsCTA;
         const int b_col = tn * BNT + static_cast<int>(rank) * C::kBCols;
-        for (int kb = a.split_kb[s]; kb < a.split_kb[s + 1]; ++kb) {
+        const int kb_lo = s < 0 ? a.split_kb[0] : a.split_kb[s];
+        const int kb_hi = s < 0 ? a.split_kb[a.splits] : a.split_kb[s + 1];
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (unit == a0.inject_unit && kb == a0.inject_kb) {
             // debug injection: stop issuing without a word, as a producer
             // that died would; the MMA issuer's bounded wait runs out
@@ -543,7 +554,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
         tc_fence_after_sync();
         // RH = 1: accumulator buffer acc; RH = 2: row half h at column h·BNT
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BNT);
-        const int kb0 = a.split_kb[s], kb1 = a.split_kb[s + 1];
+        const int kb0 = s < 0 ? a.split_kb[0] : a.split_kb[s];
+        const int kb1 = s < 0 ? a.split_kb[a.splits] : a.split_kb[s + 1];
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_bounded(&full[stage], phase, a0.wait_ns, abort_flag)) {
             if (!*abort_flag) flag_timeout(a0, abort_flag);
@@ -617,6 +629,21 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
       const int c0 = half * C::kChunks;   // this warp's first 32-column chunk
 
       if constexpr (EPI == EPI_SPLIT_SUM) {
+       if (s < 0) {
+        // a whole tile: the accumulator is the sum over every shard
+#pragma unroll 1
+        for (int c = c0; c < c0 + C::kChunks; ++c) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_base + c * 32, r);
+          tc_wait_ld();
+          const int col0 = tn * BNT + c * 32;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+          if (row_ok && col0 < a.N)
+            store_bf16x32(static_cast<__nv_bfloat16*>(a.out0) + row * a.ldo + col0, v, a.N - col0);
+        }
+       } else {
         // 1) publish this split's fp32 partial
 #pragma unroll 1
         for (int c = c0; c < c0 + C::kChunks; ++c) {
@@ -703,6 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_tc_kernel(const __grid_const
                             a.N - col0);
           }
         }
+       }
       } else if constexpr (EPI == EPI_XENT_STATS) {
         // Softmax statistics of this warp's 128-column slice of each row: the
         // maximum m, s = Σ exp(acc − m) (rescaled whenever m grows) and the
@@ -996,6 +1024,12 @@ bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return r == CUDA_SUCCESS;
 }
 
+// TP_GEMM_SPLIT_ALL=1: split-sum GEMMs split every tile (sweeps).
+bool split_all_tiles() {
+  const char* e = std::getenv("TP_GEMM_SPLIT_ALL");
+  return e && e[0] == '1';
+}
+
 // TP_GEMM_NO_TMA_STORE=1 stores the bf16 outputs from registers (sweeps).
 bool tma_store_disabled() {
   const char* e = std::getenv("TP_GEMM_NO_TMA_STORE");
@@ -1236,7 +1270,16 @@ tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& 
     }
     if (p.split_k[0] != 0 || p.split_k[p.splits] != p.K) return TP_ERR_SHAPE;
   }
-  a.num_units = a.tiles_m * a.tiles_n * a.splits;
+  // split-sum GEMMs split only the tiles of the last, partial wave (the
+  // others run their whole K range in the accumulator); per-shard partials
+  // (Zpart) split every tile.  TP_GEMM_SPLIT_ALL=1 splits every tile (sweeps).
+  a.full_tiles = 0;
+  if (p.splits > 1 && p.zpart == nullptr && !split_all_tiles()) {
+    const int tiles = a.tiles_m * a.tiles_n;
+    const int slots = num_sms() / CG;
+    a.full_tiles = tiles - tiles % slots;
+  }
+  a.num_units = a.full_tiles + (a.tiles_m * a.tiles_n - a.full_tiles) * a.splits;
   // partials requested (Zpart) go through the split epilogue even for a
   // single split: it publishes the partial and stores the (one-term) sum
   if (p.zpart != nullptr && p.epi != EPI_STORE_BF16) return TP_ERR_UNSUPPORTED;
