@@ -189,10 +189,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // Forward for rows of up to 32·CH chunks (h <= 2048): one warp per row, four
-// rows per block, the row in registers and both reductions by shuffles, so
-// no block barrier stands between a row's loads and its stores.
+// rows per block, the row in registers (hs kept packed as bf16 between the
+// passes, which is what the statistics are taken of, and unpacked again in
+// each) and both reductions by shuffles, so no block barrier stands between
+// a row's loads and its stores.
 template <int CH>
-__global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
+__global__ void __launch_bounds__(kLnThreads, 5) sp_ln_fwd_warp_kernel(
     const uint4* __restrict__ x, const uint4* __restrict__ bias, const uint4* __restrict__ residual,
     const uint4* __restrict__ gamma, const uint4* __restrict__ beta, int64_t M, int h8,
     float inv_h, float eps, DropoutRng rng, uint4* __restrict__ hs_out, uint4* __restrict__ y_out,
@@ -200,7 +202,7 @@ __global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
   const int lane = threadIdx.x & 31;
   const int64_t row = static_cast<int64_t>(blockIdx.x) * (kLnThreads / 32) + (threadIdx.x >> 5);
   if (row >= M) return;   // whole warps only
-  float hv[CH][8];
+  uint4 hp[CH];   // hs of the row, packed
   float s = 0.0f;
   // every load of the row first, so that all of them are in flight together
   uint4 xw[CH], rw[CH];
@@ -232,37 +234,43 @@ __global__ void __launch_bounds__(kLnThreads) sp_ln_fwd_warp_kernel(
       for (int i = 0; i < 8; ++i)
         t[i] = rv[i] + (((kb >> i) & 1u) ? (xv[i] + bv[i]) * rng.inv_keep : 0.0f);
       const uint4 packed = pack8(t);
+      hp[k] = packed;
       __stcs(hs_out + o, packed);
       if (keep_out)
         *reinterpret_cast<uint2*>(keep_out + o * 8) = make_uint2(
             ((kb >> 0) & 1u) | (((kb >> 1) & 1u) << 8) | (((kb >> 2) & 1u) << 16) | (((kb >> 3) & 1u) << 24),
             ((kb >> 4) & 1u) | (((kb >> 5) & 1u) << 8) | (((kb >> 6) & 1u) << 16) | (((kb >> 7) & 1u) << 24));
-      unpack8(packed, hv[k]);   // the statistics of hs as stored
+      float hv[8];
+      unpack8(packed, hv);   // the statistics of hs as stored
 #pragma unroll
-      for (int i = 0; i < 8; ++i) s += hv[k][i];
+      for (int i = 0; i < 8; ++i) s += hv[i];
     }
   }
   const float mean = warp_sum(s) * inv_h;
   float q = 0.0f;
 #pragma unroll
   for (int k = 0; k < CH; ++k) {
-    if (lane + 32 * k < h8)
+    if (lane + 32 * k < h8) {
+      float hv[8];
+      unpack8(hp[k], hv);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float d = hv[k][i] - mean;
+        const float d = hv[i] - mean;
         q = fmaf(d, d, q);
       }
+    }
   }
   const float rstd = 1.0f / sqrtf(warp_sum(q) * inv_h + eps);
 #pragma unroll
   for (int k = 0; k < CH; ++k) {
     const int c = lane + 32 * k;
     if (c < h8) {
-      float gv[8], bv[8], yv[8];
+      float gv[8], bv[8], yv[8], hv[8];
+      unpack8(hp[k], hv);
       unpack8(__ldg(gamma + c), gv);
       unpack8(__ldg(beta + c), bv);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) yv[i] = fmaf((hv[k][i] - mean) * rstd, gv[i], bv[i]);
+      for (int i = 0; i < 8; ++i) yv[i] = fmaf((hv[i] - mean) * rstd, gv[i], bv[i]);
       __stcs(y_out + row * h8 + c, pack8(yv));
     }
   }
