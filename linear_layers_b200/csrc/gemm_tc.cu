@@ -20,7 +20,10 @@
 //             pair leader one elected lane issues the MMAs;
 //   warps 2-9 epilogue: tcgen05.ld of the finished accumulator (two warps per
 //             TMEM lane quadrant, 128 columns each), fused element-wise
-//             work, stores to global memory.
+//             work, then each warp's 32 x 32 chunk out through a 64-byte-
+//             swizzled staging buffer and a TMA store (bf16 and fp32
+//             outputs), or stores from registers (split partials, outputs
+//             a tensor map cannot describe).
 // The accumulator is double buffered, so the epilogue of one tile overlaps
 // the main loop of the next.
 //
