@@ -18,6 +18,14 @@ from tests.gpu_helpers import TOL_BF16, TOL_F32, assert_close, to_dev
 
 pytestmark = pytest.mark.gpu
 
+# Per-element bound for dB from a rebuilt Y.  The forward applies GeLU to the
+# fp32 pre-activation; the rebuild only has U rounded to bf16, so every Y
+# carries U's rounding (about 2^-9 relative) on top of its own, and dB = Yᵀ·dZ
+# sums it over the tokens: worst elements of 1.8e-2 against 1.0e-2 for the
+# saved-activation dB on the same inputs, relative Frobenius 3.2e-3 against
+# 2.4e-3.  The Frobenius bound stays TOL_BF16.
+TOL_ELEM_DB_REBUILT = 2 * TOL_BF16
+
 
 def _fwd(d, N, act, offsets=None):
     st = tpl.new_status()
@@ -40,7 +48,7 @@ def test_recompute_ragged_tiles(act):
     oU, oY, _ = O.mlp_fwd(inp["X"], inp["A"], inp["bias"], inp["B"], act)
     assert_close("recomputed Y", g["Y"], oY, TOL_BF16)
     for k in ("dX", "dA", "dB", "dbias", "dU"):
-        assert_close(k, g[k], ob[k], TOL_BF16)
+        assert_close(k, g[k], ob[k], TOL_BF16, elem_tol=TOL_ELEM_DB_REBUILT if k == "dB" else None)
     for k in ("dX", "dA", "dbias", "dU"):
         assert torch.equal(g[k], ref[k]), k
 
@@ -63,7 +71,7 @@ def test_recompute_in_place_and_uneven_shards():
     assert torch.equal(U2, a["Y"])            # U2 now holds the recomputed activation
     ob = O.mlp_bwd(inp["X"], inp["A"], inp["bias"], inp["B"], inp["dZ"])
     for k in ("dX", "dA", "dB", "dbias"):
-        assert_close(k, a[k], ob[k], TOL_BF16)
+        assert_close(k, a[k], ob[k], TOL_BF16, elem_tol=TOL_ELEM_DB_REBUILT if k == "dB" else None)
 
 
 def test_recompute_fp32_path():
@@ -99,4 +107,4 @@ def test_recompute_h4096_sampled_columns():
     cols = np.sort(np.random.default_rng(3).choice(w["F"], 96, replace=False))
     c = torch.as_tensor(cols)
     ob = O.mlp_bwd(inp["X"], inp["A"][:, c], inp["bias"][c], inp["B"][c], inp["dZ"])
-    assert_close("dB[cols]", g["dB"][c.cuda()], ob["dB"], TOL_BF16)
+    assert_close("dB[cols]", g["dB"][c.cuda()], ob["dB"], TOL_BF16, elem_tol=TOL_ELEM_DB_REBUILT)
