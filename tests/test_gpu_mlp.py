@@ -171,3 +171,17 @@ def test_mlp_every_tile_shape(tile, monkeypatch):
     # long K over 8 shards: the split shard sum (two or more K ranges per tile)
     inp = tp_inputs.mlp_inputs(512, 256, 4096, w_std=0.02, bias_std=0.02, seed=22)
     _check_full(inp, 8, tpl.ACT_GELU_TANH, TOL_BF16)
+
+
+@pytest.mark.parametrize("switch", ["TP_GEMM_NO_TMA_STORE", "TP_GEMM_SPLIT_ALL"])
+def test_mlp_alternate_gemm_paths(switch, monkeypatch):
+    """The two GEMM paths the defaults leave unused: outputs stored from
+    registers instead of through staged tensor-map stores, and the shard sum
+    split on every tile instead of on the tail that does not fill the
+    persistent slots."""
+    monkeypatch.setenv(switch, "1")
+    inp = tp_inputs.mlp_inputs(300, 264, 1024, w_std=0.05, bias_std=0.02, seed=23)
+    _check_full(inp, 4, tpl.ACT_GELU_TANH, TOL_BF16, zpart=True)
+    _check_full(inp, 3, tpl.ACT_GELU_ERF, TOL_BF16, offsets=[0, 128, 448, 1024])
+    inp = tp_inputs.mlp_inputs(512, 256, 4096, w_std=0.02, bias_std=0.02, seed=24)
+    _check_full(inp, 8, tpl.ACT_GELU_TANH, TOL_BF16)

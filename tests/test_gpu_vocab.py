@@ -71,6 +71,17 @@ def test_logits_ragged():
         assert_close(f"logits shard {i}", L[:, i * 250:(i + 1) * 250], b, TOL_BF16)
 
 
+def test_logits_ragged_register_store(monkeypatch):
+    """The fp32 logits stored from registers instead of through tensor-map
+    stores (the path taken when the output is not 16-byte aligned)."""
+    monkeypatch.setenv("TP_GEMM_NO_TMA_STORE", "1")
+    inp = tp_inputs.vocab_inputs(300, 1000, 264, seed=5)
+    L, gl = guarded((300, 1000), torch.float32)
+    tpl.tp_logits_fwd(inp["H"].cuda(), inp["E"].cuda(), 4, logits=L)
+    gl.check("logits")
+    assert_close("logits", L, O.logits(inp["H"], inp["E"]), TOL_BF16)
+
+
 @pytest.mark.slow
 def test_logits_full_size_sampled_rows():
     w = tp_inputs.WORKLOADS["vocab_v50304"]
