@@ -118,18 +118,35 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
+        self.skip = 0
         self.path = os.path.join("/tmp", f"tp_clocks_{os.getpid()}.csv")
 
+    def _lines(self) -> int:
+        try:
+            with open(self.path) as f:
+                return sum(1 for line in f if line.endswith("\n"))
+        except OSError:
+            return 0
+
     def __enter__(self):
+        """Starts sampling and returns once the first sample is written (at
+        most 5 s), so that a short timed region that follows is covered."""
         try:
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "25"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
+            t0 = time.perf_counter()
+            while self._lines() == 0 and time.perf_counter() - t0 < 5.0 and self.proc.poll() is None:
+                time.sleep(0.01)
         except Exception:
             self.proc = None
         return self
+
+    def mark(self):
+        """Samples written before this call (start-up, warm-up) are left out."""
+        self.skip = self._lines()
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -146,7 +163,9 @@ class ClockSampler:
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         with open(self.path) as f:
-            for line in f:
+            for i, line in enumerate(f):
+                if i < self.skip:
+                    continue
                 parts = [p.strip() for p in line.split(",")]
                 if len(parts) < 9:
                     continue
@@ -665,19 +684,22 @@ def run_gpu(args):
            "cublas_gemm": lambda: _cublas_gemm(torch, g)}
     stream = torch.cuda.current_stream(dev)
 
-    for _ in range(args.warmup):
-        for p in parts:
-            fns[p]()
-    torch.cuda.synchronize(dev)
-    assert int(st.item()) == 0, f"device status {int(st.item())} after warm-up"
-
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
-          for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(dev)
-    launches0 = tpl.tp_launch_count()
+    # the clock sampler starts before the warm-up (nvidia-smi takes a moment
+    # to write its first sample); mark() keeps the samples of the timed steps
     with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.warmup):
+            for p in parts:
+                fns[p]()
+        torch.cuda.synchronize(dev)
+        assert int(st.item()) == 0, f"device status {int(st.item())} after warm-up"
+
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+              for _ in range(args.steps)]
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        launches0 = tpl.tp_launch_count()
+        clk.mark()
         t_wall = time.perf_counter()
         for s in range(args.steps):
             ev[s][0].record(stream)

@@ -161,6 +161,14 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {   // three-i
   return d;
 }
 
+// Maximum over the full warp in one instruction (sm_100a `redux.sync` on
+// f32; NaN inputs are dropped, as by fmaxf).
+__device__ __forceinline__ float warp_max_f32(float x) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // Gradient stores: fp32 float4, or four bf16 (round to nearest even) in 8 bytes.
 __device__ __forceinline__ void store_grad4(float* dst, int j, float4 e) {
   __stcs(reinterpret_cast<float4*>(dst) + j, e);
@@ -257,9 +265,7 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
     float mt = -CUDART_INF_F;
 #pragma unroll
     for (int r = 0; r < R; ++r) mt = max3f(max3f(mt, x[r].x, x[r].y), x[r].z, x[r].w);
-    float m_w = mt;
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) m_w = fmaxf(m_w, __shfl_xor_sync(0xffffffffu, m_w, off));
+    const float m_w = warp_max_f32(mt);
     int it = 0x7fffffff;
     if (mt == m_w) {   // only lanes holding the warp maximum search
 #pragma unroll
@@ -290,17 +296,17 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
     }
     float st = st2.x + st2.y;
 #pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) {
-      st += __shfl_xor_sync(0xffffffffu, st, off);
-      it = min(it, __shfl_xor_sync(0xffffffffu, it, off));
-    }
+    for (int off = 16; off >= 1; off >>= 1) st += __shfl_xor_sync(0xffffffffu, st, off);
+    it = __reduce_min_sync(0xffffffffu, it);
     if (lane == 0) {
       red_m2[p][warp] = m_w;
       red_s2[p][warp] = st;
       red_i2[p][warp] = it;
     }
     __syncthreads();   // also: every thread has its slice in registers
-    if (threadIdx.x == 0 && tok + 2 * nclusters < T) {   // refill two tokens ahead
+    // refill two tokens ahead: warp 1 issues it, so that warp 0, which
+    // sends the shard's record, does not wait for the copy to be issued
+    if (threadIdx.x == 32 && tok + 2 * nclusters < T) {
       fence_proxy_async_smem();
       issue(p, tok + 2 * nclusters);
     }
@@ -340,21 +346,17 @@ __global__ void __launch_bounds__(NT, R * NT <= 2048 ? 4 : 2)
       rt = q.z;
       ri = __float_as_int(q.w);
     }
-    float M = rm;
-#pragma unroll
-    for (int off = 4; off >= 1; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float M = warp_max_f32(rm);   // lanes past N hold -inf
     float term = lane < N ? rs * ex2_approx((rm - M) * kLog2e) : 0.f;
-    int bi = rm == M ? ri : 0x7fffffff;   // lowest index among the shards holding M
+    // lowest index among the shards holding M
+    const int bi = __reduce_min_sync(0xffffffffu, rm == M ? ri : 0x7fffffff);
 #pragma unroll
     for (int off = 4; off >= 1; off >>= 1) {
       term += __shfl_xor_sync(0xffffffffu, term, off);
       rt += __shfl_xor_sync(0xffffffffu, rt, off);
-      bi = min(bi, __shfl_xor_sync(0xffffffffu, bi, off));
     }
     const float S = __shfl_sync(0xffffffffu, term, 0);
     const float tgt = __shfl_sync(0xffffffffu, rt, 0);
-    M = __shfl_sync(0xffffffffu, M, 0);
-    bi = __shfl_sync(0xffffffffu, bi, 0);
     const float lse = M + logf(S);
     if (shard == 0 && threadIdx.x == 0) {
       loss[tok] = y_ok ? lse - tgt : CUDART_NAN_F;
