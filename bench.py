@@ -558,11 +558,13 @@ def _event_loop(torch, fn, n, stream, before=None):
     return total / n
 
 
-def _embed_flushed(torch, tpl, vo, stream, st, n=10):
-    """vp_embed with a 256 MB memset between calls, so the table rows it
-    reads come from HBM and not from the 126 MB L2."""
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device=vo["E"].device)
-    ms = _event_loop(torch, lambda: _embed(tpl, vo, st), n, stream, before=flush.zero_)
+def _flushed(torch, fn, dev, stream, n=10):
+    """Average ms of fn() with the 126 MB L2 flushed before every call: an
+    untimed read of a 256 MB buffer (torch.amax), so that the call's inputs
+    come from HBM and no dirty lines of the flush are written back inside
+    the timed call (a memset flush would leave 126 MB of them)."""
+    flush = torch.ones(256 << 20, dtype=torch.uint8, device=dev)
+    ms = _event_loop(torch, fn, n, stream, before=lambda: torch.amax(flush))
     del flush
     return ms
 
@@ -747,7 +749,8 @@ def run_gpu(args):
     at_ms = _side_loop(torch, fns, ATTN_PARTS, side_steps, stream, dev, st, world)
     ln_ms = _side_loop(torch, fns, LN_PARTS, side_steps, stream, dev, st, world)
 
-    embed_flush_ms = _embed_flushed(torch, tpl, vo, stream, st)
+    embed_flush_ms = _flushed(torch, fns["embed"], dev, stream)
+    ln_flush_ms = {p: _flushed(torch, fns[p], dev, stream) for p in LN_PARTS}
     libctx = (None if args.no_library_context else
               _library_context(torch, g, vo, stream, ours=(fns["mlp_fwd"], fns["mlp_bwd"])))
 
@@ -812,7 +815,7 @@ def run_gpu(args):
                                         "GBps": round(EMBED_BYTES / (embed_flush_ms / 1e3) / 1e9, 1),
                                         "frac_of_measured_hbm": round(EMBED_BYTES / (embed_flush_ms / 1e3) / 1e9
                                                                       / peaks["hbm_gbs"], 4),
-                                        "what": "a 256 MB memset before every call (untimed), 10 calls"}},
+                                        "what": "a 256 MB read before every call (untimed), 10 calls"}},
             "vocab_bwd": {
                 "what": "next row, own loop of %d iterations after the step" % side_steps,
                 "xent_bf16_grad_ms": round(bwd_ms["xent_bf16"], 4),
@@ -854,11 +857,24 @@ def run_gpu(args):
             "sp_layernorm": {
                 "what": "hs = X + dropout(Zo + b), y = LayerNorm(hs) and its backward, M=4096 "
                         "h=1600 over 4 sequence shards, p=0.1 (Philox masks regenerated in the "
-                        "backward); own loop of %d iterations" % side_steps,
+                        "backward); own loop of %d iterations: its 52-65 MB working set stays in "
+                        "the 126 MB L2 between calls, so these are L2-warm; l2_flushed has the "
+                        "HBM-bound figures" % side_steps,
                 "fwd_us": round(ln_ms["ln_fwd"] * 1e3, 2),
                 "fwd_GBps": round(LN_FWD_BYTES / (ln_ms["ln_fwd"] / 1e3) / 1e9, 1),
                 "bwd_us": round(ln_ms["ln_bwd"] * 1e3, 2),
                 "bwd_GBps": round(LN_BWD_BYTES / (ln_ms["ln_bwd"] / 1e3) / 1e9, 1),
+                "l2_flushed": {
+                    "what": "a 256 MB read before every call (untimed), 10 calls each",
+                    "fwd_us": round(ln_flush_ms["ln_fwd"] * 1e3, 2),
+                    "fwd_GBps": round(LN_FWD_BYTES / (ln_flush_ms["ln_fwd"] / 1e3) / 1e9, 1),
+                    "fwd_frac_of_measured_hbm": round(LN_FWD_BYTES / (ln_flush_ms["ln_fwd"] / 1e3) / 1e9
+                                                      / peaks["hbm_gbs"], 4),
+                    "bwd_us": round(ln_flush_ms["ln_bwd"] * 1e3, 2),
+                    "bwd_GBps": round(LN_BWD_BYTES / (ln_flush_ms["ln_bwd"] / 1e3) / 1e9, 1),
+                    "bwd_frac_of_measured_hbm": round(LN_BWD_BYTES / (ln_flush_ms["ln_bwd"] / 1e3) / 1e9
+                                                      / peaks["hbm_gbs"], 4),
+                },
                 "bytes_note": "8 B/element forward (x, residual in; hs, y out), 10 B/element "
                               "backward (dy, dhs, hs in; dx, dresidual out)",
             },
