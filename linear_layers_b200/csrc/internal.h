@@ -116,7 +116,7 @@ size_t sp_ln_bwd_ws_bytes(int64_t M, int64_t h);
 tp_status sp_ln_fwd_launch(const void* x, const void* bias, const void* residual, const void* gamma,
                            const void* beta, int64_t M, int64_t h, float p, uint64_t seed,
                            uint64_t offset, float eps, void* hs, void* y, float* mean, float* rstd,
-                           uint8_t* keep, cudaStream_t stream);
+                           uint8_t* keep, int32_t* dev_status, cudaStream_t stream);
 tp_status sp_ln_bwd_launch(const void* dy, const void* dhs_in, const void* hs, const void* gamma,
                            const float* mean, const float* rstd, int64_t M, int64_t h, float p,
                            uint64_t seed, uint64_t offset, void* dx, void* dres, float* dgamma,

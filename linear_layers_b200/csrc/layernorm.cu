@@ -21,8 +21,10 @@
 #include <cuda_bf16.h>
 
 #include <cmath>
+#include <cstdlib>
 
 #include "internal.h"
+#include "sm100_ptx.cuh"
 
 namespace tpl {
 
@@ -280,6 +282,177 @@ __global__ void __launch_bounds__(kLnThreads, 5) sp_ln_fwd_warp_kernel(
   }
 }
 
+// Staged forward (rows of up to 2048 elements): persistent CTAs, one per SM,
+// each owning a contiguous range of rows.  A row's x and residual reach
+// shared memory by bulk copy into one of `slots` row slots; the copies of
+// all the slots are issued at the start (at M=4096, h=1600 every row of the
+// range), so that every read of the kernel is in flight from its first
+// microsecond instead of one wave of warps' worth.  Warp w owns slots
+// w, w+W, ...: it waits for a slot's row, computes hs and y from shared
+// memory into registers and global memory, and refills the slot with the
+// row `slots` further on.  gamma, beta and the bias are copied once per CTA.
+// No block barrier after the start; every wait is bounded.
+constexpr int kLnMaxSlots = 64;
+
+__device__ __forceinline__ void ln_bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int CH, int W>
+__global__ void __launch_bounds__(W * 32, 1) sp_ln_fwd_staged_kernel(
+    const uint4* __restrict__ x, const uint4* __restrict__ bias, const uint4* __restrict__ residual,
+    const uint4* __restrict__ gamma, const uint4* __restrict__ beta, int64_t M, int h8,
+    int rows_per_cta, int slots, float inv_h, float eps, DropoutRng rng, uint4* __restrict__ hs_out,
+    uint4* __restrict__ y_out, float* __restrict__ mean_out, float* __restrict__ rstd_out,
+    uint8_t* __restrict__ keep_out, int32_t* dev_status, uint64_t wait_ns) {
+  extern __shared__ __align__(128) unsigned char lsm[];
+  __shared__ __align__(8) uint64_t full[kLnMaxSlots];
+  __shared__ __align__(8) uint64_t par_bar;
+  __shared__ int abort_flag;
+  // [gamma | beta | bias] then slots × [x row | residual row], h8 uint4 each
+  uint4* sg = reinterpret_cast<uint4*>(lsm);
+  uint4* sb = sg + h8;
+  uint4* sbias = sb + h8;
+  uint4* slot0 = sbias + h8;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * rows_per_cta;
+  const int64_t left = M - row0;
+  const int nrows = left < rows_per_cta ? static_cast<int>(left) : rows_per_cta;
+  const uint32_t row_bytes = static_cast<uint32_t>(h8) * 16u;
+  if (nrows <= 0) return;   // whole CTA
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(&par_bar, 1);
+    for (int sl = 0; sl < slots; ++sl) mbar_init(&full[sl], 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(&par_bar, (bias ? 3u : 2u) * row_bytes);
+    ln_bulk_load(sg, gamma, row_bytes, &par_bar);
+    ln_bulk_load(sb, beta, row_bytes, &par_bar);
+    if (bias) ln_bulk_load(sbias, bias, row_bytes, &par_bar);
+  }
+  auto fill = [&](int sl, int t) {   // one lane: the CTA's row t into slot sl
+    uint4* dst = slot0 + static_cast<size_t>(sl) * 2 * h8;
+    const int64_t g = row0 + t;
+    mbar_arrive_expect_tx(&full[sl], 2u * row_bytes);
+    ln_bulk_load(dst, x + g * h8, row_bytes, &full[sl]);
+    ln_bulk_load(dst + h8, residual + g * h8, row_bytes, &full[sl]);
+  };
+  if (lane == 0)
+    for (int sl = warp; sl < slots && sl < nrows; sl += W) fill(sl, sl);
+  // wait outcomes are made warp-uniform before the warp's shuffles
+  bool ok = __all_sync(0xffffffffu, mbar_wait_bounded<true>(&par_bar, 0u, wait_ns, &abort_flag));
+  for (int k = 0; ok; ++k) {
+    bool any = false;
+    for (int sl = warp; sl < slots; sl += W) {
+      const int t = sl + k * slots;
+      if (t >= nrows) break;
+      any = true;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded<true>(&full[sl], static_cast<uint32_t>(k) & 1u,
+                                                           wait_ns, &abort_flag))) {
+        ok = false;
+        break;
+      }
+      const uint4* xs = slot0 + static_cast<size_t>(sl) * 2 * h8;
+      const uint4* rs = xs + h8;
+      const int64_t row = row0 + t;
+      // hs of the row as stored (bf16-rounded), kept in fp32 for the two
+      // statistics passes and the normalisation; the element arithmetic
+      // runs on f32x2 pairs
+      float hf[CH][8];
+      float2 s2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int kk = 0; kk < CH; ++kk) {
+        const int c = lane + 32 * kk;
+        if (c < h8) {
+          const int64_t o = row * h8 + c;
+          float xv[8], rv[8], bv[8];
+          unpack8(xs[c], xv);
+          unpack8(rs[c], rv);
+          if (bias) {
+            unpack8(sbias[c], bv);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) bv[i] = 0.0f;
+          }
+          const uint32_t kb = keep_bits8(rng, static_cast<uint64_t>(o) * 8);
+          // hs = residual + keep·(x + bias)/(1 − p), one rounding after the product
+          float tv[8];
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const float2 xb = __fadd2_rn(make_float2(xv[i], xv[i + 1]), make_float2(bv[i], bv[i + 1]));
+            const float2 sc = make_float2(((kb >> i) & 1u) ? rng.inv_keep : 0.0f,
+                                          ((kb >> (i + 1)) & 1u) ? rng.inv_keep : 0.0f);
+            const float2 tt = __ffma2_rn(xb, sc, make_float2(rv[i], rv[i + 1]));
+            tv[i] = tt.x;
+            tv[i + 1] = tt.y;
+          }
+          const uint4 packed = pack8(tv);
+          __stcs(hs_out + o, packed);
+          if (keep_out)
+            *reinterpret_cast<uint2*>(keep_out + o * 8) = make_uint2(
+                ((kb >> 0) & 1u) | (((kb >> 1) & 1u) << 8) | (((kb >> 2) & 1u) << 16) | (((kb >> 3) & 1u) << 24),
+                ((kb >> 4) & 1u) | (((kb >> 5) & 1u) << 8) | (((kb >> 6) & 1u) << 16) | (((kb >> 7) & 1u) << 24));
+          unpack8(packed, hf[kk]);   // the statistics of hs as stored
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) s2 = __fadd2_rn(s2, make_float2(hf[kk][i], hf[kk][i + 1]));
+        }
+      }
+      // the slot's row is in registers: refill it with the row `slots` on
+      __syncwarp();
+      if (lane == 0 && t + slots < nrows) {
+        fence_proxy_async_smem();
+        fill(sl, t + slots);
+      }
+      const float mean = warp_sum(s2.x + s2.y) * inv_h;
+      const float2 nm2 = make_float2(-mean, -mean);
+      float2 q2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int kk = 0; kk < CH; ++kk) {
+        if (lane + 32 * kk < h8) {
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const float2 d = __fadd2_rn(make_float2(hf[kk][i], hf[kk][i + 1]), nm2);
+            q2 = __ffma2_rn(d, d, q2);
+          }
+        }
+      }
+      const float rstd = 1.0f / sqrtf(warp_sum(q2.x + q2.y) * inv_h + eps);
+      const float2 rs2 = make_float2(rstd, rstd);
+#pragma unroll
+      for (int kk = 0; kk < CH; ++kk) {
+        const int c = lane + 32 * kk;
+        if (c < h8) {
+          float gv[8], bv[8], yv[8];
+          unpack8(sg[c], gv);
+          unpack8(sb[c], bv);
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            const float2 xh = __fmul2_rn(__fadd2_rn(make_float2(hf[kk][i], hf[kk][i + 1]), nm2), rs2);
+            const float2 yy = __ffma2_rn(xh, make_float2(gv[i], gv[i + 1]), make_float2(bv[i], bv[i + 1]));
+            yv[i] = yy.x;
+            yv[i + 1] = yy.y;
+          }
+          __stcs(y_out + row * h8 + c, pack8(yv));
+        }
+      }
+      if (lane == 0) {
+        mean_out[row] = mean;
+        rstd_out[row] = rstd;
+      }
+    }
+    if (!any) break;
+  }
+  if (!ok && lane == 0 && dev_status) atomicOr(dev_status, TP_DEVERR_TIMEOUT);
+}
+
 // Backward, kLnBwdRows rows per block.  Pass A of a row forms Σ g and
 // Σ g·xhat (g = dy·gamma); pass B reads the row again (from L1) and writes
 // dresidual = rstd·(g − mean(g) − xhat·mean(g·xhat)) + dhs_in and
@@ -508,12 +681,77 @@ tp_status ln_fwd_warp_t(const void* x, const void* bias, const void* residual, c
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
 
+template <int CH, int W>
+tp_status ln_fwd_staged_t(const void* x, const void* bias, const void* residual, const void* gamma,
+                          const void* beta, int64_t M, int64_t h, const DropoutRng& g, float eps,
+                          void* hs, void* y, float* mean, float* rstd, uint8_t* keep,
+                          int32_t* dev_status, cudaStream_t stream) {
+  static int max_optin[64] = {0};
+  static size_t attr_set[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (max_optin[dev & 63] == 0 &&
+      cudaDeviceGetAttribute(&max_optin[dev & 63], cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+          cudaSuccess)
+    return TP_ERR_CUDA;
+  const size_t row_bytes = static_cast<size_t>(h / 8) * 16;
+  const int sms = num_sms();
+  const int64_t rows_per_cta = (M + sms - 1) / sms;
+  const int64_t grid = (M + rows_per_cta - 1) / rows_per_cta;
+  // shared memory: gamma, beta, bias and the row slots, 1 KB left for the
+  // static part (barriers)
+  const int64_t budget = static_cast<int64_t>(max_optin[dev & 63]) - 1024 - 3 * static_cast<int64_t>(row_bytes);
+  int64_t slots = budget / static_cast<int64_t>(2 * row_bytes);
+  if (slots > rows_per_cta) slots = rows_per_cta;
+  if (slots > kLnMaxSlots) slots = kLnMaxSlots;
+  if (slots < 1) return TP_ERR_UNSUPPORTED;
+  const size_t smem = (3 + 2 * static_cast<size_t>(slots)) * row_bytes;
+  if (smem > attr_set[dev & 63]) {
+    if (cudaFuncSetAttribute(sp_ln_fwd_staged_kernel<CH, W>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return TP_ERR_CUDA;
+    attr_set[dev & 63] = smem;
+  }
+  sp_ln_fwd_staged_kernel<CH, W><<<static_cast<unsigned>(grid), W * 32, smem, stream>>>(
+      static_cast<const uint4*>(x), static_cast<const uint4*>(bias),
+      static_cast<const uint4*>(residual), static_cast<const uint4*>(gamma),
+      static_cast<const uint4*>(beta), M, static_cast<int>(h / 8), static_cast<int>(rows_per_cta),
+      static_cast<int>(slots), 1.0f / static_cast<float>(h), eps, g, static_cast<uint4*>(hs),
+      static_cast<uint4*>(y), mean, rstd, keep, dev_status, wait_limit_ns());
+  note_launches(1);
+  return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+}
+
+// TP_LN_FWD_WARP=1 takes the register-only warp-per-row forward instead of
+// the staged one (sweeps).
+bool ln_fwd_warp_forced() {
+  const char* e = std::getenv("TP_LN_FWD_WARP");
+  return e && e[0] == '1';
+}
+
+
 tp_status sp_ln_fwd_launch(const void* x, const void* bias, const void* residual, const void* gamma,
                            const void* beta, int64_t M, int64_t h, float p, uint64_t seed,
                            uint64_t offset, float eps, void* hs, void* y, float* mean, float* rstd,
-                           uint8_t* keep, cudaStream_t stream) {
+                           uint8_t* keep, int32_t* dev_status, cudaStream_t stream) {
   const DropoutRng g = make_rng(p, seed, offset);
   const int64_t h8 = h / 8;
+  if (h8 <= 32 * 8 && !ln_fwd_warp_forced()) {
+// 16 warps per CTA: 32 measured slower (and spill at 7 or more chunks)
+#define TP_LN_STAGED(C) \
+  return ln_fwd_staged_t<C, 16>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, dev_status, stream)
+    switch ((h8 + 31) / 32) {
+      case 1: TP_LN_STAGED(1);
+      case 2: TP_LN_STAGED(2);
+      case 3: TP_LN_STAGED(3);
+      case 4: TP_LN_STAGED(4);
+      case 5: TP_LN_STAGED(5);
+      case 6: TP_LN_STAGED(6);
+      case 7: TP_LN_STAGED(7);
+      default: TP_LN_STAGED(8);
+    }
+#undef TP_LN_STAGED
+  }
   if (h8 <= 32 * 2)
     return ln_fwd_warp_t<2>(x, bias, residual, gamma, beta, M, h, g, eps, hs, y, mean, rstd, keep, stream);
   if (h8 <= 32 * 4)

@@ -655,7 +655,6 @@ tp_status tp_sp_dropout_add_ln_fwd(const void* x, const void* bias, const void* 
                                    int32_t N, float p, uint64_t seed, uint64_t offset, float eps,
                                    void* hs, void* y, float* mean, float* rstd, uint8_t* keep_out,
                                    int32_t* dev_status, void* stream) {
-  (void)dev_status;
   if (!x || !residual || !gamma || !beta || !hs || !y || !mean || !rstd) return TP_ERR_NULL;
   if (!dims_ok({M, h}) || N < 1 || M % N) return TP_ERR_SHAPE;
   if (!(p >= 0.0f && p < 1.0f) || !(eps > 0.0f)) return TP_ERR_SHAPE;
@@ -665,7 +664,7 @@ tp_status tp_sp_dropout_add_ln_fwd(const void* x, const void* bias, const void* 
     return TP_ERR_ALIGN;
   if (tp_status st = require_sm100()) return st;
   return sp_ln_fwd_launch(x, bias, residual, gamma, beta, M, h, p, seed, offset, eps, hs, y, mean,
-                          rstd, keep_out, as_stream(stream));
+                          rstd, keep_out, dev_status, as_stream(stream));
 }
 
 tp_status tp_sp_dropout_add_ln_bwd(const void* dy, const void* dhs_in, const void* hs,

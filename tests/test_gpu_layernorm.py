@@ -113,3 +113,34 @@ def test_layernorm_deterministic():
     _, b2 = _run(d, M, h, 4, 0.125, 1, 2, True)
     for k in ("dx", "dresidual", "dgamma", "dbeta", "dbias"):
         assert torch.equal(b1[k], b2[k]), k
+
+
+@pytest.mark.parametrize("M,h", [
+    (16384, 1600),   # more rows per CTA than row slots: every slot refilled
+    (1000, 2048),    # the widest row the staged forward takes
+    (5, 24),         # fewer rows than CTAs, three chunks per row
+])
+def test_layernorm_forward_staged_shapes(M, h):
+    """The staged forward (rows bulk-copied into shared-memory slots) at the
+    shapes that take its other paths."""
+    d = _inputs(M, h, seed=M + 7 * h)
+    seed, offset, p = 99, 5, 0.125
+    f, b = _run(d, M, h, 1, p, seed, offset, True)
+    ref = O.dropout_add_layernorm(d["x"], d["bias"], d["res"], d["gamma"], d["beta"], p, seed, offset)
+    assert np.array_equal(f["keep"].cpu().numpy().astype(bool), ref["keep"])
+    assert_close("hs", f["hs"], ref["hs"], TOL_BF16)
+    assert_close("y", f["y"], ref["y"], TOL_BF16)
+    assert_close("rstd", f["rstd"], ref["rstd"], TOL_STAT, elem_tol=2 * TOL_STAT)
+
+
+def test_layernorm_forward_warp_path(monkeypatch):
+    """The register-only warp-per-row forward (TP_LN_FWD_WARP=1), the path
+    the staged one replaced, kept for sweeps: same results."""
+    monkeypatch.setenv("TP_LN_FWD_WARP", "1")
+    M, h, p, seed, offset = 300, 1600, 0.125, 7, 3
+    d = _inputs(M, h, seed=21)
+    f, _ = _run(d, M, h, 4, p, seed, offset, False)
+    ref = O.dropout_add_layernorm(d["x"], d["bias"], d["res"], d["gamma"], d["beta"], p, seed, offset)
+    assert np.array_equal(f["keep"].cpu().numpy().astype(bool), ref["keep"])
+    assert_close("hs", f["hs"], ref["hs"], TOL_BF16)
+    assert_close("y", f["y"], ref["y"], TOL_BF16)
