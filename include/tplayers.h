@@ -479,6 +479,10 @@ TP_API tp_status tp_attention_bwd(const void* QKV, const void* ctx, const void* 
  *   x, residual, gamma, beta bf16; bias [h] bf16 nullable; h % 8 == 0,
  *   h <= 8192, pointers 16-byte aligned.  The formulas are not printed on
  *   the pages: this is the transformer's residual step as Megatron writes it.
+ *   For h <= 2048 the rows reach shared memory by bulk copy and every wait
+ *   for a copy is bounded: if one runs out, TP_DEVERR_TIMEOUT is ORed into
+ *   *dev_status (nullable) and the rows not yet computed are left as they
+ *   were.
  */
 TP_API tp_status tp_sp_dropout_add_ln_fwd(const void* x, const void* bias, const void* residual,
                                           const void* gamma, const void* beta, int64_t M,
