@@ -215,12 +215,37 @@ __global__ void __launch_bounds__(128) dact_colsum_v8_kernel(const uint4* __rest
   }
 }
 
-__global__ void dbias_finish_kernel(const float* part, int tiles, int N, float* dbias) {
-  const int n = blockIdx.x * blockDim.x + threadIdx.x;
-  if (n >= N) return;
+// dbias[n] = Σ_t part[t, n] in a fixed order: 32 columns per block, 8 row
+// groups of 32 threads; group q sums tiles q, q+8, q+16, … (four loads in
+// flight), then the 8 group sums are added in group order.
+__global__ void __launch_bounds__(256) dbias_finish_kernel(const float* part, int tiles, int N,
+                                                           float* dbias) {
+  __shared__ float red[8][33];
+  const int lane = threadIdx.x & 31, q = threadIdx.x >> 5;
+  const int n = blockIdx.x * 32 + lane;
   float s = 0.f;
-  for (int t = 0; t < tiles; ++t) s += part[static_cast<int64_t>(t) * N + n];
-  dbias[n] = s;
+  if (n < N) {
+    int t = q;
+    for (; t + 24 < tiles; t += 32) {
+      const float a = part[static_cast<int64_t>(t) * N + n];
+      const float b = part[static_cast<int64_t>(t + 8) * N + n];
+      const float c = part[static_cast<int64_t>(t + 16) * N + n];
+      const float d = part[static_cast<int64_t>(t + 24) * N + n];
+      s += a;
+      s += b;
+      s += c;
+      s += d;
+    }
+    for (; t < tiles; t += 8) s += part[static_cast<int64_t>(t) * N + n];
+  }
+  red[q][lane] = s;
+  __syncthreads();
+  if (q == 0 && n < N) {
+    float tot = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) tot += red[g][lane];
+    dbias[n] = tot;
+  }
 }
 
 }  // namespace
@@ -310,7 +335,7 @@ tp_status dact_colsum_launch(const void* dY, const void* U, int64_t M, int64_t N
 
 tp_status dbias_finish_launch(const float* part, int tiles, int N, float* dbias,
                               cudaStream_t stream) {
-  dbias_finish_kernel<<<(N + 255) / 256, 256, 0, stream>>>(part, tiles, N, dbias);
+  dbias_finish_kernel<<<(N + 31) / 32, 256, 0, stream>>>(part, tiles, N, dbias);
   note_launches(1);
   return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA;
 }
