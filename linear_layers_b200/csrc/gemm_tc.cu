@@ -68,6 +68,7 @@ struct GemmArgs {
   int M, N, K;
   int a_mn, b_mn;
   int tiles_m, tiles_n, splits, group_m;
+  int group_n;                      // > 0: bands of group_n tile columns instead of group_m rows
   int full_tiles;                   // split-sum GEMMs: the first full_tiles tiles (raster
                                     // order) take their whole K range, the rest are split
   int num_units;
@@ -236,7 +237,10 @@ __device__ __forceinline__ void dact_value_chunk(float (&v)[32], float (&u)[32],
 // -------------------------------------------------------------------------
 // tile scheduling: unit -> (tile row, tile column, split)
 // Tiles are visited in bands of group_m tile rows, column by column inside a
-// band, so that one wave of CTAs shares A rows and B columns through L2.
+// band, so that one wave of CTAs shares A rows and B columns through L2 and
+// B is read once per band; or, when B is the larger operand and a band of
+// its columns fits in L2, in bands of group_n tile columns, row by row
+// inside a band, so that A is the one read once per band.
 // Split-sum GEMMs: the first full_tiles tiles take their whole K range
 // (s = −1, stored directly); the tiles of the last, partial wave are split,
 // split-major (every tile's first K range, then every tile's second), and
@@ -254,6 +258,16 @@ __device__ __forceinline__ void unit_map(const GemmArgs& a, int unit, int& tm, i
     const int u = unit - a.full_tiles;
     s = u / rem;
     tile = a.full_tiles + (u - s * rem);
+  }
+  if (a.group_n > 0) {
+    const int per_group = a.group_n * a.tiles_m;
+    const int g = tile / per_group;
+    const int first_n = g * a.group_n;
+    const int gn = min(a.tiles_n - first_n, a.group_n);
+    const int r = tile - g * per_group;
+    tn = first_n + r % gn;
+    tm = r / gn;
+    return;
   }
   const int per_group = a.group_m * a.tiles_n;
   const int g = tile / per_group;
@@ -1027,6 +1041,12 @@ bool make_tmap_f32(CUtensorMap* m, const void* ptr, uint64_t inner, uint64_t out
   return r == CUDA_SUCCESS;
 }
 
+// TP_GEMM_NO_COLUMN_BANDS=1 keeps row bands for every GEMM (sweeps).
+bool column_bands_enabled() {
+  const char* e = std::getenv("TP_GEMM_NO_COLUMN_BANDS");
+  return !(e && e[0] == '1');
+}
+
 // TP_GEMM_SPLIT_ALL=1: split-sum GEMMs split every tile (sweeps).
 bool split_all_tiles() {
   const char* e = std::getenv("TP_GEMM_SPLIT_ALL");
@@ -1255,7 +1275,23 @@ tp_status setup_problem(const GemmProblem& p, const TileChoice& tile, GemmArgs& 
   // 7.3 GB read with 32-tile-row bands against 6.5 GB with 8); the byte
   // budget rule stays as a sweep switch
   a.group_m = CG == 2 ? 8 : 16;
+  // Column bands when B is more than twice A, a band of 16 B panels (its
+  // columns over the whole K range of a split) fits in a third of L2, and
+  // there are enough tile rows for a band to hold several waves: A is then
+  // re-read once per band instead of B once per row band (the logits GEMM:
+  // 13 reads of H, 134 MB, instead of 8 of the 412 MB table; 5.9 against
+  // 9.1 GB read in one capture).  The MLP's shapes (16 tile rows) read more
+  // with column bands, so they keep row bands.
+  a.group_n = 0;
+  {
+    const double kspan = static_cast<double>((p.K + p.splits - 1) / p.splits);
+    const double panel = static_cast<double>(BNT) * kspan * 2.0;
+    if (column_bands_enabled() && static_cast<int64_t>(p.N) > 2 * static_cast<int64_t>(p.M) &&
+        16.0 * panel <= 42.0 * 1024.0 * 1024.0 && a.tiles_n > 16 && a.tiles_m >= 32)
+      a.group_n = 16;
+  }
   if (band_budget_bytes() > 0.0) {
+    a.group_n = 0;
     const double row_bytes = static_cast<double>(rows) * ((p.K + p.splits - 1) / p.splits) * 2.0;
     const int band = static_cast<int>(band_budget_bytes() / row_bytes);
     a.group_m = band < 1 ? 1 : (band > a.tiles_m ? a.tiles_m : band);

@@ -82,6 +82,22 @@ def test_logits_ragged_register_store(monkeypatch):
     assert_close("logits", L, O.logits(inp["H"], inp["E"]), TOL_BF16)
 
 
+def test_logits_column_bands_bit_identical(monkeypatch):
+    """With 32 or more tile rows and B the larger operand the GEMM visits its
+    tiles in bands of columns; the order of the tiles changes nothing in any
+    tile's arithmetic, so the logits equal those of the row-band order bit
+    for bit (and the oracle on sampled rows)."""
+    inp = tp_inputs.vocab_inputs(8192, 20000, 128, seed=9)
+    H, E = inp["H"].cuda(), inp["E"].cuda()
+    L1 = tpl.tp_logits_fwd(H, E, 8)
+    monkeypatch.setenv("TP_GEMM_NO_COLUMN_BANDS", "1")
+    L2 = tpl.tp_logits_fwd(H, E, 8)
+    torch.cuda.synchronize()
+    assert torch.equal(L1, L2)
+    rows = torch.as_tensor(np.r_[0:16, 4000:4016, 8176:8192])
+    assert_close("logits[rows]", L1[rows.cuda()], O.logits(inp["H"][rows], inp["E"]), TOL_BF16)
+
+
 @pytest.mark.slow
 def test_logits_full_size_sampled_rows():
     w = tp_inputs.WORKLOADS["vocab_v50304"]
