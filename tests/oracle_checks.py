@@ -322,6 +322,10 @@ def check_embed_page_example(o):
     v, N, ids = g["v"], g["N"], np.array(g["ids"])
     assert [[o.even_offsets(v, N)[i], o.even_offsets(v, N)[i + 1]] for i in range(N)] == g["shard_ranges"]
     assert o.embed_owner(ids, v, N).tolist() == g["owner"]
+    # the ranges are half-open: each shard's first id is its own, its end id is the
+    # next shard's (or nobody's past the table)
+    edge = np.array([-1, 0, 149, 150, 299, 300])
+    assert o.embed_owner(edge, v, N).tolist() == [-1, 0, 0, 1, 1, -1]
     E = _rng(8).normal(size=(v, 16))
     out = o.vp_embed_sharded(ids, E, N)
     for t, i in enumerate(ids):
@@ -700,7 +704,7 @@ def check_philox_known_answers(o):
 def check_dropout_mask_properties(o):
     """Keep fraction within 5 sigma of 1 − p; p = 0 keeps everything; the mask is a
     function of (seed, offset) alone; element e uses word e mod 4 of counter e div 4."""
-    M, h, p = 512, 1000, 0.1
+    M, h, p = 511, 1001, 0.1
     k = o.dropout_keep(M, h, p, seed=1234, offset=7)
     n = M * h
     assert abs(k.mean() - (1 - p)) < 5 * math.sqrt(p * (1 - p) / n)
@@ -708,9 +712,15 @@ def check_dropout_mask_properties(o):
     assert np.array_equal(k, o.dropout_keep(M, h, p, 1234, 7))
     assert not np.array_equal(k, o.dropout_keep(M, h, p, 1234, 8))
     assert not np.array_equal(k, o.dropout_keep(M, h, p, 1235, 7))
-    w = o.philox4x32_10(np.array([2, 0, 7, 0], dtype=np.uint64), np.array([1234, 0], dtype=np.uint64))
-    e = 2 * 4 + 3                                         # counter 2, word 3
-    assert k.reshape(-1)[e] == (int(w[3]) >= int(math.floor(p * 2 ** 32)))
+    thr = int(math.floor(p * 2 ** 32))
+    flat = k.reshape(-1)
+    # every word of the first 64 counters and of the last (partial) one, each counter
+    # drawn on its own; h = 1001 makes rows start in the middle of a counter
+    for q in list(range(64)) + [(n - 1) // 4]:
+        w = o.philox4x32_10(np.array([q, 0, 7, 0], dtype=np.uint64), np.array([1234, 0], dtype=np.uint64))
+        for j in range(4):
+            if 4 * q + j < n:
+                assert flat[4 * q + j] == (int(w[j]) >= thr), (q, j)
 
 
 def check_layernorm_vs_torch(o):

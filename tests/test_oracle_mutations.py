@@ -343,6 +343,130 @@ def _m_row_bwd_dX_sign(mp):
     mp.setattr(O, "row_linear_bwd", bad)
 
 
+def _m_col_fwd_drops_bias(mp):
+    orig = O.col_linear_fwd
+    mp.setattr(O, "col_linear_fwd", lambda X, W, bias=None, act=O.ACT_NONE: orig(X, W, None, act))
+
+
+def _m_row_fwd_drops_last_shard(mp):
+    orig = O.row_linear_fwd
+
+    def bad(Xin, W, offsets=None, N=None):
+        Z, parts = orig(Xin, W, offsets, N)
+        if parts is None:
+            return Z, parts
+        return O.all_reduce_sum(parts[:-1] or parts), parts   # the g sum without the last shard
+    mp.setattr(O, "row_linear_fwd", bad)
+
+
+def _m_qkv_columns_k_v_swapped(mp):
+    orig = O.qkv_shard_columns
+
+    def bad(n_heads, head_dim, heads_per_shard):
+        perm, offs = orig(n_heads, head_dim, heads_per_shard)
+        perm = list(perm)
+        h = n_heads * head_dim
+        perm = [c + h if h <= c < 2 * h else (c - h if c >= 2 * h else c) for c in perm]
+        return perm, offs
+    mp.setattr(O, "qkv_shard_columns", bad)
+
+
+def _m_embed_owner_inclusive_range(mp):
+    def bad(ids, v, N):
+        ids = O.i64(ids)
+        offs = O.even_offsets(v, N)
+        own = np.full(ids.shape, -1, dtype=np.int64)
+        for i in range(N):
+            own[(ids >= offs[i]) & (ids <= offs[i + 1])] = i   # hi taken as inclusive
+        return own
+    mp.setattr(O, "embed_owner", bad)
+
+
+def _m_vp_embed_shard_base_off(mp):
+    def bad(ids, E, N):
+        ids, E = O.i64(ids), O.f64(E)
+        v, h = E.shape
+        offs = O.even_offsets(v, N)
+        parts = []
+        for i in range(N):
+            lo, hi = offs[i], offs[i + 1]
+            mine = (ids >= lo) & (ids < hi)
+            part = np.zeros((ids.shape[0], h))
+            part[mine] = E[np.minimum(ids[mine] - lo + (1 if i else 0), v - 1)]   # wrong base
+            parts.append(part)
+        return O.all_reduce_sum(parts)
+    mp.setattr(O, "vp_embed_sharded", bad)
+
+
+def _m_logits_sharded_wrong_rows(mp):
+    def bad(H, E, N):
+        H, E = O.f64(H), O.f64(E)
+        offs = O.even_offsets(E.shape[0], N)
+        return [H @ E[offs[N - 1 - i]:offs[N - i]].T for i in range(N)]   # shards in reverse
+    mp.setattr(O, "logits_sharded", bad)
+
+
+def _m_dropout_keep_next_word(mp):
+    orig = O.dropout_keep
+
+    def bad(M, h, p, seed, offset):
+        k = orig(M, h, p, seed, offset).reshape(-1)
+        n = k.size
+        w = np.arange(n)
+        return k[np.minimum((w // 4) * 4 + (w + 1) % 4, n - 1)].reshape(M, h)   # word e+1 mod 4
+    mp.setattr(O, "dropout_keep", bad)
+
+
+def _m_tied_grad_output_only(mp):
+    mp.setattr(O, "tied_embedding_grad", lambda dE_output, dE_input: O.f64(dE_output))
+
+
+def _m_embed_bwd_sharded_wrong_shard(mp):
+    orig = O.embed_bwd_sharded
+
+    def bad(ids, dout, v, N):
+        blocks = orig(ids, dout, v, N)
+        if isinstance(blocks, list) and len(blocks) > 1:
+            blocks = blocks[1:] + blocks[:1]     # blocks rotated by one shard
+        elif isinstance(blocks, np.ndarray):
+            blocks = np.roll(blocks, v // max(N, 1), axis=0)
+        return blocks
+    mp.setattr(O, "embed_bwd_sharded", bad)
+
+
+def _m_mlp_fwd_sharded_no_bias(mp):
+    orig = O.mlp_fwd_sharded
+    mp.setattr(O, "mlp_fwd_sharded",
+               lambda X, A, bias, B, N, offsets=None, act=O.ACT_GELU_TANH: orig(X, A, None, B, N, offsets, act))
+
+
+def _m_ln_bwd_sharded_first_shard_params(mp):
+    orig = O.dropout_add_layernorm_bwd_sharded
+
+    def bad(dy, dhs_in, hs, gamma, mean, rstd, keep, p, N):
+        r = orig(dy, dhs_in, hs, gamma, mean, rstd, keep, p, N)
+        M = O.f64(dy).shape[0]
+        first = O.dropout_add_layernorm_bwd(O.f64(dy)[: M // N], None if dhs_in is None else O.f64(dhs_in)[: M // N],
+                                            O.f64(hs)[: M // N], gamma, O.f64(mean)[: M // N],
+                                            O.f64(rstd)[: M // N], keep[: M // N], p)
+        r["dgamma"] = first["dgamma"]     # the parameter gradients without their all-reduce
+        return r
+    mp.setattr(O, "dropout_add_layernorm_bwd_sharded", bad)
+
+
+def _m_attention_sharded_bwd_no_dv(mp):
+    orig = O.attention_sharded_bwd
+
+    def bad(QKV, dctx, b, s, n_heads, head_dim, heads_per_shard, causal=True, scale=None):
+        d = orig(QKV, dctx, b, s, n_heads, head_dim, heads_per_shard, causal, scale)
+        col = 0
+        for nh in heads_per_shard:            # zero every shard's V block
+            d[:, col + 2 * nh * head_dim: col + 3 * nh * head_dim] = 0.0
+            col += 3 * nh * head_dim
+        return d
+    mp.setattr(O, "attention_sharded_bwd", bad)
+
+
 MUTATIONS = [v for k, v in sorted(globals().items()) if k.startswith("_m_")]
 
 
