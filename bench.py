@@ -949,9 +949,12 @@ def _oracle_mlp_sample(rows: int):
 def cpu_baseline(budget_s: float = 15.0):
     rows = 64
     dt, fl = _oracle_mlp_sample(rows)
-    # grow the sample toward the time budget (bounded)
-    if dt < budget_s / 4:
-        rows = int(min(1024, max(64, rows * (budget_s / 2) / max(dt, 1e-3))))
+    # grow the sample toward the time budget (bounded by the layer's 4096 rows);
+    # the small first samples carry fixed costs, so the growth is taken twice
+    for _ in range(2):
+        if dt >= budget_s / 2 or rows >= MLP["M"]:
+            break
+        rows = int(min(MLP["M"], max(64, rows * 0.8 * budget_s / max(dt, 1e-3))))
         rows = max(64, rows // 64 * 64)
         dt, fl = _oracle_mlp_sample(rows)
     return {"value": round(fl / dt / 1e12, 5), "unit": "TFLOP/s", "cores": _blas_threads(),
