@@ -3,9 +3,10 @@
 Thin ctypes binding over ``libtplayers.so`` (declared in ``include/tplayers.h``).
 Every function here has the name of the C entry point it calls and does
 argument marshalling only: it reads sizes from the tensors' shapes,
-allocates missing outputs with torch (device memory is torch's job), passes
-raw device pointers and the current CUDA stream, and raises ``TPError`` on a
-non-zero status.  All arithmetic happens in the library's CUDA kernels; there
+allocates missing outputs with torch (device memory is torch's job), checks
+that every other tensor has the shape, dtype and device those sizes imply,
+passes raw device pointers and the current CUDA stream, and raises
+``TPError`` on a non-zero status.  All arithmetic happens in the library's CUDA kernels; there
 is no CPU or PyTorch fallback, and importing a function whose library is
 missing fails loudly.
 
@@ -156,6 +157,40 @@ def _contig(*ts):
             raise ValueError("tensors must be contiguous (row-major, no padding)")
 
 
+_BF, _F32, _I64T, _I32T, _U8 = torch.bfloat16, torch.float32, torch.int64, torch.int32, torch.uint8
+
+
+def _want(dev, *specs):
+    """Check (name, tensor, shape, dtype) entries before anything is enqueued.
+
+    The library receives bare pointers and the sizes read from the leading
+    operands, so a tensor of another shape, dtype or device would be read or
+    written past its end on the GPU.  A None tensor (an optional argument)
+    passes; a None shape or dtype is not checked.  The status word must be
+    an int32 tensor on the same device."""
+    for name, t, shape, dtype in specs:
+        if t is None:
+            continue
+        if not isinstance(t, torch.Tensor):
+            raise TypeError(f"{name} must be a torch.Tensor, not {type(t).__name__}")
+        if t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the operands on {dev}")
+        if shape is not None and tuple(t.shape) != tuple(int(x) for x in shape):
+            raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if dtype is not None and t.dtype != dtype:
+            raise TypeError(f"{name} is {t.dtype}, expected {dtype}")
+
+
+def _status_spec(dev_status):
+    if dev_status is not None and isinstance(dev_status, torch.Tensor) and dev_status.numel() < 1:
+        raise ValueError("dev_status must hold at least one int32 word")
+    return ("dev_status", dev_status, None, _I32T)
+
+
+def _ws_spec(ws):
+    return ("ws", ws, None, None)
+
+
 def new_status(device="cuda") -> torch.Tensor:
     """A zeroed int32 device word for the kernels' TP_DEVERR_* bits."""
     return torch.zeros(1, dtype=torch.int32, device=device)
@@ -209,12 +244,23 @@ def tp_mlp_fwd(X, A, bias, B, N, *, shard_offsets=None, act=ACT_GELU_TANH, U=Non
     Y = torch.empty(M, F, dtype=X.dtype, device=dev) if Y is None else Y
     Z = torch.empty(M, h, dtype=X.dtype, device=dev) if Z is None else Z
     _contig(X, A, bias, B, U, Y, Z, Zpart)
+    dt = X.dtype
+    _want(dev, ("A", A, (h, F), dt), ("bias", bias, (F,), dt), ("B", B, (F, h), dt),
+          ("U", U, (M, F), dt), ("Y", Y, (M, F), dt), ("Z", Z, (M, h), dt),
+          ("Zpart", Zpart, (N, M, h), _F32), _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_MLP_FWD, M, h, F, N, dev)
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(bias), _ptr(B), M, h, F, N, offs, _dt(X),
                             act, _ptr(U), _ptr(Y), _ptr(Z), _ptr(Zpart), _ptr(ws), wsb,
                             _ptr(dev_status), _stream(dev)), "tp_mlp_fwd")
     return Z, U, Y
+
+
+def _mlp_bwd_specs(M, h, F, dt, A, B, U, Y, dZ, dU, dX, dA, dbias, dB, ws, dev_status):
+    return (("A", A, (h, F), dt), ("B", B, (F, h), dt), ("U", U, (M, F), dt),
+            ("Y", Y, (M, F), dt), ("dZ", dZ, (M, h), dt), ("dU", dU, (M, F), dt),
+            ("dX", dX, (M, h), dt), ("dA", dA, (h, F), dt), ("dbias", dbias, (F,), _F32),
+            ("dB", dB, (F, h), dt), _ws_spec(ws), _status_spec(dev_status))
 
 
 def tp_mlp_bwd(X, A, B, U, Y, dZ, N, *, shard_offsets=None, act=ACT_GELU_TANH, with_dbias=True,
@@ -231,6 +277,8 @@ def tp_mlp_bwd(X, A, B, U, Y, dZ, N, *, shard_offsets=None, act=ACT_GELU_TANH, w
     if dbias is None and with_dbias:
         dbias = torch.empty(F, dtype=torch.float32, device=dev)
     _contig(X, A, B, U, Y, dZ, dU, dX, dA, dB, dbias)
+    _want(dev, *_mlp_bwd_specs(M, h, F, dt, A, B, U, Y, dZ, dU, dX, dA, dbias, dB, ws,
+                               dev_status))
     ws, wsb = _workspace(ws, OP_MLP_BWD, M, h, F, N, dev)
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_mlp_bwd(_ptr(X), _ptr(A), _ptr(B), _ptr(U), _ptr(Y), _ptr(dZ), M, h, F, N,
@@ -257,6 +305,8 @@ def tp_mlp_bwd_recompute(X, A, B, U, dZ, N, *, Y=None, shard_offsets=None, act=A
     if dbias is None and with_dbias:
         dbias = torch.empty(F, dtype=torch.float32, device=dev)
     _contig(X, A, B, U, Y, dZ, dU, dX, dA, dB, dbias)
+    _want(dev, *_mlp_bwd_specs(M, h, F, dt, A, B, U, Y, dZ, dU, dX, dA, dbias, dB, ws,
+                               dev_status))
     ws, wsb = _workspace(ws, OP_MLP_BWD, M, h, F, N, dev)
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_mlp_bwd_recompute(_ptr(X), _ptr(A), _ptr(B), _ptr(U), _ptr(Y), _ptr(dZ), M, h,
@@ -277,6 +327,9 @@ def tp_col_linear_fwd(X, W, bias, N, *, shard_offsets=None, act=ACT_NONE, U=None
         U = torch.empty(M, Nout, dtype=X.dtype, device=dev)
     Y = torch.empty(M, Nout, dtype=X.dtype, device=dev) if Y is None else Y
     _contig(X, W, bias, U, Y)
+    dt = X.dtype
+    _want(dev, ("W", W, (K, Nout), dt), ("bias", bias, (Nout,), dt), ("U", U, (M, Nout), dt),
+          ("Y", Y, (M, Nout), dt), _status_spec(dev_status))
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_col_linear_fwd(_ptr(X), _ptr(W), _ptr(bias), M, K, Nout, N, offs, _dt(X),
                                    act, _ptr(U), _ptr(Y), _ptr(dev_status), _stream(dev)),
@@ -298,6 +351,9 @@ def tp_col_linear_bwd(X, W, U, dY, N, *, shard_offsets=None, act=ACT_NONE, with_
     if dbias is None and with_dbias:
         dbias = torch.empty(Nout, dtype=torch.float32, device=dev)
     _contig(X, W, U, dY, dU, dX, dW, dbias)
+    _want(dev, ("W", W, (K, Nout), dt), ("U", U, (M, Nout), dt), ("dY", dY, (M, Nout), dt),
+          ("dU", dU, (M, Nout), dt), ("dX", dX, (M, K), dt), ("dW", dW, (K, Nout), dt),
+          ("dbias", dbias, (Nout,), _F32), _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_COL_LINEAR_BWD, M, K, Nout, N, dev)
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_col_linear_bwd(_ptr(X), _ptr(W), _ptr(U), _ptr(dY), M, K, Nout, N, offs,
@@ -315,6 +371,9 @@ def tp_row_linear_fwd(Xin, W, N, *, shard_offsets=None, Z=None, Zpart=None, ws=N
     dev = Xin.device
     Z = torch.empty(M, Nout, dtype=Xin.dtype, device=dev) if Z is None else Z
     _contig(Xin, W, Z, Zpart)
+    dt = Xin.dtype
+    _want(dev, ("W", W, (Kin, Nout), dt), ("Z", Z, (M, Nout), dt),
+          ("Zpart", Zpart, (N, M, Nout), _F32), _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_ROW_LINEAR_FWD, M, Nout, Kin, N, dev)
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_row_linear_fwd(_ptr(Xin), _ptr(W), M, Kin, Nout, N, offs, _dt(Xin), _ptr(Z),
@@ -341,6 +400,8 @@ def tp_row_linear_fwd_noalloc(Xin, W, N, *, shard_offsets=None, Z=None, dev_stat
     dev = Xin.device
     Z = torch.empty(M, Nout, dtype=Xin.dtype, device=dev) if Z is None else Z
     _contig(Xin, W, Z)
+    dt = Xin.dtype
+    _want(dev, ("W", W, (Kin, Nout), dt), ("Z", Z, (M, Nout), dt), _status_spec(dev_status))
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_row_linear_fwd_noalloc(_ptr(Xin), _ptr(W), M, Kin, Nout, N, offs, _dt(Xin),
                                            _ptr(Z), _ptr(dev_status), _stream(dev)),
@@ -356,6 +417,9 @@ def tp_row_linear_bwd(Xin, W, dZ, N, *, shard_offsets=None, dXin=None, dW=None, 
     dXin = torch.empty(M, Kin, dtype=Xin.dtype, device=dev) if dXin is None else dXin
     dW = torch.empty(Kin, Nout, dtype=Xin.dtype, device=dev) if dW is None else dW
     _contig(Xin, W, dZ, dXin, dW)
+    dt = Xin.dtype
+    _want(dev, ("W", W, (Kin, Nout), dt), ("dZ", dZ, (M, Nout), dt), ("dXin", dXin, (M, Kin), dt),
+          ("dW", dW, (Kin, Nout), dt), _status_spec(dev_status))
     offs, keep = _offsets(shard_offsets, N)
     _check(lib().tp_row_linear_bwd(_ptr(Xin), _ptr(W), _ptr(dZ), M, Kin, Nout, N, offs, _dt(Xin),
                                    _ptr(dXin), _ptr(dW), _ptr(dev_status), _stream(dev)),
@@ -372,6 +436,7 @@ def vp_embed(ids, E, N, *, out=None, dev_status=None):
     _contig(ids, E, out)
     if ids.dtype != torch.int64:
         raise TypeError("ids must be int64")
+    _want(dev, ("ids", ids, (T,), _I64T), ("out", out, (T, h), E.dtype), _status_spec(dev_status))
     _check(lib().vp_embed(_ptr(ids), T, _ptr(E), v, h, N, _dt(E), _ptr(out), _ptr(dev_status),
                           _stream(dev)), "vp_embed")
     return out
@@ -384,9 +449,17 @@ def tp_logits_fwd(H, E, N, *, logits=None, dev_status=None):
     dev = H.device
     logits = torch.empty(T, v, dtype=torch.float32, device=dev) if logits is None else logits
     _contig(H, E, logits)
+    _want(dev, ("H", H, (T, h), _BF), ("E", E, (v, h), _BF), ("logits", logits, (T, v), _F32),
+          _status_spec(dev_status))
     _check(lib().tp_logits_fwd(_ptr(H), _ptr(E), T, h, v, N, _ptr(logits), _ptr(dev_status),
                                _stream(dev)), "tp_logits_fwd")
     return logits
+
+
+def _xent_specs(T, v, logits, targets, loss, loss_sum, argmax, dev_status):
+    return (("logits", logits, (T, v), _F32), ("targets", targets, (T,), _I64T),
+            ("loss", loss, (T,), _F32), ("loss_sum", loss_sum, (1,), _F32),
+            ("argmax", argmax, (T,), _I32T), _status_spec(dev_status))
 
 
 def vp_xent(logits, targets, N, *, grad_scale=1.0, with_grad=True, with_argmax=True,
@@ -403,6 +476,8 @@ def vp_xent(logits, targets, N, *, grad_scale=1.0, with_grad=True, with_argmax=T
     _contig(logits, targets, loss, dlogits, argmax)
     if targets.dtype != torch.int64:
         raise TypeError("targets must be int64")
+    _want(dev, *_xent_specs(T, v, logits, targets, loss, loss_sum, argmax, dev_status),
+          ("dlogits", dlogits, (T, v), _F32))
     _check(lib().vp_xent(_ptr(logits), _ptr(targets), T, v, N, float(grad_scale), _ptr(loss),
                          _ptr(loss_sum), _ptr(dlogits), _ptr(argmax), _ptr(dev_status),
                          _stream(dev)), "vp_xent")
@@ -422,6 +497,8 @@ def vp_xent_bf16_grad(logits, targets, N, *, grad_scale=1.0, with_argmax=True, l
     _contig(logits, targets, loss, dlogits, argmax)
     if targets.dtype != torch.int64:
         raise TypeError("targets must be int64")
+    _want(dev, *_xent_specs(T, v, logits, targets, loss, loss_sum, argmax, dev_status),
+          ("dlogits", dlogits, (T, v), _BF))
     _check(lib().vp_xent_bf16_grad(_ptr(logits), _ptr(targets), T, v, N, float(grad_scale),
                                    _ptr(loss), _ptr(loss_sum), _ptr(dlogits), _ptr(argmax),
                                    _ptr(dev_status), _stream(dev)), "vp_xent_bf16_grad")
@@ -436,6 +513,8 @@ def tp_logits_bwd(dlogits, H, E, N, *, dH=None, dE=None, dev_status=None):
     dH = torch.empty(T, h, dtype=H.dtype, device=dev) if dH is None else dH
     dE = torch.empty(v, h, dtype=torch.float32, device=dev) if dE is None else dE
     _contig(dlogits, H, E, dH, dE)
+    _want(dev, ("dlogits", dlogits, (T, v), _BF), ("H", H, (T, h), _BF), ("E", E, (v, h), _BF),
+          ("dH", dH, (T, h), _BF), ("dE", dE, (v, h), _F32), _status_spec(dev_status))
     _check(lib().tp_logits_bwd(_ptr(dlogits), _ptr(H), _ptr(E), T, h, v, N, _ptr(dH), _ptr(dE),
                                _ptr(dev_status), _stream(dev)), "tp_logits_bwd")
     return dH, dE
@@ -449,6 +528,8 @@ def vp_embed_bwd(ids, dout, dE, N, *, ws=None, dev_status=None):
     _contig(ids, dout, dE)
     if ids.dtype != torch.int64:
         raise TypeError("ids must be int64")
+    _want(dev, ("ids", ids, (T,), _I64T), ("dout", dout, (T, h), _BF), ("dE", dE, (v, h), _F32),
+          _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_EMBED_BWD, T, h, v, N, dev)
     _check(lib().vp_embed_bwd(_ptr(ids), _ptr(dout), T, v, h, N, _ptr(dE), _ptr(ws), wsb,
                               _ptr(dev_status), _stream(dev)), "vp_embed_bwd")
@@ -472,6 +553,9 @@ def tp_linear_xent_fwd(H, E, targets, N, *, with_argmax=True, loss=None, loss_su
     _contig(H, E, targets, loss, lse, argmax)
     if targets.dtype != torch.int64:
         raise TypeError("targets must be int64")
+    _want(dev, ("H", H, (T, h), _BF), ("E", E, (v, h), _BF), ("targets", targets, (T,), _I64T),
+          ("loss", loss, (T,), _F32), ("loss_sum", loss_sum, (1,), _F32), ("lse", lse, (T,), _F32),
+          ("argmax", argmax, (T,), _I32T), _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_LINEAR_XENT, T, h, v, N, dev)
     _check(lib().tp_linear_xent_fwd(_ptr(H), _ptr(E), _ptr(targets), T, h, v, N, _ptr(loss),
                                     _ptr(loss_sum), _ptr(lse), _ptr(argmax), _ptr(ws), wsb,
@@ -489,6 +573,8 @@ def tp_linear_xent_dlogits(H, E, targets, lse, N, *, grad_scale=1.0, dlogits=Non
     _contig(H, E, targets, lse, dlogits)
     if targets.dtype != torch.int64:
         raise TypeError("targets must be int64")
+    _want(dev, ("H", H, (T, h), _BF), ("E", E, (v, h), _BF), ("targets", targets, (T,), _I64T),
+          ("lse", lse, (T,), _F32), ("dlogits", dlogits, (T, v), _BF), _status_spec(dev_status))
     _check(lib().tp_linear_xent_dlogits(_ptr(H), _ptr(E), _ptr(targets), _ptr(lse), T, h, v, N,
                                         float(grad_scale), _ptr(dlogits), _ptr(dev_status),
                                         _stream(dev)), "tp_linear_xent_dlogits")
@@ -506,6 +592,8 @@ def tp_attention_fwd(QKV, b, s, n_heads, N, *, head_offsets=None, causal=True, s
     if with_lse and lse is None:
         lse = torch.empty(b, n_heads, s, dtype=torch.float32, device=dev)
     _contig(QKV, ctx, lse)
+    _want(dev, ("QKV", QKV, (b * s, 3 * n_heads * hd), _BF), ("ctx", ctx, (b * s, n_heads * hd), _BF),
+          ("lse", lse, (b, n_heads, s), _F32), _status_spec(dev_status))
     offs, keep = _offsets(head_offsets, N)
     _check(lib().tp_attention_fwd(_ptr(QKV), b, s, n_heads, hd, N, offs, 1 if causal else 0,
                                   float(scale) if scale else 0.0, _ptr(ctx), _ptr(lse),
@@ -528,6 +616,10 @@ def tp_sp_dropout_add_ln_fwd(x, bias, residual, gamma, beta, N, *, p=0.0, seed=0
     if with_keep and keep is None:
         keep = torch.empty(M, h, dtype=torch.uint8, device=dev)
     _contig(x, bias, residual, gamma, beta, hs, y, mean, rstd, keep)
+    _want(dev, ("x", x, (M, h), _BF), ("bias", bias, (h,), _BF), ("residual", residual, (M, h), _BF),
+          ("gamma", gamma, (h,), _BF), ("beta", beta, (h,), _BF), ("hs", hs, (M, h), _BF),
+          ("y", y, (M, h), _BF), ("mean", mean, (M,), _F32), ("rstd", rstd, (M,), _F32),
+          ("keep", keep, (M, h), _U8), _status_spec(dev_status))
     _check(lib().tp_sp_dropout_add_ln_fwd(_ptr(x), _ptr(bias), _ptr(residual), _ptr(gamma),
                                           _ptr(beta), M, h, N, float(p), int(seed), int(offset),
                                           float(eps), _ptr(hs), _ptr(y), _ptr(mean), _ptr(rstd),
@@ -549,6 +641,11 @@ def tp_sp_dropout_add_ln_bwd(dy, dhs_in, hs, gamma, mean, rstd, N, *, p=0.0, see
     if with_dbias and dbias is None:
         dbias = torch.empty(h, dtype=torch.float32, device=dev)
     _contig(dy, dhs_in, hs, gamma, mean, rstd, dx, dresidual, dgamma, dbeta, dbias)
+    _want(dev, ("dy", dy, (M, h), _BF), ("dhs_in", dhs_in, (M, h), _BF), ("hs", hs, (M, h), _BF),
+          ("gamma", gamma, (h,), _BF), ("mean", mean, (M,), _F32), ("rstd", rstd, (M,), _F32),
+          ("dx", dx, (M, h), _BF), ("dresidual", dresidual, (M, h), _BF),
+          ("dgamma", dgamma, (h,), _F32), ("dbeta", dbeta, (h,), _F32), ("dbias", dbias, (h,), _F32),
+          _ws_spec(ws), _status_spec(dev_status))
     ws, wsb = _workspace(ws, OP_SP_LN_BWD, M, h, h, N, dev)
     _check(lib().tp_sp_dropout_add_ln_bwd(_ptr(dy), _ptr(dhs_in), _ptr(hs), _ptr(gamma),
                                           _ptr(mean), _ptr(rstd), M, h, N, float(p), int(seed),
@@ -566,6 +663,9 @@ def tp_attention_bwd(QKV, ctx, dctx, lse, b, s, n_heads, N, *, head_offsets=None
     dev = QKV.device
     dQKV = torch.empty_like(QKV) if dQKV is None else dQKV
     _contig(QKV, ctx, dctx, lse, dQKV)
+    _want(dev, ("QKV", QKV, (b * s, 3 * n_heads * 64), _BF), ("ctx", ctx, (b * s, n_heads * 64), _BF),
+          ("dctx", dctx, (b * s, n_heads * 64), _BF), ("lse", lse, (b, n_heads, s), _F32),
+          ("dQKV", dQKV, (b * s, 3 * n_heads * 64), _BF), _ws_spec(ws), _status_spec(dev_status))
     offs, keep = _offsets(head_offsets, N)
     ws, wsb = _workspace(ws, OP_ATTENTION_BWD, b * s, n_heads, 64, N, dev)
     _check(lib().tp_attention_bwd(_ptr(QKV), _ptr(ctx), _ptr(dctx), _ptr(lse), b, s, n_heads, 64,
