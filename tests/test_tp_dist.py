@@ -67,6 +67,23 @@ def _worker(rank, world, port, q):
 
         ok = []
         comp = _Float64Shard(O)
+        # count the collectives: [MLP-TP] §2.3 / [TP-ILL] §2.2 put exactly one
+        # all-reduce of b·s·h elements in the MLP's forward (g) and one in its
+        # backward (f); the column-parallel block all-reduces only dX, the
+        # row-parallel block only Z
+        sent = []
+        plain_all_reduce = dist.all_reduce
+
+        def counting_all_reduce(t, *a, **k):
+            sent.append(t.numel())
+            return plain_all_reduce(t, *a, **k)
+
+        D.dist.all_reduce = counting_all_reduce
+
+        def moved(fn, *a):
+            sent.clear()
+            r = fn(*a)
+            return r, list(sent)
         F = 48
         inp = tp_inputs.mlp_inputs(10, 16, F, dtype=torch.float32, w_std=0.3, bias_std=0.1, seed=7)
         X, A, b, B, dZ = (inp[k].double() for k in ("X", "A", "bias", "B", "dZ"))
@@ -74,8 +91,9 @@ def _worker(rank, world, port, q):
         for offsets in (None, uneven):
             A_i, b_i, B_i = D.shard_mlp_weights(A, b, B, rank, world, offsets)
             layer = D.TPMLP(A_i, b_i, B_i, compute=comp)
-            Z, state = layer.forward(X)
-            g = layer.backward(X, state, dZ)
+            (Z, state), n_fwd = moved(layer.forward, X)
+            g, n_bwd = moved(layer.backward, X, state, dZ)
+            ok.append(n_fwd == [X.shape[0] * X.shape[1]] and n_bwd == [X.shape[0] * X.shape[1]])
             _, _, oZ = O.mlp_fwd(X, A, b, B)
             og = O.mlp_bwd(X, A, b, B, dZ)
             offs = D.shard_bounds(F, world, offsets)
@@ -94,9 +112,10 @@ def _worker(rank, world, port, q):
         offs = D.shard_bounds(12, world, None)
         lo, hi = offs[rank], offs[rank + 1]
         col = D.ColumnParallelLinear(Wc[:, lo:hi].contiguous(), bc[lo:hi].contiguous(), compute=comp)
-        Yi = col.forward(Xl)
+        Yi, n_cf = moved(col.forward, Xl)
         dY = torch.from_numpy(r.normal(size=(6, 12)))
-        gc = col.backward(Xl, dY[:, lo:hi].contiguous())
+        gc, n_cb = moved(col.backward, Xl, dY[:, lo:hi].contiguous())
+        ok.append(n_cf == [] and n_cb == [6 * 9])
         _, oY = O.col_linear_fwd(Xl, Wc, bc)
         ocb = O.col_linear_bwd(Xl, Wc, oY, dY)
         ok.append(np.abs(Yi.numpy() - oY[:, lo:hi]).max() < 1e-12)
@@ -105,9 +124,10 @@ def _worker(rank, world, port, q):
         ok.append(np.abs(gc["dbias"].numpy() - ocb["dbias"][lo:hi]).max() < 1e-12)
         Wr = torch.from_numpy(r.normal(size=(12, 5)))
         row = D.RowParallelLinear(Wr[lo:hi].contiguous(), compute=comp)
-        Zr = row.forward(Yi)
+        Zr, n_rf = moved(row.forward, Yi)
         dZr = torch.from_numpy(r.normal(size=(6, 5)))
-        gr = row.backward(Yi, dZr)
+        gr, n_rb = moved(row.backward, Yi, dZr)
+        ok.append(n_rf == [6 * 5] and n_rb == [])
         oZr, _ = O.row_linear_fwd(oY, Wr)
         orb = O.row_linear_bwd(oY, Wr, dZr)
         ok.append(np.abs(Zr.numpy() - oZr).max() < 1e-12)
