@@ -154,6 +154,63 @@ def test_tp_dist_gloo_ranks_match_unsharded(world):
         assert all(oks), (rank, oks)
 
 
+def _failing_worker(rank, world, port, q):
+    """Rank 1 fails between steps (raises before the forward, its process
+    ends); rank 0 must learn of it from its next collective, which ends with
+    an error within the process group's short timeout instead of waiting."""
+    import time
+    from datetime import timedelta
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=5))
+    from linear_layers_b200 import tp_dist as D
+    from oracle import tp_oracle as O
+
+    comp = _Float64Shard(O)
+    r = np.random.default_rng(3)
+    X = torch.from_numpy(r.normal(size=(4, 8)))
+    A_i = torch.from_numpy(r.normal(size=(8, 6)))
+    B_i = torch.from_numpy(r.normal(size=(6, 8)))
+    layer = D.TPMLP(A_i, None, B_i, compute=comp)
+    layer.forward(X)                      # one good step on both ranks
+    dist.barrier()
+    if rank == 1:
+        q.put((rank, "left", 0.0))
+        q.close()
+        q.join_thread()                   # the message is out before the process ends
+        os._exit(3)                       # the failure: this rank is gone
+    t0 = time.monotonic()
+    try:
+        layer.forward(X)
+        q.put((rank, "no error", time.monotonic() - t0))
+    except Exception as e:                # gloo: peer closed, or the timeout
+        q.put((rank, type(e).__name__, time.monotonic() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)                           # the broken group is not torn down
+
+
+def test_tp_dist_rank_failure_ends_the_next_collective_with_an_error():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = {}
+    for _ in procs:
+        rank, what, secs = q.get(timeout=120)
+        res[rank] = (what, secs)
+    for p in procs:
+        p.join(timeout=60)
+    assert res[1][0] == "left"
+    what, secs = res[0]
+    assert what != "no error", "the surviving rank's all-reduce completed without its peer"
+    assert secs < 30, secs                 # ended by the error, not by waiting for good
+    assert procs[1].exitcode == 3
+
+
 def test_shard_bounds_validation():
     from linear_layers_b200 import tp_dist as D
 
