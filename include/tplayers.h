@@ -29,6 +29,9 @@
  *    memory and never synchronises; all work is enqueued on `stream`
  *    (a cudaStream_t, passed as void*; NULL = legacy default stream) and the
  *    call returns before it completes.
+ *  - Every size (M, h, F, K, Nout, T, v, b·s, ...) lies in [1, 2^30]; a size
+ *    outside that range returns TP_ERR_SHAPE.  An empty batch is therefore
+ *    not a call: skip it on the host.
  *  - Argument errors are returned synchronously, before anything is
  *    enqueued.  Errors found on the device (an id or target out of range, a
  *    bounded wait that ran out) are OR-ed as TP_DEVERR_* bits into

@@ -87,6 +87,8 @@ def test_validation_errors_before_any_launch(L):
     assert _mlp_fwd(L, dt=7) == TP_ERR_DTYPE
     assert _mlp_fwd(L, act=9) == TP_ERR_DTYPE
     assert _mlp_fwd(L, M=0) == TP_ERR_SHAPE
+    assert _mlp_fwd(L, M=(1 << 30) + 1) == TP_ERR_SHAPE        # sizes are bounded by 2^30
+    assert _mlp_fwd(L, h=-8) == TP_ERR_SHAPE
     assert _mlp_fwd(L, F=250, N=4) == TP_ERR_SHAPE            # F % N without offsets
     assert _mlp_fwd(L, h=60) == TP_ERR_ALIGN                   # bf16 rows need 8 | h
     assert _mlp_fwd(L, X=ctypes.c_void_p((1 << 20) + 8)) == TP_ERR_ALIGN
